@@ -1,0 +1,412 @@
+"""KronQ per-layer hot path: plain, slow, fp64 CPU oracle.
+
+TEST INFRASTRUCTURE ONLY. This module is the yardstick the CUDA library is checked against.
+Only the test suite, the smoke check and the benchmark's CPU-baseline / reference arm may
+import it; the library itself never does, and the two share no code (the oracle uses numpy
+and scipy; the library is CUDA C++).
+
+What it computes, step by step, with the passage each step follows. Page names:
+  [KronQ-hyper]  "KronQ: LLM Quantization via Kronecker-Factored Hessian", hyper.ai summary
+                 (Method section; the only page that prints the equations).
+  [KronQ-gist]   the same paper, gist.science technical summary (Methodology, Limitations).
+
+  accumulate      H_X = E[x x^T], H_G = E[g g^T] under the K-FAC split H ~ H_X (x) H_G, and the
+                  asymmetric term E[(x - x~) x~^T]            [KronQ-hyper] Method: Fisher eq.,
+                                                              K-FAC split, asymmetric objective
+  biip            W <- S_G W S_X with S_X = diag(H_X,jj/|W_:,j|^2)^(1/4), S_G likewise on rows;
+                  then W <- U W V^T, H_X <- V H_X V^T, H_G <- U H_G U^T, dXX^T <- V dXX^T V^T
+                  with U, V random-sign Hadamard          [KronQ-hyper] Method: BiIP equations
+  score           s = tr(H_G) * tr(H_X), after BiIP          [KronQ-hyper] Method: sensitivity
+  cholinv         K = upper Cholesky factor of (H_X + lambda I)^-1, read as the "[H_X^-1]" rows
+                  of the column update                      [KronQ-hyper] Method: OBS update
+  p_matrix        P = striu(D K^T) K (GPTAQ's correction matrix; the pages name P but do not
+                  define it - this is the documented reading)
+  grid            per-output-row asymmetric min-max b-bit grid
+  quantize_layer  column-wise OBS update, literally:
+                    dW_:,p+1: = -delta_p [H_X^-1]_p,p+1: + W_:,p P_p,p+1:
+                                                             [KronQ-hyper] Method: OBS update
+  score_allocate  larger s gets more bits, greedy under an average-bit budget
+                                                  [KronQ-hyper] Method: mixed precision;
+                                                  [KronQ-gist] Experimental results (upgrade the
+                                                  higher-scored sublayer first)
+  objective       tr[H_G dW H_X dW^T] + 2 tr[H_G W D dW^T]  [KronQ-hyper] Method: objectives
+  mu_incoherence  max_ij |Q_ij| over eigenvectors Q of H (mu(H)/sqrt(d))
+                                                  [KronQ-hyper] Method: incoherence figure
+
+Precision: all continuous arithmetic is fp64. The two places where floating point decides an
+integer (the grid's integer zero point and each quantized code) are evaluated in fp32, the
+precision the CUDA kernels decide them in, so that both sides take the same decision.
+
+Readings where the pages are silent or ambiguous (each is also listed in the design notes):
+  * statistics are normalised by 1/N; H_X is built from the quantized-path input x~;
+  * the asymmetric term is D = E[(x - x~) x~^T] with factor 2 in the objective and "+" in the
+    update (exact expansion of E|W x - W^ x~|^2_{H_G});
+  * S_X and S_G are both computed from the original W; H_X, D transform as S_X^-1 . S_X^-1,
+    H_G as S_G^-1 . S_G^-1 (the only choice that leaves the objective unchanged); a zero norm or
+    zero diagonal gives scale 1;
+  * U = (1/sqrt(b)) (I (x) H_b) diag(sigma): Sylvester Hadamard blocks of b = largest power of
+    two dividing d, caller-supplied signs;
+  * damping lambda = damp_rel * mean diag(H_X after BiIP), added before factorisation;
+  * grid: lo/hi = row min/max of W' before the solve, scale = (hi-lo)/(2^b-1) (1 if hi == lo),
+    zero = rint(-lo/scale), codes clamp(rint(w/scale)+zero, 0, 2^b-1), round half to even;
+  * columns in natural order; allocation is the greedy in score_allocate.
+
+Parity pins: every function here is pinned by tests in tests/test_oracle_pins.py against
+closed forms, brute force or textbook special cases; none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import scipy.linalg as sla
+
+# flags of the incoherence step (same numeric values as the C header, re-declared here)
+SCALE_IN = 1
+SCALE_OUT = 2
+ROTATE_IN = 4
+ROTATE_OUT = 8
+BIIP_FULL = SCALE_IN | SCALE_OUT | ROTATE_IN | ROTATE_OUT
+
+
+class NotPositiveDefinite(Exception):
+    pass
+
+
+# ------------------------------------------------------------------------------------------
+# Statistics
+# ------------------------------------------------------------------------------------------
+
+def accumulate(xq, xfp=None, g=None):
+    """Raw (un-normalised) sums over the N calibration tokens (rows).
+
+    hx_sum = X~^T X~, hg_sum = G^T G, dxx_sum = (X - X~)^T X~.
+    [KronQ-hyper] Method: H_X = E[x x^T], H_G = E[g g^T] (K-FAC split of the empirical Fisher
+    E[x x^T (x) g g^T]); the asymmetric objective's input-drift term dX X^T.
+    """
+    xq = np.asarray(xq, dtype=np.float64)
+    hx = xq.T @ xq
+    hg = None
+    if g is not None:
+        g = np.asarray(g, dtype=np.float64)
+        hg = g.T @ g
+    dxx = None
+    if xfp is not None:
+        xfp = np.asarray(xfp, dtype=np.float64)
+        dxx = (xfp - xq).T @ xq
+    return hx, hg, dxx
+
+
+def fisher_kron(x, g):
+    """Empirical Fisher E[vec(dL/dW) vec(dL/dW)^T] with dL/dW = g x^T, column-stacked vec.
+
+    [KronQ-hyper] Method: Fisher equation, vec(g x^T) = x (x) g. Brute force, tiny sizes only.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    g = np.asarray(g, dtype=np.float64)
+    n = x.shape[0]
+    dim = x.shape[1] * g.shape[1]
+    f = np.zeros((dim, dim))
+    for t in range(n):
+        grad = np.outer(g[t], x[t])           # dL/dW, d_out x d_in
+        v = grad.reshape(-1, order="F")       # column-stacked vec
+        f += np.outer(v, v)
+    return f / n
+
+
+# ------------------------------------------------------------------------------------------
+# Hadamard blocks
+# ------------------------------------------------------------------------------------------
+
+def hadamard_block_size(d: int) -> int:
+    """Largest power of two dividing d (the Hadamard block size used for dimension d)."""
+    if d <= 0:
+        raise ValueError("d must be positive")
+    return d & (-d)
+
+
+def sylvester(b: int) -> np.ndarray:
+    """Sylvester Hadamard matrix of order b: [H_b]_ij = (-1)^popcount(i & j)."""
+    i = np.arange(b)
+    pc = np.zeros((b, b), dtype=np.int64)
+    a = i[:, None] & i[None, :]
+    while np.any(a):
+        pc += a & 1
+        a = a >> 1
+    return np.where(pc % 2 == 0, 1.0, -1.0)
+
+
+def transform_matrix(d: int, signs) -> np.ndarray:
+    """Dense U (or V) = (1/sqrt(b)) (I_{d/b} (x) H_b) diag(signs). Small d only."""
+    b = hadamard_block_size(d)
+    blk = np.kron(np.eye(d // b), sylvester(b)) / math.sqrt(b)
+    return blk * np.asarray(signs, dtype=np.float64)[None, :]
+
+
+def apply_transform(m, signs, axis: int):
+    """Apply T = (1/sqrt(b)) (I (x) H_b) diag(signs) along one axis of m.
+
+    axis=1 returns m T^T (rows transformed), axis=0 returns T m (columns transformed).
+    Implemented with the block structure (reshape into d/b blocks of b and multiply each by the
+    Sylvester matrix) so that large d stays tractable.
+    """
+    m = np.asarray(m, dtype=np.float64)
+    d = m.shape[axis]
+    b = hadamard_block_size(d)
+    h = sylvester(b) / math.sqrt(b)
+    s = np.asarray(signs, dtype=np.float64)
+    if axis == 1:
+        ms = m * s[None, :]
+        r = ms.reshape(m.shape[0], d // b, b) @ h.T
+        return r.reshape(m.shape[0], d)
+    ms = m * s[:, None]
+    r = np.einsum("ij,kjc->kic", h, ms.reshape(d // b, b, m.shape[1]))
+    return r.reshape(d, m.shape[1])
+
+
+# ------------------------------------------------------------------------------------------
+# Bidirectional incoherence processing
+# ------------------------------------------------------------------------------------------
+
+def biip(w, hx_sum, hg_sum=None, dxx_sum=None, inv_n=1.0, sign_in=None, sign_out=None,
+         flags=BIIP_FULL):
+    """Normalise the sums, rescale, rotate; return the processed layer and its traces.
+
+    [KronQ-hyper] Method, BiIP equations:
+      W <- S_G W S_X,  S_X = diag(H_X,jj / |W_:,j|^2)^(1/4),  S_G = diag(H_G,ii / |W_i,:|^2)^(1/4)
+      W <- U W V^T,  H_X <- V H_X V^T,  H_G <- U H_G U^T,  dXX^T <- V dXX^T V^T.
+    The Hessians follow the scaling as H_X <- S_X^-1 H_X S_X^-1, H_G <- S_G^-1 H_G S_G^-1,
+    D <- S_X^-1 D S_X^-1, which keeps tr[H_G dW H_X dW^T] unchanged.
+    Returns dict: w, hx, hg (None if not given), dxx (None if not given), s_x, s_g, tr_hx, tr_hg.
+    """
+    w0 = np.asarray(w, dtype=np.float64)
+    d_out, d_in = w0.shape
+    hx = np.asarray(hx_sum, dtype=np.float64) * inv_n
+    hg = None if hg_sum is None else np.asarray(hg_sum, dtype=np.float64) * inv_n
+    dxx = None if dxx_sum is None else np.asarray(dxx_sum, dtype=np.float64) * inv_n
+    if (flags & SCALE_OUT) and hg is None:
+        raise ValueError("output-side scaling needs H_G")
+
+    col_sq = (w0 * w0).sum(axis=0)    # |W_:,j|^2 of the original W
+    row_sq = (w0 * w0).sum(axis=1)    # |W_i,:|^2 of the original W
+    s_x = np.ones(d_in)
+    s_g = np.ones(d_out)
+    if flags & SCALE_IN:
+        dx = np.diag(hx)
+        ok = (col_sq > 0) & (dx > 0)
+        s_x[ok] = (dx[ok] / col_sq[ok]) ** 0.25
+    if flags & SCALE_OUT:
+        dg = np.diag(hg)
+        ok = (row_sq > 0) & (dg > 0)
+        s_g[ok] = (dg[ok] / row_sq[ok]) ** 0.25
+
+    wp = s_g[:, None] * w0 * s_x[None, :]
+    hx = hx / np.outer(s_x, s_x)
+    if dxx is not None:
+        dxx = dxx / np.outer(s_x, s_x)
+    if hg is not None:
+        hg = hg / np.outer(s_g, s_g)
+
+    if flags & ROTATE_IN:
+        wp = apply_transform(wp, sign_in, axis=1)                      # W V^T
+        hx = apply_transform(apply_transform(hx, sign_in, axis=0), sign_in, axis=1)  # V H V^T
+        if dxx is not None:
+            dxx = apply_transform(apply_transform(dxx, sign_in, axis=0), sign_in, axis=1)
+    if flags & ROTATE_OUT:
+        wp = apply_transform(wp, sign_out, axis=0)                     # U W
+        if hg is not None:
+            hg = apply_transform(apply_transform(hg, sign_out, axis=0), sign_out, axis=1)
+
+    tr_hx = float(np.trace(hx))
+    tr_hg = None if hg is None else float(np.trace(hg))
+    return {"w": wp, "hx": hx, "hg": hg, "dxx": dxx, "s_x": s_x, "s_g": s_g,
+            "tr_hx": tr_hx, "tr_hg": tr_hg}
+
+
+def score(tr_hx, tr_hg):
+    """s = tr(H_G) * tr(H_X)   [KronQ-hyper] Method: sensitivity score."""
+    return float(tr_hg) * float(tr_hx)
+
+
+# ------------------------------------------------------------------------------------------
+# Damped inverse factor
+# ------------------------------------------------------------------------------------------
+
+def damping(h, damp_rel: float) -> float:
+    return float(damp_rel) * float(np.mean(np.diag(h)))
+
+
+def cholinv(h, damp_rel: float = 0.01):
+    """K upper triangular with K^T K = (H + lambda I)^-1, lambda = damp_rel * mean diag H.
+
+    Plain three-step route: Cholesky of H + lambda I, the explicit inverse, then the upper
+    Cholesky factor of that inverse. K's rows are the "[H_X^-1]_p,p+1:" rows of the column
+    update ([KronQ-hyper] Method: OBS update).
+    """
+    h = np.asarray(h, dtype=np.float64)
+    d = h.shape[0]
+    a = h + damping(h, damp_rel) * np.eye(d)
+    try:
+        l = np.linalg.cholesky(a)
+    except np.linalg.LinAlgError as e:
+        raise NotPositiveDefinite(str(e))
+    linv = sla.solve_triangular(l, np.eye(d), lower=True)
+    ainv = linv.T @ linv
+    ainv = 0.5 * (ainv + ainv.T)
+    try:
+        l2 = np.linalg.cholesky(ainv)
+    except np.linalg.LinAlgError as e:
+        raise NotPositiveDefinite(str(e))
+    return l2.T.copy()
+
+
+def p_matrix(dxx, k):
+    """GPTAQ correction matrix P = striu(D K^T) K (strictly upper triangular)."""
+    m = np.asarray(dxx, dtype=np.float64) @ np.asarray(k, dtype=np.float64).T
+    return np.triu(m, 1) @ k
+
+
+# ------------------------------------------------------------------------------------------
+# Grid and column-wise solve
+# ------------------------------------------------------------------------------------------
+
+def grid(w, bits: int):
+    """Per-row asymmetric min-max grid; decisions in fp32. Returns (scale, zero) as float32."""
+    w = np.asarray(w)
+    maxq = np.float32(2 ** bits - 1)
+    lo = w.min(axis=1).astype(np.float32)
+    hi = w.max(axis=1).astype(np.float32)
+    scale = ((hi - lo) / maxq).astype(np.float32)
+    scale = np.where(hi == lo, np.float32(1.0), scale).astype(np.float32)
+    zero = np.rint((-lo) / scale).astype(np.float32)
+    return scale, zero
+
+
+def quantize_codes(col, scale, zero, bits):
+    """codes = clamp(rint(w/scale) + zero, 0, 2^b - 1), division and rounding in fp32."""
+    maxq = np.float32(2 ** bits - 1)
+    t = np.rint(col.astype(np.float32) / scale)
+    return np.clip(t + zero, np.float32(0), maxq).astype(np.float32)
+
+
+def dequantize(codes, scale, zero):
+    return (scale * (codes - zero)).astype(np.float32)
+
+
+def quantize_layer(w, k, dxx=None, bits: int = 4, follow_codes=None, tie_tol: float = 1e-3):
+    """Column-wise OBS / GPTAQ solve onto the per-row grid, literally, one column at a time.
+
+    [KronQ-hyper] Method, OBS update:
+        dW_:,p+1: = -delta_p [H_X^-1]_p,p+1: + W_:,p [P]_p,p+1:
+    with delta_p = (w_p - deq(q(w_p))) / K_pp, [H_X^-1]_p,p+1: = K_p,p+1:, W_:,p the weights
+    before quantization (after incoherence processing), P = p_matrix(dxx, k).
+
+    follow_codes: optional array of codes from another implementation. Where this oracle's
+    value sits within tie_tol grid units of a rounding boundary (a half-integer of w/scale) it
+    adopts that code instead of its own, and records a near-tie. Every other code is its own.
+    Returns dict: codes (uint8), scale, zero, w_hat (fp64), near_tie (bool mask),
+    pre (fp64: each column's value just before it was quantized).
+    """
+    w0 = np.asarray(w, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    d_out, d_in = w0.shape
+    scale, zero = grid(w0, bits)
+    p_mat = None if dxx is None else p_matrix(dxx, k)
+    cur = w0.copy()
+    codes = np.zeros((d_out, d_in), dtype=np.uint8)
+    near = np.zeros((d_out, d_in), dtype=bool)
+    pre = np.zeros((d_out, d_in))
+    for p in range(d_in):
+        col = cur[:, p].copy()
+        pre[:, p] = col
+        c = quantize_codes(col, scale, zero, bits)
+        if follow_codes is not None:
+            t = col / scale.astype(np.float64)
+            dist = np.abs(t - (np.floor(t) + 0.5))
+            tie = dist <= tie_tol
+            near[:, p] = tie
+            c = np.where(tie, np.asarray(follow_codes)[:, p].astype(np.float32), c)
+        dq = dequantize(c, scale, zero).astype(np.float64)
+        delta = (col - dq) / k[p, p]
+        if p + 1 < d_in:
+            cur[:, p + 1:] -= np.outer(delta, k[p, p + 1:])
+            if p_mat is not None:
+                cur[:, p + 1:] += np.outer(w0[:, p], p_mat[p, p + 1:])
+        cur[:, p] = dq
+        codes[:, p] = c.astype(np.uint8)
+    return {"codes": codes, "scale": scale, "zero": zero, "w_hat": cur, "near_tie": near,
+            "pre": pre}
+
+
+# ------------------------------------------------------------------------------------------
+# Objective and diagnostics
+# ------------------------------------------------------------------------------------------
+
+def objective(w, w_hat, hx, hg=None, dxx=None):
+    """tr[H_G dW H_X dW^T] + 2 tr[H_G W D dW^T], dW = W - W^ (H_G = I when not given).
+
+    [KronQ-hyper] Method: Kronecker-factored objective and its asymmetric form.
+    """
+    w = np.asarray(w, dtype=np.float64)
+    dw = w - np.asarray(w_hat, dtype=np.float64)
+    hx = np.asarray(hx, dtype=np.float64)
+    hg_ = np.eye(w.shape[0]) if hg is None else np.asarray(hg, dtype=np.float64)
+    val = np.trace(hg_ @ dw @ hx @ dw.T)
+    if dxx is not None:
+        val += 2.0 * np.trace(hg_ @ w @ np.asarray(dxx, dtype=np.float64) @ dw.T)
+    return float(val)
+
+
+def mu_incoherence(h):
+    """mu(H)/sqrt(d) = max_ij |Q_ij| over an orthonormal eigenbasis Q of H."""
+    _, q = np.linalg.eigh(np.asarray(h, dtype=np.float64))
+    return float(np.abs(q).max())
+
+
+def cv_norms(w):
+    """(CV_in, CV_out): coefficient of variation of column norms and of row norms of W."""
+    w = np.asarray(w, dtype=np.float64)
+    c = np.sqrt((w * w).sum(axis=0))
+    r = np.sqrt((w * w).sum(axis=1))
+    return float(c.std() / c.mean()), float(r.std() / r.mean())
+
+
+# ------------------------------------------------------------------------------------------
+# Mixed-precision allocation
+# ------------------------------------------------------------------------------------------
+
+def score_allocate(tr_hx, tr_hg, n_params, choices, avg_bits):
+    """Scores s_l = tr(H_G) tr(H_X) and a greedy bit allocation under an average-bit budget.
+
+    [KronQ-hyper] Method: sublayers with larger s get higher bit widths;
+    [KronQ-gist] Experimental results: the higher-scored sublayer is upgraded first.
+    Order: s descending, ties by index ascending. Budget T = floor(avg_bits * sum n) bits.
+    Every sublayer starts at min(choices); in that order each takes the largest choice that
+    keeps the total within T.
+    Returns (scores, bits).
+    """
+    tr_hx = [float(v) for v in tr_hx]
+    tr_hg = [float(v) for v in tr_hg]
+    n_params = [int(v) for v in n_params]
+    L = len(tr_hx)
+    s = [tr_hg[l] * tr_hx[l] for l in range(L)]
+    if any(math.isnan(v) for v in s):
+        raise ValueError("NaN score")
+    total = sum(n_params)
+    budget = int(math.floor(float(avg_bits) * float(total)))
+    ch = sorted(set(int(c) for c in choices))
+    bits = [ch[0]] * L
+    used = ch[0] * total
+    if used > budget:
+        raise ValueError("budget below the smallest bit width")
+    order = sorted(range(L), key=lambda l: (-s[l], l))
+    for l in order:
+        for b in reversed(ch):
+            if b <= bits[l]:
+                break
+            extra = (b - bits[l]) * n_params[l]
+            if used + extra <= budget:
+                used += extra
+                bits[l] = b
+                break
+    return s, bits
