@@ -1,0 +1,468 @@
+"""KronQ layer-path benchmark on B200.
+
+One step = the whole hot path over one LLaMA-2-7B-shaped transformer block (7 sublayers:
+q/k/v/o 4096x4096, gate/up 11008x4096, down 4096x11008; 262144 calibration tokens; 4-bit
+per-channel grid; BiIP on; X~ = X so the drift term is off):
+  Kronecker-factor sums for the 4 distinct inputs (q/k/v share one) and the 7 output-gradient
+  streams -> BiIP of every sublayer -> traces to the host -> scores and bit allocation ->
+  damped inverse factor -> column solve of every sublayer.
+Metric: quantized weight params/s (whole job: params of all ranks' blocks / max step time).
+Each rank quantizes its own block (weak scaling, no collective on the data path).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+--impl reference times the fp64 CPU oracle on a bounded sample of the same workload (see
+oracle_sample) on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "llama2_7b_block"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="kronq", choices=["kronq", "reference"])
+    ap.add_argument("--tokens", type=int, default=None, help=argparse.SUPPRESS)
+    ap.add_argument("--no-e2e", action="store_true", help=argparse.SUPPRESS)
+    ap.add_argument("--no-cpu-baseline", action="store_true", help=argparse.SUPPRESS)
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------------- oracle
+
+def oracle_sample(seconds_hint: float = 12.0):
+    """Time the fp64 oracle on a bounded sample of the block and scale it to one full step.
+
+    Sample: q_proj (4096 x 4096) with 4096 calibration tokens for the statistics, the whole
+    BiIP and damped inverse factor of that sublayer, and the column solve of 32 output rows.
+    Each stage's time is scaled to the full block by its work ratio (accumulation ~ N d^2 per
+    stream, BiIP ~ dense Hadamard cost, inverse ~ d^3, solve ~ d_out d_in^2).
+    Returns (estimated seconds per full step, description, threads).
+    """
+    import numpy as np
+    import torch
+    from threadpoolctl import threadpool_info
+
+    from oracle import kronq_oracle as O
+    from post_quantization_b200 import synth
+
+    wl = synth.WORKLOADS[WORKLOAD]
+    d = 4096
+    n_s = 4096
+    rows = 32
+    tag = ("bench-oracle",)
+    x = synth.correlated_x(n_s, d, synth.seed_for(tag, "X")).double().numpy()
+    g = synth.gradients(n_s, d, synth.seed_for(tag, "G")).double().numpy()
+    w = synth.weight(d, d, synth.seed_for(tag, "W")).double().numpy()
+    si = synth.rademacher(d, synth.seed_for(tag, "si")).numpy()
+    so = synth.rademacher(d, synth.seed_for(tag, "so")).numpy()
+
+    t0 = time.perf_counter()
+    hx, hg, _ = O.accumulate(x, None, g)
+    t_acc = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    b = O.biip(w, hx, hg, None, 1.0 / n_s, si, so, O.BIIP_FULL)
+    t_biip = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    k = O.cholinv(b["hx"], 0.01)
+    t_chol = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    O.quantize_layer(b["w"][:rows], k, None, wl.bits)
+    t_q = time.perf_counter() - t0
+
+    N = wl.n_tokens
+    # accumulation: this sample did one X and one G stream of width 4096 over n_s tokens
+    acc_work = sum(N * dd * dd for dd in wl.streams().values()) + \
+        sum(N * s.d_out * s.d_out for s in wl.sublayers)
+    acc_scale = acc_work / (2 * n_s * d * d)
+
+    def biip_cost(s):
+        bi = s.d_in & -s.d_in; bo = s.d_out & -s.d_out
+        return s.d_out * s.d_in * (bi + bo) + 2 * s.d_in * s.d_in * bi + 2 * s.d_out * s.d_out * bo
+
+    ref = synth.Sublayer("q", d, d, "x")
+    biip_scale = sum(biip_cost(s) for s in wl.sublayers) / biip_cost(ref)
+    chol_scale = sum(s.d_in ** 3 for s in wl.sublayers) / d ** 3
+    q_scale = sum(s.d_out * s.d_in ** 2 for s in wl.sublayers) / (rows * d * d)
+    est = t_acc * acc_scale + t_biip * biip_scale + t_chol * chol_scale + t_q * q_scale
+    threads = 0
+    for info in threadpool_info():
+        threads = max(threads, int(info.get("num_threads", 0)))
+    desc = (f"q_proj 4096x4096: statistics over {n_s} tokens, full BiIP and inverse factor, "
+            f"column solve of {rows} rows; stage times ({t_acc:.2f}s, {t_biip:.2f}s, "
+            f"{t_chol:.2f}s, {t_q:.2f}s) scaled by work ratios ({acc_scale:.0f}, "
+            f"{biip_scale:.1f}, {chol_scale:.1f}, {q_scale:.0f}) to one {WORKLOAD} step")
+    return est, desc, threads or (os.cpu_count() or 1), t_acc + t_biip + t_chol + t_q
+
+
+# ---------------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    def __init__(self, index: int):
+        self.index = index
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 8:
+                self.samples.append(parts)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        if not self.samples:
+            return None
+        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
+        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for s in self.samples:
+            for nm, v in zip(names, s[4:8]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------------- GPU arm
+
+class Block:
+    """Device-resident inputs and buffers of one block; `step` runs the whole path."""
+
+    def __init__(self, wl, rank, device, n_tokens, ws):
+        import torch
+
+        from post_quantization_b200 import synth
+        self.wl = wl
+        self.dev = device
+        self.n = n_tokens
+        self.ws = ws
+        tag = (WORKLOAD, "rank", rank)
+        self.x = {name: synth.correlated_x(n_tokens, d, synth.seed_for(tag, name, "X"),
+                                           device=device)
+                  for name, d in wl.streams().items()}
+        self.g = {s.name: synth.gradients(n_tokens, s.d_out, synth.seed_for(tag, s.name, "G"),
+                                          device=device) for s in wl.sublayers}
+        self.w = {s.name: synth.weight(s.d_out, s.d_in, synth.seed_for(tag, s.name, "W"),
+                                       dtype=wl.w_dtype, device=device) for s in wl.sublayers}
+        self.si = {s.name: synth.rademacher(s.d_in, synth.seed_for(tag, s.name, "si"),
+                                            device=device) for s in wl.sublayers}
+        self.so = {s.name: synth.rademacher(s.d_out, synth.seed_for(tag, s.name, "so"),
+                                            device=device) for s in wl.sublayers}
+        self.hx = {name: torch.zeros(d, d, device=device) for name, d in wl.streams().items()}
+        self.hg = {s.name: torch.zeros(s.d_out, s.d_out, device=device) for s in wl.sublayers}
+        self.results = {}
+        self.acc_events = []        # (start, end, flops) of each statistics call
+        self.bits = None
+
+    def input_bytes(self):
+        tot = 0
+        for t in list(self.x.values()) + list(self.g.values()) + list(self.w.values()):
+            tot += t.numel() * t.element_size()
+        return tot
+
+    def step(self, time_acc=False, x_src=None, g_src=None):
+        import torch
+
+        from post_quantization_b200 import kronq as K
+        from post_quantization_b200 import pipeline as P
+        wl = self.wl
+        x = x_src or self.x
+        g = g_src or self.g
+        for name, h in self.hx.items():
+            h.zero_()
+            if time_acc:
+                e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+            P.accumulate(xq=x[name], hx_sum=h, ws=self.ws)
+            if time_acc:
+                e1.record()
+                d = h.shape[0]
+                self.acc_events.append((e0, e1, self.n * d * (d + 1)))
+        for s in wl.sublayers:
+            h = self.hg[s.name]
+            h.zero_()
+            if time_acc:
+                e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+            P.accumulate(g=g[s.name], hg_sum=h, ws=self.ws)
+            if time_acc:
+                e1.record()
+                d = h.shape[0]
+                self.acc_events.append((e0, e1, self.n * d * (d + 1)))
+        inv_n = 1.0 / self.n
+        for s in wl.sublayers:
+            self.results[s.name] = P.biip(self.w[s.name], self.hx[s.x_stream], self.hg[s.name],
+                                          None, inv_n, self.si[s.name], self.so[s.name],
+                                          K.BIIP_FULL, ws=self.ws)
+        tr = torch.stack([self.results[s.name].tr for s in wl.sublayers]).cpu()
+        choices = wl.extra.get("choices", (wl.bits,))
+        avg = wl.extra.get("avg_bits", float(wl.bits))
+        _, self.bits = K.kronq_score_allocate(tr[:, 0].tolist(), tr[:, 1].tolist(),
+                                              [s.d_out * s.d_in for s in wl.sublayers], choices,
+                                              avg)
+        for s, b in zip(wl.sublayers, self.bits):
+            r = self.results[s.name]
+            P.cholinv(r, 0.01, ws=self.ws)
+            P.quantize(r, b, ws=self.ws)
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    from post_quantization_b200 import build
+    from post_quantization_b200 import kronq as K
+    from post_quantization_b200 import pipeline as P
+    from post_quantization_b200 import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=600))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    K.load_library()
+    K.kronq_device_check()
+
+    wl = synth.WORKLOADS[WORKLOAD]
+    n_tok = args.tokens or wl.n_tokens
+    ws = P.Workspace(dev)
+    blk = Block(wl, rank, dev, n_tok, ws)
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        blk.step()
+    barrier()
+    assert K.kronq_device_error() == 0
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    launches0 = K.kronq_launch_count()
+    barrier()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record()
+    for _ in range(args.steps):
+        blk.step(time_acc=True)
+    t_end.record()
+    barrier()
+    clk = clocks.stop()
+    launches = K.kronq_launch_count() - launches0
+    elapsed = t_start.elapsed_time(t_end) / 1e3
+    acc_ms = [a.elapsed_time(b) for a, b, _ in blk.acc_events]
+    acc_flops = [f for _, _, f in blk.acc_events]
+    t = torch.tensor([elapsed], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    elapsed_max = float(t)
+    params = wl.params_per_block * world
+    value = params * args.steps / elapsed_max
+
+    # ---- end to end: host inputs (pinned), host->device copies and the result read-back
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(blk, args, world, dist if world > 1 else None, barrier)
+
+    result = None
+    if rank == 0:
+        import json as _json
+        peaks = {}
+        pp = os.path.join(ROOT, "MEASURED_PEAKS.json")
+        if os.path.exists(pp):
+            peaks = _json.load(open(pp))
+        peak = peaks.get("bf16_tflops_sustained")
+        peak_src = "measured (sustained bf16)"
+        if not peak:
+            peak = 1400.0
+            peak_src = "fallback (sustained bf16)"
+        achieved = sum(acc_flops) / (sum(acc_ms) / 1e3) / 1e12
+        acc_tflops = sum(acc_flops) / (sum(acc_ms) / 1e3) / 1e12
+        result = {
+            "metric": "quantized weight params/s (BiIP+GPTAQ solve); H_X/H_G accumulate TFLOP/s",
+            "value": value,
+            "unit": "params/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": elapsed_max / args.steps * 1e3,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16 statistics, fp32 solve",
+            "data": "synthetic (seeded LLaMA-shaped activations, gradients and weights)",
+            "config": {"workload": "LLaMA-2-7B-shaped block: q/k/v/o 4096x4096, gate/up "
+                                   "11008x4096, down 4096x11008; 262144 tokens; 4-bit "
+                                   "per-channel grid; BiIP on; drift term off",
+                       "tokens": n_tok, "params_per_block": wl.params_per_block,
+                       "parallelism": f"one block per GPU x{world}",
+                       "l2": "inputs (34 GB) larger than L2"},
+            "accumulate_tflops": acc_tflops,
+            "roofline": {"bound": "tensor", "kernel": "accumulate_tc_kernel",
+                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "peak_source": peak_src, "traffic": None},
+            "gpu_launches": launches,
+            "clocks": clk,
+            "e2e": e2e,
+        }
+        if not args.no_cpu_baseline:
+            est, desc, threads, spent = oracle_sample()
+            result["cpu_baseline"] = {"value": wl.params_per_block / est, "unit": "params/s",
+                                      "cores": threads, "kind": "oracle", "sample": desc,
+                                      "sample_seconds": spent}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
+
+
+def run_e2e(blk, args, world, dist, barrier):
+    """Same step through the same API, inputs starting in pinned host memory every step."""
+    import torch
+    def pinned(v):
+        h = torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
+        h.copy_(v)
+        return h
+
+    host_x = {k: pinned(v) for k, v in blk.x.items()}
+    host_g = {k: pinned(v) for k, v in blk.g.items()}
+    dev_x = {k: torch.empty_like(v) for k, v in blk.x.items()}
+    dev_g = {k: torch.empty_like(v) for k, v in blk.g.items()}
+    # free the resident copies to keep device memory flat
+    blk.x = dev_x
+    blk.g = dev_g
+    h2d = sum(t.numel() * t.element_size() for t in list(host_x.values()) + list(host_g.values()))
+    d2h = 0
+
+    def one():
+        nonlocal d2h
+        for k, v in host_x.items():
+            dev_x[k].copy_(v, non_blocking=True)
+        for k, v in host_g.items():
+            dev_g[k].copy_(v, non_blocking=True)
+        blk.step()
+        outs = []
+        for s in blk.wl.sublayers:
+            r = blk.results[s.name]
+            outs.append(r.codes.to("cpu", non_blocking=True))
+            outs.append(r.scale.to("cpu", non_blocking=True))
+            outs.append(r.zero.to("cpu", non_blocking=True))
+        torch.cuda.current_stream().synchronize()
+        d2h = sum(o.numel() * o.element_size() for o in outs)
+
+    one()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
+    steps = max(1, min(args.steps, 3))
+    e0.record()
+    for _ in range(steps):
+        one()
+    e1.record()
+    barrier()
+    el = e0.elapsed_time(e1) / 1e3
+    t = torch.tensor([el], dtype=torch.float64, device=blk.dev)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    value = blk.wl.params_per_block * world * steps / float(t)
+    return {"value": value, "unit": "params/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps}
+
+
+# ---------------------------------------------------------------------------------- reference
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    from post_quantization_b200 import synth
+    wl = synth.WORKLOADS[WORKLOAD]
+    times = []
+    threads = 1
+    desc = ""
+    for i in range(args.warmup + args.steps):
+        est, desc, threads, spent = oracle_sample()
+        if i >= args.warmup:
+            times.append(est)
+    est = statistics.mean(times)
+    value = wl.params_per_block / est
+    return {
+        "impl": "reference",
+        "metric": "quantized weight params/s (BiIP+GPTAQ solve); H_X/H_G accumulate TFLOP/s",
+        "value": value, "unit": "params/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": est * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded LLaMA-shaped activations, gradients and weights)",
+        "config": {"workload": "LLaMA-2-7B-shaped block: q/k/v/o 4096x4096, gate/up "
+                               "11008x4096, down 4096x11008; 262144 tokens; 4-bit per-channel "
+                               "grid; BiIP on; drift term off"},
+        "cpu_baseline": {"value": value, "unit": "params/s", "cores": threads, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "params/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        res = run_reference(args)
+    else:
+        res = run_gpu(args)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,218 @@
+/*
+ * kronq.h - C ABI of the KronQ per-layer quantization hot path on NVIDIA B200 (sm_100a).
+ *
+ * KronQ quantizes one linear layer y = W x (W: d_out x d_in) with a Kronecker-factored
+ * Hessian H ~ H_X (x) H_G, bidirectional incoherence processing (BiIP), a damped inverse
+ * Cholesky factor and a column-wise OBS/GPTAQ solve, and ranks sublayers by
+ * s = tr(H_G) * tr(H_X) for mixed precision. Sources of each operation are cited per call:
+ *   [KronQ-hyper] "KronQ: LLM Quantization via Kronecker-Factored Hessian", hyper.ai summary,
+ *                 Method section (the page that prints the equations);
+ *   [KronQ-gist]  the same paper, gist.science technical summary (Methodology, Results).
+ *
+ * Conventions shared by every call
+ *   - Matrices are row-major. Pointers marked (device) are CUDA device pointers owned by the
+ *     caller; (host) pointers are ordinary host memory owned by the caller. The library never
+ *     frees or retains a pointer after the call returns.
+ *   - The library allocates no device memory. Calls that need scratch space take a caller
+ *     workspace (device, 256-byte aligned) whose minimum size is returned by the matching
+ *     kronq_*_workspace_size() query. A smaller workspace gives KRONQ_ERR_WORKSPACE.
+ *   - Device work is enqueued on `stream` and is asynchronous unless stated otherwise. A status
+ *     other than KRONQ_OK means nothing was enqueued (argument errors) or a CUDA launch failed;
+ *     faults of earlier asynchronous work surface as KRONQ_ERR_CUDA at a later call.
+ *   - bf16 arrays are IEEE bfloat16 (1 sign, 8 exponent, 7 mantissa bits) stored as uint16.
+ *   - kronq_last_error_detail() returns a thread-local text of the last failure of this thread.
+ *   - All entry points are safe to call from several host threads on distinct streams; calls
+ *     that share output buffers must be ordered by the caller.
+ */
+#ifndef KRONQ_H_
+#define KRONQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KRONQ_API __attribute__((visibility("default")))
+#else
+#define KRONQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream; binary-compatible with cudaStream_t / CUstream (NULL = legacy stream). */
+typedef struct CUstream_st* kronq_stream_t;
+
+typedef enum kronq_status {
+  KRONQ_OK = 0,
+  KRONQ_ERR_INVALID_ARG = 1,  /* null pointer, bad enum, misaligned pointer or stride */
+  KRONQ_ERR_SHAPE = 2,        /* non-positive or inconsistent sizes */
+  KRONQ_ERR_NOT_PD = 3,       /* damped H_X not positive definite (kronq_cholinv) */
+  KRONQ_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+  KRONQ_ERR_WORKSPACE = 5,    /* workspace pointer null/misaligned or smaller than required */
+  KRONQ_ERR_UNSUPPORTED = 6,  /* device is not sm_100 or a parameter is outside the supported range */
+  KRONQ_ERR_TIMEOUT = 7       /* a kernel gave up a bounded wait (see kronq_device_error) */
+} kronq_status;
+
+/* Element types of the weight input of kronq_biip. */
+enum { KRONQ_DTYPE_BF16 = 0, KRONQ_DTYPE_F32 = 1 };
+
+/* Flags of kronq_biip ([KronQ-hyper] Method, BiIP equations). */
+enum {
+  KRONQ_BIIP_SCALE_IN = 1,    /* W <- W S_X,  S_X = diag(H_X,jj / |W_:,j|^2)^(1/4)          */
+  KRONQ_BIIP_SCALE_OUT = 2,   /* W <- S_G W,  S_G = diag(H_G,ii / |W_i,:|^2)^(1/4)          */
+  KRONQ_BIIP_ROTATE_IN = 4,   /* W <- W V^T,  H_X <- V H_X V^T, dXX^T <- V dXX^T V^T         */
+  KRONQ_BIIP_ROTATE_OUT = 8,  /* W <- U W,    H_G <- U H_G U^T                               */
+  KRONQ_BIIP_WRITE_HG = 16,   /* also write the normalised, transformed H_G into `hg`        */
+  KRONQ_BIIP_FULL = 15        /* the four transforms of BiIP                                  */
+};
+
+/* Flags of kronq_cholinv. */
+enum { KRONQ_CHOLINV_SYNC = 1 };
+
+KRONQ_API const char* kronq_status_string(kronq_status status);
+KRONQ_API const char* kronq_last_error_detail(void);
+KRONQ_API int kronq_version(void);
+
+/* Checks that the current CUDA device is a compute-capability 10.0 (B200-class) GPU. */
+KRONQ_API kronq_status kronq_device_check(void);
+
+/* Number of kernels this library has launched in this process (all devices, all threads). */
+KRONQ_API uint64_t kronq_launch_count(void);
+
+/* Reads and clears the device-side error word (bounded waits that gave up). Synchronizes
+ * `stream`. *code_out = 0 when no kernel reported an error since the last call. */
+KRONQ_API kronq_status kronq_device_error(int32_t* code_out, kronq_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * 1. kronq_accumulate - Kronecker-factor sums over calibration tokens.
+ *
+ * [KronQ-hyper] Method: for y = W x with g = dL/dy, the empirical Fisher is
+ * E[x x^T (x) g g^T] ~ H_X (x) H_G with H_X = E[x x^T], H_G = E[g g^T]; the asymmetric
+ * (GPTAQ) objective adds the input-drift term dX X^T. This call adds, over n tokens,
+ *     hx_sum  += X~^T X~            (d_in x d_in)   if hx_sum  != NULL
+ *     hg_sum  += G^T G              (d_out x d_out) if hg_sum  != NULL
+ *     dxx_sum += (X - X~)^T X~      (d_in x d_in)   if dxx_sum != NULL
+ * where X~ (xq) is the input the quantized layer sees and X (xfp) the full-precision input.
+ * The sums are un-normalised (divide by the total token count later, see kronq_biip).
+ *
+ *   xq, xfp  (device, bf16) n x d_in, row stride ld_xq / ld_xfp elements (one token per row)
+ *   g        (device, bf16) n x d_out, row stride ld_g
+ *   hx_sum, dxx_sum (device, fp32) d_in x d_in contiguous; hg_sum d_out x d_out contiguous.
+ *            Both triangles of hx_sum / hg_sum are valid on return (symmetric).
+ *   Requirements: strides >= width, stride*2 bytes a multiple of 16, base pointers 16-byte
+ *   aligned; hx_sum needs xq; dxx_sum needs xq and xfp; hg_sum needs g. n = 0 is a no-op.
+ *   Accumulation: bf16 products, fp32 sums on tcgen05 tensor cores; the drift X - X~ is split
+ *   into two bf16 terms so that (X - X~)^T X~ is formed without rounding X - X~.
+ * ------------------------------------------------------------------------------------- */
+KRONQ_API size_t kronq_accumulate_workspace_size(int64_t n, int32_t d_in, int32_t d_out, int with_dxx);
+KRONQ_API kronq_status kronq_accumulate(const void* xq, int64_t ld_xq, const void* xfp, int64_t ld_xfp,
+                              const void* g, int64_t ld_g, int64_t n, int32_t d_in,
+                              int32_t d_out, float* hx_sum, float* hg_sum, float* dxx_sum,
+                              void* workspace, size_t workspace_bytes, kronq_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * 2. kronq_biip - normalisation and bidirectional incoherence processing of one sublayer.
+ *
+ * [KronQ-hyper] Method, BiIP equations:
+ *     W <- S_G W S_X,  S_X = diag([H_X]_jj / |W_:,j|^2)^(1/4),  S_G = diag([H_G]_ii / |W_i,:|^2)^(1/4)
+ *     W <- U W V^T,  H_X <- V H_X V^T,  H_G <- U H_G U^T,  dXX^T <- V dXX^T V^T
+ * with U, V random-sign Hadamard transforms, here U = (1/sqrt(b)) (I (x) H_b) diag(sign_out)
+ * (Sylvester H_b, b = largest power of two dividing d_out) and V likewise on the input side.
+ * The Hessians follow the diagonal scaling as H_X <- S_X^-1 H_X S_X^-1 (same for dXX^T) and
+ * H_G <- S_G^-1 H_G S_G^-1, which leaves tr[H_G dW H_X dW^T] unchanged. Both scales use the
+ * original W; a zero norm or zero diagonal gives scale 1. Also returns the traces used by the
+ * sensitivity score s = tr(H_G) tr(H_X) ([KronQ-hyper] Method: sensitivity), taken after BiIP.
+ *
+ *   w        (device) d_out x d_in, w_dtype KRONQ_DTYPE_BF16 or KRONQ_DTYPE_F32; not modified
+ *   w_out    (device, fp32) d_out x d_in: W' = U S_G W S_X V^T
+ *   hx       (device, fp32) d_in x d_in: in: raw sum X~^T X~; out: V S_X^-1 (inv_n hx) S_X^-1 V^T
+ *   hg       (device, fp32) d_out x d_out raw sum G^T G, or NULL (then SCALE_OUT is invalid).
+ *            Read-only unless KRONQ_BIIP_WRITE_HG, in which case it is replaced by
+ *            U S_G^-1 (inv_n hg) S_G^-1 U^T.
+ *   dxx      (device, fp32) d_in x d_in raw drift sum or NULL; out: V S_X^-1 (inv_n dxx) S_X^-1 V^T
+ *   inv_n    1 / total token count
+ *   sign_in  (device, int8 +-1) d_in; needed with ROTATE_IN. sign_out likewise d_out.
+ *   s_x, s_g (device, fp32) d_in / d_out diagonal scales (1 where the flag is off)
+ *   tr_hx, tr_hg (device, fp64, one element each): traces after BiIP; tr_hg may be NULL and is
+ *            left untouched when hg is NULL.
+ * ------------------------------------------------------------------------------------- */
+KRONQ_API size_t kronq_biip_workspace_size(int32_t d_out, int32_t d_in);
+KRONQ_API kronq_status kronq_biip(const void* w, int32_t w_dtype, float* w_out, float* hx, float* hg,
+                        float* dxx, double inv_n, const int8_t* sign_in, const int8_t* sign_out,
+                        int32_t d_out, int32_t d_in, uint32_t flags, float* s_x, float* s_g,
+                        double* tr_hx, double* tr_hg, void* workspace, size_t workspace_bytes,
+                        kronq_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * 3. kronq_cholinv - damped inverse Cholesky factor.
+ *
+ * [KronQ-hyper] Method, OBS update: the rows "[H_X^-1]_p,p+1:" of the column update are the
+ * rows of K, the upper-triangular factor with K^T K = (H_X + lambda I)^-1 (positive diagonal),
+ * lambda = damp_rel * mean(diag H_X). Computed as a blocked reverse-order Cholesky
+ * H_X + lambda I = R R^T (R upper) followed by a blocked triangular inverse K = R^-1.
+ *
+ *   h_to_k   (device, fp32) d x d, in: symmetric H_X (upper triangle read); out: K in the upper
+ *            triangle, zeros below the diagonal.
+ *   info     (device, int32): -1 when positive definite, else the index of the first pivot that
+ *            was not positive (pivots are taken from the last index down).
+ *   flags    KRONQ_CHOLINV_SYNC: synchronize `stream` and return KRONQ_ERR_NOT_PD when
+ *            info >= 0. Without it the call is asynchronous and the caller reads info.
+ *   On failure K is unspecified.
+ * ------------------------------------------------------------------------------------- */
+KRONQ_API size_t kronq_cholinv_workspace_size(int32_t d);
+KRONQ_API kronq_status kronq_cholinv(float* h_to_k, int32_t d, float damp_rel, int32_t* info,
+                           uint32_t flags, void* workspace, size_t workspace_bytes,
+                           kronq_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * 4. kronq_quantize_layer - column-wise OBS / GPTAQ solve onto a b-bit per-row grid.
+ *
+ * [KronQ-hyper] Method, OBS update (H_G cancels, Proposition 1 - the solve takes no H_G):
+ *     dW_:,p+1: = -delta_p [H_X^-1]_p,p+1: + W_:,p P_p,p+1:
+ * with delta_p = (w_p - deq(q(w_p))) / K_pp, K from kronq_cholinv and P the GPTAQ correction
+ * matrix, read as P = striu(D K^T) K with D the processed drift term (P = 0 when dxx is NULL).
+ * Because the P term uses the weights before any update, it is applied up front: the solve runs
+ * on W (I + P) and then proceeds in 128-column blocks with lazy trailing updates.
+ * Grid: per output row, lo/hi = min/max of W (before the solve), scale = (hi - lo)/(2^bits - 1)
+ * (1 if hi == lo), zero = rint(-lo/scale), code = clamp(rint(w/scale) + zero, 0, 2^bits - 1),
+ * deq = scale * (code - zero), all in fp32 with round-half-to-even.
+ *
+ *   w        (device, fp32) d_out x d_in processed weights W' (from kronq_biip); not modified
+ *   k        (device, fp32) d_in x d_in, upper triangle = K (from kronq_cholinv)
+ *   dxx      (device, fp32) d_in x d_in processed drift term, or NULL
+ *   bits     2..8;  block: column block width, 128 (others give KRONQ_ERR_UNSUPPORTED)
+ *   codes    (device, uint8) d_out x d_in;  scale, zero (device, fp32) d_out each
+ *   w_hat    (device, fp32) d_out x d_in: dequantized weights W^ (also the solve's working copy)
+ * ------------------------------------------------------------------------------------- */
+KRONQ_API size_t kronq_quantize_layer_workspace_size(int32_t d_out, int32_t d_in, int32_t block,
+                                           int with_dxx);
+KRONQ_API kronq_status kronq_quantize_layer(const float* w, const float* k, const float* dxx,
+                                  int32_t d_out, int32_t d_in, int32_t bits, int32_t block,
+                                  uint8_t* codes, float* scale, float* zero, float* w_hat,
+                                  void* workspace, size_t workspace_bytes,
+                                  kronq_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * 5. kronq_score_allocate - sensitivity scores and mixed-precision bit allocation (host).
+ *
+ * [KronQ-hyper] Method: s_l = tr(H_G^(l)) * tr(H_X^(l)), computed after BiIP; sublayers with a
+ * larger s get more bits. [KronQ-gist] Results: the higher-scored sublayer is upgraded first.
+ * Rule: budget T = floor(avg_bits * sum n_l) bits; every sublayer starts at min(choices);
+ * sublayers are visited by s descending (ties: lower index first) and each takes the largest
+ * choice that keeps the total <= T. Deterministic, integer budget arithmetic.
+ *
+ *   tr_hx, tr_hg (host, fp64) L each; n_params (host, int64) L; choices (host) n_choices widths
+ *   score_out (host, fp64) L, may be NULL; bits_out (host, int32) L
+ *   Errors: KRONQ_ERR_INVALID_ARG for a NaN score or a budget below L * min(choices).
+ * ------------------------------------------------------------------------------------- */
+KRONQ_API kronq_status kronq_score_allocate(const double* tr_hx, const double* tr_hg,
+                                  const int64_t* n_params, int32_t L, const int32_t* choices,
+                                  int32_t n_choices, double avg_bits, double* score_out,
+                                  int32_t* bits_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KRONQ_H_ */

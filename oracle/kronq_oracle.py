@@ -56,6 +56,7 @@ closed forms, brute force or textbook special cases; none is "parity unpinned".
 """
 from __future__ import annotations
 
+import functools
 import math
 
 import numpy as np
@@ -125,15 +126,22 @@ def hadamard_block_size(d: int) -> int:
     return d & (-d)
 
 
-def sylvester(b: int) -> np.ndarray:
-    """Sylvester Hadamard matrix of order b: [H_b]_ij = (-1)^popcount(i & j)."""
+@functools.lru_cache(maxsize=16)
+def _sylvester_cached(b: int) -> np.ndarray:
     i = np.arange(b)
     pc = np.zeros((b, b), dtype=np.int64)
     a = i[:, None] & i[None, :]
     while np.any(a):
         pc += a & 1
         a = a >> 1
-    return np.where(pc % 2 == 0, 1.0, -1.0)
+    h = np.where(pc % 2 == 0, 1.0, -1.0)
+    h.setflags(write=False)
+    return h
+
+
+def sylvester(b: int) -> np.ndarray:
+    """Sylvester Hadamard matrix of order b: [H_b]_ij = (-1)^popcount(i & j)."""
+    return _sylvester_cached(b)
 
 
 def transform_matrix(d: int, signs) -> np.ndarray:
@@ -160,7 +168,7 @@ def apply_transform(m, signs, axis: int):
         r = ms.reshape(m.shape[0], d // b, b) @ h.T
         return r.reshape(m.shape[0], d)
     ms = m * s[:, None]
-    r = np.einsum("ij,kjc->kic", h, ms.reshape(d // b, b, m.shape[1]))
+    r = np.matmul(h, ms.reshape(d // b, b, m.shape[1]))     # H_b times each block of rows
     return r.reshape(d, m.shape[1])
 
 

@@ -1,0 +1,336 @@
+// C ABI of the KronQ library: argument validation, workspace carving and dispatch to the
+// kernels. Declarations and the contract of every call are in include/kronq.h.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <vector>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace kq {
+
+namespace {
+thread_local char g_detail[512] = "";
+__device__ int g_device_error_word = 0;
+constexpr int kMaxDevices = 64;
+int* g_err_ptr[kMaxDevices] = {nullptr};
+}  // namespace
+
+void set_detail(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_detail, sizeof(g_detail), fmt, ap);
+  va_end(ap);
+}
+
+kronq_status fail(kronq_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_detail, sizeof(g_detail), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+std::atomic<uint64_t> g_launches{0};
+
+kronq_status check_launch(const char* what) {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(KRONQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return KRONQ_OK;
+}
+
+int* device_error_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  if (!g_err_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error_word) != cudaSuccess) return nullptr;
+    g_err_ptr[dev] = static_cast<int*>(p);
+  }
+  return g_err_ptr[dev];
+}
+
+namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+kronq_status check_ws(void* ws, size_t have, size_t need) {
+  if (need == 0) return KRONQ_OK;
+  if (!ws) return fail(KRONQ_ERR_WORKSPACE, "workspace is NULL, %zu bytes needed", need);
+  if (!aligned(ws, 256)) return fail(KRONQ_ERR_WORKSPACE, "workspace not 256-byte aligned");
+  if (have < need)
+    return fail(KRONQ_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", have, need);
+  return KRONQ_OK;
+}
+
+kronq_status check_bf16_matrix(const void* p, int64_t ld, int cols, const char* name) {
+  if (!p) return fail(KRONQ_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned(p, 16)) return fail(KRONQ_ERR_INVALID_ARG, "%s not 16-byte aligned", name);
+  if (ld < cols) return fail(KRONQ_ERR_SHAPE, "%s: stride %lld < width %d", name, (long long)ld, cols);
+  if ((ld * 2) % 16 != 0)
+    return fail(KRONQ_ERR_INVALID_ARG, "%s: stride %lld elements is not a multiple of 16 bytes",
+                name, (long long)ld);
+  return KRONQ_OK;
+}
+
+constexpr int64_t kDriftChunk = 32768;   // tokens per drift split (workspace bound)
+
+size_t drift_ld(int d_in) { return static_cast<size_t>((d_in + 7) / 8 * 8); }
+
+size_t drift_ws(int64_t n, int d_in) {
+  const int64_t rows = std::min<int64_t>(n, kDriftChunk);
+  if (rows <= 0) return 0;
+  return 2 * align256(static_cast<size_t>(rows) * drift_ld(d_in) * 2);
+}
+
+}  // namespace
+}  // namespace kq
+
+using namespace kq;
+
+extern "C" {
+
+const char* kronq_status_string(kronq_status s) {
+  switch (s) {
+    case KRONQ_OK: return "ok";
+    case KRONQ_ERR_INVALID_ARG: return "invalid argument";
+    case KRONQ_ERR_SHAPE: return "invalid shape";
+    case KRONQ_ERR_NOT_PD: return "matrix not positive definite";
+    case KRONQ_ERR_CUDA: return "CUDA error";
+    case KRONQ_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case KRONQ_ERR_UNSUPPORTED: return "unsupported device or parameter";
+    case KRONQ_ERR_TIMEOUT: return "a kernel gave up a bounded wait";
+  }
+  return "unknown status";
+}
+
+const char* kronq_last_error_detail(void) { return g_detail; }
+
+int kronq_version(void) { return 100; }
+
+uint64_t kronq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+kronq_status kronq_device_check(void) {
+  int dev = 0;
+  KQ_CUDA_TRY(cudaGetDevice(&dev));
+  int major = 0, minor = 0;
+  KQ_CUDA_TRY(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+  KQ_CUDA_TRY(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
+  if (major != 10 || minor != 0)
+    return fail(KRONQ_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a",
+                dev, major, minor);
+  return KRONQ_OK;
+}
+
+kronq_status kronq_device_error(int32_t* code_out, kronq_stream_t stream) {
+  if (!code_out) return fail(KRONQ_ERR_INVALID_ARG, "code_out is NULL");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int* w = device_error_word();
+  if (!w) return fail(KRONQ_ERR_CUDA, "device error word unavailable");
+  int host = 0;
+  KQ_CUDA_TRY(cudaMemcpyAsync(&host, w, sizeof(int), cudaMemcpyDeviceToHost, s));
+  KQ_CUDA_TRY(cudaStreamSynchronize(s));
+  *code_out = host;
+  if (host != 0) {
+    KQ_CUDA_TRY(cudaMemsetAsync(w, 0, sizeof(int), s));
+    KQ_CUDA_TRY(cudaStreamSynchronize(s));
+  }
+  return KRONQ_OK;
+}
+
+// ----------------------------------------------------------------------------- accumulate
+size_t kronq_accumulate_workspace_size(int64_t n, int32_t d_in, int32_t d_out, int with_dxx) {
+  (void)d_out;
+  if (!with_dxx || n <= 0 || d_in <= 0) return 0;
+  return drift_ws(n, d_in);
+}
+
+kronq_status kronq_accumulate(const void* xq, int64_t ld_xq, const void* xfp, int64_t ld_xfp,
+                              const void* g, int64_t ld_g, int64_t n, int32_t d_in,
+                              int32_t d_out, float* hx_sum, float* hg_sum, float* dxx_sum,
+                              void* workspace, size_t workspace_bytes, kronq_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (n < 0) return fail(KRONQ_ERR_SHAPE, "n < 0");
+  if (!hx_sum && !hg_sum && !dxx_sum) return fail(KRONQ_ERR_INVALID_ARG, "no output requested");
+  if ((hx_sum || dxx_sum) && d_in <= 0) return fail(KRONQ_ERR_SHAPE, "d_in <= 0");
+  if (hg_sum && d_out <= 0) return fail(KRONQ_ERR_SHAPE, "d_out <= 0");
+  if (hx_sum || dxx_sum) KQ_TRY(check_bf16_matrix(xq, ld_xq, d_in, "xq"));
+  if (dxx_sum) KQ_TRY(check_bf16_matrix(xfp, ld_xfp, d_in, "xfp"));
+  if (hg_sum) KQ_TRY(check_bf16_matrix(g, ld_g, d_out, "g"));
+  for (const float* o : {hx_sum, hg_sum, dxx_sum})
+    if (o && !aligned(o, 16)) return fail(KRONQ_ERR_INVALID_ARG, "output not 16-byte aligned");
+  if (dxx_sum) KQ_TRY(check_ws(workspace, workspace_bytes, drift_ws(n, d_in)));
+  KQ_TRY(kronq_device_check());
+  if (n == 0) return KRONQ_OK;
+
+  if (hx_sum) {
+    KQ_TRY(launch_accumulate_tc(xq, ld_xq, xq, ld_xq, n, d_in, d_in, hx_sum, d_in, true, s));
+    KQ_TRY(launch_mirror_upper(hx_sum, d_in, d_in, s));
+  }
+  if (hg_sum) {
+    KQ_TRY(launch_accumulate_tc(g, ld_g, g, ld_g, n, d_out, d_out, hg_sum, d_out, true, s));
+    KQ_TRY(launch_mirror_upper(hg_sum, d_out, d_out, s));
+  }
+  if (dxx_sum) {
+    const int64_t ld = static_cast<int64_t>(drift_ld(d_in));
+    const int64_t rows = std::min<int64_t>(n, kDriftChunk);
+    uint8_t* hi = static_cast<uint8_t*>(workspace);
+    uint8_t* lo = hi + align256(static_cast<size_t>(rows) * ld * 2);
+    const uint16_t* xq16 = static_cast<const uint16_t*>(xq);
+    const uint16_t* xf16 = static_cast<const uint16_t*>(xfp);
+    for (int64_t t0 = 0; t0 < n; t0 += kDriftChunk) {
+      const int64_t cnt = std::min<int64_t>(kDriftChunk, n - t0);
+      KQ_TRY(launch_drift_split(xf16 + t0 * ld_xfp, ld_xfp, xq16 + t0 * ld_xq, ld_xq, cnt, d_in, hi,
+                                lo, ld, s));
+      KQ_TRY(launch_accumulate_tc(hi, ld, xq16 + t0 * ld_xq, ld_xq, cnt, d_in, d_in, dxx_sum, d_in,
+                                  false, s));
+      KQ_TRY(launch_accumulate_tc(lo, ld, xq16 + t0 * ld_xq, ld_xq, cnt, d_in, d_in, dxx_sum, d_in,
+                                  false, s));
+    }
+  }
+  return KRONQ_OK;
+}
+
+// ----------------------------------------------------------------------------- biip
+size_t kronq_biip_workspace_size(int32_t d_out, int32_t d_in) {
+  if (d_out <= 0 || d_in <= 0) return 0;
+  return biip_workspace_bytes(d_out, d_in);
+}
+
+kronq_status kronq_biip(const void* w, int32_t w_dtype, float* w_out, float* hx, float* hg,
+                        float* dxx, double inv_n, const int8_t* sign_in, const int8_t* sign_out,
+                        int32_t d_out, int32_t d_in, uint32_t flags, float* s_x, float* s_g,
+                        double* tr_hx, double* tr_hg, void* workspace, size_t workspace_bytes,
+                        kronq_stream_t stream) {
+  if (d_out <= 0 || d_in <= 0) return fail(KRONQ_ERR_SHAPE, "d_out and d_in must be positive");
+  if (!w || !w_out || !hx || !s_x || !s_g || !tr_hx)
+    return fail(KRONQ_ERR_INVALID_ARG, "w, w_out, hx, s_x, s_g and tr_hx are required");
+  if (w_dtype != KRONQ_DTYPE_BF16 && w_dtype != KRONQ_DTYPE_F32)
+    return fail(KRONQ_ERR_INVALID_ARG, "w_dtype must be KRONQ_DTYPE_BF16 or KRONQ_DTYPE_F32");
+  if (flags & ~static_cast<uint32_t>(31))
+    return fail(KRONQ_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+  if ((flags & KRONQ_BIIP_SCALE_OUT) && !hg)
+    return fail(KRONQ_ERR_INVALID_ARG, "KRONQ_BIIP_SCALE_OUT needs hg");
+  if ((flags & KRONQ_BIIP_ROTATE_IN) && !sign_in)
+    return fail(KRONQ_ERR_INVALID_ARG, "KRONQ_BIIP_ROTATE_IN needs sign_in");
+  if ((flags & KRONQ_BIIP_ROTATE_OUT) && !sign_out)
+    return fail(KRONQ_ERR_INVALID_ARG, "KRONQ_BIIP_ROTATE_OUT needs sign_out");
+  if (!(inv_n > 0.0) || !std::isfinite(inv_n)) return fail(KRONQ_ERR_INVALID_ARG, "inv_n must be > 0");
+  if (w == w_out) return fail(KRONQ_ERR_INVALID_ARG, "w and w_out must not alias");
+  KQ_TRY(check_ws(workspace, workspace_bytes, biip_workspace_bytes(d_out, d_in)));
+  KQ_TRY(kronq_device_check());
+  BiipArgs a{w, w_dtype, w_out, hx, hg, dxx, inv_n, sign_in, sign_out, d_out, d_in, flags,
+             s_x, s_g, tr_hx, tr_hg};
+  return run_biip(a, workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+// ----------------------------------------------------------------------------- cholinv
+size_t kronq_cholinv_workspace_size(int32_t d) {
+  if (d <= 0) return 0;
+  return cholinv_workspace_bytes(d);
+}
+
+kronq_status kronq_cholinv(float* h_to_k, int32_t d, float damp_rel, int32_t* info,
+                           uint32_t flags, void* workspace, size_t workspace_bytes,
+                           kronq_stream_t stream) {
+  if (d <= 0) return fail(KRONQ_ERR_SHAPE, "d must be positive");
+  if (!h_to_k || !info) return fail(KRONQ_ERR_INVALID_ARG, "h_to_k and info are required");
+  if (!(damp_rel >= 0.f) || !std::isfinite(damp_rel))
+    return fail(KRONQ_ERR_INVALID_ARG, "damp_rel must be finite and >= 0");
+  if (flags & ~static_cast<uint32_t>(KRONQ_CHOLINV_SYNC))
+    return fail(KRONQ_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+  KQ_TRY(check_ws(workspace, workspace_bytes, cholinv_workspace_bytes(d)));
+  KQ_TRY(kronq_device_check());
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  KQ_TRY(run_cholinv(h_to_k, d, damp_rel, info, workspace, s));
+  if (flags & KRONQ_CHOLINV_SYNC) {
+    int32_t host = -1;
+    KQ_CUDA_TRY(cudaMemcpyAsync(&host, info, sizeof(int32_t), cudaMemcpyDeviceToHost, s));
+    KQ_CUDA_TRY(cudaStreamSynchronize(s));
+    if (host >= 0)
+      return fail(KRONQ_ERR_NOT_PD, "pivot %d of the damped H_X is not positive", host);
+  }
+  return KRONQ_OK;
+}
+
+// ----------------------------------------------------------------------------- quantize
+size_t kronq_quantize_layer_workspace_size(int32_t d_out, int32_t d_in, int32_t block,
+                                           int with_dxx) {
+  if (d_out <= 0 || d_in <= 0) return 0;
+  return quantize_workspace_bytes(d_out, d_in, block, with_dxx != 0);
+}
+
+kronq_status kronq_quantize_layer(const float* w, const float* k, const float* dxx,
+                                  int32_t d_out, int32_t d_in, int32_t bits, int32_t block,
+                                  uint8_t* codes, float* scale, float* zero, float* w_hat,
+                                  void* workspace, size_t workspace_bytes,
+                                  kronq_stream_t stream) {
+  if (d_out <= 0 || d_in <= 0) return fail(KRONQ_ERR_SHAPE, "d_out and d_in must be positive");
+  if (!w || !k || !codes || !scale || !zero || !w_hat)
+    return fail(KRONQ_ERR_INVALID_ARG, "w, k, codes, scale, zero and w_hat are required");
+  if (bits < 2 || bits > 8) return fail(KRONQ_ERR_UNSUPPORTED, "bits must be in 2..8");
+  if (block != 128) return fail(KRONQ_ERR_UNSUPPORTED, "block must be 128");
+  if (w == w_hat) return fail(KRONQ_ERR_INVALID_ARG, "w and w_hat must not alias");
+  KQ_TRY(check_ws(workspace, workspace_bytes,
+                  quantize_workspace_bytes(d_out, d_in, block, dxx != nullptr)));
+  KQ_TRY(kronq_device_check());
+  return run_quantize(w, k, dxx, d_out, d_in, bits, block, codes, scale, zero, w_hat, workspace,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+// ----------------------------------------------------------------------------- allocation
+kronq_status kronq_score_allocate(const double* tr_hx, const double* tr_hg,
+                                  const int64_t* n_params, int32_t L, const int32_t* choices,
+                                  int32_t n_choices, double avg_bits, double* score_out,
+                                  int32_t* bits_out) {
+  if (L <= 0 || n_choices <= 0) return fail(KRONQ_ERR_SHAPE, "L and n_choices must be positive");
+  if (!tr_hx || !tr_hg || !n_params || !choices || !bits_out)
+    return fail(KRONQ_ERR_INVALID_ARG, "null pointer");
+  std::vector<double> s(L);
+  int64_t total = 0;
+  for (int l = 0; l < L; ++l) {
+    s[l] = tr_hg[l] * tr_hx[l];
+    if (std::isnan(s[l])) return fail(KRONQ_ERR_INVALID_ARG, "score of sublayer %d is NaN", l);
+    if (n_params[l] < 0) return fail(KRONQ_ERR_SHAPE, "n_params[%d] < 0", l);
+    total += n_params[l];
+  }
+  std::vector<int32_t> ch(choices, choices + n_choices);
+  std::sort(ch.begin(), ch.end());
+  ch.erase(std::unique(ch.begin(), ch.end()), ch.end());
+  if (ch.front() <= 0) return fail(KRONQ_ERR_INVALID_ARG, "bit widths must be positive");
+  const int64_t budget = static_cast<int64_t>(std::floor(avg_bits * static_cast<double>(total)));
+  int64_t used = static_cast<int64_t>(ch.front()) * total;
+  if (used > budget)
+    return fail(KRONQ_ERR_INVALID_ARG, "budget %lld bits is below the smallest width",
+                (long long)budget);
+  std::vector<int> order(L);
+  for (int l = 0; l < L; ++l) order[l] = l;
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) {
+    if (s[a] != s[b]) return s[a] > s[b];
+    return a < b;
+  });
+  for (int l = 0; l < L; ++l) bits_out[l] = ch.front();
+  for (int l : order) {
+    for (auto it = ch.rbegin(); it != ch.rend(); ++it) {
+      const int b = *it;
+      if (b <= bits_out[l]) break;
+      const int64_t extra = static_cast<int64_t>(b - bits_out[l]) * n_params[l];
+      if (used + extra <= budget) {
+        used += extra;
+        bits_out[l] = b;
+        break;
+      }
+    }
+  }
+  if (score_out)
+    for (int l = 0; l < L; ++l) score_out[l] = s[l];
+  return KRONQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,411 @@
+// Kronecker-factor accumulation on 5th-generation tensor cores.
+//
+// KronQ (hyper.ai summary), Method: H_X = E[x x^T] and H_G = E[g g^T] are the two Kronecker
+// factors of the empirical Fisher; the GPTAQ asymmetric objective adds the drift term dX X^T.
+// Over a chunk of tokens these are C += A^T B with A, B token-major (one token per row), i.e.
+// both tensor-core operands are MN-major.
+//
+// Kernel: persistent, one CTA per SM, warp-specialised.
+//   warp 0        TMA producer: loads 64-token x 64-column boxes (128-byte swizzle) of A and B
+//                 into a 4-stage shared-memory ring (no multicast).
+//   warp 1        TMEM allocator + MMA issuer: tcgen05.mma kind::f16, M=128, N=256, K=16,
+//                 bf16 x bf16 -> fp32 in TMEM; two 256-column accumulators so the epilogue of
+//                 one work unit overlaps the main loop of the next.
+//   warps 2..5    epilogue: tcgen05.ld the accumulator, add it into C with vector atomics (the
+//                 call's contract is "+=", and split-K partial sums combine the same way).
+// Work unit = (output tile, token chunk). For symmetric outputs only tiles touching the upper
+// triangle are computed and a mirror kernel fills the strict lower triangle afterwards.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace kq {
+
+namespace acc {
+constexpr int BM = 128;             // output rows per tile (MMA M)
+constexpr int BN = 256;             // output cols per tile (MMA N)
+constexpr int BK = 64;              // tokens per pipeline stage
+constexpr int UK = 16;              // tokens per MMA instruction
+constexpr int STAGES = 4;
+constexpr int BOX = 64;             // columns per TMA box (128 bytes of bf16)
+constexpr int BOX_BYTES = BOX * BK * 2;          // 8 KB
+constexpr int A_BOXES = BM / BOX;                // 2
+constexpr int B_BOXES = BN / BOX;                // 4
+constexpr int STAGE_BYTES = (A_BOXES + B_BOXES) * BOX_BYTES;   // 48 KB
+constexpr int THREADS = 192;
+constexpr int TMEM_COLS = 512;      // 2 accumulators x 256 fp32 columns
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+}  // namespace acc
+
+struct AccParams {
+  float* c;
+  int64_t ldc;
+  int m, n;               // output rows / cols
+  int64_t k;              // tokens
+  int tiles_m, tiles_n;
+  int symmetric;          // 1: only tiles that touch the upper triangle
+  int num_tiles;          // tiles actually computed
+  int kblocks_per_unit;   // BK-blocks per token chunk
+  int k_splits;
+  int num_units;
+  int* err;
+};
+
+// Map a computed-tile index to (tm, tn). Symmetric: row tm holds tiles tn >= tn_min(tm).
+__device__ __forceinline__ void tile_coords(const AccParams& p, int t, int& tm, int& tn) {
+  if (!p.symmetric) {
+    tm = t / p.tiles_n;
+    tn = t % p.tiles_n;
+    return;
+  }
+  int r = 0;
+  for (;;) {
+    const int tn_min = (r * acc::BM) / acc::BN;
+    const int cnt = p.tiles_n - tn_min;
+    if (t < cnt) {
+      tm = r;
+      tn = tn_min + t;
+      return;
+    }
+    t -= cnt;
+    ++r;
+  }
+}
+
+__global__ void __launch_bounds__(acc::THREADS, 1)
+    accumulate_tc_kernel(const __grid_constant__ CUtensorMap tma_a,
+                         const __grid_constant__ CUtensorMap tma_b, const AccParams p) {
+  using namespace acc;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte alignment for the 128-byte swizzle atoms
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* full = bars;                  // [STAGES]
+  uint64_t* empty = bars + STAGES;        // [STAGES]
+  uint64_t* tfull = bars + 2 * STAGES;    // [2]
+  uint64_t* tempty = bars + 2 * STAGES + 2;   // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tma_a);
+    prefetch_tensormap(&tma_b);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int kblocks_total = static_cast<int>((p.k + BK - 1) / BK);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+        const int split = u / p.num_tiles;
+        const int t = u % p.num_tiles;
+        int tm, tn;
+        tile_coords(p, t, tm, tn);
+        const int kb0 = split * p.kblocks_per_unit;
+        const int kb1 = min(kblocks_total, kb0 + p.kblocks_per_unit);
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.err, DEV_ERR_TMA_WAIT)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+          const int y = kb * BK;
+#pragma unroll
+          for (int b = 0; b < A_BOXES; ++b)
+            tma_load_2d(st + b * BOX_BYTES, &tma_a, &full[s], tm * BM + b * BOX, y);
+#pragma unroll
+          for (int b = 0; b < B_BOXES; ++b)
+            tma_load_2d(st + (A_BOXES + b) * BOX_BYTES, &tma_b, &full[s], tn * BN + b * BOX, y);
+        }
+      }
+      if (!ok) {
+        // aborted: let the copies still in flight land before the CTA exits
+        for (uint32_t j = it > STAGES ? it - STAGES : 0; j < it; ++j)
+          mbar_drain(&full[j % STAGES], (j / STAGES) & 1u, 1000000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32_mn_mn(BM, BN);
+      uint32_t it = 0;
+      uint32_t ui = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x, ++ui) {
+        const int split = u / p.num_tiles;
+        const int kb0 = split * p.kblocks_per_unit;
+        const int kb1 = min(kblocks_total, kb0 + p.kblocks_per_unit);
+        const uint32_t a = ui & 1u;
+        const uint32_t aph = (ui >> 1) & 1u;
+        if (!mbar_wait(&tempty[a], aph ^ 1u, abort_flag, p.err, DEV_ERR_MMA_WAIT)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + a * BN;
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          if (!mbar_wait(&full[s], ph, abort_flag, p.err, DEV_ERR_MMA_WAIT)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(smem + s * STAGE_BYTES);
+          const uint32_t b_base = a_base + A_BOXES * BOX_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / UK; ++kk) {
+            // MN-major, 128B swizzle: 8 token rows of 128 bytes form one 1 KB atom (SBO);
+            // successive 64-column boxes are one box apart (LBO).
+            const uint32_t koff = kk * UK * 128;
+            const uint64_t ad = smem_desc_sw128(a_base + koff, BOX_BYTES, 1024);
+            const uint64_t bd = smem_desc_sw128(b_base + koff, BOX_BYTES, 1024);
+            umma_f16(d_tmem, ad, bd, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty[s]);   // frees the stage once these MMAs have read it
+        }
+        if (!ok) break;
+        umma_commit(&tfull[a]);     // accumulator ready for the epilogue
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue (warps 2..5)
+    const int q = warp & 3;            // TMEM lane quarter this warp may access
+    uint32_t ui = 0;
+    for (int u = blockIdx.x; u < p.num_units; u += gridDim.x, ++ui) {
+      const int t = u % p.num_tiles;
+      int tm, tn;
+      tile_coords(p, t, tm, tn);
+      const uint32_t a = ui & 1u;
+      const uint32_t aph = (ui >> 1) & 1u;
+      // one lane waits, the warp follows its verdict (tcgen05.ld needs a converged warp)
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(&tfull[a], aph, abort_flag, p.err, DEV_ERR_EPI_WAIT) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      __syncwarp();
+      if (!ok) break;
+      tc_fence_after();
+      const int row = tm * BM + q * 32 + lane;
+      const uint32_t taddr = tmem_base + ((q * 32u) << 16) + a * BN;
+#pragma unroll 1
+      for (int cb = 0; cb < BN / 32; ++cb) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(taddr + cb * 32, v);
+        tmem_ld_wait();
+        const int col0 = tn * BN + cb * 32;
+        if (row < p.m && col0 < p.n) {
+          float* dst = p.c + static_cast<int64_t>(row) * p.ldc + col0;
+          if (col0 + 32 <= p.n && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+              float4 f = make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
+                                     __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+              atomicAdd(reinterpret_cast<float4*>(dst + j), f);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (col0 + j < p.n) atomicAdd(dst + j, __uint_as_float(v[j]));
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[a]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// Fill the strict lower triangle of a symmetric d x d matrix from its upper triangle.
+__global__ void mirror_upper_kernel(float* c, int64_t ldc, int d) {
+  __shared__ float tile[32][33];
+  const int bi = blockIdx.y, bj = blockIdx.x;   // destination tile (row block bi, col block bj)
+  if (bj > bi) return;
+  const int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
+  // read source tile (bj, bi) from the upper triangle
+  for (int r = ty; r < 32; r += 8) {
+    const int i = bj * 32 + r, j = bi * 32 + tx;
+    if (i < d && j < d) tile[r][tx] = c[static_cast<int64_t>(i) * ldc + j];
+  }
+  __syncthreads();
+  for (int r = ty; r < 32; r += 8) {
+    const int i = bi * 32 + r, j = bj * 32 + tx;
+    if (i < d && j < d && i > j) c[static_cast<int64_t>(i) * ldc + j] = tile[tx][r];
+  }
+}
+
+// X - X~ split into two bf16 terms: hi = bf16(x - xq), lo = bf16((x - xq) - hi).
+__global__ void drift_split_kernel(const __nv_bfloat16* __restrict__ xfp, int64_t ld_xfp,
+                                   const __nv_bfloat16* __restrict__ xq, int64_t ld_xq,
+                                   int64_t rows, int cols, __nv_bfloat16* __restrict__ hi,
+                                   __nv_bfloat16* __restrict__ lo, int64_t ld_out) {
+  const int64_t total = rows * cols;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / cols;
+    const int c = static_cast<int>(i - r * cols);
+    const float d = __bfloat162float(xfp[r * ld_xfp + c]) - __bfloat162float(xq[r * ld_xq + c]);
+    const __nv_bfloat16 h = __float2bfloat16_rn(d);
+    hi[r * ld_out + c] = h;
+    lo[r * ld_out + c] = __float2bfloat16_rn(d - __bfloat162float(h));
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------------------------
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// Tensor map over a rows x cols bf16 matrix (row stride ld elements), 64 x 64 boxes, 128B swizzle.
+kronq_status make_map(CUtensorMap* map, const void* base, int64_t rows, int cols, int64_t ld) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return fail(KRONQ_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(acc::BOX), static_cast<cuuint32_t>(acc::BK)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(KRONQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return KRONQ_OK;
+}
+
+int num_sms() {
+  static int sms = 0;
+  if (!sms) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
+  }
+  return sms;
+}
+
+}  // namespace
+
+// C (m x n, fp32, ldc) += A^T B with A: k x m bf16 (ld_a), B: k x n bf16 (ld_b).
+kronq_status launch_accumulate_tc(const void* a, int64_t ld_a, const void* b, int64_t ld_b,
+                                  int64_t k, int m, int n, float* c, int64_t ldc, bool symmetric,
+                                  cudaStream_t stream) {
+  using namespace acc;
+  if (k <= 0 || m <= 0 || n <= 0) return KRONQ_OK;
+  CUtensorMap ma, mb;
+  KQ_TRY(make_map(&ma, a, k, m, ld_a));
+  KQ_TRY(make_map(&mb, b, k, n, ld_b));
+
+  AccParams p{};
+  p.c = c;
+  p.ldc = ldc;
+  p.m = m;
+  p.n = n;
+  p.k = k;
+  p.tiles_m = (m + BM - 1) / BM;
+  p.tiles_n = (n + BN - 1) / BN;
+  p.symmetric = symmetric ? 1 : 0;
+  if (symmetric) {
+    int cnt = 0;
+    for (int r = 0; r < p.tiles_m; ++r) cnt += p.tiles_n - (r * BM) / BN;
+    p.num_tiles = cnt;
+  } else {
+    p.num_tiles = p.tiles_m * p.tiles_n;
+  }
+  const int sms = num_sms();
+  const int kblocks = static_cast<int>((k + BK - 1) / BK);
+  // Token chunk per unit: about 16K tokens, fewer when there are too few tiles to fill the GPU.
+  int per = 256;
+  while (per > 8 && static_cast<int64_t>(p.num_tiles) * ((kblocks + per - 1) / per) < 8 * sms)
+    per >>= 1;
+  if (per > kblocks) per = kblocks;
+  p.kblocks_per_unit = per;
+  p.k_splits = (kblocks + per - 1) / per;
+  p.num_units = p.num_tiles * p.k_splits;
+  p.err = device_error_word();
+  if (!p.err) return fail(KRONQ_ERR_CUDA, "device error word unavailable");
+
+  static bool attr_set = false;
+  if (!attr_set) {
+    KQ_CUDA_TRY(cudaFuncSetAttribute(accumulate_tc_kernel,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
+    attr_set = true;
+  }
+  const int grid = p.num_units < sms ? p.num_units : sms;
+  accumulate_tc_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(ma, mb, p);
+  KQ_TRY(check_launch("accumulate_tc_kernel"));
+  return KRONQ_OK;
+}
+
+kronq_status launch_mirror_upper(float* c, int64_t ldc, int d, cudaStream_t stream) {
+  const int t = (d + 31) / 32;
+  mirror_upper_kernel<<<dim3(t, t), dim3(32, 8), 0, stream>>>(c, ldc, d);
+  return check_launch("mirror_upper_kernel");
+}
+
+kronq_status launch_drift_split(const void* xfp, int64_t ld_xfp, const void* xq, int64_t ld_xq,
+                                int64_t rows, int cols, void* hi, void* lo, int64_t ld_out,
+                                cudaStream_t stream) {
+  const int64_t total = rows * cols;
+  if (total <= 0) return KRONQ_OK;
+  int64_t blocks = (total + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  drift_split_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(xfp), ld_xfp, static_cast<const __nv_bfloat16*>(xq), ld_xq,
+      rows, cols, static_cast<__nv_bfloat16*>(hi), static_cast<__nv_bfloat16*>(lo), ld_out);
+  return check_launch("drift_split_kernel");
+}
+
+}  // namespace kq

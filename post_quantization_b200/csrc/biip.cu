@@ -1,0 +1,335 @@
+// Bidirectional incoherence processing (BiIP) of one sublayer.
+//
+// KronQ (hyper.ai summary), Method, BiIP equations:
+//   W <- S_G W S_X,  S_X = diag(H_X,jj / |W_:,j|^2)^(1/4),  S_G = diag(H_G,ii / |W_i,:|^2)^(1/4)
+//   W <- U W V^T,  H_X <- V H_X V^T,  H_G <- U H_G U^T,  dXX^T <- V dXX^T V^T
+// with U, V = (1/sqrt(b)) (I (x) H_b) diag(random signs), H_b Sylvester, b = largest power of
+// two dividing the dimension. The Hessians follow the scaling as S^-1 H S^-1.
+//
+// Passes (all bandwidth-bound):
+//   norms   one read of W: |W_:,j|^2 and |W_i,:|^2 (fp64 sums)
+//   scales  S_X, S_G, the per-row / per-column factors of the passes below, traces
+//   rows    for every row: multiply by row and column factors, FWHT along the row in b-blocks
+//   cols    for every b-row block of every column: FWHT along the column (in place)
+// W' = rows(W) then cols; H_X and dXX^T = rows then cols (in place); H_G likewise if asked.
+#include <cuda_bf16.h>
+
+#include <cmath>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace kq {
+
+namespace {
+
+constexpr int kNormRows = 64;
+constexpr int kNormCols = 256;
+
+template <typename T>
+__device__ __forceinline__ float load_as_float(const T* p, int64_t i);
+template <>
+__device__ __forceinline__ float load_as_float<float>(const float* p, int64_t i) {
+  return p[i];
+}
+template <>
+__device__ __forceinline__ float load_as_float<__nv_bfloat16>(const __nv_bfloat16* p, int64_t i) {
+  return __bfloat162float(p[i]);
+}
+
+// Partial squared column and row norms of a 64 x 256 tile, added into fp64 accumulators.
+template <typename T>
+__global__ void __launch_bounds__(256) colrow_norms_kernel(const T* __restrict__ w, int rows,
+                                                           int cols, double* __restrict__ col_sq,
+                                                           double* __restrict__ row_sq) {
+  __shared__ float part[8][kNormRows];
+  const int c = blockIdx.x * kNormCols + threadIdx.x;
+  const int r0 = blockIdx.y * kNormRows;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float colacc = 0.f;
+  for (int r = 0; r < kNormRows; ++r) {
+    const int row = r0 + r;
+    float v = 0.f;
+    if (row < rows && c < cols) v = load_as_float(w, static_cast<int64_t>(row) * cols + c);
+    const float sq = v * v;
+    colacc += sq;
+    float rs = sq;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) rs += __shfl_xor_sync(0xffffffffu, rs, o);
+    if (lane == 0) part[warp][r] = rs;
+  }
+  if (c < cols) atomicAdd(&col_sq[c], static_cast<double>(colacc));
+  __syncthreads();
+  if (threadIdx.x < kNormRows) {
+    const int row = r0 + threadIdx.x;
+    float s = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) s += part[k][threadIdx.x];
+    if (row < rows) atomicAdd(&row_sq[row], static_cast<double>(s));
+  }
+}
+
+// (diag * inv_n / norm_sq)^(1/4), or 1 where either is not positive.
+__device__ __forceinline__ double biip_scale(double diag_raw, double inv_n, double norm_sq) {
+  const double dg = diag_raw * inv_n;
+  if (!(dg > 0.0) || !(norm_sq > 0.0)) return 1.0;
+  return sqrt(sqrt(dg / norm_sq));
+}
+
+// Scales and factor vectors for one side (d entries).
+//   s        = S (fp32 output)
+//   fw       = S * sign            (factor on W)
+//   fh       = sign / S            (factor on the Hessian, both sides)
+__global__ void side_scales_kernel(int d, const float* __restrict__ h, const double* __restrict__ nsq,
+                                   double inv_n, int do_scale, const int8_t* __restrict__ sign,
+                                   float* __restrict__ s_out, float* __restrict__ fw,
+                                   float* __restrict__ fh) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= d) return;
+  double s = 1.0;
+  if (do_scale) s = biip_scale(h[static_cast<int64_t>(i) * d + i], inv_n, nsq[i]);
+  const double sg = sign ? static_cast<double>(sign[i]) : 1.0;
+  s_out[i] = static_cast<float>(s);
+  fw[i] = static_cast<float>(s * sg);
+  fh[i] = static_cast<float>(sg / s);
+}
+
+// tr(S^-1 (inv_n H) S^-1) = sum_i inv_n H_ii / s_i^2, in fp64 (one block).
+__global__ void side_trace_kernel(int d, const float* __restrict__ h, const double* __restrict__ nsq,
+                                  double inv_n, int do_scale, double* __restrict__ tr) {
+  __shared__ double red[32];
+  double acc = 0.0;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) {
+    const double hii = static_cast<double>(h[static_cast<int64_t>(i) * d + i]) * inv_n;
+    double s = 1.0;
+    if (do_scale) s = biip_scale(h[static_cast<int64_t>(i) * d + i], inv_n, nsq[i]);
+    acc += hii / (s * s);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    double v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (threadIdx.x == 0) *tr = v;
+  }
+}
+
+// Row pass over a rows x cols matrix seen as a flat array of b-blocks (b divides cols):
+// dst = FWHT_b(src * row_factor[r] * col_factor[c] * scalar) / sqrt(b), one chunk per CTA.
+template <typename T>
+__global__ void __launch_bounds__(256) fwht_rows_kernel(const T* src, float* dst, int64_t rows,
+                                                        int64_t cols, const float* __restrict__ row_f,
+                                                        const float* __restrict__ col_f, float scalar,
+                                                        int log2b, int chunk, float out_scale) {
+  extern __shared__ float sbuf[];
+  const int64_t total = rows * cols;
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * chunk;
+  for (int e = threadIdx.x; e < chunk; e += blockDim.x) {
+    const int64_t f = base + e;
+    float v = 0.f;
+    if (f < total) {
+      const int64_t r = f / cols;
+      const int64_t c = f - r * cols;
+      v = load_as_float(src, f) * scalar;
+      if (row_f) v *= row_f[r];
+      if (col_f) v *= col_f[c];
+    }
+    sbuf[e] = v;
+  }
+  __syncthreads();
+  const int half = chunk >> 1;
+  for (int h = 0; h < log2b; ++h) {
+    const int lowmask = (1 << h) - 1;
+    for (int p = threadIdx.x; p < half; p += blockDim.x) {
+      const int i = ((p >> h) << (h + 1)) | (p & lowmask);
+      const int j = i | (1 << h);
+      const float a = sbuf[i], b = sbuf[j];
+      sbuf[i] = a + b;
+      sbuf[j] = a - b;
+    }
+    __syncthreads();
+  }
+  for (int e = threadIdx.x; e < chunk; e += blockDim.x) {
+    const int64_t f = base + e;
+    if (f < total) dst[f] = sbuf[e] * out_scale;
+  }
+}
+
+// Column pass, in place: for each column, FWHT along rows in blocks of b; tile = b x cw.
+__global__ void __launch_bounds__(256) fwht_cols_kernel(float* m, int64_t rows, int64_t cols,
+                                                        int log2b, int cw, float out_scale) {
+  extern __shared__ float sbuf[];
+  const int b = 1 << log2b;
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * cw;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * b;
+  const int n = b * cw;
+  for (int e = threadIdx.x; e < n; e += blockDim.x) {
+    const int r = e / cw, c = e - r * cw;
+    float v = 0.f;
+    if (c0 + c < cols) v = m[(r0 + r) * cols + c0 + c];
+    sbuf[e] = v;
+  }
+  __syncthreads();
+  const int pairs = (b >> 1) * cw;
+  for (int h = 0; h < log2b; ++h) {
+    const int lowmask = (1 << h) - 1;
+    for (int q = threadIdx.x; q < pairs; q += blockDim.x) {
+      const int c = q % cw, p = q / cw;
+      const int i = ((p >> h) << (h + 1)) | (p & lowmask);
+      const int j = i | (1 << h);
+      const float a = sbuf[i * cw + c], bb = sbuf[j * cw + c];
+      sbuf[i * cw + c] = a + bb;
+      sbuf[j * cw + c] = a - bb;
+    }
+    __syncthreads();
+  }
+  for (int e = threadIdx.x; e < n; e += blockDim.x) {
+    const int r = e / cw, c = e - r * cw;
+    if (c0 + c < cols) m[(r0 + r) * cols + c0 + c] = sbuf[e] * out_scale;
+  }
+}
+
+int ilog2_pow2(int b) {
+  int l = 0;
+  while ((1 << l) < b) ++l;
+  return l;
+}
+
+int largest_pow2_divisor(int d) { return d & (-d); }
+
+template <typename T>
+kronq_status row_pass(const T* src, float* dst, int64_t rows, int64_t cols, const float* row_f,
+                      const float* col_f, float scalar, int b, cudaStream_t stream) {
+  const int chunk = b > 4096 ? b : 4096;
+  const int64_t total = rows * cols;
+  const int64_t blocks = (total + chunk - 1) / chunk;
+  const size_t smem = static_cast<size_t>(chunk) * sizeof(float);
+  const float out_scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(b)));
+  if (smem > 48 * 1024)
+    KQ_CUDA_TRY(cudaFuncSetAttribute(fwht_rows_kernel<T>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  fwht_rows_kernel<T><<<static_cast<unsigned>(blocks), 256, smem, stream>>>(
+      src, dst, rows, cols, row_f, col_f, scalar, ilog2_pow2(b), chunk, out_scale);
+  return check_launch("fwht_rows_kernel");
+}
+
+kronq_status col_pass(float* m, int64_t rows, int64_t cols, int b, cudaStream_t stream) {
+  if (b <= 1) return KRONQ_OK;
+  int cw = 32768 / b;
+  if (cw > 64) cw = 64;
+  if (cw < 1) cw = 1;
+  const size_t smem = static_cast<size_t>(b) * cw * sizeof(float);
+  const float out_scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(b)));
+  if (smem > 48 * 1024)
+    KQ_CUDA_TRY(cudaFuncSetAttribute(fwht_cols_kernel,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  dim3 grid(static_cast<unsigned>((cols + cw - 1) / cw), static_cast<unsigned>(rows / b));
+  fwht_cols_kernel<<<grid, 256, smem, stream>>>(m, rows, cols, ilog2_pow2(b), cw, out_scale);
+  return check_launch("fwht_cols_kernel");
+}
+
+struct BiipWs {
+  double* col_sq;   // d_in
+  double* row_sq;   // d_out
+  float* fw_in;     // d_in   S_X * sign_in
+  float* fh_in;     // d_in   sign_in / S_X
+  float* fw_out;    // d_out  S_G * sign_out
+  float* fh_out;    // d_out  sign_out / S_G
+};
+
+BiipWs carve(void* ws, int d_out, int d_in) {
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  BiipWs w;
+  w.col_sq = reinterpret_cast<double*>(p);
+  p += align256(sizeof(double) * d_in);
+  w.row_sq = reinterpret_cast<double*>(p);
+  p += align256(sizeof(double) * d_out);
+  w.fw_in = reinterpret_cast<float*>(p);
+  p += align256(sizeof(float) * d_in);
+  w.fh_in = reinterpret_cast<float*>(p);
+  p += align256(sizeof(float) * d_in);
+  w.fw_out = reinterpret_cast<float*>(p);
+  p += align256(sizeof(float) * d_out);
+  w.fh_out = reinterpret_cast<float*>(p);
+  return w;
+}
+
+}  // namespace
+
+size_t biip_workspace_bytes(int d_out, int d_in) {
+  return align256(sizeof(double) * d_in) + align256(sizeof(double) * d_out) +
+         2 * align256(sizeof(float) * d_in) + 2 * align256(sizeof(float) * d_out);
+}
+
+kronq_status run_biip(const BiipArgs& a, void* ws_raw, cudaStream_t stream) {
+  const BiipWs ws = carve(ws_raw, a.d_out, a.d_in);
+  const bool scale_in = a.flags & KRONQ_BIIP_SCALE_IN;
+  const bool scale_out = a.flags & KRONQ_BIIP_SCALE_OUT;
+  const bool rot_in = a.flags & KRONQ_BIIP_ROTATE_IN;
+  const bool rot_out = a.flags & KRONQ_BIIP_ROTATE_OUT;
+  const bool write_hg = (a.flags & KRONQ_BIIP_WRITE_HG) && a.hg;
+  const int b_in = rot_in ? largest_pow2_divisor(a.d_in) : 1;
+  const int b_out = rot_out ? largest_pow2_divisor(a.d_out) : 1;
+
+  // 1. squared column / row norms of the original W
+  KQ_CUDA_TRY(cudaMemsetAsync(ws.col_sq, 0, sizeof(double) * a.d_in, stream));
+  KQ_CUDA_TRY(cudaMemsetAsync(ws.row_sq, 0, sizeof(double) * a.d_out, stream));
+  {
+    dim3 grid((a.d_in + kNormCols - 1) / kNormCols, (a.d_out + kNormRows - 1) / kNormRows);
+    if (a.w_dtype == KRONQ_DTYPE_BF16)
+      colrow_norms_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
+          static_cast<const __nv_bfloat16*>(a.w), a.d_out, a.d_in, ws.col_sq, ws.row_sq);
+    else
+      colrow_norms_kernel<float><<<grid, 256, 0, stream>>>(static_cast<const float*>(a.w),
+                                                           a.d_out, a.d_in, ws.col_sq, ws.row_sq);
+    KQ_TRY(check_launch("colrow_norms_kernel"));
+  }
+
+  // 2. scales, factors and traces (from the un-transformed diagonals)
+  side_scales_kernel<<<(a.d_in + 255) / 256, 256, 0, stream>>>(
+      a.d_in, a.hx, ws.col_sq, a.inv_n, scale_in, rot_in ? a.sign_in : nullptr, a.s_x, ws.fw_in,
+      ws.fh_in);
+  KQ_TRY(check_launch("side_scales_kernel(in)"));
+  side_trace_kernel<<<1, 1024, 0, stream>>>(a.d_in, a.hx, ws.col_sq, a.inv_n, scale_in, a.tr_hx);
+  KQ_TRY(check_launch("side_trace_kernel(in)"));
+  side_scales_kernel<<<(a.d_out + 255) / 256, 256, 0, stream>>>(
+      a.d_out, a.hg, ws.row_sq, a.inv_n, scale_out, rot_out ? a.sign_out : nullptr, a.s_g,
+      ws.fw_out, ws.fh_out);
+  KQ_TRY(check_launch("side_scales_kernel(out)"));
+  if (a.hg && a.tr_hg) {
+    side_trace_kernel<<<1, 1024, 0, stream>>>(a.d_out, a.hg, ws.row_sq, a.inv_n, scale_out,
+                                              a.tr_hg);
+    KQ_TRY(check_launch("side_trace_kernel(out)"));
+  }
+
+  // 3. W' = U S_G W S_X V^T: row pass (scales, output signs, input-side FWHT), column pass
+  if (a.w_dtype == KRONQ_DTYPE_BF16)
+    KQ_TRY(row_pass(static_cast<const __nv_bfloat16*>(a.w), a.w_out, a.d_out, a.d_in, ws.fw_out,
+                    ws.fw_in, 1.0f, b_in, stream));
+  else
+    KQ_TRY(row_pass(static_cast<const float*>(a.w), a.w_out, a.d_out, a.d_in, ws.fw_out, ws.fw_in,
+                    1.0f, b_in, stream));
+  KQ_TRY(col_pass(a.w_out, a.d_out, a.d_in, b_out, stream));
+
+  // 4. H_X <- V S_X^-1 (inv_n H_X) S_X^-1 V^T, same for dXX^T; H_G if asked
+  const float inv_n = static_cast<float>(a.inv_n);
+  KQ_TRY(row_pass(static_cast<const float*>(a.hx), a.hx, a.d_in, a.d_in, ws.fh_in, ws.fh_in, inv_n,
+                  b_in, stream));
+  KQ_TRY(col_pass(a.hx, a.d_in, a.d_in, b_in, stream));
+  if (a.dxx) {
+    KQ_TRY(row_pass(static_cast<const float*>(a.dxx), a.dxx, a.d_in, a.d_in, ws.fh_in, ws.fh_in,
+                    inv_n, b_in, stream));
+    KQ_TRY(col_pass(a.dxx, a.d_in, a.d_in, b_in, stream));
+  }
+  if (write_hg) {
+    KQ_TRY(row_pass(static_cast<const float*>(a.hg), a.hg, a.d_out, a.d_out, ws.fh_out, ws.fh_out,
+                    inv_n, b_out, stream));
+    KQ_TRY(col_pass(a.hg, a.d_out, a.d_out, b_out, stream));
+  }
+  return KRONQ_OK;
+}
+
+}  // namespace kq

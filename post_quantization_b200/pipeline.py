@@ -1,0 +1,102 @@
+"""Orchestration of the KronQ layer path over the C ABI (buffers and call order only).
+
+A sublayer goes through: Kronecker-factor sums -> BiIP -> damped inverse factor -> column
+solve; a block or stack adds the trace-product scores and the bit allocation in between. Every
+arithmetic step is one of the five library calls; this module only allocates device buffers
+with torch and sequences the calls on one stream.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+
+from . import kronq as K
+
+
+@dataclass
+class SublayerResult:
+    w_prime: torch.Tensor     # W' = U S_G W S_X V^T (fp32)
+    hx: torch.Tensor          # H_X' (fp32), overwritten by K after cholinv
+    s_x: torch.Tensor
+    s_g: torch.Tensor
+    tr: torch.Tensor          # [tr H_X', tr H_G'] fp64 on device
+    dxx: torch.Tensor | None
+    info: torch.Tensor
+    codes: torch.Tensor | None = None
+    scale: torch.Tensor | None = None
+    zero: torch.Tensor | None = None
+    w_hat: torch.Tensor | None = None
+
+
+class Workspace:
+    """One device scratch buffer, grown on demand and reused by every call on one stream."""
+
+    def __init__(self, device):
+        self.device = device
+        self.buf = torch.empty(0, dtype=torch.uint8, device=device)
+
+    def get(self, nbytes: int):
+        if nbytes == 0:
+            return None
+        if self.buf.numel() < nbytes + 256:
+            self.buf = torch.empty(nbytes + 256, dtype=torch.uint8, device=self.device)
+        off = (-self.buf.data_ptr()) % 256
+        return self.buf[off:off + nbytes]
+
+
+def accumulate(xq=None, xfp=None, g=None, hx_sum=None, hg_sum=None, dxx_sum=None, ws=None,
+               stream=None):
+    n = (xq if xq is not None else g).shape[0]
+    d_in = xq.shape[1] if xq is not None else 0
+    d_out = g.shape[1] if g is not None else 0
+    wsz = K.kronq_accumulate_workspace_size(n, d_in, d_out, dxx_sum is not None)
+    K.kronq_accumulate(xq, xfp, g, hx_sum, hg_sum, dxx_sum,
+                       workspace=ws.get(wsz) if ws is not None else None, stream=stream)
+
+
+def biip(w, hx_sum, hg_sum, dxx_sum, inv_n, sign_in, sign_out, flags=K.BIIP_FULL, ws=None,
+         stream=None, copy_hx=True):
+    """Runs kronq_biip on copies of the sums (hx is copied unless copy_hx is False)."""
+    dev = w.device
+    d_out, d_in = w.shape
+    hx = hx_sum.clone() if copy_hx else hx_sum
+    dxx = dxx_sum.clone() if dxx_sum is not None else None
+    w_out = torch.empty(d_out, d_in, dtype=torch.float32, device=dev)
+    s_x = torch.empty(d_in, dtype=torch.float32, device=dev)
+    s_g = torch.empty(d_out, dtype=torch.float32, device=dev)
+    tr = torch.zeros(2, dtype=torch.float64, device=dev)
+    wsz = K.kronq_biip_workspace_size(d_out, d_in)
+    K.kronq_biip(w, w_out, hx, hg_sum, dxx, inv_n, sign_in, sign_out, flags, s_x, s_g, tr[0:1],
+                 tr[1:2] if hg_sum is not None else None,
+                 workspace=ws.get(wsz) if ws is not None else None, stream=stream)
+    info = torch.empty(1, dtype=torch.int32, device=dev)
+    return SublayerResult(w_out, hx, s_x, s_g, tr, dxx, info)
+
+
+def cholinv(r: SublayerResult, damp_rel=0.01, ws=None, stream=None, sync=False):
+    d = r.hx.shape[0]
+    wsz = K.kronq_cholinv_workspace_size(d)
+    K.kronq_cholinv(r.hx, damp_rel, r.info, K.CHOLINV_SYNC if sync else 0,
+                    workspace=ws.get(wsz) if ws is not None else None, stream=stream)
+
+
+def quantize(r: SublayerResult, bits: int, ws=None, stream=None):
+    d_out, d_in = r.w_prime.shape
+    dev = r.w_prime.device
+    if r.codes is None:
+        r.codes = torch.empty(d_out, d_in, dtype=torch.uint8, device=dev)
+        r.scale = torch.empty(d_out, dtype=torch.float32, device=dev)
+        r.zero = torch.empty(d_out, dtype=torch.float32, device=dev)
+        r.w_hat = torch.empty(d_out, d_in, dtype=torch.float32, device=dev)
+    wsz = K.kronq_quantize_layer_workspace_size(d_out, d_in, 128, r.dxx is not None)
+    K.kronq_quantize_layer(r.w_prime, r.hx, r.dxx, bits, r.codes, r.scale, r.zero, r.w_hat,
+                           workspace=ws.get(wsz) if ws is not None else None, stream=stream)
+
+
+def quantize_sublayer(w, hx_sum, hg_sum, dxx_sum, inv_n, sign_in, sign_out, bits,
+                      flags=K.BIIP_FULL, damp_rel=0.01, ws=None, stream=None):
+    r = biip(w, hx_sum, hg_sum, dxx_sum, inv_n, sign_in, sign_out, flags, ws, stream)
+    cholinv(r, damp_rel, ws, stream)
+    quantize(r, bits, ws, stream)
+    return r

@@ -1,0 +1,139 @@
+"""Host-side checks of the C ABI library (no GPU needed).
+
+The library must load, export every entry point include/kronq.h declares, reject bad
+arguments before touching a device, and run the (host-only) score/allocation call bit-exactly
+like the oracle.
+"""
+import json
+import math
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import kronq_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def K():
+    from post_quantization_b200 import build
+    build.build()
+    from post_quantization_b200 import kronq
+    kronq.load_library()
+    return kronq
+
+
+def header_symbols():
+    src = open(os.path.join(ROOT, "include", "kronq.h")).read()
+    return sorted(set(re.findall(r"\b(kronq_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(K):
+    import ctypes
+    lib = ctypes.CDLL(K.LIB_PATH)
+    declared = header_symbols()
+    assert len(declared) >= 14
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert set(declared) == set(K.SYMBOLS)
+
+
+def test_only_kronq_symbols_exported(K):
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", K.LIB_PATH], capture_output=True,
+                         text=True).stdout
+    names = [l.split()[-1] for l in out.splitlines() if " T " in l]
+    assert names and all(n.startswith("kronq_") for n in names), names
+
+
+def test_status_strings(K):
+    assert K.kronq_status_string(K.OK) == "ok"
+    assert "positive definite" in K.kronq_status_string(K.ERR_NOT_PD)
+    assert K.kronq_version() >= 100
+
+
+def test_workspace_queries(K):
+    assert K.kronq_biip_workspace_size(4096, 11008) > 0
+    assert K.kronq_cholinv_workspace_size(4096) >= 4096 * 64 * 4
+    assert K.kronq_quantize_layer_workspace_size(4096, 4096, 128, False) >= 4096 * 128 * 4
+    assert (K.kronq_quantize_layer_workspace_size(64, 64, 128, True)
+            > K.kronq_quantize_layer_workspace_size(64, 64, 128, False))
+    assert K.kronq_accumulate_workspace_size(1000, 256, 256, False) == 0
+    assert K.kronq_accumulate_workspace_size(1000, 256, 256, True) > 0
+    assert K.kronq_biip_workspace_size(0, 5) == 0
+
+
+def test_argument_errors_before_device(K):
+    lib = K.load_library()
+    # quantize: bad bits / block / missing pointers, no device touched
+    assert lib.kronq_quantize_layer(8, 8, None, 16, 16, 9, 128, 8, 8, 8, 16, None, 0, None) \
+        == K.ERR_UNSUPPORTED
+    assert lib.kronq_quantize_layer(8, 8, None, 16, 16, 4, 64, 8, 8, 8, 16, None, 0, None) \
+        == K.ERR_UNSUPPORTED
+    assert lib.kronq_quantize_layer(None, 8, None, 16, 16, 4, 128, 8, 8, 8, 16, None, 0, None) \
+        == K.ERR_INVALID_ARG
+    assert lib.kronq_quantize_layer(8, 8, None, 0, 16, 4, 128, 8, 8, 8, 16, None, 0, None) \
+        == K.ERR_SHAPE
+    # biip: SCALE_OUT without hg, rotation without signs, bad dtype, aliasing
+    args = [16, 0, 32, 48, None, None, 1.0, None, None, 4, 4]
+    tail = [64, 80, 96, 112, None, 0, None]
+    assert lib.kronq_biip(*args, K.BIIP_SCALE_OUT, *tail) == K.ERR_INVALID_ARG
+    assert lib.kronq_biip(*args, K.BIIP_ROTATE_IN, *tail) == K.ERR_INVALID_ARG
+    bad = list(args); bad[1] = 7
+    assert lib.kronq_biip(*bad, 0, *tail) == K.ERR_INVALID_ARG
+    assert lib.kronq_biip(*args, 1 << 8, *tail) == K.ERR_INVALID_ARG
+    # cholinv: negative damping, missing info
+    assert lib.kronq_cholinv(16, 4, -1.0, 32, 0, None, 0, None) == K.ERR_INVALID_ARG
+    assert lib.kronq_cholinv(16, 4, 0.01, None, 0, None, 0, None) == K.ERR_INVALID_ARG
+    assert lib.kronq_cholinv(16, 0, 0.01, 32, 0, None, 0, None) == K.ERR_SHAPE
+    # accumulate: misaligned stride (bf16 stride must be a multiple of 8 elements)
+    assert lib.kronq_accumulate(256, 12, None, 0, None, 0, 10, 12, 0, 512, None, None, None, 0,
+                                None) == K.ERR_INVALID_ARG
+    assert lib.kronq_accumulate(256, 16, None, 0, None, 0, 10, 12, 0, None, None, None, None, 0,
+                                None) == K.ERR_INVALID_ARG
+    assert "no output" in lib.kronq_last_error_detail().decode()
+
+
+def test_allocation_matches_golden_and_oracle(K):
+    with open(os.path.join(ROOT, "tests", "golden", "allocation_cases.json")) as f:
+        for c in json.load(f)["cases"]:
+            s, bits = K.kronq_score_allocate(c["tr_hx"], c["tr_hg"], c["n_params"], c["choices"],
+                                             c["avg_bits"])
+            assert bits == c["bits"], c["name"]
+    r = np.random.default_rng(7)
+    for trial in range(200):
+        L = int(r.integers(1, 40))
+        tr_hx = r.lognormal(0, 2, L)
+        tr_hg = r.lognormal(0, 2, L)
+        if trial % 5 == 0:                      # ties
+            tr_hx[: L // 2] = 1.0; tr_hg[: L // 2] = 2.0
+        n = r.integers(1, 10_000_000, L)
+        choices = sorted(set(r.choice([1, 2, 3, 4, 5, 6, 8], int(r.integers(1, 4)), replace=False)))
+        avg = float(min(choices) + r.uniform(0, max(choices) - min(choices) + 0.5))
+        s_o, b_o = O.score_allocate(tr_hx, tr_hg, n, choices, avg)
+        s_k, b_k = K.kronq_score_allocate(tr_hx, tr_hg, n, choices, avg)
+        assert b_k == b_o
+        assert s_k == s_o
+
+
+def test_allocation_errors(K):
+    with pytest.raises(K.KronqError) as e:
+        K.kronq_score_allocate([float("nan")], [1.0], [10], [2, 3], 3.0)
+    assert e.value.status == K.ERR_INVALID_ARG
+    with pytest.raises(K.KronqError):
+        K.kronq_score_allocate([1.0], [1.0], [10], [2, 3], 1.0)
+
+
+def test_llama2_stack_allocation_shape(K):
+    # 224 sublayers of LLaMA-2-7B shapes at 2.5 average bits from {2, 3, 4}
+    from post_quantization_b200 import synth
+    wl = synth.WORKLOADS["llama2_7b_stack"]
+    sizes = [s.d_out * s.d_in for s in wl.sublayers] * wl.n_blocks
+    r = np.random.default_rng(3)
+    tr_hx = r.lognormal(0, 1, len(sizes)); tr_hg = r.lognormal(0, 3, len(sizes))
+    s, bits = K.kronq_score_allocate(tr_hx, tr_hg, sizes, [2, 3, 4], 2.5)
+    assert sum(b * n for b, n in zip(bits, sizes)) <= math.floor(2.5 * sum(sizes))
+    assert bits == O.score_allocate(tr_hx, tr_hg, sizes, [2, 3, 4], 2.5)[1]

@@ -1,0 +1,303 @@
+"""CUDA path vs fp64 oracle, element by element, through the C ABI.
+
+Bars (written in each test): relative Frobenius error <= 1e-3 for H_X, H_G, D, W', scales,
+traces, K and W^; codes: the oracle runs in follow mode (it adopts the GPU's code only where its
+own value lies within 1e-3 grid units of a rounding boundary) and must then agree on every code,
+with near-ties <= 0.1% of entries; grid scale/zero bit-exact when both sides see the same W'.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import kronq_oracle as O
+from post_quantization_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-3
+
+
+@pytest.fixture(scope="module")
+def K():
+    from post_quantization_b200 import build
+    build.build()
+    from post_quantization_b200 import kronq
+    kronq.load_library()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    kronq.kronq_device_check()
+    return kronq
+
+
+@pytest.fixture(scope="module")
+def P(K):
+    from post_quantization_b200 import pipeline
+    return pipeline
+
+
+def rel(a, b):
+    a = np.asarray(a, dtype=np.float64); b = np.asarray(b, dtype=np.float64)
+    nb = np.linalg.norm(b)
+    return float(np.linalg.norm(a - b) / (nb if nb > 0 else 1.0))
+
+
+def h64(t):
+    return t.detach().double().cpu().numpy()
+
+
+def layer_inputs(d_out, d_in, n, drift="abs0.01", w_dtype=torch.float32, tag="t", dev="cuda"):
+    xfp = synth.correlated_x(n, d_in, synth.seed_for(tag, "X"), device=dev)
+    if drift == "none":
+        xq = xfp
+    elif drift.startswith("abs"):
+        xq = synth.perturbed(xfp, synth.seed_for(tag, "Xq"), abs_std=float(drift[3:]))
+    else:
+        xq = synth.perturbed(xfp, synth.seed_for(tag, "Xq"), rel_std=float(drift[3:]))
+    g = synth.gradients(n, d_out, synth.seed_for(tag, "G"), device=dev)
+    w = synth.weight(d_out, d_in, synth.seed_for(tag, "W"), dtype=w_dtype, device=dev)
+    si = synth.rademacher(d_in, synth.seed_for(tag, "si"), device=dev)
+    so = synth.rademacher(d_out, synth.seed_for(tag, "so"), device=dev)
+    return xq, xfp, g, w, si, so
+
+
+def gpu_sums(K, xq, xfp, g, with_dxx=True):
+    d_in = xq.shape[1]; d_out = g.shape[1]
+    hx = torch.zeros(d_in, d_in, device="cuda"); hg = torch.zeros(d_out, d_out, device="cuda")
+    dxx = torch.zeros(d_in, d_in, device="cuda") if with_dxx else None
+    K.kronq_accumulate(xq, xfp if with_dxx else None, g, hx, hg, dxx)
+    torch.cuda.synchronize()
+    return hx, hg, dxx
+
+
+# ------------------------------------------------------------------------------ accumulate
+
+@pytest.mark.parametrize("n,d_in,d_out", [(2048, 256, 256), (1000, 200, 72), (77, 64, 136),
+                                          (4100, 384, 520), (64, 8, 16)])
+def test_accumulate_matches_oracle(K, n, d_in, d_out):
+    xq, xfp, g, *_ = layer_inputs(d_out, d_in, n, tag=("acc", n, d_in, d_out))
+    hx, hg, dxx = gpu_sums(K, xq, xfp, g)
+    ohx, ohg, odxx = O.accumulate(h64(xq), h64(xfp), h64(g))
+    assert rel(h64(hx), ohx) <= TOL
+    assert rel(h64(hg), ohg) <= TOL
+    assert rel(h64(dxx), odxx) <= TOL
+    assert torch.equal(hx, hx.T) and torch.equal(hg, hg.T)
+    print("rel err hx %.2e hg %.2e dxx %.2e" % (rel(h64(hx), ohx), rel(h64(hg), ohg),
+                                                  rel(h64(dxx), odxx)))
+
+
+def test_accumulate_is_additive_and_strided(K):
+    n, d = 3000, 130
+    base = torch.zeros(n, 136, dtype=torch.bfloat16, device="cuda")
+    base[:, :d] = synth.correlated_x(n, d, synth.seed_for("strided"), device="cuda")
+    x = base[:, :d]                                   # row stride 136, width 130
+    h1 = torch.zeros(d, d, device="cuda")
+    K.kronq_accumulate(x, None, None, h1)
+    h2 = torch.zeros(d, d, device="cuda")
+    K.kronq_accumulate(x[:1234], None, None, h2)
+    K.kronq_accumulate(x[1234:], None, None, h2)
+    torch.cuda.synchronize()
+    o = O.accumulate(h64(x))[0]
+    assert rel(h64(h1), o) <= TOL and rel(h64(h2), o) <= TOL
+    # n = 0 is a no-op
+    K.kronq_accumulate(x[:0], None, None, h2)
+    torch.cuda.synchronize()
+    assert rel(h64(h2), o) <= TOL
+
+
+@pytest.mark.parametrize("d", [4096, 11008])
+def test_accumulate_llama_width_sampled(K, d):
+    # LLaMA-2-7B widths (hidden 4096, MLP 11008), 16384 tokens, 16 sampled 128 x 128 tiles
+    n = 16384
+    x = synth.correlated_x(n, d, synth.seed_for("acc-full", d), device="cuda")
+    h = torch.zeros(d, d, device="cuda")
+    K.kronq_accumulate(x, None, None, h)
+    torch.cuda.synchronize()
+    r = np.random.default_rng(d)
+    xc = x.float()
+    for _ in range(16):
+        i0 = int(r.integers(0, d // 128)) * 128; j0 = int(r.integers(0, d // 128)) * 128
+        a = xc[:, i0:i0 + 128].double().cpu().numpy(); b = xc[:, j0:j0 + 128].double().cpu().numpy()
+        assert rel(h64(h[i0:i0 + 128, j0:j0 + 128]), a.T @ b) <= TOL
+    tr = float(np.sum(h64(x) ** 2))
+    assert abs(float(torch.trace(h.double())) - tr) <= TOL * tr
+
+
+# ------------------------------------------------------------------------------ biip
+
+def run_biip(K, P, w, hx_sum, hg_sum, dxx_sum, inv_n, si, so, flags):
+    r = P.biip(w, hx_sum, hg_sum, dxx_sum, inv_n, si, so, flags)
+    torch.cuda.synchronize()
+    return r
+
+
+@pytest.mark.parametrize("flags", [0, 1 | 2, 4 | 8, 15, 15 | 16])
+@pytest.mark.parametrize("shape", [(256, 256), (200, 96), (72, 520)])
+@pytest.mark.parametrize("w_dtype", [torch.float32, torch.bfloat16])
+def test_biip_matches_oracle(K, P, flags, shape, w_dtype):
+    d_out, d_in = shape
+    n = 1024
+    xq, xfp, g, w, si, so = layer_inputs(d_out, d_in, n, w_dtype=w_dtype,
+                                         tag=("biip", d_out, d_in))
+    hx, hg, dxx = gpu_sums(K, xq, xfp, g)
+    hg_in = hg.clone()
+    r = run_biip(K, P, w, hx, hg_in, dxx, 1.0 / n, si, so, flags)
+    o = O.biip(h64(w), h64(hx), h64(hg), h64(dxx), 1.0 / n, h64(si), h64(so), flags & 15)
+    assert rel(h64(r.w_prime), o["w"]) <= TOL
+    assert rel(h64(r.hx), o["hx"]) <= TOL
+    assert rel(h64(r.dxx), o["dxx"]) <= TOL
+    assert rel(h64(r.s_x), o["s_x"]) <= TOL and rel(h64(r.s_g), o["s_g"]) <= TOL
+    assert abs(float(r.tr[0]) - o["tr_hx"]) <= TOL * abs(o["tr_hx"])
+    assert abs(float(r.tr[1]) - o["tr_hg"]) <= TOL * abs(o["tr_hg"])
+    if flags & 16:
+        assert rel(h64(hg_in), o["hg"]) <= TOL
+    else:
+        assert torch.equal(hg_in, hg)          # read-only without WRITE_HG
+
+
+def test_biip_llama_gate_shape(K, P):
+    # gate_proj of LLaMA-2-7B: 11008 x 4096 (output Hadamard blocks of 256, input 4096)
+    d_out, d_in, n = 11008, 4096, 4096
+    xq, _, g, w, si, so = layer_inputs(d_out, d_in, n, drift="none", w_dtype=torch.bfloat16,
+                                       tag="biip-gate")
+    hx = torch.zeros(d_in, d_in, device="cuda"); hg = torch.zeros(d_out, d_out, device="cuda")
+    K.kronq_accumulate(xq, None, g, hx, hg)
+    r = run_biip(K, P, w, hx, hg, None, 1.0 / n, si, so, 15)
+    o = O.biip(h64(w), h64(hx), h64(hg), None, 1.0 / n, h64(si), h64(so), 15)
+    assert rel(h64(r.w_prime), o["w"]) <= TOL
+    assert rel(h64(r.hx), o["hx"]) <= TOL
+    assert rel(h64(r.s_g), o["s_g"]) <= TOL
+    assert abs(float(r.tr[1]) - o["tr_hg"]) <= TOL * o["tr_hg"]
+
+
+# ------------------------------------------------------------------------------ cholinv
+
+def spd_gpu(d, seed, cond=1e3):
+    r = np.random.default_rng(seed)
+    q, _ = np.linalg.qr(r.standard_normal((d, d)))
+    ev = np.exp(r.uniform(0, math.log(cond), d))
+    return torch.tensor((q * ev) @ q.T, dtype=torch.float32, device="cuda")
+
+
+@pytest.mark.parametrize("d", [256, 200, 65, 64, 1, 513])
+def test_cholinv_matches_oracle(K, d):
+    h = spd_gpu(d, d)
+    o = O.cholinv(h64(h), 0.01)
+    k = h.clone()
+    info = torch.empty(1, dtype=torch.int32, device="cuda")
+    K.kronq_cholinv(k, 0.01, info, K.CHOLINV_SYNC)
+    assert int(info) == -1
+    assert rel(h64(k), o) <= TOL
+    assert torch.all(torch.tril(k, -1) == 0)
+
+
+@pytest.mark.parametrize("d", [4096, 11008])
+def test_cholinv_llama_width_residual(K, d):
+    n = 3 * d
+    x = synth.correlated_x(n, d, synth.seed_for("chol", d), device="cuda")
+    h = torch.zeros(d, d, device="cuda")
+    K.kronq_accumulate(x, None, None, h)
+    h /= n
+    k = h.clone()
+    info = torch.empty(1, dtype=torch.int32, device="cuda")
+    K.kronq_cholinv(k, 0.01, info, K.CHOLINV_SYNC)
+    hd = h64(h); kd = h64(k)
+    lam = 0.01 * np.mean(np.diag(hd))
+    a = hd + lam * np.eye(d)
+    r = np.random.default_rng(0)
+    for _ in range(8):
+        v = r.standard_normal(d)
+        res = kd.T @ (kd @ (a @ v)) - v
+        assert np.linalg.norm(res) <= TOL * np.linalg.norm(v)
+    assert np.all(np.diag(kd) > 0)
+
+
+def test_cholinv_not_positive_definite(K):
+    h = torch.eye(96, device="cuda")
+    h[40, 40] = -1000.0
+    info = torch.empty(1, dtype=torch.int32, device="cuda")
+    with pytest.raises(K.KronqError) as e:
+        K.kronq_cholinv(h, 0.0, info, K.CHOLINV_SYNC)
+    assert e.value.status == K.ERR_NOT_PD
+    assert int(info) == 40
+    # asynchronous form reports through info only
+    h2 = torch.eye(96, device="cuda"); h2[5, 5] = -1.0
+    K.kronq_cholinv(h2, 0.0, info, 0)
+    torch.cuda.synchronize()
+    assert int(info) == 5
+
+
+# ------------------------------------------------------------------------------ quantize
+
+def check_codes(gpu, oracle_res, total):
+    mism = (h64(gpu) != oracle_res["codes"]).sum()
+    assert mism == 0, f"{mism} codes differ away from rounding boundaries"
+    assert oracle_res["near_tie"].sum() <= 1e-3 * total
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+@pytest.mark.parametrize("with_dxx", [False, True])
+@pytest.mark.parametrize("shape", [(256, 256), (96, 200), (130, 384)])
+def test_quantize_matches_oracle(K, P, bits, with_dxx, shape):
+    d_out, d_in = shape
+    n = 2048
+    xq, xfp, g, w, si, so = layer_inputs(d_out, d_in, n, drift="rel0.05", tag=("q", shape))
+    hx, hg, dxx = gpu_sums(K, xq, xfp, g, with_dxx=with_dxx)
+    r = P.biip(w, hx, hg, dxx, 1.0 / n, si, so, 15)
+    wp = r.w_prime.clone(); dxx_p = None if dxx is None else r.dxx.clone()
+    P.cholinv(r, 0.01, sync=True)
+    kk = r.hx.clone()
+    P.quantize(r, bits)
+    torch.cuda.synchronize()
+    o = O.quantize_layer(h64(wp), h64(kk), None if dxx_p is None else h64(dxx_p), bits,
+                         follow_codes=h64(r.codes))
+    assert np.array_equal(h64(r.scale), o["scale"].astype(np.float64))
+    assert np.array_equal(h64(r.zero), o["zero"].astype(np.float64))
+    check_codes(r.codes, o, d_out * d_in)
+    assert rel(h64(r.w_hat), o["w_hat"]) <= TOL
+
+
+def test_quantize_llama_shape_sampled_rows(K, P):
+    # q_proj of LLaMA-2-7B (4096 x 4096), 4 bits: 48 random rows re-run by the oracle from the
+    # GPU's K and W' (rows are independent given K)
+    d_out = d_in = 4096
+    n = 8192
+    xq, _, g, w, si, so = layer_inputs(d_out, d_in, n, drift="none", w_dtype=torch.bfloat16,
+                                       tag="q-full")
+    hx = torch.zeros(d_in, d_in, device="cuda"); hg = torch.zeros(d_out, d_out, device="cuda")
+    K.kronq_accumulate(xq, None, g, hx, hg)
+    r = P.biip(w, hx, hg, None, 1.0 / n, si, so, 15)
+    wp = r.w_prime.clone()
+    P.cholinv(r, 0.01, sync=True)
+    P.quantize(r, 4)
+    torch.cuda.synchronize()
+    rows = np.random.default_rng(1).choice(d_out, 48, replace=False)
+    o = O.quantize_layer(h64(wp[rows]), h64(r.hx), None, 4, follow_codes=h64(r.codes[rows]))
+    check_codes(r.codes[rows], o, 48 * d_in)
+    assert rel(h64(r.w_hat[rows]), o["w_hat"]) <= TOL
+
+
+# ------------------------------------------------------------------------------ end to end
+
+@pytest.mark.parametrize("flags", [0, 15])
+def test_layer256_end_to_end(K, P, flags):
+    # single 256 x 256 layer, 2048 tokens, fp32 W, X~ = X + N(0, 0.01^2), 2 bits, damp 0.01
+    d = 256; n = 2048; bits = 2
+    xq, xfp, g, w, si, so = layer_inputs(d, d, n, drift="abs0.01", tag="layer256")
+    hx, hg, dxx = gpu_sums(K, xq, xfp, g)
+    r = P.quantize_sublayer(w, hx, hg, dxx, 1.0 / n, si, so, bits, flags=flags)
+    torch.cuda.synchronize()
+    ohx, ohg, odxx = O.accumulate(h64(xq), h64(xfp), h64(g))
+    ob = O.biip(h64(w), ohx, ohg, odxx, 1.0 / n, h64(si), h64(so), flags)
+    ok = O.cholinv(ob["hx"], 0.01)
+    oq = O.quantize_layer(ob["w"], ok, ob["dxx"], bits, follow_codes=h64(r.codes))
+    check_codes(r.codes, oq, d * d)
+    assert rel(h64(r.w_hat), oq["w_hat"]) <= TOL
+    hg_p = ob["hg"]
+    j_gpu = O.objective(ob["w"], h64(r.w_hat), ob["hx"], hg_p, ob["dxx"])
+    j_ora = O.objective(ob["w"], oq["w_hat"], ob["hx"], hg_p, ob["dxx"])
+    assert abs(j_gpu - j_ora) <= TOL * abs(j_ora)
+
+
+def test_no_device_error_recorded(K):
+    assert K.kronq_device_error() == 0
