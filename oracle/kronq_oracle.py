@@ -311,9 +311,10 @@ def quantize_layer(w, k, dxx=None, bits: int = 4, follow_codes=None, tie_tol: fl
 
     follow_codes: optional array of codes from another implementation. Where this oracle's
     value sits within tie_tol grid units of a rounding boundary (a half-integer of w/scale) it
-    adopts that code instead of its own, and records a near-tie. Every other code is its own.
+    adopts that code instead of its own, and records a near-tie; where it adopts a code that
+    differs from its own decision it also records a disagreement. Every other code is its own.
     Returns dict: codes (uint8), scale, zero, w_hat (fp64), near_tie (bool mask),
-    pre (fp64: each column's value just before it was quantized).
+    disagree (bool mask), pre (fp64: each column's value just before it was quantized).
     """
     w0 = np.asarray(w, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
@@ -323,6 +324,7 @@ def quantize_layer(w, k, dxx=None, bits: int = 4, follow_codes=None, tie_tol: fl
     cur = w0.copy()
     codes = np.zeros((d_out, d_in), dtype=np.uint8)
     near = np.zeros((d_out, d_in), dtype=bool)
+    disagree = np.zeros((d_out, d_in), dtype=bool)
     pre = np.zeros((d_out, d_in))
     for p in range(d_in):
         col = cur[:, p].copy()
@@ -333,7 +335,9 @@ def quantize_layer(w, k, dxx=None, bits: int = 4, follow_codes=None, tie_tol: fl
             dist = np.abs(t - (np.floor(t) + 0.5))
             tie = dist <= tie_tol
             near[:, p] = tie
-            c = np.where(tie, np.asarray(follow_codes)[:, p].astype(np.float32), c)
+            other = np.asarray(follow_codes)[:, p].astype(np.float32)
+            disagree[:, p] = tie & (other != c)
+            c = np.where(tie, other, c)
         dq = dequantize(c, scale, zero).astype(np.float64)
         delta = (col - dq) / k[p, p]
         if p + 1 < d_in:
@@ -343,7 +347,7 @@ def quantize_layer(w, k, dxx=None, bits: int = 4, follow_codes=None, tie_tol: fl
         cur[:, p] = dq
         codes[:, p] = c.astype(np.uint8)
     return {"codes": codes, "scale": scale, "zero": zero, "w_hat": cur, "near_tie": near,
-            "pre": pre}
+            "disagree": disagree, "pre": pre}
 
 
 # ------------------------------------------------------------------------------------------

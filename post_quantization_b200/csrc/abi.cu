@@ -158,6 +158,7 @@ kronq_status kronq_accumulate(const void* xq, int64_t ld_xq, const void* xfp, in
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (n < 0) return fail(KRONQ_ERR_SHAPE, "n < 0");
   if (!hx_sum && !hg_sum && !dxx_sum) return fail(KRONQ_ERR_INVALID_ARG, "no output requested");
+  if (n == 0) return KRONQ_OK;   // nothing to add (inputs may be empty/NULL)
   if ((hx_sum || dxx_sum) && d_in <= 0) return fail(KRONQ_ERR_SHAPE, "d_in <= 0");
   if (hg_sum && d_out <= 0) return fail(KRONQ_ERR_SHAPE, "d_out <= 0");
   if (hx_sum || dxx_sum) KQ_TRY(check_bf16_matrix(xq, ld_xq, d_in, "xq"));
@@ -167,7 +168,6 @@ kronq_status kronq_accumulate(const void* xq, int64_t ld_xq, const void* xfp, in
     if (o && !aligned(o, 16)) return fail(KRONQ_ERR_INVALID_ARG, "output not 16-byte aligned");
   if (dxx_sum) KQ_TRY(check_ws(workspace, workspace_bytes, drift_ws(n, d_in)));
   KQ_TRY(kronq_device_check());
-  if (n == 0) return KRONQ_OK;
 
   if (hx_sum) {
     KQ_TRY(launch_accumulate_tc(xq, ld_xq, xq, ld_xq, n, d_in, d_in, hx_sum, d_in, true, s));

@@ -46,6 +46,16 @@ def h64(t):
     return t.detach().double().cpu().numpy()
 
 
+def padded(t):
+    """Same values in storage whose row stride is a multiple of 8 elements (16 bytes)."""
+    c = t.shape[1]
+    if c % 8 == 0:
+        return t
+    base = torch.zeros(t.shape[0], (c + 7) // 8 * 8, dtype=t.dtype, device=t.device)
+    base[:, :c] = t
+    return base[:, :c]
+
+
 def layer_inputs(d_out, d_in, n, drift="abs0.01", w_dtype=torch.float32, tag="t", dev="cuda"):
     xfp = synth.correlated_x(n, d_in, synth.seed_for(tag, "X"), device=dev)
     if drift == "none":
@@ -58,7 +68,7 @@ def layer_inputs(d_out, d_in, n, drift="abs0.01", w_dtype=torch.float32, tag="t"
     w = synth.weight(d_out, d_in, synth.seed_for(tag, "W"), dtype=w_dtype, device=dev)
     si = synth.rademacher(d_in, synth.seed_for(tag, "si"), device=dev)
     so = synth.rademacher(d_out, synth.seed_for(tag, "so"), device=dev)
-    return xq, xfp, g, w, si, so
+    return padded(xq), padded(xfp), padded(g), w, si, so
 
 
 def gpu_sums(K, xq, xfp, g, with_dxx=True):
@@ -230,9 +240,14 @@ def test_cholinv_not_positive_definite(K):
 # ------------------------------------------------------------------------------ quantize
 
 def check_codes(gpu, oracle_res, total):
+    # every code the oracle decides on its own (away from a rounding boundary) must match, and
+    # the oracle's own decision may differ from the GPU's on at most 0.1% of entries, all of
+    # them within 1e-3 grid units of a boundary
     mism = (h64(gpu) != oracle_res["codes"]).sum()
     assert mism == 0, f"{mism} codes differ away from rounding boundaries"
-    assert oracle_res["near_tie"].sum() <= 1e-3 * total
+    dis = int(oracle_res["disagree"].sum())
+    print(f"near-ties {int(oracle_res['near_tie'].sum())}, disagreements {dis} of {total}")
+    assert dis <= 1e-3 * total
 
 
 @pytest.mark.parametrize("bits", [2, 3, 4, 8])

@@ -385,6 +385,9 @@ def test_follow_mode_adopts_only_near_ties():
     other = (base["codes"].astype(int) + 1) % 4
     fol = O.quantize_layer(w, k, None, 2, follow_codes=other)
     assert np.array_equal(fol["codes"] != base["codes"], fol["near_tie"] & (fol["codes"] != base["codes"]))
+    assert not same["disagree"].any()
+    # a disagreement is recorded exactly where a different code was adopted at a near-tie
+    assert np.array_equal(fol["disagree"][:, 0], fol["near_tie"][:, 0] & (other[:, 0] != base["codes"][:, 0]))
 
 
 # ------------------------------------------------------------------ incoherence figure (P10)
