@@ -2,15 +2,18 @@
 //
 // KronQ (hyper.ai summary), Method, OBS update: the rows "[H_X^-1]_p,p+1:" that the column
 // update subtracts are the rows of K. Route: reverse-order (UL) Cholesky H + lambda I = R R^T
-// with R upper, blocked from the bottom-right corner, then the blocked triangular inverse
-// K = R^-1 (by uniqueness of the Cholesky factorization, K is the upper Cholesky factor of the
-// damped inverse). lambda = damp_rel * mean(diag H).
+// with R upper, and K = R^-1 (by uniqueness of the Cholesky factorization, K is the upper
+// Cholesky factor of the damped inverse). lambda = damp_rel * mean(diag H).
 //
-// Per 64-wide block (from the last one up):
-//   diag    one CTA factors the block (A22 = R22 R22^T) and inverts it (K22 = R22^-1) in smem
-//   panel   R12 = A12 K22^T                       (fp32 GEMM)
-//   update  A11 -= R12 R12^T, upper triangle only (fp32 GEMM)
-// then, per block row from the bottom:  K_i,>i = -K_ii (R_i,>i K_>i,>i).
+// Recursive blocked algorithm on a diagonal block A = [[A11, A12], [A12^T, A22]] (upper triangle
+// stored, lower triangle zero), which it overwrites with K:
+//   K22 = chol_inv(A22)
+//   R12 = A12 K22^T                 (A12 = R12 R22^T)
+//   A11 <- A11 - R12 R12^T          (upper triangle)
+//   K11 = chol_inv(A11)
+//   K12 = -K11 R12 K22              ([[R11, R12], [0, R22]]^-1)
+// Leaves of at most 64 columns are factored and inverted in shared memory by one CTA. The four
+// products per level are large square fp32 GEMMs that skip the zero triangles of K.
 #include <cmath>
 
 #include "common.cuh"
@@ -55,61 +58,56 @@ __global__ void prep_kernel(float* __restrict__ a, int d, const float* __restric
   }
 }
 
-// Factor the nb x nb diagonal block at (j0, j0): A22 = R R^T (R upper), write K22 = R^-1.
-__global__ void __launch_bounds__(256) ul_diag_kernel(float* __restrict__ a, int d, int j0, int nb,
-                                                      int32_t* __restrict__ info) {
-  __shared__ float S[NB][NB + 1];
-  __shared__ float Kt[NB][NB + 1];
-  __shared__ int failed;
+// Leaf: factor the nb x nb diagonal block at a (ld) as A = R R^T (R upper) and overwrite its
+// upper triangle with K = R^-1. One CTA of 256 threads.
+__global__ void __launch_bounds__(256) leaf_kernel(float* __restrict__ a, int64_t ld, int nb,
+                                                   int j0, int32_t* __restrict__ info) {
+  __shared__ float S[NB][NB + 1];   // running block (upper triangle), then the inverse K
+  __shared__ float R[NB][NB + 1];   // factor R
   if (*info >= 0) return;
   const int tid = threadIdx.x;
-  if (tid == 0) failed = 0;
   for (int e = tid; e < NB * NB; e += blockDim.x) {
     const int i = e / NB, k = e % NB;
-    float v = 0.f;
-    if (i < nb && k < nb && k >= i) v = a[static_cast<int64_t>(j0 + i) * d + j0 + k];
-    if (i >= nb || k >= nb) v = (i == k) ? 1.f : 0.f;
-    S[i][k] = v;
-    Kt[i][k] = 0.f;
+    S[i][k] = (i < nb && k < nb && k >= i) ? a[i * ld + k] : 0.f;
+    R[i][k] = 0.f;
   }
   __syncthreads();
-  // column c from the last to the first
-  const int col = tid & (NB - 1);   // thread's column in the trailing update
-  const int half = tid / NB;        // 0..3: strided rows
+  // UL factorization, column c from the last to the first; one barrier per column.
+  const int kc = tid & (NB - 1);   // this thread's column in the update
+  const int i0 = tid >> 6;         // and its first row (rows i0, i0 + 4, ...)
   for (int c = nb - 1; c >= 0; --c) {
-    if (tid == 0) {
-      const float piv = S[c][c];
-      if (!(piv > 0.f) || !isfinite(piv)) {
-        failed = 1;
-        *info = j0 + c;
-      } else {
-        S[c][c] = sqrtf(piv);
-      }
+    const float piv = S[c][c];
+    if (!(piv > 0.f) || !isfinite(piv)) {
+      if (tid == 0) *info = j0 + c;
+      return;                       // uniform: every thread read the same pivot
     }
-    __syncthreads();
-    if (failed) return;
-    const float r = S[c][c];
-    for (int i = tid; i < c; i += blockDim.x) S[i][c] = S[i][c] / r;
-    __syncthreads();
-    if (col < c) {
-      const float rk = S[col][c];
-      for (int i = half; i <= col; i += 4) S[i][col] -= S[i][c] * rk;
+    const float inv = 1.f / piv;
+    if (tid < c) R[tid][c] = S[tid][c] * rsqrtf(piv);
+    if (tid == c) R[c][c] = sqrtf(piv);
+    if (kc < c) {
+      const float s_kc = S[kc][c] * inv;
+      for (int i = i0; i <= kc; i += 4) S[i][kc] -= S[i][c] * s_kc;
     }
     __syncthreads();
   }
-  // K = R^-1, one row of K per step from the bottom: K_ij = (delta_ij - sum_{l>i} R_il K_lj) / R_ii
+  // K = R^-1 row by row from the bottom: K_ij = (delta_ij - sum_{i<l<=j} R_il K_lj) / R_ii.
+  // Four threads share one column's dot product. K reuses the storage of S.
+  float(*Kt)[NB + 1] = S;
+  for (int e = tid; e < NB * NB; e += blockDim.x) Kt[e / NB][e % NB] = 0.f;
+  __syncthreads();
+  const int j = tid >> 2, part = tid & 3;
   for (int i = nb - 1; i >= 0; --i) {
-    for (int j = tid; j < nb; j += blockDim.x) {
-      if (j < i) continue;
-      float s = (i == j) ? 1.f : 0.f;
-      for (int l = i + 1; l <= j; ++l) s -= S[i][l] * Kt[l][j];
-      Kt[i][j] = s / S[i][i];
-    }
+    float s = 0.f;
+    if (j < nb && j > i)
+      for (int l = i + 1 + part; l <= j; l += 4) s += R[i][l] * Kt[l][j];
+    s += __shfl_xor_sync(0xffffffffu, s, 1);
+    s += __shfl_xor_sync(0xffffffffu, s, 2);
+    if (part == 0 && j < nb && j >= i) Kt[i][j] = ((i == j ? 1.f : 0.f) - s) / R[i][i];
     __syncthreads();
   }
   for (int e = tid; e < nb * nb; e += blockDim.x) {
     const int i = e / nb, k = e % nb;
-    a[static_cast<int64_t>(j0 + i) * d + j0 + k] = (k >= i) ? Kt[i][k] : 0.f;
+    a[i * ld + k] = (k >= i) ? Kt[i][k] : 0.f;
   }
 }
 
@@ -124,17 +122,60 @@ __global__ void copy_panel_kernel(const float* __restrict__ src, int64_t lds, fl
   }
 }
 
+struct Ctx {
+  int64_t ld;
+  float* ws;        // at least (n/2)^2 floats
+  int32_t* info;
+  cudaStream_t stream;
+};
+
+// Overwrite the n x n diagonal block at a (global index j0) with K.
+kronq_status chol_inv_rec(const Ctx& c, float* a, int n, int j0) {
+  if (n <= NB) {
+    leaf_kernel<<<1, 256, 0, c.stream>>>(a, c.ld, n, j0, c.info);
+    return check_launch("leaf_kernel");
+  }
+  // bottom-right part: a multiple of NB columns, about half
+  int n2 = ((n / 2 + NB - 1) / NB) * NB;
+  if (n2 >= n) n2 = n - NB;
+  const int n1 = n - n2;
+  float* a11 = a;
+  float* a12 = a + n1;
+  float* a22 = a + static_cast<int64_t>(n1) * c.ld + n1;
+  const int64_t ld = c.ld;
+  KQ_TRY(chol_inv_rec(c, a22, n2, j0 + n1));                                    // K22
+  KQ_TRY(sgemm(false, true, n1, n2, n2, 1.f, a12, ld, a22, ld, 0.f, c.ws, n2, false, c.info,
+               c.stream, GEMM_B_LOWER));                                        // R12 = A12 K22^T
+  {
+    int64_t blocks = (static_cast<int64_t>(n1) * n2 + 255) / 256;
+    if (blocks > 8192) blocks = 8192;
+    copy_panel_kernel<<<static_cast<int>(blocks), 256, 0, c.stream>>>(c.ws, n2, a12, ld, n1, n2);
+    KQ_TRY(check_launch("copy_panel_kernel"));
+  }
+  KQ_TRY(sgemm(false, true, n1, n1, n2, -1.f, a12, ld, a12, ld, 1.f, a11, ld, true, c.info,
+               c.stream));                                                      // A11 -= R12 R12^T
+  KQ_TRY(chol_inv_rec(c, a11, n1, j0));                                         // K11
+  KQ_TRY(sgemm(false, false, n1, n2, n2, 1.f, a12, ld, a22, ld, 0.f, c.ws, n2, false, c.info,
+               c.stream, GEMM_B_UPPER));                                        // T = R12 K22
+  KQ_TRY(sgemm(false, false, n1, n2, n1, -1.f, a11, ld, c.ws, n2, 0.f, a12, ld, false, c.info,
+               c.stream, GEMM_A_UPPER));                                        // K12 = -K11 T
+  return KRONQ_OK;
+}
+
+size_t ws_floats(int d) {
+  const size_t h = static_cast<size_t>(d / 2 + NB);
+  return h * h;
+}
+
 }  // namespace
 
-size_t cholinv_workspace_bytes(int d) {
-  return align256(sizeof(float) * static_cast<size_t>(d) * NB) + 256;
-}
+size_t cholinv_workspace_bytes(int d) { return align256(sizeof(float) * ws_floats(d)) + 256; }
 
 kronq_status run_cholinv(float* a, int d, float damp_rel, int32_t* info, void* ws,
                          cudaStream_t stream) {
-  float* panel = static_cast<float*>(ws);   // up to d x NB
+  float* scratch = static_cast<float*>(ws);
   float* lam = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
-                                        align256(sizeof(float) * static_cast<size_t>(d) * NB));
+                                        align256(sizeof(float) * ws_floats(d)));
   damping_kernel<<<1, 1024, 0, stream>>>(a, d, damp_rel, lam, info);
   KQ_TRY(check_launch("damping_kernel"));
   {
@@ -142,42 +183,8 @@ kronq_status run_cholinv(float* a, int d, float damp_rel, int32_t* info, void* w
     prep_kernel<<<grid, 256, 0, stream>>>(a, d, lam);
     KQ_TRY(check_launch("prep_kernel"));
   }
-  // factorization, blocks from the bottom-right corner
-  for (int j1 = d; j1 > 0; j1 -= NB) {
-    const int j0 = j1 > NB ? j1 - NB : 0;
-    const int nb = j1 - j0;
-    ul_diag_kernel<<<1, 256, 0, stream>>>(a, d, j0, nb, info);
-    KQ_TRY(check_launch("ul_diag_kernel"));
-    if (j0 == 0) break;
-    // R12 = A12 K22^T  -> panel (j0 x nb), then back into A12
-    KQ_TRY(sgemm(false, true, j0, nb, nb, 1.f, a + j0, d, a + static_cast<int64_t>(j0) * d + j0,
-                 d, 0.f, panel, nb, false, info, stream));
-    {
-      int64_t blocks = (static_cast<int64_t>(j0) * nb + 255) / 256;
-      if (blocks > 4096) blocks = 4096;
-      copy_panel_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(panel, nb, a + j0, d, j0, nb);
-      KQ_TRY(check_launch("copy_panel_kernel"));
-    }
-    // A11 -= R12 R12^T (upper triangle)
-    KQ_TRY(sgemm(false, true, j0, j0, nb, -1.f, panel, nb, panel, nb, 1.f, a, d, true, info,
-                 stream));
-  }
-  // inversion, block rows from the bottom: K_i,>i = -K_ii (R_i,>i K_>i,>i)
-  for (int i1 = d; i1 > 0;) {
-    const int i0 = i1 > NB ? i1 - NB : 0;   // same block boundaries as the factorization
-    const int nbi = i1 - i0;
-    const int m = d - i1;
-    if (m > 0) {
-      // T = R_i,>i K_>i,>i  (nbi x m)
-      KQ_TRY(sgemm(false, false, nbi, m, m, 1.f, a + static_cast<int64_t>(i0) * d + i1, d,
-                   a + static_cast<int64_t>(i1) * d + i1, d, 0.f, panel, m, false, info, stream));
-      // K_i,>i = -K_ii T
-      KQ_TRY(sgemm(false, false, nbi, m, nbi, -1.f, a + static_cast<int64_t>(i0) * d + i0, d,
-                   panel, m, 0.f, a + static_cast<int64_t>(i0) * d + i1, d, false, info, stream));
-    }
-    i1 = i0;
-  }
-  return KRONQ_OK;
+  Ctx c{d, scratch, info, stream};
+  return chol_inv_rec(c, a, d, 0);
 }
 
 }  // namespace kq

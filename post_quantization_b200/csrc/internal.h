@@ -53,9 +53,16 @@ kronq_status run_quantize(const float* w, const float* k, const float* dxx, int 
 //   op(A) is M x K: A stored M x K (lda) or, when ta, K x M.
 //   op(B) is K x N: B stored K x N (ldb) or, when tb, N x K.
 //   upper_only: only elements with col >= row are written (tiles fully below are skipped).
+//   tri: zero structure of the operands (the zeros must be stored), used to skip K ranges:
+//     GEMM_A_UPPER  op(A)[m][k] = 0 for k < m
+//     GEMM_B_UPPER  op(B)[k][n] = 0 for k > n
+//     GEMM_B_LOWER  op(B)[k][n] = 0 for k < n
+//   skip_if_nonneg: device int; the kernel does nothing when it holds a value >= 0.
+enum { GEMM_A_UPPER = 1, GEMM_B_UPPER = 2, GEMM_B_LOWER = 4 };
 kronq_status sgemm(bool ta, bool tb, int m, int n, int k, float alpha, const float* a,
                    int64_t lda, const float* b, int64_t ldb, float beta, float* c, int64_t ldc,
-                   bool upper_only, const int32_t* skip_if_nonneg, cudaStream_t stream);
+                   bool upper_only, const int32_t* skip_if_nonneg, cudaStream_t stream,
+                   int tri = 0);
 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 

@@ -22,7 +22,7 @@ namespace kq {
 namespace {
 
 constexpr int QB = 128;        // column block
-constexpr int QROWS = 32;      // rows per CTA in the block solve
+constexpr int QROWS = 128;     // rows (= threads) per CTA in the block solve
 constexpr int QSUB = 32;       // columns per register-resident sub-block
 
 // Per-row grid from W (before the solve), all decisions in fp32:
@@ -73,25 +73,51 @@ __global__ void __launch_bounds__(QROWS) block_solve_kernel(
   float* Ks = sm;                              // QB x QB block of K (padding = identity)
   float* St = Ks + QB * QB;                    // QROWS x (QB + 1): running row values
   float* Dt = St + QROWS * (QB + 1);           // QROWS x (QB + 1): errors
+  float* Rd = Dt + QROWS * (QB + 1);           // QB reciprocals of K's diagonal
   const int tid = threadIdx.x;
   const int row0 = blockIdx.x * QROWS;
   const int rows = min(QROWS, d_out - row0);
 
-  for (int e = tid; e < QB * QB; e += blockDim.x) {
-    const int i = e / QB, j = e % QB;
-    float v;
-    if (i < bw && j < bw)
-      v = (j >= i) ? k[static_cast<int64_t>(b0 + i) * d_in + b0 + j] : 0.f;
-    else
-      v = (i == j) ? 1.f : 0.f;
-    Ks[e] = v;
+  // K block (rows/cols beyond bw become identity so that padding never feeds back) and the
+  // rows' block of running weights, with 16-byte loads where the layout allows
+  const bool vec = (d_in % 4 == 0) && bw == QB &&
+                   ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(w_hat)) & 15u) == 0;
+  if (vec) {
+    for (int e = tid; e < QB * QB / 4; e += blockDim.x) {
+      const int i = e / (QB / 4), j4 = (e % (QB / 4)) * 4;
+      float4 v = *reinterpret_cast<const float4*>(k + static_cast<int64_t>(b0 + i) * d_in + b0 + j4);
+      if (j4 + 0 < i) v.x = 0.f;
+      if (j4 + 1 < i) v.y = 0.f;
+      if (j4 + 2 < i) v.z = 0.f;
+      if (j4 + 3 < i) v.w = 0.f;
+      *reinterpret_cast<float4*>(Ks + i * QB + j4) = v;
+    }
+    for (int e = tid; e < QROWS * QB / 4; e += blockDim.x) {
+      const int r = e / (QB / 4), c4 = (e % (QB / 4)) * 4;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (r < rows) v = *reinterpret_cast<const float4*>(w_hat + static_cast<int64_t>(row0 + r) * d_in + b0 + c4);
+      float* dst = St + r * (QB + 1) + c4;
+      dst[0] = v.x; dst[1] = v.y; dst[2] = v.z; dst[3] = v.w;
+    }
+  } else {
+    for (int e = tid; e < QB * QB; e += blockDim.x) {
+      const int i = e / QB, j = e % QB;
+      float v;
+      if (i < bw && j < bw)
+        v = (j >= i) ? k[static_cast<int64_t>(b0 + i) * d_in + b0 + j] : 0.f;
+      else
+        v = (i == j) ? 1.f : 0.f;
+      Ks[e] = v;
+    }
+    for (int e = tid; e < QROWS * QB; e += blockDim.x) {
+      const int r = e / QB, c = e % QB;
+      float v = 0.f;
+      if (r < rows && c < bw) v = w_hat[static_cast<int64_t>(row0 + r) * d_in + b0 + c];
+      St[r * (QB + 1) + c] = v;
+    }
   }
-  for (int e = tid; e < QROWS * QB; e += blockDim.x) {
-    const int r = e / QB, c = e % QB;
-    float v = 0.f;
-    if (r < rows && c < bw) v = w_hat[static_cast<int64_t>(row0 + r) * d_in + b0 + c];
-    St[r * (QB + 1) + c] = v;
-  }
+  __syncthreads();
+  if (tid < QB) Rd[tid] = 1.f / Ks[tid * QB + tid];
   __syncthreads();
 
   const int row = row0 + tid;
@@ -114,7 +140,7 @@ __global__ void __launch_bounds__(QROWS) block_solve_kernel(
       code = fminf(fmaxf(code, 0.f), maxq);
       const float dq = __fmul_rn(sc, __fsub_rn(code, zr));
       const float* kr = Ks + (sb + p) * QB + sb;
-      err[p] = __fdiv_rn(__fsub_rn(w[p], dq), kr[p]);
+      err[p] = __fsub_rn(w[p], dq) * Rd[sb + p];
 #pragma unroll
       for (int j = p + 1; j < QSUB; ++j) w[j] = fmaf(-err[p], kr[j], w[j]);
       w[p] = dq;
@@ -191,7 +217,7 @@ kronq_status run_quantize(const float* w, const float* k, const float* dxx, int 
     float* t1 = reinterpret_cast<float*>(p);
     // M = D K^T, striu(M)
     KQ_TRY(sgemm(false, true, d_in, d_in, d_in, 1.f, dxx, d_in, k, d_in, 0.f, mm, d_in, false,
-                 nullptr, stream));
+                 nullptr, stream, GEMM_B_LOWER));
     {
       dim3 g((d_in + 255) / 256, d_in);
       striu_kernel<<<g, 256, 0, stream>>>(mm, d_in);
@@ -199,13 +225,13 @@ kronq_status run_quantize(const float* w, const float* k, const float* dxx, int 
     }
     // W~ = W + (W striu(M)) K
     KQ_TRY(sgemm(false, false, d_out, d_in, d_in, 1.f, w, d_in, mm, d_in, 0.f, t1, d_in, false,
-                 nullptr, stream));
+                 nullptr, stream, GEMM_B_UPPER));
     KQ_TRY(sgemm(false, false, d_out, d_in, d_in, 1.f, t1, d_in, k, d_in, 1.f, w_hat, d_in, false,
-                 nullptr, stream));
+                 nullptr, stream, GEMM_B_UPPER));
   }
 
   static bool attr = false;
-  const size_t smem = sizeof(float) * (QB * QB + 2 * QROWS * (QB + 1));
+  const size_t smem = sizeof(float) * (QB * QB + 2 * QROWS * (QB + 1) + QB);
   if (!attr) {
     KQ_CUDA_TRY(cudaFuncSetAttribute(block_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)smem));

@@ -19,10 +19,17 @@ __global__ void __launch_bounds__(256) sgemm_kernel(int M, int N, int K, float a
                                                     const float* __restrict__ A, int64_t lda,
                                                     const float* __restrict__ B, int64_t ldb,
                                                     float beta, float* __restrict__ C, int64_t ldc,
-                                                    int upper_only, const int32_t* skip) {
+                                                    int upper_only, int tri,
+                                                    const int32_t* skip) {
   if (skip && *skip >= 0) return;
   const int bm = blockIdx.y * TM, bn = blockIdx.x * TN;
   if (upper_only && bm > bn + TN - 1) return;
+  // K range that can be non-zero for this tile when an operand is triangular
+  int k_lo = 0, k_hi = K;
+  if (tri & GEMM_A_UPPER) k_lo = max(k_lo, bm);
+  if (tri & GEMM_B_LOWER) k_lo = max(k_lo, bn);
+  if (tri & GEMM_B_UPPER) k_hi = min(k_hi, bn + TN);
+  k_lo = (k_lo / TK) * TK;
   __shared__ __align__(16) float As[TK][TM + 4];
   __shared__ __align__(16) float Bs[TK][TN + 4];
   const int tid = threadIdx.x;
@@ -33,7 +40,7 @@ __global__ void __launch_bounds__(256) sgemm_kernel(int M, int N, int K, float a
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
 
-  for (int k0 = 0; k0 < K; k0 += TK) {
+  for (int k0 = k_lo; k0 < k_hi; k0 += TK) {
     // ---- stage op(A)[bm:bm+128, k0:k0+8] as As[k][m]
     if (!TA) {
       const int m = tid >> 1, kq = (tid & 1) * 4;
@@ -108,22 +115,22 @@ __global__ void __launch_bounds__(256) sgemm_kernel(int M, int N, int K, float a
 
 kronq_status sgemm(bool ta, bool tb, int m, int n, int k, float alpha, const float* a,
                    int64_t lda, const float* b, int64_t ldb, float beta, float* c, int64_t ldc,
-                   bool upper_only, const int32_t* skip, cudaStream_t stream) {
+                   bool upper_only, const int32_t* skip, cudaStream_t stream, int tri) {
   if (m <= 0 || n <= 0) return KRONQ_OK;
   dim3 grid((n + TN - 1) / TN, (m + TM - 1) / TM);
   const int up = upper_only ? 1 : 0;
   if (!ta && !tb)
     sgemm_kernel<false, false><<<grid, 256, 0, stream>>>(m, n, k, alpha, a, lda, b, ldb, beta, c,
-                                                         ldc, up, skip);
+                                                         ldc, up, tri, skip);
   else if (!ta && tb)
     sgemm_kernel<false, true><<<grid, 256, 0, stream>>>(m, n, k, alpha, a, lda, b, ldb, beta, c,
-                                                        ldc, up, skip);
+                                                        ldc, up, tri, skip);
   else if (ta && !tb)
     sgemm_kernel<true, false><<<grid, 256, 0, stream>>>(m, n, k, alpha, a, lda, b, ldb, beta, c,
-                                                        ldc, up, skip);
+                                                        ldc, up, tri, skip);
   else
     sgemm_kernel<true, true><<<grid, 256, 0, stream>>>(m, n, k, alpha, a, lda, b, ldb, beta, c,
-                                                       ldc, up, skip);
+                                                       ldc, up, tri, skip);
   return check_launch("sgemm_kernel");
 }
 
