@@ -144,6 +144,27 @@ KRONQ_API kronq_status kronq_biip(const void* w, int32_t w_dtype, float* w_out, 
                         double* tr_hx, double* tr_hg, void* workspace, size_t workspace_bytes,
                         kronq_stream_t stream);
 
+/* kronq_biip_noalloc - kronq_biip for callers that cannot allocate device memory.
+ *
+ * The paper has no counterpart to this call; it exists for deployment. Some callers cannot call
+ * cudaMalloc or hand the library a workspace: code running while a CUDA graph is being captured,
+ * plug-ins and host runtimes that only see buffers handed to them by their host framework, and
+ * services that reserve all device memory up front. This variant takes the same arguments as
+ * kronq_biip minus the workspace and uses a fixed scratch array of 1 MiB that lives in device
+ * memory (every GPU that loads this library holds it until the process exits). That limits it
+ * to 16 * (d_out + d_in) + about 1.5 KB <= 1 MiB (d_out + d_in up to about 65000, every LLaMA
+ * shape); larger layers get KRONQ_ERR_UNSUPPORTED with the needed size in the error detail.
+ * The first call on a device looks up the array's device address; make that first call before
+ * any stream capture. All calls in the process share the one array, so calls whose execution
+ * overlaps on the GPU (several streams or threads) race on it and must be ordered by the caller.
+ * The array keeps the last call's contents; the call clears what it needs cleared itself. */
+KRONQ_API kronq_status kronq_biip_noalloc(const void* w, int32_t w_dtype, float* w_out, float* hx,
+                                          float* hg, float* dxx, double inv_n,
+                                          const int8_t* sign_in, const int8_t* sign_out,
+                                          int32_t d_out, int32_t d_in, uint32_t flags,
+                                          float* s_x, float* s_g, double* tr_hx, double* tr_hg,
+                                          kronq_stream_t stream);
+
 /* ---------------------------------------------------------------------------------------
  * 3. kronq_cholinv - damped inverse Cholesky factor.
  *

@@ -15,6 +15,7 @@
 #include <cuda_bf16.h>
 
 #include <cmath>
+#include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
@@ -333,3 +334,52 @@ kronq_status run_biip(const BiipArgs& a, void* ws_raw, cudaStream_t stream) {
 }
 
 }  // namespace kq
+
+// ---------------------------------------------------------------------------------------------
+// Variant of kronq_biip that allocates nothing: its scratch is a fixed array in device memory
+// that every GPU holds from the moment this library is loaded until the process exits.
+// ---------------------------------------------------------------------------------------------
+namespace {
+constexpr size_t kBiipStaticScratchBytes = size_t(1) << 20;   // 1 MiB
+__device__ __align__(256) unsigned char g_biip_static_scratch[kBiipStaticScratchBytes];
+constexpr int kMaxScratchDevices = 64;
+void* g_biip_static_ptr[kMaxScratchDevices] = {nullptr};
+std::mutex g_biip_static_mu;
+}  // namespace
+
+extern "C" kronq_status kronq_biip_noalloc(const void* w, int32_t w_dtype, float* w_out, float* hx,
+                                           float* hg, float* dxx, double inv_n,
+                                           const int8_t* sign_in, const int8_t* sign_out,
+                                           int32_t d_out, int32_t d_in, uint32_t flags,
+                                           float* s_x, float* s_g, double* tr_hx, double* tr_hg,
+                                           kronq_stream_t stream) {
+  if (d_out <= 0 || d_in <= 0)
+    return kq::fail(KRONQ_ERR_SHAPE, "d_out and d_in must be positive");
+  const size_t need = kq::biip_workspace_bytes(d_out, d_in);
+  if (need > kBiipStaticScratchBytes)
+    return kq::fail(KRONQ_ERR_UNSUPPORTED,
+                    "kronq_biip_noalloc: d_out + d_in too large for the %zu-byte static scratch "
+                    "(%zu bytes needed); use kronq_biip with a workspace",
+                    kBiipStaticScratchBytes, need);
+  int dev = 0;
+  KQ_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxScratchDevices)
+    return kq::fail(KRONQ_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  void* scratch = nullptr;
+  {
+    // first call on this device: look up the device address of the static array
+    std::lock_guard<std::mutex> lock(g_biip_static_mu);
+    if (!g_biip_static_ptr[dev]) {
+      void* p = nullptr;
+      const cudaError_t e = cudaGetSymbolAddress(&p, g_biip_static_scratch);
+      if (e != cudaSuccess || !p)
+        return kq::fail(KRONQ_ERR_CUDA, "cudaGetSymbolAddress(static scratch): %s",
+                        cudaGetErrorString(e));
+      g_biip_static_ptr[dev] = p;
+    }
+    scratch = g_biip_static_ptr[dev];
+  }
+  return kronq_biip(w, w_dtype, w_out, hx, hg, dxx, inv_n, sign_in, sign_out, d_out, d_in, flags,
+                    s_x, s_g, tr_hx, tr_hg, scratch, kBiipStaticScratchBytes, stream);
+}
+

@@ -42,7 +42,7 @@ SYMBOLS = (
     "kronq_status_string", "kronq_last_error_detail", "kronq_version", "kronq_device_check",
     "kronq_device_error", "kronq_launch_count",
     "kronq_accumulate_workspace_size", "kronq_accumulate",
-    "kronq_biip_workspace_size", "kronq_biip",
+    "kronq_biip_workspace_size", "kronq_biip", "kronq_biip_noalloc",
     "kronq_cholinv_workspace_size", "kronq_cholinv",
     "kronq_quantize_layer_workspace_size", "kronq_quantize_layer",
     "kronq_score_allocate",
@@ -91,6 +91,9 @@ def load_library(path: str = LIB_PATH):
         "kronq_biip": (c_i32, [c_void_p, c_i32, c_void_p, c_void_p, c_void_p, c_void_p, c_dbl,
                                c_void_p, c_void_p, c_i32, c_i32, c_u32, c_void_p, c_void_p,
                                c_void_p, c_void_p, c_void_p, c_sz, c_void_p]),
+        "kronq_biip_noalloc": (c_i32, [c_void_p, c_i32, c_void_p, c_void_p, c_void_p, c_void_p,
+                                       c_dbl, c_void_p, c_void_p, c_i32, c_i32, c_u32, c_void_p,
+                                       c_void_p, c_void_p, c_void_p, c_void_p]),
         "kronq_cholinv_workspace_size": (c_sz, [c_i32]),
         "kronq_cholinv": (c_i32, [c_void_p, c_i32, c_flt, c_void_p, c_u32, c_void_p, c_sz,
                                   c_void_p]),
