@@ -5,7 +5,8 @@ q/k/v/o 4096x4096, gate/up 11008x4096, down 4096x11008; 262144 calibration token
 per-channel grid; BiIP on; X~ = X so the drift term is off):
   Kronecker-factor sums for the 4 distinct inputs (q/k/v share one) and the 7 output-gradient
   streams -> BiIP of every sublayer -> traces to the host -> scores and bit allocation ->
-  damped inverse factor -> column solve of every sublayer.
+  damped inverse factor -> column solve of every sublayer. The per-sublayer steps of the 7
+  sublayers run side by side on one CUDA stream each.
 Metric: quantized weight params/s (whole job: params of all ranks' blocks / max step time).
 Each rank quantizes its own block (weak scaling, no collective on the data path).
 
@@ -196,6 +197,7 @@ class Block:
         self.results = {}
         self.acc_events = []        # (start, end, flops) of each statistics call
         self.bits = None
+        self.streams = None         # one stream per sublayer for the per-sublayer steps
 
     def input_bytes(self):
         tot = 0
@@ -233,20 +235,20 @@ class Block:
                 d = h.shape[0]
                 self.acc_events.append((e0, e1, self.n * d * (d + 1)))
         inv_n = 1.0 / self.n
-        for s in wl.sublayers:
-            self.results[s.name] = P.biip(self.w[s.name], self.hx[s.x_stream], self.hg[s.name],
-                                          None, inv_n, self.si[s.name], self.so[s.name],
-                                          K.BIIP_FULL, ws=self.ws)
+        if self.streams is None:
+            self.streams = P.SublayerStreams(len(wl.sublayers), self.dev)
+        res = self.streams.biip([(self.w[s.name], self.hx[s.x_stream], self.hg[s.name], None,
+                                  inv_n, self.si[s.name], self.so[s.name], K.BIIP_FULL)
+                                 for s in wl.sublayers])
+        for s, r in zip(wl.sublayers, res):
+            self.results[s.name] = r
         tr = torch.stack([self.results[s.name].tr for s in wl.sublayers]).cpu()
         choices = wl.extra.get("choices", (wl.bits,))
         avg = wl.extra.get("avg_bits", float(wl.bits))
         _, self.bits = K.kronq_score_allocate(tr[:, 0].tolist(), tr[:, 1].tolist(),
                                               [s.d_out * s.d_in for s in wl.sublayers], choices,
                                               avg)
-        for s, b in zip(wl.sublayers, self.bits):
-            r = self.results[s.name]
-            P.cholinv(r, 0.01, ws=self.ws)
-            P.quantize(r, b, ws=self.ws)
+        self.streams.solve([self.results[s.name] for s in wl.sublayers], self.bits, 0.01)
 
 
 def run_gpu(args):

@@ -191,16 +191,21 @@ __device__ __forceinline__ void tmem_ld_wait() {
 }
 
 // Shared-memory matrix descriptor (sm_100 format): start address, leading/stride byte offsets,
-// descriptor version 1, 128-byte swizzle.
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes,
-                                                    uint32_t sbo_bytes) {
+// descriptor version 1, swizzle layout (2 = 128-byte swizzle with 16-byte atoms, 1 = 128-byte
+// swizzle with 32-byte atoms, the layout of MN-major 32-bit operands).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes,
+                                              uint32_t sbo_bytes, uint32_t layout) {
   uint64_t d = 0;
   d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
   d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
   d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
-  d |= 1ull << 46;   // descriptor version (Blackwell)
-  d |= 2ull << 61;   // layout: 128-byte swizzle
+  d |= 1ull << 46;                                   // descriptor version (Blackwell)
+  d |= static_cast<uint64_t>(layout & 7u) << 61;     // swizzle layout
   return d;
+}
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes,
+                                                    uint32_t sbo_bytes) {
+  return smem_desc(saddr, lbo_bytes, sbo_bytes, 2u);
 }
 
 // Instruction descriptor for kind::f16 with bf16 A/B, fp32 D, both operands MN-major.

@@ -49,21 +49,54 @@ kronq_status run_quantize(const float* w, const float* k, const float* dxx, int 
                           int bits, int block, uint8_t* codes, float* scale, float* zero,
                           float* w_hat, void* ws, cudaStream_t stream);
 
-// sgemm.cu: C = alpha * op(A) op(B) + beta * C, fp32 on CUDA cores.
-//   op(A) is M x K: A stored M x K (lda) or, when ta, K x M.
-//   op(B) is K x N: B stored K x N (ldb) or, when tb, N x K.
-//   upper_only: only elements with col >= row are written (tiles fully below are skipped).
-//   tri: zero structure of the operands (the zeros must be stored), used to skip K ranges:
-//     GEMM_A_UPPER  op(A)[m][k] = 0 for k < m
-//     GEMM_B_UPPER  op(B)[k][n] = 0 for k > n
-//     GEMM_B_LOWER  op(B)[k][n] = 0 for k < n
-//   skip_if_nonneg: device int; the kernel does nothing when it holds a value >= 0.
+// Zero structure of GEMM operands (the zeros must be stored), used to skip K ranges:
+//   GEMM_A_UPPER  A[m][k] = 0 for k < m
+//   GEMM_B_UPPER  op(B)[k][n] = 0 for k > n
+//   GEMM_B_LOWER  op(B)[k][n] = 0 for k < n
 enum { GEMM_A_UPPER = 1, GEMM_B_UPPER = 2, GEMM_B_LOWER = 4 };
-kronq_status sgemm(bool ta, bool tb, int m, int n, int k, float alpha, const float* a,
-                   int64_t lda, const float* b, int64_t ldb, float beta, float* c, int64_t ldc,
-                   bool upper_only, const int32_t* skip_if_nonneg, cudaStream_t stream,
-                   int tri = 0);
+
+// tgemm.cu: fp32-accurate GEMM on tcgen05 tensor cores (three tf32 passes on split operands).
+//   An operand x is first split into hi = tf32(x) and lo = x - hi (split_tf32), both row-major
+//   with stride ld (a multiple of 4 floats, 16-byte aligned base).
+//   C = alpha * A B + beta * C with A: m x k (k contiguous); B: n x k (k contiguous) or, when
+//   b_mn_major, k x n (n contiguous). upper_only / tri / skip as for the zero-structure flags.
+struct SplitF32 {
+  float* hi;
+  float* lo;
+  int64_t ld;
+};
+kronq_status split_tf32(const float* src, int64_t lds, int rows, int cols, SplitF32 dst,
+                        cudaStream_t stream);
+// two matrices in one launch
+kronq_status split_tf32_2(const float* src0, int64_t lds0, int rows0, int cols0, SplitF32 dst0,
+                          const float* src1, int64_t lds1, int rows1, int cols1, SplitF32 dst1,
+                          cudaStream_t stream);
+kronq_status tgemm(int m, int n, int k, float alpha, SplitF32 a, SplitF32 b, bool b_mn_major,
+                   float beta, float* c, int64_t ldc, bool upper_only, int tri,
+                   const int32_t* skip, cudaStream_t stream);
 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+inline int64_t pad4(int64_t x) { return (x + 3) & ~static_cast<int64_t>(3); }
+
+// Bump allocator over a workspace region (256-byte aligned pieces).
+struct Carve {
+  uint8_t* p;
+  float* floats(size_t n) {
+    float* r = reinterpret_cast<float*>(p);
+    p += align256(n * sizeof(float));
+    return r;
+  }
+  SplitF32 split(int rows, int cols) {
+    const int64_t ld = pad4(cols);
+    SplitF32 s;
+    s.hi = floats(static_cast<size_t>(rows) * ld);
+    s.lo = floats(static_cast<size_t>(rows) * ld);
+    s.ld = ld;
+    return s;
+  }
+};
+inline size_t split_bytes(int rows, int cols) {
+  return 2 * align256(static_cast<size_t>(rows) * pad4(cols) * sizeof(float));
+}
 
 }  // namespace kq

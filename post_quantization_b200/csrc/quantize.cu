@@ -6,10 +6,10 @@
 // (H_G cancels from the update, Proposition 1, so the solve never sees H_G). P is the GPTAQ
 // correction matrix, read as P = striu(D K^T) K. Its term uses the weights before any update,
 // so its total contribution to column j, sum_{p<j} W_:,p P_p,j, is known in advance: the solve
-// is GPTQ on W~ = W + W P, which this file forms up front with fp32 GEMMs.
+// is GPTQ on W~ = W + W P, which this file forms up front (fp32-accurate tensor-core GEMMs).
 //
-// Solve: 128-column blocks. Inside a block every output row is independent given K, so one
-// thread owns one row and walks the block's columns in order (quantize, error, update the
+// Solve: 128-column blocks. Inside a block every output row is independent given K; four
+// threads share a row and walk the block's columns in order (quantize, error, update the
 // remaining columns of the block). After the block the rest of every row is updated lazily with
 // one GEMM: W~[:, e:] -= Delta_blk K[blk, e:].
 #include <cmath>
@@ -22,8 +22,10 @@ namespace kq {
 namespace {
 
 constexpr int QB = 128;        // column block
-constexpr int QROWS = 128;     // rows (= threads) per CTA in the block solve
-constexpr int QSUB = 32;       // columns per register-resident sub-block
+constexpr int QROWS = 32;      // rows per CTA in the block solve
+constexpr int QT = 4;          // threads per row
+constexpr int QW = QB / QT;    // columns per thread
+constexpr int KS_LD = QT * (QW + 1);   // padded row of the K block in shared memory
 
 // Per-row grid from W (before the solve), all decisions in fp32:
 // scale = (hi - lo) / (2^b - 1) (1 if hi == lo), zero = rint(-lo / scale).
@@ -59,45 +61,38 @@ __global__ void striu_kernel(float* __restrict__ m, int d) {
     m[static_cast<int64_t>(i) * d + j] = 0.f;
 }
 
-// One 128-column block of the solve for QROWS rows (one thread per row).
-// The block is walked in four 32-column sub-blocks: the current sub-block lives in registers
-// (fully unrolled), the rest of the thread's row waits in shared memory and receives the
-// sub-block's errors in one pass after it.
+// One 128-column block of the solve for QROWS rows. Four threads share a row, each holding 32
+// of the block's columns in registers. At column p the thread that owns it quantizes it and
+// hands the scaled error to the other three (a shuffle within the group of four), and every
+// thread updates its own columns to the right of p. The K block sits in shared memory with
+// 33-float quarters so that the four threads of a row read from different banks.
 //   w_hat  d_out x d_in running weights (in: current values, out: dequantized for the block)
-//   delta  d_out x QB errors scaled by 1/K_pp (input of the lazy trailing update)
-__global__ void __launch_bounds__(QROWS) block_solve_kernel(
+//   delta  d_out x QB errors scaled by 1/K_pp, written split as tf32 hi + lo (the operand of
+//          the lazy trailing update on the tensor cores)
+__global__ void __launch_bounds__(QROWS * QT) block_solve_kernel(
     float* __restrict__ w_hat, const float* __restrict__ k, int d_out, int d_in, int b0, int bw,
     const float* __restrict__ scale, const float* __restrict__ zero, float maxq,
-    uint8_t* __restrict__ codes, float* __restrict__ delta) {
+    uint8_t* __restrict__ codes, float* __restrict__ delta_hi, float* __restrict__ delta_lo) {
   extern __shared__ float sm[];
-  float* Ks = sm;                              // QB x QB block of K (padding = identity)
-  float* St = Ks + QB * QB;                    // QROWS x (QB + 1): running row values
-  float* Dt = St + QROWS * (QB + 1);           // QROWS x (QB + 1): errors
-  float* Rd = Dt + QROWS * (QB + 1);           // QB reciprocals of K's diagonal
+  float* Ks = sm;                      // QB rows x KS_LD
+  float* Rd = sm + QB * KS_LD;         // QB reciprocals of K's diagonal
   const int tid = threadIdx.x;
-  const int row0 = blockIdx.x * QROWS;
-  const int rows = min(QROWS, d_out - row0);
+  const int lane = tid & 31;
+  const int q = tid % QT;              // column quarter of this thread
+  const int row = blockIdx.x * QROWS + tid / QT;
+  const bool active = row < d_out;
 
-  // K block (rows/cols beyond bw become identity so that padding never feeds back) and the
-  // rows' block of running weights, with 16-byte loads where the layout allows
-  const bool vec = (d_in % 4 == 0) && bw == QB &&
-                   ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(w_hat)) & 15u) == 0;
-  if (vec) {
+  // K block (rows/cols beyond bw become identity so that padding never feeds back)
+  const bool kvec = (d_in % 4 == 0) && bw == QB && (reinterpret_cast<uintptr_t>(k) & 15u) == 0;
+  if (kvec) {
     for (int e = tid; e < QB * QB / 4; e += blockDim.x) {
       const int i = e / (QB / 4), j4 = (e % (QB / 4)) * 4;
-      float4 v = *reinterpret_cast<const float4*>(k + static_cast<int64_t>(b0 + i) * d_in + b0 + j4);
-      if (j4 + 0 < i) v.x = 0.f;
-      if (j4 + 1 < i) v.y = 0.f;
-      if (j4 + 2 < i) v.z = 0.f;
-      if (j4 + 3 < i) v.w = 0.f;
-      *reinterpret_cast<float4*>(Ks + i * QB + j4) = v;
-    }
-    for (int e = tid; e < QROWS * QB / 4; e += blockDim.x) {
-      const int r = e / (QB / 4), c4 = (e % (QB / 4)) * 4;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (r < rows) v = *reinterpret_cast<const float4*>(w_hat + static_cast<int64_t>(row0 + r) * d_in + b0 + c4);
-      float* dst = St + r * (QB + 1) + c4;
-      dst[0] = v.x; dst[1] = v.y; dst[2] = v.z; dst[3] = v.w;
+      const float4 v = *reinterpret_cast<const float4*>(k + static_cast<int64_t>(b0 + i) * d_in + b0 + j4);
+      float* dst = Ks + i * KS_LD + (j4 >> 5) * (QW + 1) + (j4 & 31);
+      dst[0] = (j4 + 0 >= i) ? v.x : 0.f;
+      dst[1] = (j4 + 1 >= i) ? v.y : 0.f;
+      dst[2] = (j4 + 2 >= i) ? v.z : 0.f;
+      dst[3] = (j4 + 3 >= i) ? v.w : 0.f;
     }
   } else {
     for (int e = tid; e < QB * QB; e += blockDim.x) {
@@ -107,79 +102,75 @@ __global__ void __launch_bounds__(QROWS) block_solve_kernel(
         v = (j >= i) ? k[static_cast<int64_t>(b0 + i) * d_in + b0 + j] : 0.f;
       else
         v = (i == j) ? 1.f : 0.f;
-      Ks[e] = v;
-    }
-    for (int e = tid; e < QROWS * QB; e += blockDim.x) {
-      const int r = e / QB, c = e % QB;
-      float v = 0.f;
-      if (r < rows && c < bw) v = w_hat[static_cast<int64_t>(row0 + r) * d_in + b0 + c];
-      St[r * (QB + 1) + c] = v;
+      Ks[i * KS_LD + (j >> 5) * (QW + 1) + (j & 31)] = v;
     }
   }
   __syncthreads();
-  if (tid < QB) Rd[tid] = 1.f / Ks[tid * QB + tid];
+  if (tid < QB) Rd[tid] = 1.f / Ks[tid * KS_LD + (tid >> 5) * (QW + 1) + (tid & 31)];
   __syncthreads();
 
-  const int row = row0 + tid;
-  const bool active = tid < rows;
+  // this thread's 32 columns of its row
+  float w[QW];
+  float* wrow = w_hat + static_cast<int64_t>(row) * d_in + b0 + QW * q;
+  const bool wvec = active && bw == QB && ((reinterpret_cast<uintptr_t>(wrow) & 15u) == 0);
+  if (wvec) {
+#pragma unroll
+    for (int j = 0; j < QW; j += 4) {
+      const float4 v = *reinterpret_cast<const float4*>(wrow + j);
+      w[j] = v.x; w[j + 1] = v.y; w[j + 2] = v.z; w[j + 3] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < QW; ++j) w[j] = (active && QW * q + j < bw) ? wrow[j] : 0.f;
+  }
   const float sc = active ? scale[row] : 1.f;
   const float zr = active ? zero[row] : 0.f;
-  float* my = St + tid * (QB + 1);
-  float* myd = Dt + tid * (QB + 1);
-  uint32_t packed[QB / 4];
+  float err[QW];
+  uint32_t packed[QW / 4];
+#pragma unroll
+  for (int j = 0; j < QW / 4; ++j) packed[j] = 0u;
 
-#pragma unroll 1
-  for (int sb = 0; sb < QB; sb += QSUB) {
-    float w[QSUB], err[QSUB];
 #pragma unroll
-    for (int c = 0; c < QSUB; ++c) w[c] = my[sb + c];
-#pragma unroll
-    for (int p = 0; p < QSUB; ++p) {
-      const float t = __fdiv_rn(w[p], sc);
+  for (int p = 0; p < QB; ++p) {
+    const int qo = p / QW, lp = p % QW;   // owner quarter and its local column (compile time)
+    float e = 0.f;
+    if (q == qo) {
+      const float t = __fdiv_rn(w[lp], sc);
       float code = __fadd_rn(rintf(t), zr);
       code = fminf(fmaxf(code, 0.f), maxq);
       const float dq = __fmul_rn(sc, __fsub_rn(code, zr));
-      const float* kr = Ks + (sb + p) * QB + sb;
-      err[p] = __fsub_rn(w[p], dq) * Rd[sb + p];
-#pragma unroll
-      for (int j = p + 1; j < QSUB; ++j) w[j] = fmaf(-err[p], kr[j], w[j]);
-      w[p] = dq;
-      const int cc = sb + p;
-      if ((p & 3) == 0) packed[cc >> 2] = 0u;
-      packed[cc >> 2] |= (static_cast<uint32_t>(code) & 0xFFu) << (8 * (p & 3));
+      e = __fsub_rn(w[lp], dq) * Rd[p];
+      w[lp] = dq;
+      err[lp] = e;
+      packed[lp / 4] |= (static_cast<uint32_t>(code) & 0xFFu) << (8 * (lp % 4));
     }
+    e = __shfl_sync(0xffffffffu, e, (lane & ~(QT - 1)) | qo);
+    if (q >= qo) {
+      const float* kr = Ks + p * KS_LD + q * (QW + 1);
 #pragma unroll
-    for (int c = 0; c < QSUB; ++c) {
-      my[sb + c] = w[c];
-      myd[sb + c] = err[c];
-    }
-    // the sub-block's errors reach the rest of the block
-#pragma unroll 2
-    for (int j = sb + QSUB; j < QB; ++j) {
-      float acc = my[j];
-#pragma unroll
-      for (int p = 0; p < QSUB; ++p) acc = fmaf(-err[p], Ks[(sb + p) * QB + j], acc);
-      my[j] = acc;
+      for (int j = 0; j < QW; ++j)
+        if (QW * q + j > p) w[j] = fmaf(-e, kr[j], w[j]);
     }
   }
-  __syncthreads();
-  for (int e = tid; e < QROWS * QB; e += blockDim.x) {
-    const int r = e / QB, c = e % QB;
-    if (r < rows) {
-      delta[static_cast<int64_t>(row0 + r) * QB + c] = (c < bw) ? Dt[r * (QB + 1) + c] : 0.f;
-      if (c < bw) w_hat[static_cast<int64_t>(row0 + r) * d_in + b0 + c] = St[r * (QB + 1) + c];
-    }
-  }
+
   if (active) {
-    uint8_t* cr = codes + static_cast<int64_t>(row) * d_in + b0;
-    if (bw == QB && (reinterpret_cast<uintptr_t>(cr) & 15u) == 0) {
 #pragma unroll
-      for (int c = 0; c < QB / 16; ++c)
-        reinterpret_cast<uint4*>(cr)[c] =
-            make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+    for (int j = 0; j < QW; ++j) {
+      const int c = QW * q + j;
+      if (c < bw) wrow[j] = w[j];
+      const float dv = c < bw ? err[j] : 0.f;
+      uint32_t h;
+      asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(h) : "f"(dv));
+      delta_hi[static_cast<int64_t>(row) * QB + c] = __uint_as_float(h);
+      delta_lo[static_cast<int64_t>(row) * QB + c] = dv - __uint_as_float(h);
+    }
+    uint8_t* cr = codes + static_cast<int64_t>(row) * d_in + b0 + QW * q;
+    if (bw == QB && (reinterpret_cast<uintptr_t>(cr) & 15u) == 0) {
+      reinterpret_cast<uint4*>(cr)[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      reinterpret_cast<uint4*>(cr)[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
     } else {
-      for (int c = 0; c < bw; ++c)
-        cr[c] = static_cast<uint8_t>((packed[c >> 2] >> (8 * (c & 3))) & 0xFFu);
+      for (int j = 0; j < QW; ++j)
+        if (QW * q + j < bw) cr[j] = static_cast<uint8_t>((packed[j >> 2] >> (8 * (j & 3))) & 0xFFu);
     }
   }
 }
@@ -188,10 +179,15 @@ __global__ void __launch_bounds__(QROWS) block_solve_kernel(
 
 size_t quantize_workspace_bytes(int d_out, int d_in, int block, bool with_dxx) {
   (void)block;
-  size_t b = align256(sizeof(float) * static_cast<size_t>(d_out) * QB);   // delta
+  size_t b = split_bytes(d_in, d_in);        // K, split once per layer
+  b += split_bytes(d_out, QB);               // block errors
   if (with_dxx) {
-    b += align256(sizeof(float) * static_cast<size_t>(d_in) * d_in);      // M = striu(D K^T)
-    b += align256(sizeof(float) * static_cast<size_t>(d_out) * d_in);     // W striu(M)
+    const size_t r1 = split_bytes(d_in, d_in) > split_bytes(d_out, d_in) ? split_bytes(d_in, d_in)
+                                                                         : split_bytes(d_out, d_in);
+    b += r1;                                                           // D / W / W striu(M) splits
+    b += align256(sizeof(float) * static_cast<size_t>(d_in) * d_in);   // M = striu(D K^T)
+    b += split_bytes(d_in, d_in);                                      // M split
+    b += align256(sizeof(float) * static_cast<size_t>(d_out) * d_in); // W striu(M)
   }
   return b;
 }
@@ -201,37 +197,59 @@ kronq_status run_quantize(const float* w, const float* k, const float* dxx, int 
                           float* w_hat, void* ws, cudaStream_t stream) {
   (void)block;
   const float maxq = static_cast<float>((1 << bits) - 1);
-  uint8_t* p = static_cast<uint8_t*>(ws);
-  float* delta = reinterpret_cast<float*>(p);
-  p += align256(sizeof(float) * static_cast<size_t>(d_out) * QB);
+  Carve cv{static_cast<uint8_t*>(ws)};
+  SplitF32 ks = cv.split(d_in, d_in);
+  SplitF32 ds = cv.split(d_out, QB);
 
   // grid from W before the solve
   grid_kernel<<<(d_out + 7) / 8, 256, 0, stream>>>(w, d_out, d_in, maxq, scale, zero);
   KQ_TRY(check_launch("grid_kernel"));
+  KQ_TRY(split_tf32(k, d_in, d_in, d_in, ks, stream));
 
   KQ_CUDA_TRY(cudaMemcpyAsync(w_hat, w, sizeof(float) * static_cast<size_t>(d_out) * d_in,
                               cudaMemcpyDeviceToDevice, stream));
   if (dxx) {
-    float* mm = reinterpret_cast<float*>(p);
-    p += align256(sizeof(float) * static_cast<size_t>(d_in) * d_in);
-    float* t1 = reinterpret_cast<float*>(p);
+    uint8_t* r1_base = cv.p;
+    const size_t r1 = split_bytes(d_in, d_in) > split_bytes(d_out, d_in) ? split_bytes(d_in, d_in)
+                                                                         : split_bytes(d_out, d_in);
+    cv.p += r1;
+    float* mm = cv.floats(static_cast<size_t>(d_in) * d_in);
+    SplitF32 ms = cv.split(d_in, d_in);
+    float* t1 = cv.floats(static_cast<size_t>(d_out) * d_in);
     // M = D K^T, striu(M)
-    KQ_TRY(sgemm(false, true, d_in, d_in, d_in, 1.f, dxx, d_in, k, d_in, 0.f, mm, d_in, false,
-                 nullptr, stream, GEMM_B_LOWER));
+    {
+      Carve r{r1_base};
+      SplitF32 dsp = r.split(d_in, d_in);
+      KQ_TRY(split_tf32(dxx, d_in, d_in, d_in, dsp, stream));
+      KQ_TRY(tgemm(d_in, d_in, d_in, 1.f, dsp, ks, false, 0.f, mm, d_in, false, GEMM_B_LOWER,
+                   nullptr, stream));
+    }
     {
       dim3 g((d_in + 255) / 256, d_in);
       striu_kernel<<<g, 256, 0, stream>>>(mm, d_in);
       KQ_TRY(check_launch("striu_kernel"));
     }
-    // W~ = W + (W striu(M)) K
-    KQ_TRY(sgemm(false, false, d_out, d_in, d_in, 1.f, w, d_in, mm, d_in, 0.f, t1, d_in, false,
-                 nullptr, stream, GEMM_B_UPPER));
-    KQ_TRY(sgemm(false, false, d_out, d_in, d_in, 1.f, t1, d_in, k, d_in, 1.f, w_hat, d_in, false,
-                 nullptr, stream, GEMM_B_UPPER));
+    KQ_TRY(split_tf32(mm, d_in, d_in, d_in, ms, stream));
+    // T1 = W striu(M)
+    {
+      Carve r{r1_base};
+      SplitF32 wsp = r.split(d_out, d_in);
+      KQ_TRY(split_tf32(w, d_in, d_out, d_in, wsp, stream));
+      KQ_TRY(tgemm(d_out, d_in, d_in, 1.f, wsp, ms, true, 0.f, t1, d_in, false, GEMM_B_UPPER,
+                   nullptr, stream));
+    }
+    // W~ = W + T1 K
+    {
+      Carve r{r1_base};
+      SplitF32 tsp = r.split(d_out, d_in);
+      KQ_TRY(split_tf32(t1, d_in, d_out, d_in, tsp, stream));
+      KQ_TRY(tgemm(d_out, d_in, d_in, 1.f, tsp, ks, true, 1.f, w_hat, d_in, false, GEMM_B_UPPER,
+                   nullptr, stream));
+    }
   }
 
   static bool attr = false;
-  const size_t smem = sizeof(float) * (QB * QB + 2 * QROWS * (QB + 1) + QB);
+  const size_t smem = sizeof(float) * (QB * KS_LD + QB);
   if (!attr) {
     KQ_CUDA_TRY(cudaFuncSetAttribute(block_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)smem));
@@ -239,14 +257,15 @@ kronq_status run_quantize(const float* w, const float* k, const float* dxx, int 
   }
   for (int b0 = 0; b0 < d_in; b0 += QB) {
     const int bw = d_in - b0 < QB ? d_in - b0 : QB;
-    block_solve_kernel<<<(d_out + QROWS - 1) / QROWS, QROWS, smem, stream>>>(
-        w_hat, k, d_out, d_in, b0, bw, scale, zero, maxq, codes, delta);
+    block_solve_kernel<<<(d_out + QROWS - 1) / QROWS, QROWS * QT, smem, stream>>>(
+        w_hat, k, d_out, d_in, b0, bw, scale, zero, maxq, codes, ds.hi, ds.lo);
     KQ_TRY(check_launch("block_solve_kernel"));
     const int e = b0 + bw;
     if (e < d_in) {
       // W~[:, e:] -= Delta K[b0:e, e:]
-      KQ_TRY(sgemm(false, false, d_out, d_in - e, bw, -1.f, delta, QB,
-                   k + static_cast<int64_t>(b0) * d_in + e, d_in, 1.f, w_hat + e, d_in, false,
+      SplitF32 kb{ks.hi + static_cast<int64_t>(b0) * ks.ld + e,
+                  ks.lo + static_cast<int64_t>(b0) * ks.ld + e, ks.ld};
+      KQ_TRY(tgemm(d_out, d_in - e, bw, -1.f, ds, kb, true, 1.f, w_hat + e, d_in, false, 0,
                    nullptr, stream));
     }
   }

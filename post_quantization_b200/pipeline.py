@@ -3,7 +3,8 @@
 A sublayer goes through: Kronecker-factor sums -> BiIP -> damped inverse factor -> column
 solve; a block or stack adds the trace-product scores and the bit allocation in between. Every
 arithmetic step is one of the five library calls; this module only allocates device buffers
-with torch and sequences the calls on one stream.
+with torch and sequences the calls, on the caller's stream or, for the independent sublayers of
+a block, on one stream per sublayer (SublayerStreams).
 """
 from __future__ import annotations
 
@@ -100,3 +101,42 @@ def quantize_sublayer(w, hx_sum, hg_sum, dxx_sum, inv_n, sign_in, sign_out, bits
     cholinv(r, damp_rel, ws, stream)
     quantize(r, bits, ws, stream)
     return r
+
+
+class SublayerStreams:
+    """Runs the per-sublayer steps of a block on one CUDA stream per sublayer.
+
+    The sublayers of a block are independent once their statistics exist, and each of their
+    kernel chains (BiIP passes, the recursive inverse factor, the column solve) leaves most of
+    the GPU idle on its own, so they run side by side. Each stream has its own workspace. Every
+    method makes its streams wait for the caller's stream first and makes the caller's stream
+    wait for all of them before it returns.
+    """
+
+    def __init__(self, count: int, device):
+        self.streams = [torch.cuda.Stream(device=device) for _ in range(count)]
+        self.ws = [Workspace(device) for _ in range(count)]
+
+    def _fan_out(self, jobs, fn):
+        main = torch.cuda.current_stream()
+        out = []
+        for i, job in enumerate(jobs):
+            s = self.streams[i % len(self.streams)]
+            s.wait_stream(main)
+            with torch.cuda.stream(s):
+                out.append(fn(job, self.ws[i % len(self.ws)]))
+        for s in self.streams:
+            main.wait_stream(s)
+        return out
+
+    def biip(self, jobs):
+        """jobs: (w, hx_sum, hg_sum, dxx_sum, inv_n, sign_in, sign_out, flags) per sublayer."""
+        return self._fan_out(jobs, lambda j, ws: biip(*j, ws=ws))
+
+    def solve(self, results, bits, damp_rel=0.01):
+        def one(job, ws):
+            r, b = job
+            cholinv(r, damp_rel, ws)
+            quantize(r, b, ws)
+            return r
+        return self._fan_out(list(zip(results, bits)), one)
