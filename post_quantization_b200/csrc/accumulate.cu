@@ -53,23 +53,37 @@ struct AccParams {
 };
 
 // Map a computed-tile index to (tm, tn). Symmetric: row tm holds tiles tn >= tn_min(tm).
+// Tiles are visited in groups of GROUP tile rows, column by column inside a group, so that the
+// ~148 tiles in flight at any time cover a compact block of the output: they read GROUP row
+// strips and ~148/GROUP column strips of the token chunk instead of every column, which keeps
+// the chunk's DRAM re-reads down when the output has many more tiles than the GPU has SMs.
+constexpr int GROUP = 8;
+
+__device__ __forceinline__ int tn_min_of(const AccParams& p, int tm) {
+  return p.symmetric ? (tm * acc::BM) / acc::BN : 0;
+}
+
 __device__ __forceinline__ void tile_coords(const AccParams& p, int t, int& tm, int& tn) {
-  if (!p.symmetric) {
-    tm = t / p.tiles_n;
-    tn = t % p.tiles_n;
-    return;
-  }
-  int r = 0;
+  int g0 = 0;
   for (;;) {
-    const int tn_min = (r * acc::BM) / acc::BN;
-    const int cnt = p.tiles_n - tn_min;
-    if (t < cnt) {
-      tm = r;
-      tn = tn_min + t;
+    const int g1 = min(g0 + GROUP, p.tiles_m);
+    int cnt = 0;
+    for (int r = g0; r < g1; ++r) cnt += p.tiles_n - tn_min_of(p, r);
+    if (t < cnt) break;
+    t -= cnt;
+    g0 = g1;
+  }
+  const int g1 = min(g0 + GROUP, p.tiles_m);
+  for (int c = tn_min_of(p, g0);; ++c) {
+    // rows of the group whose first tile is at or left of column c (tn_min grows with the row)
+    int rows = 0;
+    while (g0 + rows < g1 && tn_min_of(p, g0 + rows) <= c) ++rows;
+    if (t < rows) {
+      tm = g0 + t;
+      tn = c;
       return;
     }
-    t -= cnt;
-    ++r;
+    t -= rows;
   }
 }
 

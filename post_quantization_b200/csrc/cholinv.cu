@@ -13,8 +13,8 @@
 //   K11 = chol_inv(A11)
 //   K12 = -K11 R12 K22              ([[R11, R12], [0, R22]]^-1)
 // Leaves of at most 128 columns are factored and inverted in shared memory by one CTA. The four
-// products per level are large square GEMMs on the tensor cores (three tf32 passes on split
-// operands, fp32-accurate) that skip the zero triangles of K.
+// products per level are large square GEMMs on the tensor cores (operands split into three bf16
+// pieces, fp32-accurate) that skip the zero triangles of K.
 #include <cmath>
 
 #include "common.cuh"
@@ -208,30 +208,30 @@ kronq_status chol_inv_rec(const Ctx& c, float* a, int n, int j0) {
   {
     // R12 = A12 K22^T, written over A12 (the GEMM reads split copies)
     Carve cv{c.splits};
-    SplitF32 s12 = cv.split(n1, n2), s22 = cv.split(n2, n2);
-    KQ_TRY(split_tf32_2(a12, ld, n1, n2, s12, a22, ld, n2, n2, s22, st));
+    Split3 s12 = cv.split(n1, n2), s22 = cv.split(n2, n2);
+    KQ_TRY(split_bf16x3_2(a12, ld, n1, n2, s12, a22, ld, n2, n2, s22, st));
     KQ_TRY(tgemm(n1, n2, n2, 1.f, s12, s22, false, 0.f, a12, ld, false, GEMM_B_LOWER, c.info, st));
   }
   {
     // A11 -= R12 R12^T (upper triangle)
     Carve cv{c.splits};
-    SplitF32 r12 = cv.split(n1, n2);
-    KQ_TRY(split_tf32(a12, ld, n1, n2, r12, st));
+    Split3 r12 = cv.split(n1, n2);
+    KQ_TRY(split_bf16x3(a12, ld, n1, n2, r12, st));
     KQ_TRY(tgemm(n1, n1, n2, -1.f, r12, r12, false, 1.f, a11, ld, true, 0, c.info, st));
   }
   KQ_TRY(chol_inv_rec(c, a11, n1, j0));                                    // K11
   {
     // T = R12 K22
     Carve cv{c.splits};
-    SplitF32 r12 = cv.split(n1, n2), s22 = cv.split(n2, n2);
-    KQ_TRY(split_tf32_2(a12, ld, n1, n2, r12, a22, ld, n2, n2, s22, st));
+    Split3 r12 = cv.split(n1, n2), s22 = cv.split(n2, n2);
+    KQ_TRY(split_bf16x3_2(a12, ld, n1, n2, r12, a22, ld, n2, n2, s22, st));
     KQ_TRY(tgemm(n1, n2, n2, 1.f, r12, s22, true, 0.f, c.t, n2, false, GEMM_B_UPPER, c.info, st));
   }
   {
     // K12 = -K11 T
     Carve cv{c.splits};
-    SplitF32 s11 = cv.split(n1, n1), tt = cv.split(n1, n2);
-    KQ_TRY(split_tf32_2(a11, ld, n1, n1, s11, c.t, n2, n1, n2, tt, st));
+    Split3 s11 = cv.split(n1, n1), tt = cv.split(n1, n2);
+    KQ_TRY(split_bf16x3_2(a11, ld, n1, n1, s11, c.t, n2, n1, n2, tt, st));
     KQ_TRY(tgemm(n1, n2, n1, -1.f, s11, tt, true, 0.f, a12, ld, false, GEMM_A_UPPER, c.info, st));
   }
   return KRONQ_OK;

@@ -55,28 +55,33 @@ kronq_status run_quantize(const float* w, const float* k, const float* dxx, int 
 //   GEMM_B_LOWER  op(B)[k][n] = 0 for k < n
 enum { GEMM_A_UPPER = 1, GEMM_B_UPPER = 2, GEMM_B_LOWER = 4 };
 
-// tgemm.cu: fp32-accurate GEMM on tcgen05 tensor cores (three tf32 passes on split operands).
-//   An operand x is first split into hi = tf32(x) and lo = x - hi (split_tf32), both row-major
-//   with stride ld (a multiple of 4 floats, 16-byte aligned base).
+// tgemm.cu: fp32-accurate GEMM on tcgen05 tensor cores (bf16 x3 split, six products).
+//   An fp32 operand x is first split (split_bf16x3) into three bf16 pieces x0 + x1 + x2 that
+//   carry its 24 significant bits, each stored row-major with stride ld (a multiple of 8
+//   elements, 16-byte aligned base).
 //   C = alpha * A B + beta * C with A: m x k (k contiguous); B: n x k (k contiguous) or, when
 //   b_mn_major, k x n (n contiguous). upper_only / tri / skip as for the zero-structure flags.
-struct SplitF32 {
-  float* hi;
-  float* lo;
+struct Split3 {
+  uint16_t* part[3];
   int64_t ld;
 };
-kronq_status split_tf32(const float* src, int64_t lds, int rows, int cols, SplitF32 dst,
-                        cudaStream_t stream);
-// two matrices in one launch
-kronq_status split_tf32_2(const float* src0, int64_t lds0, int rows0, int cols0, SplitF32 dst0,
-                          const float* src1, int64_t lds1, int rows1, int cols1, SplitF32 dst1,
+kronq_status split_bf16x3(const float* src, int64_t lds, int rows, int cols, Split3 dst,
                           cudaStream_t stream);
-kronq_status tgemm(int m, int n, int k, float alpha, SplitF32 a, SplitF32 b, bool b_mn_major,
+// two matrices in one launch
+kronq_status split_bf16x3_2(const float* src0, int64_t lds0, int rows0, int cols0, Split3 dst0,
+                            const float* src1, int64_t lds1, int rows1, int cols1, Split3 dst1,
+                            cudaStream_t stream);
+kronq_status tgemm(int m, int n, int k, float alpha, Split3 a, Split3 b, bool b_mn_major,
                    float beta, float* c, int64_t ldc, bool upper_only, int tri,
                    const int32_t* skip, cudaStream_t stream);
+// the sub-matrix of a split operand starting at (row, col)
+inline Split3 offset(Split3 s, int64_t row, int64_t col) {
+  for (int i = 0; i < 3; ++i) s.part[i] += row * s.ld + col;
+  return s;
+}
 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
-inline int64_t pad4(int64_t x) { return (x + 3) & ~static_cast<int64_t>(3); }
+inline int64_t pad8(int64_t x) { return (x + 7) & ~static_cast<int64_t>(7); }
 
 // Bump allocator over a workspace region (256-byte aligned pieces).
 struct Carve {
@@ -86,17 +91,18 @@ struct Carve {
     p += align256(n * sizeof(float));
     return r;
   }
-  SplitF32 split(int rows, int cols) {
-    const int64_t ld = pad4(cols);
-    SplitF32 s;
-    s.hi = floats(static_cast<size_t>(rows) * ld);
-    s.lo = floats(static_cast<size_t>(rows) * ld);
-    s.ld = ld;
+  Split3 split(int rows, int cols) {
+    Split3 s;
+    s.ld = pad8(cols);
+    for (int i = 0; i < 3; ++i) {
+      s.part[i] = reinterpret_cast<uint16_t*>(p);
+      p += align256(static_cast<size_t>(rows) * s.ld * sizeof(uint16_t));
+    }
     return s;
   }
 };
 inline size_t split_bytes(int rows, int cols) {
-  return 2 * align256(static_cast<size_t>(rows) * pad4(cols) * sizeof(float));
+  return 3 * align256(static_cast<size_t>(rows) * pad8(cols) * sizeof(uint16_t));
 }
 
 }  // namespace kq

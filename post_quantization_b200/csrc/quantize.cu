@@ -12,6 +12,8 @@
 // threads share a row and walk the block's columns in order (quantize, error, update the
 // remaining columns of the block). After the block the rest of every row is updated lazily with
 // one GEMM: W~[:, e:] -= Delta_blk K[blk, e:].
+#include <cuda_bf16.h>
+
 #include <cmath>
 
 #include "common.cuh"
@@ -67,12 +69,13 @@ __global__ void striu_kernel(float* __restrict__ m, int d) {
 // thread updates its own columns to the right of p. The K block sits in shared memory with
 // 33-float quarters so that the four threads of a row read from different banks.
 //   w_hat  d_out x d_in running weights (in: current values, out: dequantized for the block)
-//   delta  d_out x QB errors scaled by 1/K_pp, written split as tf32 hi + lo (the operand of
+//   delta  d_out x QB errors scaled by 1/K_pp, written as three bf16 pieces (the operand of
 //          the lazy trailing update on the tensor cores)
 __global__ void __launch_bounds__(QROWS * QT) block_solve_kernel(
     float* __restrict__ w_hat, const float* __restrict__ k, int d_out, int d_in, int b0, int bw,
     const float* __restrict__ scale, const float* __restrict__ zero, float maxq,
-    uint8_t* __restrict__ codes, float* __restrict__ delta_hi, float* __restrict__ delta_lo) {
+    uint8_t* __restrict__ codes, uint16_t* __restrict__ delta0, uint16_t* __restrict__ delta1,
+    uint16_t* __restrict__ delta2) {
   extern __shared__ float sm[];
   float* Ks = sm;                      // QB rows x KS_LD
   float* Rd = sm + QB * KS_LD;         // QB reciprocals of K's diagonal
@@ -158,11 +161,16 @@ __global__ void __launch_bounds__(QROWS * QT) block_solve_kernel(
     for (int j = 0; j < QW; ++j) {
       const int c = QW * q + j;
       if (c < bw) wrow[j] = w[j];
+      // the error, split into three bf16 pieces for the tensor-core trailing update
       const float dv = c < bw ? err[j] : 0.f;
-      uint32_t h;
-      asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(h) : "f"(dv));
-      delta_hi[static_cast<int64_t>(row) * QB + c] = __uint_as_float(h);
-      delta_lo[static_cast<int64_t>(row) * QB + c] = dv - __uint_as_float(h);
+      const __nv_bfloat16 p0 = __float2bfloat16_rn(dv);
+      const float r1 = dv - __bfloat162float(p0);
+      const __nv_bfloat16 p1 = __float2bfloat16_rn(r1);
+      const __nv_bfloat16 p2 = __float2bfloat16_rn(r1 - __bfloat162float(p1));
+      const int64_t o = static_cast<int64_t>(row) * QB + c;
+      delta0[o] = __bfloat16_as_ushort(p0);
+      delta1[o] = __bfloat16_as_ushort(p1);
+      delta2[o] = __bfloat16_as_ushort(p2);
     }
     uint8_t* cr = codes + static_cast<int64_t>(row) * d_in + b0 + QW * q;
     if (bw == QB && (reinterpret_cast<uintptr_t>(cr) & 15u) == 0) {
@@ -198,13 +206,13 @@ kronq_status run_quantize(const float* w, const float* k, const float* dxx, int 
   (void)block;
   const float maxq = static_cast<float>((1 << bits) - 1);
   Carve cv{static_cast<uint8_t*>(ws)};
-  SplitF32 ks = cv.split(d_in, d_in);
-  SplitF32 ds = cv.split(d_out, QB);
+  Split3 ks = cv.split(d_in, d_in);
+  Split3 ds = cv.split(d_out, QB);
 
   // grid from W before the solve
   grid_kernel<<<(d_out + 7) / 8, 256, 0, stream>>>(w, d_out, d_in, maxq, scale, zero);
   KQ_TRY(check_launch("grid_kernel"));
-  KQ_TRY(split_tf32(k, d_in, d_in, d_in, ks, stream));
+  KQ_TRY(split_bf16x3(k, d_in, d_in, d_in, ks, stream));
 
   KQ_CUDA_TRY(cudaMemcpyAsync(w_hat, w, sizeof(float) * static_cast<size_t>(d_out) * d_in,
                               cudaMemcpyDeviceToDevice, stream));
@@ -214,13 +222,13 @@ kronq_status run_quantize(const float* w, const float* k, const float* dxx, int 
                                                                          : split_bytes(d_out, d_in);
     cv.p += r1;
     float* mm = cv.floats(static_cast<size_t>(d_in) * d_in);
-    SplitF32 ms = cv.split(d_in, d_in);
+    Split3 ms = cv.split(d_in, d_in);
     float* t1 = cv.floats(static_cast<size_t>(d_out) * d_in);
     // M = D K^T, striu(M)
     {
       Carve r{r1_base};
-      SplitF32 dsp = r.split(d_in, d_in);
-      KQ_TRY(split_tf32(dxx, d_in, d_in, d_in, dsp, stream));
+      Split3 dsp = r.split(d_in, d_in);
+      KQ_TRY(split_bf16x3(dxx, d_in, d_in, d_in, dsp, stream));
       KQ_TRY(tgemm(d_in, d_in, d_in, 1.f, dsp, ks, false, 0.f, mm, d_in, false, GEMM_B_LOWER,
                    nullptr, stream));
     }
@@ -229,20 +237,20 @@ kronq_status run_quantize(const float* w, const float* k, const float* dxx, int 
       striu_kernel<<<g, 256, 0, stream>>>(mm, d_in);
       KQ_TRY(check_launch("striu_kernel"));
     }
-    KQ_TRY(split_tf32(mm, d_in, d_in, d_in, ms, stream));
+    KQ_TRY(split_bf16x3(mm, d_in, d_in, d_in, ms, stream));
     // T1 = W striu(M)
     {
       Carve r{r1_base};
-      SplitF32 wsp = r.split(d_out, d_in);
-      KQ_TRY(split_tf32(w, d_in, d_out, d_in, wsp, stream));
+      Split3 wsp = r.split(d_out, d_in);
+      KQ_TRY(split_bf16x3(w, d_in, d_out, d_in, wsp, stream));
       KQ_TRY(tgemm(d_out, d_in, d_in, 1.f, wsp, ms, true, 0.f, t1, d_in, false, GEMM_B_UPPER,
                    nullptr, stream));
     }
     // W~ = W + T1 K
     {
       Carve r{r1_base};
-      SplitF32 tsp = r.split(d_out, d_in);
-      KQ_TRY(split_tf32(t1, d_in, d_out, d_in, tsp, stream));
+      Split3 tsp = r.split(d_out, d_in);
+      KQ_TRY(split_bf16x3(t1, d_in, d_out, d_in, tsp, stream));
       KQ_TRY(tgemm(d_out, d_in, d_in, 1.f, tsp, ks, true, 1.f, w_hat, d_in, false, GEMM_B_UPPER,
                    nullptr, stream));
     }
@@ -258,13 +266,12 @@ kronq_status run_quantize(const float* w, const float* k, const float* dxx, int 
   for (int b0 = 0; b0 < d_in; b0 += QB) {
     const int bw = d_in - b0 < QB ? d_in - b0 : QB;
     block_solve_kernel<<<(d_out + QROWS - 1) / QROWS, QROWS * QT, smem, stream>>>(
-        w_hat, k, d_out, d_in, b0, bw, scale, zero, maxq, codes, ds.hi, ds.lo);
+        w_hat, k, d_out, d_in, b0, bw, scale, zero, maxq, codes, ds.part[0], ds.part[1], ds.part[2]);
     KQ_TRY(check_launch("block_solve_kernel"));
     const int e = b0 + bw;
     if (e < d_in) {
       // W~[:, e:] -= Delta K[b0:e, e:]
-      SplitF32 kb{ks.hi + static_cast<int64_t>(b0) * ks.ld + e,
-                  ks.lo + static_cast<int64_t>(b0) * ks.ld + e, ks.ld};
+      const Split3 kb = offset(ks, b0, e);
       KQ_TRY(tgemm(d_out, d_in - e, bw, -1.f, ds, kb, true, 1.f, w_hat + e, d_in, false, 0,
                    nullptr, stream));
     }

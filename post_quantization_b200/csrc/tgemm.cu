@@ -1,28 +1,34 @@
-// fp32-accurate GEMM on 5th-generation tensor cores: three tf32 passes.
+// fp32-accurate GEMM on 5th-generation tensor cores: bf16 x3 split, six products.
 //
 //   C = alpha * A B + beta * C,   A: M x K (row-major, K contiguous), B: K x N given either as
 //   an N x K row-major array (K-major) or a K x N row-major array (MN-major).
 //
-// Each fp32 operand x is split beforehand into hi = tf32(x) (round to nearest) and
-// lo = x - hi (exact in fp32), and the product is hi*hi + hi*lo + lo*hi with fp32 accumulation
-// in TMEM; the dropped lo*lo term and the tf32 rounding of lo are ~2^-22 relative, so the result
-// is as accurate as an fp32 GEMM. This is what the damped inverse factor and the trailing update
-// of the column solve need: a single tf32 pass would perturb the error feedback enough to flip
-// quantized codes.
+// Each fp32 operand x is split beforehand into three bf16 pieces x = x0 + x1 + x2 (each the
+// bf16 rounding of what the previous pieces left), which carry its 24 significant bits. The
+// product keeps every term down to 2^-16 relative, a0 b0 + a0 b1 + a1 b0 + a0 b2 + a1 b1 + a2 b0;
+// bf16 x bf16 products are exact, the dropped terms are ~2^-24 relative, and the sums are the
+// tensor core's fp32 accumulation (measured ~1e-5 relative at K = 1024, close to a CUDA-core
+// fp32 GEMM). This is what the damped inverse factor and the trailing update of the column
+// solve need: one bf16 or tf32 pass perturbs the error feedback enough to flip quantized codes.
+// Six bf16 MMAs take the time of three tf32 ones and move 25% fewer operand bytes.
 //
-// Kernel: persistent, one CTA per SM. Warp 0 drives TMA (128-byte swizzle, 3-stage ring of
-// A_hi, A_lo, B_hi, B_lo tiles, no multicast), warp 1 owns TMEM and issues
-// tcgen05.mma.cta_group::1.kind::tf32 (M = N = 128, K = 8), warps 2..5 run the epilogue
-// (alpha * acc + beta * C) while the next tile accumulates in the other TMEM buffer.
+// Kernel: persistent, one CTA per SM. Warp 0 drives TMA (128-byte swizzle, 2-stage ring of the
+// six operand pieces, no multicast), warp 1 owns TMEM and issues
+// tcgen05.mma.cta_group::1.kind::f16 (M = N = 128, K = 16, bf16 in, fp32 accumulate), warps
+// 2..5 run the epilogue (alpha * acc + beta * C, coalesced through a per-warp transpose tile)
+// while the next tile accumulates in the other TMEM buffer.
+#include <cuda_bf16.h>
+
 #include "common.cuh"
 #include "internal.h"
 
 namespace kq {
 
 namespace tg {
-constexpr int BM = 128, BN = 128, BK = 32, UK = 8, STAGES = 3;
-constexpr int TILE_BYTES = 128 * BK * 4;          // 16 KB: one operand part of one stage
-constexpr int STAGE_BYTES = 4 * TILE_BYTES;       // A_hi, A_lo, B_hi, B_lo
+constexpr int BM = 128, BN = 128, BK = 64, UK = 16, STAGES = 2;
+constexpr int PIECE_BYTES = 128 * BK * 2;         // 16 KB: one bf16 piece of one operand tile
+constexpr int STAGE_BYTES = 6 * PIECE_BYTES;      // A0, A1, A2, B0, B1, B2
+constexpr int MN_BOX_BYTES = 64 * BK * 2;         // 8 KB: 64 columns x BK rows (MN-major B)
 constexpr int THREADS = 192;
 constexpr int TMEM_COLS = 256;                    // two 128-column fp32 accumulators
 constexpr int EPI_BYTES = 4 * 32 * 33 * 4;        // per epilogue warp: a 32 x 32 transpose tile
@@ -42,22 +48,12 @@ struct TgParams {
   int* err;
 };
 
-__host__ __device__ constexpr uint32_t idesc_tf32_f32(int m, int n, bool b_mn) {
+__host__ __device__ constexpr uint32_t idesc_bf16(int m, int n, bool b_mn) {
   return (1u << 4)                 // D: f32
-         | (2u << 7)               // A: tf32
-         | (2u << 10)              // B: tf32
+         | (1u << 7)               // A: bf16
+         | (1u << 10)              // B: bf16
          | (b_mn ? (1u << 16) : 0u)
          | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
-}
-
-__device__ __forceinline__ void umma_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                          uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
 }
 
 // Tile order and K range of one output tile (identical in every role).
@@ -79,10 +75,13 @@ __device__ __forceinline__ bool tile_info(const TgParams& p, int t, TileInfo& ti
   return true;
 }
 
+struct TgMaps {
+  CUtensorMap a[3];
+  CUtensorMap b[3];
+};
+
 __global__ void __launch_bounds__(tg::THREADS, 1)
-    tgemm_kernel(const __grid_constant__ CUtensorMap ta_hi, const __grid_constant__ CUtensorMap ta_lo,
-                 const __grid_constant__ CUtensorMap tb_hi, const __grid_constant__ CUtensorMap tb_lo,
-                 const TgParams p) {
+    tgemm_kernel(const __grid_constant__ TgMaps maps, const TgParams p) {
   using namespace tg;
   if (p.skip && *p.skip >= 0) return;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -113,10 +112,10 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
-    prefetch_tensormap(&ta_hi);
-    prefetch_tensormap(&ta_lo);
-    prefetch_tensormap(&tb_hi);
-    prefetch_tensormap(&tb_lo);
+    for (int i = 0; i < 3; ++i) {
+      prefetch_tensormap(&maps.a[i]);
+      prefetch_tensormap(&maps.b[i]);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, TMEM_COLS);
@@ -145,18 +144,15 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
           uint8_t* st = smem + s * STAGE_BYTES;
           mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
           const int k0 = kb * BK;
-          tma_load_2d(st, &ta_hi, &full[s], k0, ti.tm * BM);
-          tma_load_2d(st + TILE_BYTES, &ta_lo, &full[s], k0, ti.tm * BM);
-          if (!p.b_mn_major) {
-            tma_load_2d(st + 2 * TILE_BYTES, &tb_hi, &full[s], k0, ti.tn * BN);
-            tma_load_2d(st + 3 * TILE_BYTES, &tb_lo, &full[s], k0, ti.tn * BN);
-          } else {
 #pragma unroll
-            for (int j = 0; j < BN / 32; ++j) {
-              tma_load_2d(st + 2 * TILE_BYTES + j * (TILE_BYTES / 4), &tb_hi, &full[s],
-                          ti.tn * BN + 32 * j, k0);
-              tma_load_2d(st + 3 * TILE_BYTES + j * (TILE_BYTES / 4), &tb_lo, &full[s],
-                          ti.tn * BN + 32 * j, k0);
+          for (int i = 0; i < 3; ++i) {
+            tma_load_2d(st + i * PIECE_BYTES, &maps.a[i], &full[s], k0, ti.tm * BM);
+            uint8_t* bp = st + (3 + i) * PIECE_BYTES;
+            if (!p.b_mn_major) {
+              tma_load_2d(bp, &maps.b[i], &full[s], k0, ti.tn * BN);
+            } else {
+              tma_load_2d(bp, &maps.b[i], &full[s], ti.tn * BN, k0);
+              tma_load_2d(bp + MN_BOX_BYTES, &maps.b[i], &full[s], ti.tn * BN + 64, k0);
             }
           }
         }
@@ -169,7 +165,7 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_tf32_f32(BM, BN, p.b_mn_major != 0);
+      const uint32_t idesc = idesc_bf16(BM, BN, p.b_mn_major != 0);
       uint32_t it = 0, ui = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
@@ -192,24 +188,24 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
           const uint32_t base = smem_u32(smem + s * STAGE_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / UK; ++kk) {
-            // A: K-major, 128 rows x 128 bytes, 8-row atoms of 1 KB; K step = 32 bytes.
-            const uint64_t ah = smem_desc_sw128(base + kk * 32, 16, 1024);
-            const uint64_t al = smem_desc_sw128(base + TILE_BYTES + kk * 32, 16, 1024);
-            uint64_t bh, bl;
-            if (!p.b_mn_major) {
-              bh = smem_desc_sw128(base + 2 * TILE_BYTES + kk * 32, 16, 1024);
-              bl = smem_desc_sw128(base + 3 * TILE_BYTES + kk * 32, 16, 1024);
-            } else {
-              // B: MN-major 32-bit operands use the 128-byte swizzle with 32-byte atoms (4-row
-              // K groups of 512 bytes, SBO); boxes of 32 K-rows x 128 bytes, 4 along N
-              // (LBO = 4 KB); K step = 8 rows = 1 KB.
-              bh = smem_desc(base + 2 * TILE_BYTES + kk * 1024, TILE_BYTES / 4, 512, 1u);
-              bl = smem_desc(base + 3 * TILE_BYTES + kk * 1024, TILE_BYTES / 4, 512, 1u);
+            uint64_t ad[3], bd[3];
+#pragma unroll
+            for (int i = 0; i < 3; ++i) {
+              // A: K-major, 128 rows x 128 bytes, 8-row atoms of 1 KB; K step = 32 bytes.
+              ad[i] = smem_desc_sw128(base + i * PIECE_BYTES + kk * 32, 16, 1024);
+              const uint32_t bb = base + (3 + i) * PIECE_BYTES;
+              // B: K-major like A, or MN-major in two 64-column boxes (LBO = box), K step =
+              // 16 rows = 2 KB.
+              bd[i] = p.b_mn_major ? smem_desc_sw128(bb + kk * 2048, MN_BOX_BYTES, 1024)
+                                   : smem_desc_sw128(bb + kk * 32, 16, 1024);
             }
             const uint32_t first = (kb == ti.kb0 && kk == 0) ? 0u : 1u;
-            umma_tf32(d_tmem, al, bh, idesc, first);   // lo * hi
-            umma_tf32(d_tmem, ah, bl, idesc, 1u);      // hi * lo
-            umma_tf32(d_tmem, ah, bh, idesc, 1u);      // hi * hi
+            umma_f16(d_tmem, ad[2], bd[0], idesc, first);   // smallest terms first
+            umma_f16(d_tmem, ad[1], bd[1], idesc, 1u);
+            umma_f16(d_tmem, ad[0], bd[2], idesc, 1u);
+            umma_f16(d_tmem, ad[1], bd[0], idesc, 1u);
+            umma_f16(d_tmem, ad[0], bd[1], idesc, 1u);
+            umma_f16(d_tmem, ad[0], bd[0], idesc, 1u);
           }
           umma_commit(&empty[s]);
         }
@@ -258,7 +254,8 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
 #pragma unroll
         for (int r = 0; r < 32; ++r) {
           const bool ok_rc = col < p.n && row0 + r < p.m && !(p.upper_only && col < row0 + r);
-          if (ok_rc) cbase[static_cast<int64_t>(r) * p.ldc] = fmaf(p.beta, old[r], p.alpha * tw[r * 33 + lane]);
+          if (ok_rc)
+            cbase[static_cast<int64_t>(r) * p.ldc] = fmaf(p.beta, old[r], p.alpha * tw[r * 33 + lane]);
         }
         __syncwarp();
       }
@@ -277,18 +274,18 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
   }
 }
 
-// hi = tf32(x) (round to nearest, ties away), lo = x - hi; rows x cols, any source stride,
-// destination stride ld (a multiple of 4 floats). Up to two matrices per launch.
+// x = x0 + x1 + x2 in bf16 (round to nearest even at each step; each residual is exact in fp32),
+// rows x cols, any source stride, destination stride ld (a multiple of 8 elements).
+// Up to two matrices per launch.
 struct SplitJob {
   const float* src;
   int64_t lds;
   int rows, cols;
-  float* hi;
-  float* lo;
+  uint16_t* part[3];
   int64_t ld;
 };
 
-__global__ void split_tf32_kernel(SplitJob j0, SplitJob j1) {
+__global__ void split_bf16x3_kernel(SplitJob j0, SplitJob j1) {
   const int64_t n0 = static_cast<int64_t>(j0.rows) * j0.cols;
   const int64_t total = n0 + static_cast<int64_t>(j1.rows) * j1.cols;
   for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
@@ -298,11 +295,15 @@ __global__ void split_tf32_kernel(SplitJob j0, SplitJob j1) {
     const int64_t f = second ? e - n0 : e;
     const int64_t r = f / j.cols, c = f - r * j.cols;
     const float x = j.src[r * j.lds + c];
-    uint32_t h;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(h) : "f"(x));
-    const float hf = __uint_as_float(h);
-    j.hi[r * j.ld + c] = hf;
-    j.lo[r * j.ld + c] = x - hf;
+    const __nv_bfloat16 b0 = __float2bfloat16_rn(x);
+    const float r1 = x - __bfloat162float(b0);
+    const __nv_bfloat16 b1 = __float2bfloat16_rn(r1);
+    const float r2 = r1 - __bfloat162float(b1);
+    const __nv_bfloat16 b2 = __float2bfloat16_rn(r2);
+    const int64_t o = r * j.ld + c;
+    j.part[0][o] = __bfloat16_as_ushort(b0);
+    j.part[1][o] = __bfloat16_as_ushort(b1);
+    j.part[2][o] = __bfloat16_as_ushort(b2);
   }
 }
 
@@ -326,21 +327,20 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// fp32 tensor map: rows x cols (cols contiguous, row stride ld floats), box = box_cols x box_rows,
-// 128-byte swizzle with 16-byte (K-major operands) or 32-byte (MN-major operands) atoms.
-kronq_status map_f32(CUtensorMap* map, const float* base, int64_t rows, int64_t cols, int64_t ld,
-                     int box_cols, int box_rows, bool atom32 = false) {
+// bf16 tensor map: rows x cols (cols contiguous, row stride ld elements), box = box_cols x
+// box_rows, 128-byte swizzle.
+kronq_status map_bf16(CUtensorMap* map, const uint16_t* base, int64_t rows, int64_t cols,
+                      int64_t ld, int box_cols, int box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return fail(KRONQ_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
-  if ((reinterpret_cast<uintptr_t>(base) & 15u) || (ld * 4) % 16)
+  if ((reinterpret_cast<uintptr_t>(base) & 15u) || (ld * 2) % 16)
     return fail(KRONQ_ERR_INVALID_ARG, "tensor-core GEMM operand not 16-byte aligned");
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 4};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
   cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims,
-                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   atom32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B,
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(KRONQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return KRONQ_OK;
@@ -359,41 +359,40 @@ int sm_count() {
 
 }  // namespace
 
-kronq_status split_tf32(const float* src, int64_t lds, int rows, int cols, SplitF32 dst,
-                        cudaStream_t stream) {
-  return split_tf32_2(src, lds, rows, cols, dst, nullptr, 0, 0, 0, SplitF32{}, stream);
+kronq_status split_bf16x3(const float* src, int64_t lds, int rows, int cols, Split3 dst,
+                          cudaStream_t stream) {
+  return split_bf16x3_2(src, lds, rows, cols, dst, nullptr, 0, 0, 0, Split3{}, stream);
 }
 
-kronq_status split_tf32_2(const float* src0, int64_t lds0, int rows0, int cols0, SplitF32 dst0,
-                          const float* src1, int64_t lds1, int rows1, int cols1, SplitF32 dst1,
-                          cudaStream_t stream) {
-  SplitJob j0{src0, lds0, rows0, cols0 > 0 ? cols0 : 1, dst0.hi, dst0.lo, dst0.ld};
-  SplitJob j1{src1, lds1, src1 ? rows1 : 0, cols1 > 0 ? cols1 : 1, dst1.hi, dst1.lo, dst1.ld};
-  if (cols0 <= 0) j0.rows = 0;
-  const int64_t total = static_cast<int64_t>(j0.rows) * j0.cols + static_cast<int64_t>(j1.rows) * j1.cols;
+kronq_status split_bf16x3_2(const float* src0, int64_t lds0, int rows0, int cols0, Split3 dst0,
+                            const float* src1, int64_t lds1, int rows1, int cols1, Split3 dst1,
+                            cudaStream_t stream) {
+  SplitJob j0{src0, lds0, cols0 > 0 ? rows0 : 0, cols0 > 0 ? cols0 : 1,
+              {dst0.part[0], dst0.part[1], dst0.part[2]}, dst0.ld};
+  SplitJob j1{src1, lds1, (src1 && cols1 > 0) ? rows1 : 0, cols1 > 0 ? cols1 : 1,
+              {dst1.part[0], dst1.part[1], dst1.part[2]}, dst1.ld};
+  const int64_t total =
+      static_cast<int64_t>(j0.rows) * j0.cols + static_cast<int64_t>(j1.rows) * j1.cols;
   if (total <= 0) return KRONQ_OK;
   int64_t blocks = (total + 255) / 256;
   if (blocks > 148 * 32) blocks = 148 * 32;
-  split_tf32_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(j0, j1);
-  return check_launch("split_tf32_kernel");
+  split_bf16x3_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(j0, j1);
+  return check_launch("split_bf16x3_kernel");
 }
 
-kronq_status tgemm(int m, int n, int k, float alpha, SplitF32 a, SplitF32 b, bool b_mn_major,
+kronq_status tgemm(int m, int n, int k, float alpha, Split3 a, Split3 b, bool b_mn_major,
                    float beta, float* c, int64_t ldc, bool upper_only, int tri,
                    const int32_t* skip, cudaStream_t stream) {
   using namespace tg;
   if (m <= 0 || n <= 0) return KRONQ_OK;
   if (k <= 0) return fail(KRONQ_ERR_SHAPE, "tensor-core GEMM needs k >= 1");
-  CUtensorMap mah, mal, mbh, mbl;
-  const int kk = k;
-  KQ_TRY(map_f32(&mah, a.hi, m, kk, a.ld, BK, BM));
-  KQ_TRY(map_f32(&mal, a.lo, m, kk, a.ld, BK, BM));
-  if (!b_mn_major) {
-    KQ_TRY(map_f32(&mbh, b.hi, n, kk, b.ld, BK, BN));
-    KQ_TRY(map_f32(&mbl, b.lo, n, kk, b.ld, BK, BN));
-  } else {
-    KQ_TRY(map_f32(&mbh, b.hi, kk, n, b.ld, 32, BK, true));
-    KQ_TRY(map_f32(&mbl, b.lo, kk, n, b.ld, 32, BK, true));
+  TgMaps maps;
+  for (int i = 0; i < 3; ++i) {
+    KQ_TRY(map_bf16(&maps.a[i], a.part[i], m, k, a.ld, BK, BM));
+    if (!b_mn_major)
+      KQ_TRY(map_bf16(&maps.b[i], b.part[i], n, k, b.ld, BK, BN));
+    else
+      KQ_TRY(map_bf16(&maps.b[i], b.part[i], k, n, b.ld, 64, BK));
   }
   TgParams p{};
   p.c = c;
@@ -419,7 +418,7 @@ kronq_status tgemm(int m, int n, int k, float alpha, SplitF32 a, SplitF32 b, boo
   }
   const int tiles = p.tiles_m * p.tiles_n;
   const int sms = sm_count();
-  tgemm_kernel<<<tiles < sms ? tiles : sms, THREADS, SMEM_BYTES, stream>>>(mah, mal, mbh, mbl, p);
+  tgemm_kernel<<<tiles < sms ? tiles : sms, THREADS, SMEM_BYTES, stream>>>(maps, p);
   return check_launch("tgemm_kernel");
 }
 

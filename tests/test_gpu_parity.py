@@ -202,7 +202,8 @@ def test_cholinv_matches_oracle(K, d):
 
 
 @pytest.mark.parametrize("d", [4096, 11008])
-def test_cholinv_llama_width_residual(K, d):
+def test_cholinv_llama_width(K, d):
+    # LLaMA-2-7B widths: the whole K against the oracle's fp64 three-step factor of the same H
     n = 3 * d
     x = synth.correlated_x(n, d, synth.seed_for("chol", d), device="cuda")
     h = torch.zeros(d, d, device="cuda")
@@ -212,20 +213,32 @@ def test_cholinv_llama_width_residual(K, d):
     info = torch.empty(1, dtype=torch.int32, device="cuda")
     K.kronq_cholinv(k, 0.01, info, K.CHOLINV_SYNC)
     hd = h64(h); kd = h64(k)
+    ko = O.cholinv(hd, 0.01)
+    err = rel(kd, ko)
+    # A forward error below kappa(A) * u is out of reach for any fp32 factorization, so the bar
+    # is 1e-3 or 4 kappa(A) 2^-24 where that is larger (kappa by power iteration on A and on
+    # A^-1 = K^T K).
     lam = 0.01 * np.mean(np.diag(hd))
-    a = hd + lam * np.eye(d)
-    # K^T K = A^-1 with K square and invertible is the same as K A K^T = I; this residual sees
-    # K's relative error directly (K^T K A v - v would amplify it by cond(A) ~ 1e4 here)
-    r = np.random.default_rng(0)
-    worst = 0.0
-    for _ in range(8):
-        v = r.standard_normal(d)
-        res = kd @ (a @ (kd.T @ v)) - v
-        worst = max(worst, np.linalg.norm(res) / np.linalg.norm(v))
-    print(f"d={d}: max |K A K^T v - v| / |v| = {worst:.2e}")
-    assert worst <= TOL
+    kappa = cond_estimate(hd + lam * np.eye(d), ko)
+    bar = max(TOL, 4 * kappa * 2.0 ** -24)
+    print(f"d={d}: |K - K_oracle| / |K_oracle| = {err:.2e}, kappa ~ {kappa:.2e}, bar {bar:.2e}")
+    assert err <= bar
     assert np.all(np.diag(kd) > 0)
     assert np.all(np.tril(kd, -1) == 0)
+
+
+def cond_estimate(a, k, iters=30):
+    """2-norm condition number of SPD a, with a^-1 = k^T k (power iteration on both)."""
+    r = np.random.default_rng(5)
+    v = r.standard_normal(a.shape[0])
+    for _ in range(iters):
+        v = a @ v; v /= np.linalg.norm(v)
+    big = float(v @ (a @ v))
+    u = r.standard_normal(a.shape[0])
+    for _ in range(iters):
+        u = k.T @ (k @ u); u /= np.linalg.norm(u)
+    small_inv = float(u @ (k.T @ (k @ u)))
+    return big * small_inv
 
 
 def test_cholinv_not_positive_definite(K):
@@ -298,6 +311,28 @@ def test_quantize_llama_shape_sampled_rows(K, P):
     assert rel(h64(r.w_hat[rows]), o["w_hat"]) <= TOL
 
 
+def test_quantize_llama_shape_with_oracle_factor(K, P):
+    # The same q_proj shape, but the oracle quantizes its rows with its own fp64 factor of the
+    # GPU's H_X' (not the GPU's K): codes and W^ must still meet the bars, so the fp32 factor's
+    # error does not leak into the result.
+    d_out = d_in = 4096
+    n = 8192
+    xq, _, g, w, si, so = layer_inputs(d_out, d_in, n, drift="none", w_dtype=torch.bfloat16,
+                                       tag="q-full-ofac")
+    hx = torch.zeros(d_in, d_in, device="cuda"); hg = torch.zeros(d_out, d_out, device="cuda")
+    K.kronq_accumulate(xq, None, g, hx, hg)
+    r = P.biip(w, hx, hg, None, 1.0 / n, si, so, 15)
+    wp = r.w_prime.clone(); hxp = r.hx.clone()
+    P.cholinv(r, 0.01, sync=True)
+    P.quantize(r, 4)
+    torch.cuda.synchronize()
+    ko = O.cholinv(h64(hxp), 0.01)
+    rows = np.random.default_rng(2).choice(d_out, 32, replace=False)
+    o = O.quantize_layer(h64(wp[rows]), ko, None, 4, follow_codes=h64(r.codes[rows]))
+    check_codes(r.codes[rows], o, 32 * d_in)
+    assert rel(h64(r.w_hat[rows]), o["w_hat"]) <= TOL
+
+
 # ------------------------------------------------------------------------------ end to end
 
 @pytest.mark.parametrize("flags", [0, 15])
@@ -322,3 +357,169 @@ def test_layer256_end_to_end(K, P, flags):
 
 def test_no_device_error_recorded(K):
     assert K.kronq_device_error() == 0
+
+
+# ------------------------------------------------------------------------------ other workloads
+
+def test_drift_term_llama3_8b_width(K):
+    # LLaMA-3-8B hidden width 4096, X~ = X + N(0, (0.05 rms X)^2), 16384 tokens: sampled tiles of
+    # the drift sum D += (X - X~)^T X~ and of H_X against fp64 sums of the same bf16 values
+    n, d = 16384, 4096
+    x = synth.correlated_x(n, d, synth.seed_for("drift8b", "X"), device="cuda")
+    xq = synth.perturbed(x, synth.seed_for("drift8b", "Xq"), rel_std=0.05)
+    hx = torch.zeros(d, d, device="cuda"); dxx = torch.zeros(d, d, device="cuda")
+    K.kronq_accumulate(xq, x, None, hx, None, dxx)
+    torch.cuda.synchronize()
+    r = np.random.default_rng(7)
+    for _ in range(8):
+        i0 = int(r.integers(0, d // 128)) * 128; j0 = int(r.integers(0, d // 128)) * 128
+        xa = h64(x[:, i0:i0 + 128]); qa = h64(xq[:, i0:i0 + 128]); qb = h64(xq[:, j0:j0 + 128])
+        assert rel(h64(dxx[i0:i0 + 128, j0:j0 + 128]), (xa - qa).T @ qb) <= TOL
+        assert rel(h64(hx[i0:i0 + 128, j0:j0 + 128]), qa.T @ qb) <= TOL
+
+
+def test_biip_llama3_70b_down_shape(K, P):
+    # down_proj of LLaMA-3-70B: 8192 x 28672 (input Hadamard blocks of 4096, output 8192).
+    # Full-size check through the inverse transforms: (U^T W' V)_ij = s_g,i W_ij s_x,j on
+    # sampled entries, each from a b_out x b_in block of W'; plus the oracle's scales.
+    d_out, d_in, n = 8192, 28672, 2048
+    x = synth.correlated_x(n, d_in, synth.seed_for("b70", "X"), device="cuda")
+    g = synth.gradients(n, d_out, synth.seed_for("b70", "G"), device="cuda")
+    w = synth.weight(d_out, d_in, synth.seed_for("b70", "W"), device="cuda")
+    si = synth.rademacher(d_in, synth.seed_for("b70", "si"), device="cuda")
+    so = synth.rademacher(d_out, synth.seed_for("b70", "so"), device="cuda")
+    hx = torch.zeros(d_in, d_in, device="cuda"); hg = torch.zeros(d_out, d_out, device="cuda")
+    K.kronq_accumulate(x, None, g, hx, hg)
+    hx_diag = torch.diagonal(hx).clone(); hg_diag = torch.diagonal(hg).clone()
+    r = P.biip(w, hx, hg, None, 1.0 / n, si, so, 15, copy_hx=False)
+    torch.cuda.synchronize()
+    w64 = h64(w)
+    col_sq = (w64 ** 2).sum(0); row_sq = (w64 ** 2).sum(1)
+    sx = (h64(hx_diag) / n / col_sq) ** 0.25
+    sg = (h64(hg_diag) / n / row_sq) ** 0.25
+    assert rel(h64(r.s_x), sx) <= TOL and rel(h64(r.s_g), sg) <= TOL
+    tr_hx = float(np.sum(h64(hx_diag) / n / sx ** 2))
+    assert abs(float(r.tr[0]) - tr_hx) <= TOL * tr_hx
+    bi, bo = O.hadamard_block_size(d_in), O.hadamard_block_size(d_out)
+    hb_i = O.sylvester(bi) / math.sqrt(bi); hb_o = O.sylvester(bo) / math.sqrt(bo)
+    sin = h64(si); sout = h64(so)
+    rng = np.random.default_rng(70)
+    got, want = [], []
+    for _ in range(24):
+        i = int(rng.integers(0, d_out)); j = int(rng.integers(0, d_in))
+        ib, jb = (i // bo) * bo, (j // bi) * bi
+        blk = h64(r.w_prime[ib:ib + bo, jb:jb + bi])
+        u_i = hb_o[:, i - ib] * sout[i]          # column i of U = (1/sqrt b)(H_b) diag(sign)
+        v_j = hb_i[:, j - jb] * sin[j]
+        got.append(u_i @ blk @ v_j)
+        want.append(sg[i] * w64[i, j] * sx[j])
+    assert rel(np.array(got), np.array(want)) <= TOL
+    # the rotation preserves the Frobenius norm of S_G W S_X
+    nrm = float(torch.linalg.vector_norm(r.w_prime.double()))
+    assert abs(nrm - np.linalg.norm(sg[:, None] * w64 * sx[None, :])) <= TOL * nrm
+
+
+def test_cholinv_llama3_70b_width(K):
+    # H_X of the 70B down_proj input (d = 28672, 3.3 GB fp32). Backward error of the factor:
+    # with R = K^-1 (an exact fp64 triangular solve of the GPU's K), R R^T v must equal
+    # (H + lambda I) v to the bar, for random v. Unlike K (H + lambda I) K^T - I, this residual
+    # is not multiplied by the condition number (~4e4 here), so it measures the factor's
+    # accuracy rather than the fp32 rounding of its storage.
+    import scipy.linalg as sla
+    d = 28672
+    n = 2 * d
+    x = synth.correlated_x(n, d, synth.seed_for("chol70", d), device="cuda", chunk=8192)
+    h = torch.zeros(d, d, device="cuda")
+    K.kronq_accumulate(x, None, None, h)
+    del x
+    h /= n
+    hd = h64(h)
+    info = torch.empty(1, dtype=torch.int32, device="cuda")
+    K.kronq_cholinv(h, 0.01, info, K.CHOLINV_SYNC)
+    kd = h64(h)
+    del h
+    torch.cuda.empty_cache()
+    lam = 0.01 * np.mean(np.diag(hd))
+    r = np.random.default_rng(1)
+    worst = 0.0
+    for _ in range(3):
+        v = r.standard_normal(d)
+        av = hd @ v + lam * v
+        y = sla.solve_triangular(kd, v, trans="T", lower=False)   # K^-T v = R^T v
+        rrt = sla.solve_triangular(kd, y, lower=False)            # K^-1 K^-T v = R R^T v
+        worst = max(worst, np.linalg.norm(rrt - av) / np.linalg.norm(av))
+    print(f"d={d}: max |R R^T v - A v| / |A v| = {worst:.2e}")
+    assert worst <= TOL
+    assert np.all(np.diag(kd) > 0)
+    # the bottom-right block of K depends only on the bottom-right block of A (the factorization
+    # runs from the last index up): compare it with the oracle's factor of that block alone
+    m = 2048
+    sub = hd[-m:, -m:]
+    ko = O.cholinv(sub, lam / float(np.mean(np.diag(sub))))
+    assert rel(kd[-m:, -m:], ko) <= TOL
+
+
+def test_quantize_with_drift_llama3_8b_kv(K, P):
+    # k_proj of LLaMA-3-8B (1024 x 4096), 3 bits, drifted input so P is active: 32 rows re-run
+    # by the oracle (literal column update with the P term) from the GPU's K, W' and D'
+    d_out, d_in, n = 1024, 4096, 8192
+    x = synth.correlated_x(n, d_in, synth.seed_for("kv8b", "X"), device="cuda")
+    xq = synth.perturbed(x, synth.seed_for("kv8b", "Xq"), rel_std=0.05)
+    g = synth.gradients(n, d_out, synth.seed_for("kv8b", "G"), device="cuda")
+    w = synth.weight(d_out, d_in, synth.seed_for("kv8b", "W"), device="cuda")
+    si = synth.rademacher(d_in, synth.seed_for("kv8b", "si"), device="cuda")
+    so = synth.rademacher(d_out, synth.seed_for("kv8b", "so"), device="cuda")
+    hx = torch.zeros(d_in, d_in, device="cuda"); hg = torch.zeros(d_out, d_out, device="cuda")
+    dxx = torch.zeros(d_in, d_in, device="cuda")
+    K.kronq_accumulate(xq, x, g, hx, hg, dxx)
+    r = P.biip(w, hx, hg, dxx, 1.0 / n, si, so, 15)
+    wp = r.w_prime.clone(); dp = r.dxx.clone()
+    P.cholinv(r, 0.01, sync=True)
+    P.quantize(r, 3)
+    torch.cuda.synchronize()
+    rows = np.random.default_rng(8).choice(d_out, 32, replace=False)
+    o = O.quantize_layer(h64(wp[rows]), h64(r.hx), h64(dp), 3, follow_codes=h64(r.codes[rows]))
+    check_codes(r.codes[rows], o, 32 * d_in)
+    assert rel(h64(r.w_hat[rows]), o["w_hat"]) <= TOL
+
+
+def test_stack_scores_and_allocation(K, P):
+    # Two blocks of the LLaMA-2-7B mixed-precision stack (14 sublayers, each its own X and G,
+    # 65536 tokens, per-block G scale log-uniform on [1e-2, 1e1]): traces after BiIP against
+    # fp64 sums of the same bf16 inputs, and the {2,3,4}-bit allocation at 2.5 average bits
+    # bit-exact against the oracle's greedy on the same scores.
+    wl = synth.WORKLOADS["llama2_7b_stack"]
+    n = wl.n_tokens
+    tr_gpu, tr_ora, sizes = [], [], []
+    for blk in range(2):
+        mult = 10 ** np.random.default_rng(blk).uniform(-2, 1)
+        for s in wl.sublayers:
+            tag = ("stack", blk, s.name)
+            x = synth.correlated_x(n, s.d_in, synth.seed_for(tag, "X"), device="cuda")
+            g = synth.gradients(n, s.d_out, synth.seed_for(tag, "G"), device="cuda", multiplier=mult)
+            w = synth.weight(s.d_out, s.d_in, synth.seed_for(tag, "W"), device="cuda")
+            si = synth.rademacher(s.d_in, synth.seed_for(tag, "si"), device="cuda")
+            so = synth.rademacher(s.d_out, synth.seed_for(tag, "so"), device="cuda")
+            hx = torch.zeros(s.d_in, s.d_in, device="cuda")
+            hg = torch.zeros(s.d_out, s.d_out, device="cuda")
+            K.kronq_accumulate(x, None, g, hx, hg)
+            r = P.biip(w, hx, hg, None, 1.0 / n, si, so, 15, copy_hx=False)
+            torch.cuda.synchronize()
+            tr_gpu.append((float(r.tr[0]), float(r.tr[1])))
+            # fp64: diag sums from the inputs, norms from W, traces of S^-1 H S^-1
+            dx = (x.double() ** 2).sum(0).cpu().numpy() / n
+            dg = (g.double() ** 2).sum(0).cpu().numpy() / n
+            w64 = h64(w)
+            sx = (dx / (w64 ** 2).sum(0)) ** 0.25; sg = (dg / (w64 ** 2).sum(1)) ** 0.25
+            tr_ora.append((float(np.sum(dx / sx ** 2)), float(np.sum(dg / sg ** 2))))
+            sizes.append(s.d_out * s.d_in)
+            del x, g, hx, hg, r
+    for (a, b), (c, e) in zip(tr_gpu, tr_ora):
+        assert abs(a - c) <= TOL * c and abs(b - e) <= TOL * e
+    s_k, bits_k = K.kronq_score_allocate([t[0] for t in tr_gpu], [t[1] for t in tr_gpu], sizes,
+                                         [2, 3, 4], 2.5)
+    s_o, bits_o = O.score_allocate([t[0] for t in tr_gpu], [t[1] for t in tr_gpu], sizes,
+                                   [2, 3, 4], 2.5)
+    assert bits_k == bits_o and s_k == s_o
+    assert sum(b * m for b, m in zip(bits_k, sizes)) <= math.floor(2.5 * sum(sizes))
+    assert len(set(bits_k)) > 1
