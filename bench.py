@@ -331,6 +331,11 @@ def run_gpu(args):
             peak = 1400.0
             peak_src = "fallback (sustained bf16)"
         achieved = sum(acc_flops) / (sum(acc_ms) / 1e3) / 1e12
+        # DRAM bytes (read + write) per accumulate_tc_kernel launch, averaged over a step's 8
+        # launches at d = 4096 and 3 at d = 11008; from ncu captures of this kernel version at
+        # the same 16384-token work units, scaled to 262144 tokens (see the accumulate summary
+        # under profiles/)
+        traffic = 16.7e9 if n_tok == 262144 else None
         acc_tflops = sum(acc_flops) / (sum(acc_ms) / 1e3) / 1e12
         result = {
             "metric": "quantized weight params/s (BiIP+GPTAQ solve); H_X/H_G accumulate TFLOP/s",
@@ -354,7 +359,8 @@ def run_gpu(args):
             "accumulate_tflops": acc_tflops,
             "roofline": {"bound": "tensor", "kernel": "accumulate_tc_kernel",
                          "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "peak_source": peak_src, "traffic": None},
+                         "frac": achieved / peak, "peak_source": peak_src, "traffic": traffic,
+                         "traffic_unit": "bytes per launch"},
             "gpu_launches": launches,
             "clocks": clk,
             "e2e": e2e,
