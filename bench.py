@@ -306,10 +306,8 @@ def run_gpu(args):
     elapsed = t_start.elapsed_time(t_end) / 1e3
     acc_ms = [a.elapsed_time(b) for a, b, _ in blk.acc_events]
     acc_flops = [f for _, _, f in blk.acc_events]
-    t = torch.tensor([elapsed], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    elapsed_max = float(t)
+    from post_quantization_b200 import dist as D
+    elapsed_max = D.max_over_ranks(elapsed, device=dev)
     params = wl.params_per_block * world
     value = params * args.steps / elapsed_max
 
