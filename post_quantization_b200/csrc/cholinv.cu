@@ -60,124 +60,206 @@ __global__ void prep_kernel(float* __restrict__ a, int d, const float* __restric
 }
 
 // Leaf: factor the nb x nb diagonal block at a (ld) as A = R R^T (R upper) and overwrite its
-// upper triangle with K = R^-1. One CTA of 512 threads; thread t keeps the 4 x 8 block
-// rows 4*(t/16) .. +3, columns 8*(t%16) .. +7 in registers. Both sweeps are right-looking with
-// one barrier per column; the column (row) that drives a step is published in shared memory by
-// the threads that own it:
-//   factor   c = nb-1 .. 0:  u = S_:c;  R_:c = u / sqrt(u_c);  S_ik -= u_i u_k / u_c  (i <= k < c)
-//   inverse  i = nb-1 .. 0:  K_ij = (delta_ij - acc_ij) / R_ii (j >= i);  acc_rj += R_ri K_ij (r < i)
+// upper triangle with K = R^-1 (strict lower triangle := 0). One CTA of 512 threads; the block is
+// padded to 128 with an identity bottom-right part, which factors to itself and leaves the rest
+// unchanged.
+//
+// Blocked by 32-column panels P = [p0, p0 + 32), right to left, on the Schur-updated matrix S:
+//   S_PP = R_PP R_PP^T and K_PP = R_PP^-1      one warp, in registers (shuffles, no barriers)
+//   R_{<p0,P} = S_{<p0,P} K_PP^T               (S_{<p0,P} = R_{<p0,P} R_PP^T)
+//   S_{<p0,<p0} -= R_{<p0,P} R_{<p0,P}^T        (upper triangle)
+// then the off-diagonal blocks of K = R^-1 by block rows, bottom up:
+//   K_ij = -K_ii sum_{l=i+1..j} R_il K_lj       (j > i; from R K = I)
+// The products run from shared memory, a 16 x 32 tile per warp with a 4 x 4 register block per
+// lane. K's blocks are kept transposed in the (otherwise free) lower part of the R buffer, so
+// every product reads both operands along rows.
 constexpr int LEAF_THREADS = 512;
-constexpr int LD_R = NB + 1;
-constexpr size_t LEAF_SMEM = sizeof(float) * (NB * LD_R + 4 * NB);
+constexpr int PW = 32;                  // panel width
+constexpr int LDS = NB + 4;             // row stride: 16-byte rows, consecutive rows 4 banks apart
+constexpr int LDT = PW + 4;
+constexpr size_t LEAF_SMEM = sizeof(float) * (2 * NB * LDS + (NB - PW) * LDT) + 16;
+
+// acc[i][j] += sum_{m in [m0, m1)} X[r_i][m] * Y[c_j][m] for this lane's rows r_i = tr + ly + 4i
+// and columns c_j = tc + lx + 8j of a 16 x 32 warp tile (m0, m1 multiples of 4). Both reads are
+// conflict-free: the 4 (8) distinct rows of one read sit 4 banks apart.
+__device__ __forceinline__ void tile_acc(float (&acc)[4][4], const float* __restrict__ x, int ldx,
+                                         const float* __restrict__ y, int ldy, int tr, int tc,
+                                         int m0, int m1, int lane) {
+  const int ly = lane >> 3, lx = lane & 7;
+  const float* xr = x + (tr + ly) * ldx;
+  const float* yr = y + (tc + lx) * ldy;
+#pragma unroll 2
+  for (int m = m0; m < m1; m += 4) {
+    float4 xv[4], yv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) xv[i] = *reinterpret_cast<const float4*>(xr + 4 * i * ldx + m);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) yv[j] = *reinterpret_cast<const float4*>(yr + 8 * j * ldy + m);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        acc[i][j] = fmaf(xv[i].x, yv[j].x, acc[i][j]);
+        acc[i][j] = fmaf(xv[i].y, yv[j].y, acc[i][j]);
+        acc[i][j] = fmaf(xv[i].z, yv[j].z, acc[i][j]);
+        acc[i][j] = fmaf(xv[i].w, yv[j].w, acc[i][j]);
+      }
+  }
+}
+
+__device__ __forceinline__ void zero4x4(float (&acc)[4][4]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+}
 
 __global__ void __launch_bounds__(LEAF_THREADS, 1) leaf_kernel(float* __restrict__ a, int64_t ld,
                                                             int nb, int j0,
                                                             int32_t* __restrict__ info) {
-  extern __shared__ float leaf_smem[];
-  float* R = leaf_smem;                 // NB x LD_R: the factor R
-  float* pub = leaf_smem + NB * LD_R;   // 2 x NB double-buffered published column / row
+  extern __shared__ __align__(16) float leaf_smem[];
+  float* S = leaf_smem;                 // NB x LDS: S (upper), then K_ii in the diagonal blocks
+  float* R = S + NB * LDS;              // NB x LDS: R off-diagonal blocks (upper), K^T (lower)
+  float* T = R + NB * LDS;              // (NB - PW) x LDT: one block row of sum R_il K_lj, transposed
+  int* bad = reinterpret_cast<int*>(T + (NB - PW) * LDT);
   if (*info >= 0) return;
-  const int tid = threadIdx.x;
-  const int r0 = 4 * (tid >> 4);        // first owned row
-  const int c0 = 8 * (tid & 15);        // first owned column
-  float s[4][8];
-#pragma unroll
-  for (int r = 0; r < 4; ++r)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int i = r0 + r, k = c0 + j;
-      s[r][j] = (i < nb && k < nb && k >= i) ? a[i * ld + k] : 0.f;
-    }
-  for (int e = tid; e < NB * LD_R; e += blockDim.x) R[e] = 0.f;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int ly = lane >> 3, lx = lane & 7;
+  constexpr int NWARPS = LEAF_THREADS / 32;
+
+  for (int e = tid; e < NB * NB; e += LEAF_THREADS) {
+    const int r = e / NB, c = e % NB;
+    float v;
+    if (r < nb && c < nb)
+      v = c >= r ? a[r * ld + c] : 0.f;
+    else
+      v = r == c ? 1.f : 0.f;
+    S[r * LDS + c] = v;
+    if (r > c && (r >> 5) != (c >> 5) && r < nb && c < nb) a[r * ld + c] = 0.f;
+  }
+  if (tid == 0) *bad = -1;
   __syncthreads();
 
-  for (int c = nb - 1; c >= 0; --c) {
-    float* u = pub + (c & 1) * NB;
-    if ((c >> 3) == (tid & 15)) {            // owners of column c publish it
+  for (int p0 = NB - PW; p0 >= 0; p0 -= PW) {
+    if (warp == 0) {
+      // lane k holds column k of the symmetric panel block (both triangles, so that the
+      // multiplier S_ck of lane k is a register with a compile-time index)
+      float s[PW];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        // pick s[r][c % 8] with masks (an indexed read would move s to local memory)
-        int vi = 0;
-        const int cj = c & 7;
+      for (int i = 0; i < PW; ++i) {
+        const int r = i < lane ? i : lane, c = i < lane ? lane : i;
+        s[i] = S[(p0 + r) * LDS + p0 + c];
+      }
+      float mypiv = 1.f;
+      int fail = -1;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) vi |= __float_as_int(s[r][j]) & -static_cast<int>(j == cj);
-        u[r0 + r] = __int_as_float(vi);
+      for (int c = PW - 1; c >= 0; --c) {
+        const float piv = __shfl_sync(0xffffffffu, s[c], c);
+        if (!(piv > 0.f) || !isfinite(piv)) {   // uniform: every lane has the same pivot
+          fail = c;
+          break;
+        }
+        mypiv = lane == c ? piv : mypiv;
+        const float f = s[c] * __frcp_rn(piv);
+#pragma unroll
+        for (int i = c - 1; i >= 0; --i) {
+          const float v = __shfl_sync(0xffffffffu, s[i], c);
+          if (lane < c) s[i] = fmaf(-v, f, s[i]);
+        }
+      }
+      if (fail >= 0) {
+        if (lane == 0) *bad = p0 + fail;
+      } else {
+        // lane k: column k of R_PP, then column k of K_PP = R_PP^-1 by right-looking substitution
+        const float rs = rsqrtf(mypiv), sq = sqrtf(mypiv);
+#pragma unroll
+        for (int i = 0; i < PW; ++i) s[i] = i < lane ? s[i] * rs : (i == lane ? sq : 0.f);
+        float k[PW];
+#pragma unroll
+        for (int i = 0; i < PW; ++i) k[i] = 0.f;
+#pragma unroll
+        for (int i = PW - 1; i >= 0; --i) {
+          const float rii = __shfl_sync(0xffffffffu, s[i], i);
+          k[i] = ((lane == i ? 1.f : 0.f) - k[i]) * __frcp_rn(rii);
+#pragma unroll
+          for (int r = 0; r < i; ++r) k[r] = fmaf(__shfl_sync(0xffffffffu, s[r], i), k[i], k[r]);
+        }
+#pragma unroll
+        for (int i = 0; i < PW; ++i) {
+          S[(p0 + i) * LDS + p0 + lane] = k[i];        // K_PP
+          R[(p0 + lane) * LDS + p0 + i] = k[i];        // K_PP^T
+          if (p0 + i < nb && p0 + lane < nb) a[(p0 + i) * ld + p0 + lane] = k[i];
+        }
       }
     }
     __syncthreads();
-    const float piv = u[c];
-    if (!(piv > 0.f) || !isfinite(piv)) {
-      if (tid == 0) *info = j0 + c;
-      return;                                // uniform: every thread read the same pivot
+    if (*bad >= 0) {
+      if (tid == 0 && *bad < nb) *info = j0 + *bad;
+      return;                                  // uniform
     }
-    const float inv = 1.f / piv;
-    if (tid < c) R[tid * LD_R + c] = u[tid] * rsqrtf(piv);
-    if (tid == c) R[c * LD_R + c] = sqrtf(piv);
-    // only blocks that meet the shrinking triangle i <= k < c have work
-    if (c0 < c && r0 <= c0 + 7) {
-      float ui[4], uk[8];
+    if (p0 == 0) break;
+    // R_{<p0,P} = S_{<p0,P} K_PP^T: p0 / 16 tiles of 16 x 32
+    for (int t = warp; t < p0 / 16; t += NWARPS) {
+      float acc[4][4];
+      zero4x4(acc);
+      tile_acc(acc, S + p0, LDS, S + p0 * LDS + p0, LDS, 16 * t, 0, 0, PW, lane);
 #pragma unroll
-      for (int r = 0; r < 4; ++r) ui[r] = u[r0 + r] * inv;
+      for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int j = 0; j < 8; ++j) uk[j] = u[c0 + j];
+        for (int j = 0; j < 4; ++j) R[(16 * t + ly + 4 * i) * LDS + p0 + lx + 8 * j] = acc[i][j];
+    }
+    __syncthreads();
+    // S_{<p0,<p0} -= R_{<p0,P} R_{<p0,P}^T on the tiles that meet the upper triangle
+    {
+      const int tcols = p0 / 32, ntiles = (p0 / 16) * tcols;
+      for (int t = warp; t < ntiles; t += NWARPS) {
+        const int tr = 16 * (t / tcols), tc = 32 * (t % tcols);
+        if (tr >= tc + 32) continue;
+        float acc[4][4];
+        zero4x4(acc);
+        tile_acc(acc, R + p0, LDS, R + p0, LDS, tr, tc, 0, PW, lane);
 #pragma unroll
-      for (int r = 0; r < 4; ++r)
+        for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int i = r0 + r, k = c0 + j;
-          if (k < c && i <= k) s[r][j] -= ui[r] * uk[j];
+          for (int j = 0; j < 4; ++j) S[(tr + ly + 4 * i) * LDS + tc + lx + 8 * j] -= acc[i][j];
+      }
+    }
+    __syncthreads();
+  }
+
+  // K_ij (j > i), block rows bottom up
+  for (int bi = NB / PW - 2; bi >= 0; --bi) {
+    const int i0 = PW * bi, nj = NB / PW - 1 - bi;
+    // T_ij = sum_{l=i+1..j} R_il K_lj, stored transposed: T[32 (j - i - 1) + c][r]
+    for (int t = warp; t < 2 * nj; t += NWARPS) {
+      const int jj = t >> 1, tr = i0 + 16 * (t & 1), tc = i0 + PW * (jj + 1);
+      float acc[4][4];
+      zero4x4(acc);
+      tile_acc(acc, R, LDS, R, LDS, tr, tc, i0 + PW, tc + PW, lane);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          T[(PW * jj + lx + 8 * j) * LDT + tr - i0 + ly + 4 * i] = acc[i][j];
+    }
+    __syncthreads();
+    // K_ij = -K_ii T_ij: into K^T (lower part of R) and to global memory
+    for (int t = warp; t < 2 * nj; t += NWARPS) {
+      const int jj = t >> 1, tr = i0 + 16 * (t & 1), tc = i0 + PW * (jj + 1);
+      float acc[4][4];
+      zero4x4(acc);
+      tile_acc(acc, S + i0, LDS, T + PW * jj * LDT, LDT, tr, 0, 0, PW, lane);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int r = tr + ly + 4 * i, c = tc + lx + 8 * j;
+          R[c * LDS + r] = -acc[i][j];
+          if (r < nb && c < nb) a[r * ld + c] = -acc[i][j];
         }
     }
-  }
-  __syncthreads();   // R complete
-
-  // inverse: the registers now accumulate, and end up holding K
-#pragma unroll
-  for (int r = 0; r < 4; ++r)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) s[r][j] = 0.f;
-  for (int i = nb - 1; i >= 0; --i) {
-    float* kr = pub + (i & 1) * NB;
-    if ((i >> 2) == (tid >> 4)) {            // owners of row i finish it and publish it
-      const float rinv = 1.f / R[i * LD_R + i];
-      const int ir = i & 3;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int k = c0 + j;
-        float acc = s[0][j];
-        acc = ir == 1 ? s[1][j] : acc;
-        acc = ir == 2 ? s[2][j] : acc;
-        acc = ir == 3 ? s[3][j] : acc;
-        const float v = (k >= i && k < nb) ? ((k == i ? 1.f : 0.f) - acc) * rinv : 0.f;
-        s[0][j] = ir == 0 ? v : s[0][j];
-        s[1][j] = ir == 1 ? v : s[1][j];
-        s[2][j] = ir == 2 ? v : s[2][j];
-        s[3][j] = ir == 3 ? v : s[3][j];
-        kr[k] = v;
-      }
-    }
     __syncthreads();
-    // rows above i, columns from i on
-    if (r0 < i && c0 + 7 >= i) {
-      float rri[4], kij[8];
-#pragma unroll
-      for (int r = 0; r < 4; ++r) rri[r] = R[(r0 + r) * LD_R + i];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) kij[j] = kr[c0 + j];
-#pragma unroll
-      for (int r = 0; r < 4; ++r)
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          if (r0 + r < i) s[r][j] += rri[r] * kij[j];
-    }
   }
-#pragma unroll
-  for (int r = 0; r < 4; ++r)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int i = r0 + r, k = c0 + j;
-      if (i < nb && k < nb) a[i * ld + k] = (k >= i) ? s[r][j] : 0.f;
-    }
 }
 
 struct Ctx {

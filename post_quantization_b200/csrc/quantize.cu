@@ -27,7 +27,8 @@ constexpr int QB = 128;        // column block
 constexpr int QROWS = 32;      // rows per CTA in the block solve
 constexpr int QT = 4;          // threads per row
 constexpr int QW = QB / QT;    // columns per thread
-constexpr int KS_LD = QT * (QW + 1);   // padded row of the K block in shared memory
+constexpr int KQ = QW + 4;     // padded quarter row (16-byte aligned, quarters 4 banks apart)
+constexpr int KS_LD = QT * KQ; // row of the K block in shared memory
 
 // Per-row grid from W (before the solve), all decisions in fp32:
 // scale = (hi - lo) / (2^b - 1) (1 if hi == lo), zero = rint(-lo / scale).
@@ -66,8 +67,9 @@ __global__ void striu_kernel(float* __restrict__ m, int d) {
 // One 128-column block of the solve for QROWS rows. Four threads share a row, each holding 32
 // of the block's columns in registers. At column p the thread that owns it quantizes it and
 // hands the scaled error to the other three (a shuffle within the group of four), and every
-// thread updates its own columns to the right of p. The K block sits in shared memory with
-// 33-float quarters so that the four threads of a row read from different banks.
+// thread updates its own columns to the right of p. The K block sits in shared memory in
+// 36-float quarters: 16-byte aligned for vector reads, and the four threads of a row read from
+// different banks.
 //   w_hat  d_out x d_in running weights (in: current values, out: dequantized for the block)
 //   delta  d_out x QB errors scaled by 1/K_pp, written as three bf16 pieces (the operand of
 //          the lazy trailing update on the tensor cores)
@@ -91,7 +93,7 @@ __global__ void __launch_bounds__(QROWS * QT) block_solve_kernel(
     for (int e = tid; e < QB * QB / 4; e += blockDim.x) {
       const int i = e / (QB / 4), j4 = (e % (QB / 4)) * 4;
       const float4 v = *reinterpret_cast<const float4*>(k + static_cast<int64_t>(b0 + i) * d_in + b0 + j4);
-      float* dst = Ks + i * KS_LD + (j4 >> 5) * (QW + 1) + (j4 & 31);
+      float* dst = Ks + i * KS_LD + (j4 >> 5) * KQ + (j4 & 31);
       dst[0] = (j4 + 0 >= i) ? v.x : 0.f;
       dst[1] = (j4 + 1 >= i) ? v.y : 0.f;
       dst[2] = (j4 + 2 >= i) ? v.z : 0.f;
@@ -105,11 +107,11 @@ __global__ void __launch_bounds__(QROWS * QT) block_solve_kernel(
         v = (j >= i) ? k[static_cast<int64_t>(b0 + i) * d_in + b0 + j] : 0.f;
       else
         v = (i == j) ? 1.f : 0.f;
-      Ks[i * KS_LD + (j >> 5) * (QW + 1) + (j & 31)] = v;
+      Ks[i * KS_LD + (j >> 5) * KQ + (j & 31)] = v;
     }
   }
   __syncthreads();
-  if (tid < QB) Rd[tid] = 1.f / Ks[tid * KS_LD + (tid >> 5) * (QW + 1) + (tid & 31)];
+  if (tid < QB) Rd[tid] = 1.f / Ks[tid * KS_LD + (tid >> 5) * KQ + (tid & 31)];
   __syncthreads();
 
   // this thread's 32 columns of its row
@@ -148,11 +150,28 @@ __global__ void __launch_bounds__(QROWS * QT) block_solve_kernel(
       packed[lp / 4] |= (static_cast<uint32_t>(code) & 0xFFu) << (8 * (lp % 4));
     }
     e = __shfl_sync(0xffffffffu, e, (lane & ~(QT - 1)) | qo);
-    if (q >= qo) {
-      const float* kr = Ks + p * KS_LD + q * (QW + 1);
+    // quarters right of the owner update all 32 columns; the owner only those right of p
+    // (a compile-time range); quarters to the left have nothing right of p
+    const float4* kr = reinterpret_cast<const float4*>(Ks + p * KS_LD + q * KQ);
+    if (q > qo) {
 #pragma unroll
-      for (int j = 0; j < QW; ++j)
-        if (QW * q + j > p) w[j] = fmaf(-e, kr[j], w[j]);
+      for (int j4 = 0; j4 < QW / 4; ++j4) {
+        const float4 kv = kr[j4];
+        w[4 * j4] = fmaf(-e, kv.x, w[4 * j4]);
+        w[4 * j4 + 1] = fmaf(-e, kv.y, w[4 * j4 + 1]);
+        w[4 * j4 + 2] = fmaf(-e, kv.z, w[4 * j4 + 2]);
+        w[4 * j4 + 3] = fmaf(-e, kv.w, w[4 * j4 + 3]);
+      }
+    } else if (q == qo) {
+#pragma unroll
+      for (int j4 = 0; j4 < QW / 4; ++j4) {
+        if (4 * j4 + 3 <= lp) continue;       // compile time
+        const float4 kv = kr[j4];
+        if (4 * j4 > lp) w[4 * j4] = fmaf(-e, kv.x, w[4 * j4]);
+        if (4 * j4 + 1 > lp) w[4 * j4 + 1] = fmaf(-e, kv.y, w[4 * j4 + 1]);
+        if (4 * j4 + 2 > lp) w[4 * j4 + 2] = fmaf(-e, kv.z, w[4 * j4 + 2]);
+        if (4 * j4 + 3 > lp) w[4 * j4 + 3] = fmaf(-e, kv.w, w[4 * j4 + 3]);
+      }
     }
   }
 
