@@ -236,10 +236,15 @@ class Block:
                 self.acc_events.append((e0, e1, self.n * d * (d + 1)))
         inv_n = 1.0 / self.n
         if self.streams is None:
+            # the per-sublayer phases (BiIP; inverse factor + column solve) run side by side on
+            # one stream per sublayer, each phase captured once as a CUDA graph and replayed
             self.streams = P.SublayerStreams(len(wl.sublayers), self.dev)
-        res = self.streams.biip([(self.w[s.name], self.hx[s.x_stream], self.hg[s.name], None,
-                                  inv_n, self.si[s.name], self.so[s.name], K.BIIP_FULL)
-                                 for s in wl.sublayers])
+            jobs = [(self.w[s.name], self.hx[s.x_stream], self.hg[s.name], None, inv_n,
+                     self.si[s.name], self.so[s.name], K.BIIP_FULL) for s in wl.sublayers]
+            self.biip_phase = P.CapturedPhase(lambda: self.streams.biip(jobs))
+            self.solve_phases = {}
+            self.solve_res = None
+        res = self.biip_phase()
         for s, r in zip(wl.sublayers, res):
             self.results[s.name] = r
         tr = torch.stack([self.results[s.name].tr for s in wl.sublayers]).cpu()
@@ -248,7 +253,15 @@ class Block:
         _, self.bits = K.kronq_score_allocate(tr[:, 0].tolist(), tr[:, 1].tolist(),
                                               [s.d_out * s.d_in for s in wl.sublayers], choices,
                                               avg)
-        self.streams.solve([self.results[s.name] for s in wl.sublayers], self.bits, 0.01)
+        if self.solve_res is not res:       # a new BiIP output set: new solve graphs
+            self.solve_res = res
+            self.solve_phases = {}
+        key = tuple(self.bits)
+        if key not in self.solve_phases:
+            bits = list(self.bits)
+            self.solve_phases[key] = P.CapturedPhase(
+                lambda: self.streams.solve(res, bits, 0.01))
+        self.solve_phases[key]()
 
 
 def run_gpu(args):
@@ -292,7 +305,7 @@ def run_gpu(args):
 
     clocks = ClockSampler(local)
     clocks.start()
-    launches0 = K.kronq_launch_count()
+    launches0 = K.kronq_launch_count() + P.replayed_launches()
     barrier()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
@@ -302,7 +315,7 @@ def run_gpu(args):
     t_end.record()
     barrier()
     clk = clocks.stop()
-    launches = K.kronq_launch_count() - launches0
+    launches = K.kronq_launch_count() + P.replayed_launches() - launches0
     elapsed = t_start.elapsed_time(t_end) / 1e3
     acc_ms = [a.elapsed_time(b) for a, b, _ in blk.acc_events]
     acc_flops = [f for _, _, f in blk.acc_events]

@@ -120,22 +120,34 @@ __global__ void __launch_bounds__(LEAF_THREADS, 1) leaf_kernel(float* __restrict
   extern __shared__ __align__(16) float leaf_smem[];
   float* S = leaf_smem;                 // NB x LDS: S (upper), then K_ii in the diagonal blocks
   float* R = S + NB * LDS;              // NB x LDS: R off-diagonal blocks (upper), K^T (lower)
-  float* T = R + NB * LDS;              // (NB - PW) x LDT: one block row of sum R_il K_lj, transposed
+  float* T = R + NB * LDS;              // (NB - PW) x LDT: one block row of sum R_il K_lj,
+                                        // transposed (the panel warp's scratch before that)
   int* bad = reinterpret_cast<int*>(T + (NB - PW) * LDT);
   if (*info >= 0) return;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int ly = lane >> 3, lx = lane & 7;
   constexpr int NWARPS = LEAF_THREADS / 32;
 
-  for (int e = tid; e < NB * NB; e += LEAF_THREADS) {
-    const int r = e / NB, c = e % NB;
-    float v;
-    if (r < nb && c < nb)
-      v = c >= r ? a[r * ld + c] : 0.f;
-    else
-      v = r == c ? 1.f : 0.f;
-    S[r * LDS + c] = v;
-    if (r > c && (r >> 5) != (c >> 5) && r < nb && c < nb) a[r * ld + c] = 0.f;
+  // the loads of a batch in flight together, then their stores (the zero fill goes through the
+  // same pointer, so it must not sit between loads)
+  constexpr int PER = NB * NB / LEAF_THREADS, BATCH = 16;
+#pragma unroll 1
+  for (int u0 = 0; u0 < PER; u0 += BATCH) {
+    float v[BATCH];
+#pragma unroll
+    for (int u = 0; u < BATCH; ++u) {
+      const int r = (tid >> 7) + (u0 + u) * (LEAF_THREADS / NB), c = tid & (NB - 1);
+      if (r < nb && c < nb)
+        v[u] = c >= r ? a[r * ld + c] : 0.f;
+      else
+        v[u] = r == c ? 1.f : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < BATCH; ++u) {
+      const int r = (tid >> 7) + (u0 + u) * (LEAF_THREADS / NB), c = tid & (NB - 1);
+      S[r * LDS + c] = v[u];
+      if (r > c && (r >> 5) != (c >> 5) && r < nb && c < nb) a[r * ld + c] = 0.f;
+    }
   }
   if (tid == 0) *bad = -1;
   __syncthreads();
@@ -143,7 +155,11 @@ __global__ void __launch_bounds__(LEAF_THREADS, 1) leaf_kernel(float* __restrict
   for (int p0 = NB - PW; p0 >= 0; p0 -= PW) {
     if (warp == 0) {
       // lane k holds column k of the symmetric panel block (both triangles, so that the
-      // multiplier S_ck of lane k is a register with a compile-time index)
+      // multiplier S_ck of lane k is a register with a compile-time index). The column that
+      // drives a step is published in shared memory by its lane and read back as broadcasts;
+      // T is free until the off-diagonal blocks of K are formed.
+      float* pub = T;                  // PW x LDT: published columns of the factor step
+      float* rt = T + PW * LDT;        // PW x LDT: R_PP^T, 1/R_ii in the padding column PW
       float s[PW];
 #pragma unroll
       for (int i = 0; i < PW; ++i) {
@@ -154,42 +170,66 @@ __global__ void __launch_bounds__(LEAF_THREADS, 1) leaf_kernel(float* __restrict
       int fail = -1;
 #pragma unroll
       for (int c = PW - 1; c >= 0; --c) {
-        const float piv = __shfl_sync(0xffffffffu, s[c], c);
-        if (!(piv > 0.f) || !isfinite(piv)) {   // uniform: every lane has the same pivot
-          fail = c;
-          break;
-        }
-        mypiv = lane == c ? piv : mypiv;
-        const float f = s[c] * __frcp_rn(piv);
+        if (lane == c) {
 #pragma unroll
-        for (int i = c - 1; i >= 0; --i) {
-          const float v = __shfl_sync(0xffffffffu, s[i], c);
-          if (lane < c) s[i] = fmaf(-v, f, s[i]);
+          for (int i4 = 0; i4 <= c / 4; ++i4)
+            *reinterpret_cast<float4*>(pub + c * LDT + 4 * i4) =
+                make_float4(s[4 * i4], s[4 * i4 + 1], s[4 * i4 + 2], s[4 * i4 + 3]);
+        }
+        __syncwarp();
+        const float piv = pub[c * LDT + c];
+        if (fail < 0 && !(piv > 0.f && isfinite(piv))) fail = c;   // the same on every lane
+        mypiv = lane == c ? piv : mypiv;
+        const float rp = rsqrtf(piv);
+        // finished columns (lanes >= c) take a zero multiplier and stay as they are
+        const float f = lane < c ? s[c] * (rp * rp) : 0.f;
+#pragma unroll
+        for (int i4 = 0; i4 < (c + 3) / 4; ++i4) {
+          const float4 v = *reinterpret_cast<const float4*>(pub + c * LDT + 4 * i4);
+          if (4 * i4 < c) s[4 * i4] = fmaf(-v.x, f, s[4 * i4]);
+          if (4 * i4 + 1 < c) s[4 * i4 + 1] = fmaf(-v.y, f, s[4 * i4 + 1]);
+          if (4 * i4 + 2 < c) s[4 * i4 + 2] = fmaf(-v.z, f, s[4 * i4 + 2]);
+          if (4 * i4 + 3 < c) s[4 * i4 + 3] = fmaf(-v.w, f, s[4 * i4 + 3]);
         }
       }
       if (fail >= 0) {
         if (lane == 0) *bad = p0 + fail;
       } else {
-        // lane k: column k of R_PP, then column k of K_PP = R_PP^-1 by right-looking substitution
+        // lane k: column k of R_PP (row k of R_PP^T), then column k of K_PP = R_PP^-1 by
+        // right-looking substitution, reading column i of R_PP as broadcasts
         const float rs = rsqrtf(mypiv), sq = sqrtf(mypiv);
 #pragma unroll
         for (int i = 0; i < PW; ++i) s[i] = i < lane ? s[i] * rs : (i == lane ? sq : 0.f);
+#pragma unroll
+        for (int i4 = 0; i4 < PW / 4; ++i4)
+          *reinterpret_cast<float4*>(rt + lane * LDT + 4 * i4) =
+              make_float4(s[4 * i4], s[4 * i4 + 1], s[4 * i4 + 2], s[4 * i4 + 3]);
+        rt[lane * LDT + PW] = rs;      // 1 / R_kk
+        __syncwarp();
         float k[PW];
 #pragma unroll
         for (int i = 0; i < PW; ++i) k[i] = 0.f;
 #pragma unroll
         for (int i = PW - 1; i >= 0; --i) {
-          const float rii = __shfl_sync(0xffffffffu, s[i], i);
-          k[i] = ((lane == i ? 1.f : 0.f) - k[i]) * __frcp_rn(rii);
+          k[i] = ((lane == i ? 1.f : 0.f) - k[i]) * rt[i * LDT + PW];
 #pragma unroll
-          for (int r = 0; r < i; ++r) k[r] = fmaf(__shfl_sync(0xffffffffu, s[r], i), k[i], k[r]);
+          for (int r4 = 0; r4 < (i + 3) / 4; ++r4) {
+            const float4 v = *reinterpret_cast<const float4*>(rt + i * LDT + 4 * r4);
+            if (4 * r4 < i) k[4 * r4] = fmaf(v.x, k[i], k[4 * r4]);
+            if (4 * r4 + 1 < i) k[4 * r4 + 1] = fmaf(v.y, k[i], k[4 * r4 + 1]);
+            if (4 * r4 + 2 < i) k[4 * r4 + 2] = fmaf(v.z, k[i], k[4 * r4 + 2]);
+            if (4 * r4 + 3 < i) k[4 * r4 + 3] = fmaf(v.w, k[i], k[4 * r4 + 3]);
+          }
         }
 #pragma unroll
         for (int i = 0; i < PW; ++i) {
           S[(p0 + i) * LDS + p0 + lane] = k[i];        // K_PP
-          R[(p0 + lane) * LDS + p0 + i] = k[i];        // K_PP^T
           if (p0 + i < nb && p0 + lane < nb) a[(p0 + i) * ld + p0 + lane] = k[i];
         }
+#pragma unroll
+        for (int i4 = 0; i4 < PW / 4; ++i4)            // K_PP^T
+          *reinterpret_cast<float4*>(R + (p0 + lane) * LDS + p0 + 4 * i4) =
+              make_float4(k[4 * i4], k[4 * i4 + 1], k[4 * i4 + 2], k[4 * i4 + 3]);
       }
     }
     __syncthreads();

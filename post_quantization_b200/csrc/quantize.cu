@@ -8,9 +8,9 @@
 // so its total contribution to column j, sum_{p<j} W_:,p P_p,j, is known in advance: the solve
 // is GPTQ on W~ = W + W P, which this file forms up front (fp32-accurate tensor-core GEMMs).
 //
-// Solve: 128-column blocks. Inside a block every output row is independent given K; four
-// threads share a row and walk the block's columns in order (quantize, error, update the
-// remaining columns of the block). After the block the rest of every row is updated lazily with
+// Solve: 128-column blocks. Inside a block every output row is independent given K; one lane
+// per row walks the block's columns in order (quantize, error, update the remaining columns of
+// the block), the four warps of a CTA each holding a quarter of the block's columns. After the block the rest of every row is updated lazily with
 // one GEMM: W~[:, e:] -= Delta_blk K[blk, e:].
 #include <cuda_bf16.h>
 
@@ -25,10 +25,10 @@ namespace {
 
 constexpr int QB = 128;        // column block
 constexpr int QROWS = 32;      // rows per CTA in the block solve
-constexpr int QT = 4;          // threads per row
+constexpr int QT = 4;          // warps per CTA: one column quarter each
 constexpr int QW = QB / QT;    // columns per thread
-constexpr int KQ = QW + 4;     // padded quarter row (16-byte aligned, quarters 4 banks apart)
-constexpr int KS_LD = QT * KQ; // row of the K block in shared memory
+constexpr int KS_LD = QB + 4;  // row of the K block in shared memory (16-byte aligned)
+constexpr int E_LD = QB + 1;   // row of the error block (odd: one bank per lane)
 
 // Per-row grid from W (before the solve), all decisions in fp32:
 // scale = (hi - lo) / (2^b - 1) (1 if hi == lo), zero = rint(-lo / scale).
@@ -64,12 +64,13 @@ __global__ void striu_kernel(float* __restrict__ m, int d) {
     m[static_cast<int64_t>(i) * d + j] = 0.f;
 }
 
-// One 128-column block of the solve for QROWS rows. Four threads share a row, each holding 32
-// of the block's columns in registers. At column p the thread that owns it quantizes it and
-// hands the scaled error to the other three (a shuffle within the group of four), and every
-// thread updates its own columns to the right of p. The K block sits in shared memory in
-// 36-float quarters: 16-byte aligned for vector reads, and the four threads of a row read from
-// different banks.
+// One 128-column block of the solve for QROWS rows: lane l of every warp owns row
+// blockIdx.x * QROWS + l, and warp q owns the block's column quarter [32q, 32q + 32) of it, in
+// registers. Quarter by quarter, its warp walks the 32 columns in order (quantize, scaled error,
+// update its own columns to the right) with no exchange, parks the errors in shared memory, and
+// after one barrier every later quarter subtracts those 32 errors times the matching K rows.
+// K rows are read as broadcasts (every lane of a warp reads the same row), so the solve is bound
+// by the per-column dependency chain, not by shared memory.
 //   w_hat  d_out x d_in running weights (in: current values, out: dequantized for the block)
 //   delta  d_out x QB errors scaled by 1/K_pp, written as three bf16 pieces (the operand of
 //          the lazy trailing update on the tensor cores)
@@ -78,13 +79,14 @@ __global__ void __launch_bounds__(QROWS * QT) block_solve_kernel(
     const float* __restrict__ scale, const float* __restrict__ zero, float maxq,
     uint8_t* __restrict__ codes, uint16_t* __restrict__ delta0, uint16_t* __restrict__ delta1,
     uint16_t* __restrict__ delta2) {
-  extern __shared__ float sm[];
-  float* Ks = sm;                      // QB rows x KS_LD
-  float* Rd = sm + QB * KS_LD;         // QB reciprocals of K's diagonal
+  extern __shared__ __align__(16) float sm[];
+  float* Ks = sm;                      // QB x KS_LD: the K block
+  float* E = Ks + QB * KS_LD;          // QROWS x E_LD: scaled errors of the block
+  float* Rd = E + QROWS * E_LD;        // QB reciprocals of K's diagonal
   const int tid = threadIdx.x;
   const int lane = tid & 31;
-  const int q = tid % QT;              // column quarter of this thread
-  const int row = blockIdx.x * QROWS + tid / QT;
+  const int q = tid >> 5;              // column quarter of this warp
+  const int row = blockIdx.x * QROWS + lane;
   const bool active = row < d_out;
 
   // K block (rows/cols beyond bw become identity so that padding never feeds back)
@@ -93,11 +95,9 @@ __global__ void __launch_bounds__(QROWS * QT) block_solve_kernel(
     for (int e = tid; e < QB * QB / 4; e += blockDim.x) {
       const int i = e / (QB / 4), j4 = (e % (QB / 4)) * 4;
       const float4 v = *reinterpret_cast<const float4*>(k + static_cast<int64_t>(b0 + i) * d_in + b0 + j4);
-      float* dst = Ks + i * KS_LD + (j4 >> 5) * KQ + (j4 & 31);
-      dst[0] = (j4 + 0 >= i) ? v.x : 0.f;
-      dst[1] = (j4 + 1 >= i) ? v.y : 0.f;
-      dst[2] = (j4 + 2 >= i) ? v.z : 0.f;
-      dst[3] = (j4 + 3 >= i) ? v.w : 0.f;
+      *reinterpret_cast<float4*>(Ks + i * KS_LD + j4) =
+          make_float4(j4 >= i ? v.x : 0.f, j4 + 1 >= i ? v.y : 0.f, j4 + 2 >= i ? v.z : 0.f,
+                      j4 + 3 >= i ? v.w : 0.f);
     }
   } else {
     for (int e = tid; e < QB * QB; e += blockDim.x) {
@@ -107,14 +107,13 @@ __global__ void __launch_bounds__(QROWS * QT) block_solve_kernel(
         v = (j >= i) ? k[static_cast<int64_t>(b0 + i) * d_in + b0 + j] : 0.f;
       else
         v = (i == j) ? 1.f : 0.f;
-      Ks[i * KS_LD + (j >> 5) * KQ + (j & 31)] = v;
+      Ks[i * KS_LD + j] = v;
     }
   }
   __syncthreads();
-  if (tid < QB) Rd[tid] = 1.f / Ks[tid * KS_LD + (tid >> 5) * KQ + (tid & 31)];
-  __syncthreads();
+  if (tid < QB) Rd[tid] = 1.f / Ks[tid * KS_LD + tid];
 
-  // this thread's 32 columns of its row
+  // this lane's 32 columns of its row
   float w[QW];
   float* wrow = w_hat + static_cast<int64_t>(row) * d_in + b0 + QW * q;
   const bool wvec = active && bw == QB && ((reinterpret_cast<uintptr_t>(wrow) & 15u) == 0);
@@ -134,62 +133,87 @@ __global__ void __launch_bounds__(QROWS * QT) block_solve_kernel(
   uint32_t packed[QW / 4];
 #pragma unroll
   for (int j = 0; j < QW / 4; ++j) packed[j] = 0u;
+  float* erow = E + lane * E_LD;
+  __syncthreads();   // Rd
 
-#pragma unroll
-  for (int p = 0; p < QB; ++p) {
-    const int qo = p / QW, lp = p % QW;   // owner quarter and its local column (compile time)
-    float e = 0.f;
+  for (int qo = 0; qo < QT; ++qo) {
     if (q == qo) {
-      const float t = __fdiv_rn(w[lp], sc);
-      float code = __fadd_rn(rintf(t), zr);
-      code = fminf(fmaxf(code, 0.f), maxq);
-      const float dq = __fmul_rn(sc, __fsub_rn(code, zr));
-      e = __fsub_rn(w[lp], dq) * Rd[p];
-      w[lp] = dq;
-      err[lp] = e;
-      packed[lp / 4] |= (static_cast<uint32_t>(code) & 0xFFu) << (8 * (lp % 4));
-    }
-    e = __shfl_sync(0xffffffffu, e, (lane & ~(QT - 1)) | qo);
-    // quarters right of the owner update all 32 columns; the owner only those right of p
-    // (a compile-time range); quarters to the left have nothing right of p
-    const float4* kr = reinterpret_cast<const float4*>(Ks + p * KS_LD + q * KQ);
-    if (q > qo) {
 #pragma unroll
-      for (int j4 = 0; j4 < QW / 4; ++j4) {
-        const float4 kv = kr[j4];
-        w[4 * j4] = fmaf(-e, kv.x, w[4 * j4]);
-        w[4 * j4 + 1] = fmaf(-e, kv.y, w[4 * j4 + 1]);
-        w[4 * j4 + 2] = fmaf(-e, kv.z, w[4 * j4 + 2]);
-        w[4 * j4 + 3] = fmaf(-e, kv.w, w[4 * j4 + 3]);
+      for (int lp = 0; lp < QW; ++lp) {
+        const int p = QW * qo + lp;
+        const float t = __fdiv_rn(w[lp], sc);
+        float code = __fadd_rn(rintf(t), zr);
+        code = fminf(fmaxf(code, 0.f), maxq);
+        const float dq = __fmul_rn(sc, __fsub_rn(code, zr));
+        const float e = __fsub_rn(w[lp], dq) * Rd[p];
+        w[lp] = dq;
+        err[lp] = e;
+        erow[p] = e;
+        packed[lp / 4] |= (static_cast<uint32_t>(code) & 0xFFu) << (8 * (lp % 4));
+        // own columns right of lp (a compile-time range)
+        const float4* kr = reinterpret_cast<const float4*>(Ks + p * KS_LD + QW * qo);
+#pragma unroll
+        for (int j4 = 0; j4 < QW / 4; ++j4) {
+          if (4 * j4 + 3 <= lp) continue;
+          const float4 kv = kr[j4];
+          if (4 * j4 > lp) w[4 * j4] = fmaf(-e, kv.x, w[4 * j4]);
+          if (4 * j4 + 1 > lp) w[4 * j4 + 1] = fmaf(-e, kv.y, w[4 * j4 + 1]);
+          if (4 * j4 + 2 > lp) w[4 * j4 + 2] = fmaf(-e, kv.z, w[4 * j4 + 2]);
+          if (4 * j4 + 3 > lp) w[4 * j4 + 3] = fmaf(-e, kv.w, w[4 * j4 + 3]);
+        }
       }
-    } else if (q == qo) {
+    }
+    __syncthreads();
+    if (q > qo) {
+      // the finished quarter's 32 errors, applied to this warp's columns
+#pragma unroll 4
+      for (int p = QW * qo; p < QW * qo + QW; ++p) {
+        const float e = erow[p];
+        const float4* kr = reinterpret_cast<const float4*>(Ks + p * KS_LD + QW * q);
 #pragma unroll
-      for (int j4 = 0; j4 < QW / 4; ++j4) {
-        if (4 * j4 + 3 <= lp) continue;       // compile time
-        const float4 kv = kr[j4];
-        if (4 * j4 > lp) w[4 * j4] = fmaf(-e, kv.x, w[4 * j4]);
-        if (4 * j4 + 1 > lp) w[4 * j4 + 1] = fmaf(-e, kv.y, w[4 * j4 + 1]);
-        if (4 * j4 + 2 > lp) w[4 * j4 + 2] = fmaf(-e, kv.z, w[4 * j4 + 2]);
-        if (4 * j4 + 3 > lp) w[4 * j4 + 3] = fmaf(-e, kv.w, w[4 * j4 + 3]);
+        for (int j4 = 0; j4 < QW / 4; ++j4) {
+          const float4 kv = kr[j4];
+          w[4 * j4] = fmaf(-e, kv.x, w[4 * j4]);
+          w[4 * j4 + 1] = fmaf(-e, kv.y, w[4 * j4 + 1]);
+          w[4 * j4 + 2] = fmaf(-e, kv.z, w[4 * j4 + 2]);
+          w[4 * j4 + 3] = fmaf(-e, kv.w, w[4 * j4 + 3]);
+        }
       }
     }
   }
 
   if (active) {
+    if (wvec) {
 #pragma unroll
-    for (int j = 0; j < QW; ++j) {
-      const int c = QW * q + j;
-      if (c < bw) wrow[j] = w[j];
-      // the error, split into three bf16 pieces for the tensor-core trailing update
-      const float dv = c < bw ? err[j] : 0.f;
-      const __nv_bfloat16 p0 = __float2bfloat16_rn(dv);
-      const float r1 = dv - __bfloat162float(p0);
-      const __nv_bfloat16 p1 = __float2bfloat16_rn(r1);
-      const __nv_bfloat16 p2 = __float2bfloat16_rn(r1 - __bfloat162float(p1));
-      const int64_t o = static_cast<int64_t>(row) * QB + c;
-      delta0[o] = __bfloat16_as_ushort(p0);
-      delta1[o] = __bfloat16_as_ushort(p1);
-      delta2[o] = __bfloat16_as_ushort(p2);
+      for (int j = 0; j < QW; j += 4)
+        *reinterpret_cast<float4*>(wrow + j) = make_float4(w[j], w[j + 1], w[j + 2], w[j + 3]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < QW; ++j)
+        if (QW * q + j < bw) wrow[j] = w[j];
+    }
+    // the errors, split into three bf16 pieces for the tensor-core trailing update
+    // (8 columns per 16-byte store; the row's 32 columns start on a 64-byte boundary)
+    const int64_t o = static_cast<int64_t>(row) * QB + QW * q;
+#pragma unroll
+    for (int j8 = 0; j8 < QW; j8 += 8) {
+      uint32_t h0[4], h1[4], h2[4];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float dv = QW * q + j8 + u < bw ? err[j8 + u] : 0.f;
+        const __nv_bfloat16 p0 = __float2bfloat16_rn(dv);
+        const float r1 = dv - __bfloat162float(p0);
+        const __nv_bfloat16 p1 = __float2bfloat16_rn(r1);
+        const __nv_bfloat16 p2 = __float2bfloat16_rn(r1 - __bfloat162float(p1));
+        const int sh = 16 * (u & 1);
+        if ((u & 1) == 0) { h0[u >> 1] = 0u; h1[u >> 1] = 0u; h2[u >> 1] = 0u; }
+        h0[u >> 1] |= static_cast<uint32_t>(__bfloat16_as_ushort(p0)) << sh;
+        h1[u >> 1] |= static_cast<uint32_t>(__bfloat16_as_ushort(p1)) << sh;
+        h2[u >> 1] |= static_cast<uint32_t>(__bfloat16_as_ushort(p2)) << sh;
+      }
+      *reinterpret_cast<uint4*>(delta0 + o + j8) = make_uint4(h0[0], h0[1], h0[2], h0[3]);
+      *reinterpret_cast<uint4*>(delta1 + o + j8) = make_uint4(h1[0], h1[1], h1[2], h1[3]);
+      *reinterpret_cast<uint4*>(delta2 + o + j8) = make_uint4(h2[0], h2[1], h2[2], h2[3]);
     }
     uint8_t* cr = codes + static_cast<int64_t>(row) * d_in + b0 + QW * q;
     if (bw == QB && (reinterpret_cast<uintptr_t>(cr) & 15u) == 0) {
@@ -276,7 +300,7 @@ kronq_status run_quantize(const float* w, const float* k, const float* dxx, int 
   }
 
   static bool attr = false;
-  const size_t smem = sizeof(float) * (QB * KS_LD + QB);
+  const size_t smem = sizeof(float) * (QB * KS_LD + QROWS * E_LD + QB);
   if (!attr) {
     KQ_CUDA_TRY(cudaFuncSetAttribute(block_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)smem));
