@@ -10,7 +10,10 @@
 //   norms   one read of W: |W_:,j|^2 and |W_i,:|^2 (fp64 sums)
 //   scales  S_X, S_G, the per-row / per-column factors of the passes below, traces
 //   rows    for every row: multiply by row and column factors, FWHT along the row in b-blocks
-//   cols    for every b-row block of every column: FWHT along the column (in place)
+//   cols    for every b-row block of every column: FWHT along the column (in place; one pass
+//           for b <= 256, two for larger b)
+// The passes work in registers (16-point butterflies per thread) with a shared-memory exchange
+// between groups of four stages; b outside [16, 16384] takes plain shared-memory kernels.
 // W' = rows(W) then cols; H_X and dXX^T = rows then cols (in place); H_G likewise if asked.
 #include <cuda_bf16.h>
 
@@ -193,6 +196,170 @@ __global__ void __launch_bounds__(256) fwht_cols_kernel(float* m, int64_t rows, 
   }
 }
 
+// ---- register-radix passes (16 <= b <= 16384) ----
+//
+// Row pass: one CTA per chunk of C = max(b, 4096) consecutive elements (whole b-blocks),
+// C / 16 threads. Round 0 takes 16 consecutive elements per thread straight from global
+// memory and transforms index bits 0-3 in registers; round R takes the 16 elements whose index
+// differs in bits 4R..4R+3 (stride 16^R) from shared memory. The last round writes to global
+// memory, coalesced. log2(b) stages cost ceil(log2(b) / 4) - 1 shared-memory round trips.
+//
+// Column pass: a P-point transform along rows r_base + rs * j (j < P) of a tile of 32
+// columns, P in [16, 256]. b <= 256 is one pass (P = b, rs = 1); larger b is two passes,
+// 64-point over consecutive rows, then (b / 64)-point at row stride 64
+// (H_b = (H_{b/64} (x) I_64)(I_{b/64} (x) H_64)). Every global access is a 128-byte row segment.
+
+// 16-point Walsh-Hadamard butterflies on the low nbits bits of the register index.
+__device__ __forceinline__ void fwht16(float (&x)[16], int nbits) {
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    if (h < nbits) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        if (j & (1 << h)) continue;
+        const float a = x[j], b = x[j | (1 << h)];
+        x[j] = a + b;
+        x[j | (1 << h)] = a - b;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ int pad16(int i) { return i + (i >> 4); }
+
+__device__ __forceinline__ void load16(const float* p, bool vec, float (&x)[16]) {
+  if (vec) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 v = reinterpret_cast<const float4*>(p)[q];
+      x[4 * q] = v.x; x[4 * q + 1] = v.y; x[4 * q + 2] = v.z; x[4 * q + 3] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 16; ++k) x[k] = p[k];
+  }
+}
+
+__device__ __forceinline__ void load16(const __nv_bfloat16* p, bool vec, float (&x)[16]) {
+  if (vec) {
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const uint4 v = reinterpret_cast<const uint4*>(p)[q];
+      const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        x[8 * q + 2 * e] = __uint_as_float(u[e] << 16);
+        x[8 * q + 2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 16; ++k) x[k] = __bfloat162float(p[k]);
+  }
+}
+
+// src may equal dst (every element is read before the chunk's first write).
+template <typename T>
+__global__ void __launch_bounds__(1024) fwht_rows_reg_kernel(
+    const T* src, float* dst, int64_t total, int64_t cols, const float* __restrict__ row_f,
+    const float* __restrict__ col_f, float scalar, int log2b, int chunk, float out_scale,
+    int vec) {
+  extern __shared__ float sb[];
+  const int t = threadIdx.x;
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * chunk;
+  const int rounds = (log2b + 3) >> 2;
+  float x[16];
+  const int64_t f0 = base + 16 * t;
+  if (f0 < total) {   // total is a multiple of b >= 16, so a group is all in or all out
+    load16(src + f0, vec != 0, x);
+    const int64_t r = f0 / cols;
+    const int64_t c0 = f0 - r * cols;
+    const float rf = row_f ? scalar * row_f[r] : scalar;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) x[k] *= col_f ? rf * col_f[c0 + k] : rf;
+  } else {
+#pragma unroll
+    for (int k = 0; k < 16; ++k) x[k] = 0.f;
+  }
+  fwht16(x, log2b < 4 ? log2b : 4);
+  if (rounds == 1) {
+    if (f0 < total) {
+#pragma unroll
+      for (int k = 0; k < 16; ++k) dst[f0 + k] = x[k] * out_scale;
+    }
+    return;
+  }
+#pragma unroll
+  for (int k = 0; k < 16; ++k) sb[pad16(16 * t + k)] = x[k];
+  for (int R = 1; R < rounds; ++R) {
+    __syncthreads();
+    const int sh = 4 * R, s = 1 << sh;
+    const int lo = (t & (s - 1)) + ((t >> sh) << (sh + 4));
+#pragma unroll
+    for (int k = 0; k < 16; ++k) x[k] = sb[pad16(lo + s * k)];
+    const int nbits = log2b - sh < 4 ? log2b - sh : 4;
+    fwht16(x, nbits);
+    if (R == rounds - 1) {
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const int64_t f = base + lo + static_cast<int64_t>(s) * k;
+        if (f < total) dst[f] = x[k] * out_scale;
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < 16; ++k) sb[pad16(lo + s * k)] = x[k];
+    }
+  }
+}
+
+// P-point transform along rows r_base + rs * j of 32 columns, in place; 2P threads.
+constexpr int kColTile = 32;
+__global__ void __launch_bounds__(512) fwht_cols_reg_kernel(float* m, int64_t rows, int64_t cols,
+                                                            int log2p, int rs, float out_scale) {
+  extern __shared__ float sb[];
+  const int P = 1 << log2p;
+  const int t = threadIdx.x;
+  const int c = t & (kColTile - 1);
+  const int64_t col = static_cast<int64_t>(blockIdx.x) * kColTile + c;
+  const bool cin = col < cols;
+  const int y = blockIdx.y;
+  const int64_t r_base = static_cast<int64_t>(y / rs) * P * rs + (y % rs);
+  constexpr int LDT = kColTile + 1;
+  float x[16];
+  {
+    const int jg = t / kColTile;   // round 0: rows 16 jg .. 16 jg + 15
+#pragma unroll
+    for (int k = 0; k < 16; ++k)
+      x[k] = cin ? m[(r_base + static_cast<int64_t>(rs) * (16 * jg + k)) * cols + col] : 0.f;
+    fwht16(x, 4);
+    if (log2p == 4) {
+      if (cin) {
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+          m[(r_base + static_cast<int64_t>(rs) * (16 * jg + k)) * cols + col] = x[k] * out_scale;
+      }
+      return;
+    }
+#pragma unroll
+    for (int k = 0; k < 16; ++k) sb[(16 * jg + k) * LDT + c] = x[k];
+  }
+  __syncthreads();
+  // round 1: bits 4.. of j; groups (c, jl), jl in [0, 16), P / 16 elements each
+  const int M = P >> 4, per = 256 / P, q = t / kColTile;
+  for (int u = 0; u < per; ++u) {
+    const int jl = q * per + u;
+#pragma unroll
+    for (int mm = 0; mm < 16; ++mm) x[mm] = mm < M ? sb[(jl + 16 * mm) * LDT + c] : 0.f;
+    fwht16(x, log2p - 4);
+    if (cin) {
+#pragma unroll
+      for (int mm = 0; mm < 16; ++mm)
+        if (mm < M)
+          m[(r_base + static_cast<int64_t>(rs) * (jl + 16 * mm)) * cols + col] = x[mm] * out_scale;
+    }
+  }
+}
+
 int ilog2_pow2(int b) {
   int l = 0;
   while ((1 << l) < b) ++l;
@@ -207,8 +374,20 @@ kronq_status row_pass(const T* src, float* dst, int64_t rows, int64_t cols, cons
   const int chunk = b > 4096 ? b : 4096;
   const int64_t total = rows * cols;
   const int64_t blocks = (total + chunk - 1) / chunk;
-  const size_t smem = static_cast<size_t>(chunk) * sizeof(float);
   const float out_scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(b)));
+  if (b >= 16 && b <= 16384) {
+    const int threads = chunk / 16;
+    const size_t smem = static_cast<size_t>(chunk + chunk / 16) * sizeof(float);
+    if (smem > 48 * 1024)
+      KQ_CUDA_TRY(cudaFuncSetAttribute(fwht_rows_reg_kernel<T>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    const int vec = (reinterpret_cast<uintptr_t>(src) & 15u) == 0 &&
+                    (reinterpret_cast<uintptr_t>(dst) & 15u) == 0;
+    fwht_rows_reg_kernel<T><<<static_cast<unsigned>(blocks), threads, smem, stream>>>(
+        src, dst, total, cols, row_f, col_f, scalar, ilog2_pow2(b), chunk, out_scale, vec);
+    return check_launch("fwht_rows_reg_kernel");
+  }
+  const size_t smem = static_cast<size_t>(chunk) * sizeof(float);
   if (smem > 48 * 1024)
     KQ_CUDA_TRY(cudaFuncSetAttribute(fwht_rows_kernel<T>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
@@ -217,13 +396,31 @@ kronq_status row_pass(const T* src, float* dst, int64_t rows, int64_t cols, cons
   return check_launch("fwht_rows_kernel");
 }
 
+// One P-point column pass (P in [16, 256]) at row stride rs.
+kronq_status col_pass_reg(float* m, int64_t rows, int64_t cols, int log2p, int rs, float out_scale,
+                          cudaStream_t stream) {
+  const int P = 1 << log2p;
+  const size_t smem = static_cast<size_t>(P) * (kColTile + 1) * sizeof(float);
+  dim3 grid(static_cast<unsigned>((cols + kColTile - 1) / kColTile),
+            static_cast<unsigned>(rows / P));
+  fwht_cols_reg_kernel<<<grid, 2 * P, smem, stream>>>(m, rows, cols, log2p, rs, out_scale);
+  return check_launch("fwht_cols_reg_kernel");
+}
+
 kronq_status col_pass(float* m, int64_t rows, int64_t cols, int b, cudaStream_t stream) {
   if (b <= 1) return KRONQ_OK;
+  const float out_scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(b)));
+  if (b >= 16 && b <= 16384) {
+    const int L = ilog2_pow2(b);
+    if (L <= 8) return col_pass_reg(m, rows, cols, L, 1, out_scale, stream);
+    const int l1 = (L + 1) / 2, l2 = L / 2;   // H_b = (H_P2 (x) I_P1)(I_P2 (x) H_P1)
+    KQ_TRY(col_pass_reg(m, rows, cols, l1, 1, 1.0f, stream));
+    return col_pass_reg(m, rows, cols, l2, 1 << l1, out_scale, stream);
+  }
   int cw = 32768 / b;
   if (cw > 64) cw = 64;
   if (cw < 1) cw = 1;
   const size_t smem = static_cast<size_t>(b) * cw * sizeof(float);
-  const float out_scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(b)));
   if (smem > 48 * 1024)
     KQ_CUDA_TRY(cudaFuncSetAttribute(fwht_cols_kernel,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
