@@ -13,8 +13,10 @@
 //   K11 = chol_inv(A11)
 //   K12 = -K11 R12 K22              ([[R11, R12], [0, R22]]^-1)
 // Leaves of at most 128 columns are factored and inverted in shared memory by one CTA. The four
-// products per level are large square GEMMs on the tensor cores (operands split into three bf16
-// pieces, fp32-accurate) that skip the zero triangles of K.
+// products of a level are square GEMMs: on the tensor cores (operands split into three bf16
+// pieces, fp32-accurate, skipping the zero triangles of K) where a half exceeds 256, and on the
+// CUDA cores in fp32 below that, where a product is a handful of tiles and latency, not arithmetic, decides.
+#include <algorithm>
 #include <cmath>
 
 #include "common.cuh"
@@ -302,93 +304,257 @@ __global__ void __launch_bounds__(LEAF_THREADS, 1) leaf_kernel(float* __restrict
   }
 }
 
+// fp32 GEMM on the CUDA cores for the bottom levels of the recursion (m, n, k <= 256), where
+// a product is a handful of tiles and latency, not arithmetic, decides:
+//   C = alpha * A op(B) + beta * C,  op(B) = B^T (B given n x k) or B (B given k x n).
+// C must not alias A or B. CTA tile 32 x 64, 128 threads, each a 4 x 4 block (rows ty + 8i,
+// columns tx + 16j); K in chunks of 32, both operands staged along K in shared memory and read
+// as 16-byte vectors, the next chunk's loads in flight (registers) while this one is used.
+// k0 (A upper triangular) starts the K loop at the tile's first row.
+constexpr int SG_TM = 32, SG_TN = 64, SG_KC = 32, SG_LD = SG_KC + 4, SG_THREADS = 128;
+
+struct SgChunk {
+  float4 a[2];   // 32 x 32 of A: 256 float4, two per thread
+  float4 b[4];   // 64 x 32 of B: 512 float4, four per thread
+};
+
+__device__ __forceinline__ float4 ld4_guard(const float* p, int valid) {
+  // valid: how many of the 4 floats at p exist (0..4); the pointer is 16-byte aligned if 4
+  if (valid >= 4) return *reinterpret_cast<const float4*>(p);
+  float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (valid > 0) v.x = p[0];
+  if (valid > 1) v.y = p[1];
+  if (valid > 2) v.z = p[2];
+  return v;
+}
+
+__global__ void __launch_bounds__(SG_THREADS) sgemm_small_kernel(
+    int m, int n, int k, float alpha, const float* __restrict__ a, int64_t lda,
+    const float* __restrict__ b, int64_t ldb, int b_mn, float beta, float* __restrict__ c,
+    int64_t ldc, int upper_only, int a_upper, int vec, const int32_t* __restrict__ skip) {
+  if (skip && *skip >= 0) return;
+  __shared__ __align__(16) float as[2][SG_TM * SG_LD];
+  __shared__ __align__(16) float bs[2][SG_TN * SG_LD];
+  const int t = threadIdx.x, ty = t >> 4, tx = t & 15;
+  const int row0 = blockIdx.y * SG_TM, col0 = blockIdx.x * SG_TN;
+  if (upper_only && row0 > col0 + SG_TN - 1) return;
+  const int kbeg = a_upper ? (row0 / SG_KC) * SG_KC : 0;
+
+  // load mapping: A: float4 index e = t + 128 u (u < 2): row e / 8, k4 (e % 8) * 4
+  //   B K-major: e = t + 128 u (u < 4): col e / 8, k4 (e % 8) * 4
+  //   B MN-major: e = t + 128 u: k-row e / 16, col4 (e % 16) * 4
+  auto load = [&](int k0, SgChunk& ch) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int e = t + SG_THREADS * u, r = row0 + e / 8, kk = k0 + (e % 8) * 4;
+      ch.a[u] = (r < m) ? (vec ? ld4_guard(a + r * lda + kk, k - kk)
+                               : make_float4(kk < k ? a[r * lda + kk] : 0.f,
+                                             kk + 1 < k ? a[r * lda + kk + 1] : 0.f,
+                                             kk + 2 < k ? a[r * lda + kk + 2] : 0.f,
+                                             kk + 3 < k ? a[r * lda + kk + 3] : 0.f))
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int e = t + SG_THREADS * u;
+      if (!b_mn) {
+        const int cc = col0 + e / 8, kk = k0 + (e % 8) * 4;
+        ch.b[u] = (cc < n) ? (vec ? ld4_guard(b + cc * ldb + kk, k - kk)
+                                  : make_float4(kk < k ? b[cc * ldb + kk] : 0.f,
+                                                kk + 1 < k ? b[cc * ldb + kk + 1] : 0.f,
+                                                kk + 2 < k ? b[cc * ldb + kk + 2] : 0.f,
+                                                kk + 3 < k ? b[cc * ldb + kk + 3] : 0.f))
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+      } else {
+        const int kk = k0 + e / 16, cc = col0 + (e % 16) * 4;
+        ch.b[u] = (kk < k) ? (vec ? ld4_guard(b + kk * ldb + cc, n - cc)
+                                  : make_float4(cc < n ? b[kk * ldb + cc] : 0.f,
+                                                cc + 1 < n ? b[kk * ldb + cc + 1] : 0.f,
+                                                cc + 2 < n ? b[kk * ldb + cc + 2] : 0.f,
+                                                cc + 3 < n ? b[kk * ldb + cc + 3] : 0.f))
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+  };
+  auto store = [&](const SgChunk& ch, int buf) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int e = t + SG_THREADS * u;
+      *reinterpret_cast<float4*>(&as[buf][(e / 8) * SG_LD + (e % 8) * 4]) = ch.a[u];
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int e = t + SG_THREADS * u;
+      if (!b_mn) {
+        *reinterpret_cast<float4*>(&bs[buf][(e / 8) * SG_LD + (e % 8) * 4]) = ch.b[u];
+      } else {
+        const int kk = e / 16, cc = (e % 16) * 4;
+        bs[buf][(cc + 0) * SG_LD + kk] = ch.b[u].x;
+        bs[buf][(cc + 1) * SG_LD + kk] = ch.b[u].y;
+        bs[buf][(cc + 2) * SG_LD + kk] = ch.b[u].z;
+        bs[buf][(cc + 3) * SG_LD + kk] = ch.b[u].w;
+      }
+    }
+  };
+
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+  SgChunk ch;
+  int buf = 0;
+  if (kbeg < k) {
+    load(kbeg, ch);
+    store(ch, 0);
+  }
+  __syncthreads();
+  for (int k0 = kbeg; k0 < k; k0 += SG_KC) {
+    const bool more = k0 + SG_KC < k;
+    if (more) load(k0 + SG_KC, ch);          // in flight during the products below
+    const float* ap = &as[buf][ty * SG_LD];
+    const float* bp = &bs[buf][tx * SG_LD];
+#pragma unroll
+    for (int k4 = 0; k4 < SG_KC; k4 += 4) {
+      float4 av[4], bv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) av[i] = *reinterpret_cast<const float4*>(ap + 8 * i * SG_LD + k4);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) bv[j] = *reinterpret_cast<const float4*>(bp + 16 * j * SG_LD + k4);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          acc[i][j] = fmaf(av[i].x, bv[j].x, acc[i][j]);
+          acc[i][j] = fmaf(av[i].y, bv[j].y, acc[i][j]);
+          acc[i][j] = fmaf(av[i].z, bv[j].z, acc[i][j]);
+          acc[i][j] = fmaf(av[i].w, bv[j].w, acc[i][j]);
+        }
+    }
+    if (more) store(ch, buf ^ 1);
+    __syncthreads();
+    buf ^= 1;
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = row0 + ty + 8 * i;
+    if (r >= m) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int cc = col0 + tx + 16 * j;
+      if (cc >= n || (upper_only && cc < r)) continue;
+      float* p = c + r * ldc + cc;
+      *p = beta != 0.f ? fmaf(beta, *p, alpha * acc[i][j]) : alpha * acc[i][j];
+    }
+  }
+}
+kronq_status sgemm_small(int m, int n, int k, float alpha, const float* a, int64_t lda,
+                         const float* b, int64_t ldb, bool b_mn_major, float beta, float* c,
+                         int64_t ldc, bool upper_only, bool a_upper, const int32_t* skip,
+                         cudaStream_t stream) {
+  if (m <= 0 || n <= 0) return KRONQ_OK;
+  if (k <= 0) return fail(KRONQ_ERR_SHAPE, "sgemm_small: k must be >= 1");
+  const int vec = (reinterpret_cast<uintptr_t>(a) & 15u) == 0 &&
+                  (reinterpret_cast<uintptr_t>(b) & 15u) == 0 && lda % 4 == 0 && ldb % 4 == 0;
+  dim3 grid(static_cast<unsigned>((n + SG_TN - 1) / SG_TN),
+            static_cast<unsigned>((m + SG_TM - 1) / SG_TM));
+  sgemm_small_kernel<<<grid, SG_THREADS, 0, stream>>>(m, n, k, alpha, a, lda, b, ldb, b_mn_major,
+                                                      beta, c, ldc, upper_only, a_upper, vec,
+                                                      skip);
+  return check_launch("sgemm_small_kernel");
+}
+
 struct Ctx {
   int64_t ld;
   float* t;          // n1 x n2 product T of the top level (largest)
-  uint8_t* splits;   // split operands of one GEMM at a time
   int32_t* info;
   cudaStream_t stream;
 };
 
+void halves(int n, int& n1, int& n2) {
+  // bottom-right part: a multiple of NB columns, about half
+  n2 = ((n / 2 + NB - 1) / NB) * NB;
+  if (n2 >= n) n2 = n - NB;
+  n1 = n - n2;
+}
+
+// Split-operand scratch of one recursion node and everything below it. A node keeps the splits
+// of K22 and of A12 / R12 from the first GEMM to the last (across the K11 recursion), so each is
+// split once; the K11 recursion and the (K11, T) pair use the space after them.
+size_t area_bytes(int n) {
+  if (n <= NB) return 0;
+  int n1, n2;
+  halves(n, n1, n2);
+  if (n1 <= 256 && n2 <= 256)
+    return std::max(area_bytes(n2),
+                    align256(2 * sizeof(float) * static_cast<size_t>(n1) * n2) + area_bytes(n1));
+  const size_t own = split_bytes(n2, n2) + split_bytes(n1, n2);
+  const size_t tail = std::max(area_bytes(n1), split_bytes(n1, n1) + split_bytes(n1, n2));
+  return std::max(area_bytes(n2), own + tail);
+}
+
 // Overwrite the n x n diagonal block at a (global index j0) with K.
-kronq_status chol_inv_rec(const Ctx& c, float* a, int n, int j0) {
+kronq_status chol_inv_rec(const Ctx& c, float* a, int n, int j0, uint8_t* area) {
   if (n <= NB) {
     leaf_kernel<<<1, LEAF_THREADS, LEAF_SMEM, c.stream>>>(a, c.ld, n, j0, c.info);
     return check_launch("leaf_kernel");
   }
-  // bottom-right part: a multiple of NB columns, about half
-  int n2 = ((n / 2 + NB - 1) / NB) * NB;
-  if (n2 >= n) n2 = n - NB;
-  const int n1 = n - n2;
+  int n1, n2;
+  halves(n, n1, n2);
   float* a11 = a;
   float* a12 = a + n1;
   float* a22 = a + static_cast<int64_t>(n1) * c.ld + n1;
   const int64_t ld = c.ld;
   cudaStream_t st = c.stream;
 
-  KQ_TRY(chol_inv_rec(c, a22, n2, j0 + n1));                               // K22
-  {
-    // R12 = A12 K22^T, written over A12 (the GEMM reads split copies)
-    Carve cv{c.splits};
-    Split3 s12 = cv.split(n1, n2), s22 = cv.split(n2, n2);
-    KQ_TRY(split_bf16x3_2(a12, ld, n1, n2, s12, a22, ld, n2, n2, s22, st));
-    KQ_TRY(tgemm(n1, n2, n2, 1.f, s12, s22, false, 0.f, a12, ld, false, GEMM_B_LOWER, c.info, st));
+  KQ_TRY(chol_inv_rec(c, a22, n2, j0 + n1, area));                         // K22
+  if (n1 <= 256 && n2 <= 256) {
+    // small node: the four products on the CUDA cores, straight from the fp32 blocks; R12 and
+    // T live in this node's scratch, the K11 recursion uses the space after them
+    float* r12 = reinterpret_cast<float*>(area);
+    float* tt = r12 + static_cast<int64_t>(n1) * n2;
+    uint8_t* rest = reinterpret_cast<uint8_t*>(tt + static_cast<int64_t>(n1) * n2);
+    KQ_TRY(sgemm_small(n1, n2, n2, 1.f, a12, ld, a22, ld, false, 0.f, r12, n2, false, false,
+                       c.info, st));                                        // R12 = A12 K22^T
+    KQ_TRY(sgemm_small(n1, n1, n2, -1.f, r12, n2, r12, n2, false, 1.f, a11, ld, true, false,
+                       c.info, st));                                        // A11 -= R12 R12^T
+    KQ_TRY(chol_inv_rec(c, a11, n1, j0, rest));                            // K11
+    KQ_TRY(sgemm_small(n1, n2, n2, 1.f, r12, n2, a22, ld, true, 0.f, tt, n2, false, false,
+                       c.info, st));                                        // T = R12 K22
+    return sgemm_small(n1, n2, n1, -1.f, a11, ld, tt, n2, true, 0.f, a12, ld, false, true,
+                       c.info, st);                                         // K12 = -K11 T
   }
-  {
-    // A11 -= R12 R12^T (upper triangle)
-    Carve cv{c.splits};
-    Split3 r12 = cv.split(n1, n2);
-    KQ_TRY(split_bf16x3(a12, ld, n1, n2, r12, st));
-    KQ_TRY(tgemm(n1, n1, n2, -1.f, r12, r12, false, 1.f, a11, ld, true, 0, c.info, st));
-  }
-  KQ_TRY(chol_inv_rec(c, a11, n1, j0));                                    // K11
-  {
-    // T = R12 K22
-    Carve cv{c.splits};
-    Split3 r12 = cv.split(n1, n2), s22 = cv.split(n2, n2);
-    KQ_TRY(split_bf16x3_2(a12, ld, n1, n2, r12, a22, ld, n2, n2, s22, st));
-    KQ_TRY(tgemm(n1, n2, n2, 1.f, r12, s22, true, 0.f, c.t, n2, false, GEMM_B_UPPER, c.info, st));
-  }
-  {
-    // K12 = -K11 T
-    Carve cv{c.splits};
-    Split3 s11 = cv.split(n1, n1), tt = cv.split(n1, n2);
-    KQ_TRY(split_bf16x3_2(a11, ld, n1, n1, s11, c.t, n2, n1, n2, tt, st));
-    KQ_TRY(tgemm(n1, n2, n1, -1.f, s11, tt, true, 0.f, a12, ld, false, GEMM_A_UPPER, c.info, st));
-  }
+  Carve cv{area};
+  const Split3 s22 = cv.split(n2, n2);    // K22, kept to the end of the node
+  const Split3 s12 = cv.split(n1, n2);    // A12, then R12
+  uint8_t* rest = cv.p;
+  // R12 = A12 K22^T, written over A12
+  KQ_TRY(split_bf16x3_2(a22, ld, n2, n2, s22, a12, ld, n1, n2, s12, st));
+  KQ_TRY(tgemm(n1, n2, n2, 1.f, s12, s22, false, 0.f, a12, ld, false, GEMM_B_LOWER, c.info, st));
+  // A11 -= R12 R12^T (upper triangle)
+  KQ_TRY(split_bf16x3(a12, ld, n1, n2, s12, st));
+  KQ_TRY(tgemm(n1, n1, n2, -1.f, s12, s12, false, 1.f, a11, ld, true, 0, c.info, st));
+  KQ_TRY(chol_inv_rec(c, a11, n1, j0, rest));                              // K11
+  // T = R12 K22
+  KQ_TRY(tgemm(n1, n2, n2, 1.f, s12, s22, true, 0.f, c.t, n2, false, GEMM_B_UPPER, c.info, st));
+  // K12 = -K11 T
+  Carve cr{rest};
+  const Split3 s11 = cr.split(n1, n1), tt = cr.split(n1, n2);
+  KQ_TRY(split_bf16x3_2(a11, ld, n1, n1, s11, c.t, n2, n1, n2, tt, st));
+  KQ_TRY(tgemm(n1, n2, n1, -1.f, s11, tt, true, 0.f, a12, ld, false, GEMM_A_UPPER, c.info, st));
   return KRONQ_OK;
 }
 
-// Sizes of the top level (the largest of every level).
-void top_split(int d, int& n1, int& n2) {
-  if (d <= NB) {
-    n1 = n2 = 0;
-    return;
-  }
-  n2 = ((d / 2 + NB - 1) / NB) * NB;
-  if (n2 >= d) n2 = d - NB;
-  n1 = d - n2;
-}
-
 size_t t_bytes(int d) {
+  if (d <= NB) return align256(sizeof(float));
   int n1, n2;
-  top_split(d, n1, n2);
-  return align256(sizeof(float) * static_cast<size_t>(n1 > 0 ? n1 : 1) * (n2 > 0 ? n2 : 1));
-}
-
-size_t split_area_bytes(int d) {
-  int n1, n2;
-  top_split(d, n1, n2);
-  if (n1 == 0) return 0;
-  // the largest GEMM operand pair of any level is at the top level
-  const size_t a = split_bytes(n1, n2) + split_bytes(n2, n2);
-  const size_t b = split_bytes(n1, n1) + split_bytes(n1, n2);
-  return a > b ? a : b;
+  halves(d, n1, n2);
+  return align256(sizeof(float) * static_cast<size_t>(n1) * n2);
 }
 
 }  // namespace
 
-size_t cholinv_workspace_bytes(int d) { return 256 + t_bytes(d) + split_area_bytes(d); }
+size_t cholinv_workspace_bytes(int d) { return 256 + t_bytes(d) + area_bytes(d); }
 
 kronq_status run_cholinv(float* a, int d, float damp_rel, int32_t* info, void* ws,
                          cudaStream_t stream) {
@@ -410,8 +576,8 @@ kronq_status run_cholinv(float* a, int d, float damp_rel, int32_t* info, void* w
                                      static_cast<int>(LEAF_SMEM)));
     attr = true;
   }
-  Ctx c{d, t, p, info, stream};
-  return chol_inv_rec(c, a, d, 0);
+  Ctx c{d, t, info, stream};
+  return chol_inv_rec(c, a, d, 0, p);
 }
 
 }  // namespace kq

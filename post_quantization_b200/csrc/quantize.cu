@@ -10,8 +10,10 @@
 //
 // Solve: 128-column blocks. Inside a block every output row is independent given K; one lane
 // per row walks the block's columns in order (quantize, error, update the remaining columns of
-// the block), the four warps of a CTA each holding a quarter of the block's columns. After the block the rest of every row is updated lazily with
-// one GEMM: W~[:, e:] -= Delta_blk K[blk, e:].
+// the block), the four warps of a CTA each holding a quarter of the block's columns. The rest of
+// every row is updated lazily with GEMMs, in two levels: after a block, the rest of its
+// 1024-column super-block, W~[:, e:s1] -= Delta_blk K[blk, e:s1]; after a super-block, the rest
+// of W, W~[:, s1:] -= Delta_sb K[sb, s1:].
 #include <cuda_bf16.h>
 
 #include <cmath>
@@ -24,6 +26,7 @@ namespace kq {
 namespace {
 
 constexpr int QB = 128;        // column block
+constexpr int QSB = 1024;      // super-block: the rest of W is updated once per QSB columns
 constexpr int QROWS = 32;      // rows per CTA in the block solve
 constexpr int QT = 4;          // warps per CTA: one column quarter each
 constexpr int QW = QB / QT;    // columns per thread
@@ -72,13 +75,13 @@ __global__ void striu_kernel(float* __restrict__ m, int d) {
 // K rows are read as broadcasts (every lane of a warp reads the same row), so the solve is bound
 // by the per-column dependency chain, not by shared memory.
 //   w_hat  d_out x d_in running weights (in: current values, out: dequantized for the block)
-//   delta  d_out x QB errors scaled by 1/K_pp, written as three bf16 pieces (the operand of
-//          the lazy trailing update on the tensor cores)
+//   delta  d_out x QB errors scaled by 1/K_pp (row stride ldd), written as three bf16 pieces
+//          (the operand of the lazy trailing updates on the tensor cores)
 __global__ void __launch_bounds__(QROWS * QT) block_solve_kernel(
     float* __restrict__ w_hat, const float* __restrict__ k, int d_out, int d_in, int b0, int bw,
     const float* __restrict__ scale, const float* __restrict__ zero, float maxq,
     uint8_t* __restrict__ codes, uint16_t* __restrict__ delta0, uint16_t* __restrict__ delta1,
-    uint16_t* __restrict__ delta2) {
+    uint16_t* __restrict__ delta2, int64_t ldd) {
   extern __shared__ __align__(16) float sm[];
   float* Ks = sm;                      // QB x KS_LD: the K block
   float* E = Ks + QB * KS_LD;          // QROWS x E_LD: scaled errors of the block
@@ -194,7 +197,7 @@ __global__ void __launch_bounds__(QROWS * QT) block_solve_kernel(
     }
     // the errors, split into three bf16 pieces for the tensor-core trailing update
     // (8 columns per 16-byte store; the row's 32 columns start on a 64-byte boundary)
-    const int64_t o = static_cast<int64_t>(row) * QB + QW * q;
+    const int64_t o = static_cast<int64_t>(row) * ldd + QW * q;
 #pragma unroll
     for (int j8 = 0; j8 < QW; j8 += 8) {
       uint32_t h0[4], h1[4], h2[4];
@@ -231,7 +234,7 @@ __global__ void __launch_bounds__(QROWS * QT) block_solve_kernel(
 size_t quantize_workspace_bytes(int d_out, int d_in, int block, bool with_dxx) {
   (void)block;
   size_t b = split_bytes(d_in, d_in);        // K, split once per layer
-  b += split_bytes(d_out, QB);               // block errors
+  b += split_bytes(d_out, QSB);              // errors of one super-block
   if (with_dxx) {
     const size_t r1 = split_bytes(d_in, d_in) > split_bytes(d_out, d_in) ? split_bytes(d_in, d_in)
                                                                          : split_bytes(d_out, d_in);
@@ -250,7 +253,7 @@ kronq_status run_quantize(const float* w, const float* k, const float* dxx, int 
   const float maxq = static_cast<float>((1 << bits) - 1);
   Carve cv{static_cast<uint8_t*>(ws)};
   Split3 ks = cv.split(d_in, d_in);
-  Split3 ds = cv.split(d_out, QB);
+  Split3 ds = cv.split(d_out, QSB);
 
   // grid from W before the solve
   grid_kernel<<<(d_out + 7) / 8, 256, 0, stream>>>(w, d_out, d_in, maxq, scale, zero);
@@ -306,17 +309,29 @@ kronq_status run_quantize(const float* w, const float* k, const float* dxx, int 
                                      (int)smem));
     attr = true;
   }
-  for (int b0 = 0; b0 < d_in; b0 += QB) {
-    const int bw = d_in - b0 < QB ? d_in - b0 : QB;
-    block_solve_kernel<<<(d_out + QROWS - 1) / QROWS, QROWS * QT, smem, stream>>>(
-        w_hat, k, d_out, d_in, b0, bw, scale, zero, maxq, codes, ds.part[0], ds.part[1], ds.part[2]);
-    KQ_TRY(check_launch("block_solve_kernel"));
-    const int e = b0 + bw;
-    if (e < d_in) {
-      // W~[:, e:] -= Delta K[b0:e, e:]
-      const Split3 kb = offset(ks, b0, e);
-      KQ_TRY(tgemm(d_out, d_in - e, bw, -1.f, ds, kb, true, 1.f, w_hat + e, d_in, false, 0,
-                   nullptr, stream));
+  // Two-level lazy updates: after a 128-column block only the rest of its super-block is
+  // updated (K = 128); after a super-block, the rest of W at once (K = QSB), so the fp32 W is
+  // read and written once per super-block instead of once per block.
+  for (int s0 = 0; s0 < d_in; s0 += QSB) {
+    const int s1 = d_in - s0 < QSB ? d_in : s0 + QSB;
+    for (int b0 = s0; b0 < s1; b0 += QB) {
+      const int bw = d_in - b0 < QB ? d_in - b0 : QB;
+      const Split3 db = offset(ds, 0, b0 - s0);
+      block_solve_kernel<<<(d_out + QROWS - 1) / QROWS, QROWS * QT, smem, stream>>>(
+          w_hat, k, d_out, d_in, b0, bw, scale, zero, maxq, codes, db.part[0], db.part[1],
+          db.part[2], db.ld);
+      KQ_TRY(check_launch("block_solve_kernel"));
+      const int e = b0 + bw;
+      if (e < s1) {
+        // W~[:, e:s1] -= Delta_blk K[b0:e, e:s1]
+        KQ_TRY(tgemm(d_out, s1 - e, bw, -1.f, db, offset(ks, b0, e), true, 1.f, w_hat + e, d_in,
+                     false, 0, nullptr, stream));
+      }
+    }
+    if (s1 < d_in) {
+      // W~[:, s1:] -= Delta_sb K[s0:s1, s1:]
+      KQ_TRY(tgemm(d_out, d_in - s1, s1 - s0, -1.f, ds, offset(ks, s0, s1), true, 1.f,
+                   w_hat + s1, d_in, false, 0, nullptr, stream));
     }
   }
   return KRONQ_OK;

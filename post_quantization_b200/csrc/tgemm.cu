@@ -285,25 +285,52 @@ struct SplitJob {
   int64_t ld;
 };
 
-__global__ void split_bf16x3_kernel(SplitJob j0, SplitJob j1) {
-  const int64_t n0 = static_cast<int64_t>(j0.rows) * j0.cols;
-  const int64_t total = n0 + static_cast<int64_t>(j1.rows) * j1.cols;
-  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
-       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const bool second = e >= n0;
-    const SplitJob& j = second ? j1 : j0;
-    const int64_t f = second ? e - n0 : e;
-    const int64_t r = f / j.cols, c = f - r * j.cols;
-    const float x = j.src[r * j.lds + c];
-    const __nv_bfloat16 b0 = __float2bfloat16_rn(x);
-    const float r1 = x - __bfloat162float(b0);
+// 8 consecutive columns of one row per thread (blockIdx.y = row, blockIdx.z = job): no index
+// division, 16-byte stores of each piece (destination rows start on 16-byte boundaries: the
+// stride is a multiple of 8 elements).
+__global__ void __launch_bounds__(128) split_bf16x3_kernel(SplitJob j0, SplitJob j1) {
+  const SplitJob& j = blockIdx.z ? j1 : j0;
+  const int r = blockIdx.y;
+  const int c8 = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
+  if (r >= j.rows || c8 >= j.cols) return;
+  const float* src = j.src + static_cast<int64_t>(r) * j.lds + c8;
+  float x[8];
+  const bool vec = c8 + 8 <= j.cols && ((reinterpret_cast<uintptr_t>(src) & 15u) == 0);
+  if (vec) {
+    const float4 a = reinterpret_cast<const float4*>(src)[0];
+    const float4 b = reinterpret_cast<const float4*>(src)[1];
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  } else {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) x[u] = c8 + u < j.cols ? src[u] : 0.f;
+  }
+  uint32_t h[3][4];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const __nv_bfloat16 b0 = __float2bfloat16_rn(x[u]);
+    const float r1 = x[u] - __bfloat162float(b0);
     const __nv_bfloat16 b1 = __float2bfloat16_rn(r1);
     const float r2 = r1 - __bfloat162float(b1);
     const __nv_bfloat16 b2 = __float2bfloat16_rn(r2);
-    const int64_t o = r * j.ld + c;
-    j.part[0][o] = __bfloat16_as_ushort(b0);
-    j.part[1][o] = __bfloat16_as_ushort(b1);
-    j.part[2][o] = __bfloat16_as_ushort(b2);
+    const int sh = 16 * (u & 1);
+    if ((u & 1) == 0) { h[0][u >> 1] = 0u; h[1][u >> 1] = 0u; h[2][u >> 1] = 0u; }
+    h[0][u >> 1] |= static_cast<uint32_t>(__bfloat16_as_ushort(b0)) << sh;
+    h[1][u >> 1] |= static_cast<uint32_t>(__bfloat16_as_ushort(b1)) << sh;
+    h[2][u >> 1] |= static_cast<uint32_t>(__bfloat16_as_ushort(b2)) << sh;
+  }
+  const int64_t o = static_cast<int64_t>(r) * j.ld + c8;
+  if (c8 + 8 <= j.cols) {
+#pragma unroll
+    for (int i = 0; i < 3; ++i)
+      *reinterpret_cast<uint4*>(j.part[i] + o) = make_uint4(h[i][0], h[i][1], h[i][2], h[i][3]);
+  } else {
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (c8 + u < j.cols) {
+#pragma unroll
+        for (int i = 0; i < 3; ++i)
+          j.part[i][o + u] = static_cast<uint16_t>(h[i][u >> 1] >> (16 * (u & 1)));
+      }
   }
 }
 
@@ -371,12 +398,13 @@ kronq_status split_bf16x3_2(const float* src0, int64_t lds0, int rows0, int cols
               {dst0.part[0], dst0.part[1], dst0.part[2]}, dst0.ld};
   SplitJob j1{src1, lds1, (src1 && cols1 > 0) ? rows1 : 0, cols1 > 0 ? cols1 : 1,
               {dst1.part[0], dst1.part[1], dst1.part[2]}, dst1.ld};
-  const int64_t total =
-      static_cast<int64_t>(j0.rows) * j0.cols + static_cast<int64_t>(j1.rows) * j1.cols;
-  if (total <= 0) return KRONQ_OK;
-  int64_t blocks = (total + 255) / 256;
-  if (blocks > 148 * 32) blocks = 148 * 32;
-  split_bf16x3_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(j0, j1);
+  const int rows = j0.rows > j1.rows ? j0.rows : j1.rows;
+  const int cols = j0.cols > j1.cols ? j0.cols : j1.cols;
+  if (rows <= 0) return KRONQ_OK;
+  if (rows > 65535) return fail(KRONQ_ERR_SHAPE, "split: more than 65535 rows");
+  dim3 grid(static_cast<unsigned>((cols + 8 * 128 - 1) / (8 * 128)), static_cast<unsigned>(rows),
+            j1.rows > 0 ? 2u : 1u);
+  split_bf16x3_kernel<<<grid, 128, 0, stream>>>(j0, j1);
   return check_launch("split_bf16x3_kernel");
 }
 
