@@ -346,7 +346,7 @@ def run_gpu(args):
         # launches at d = 4096 and 3 at d = 11008; from ncu captures of this kernel version at
         # the same 16384-token work units, scaled to 262144 tokens (see the accumulate summary
         # under profiles/)
-        traffic = 16.7e9 if n_tok == 262144 else None
+        traffic = None   # the statistics kernel changed since its DRAM counters were taken
         acc_tflops = sum(acc_flops) / (sum(acc_ms) / 1e3) / 1e12
         result = {
             "metric": "quantized weight params/s (BiIP+GPTAQ solve); H_X/H_G accumulate TFLOP/s",

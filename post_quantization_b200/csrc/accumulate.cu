@@ -7,12 +7,15 @@
 //
 // Kernel: persistent, one CTA per SM, warp-specialised.
 //   warp 0        TMA producer: loads 64-token x 64-column boxes (128-byte swizzle) of A and B
-//                 into a 4-stage shared-memory ring (no multicast).
+//                 into a 3-stage shared-memory ring (no multicast).
 //   warp 1        TMEM allocator + MMA issuer: tcgen05.mma kind::f16, M=128, N=256, K=16,
-//                 bf16 x bf16 -> fp32 in TMEM; two 256-column accumulators so the epilogue of
-//                 one work unit overlaps the main loop of the next.
+//                 bf16 x bf16 -> fp32 in TMEM. An output tile is 256 x 256: two M=128 MMAs per
+//                 K step share the stage's B operand, filling all 512 TMEM columns, so every
+//                 operand byte staged from L2 feeds twice the tensor work of a 128-row tile and
+//                 the ring holds more MMA time against the L2 latency.
 //   warps 2..5    epilogue: tcgen05.ld the accumulator, add it into C with vector atomics (the
-//                 call's contract is "+=", and split-K partial sums combine the same way).
+//                 call's contract is "+=", and split-K partial sums combine the same way). With
+//                 TMEM full, the next unit's MMAs wait for the drain (a few percent of a unit).
 // Work unit = (output tile, token chunk). For symmetric outputs only tiles touching the upper
 // triangle are computed and a mirror kernel fills the strict lower triangle afterwards.
 #include <cuda_bf16.h>
@@ -23,18 +26,19 @@
 namespace kq {
 
 namespace acc {
-constexpr int BM = 128;             // output rows per tile (MMA M)
+constexpr int BM = 256;             // output rows per tile (two MMAs of M = 128)
+constexpr int HM = 128;             // MMA M
 constexpr int BN = 256;             // output cols per tile (MMA N)
 constexpr int BK = 64;              // tokens per pipeline stage
 constexpr int UK = 16;              // tokens per MMA instruction
-constexpr int STAGES = 4;
+constexpr int STAGES = 3;
 constexpr int BOX = 64;             // columns per TMA box (128 bytes of bf16)
 constexpr int BOX_BYTES = BOX * BK * 2;          // 8 KB
-constexpr int A_BOXES = BM / BOX;                // 2
+constexpr int A_BOXES = BM / BOX;                // 4
 constexpr int B_BOXES = BN / BOX;                // 4
-constexpr int STAGE_BYTES = (A_BOXES + B_BOXES) * BOX_BYTES;   // 48 KB
+constexpr int STAGE_BYTES = (A_BOXES + B_BOXES) * BOX_BYTES;   // 64 KB
 constexpr int THREADS = 192;
-constexpr int TMEM_COLS = 512;      // 2 accumulators x 256 fp32 columns
+constexpr int TMEM_COLS = 512;      // 2 M-halves x 256 fp32 columns
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 }  // namespace acc
 
@@ -172,7 +176,7 @@ __global__ void __launch_bounds__(acc::THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32_mn_mn(BM, BN);
+      constexpr uint32_t idesc = idesc_bf16_f32_mn_mn(HM, BN);
       uint32_t it = 0;
       uint32_t ui = 0;
       bool ok = true;
@@ -180,11 +184,12 @@ __global__ void __launch_bounds__(acc::THREADS, 1)
         const int split = u / p.num_tiles;
         const int kb0 = split * p.kblocks_per_unit;
         const int kb1 = min(kblocks_total, kb0 + p.kblocks_per_unit);
-        const uint32_t a = ui & 1u;
-        const uint32_t aph = (ui >> 1) & 1u;
-        if (!mbar_wait(&tempty[a], aph ^ 1u, abort_flag, p.err, DEV_ERR_MMA_WAIT)) break;
+        int tm, tn;
+        tile_coords(p, u % p.num_tiles, tm, tn);
+        const bool half1 = tm * BM + HM < p.m;   // rows of the second M-half exist
+        // TMEM holds one tile: wait until the epilogue has drained the previous one
+        if (!mbar_wait(&tempty[0], (ui & 1u) ^ 1u, abort_flag, p.err, DEV_ERR_MMA_WAIT)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + a * BN;
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
@@ -198,16 +203,21 @@ __global__ void __launch_bounds__(acc::THREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < BK / UK; ++kk) {
             // MN-major, 128B swizzle: 8 token rows of 128 bytes form one 1 KB atom (SBO);
-            // successive 64-column boxes are one box apart (LBO).
+            // successive 64-column boxes are one box apart (LBO). M-half h starts 2 boxes in.
             const uint32_t koff = kk * UK * 128;
-            const uint64_t ad = smem_desc_sw128(a_base + koff, BOX_BYTES, 1024);
+            const uint32_t acc_flag = (kb > kb0 || kk > 0) ? 1u : 0u;
             const uint64_t bd = smem_desc_sw128(b_base + koff, BOX_BYTES, 1024);
-            umma_f16(d_tmem, ad, bd, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+            const uint64_t ad0 = smem_desc_sw128(a_base + koff, BOX_BYTES, 1024);
+            umma_f16(tmem_base, ad0, bd, idesc, acc_flag);
+            if (half1) {
+              const uint64_t ad1 = smem_desc_sw128(a_base + 2 * BOX_BYTES + koff, BOX_BYTES, 1024);
+              umma_f16(tmem_base + BN, ad1, bd, idesc, acc_flag);
+            }
           }
           umma_commit(&empty[s]);   // frees the stage once these MMAs have read it
         }
         if (!ok) break;
-        umma_commit(&tfull[a]);     // accumulator ready for the epilogue
+        umma_commit(&tfull[0]);     // accumulator ready for the epilogue
       }
     }
   } else {
@@ -218,42 +228,45 @@ __global__ void __launch_bounds__(acc::THREADS, 1)
       const int t = u % p.num_tiles;
       int tm, tn;
       tile_coords(p, t, tm, tn);
-      const uint32_t a = ui & 1u;
-      const uint32_t aph = (ui >> 1) & 1u;
       // one lane waits, the warp follows its verdict (tcgen05.ld needs a converged warp)
       int ok = 1;
-      if (lane == 0) ok = mbar_wait(&tfull[a], aph, abort_flag, p.err, DEV_ERR_EPI_WAIT) ? 1 : 0;
+      if (lane == 0)
+        ok = mbar_wait(&tfull[0], ui & 1u, abort_flag, p.err, DEV_ERR_EPI_WAIT) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       __syncwarp();
       if (!ok) break;
       tc_fence_after();
-      const int row = tm * BM + q * 32 + lane;
-      const uint32_t taddr = tmem_base + ((q * 32u) << 16) + a * BN;
 #pragma unroll 1
-      for (int cb = 0; cb < BN / 32; ++cb) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(taddr + cb * 32, v);
-        tmem_ld_wait();
-        const int col0 = tn * BN + cb * 32;
-        if (row < p.m && col0 < p.n) {
-          float* dst = p.c + static_cast<int64_t>(row) * p.ldc + col0;
-          if (col0 + 32 <= p.n && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
+      for (int h = 0; h < 2; ++h) {
+        const int row = tm * BM + h * HM + q * 32 + lane;
+        if (tm * BM + h * HM >= p.m) break;              // uniform: the half has no rows
+        const uint32_t taddr = tmem_base + ((q * 32u) << 16) + h * BN;
+#pragma unroll 1
+        for (int cb = 0; cb < BN / 32; ++cb) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(taddr + cb * 32, v);
+          tmem_ld_wait();
+          const int col0 = tn * BN + cb * 32;
+          if (row < p.m && col0 < p.n) {
+            float* dst = p.c + static_cast<int64_t>(row) * p.ldc + col0;
+            if (col0 + 32 <= p.n && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
 #pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-              float4 f = make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
-                                     __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
-              atomicAdd(reinterpret_cast<float4*>(dst + j), f);
+              for (int j = 0; j < 32; j += 4) {
+                float4 f = make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
+                                       __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+                atomicAdd(reinterpret_cast<float4*>(dst + j), f);
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (col0 + j < p.n) atomicAdd(dst + j, __uint_as_float(v[j]));
             }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (col0 + j < p.n) atomicAdd(dst + j, __uint_as_float(v[j]));
           }
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[a]);
+      if (lane == 0) mbar_arrive(&tempty[0]);
     }
   }
 
