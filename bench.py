@@ -343,10 +343,10 @@ def run_gpu(args):
             peak_src = "fallback (sustained bf16)"
         achieved = sum(acc_flops) / (sum(acc_ms) / 1e3) / 1e12
         # DRAM bytes (read + write) per accumulate_tc_kernel launch, averaged over a step's 8
-        # launches at d = 4096 and 3 at d = 11008; from ncu captures of this kernel version at
-        # the same 16384-token work units, scaled to 262144 tokens (see the accumulate summary
-        # under profiles/)
-        traffic = None   # the statistics kernel changed since its DRAM counters were taken
+        # launches at d = 4096 and 3 at d = 11008: ncu captures of this kernel version at
+        # d = 4096 / 262144 tokens (5.51 GB) and d = 11008 / 131072 tokens (21.2 GB, x2 for
+        # 262144 tokens); the accumulate summary under profiles/ has the commands
+        traffic = 15.6e9 if n_tok == 262144 else None
         acc_tflops = sum(acc_flops) / (sum(acc_ms) / 1e3) / 1e12
         result = {
             "metric": "quantized weight params/s (BiIP+GPTAQ solve); H_X/H_G accumulate TFLOP/s",
