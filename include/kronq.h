@@ -80,6 +80,15 @@ KRONQ_API kronq_status kronq_device_check(void);
 /* Number of kernels this library has launched in this process (all devices, all threads). */
 KRONQ_API uint64_t kronq_launch_count(void);
 
+/* SM budget for the persistent kernels (the statistics kernel of kronq_accumulate and the
+ * tensor-core GEMMs inside kronq_cholinv and kronq_quantize_layer): launches made while a budget
+ * of n > 0 is set use at most n CTAs, one per SM, so that work on other streams keeps the rest
+ * of the GPU. 0 (the default) lifts it. Process-wide, read at launch time (a captured CUDA graph
+ * keeps the grid it was captured with); it changes no result. Not a reservation: nothing stops
+ * other kernels from using the budgeted SMs. */
+KRONQ_API void kronq_set_sm_budget(int32_t sms);
+KRONQ_API int32_t kronq_sm_budget(void);
+
 /* Reads and clears the device-side error word (bounded waits that gave up). Synchronizes
  * `stream`. *code_out = 0 when no kernel reported an error since the last call. */
 KRONQ_API kronq_status kronq_device_error(int32_t* code_out, kronq_stream_t stream);

@@ -37,6 +37,27 @@ kronq_status fail(kronq_status s, const char* fmt, ...) {
 }
 
 std::atomic<uint64_t> g_launches{0};
+std::atomic<int> g_sm_budget{0};
+
+int device_sms() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+    sms = 148;
+  return sms;
+}
+
+int sm_budget() {
+  static thread_local int cached_dev = -1, cached_sms = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev != cached_dev) {
+    cached_sms = device_sms();
+    cached_dev = dev;
+  }
+  const int b = g_sm_budget.load(std::memory_order_relaxed);
+  return (b > 0 && b < cached_sms) ? b : cached_sms;
+}
 
 kronq_status check_launch(const char* what) {
   g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -115,6 +136,10 @@ const char* kronq_last_error_detail(void) { return g_detail; }
 int kronq_version(void) { return 100; }
 
 uint64_t kronq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+void kronq_set_sm_budget(int32_t sms) { kq::g_sm_budget.store(sms > 0 ? sms : 0); }
+
+int32_t kronq_sm_budget(void) { return kq::g_sm_budget.load(); }
 
 kronq_status kronq_device_check(void) {
   int dev = 0;

@@ -410,7 +410,8 @@ kronq_status launch_accumulate_tc(const void* a, int64_t ld_a, const void* b, in
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
     attr_set = true;
   }
-  const int grid = p.num_units < sms ? p.num_units : sms;
+  const int budget = sm_budget();
+  const int grid = p.num_units < budget ? p.num_units : budget;
   accumulate_tc_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(ma, mb, p);
   KQ_TRY(check_launch("accumulate_tc_kernel"));
   return KRONQ_OK;

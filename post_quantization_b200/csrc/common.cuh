@@ -33,6 +33,9 @@ kronq_status check_launch(const char* what);
 
 // Device-side error word: kernels that give up a bounded wait record a code here.
 int* device_error_word();   // device address of the word (current device)
+// SMs that persistent kernels may size their grids to: the device's SM count, or less while
+// kronq_set_sm_budget has set a budget (read at launch time).
+int sm_budget();
 
 // Error codes a kernel can record.
 enum DeviceError : int {

@@ -373,16 +373,6 @@ kronq_status map_bf16(CUtensorMap* map, const uint16_t* base, int64_t rows, int6
   return KRONQ_OK;
 }
 
-int sm_count() {
-  static int sms = 0;
-  if (!sms) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms <= 0) sms = 148;
-  }
-  return sms;
-}
 
 }  // namespace
 
@@ -444,9 +434,22 @@ kronq_status tgemm(int m, int n, int k, float alpha, Split3 a, Split3 b, bool b_
                                      SMEM_BYTES));
     attr = true;
   }
+  // As few CTAs as the minimal number of tile waves needs: each CTA holds a whole SM (shared
+  // memory), and SMs this GEMM does not need stay free for other streams' work.
   const int tiles = p.tiles_m * p.tiles_n;
-  const int sms = sm_count();
-  tgemm_kernel<<<tiles < sms ? tiles : sms, THREADS, SMEM_BYTES, stream>>>(maps, p);
+  int work = tiles;
+  if (upper_only) {
+    work = 0;
+    for (int tm = 0; tm < p.tiles_m; ++tm)
+      for (int tn = 0; tn < p.tiles_n; ++tn)
+        if (tm * BM <= tn * BN + BN - 1) ++work;
+  }
+  const int sms = sm_budget();
+  const int waves = (work + sms - 1) / sms;
+  int grid = waves > 0 ? (tiles + waves - 1) / waves : 1;
+  if (grid > sms) grid = sms;
+  if (grid < 1) grid = 1;
+  tgemm_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(maps, p);
   return check_launch("tgemm_kernel");
 }
 

@@ -40,7 +40,7 @@ CHOLINV_SYNC = 1
 # every exported symbol of include/kronq.h
 SYMBOLS = (
     "kronq_status_string", "kronq_last_error_detail", "kronq_version", "kronq_device_check",
-    "kronq_device_error", "kronq_launch_count",
+    "kronq_device_error", "kronq_launch_count", "kronq_set_sm_budget", "kronq_sm_budget",
     "kronq_accumulate_workspace_size", "kronq_accumulate",
     "kronq_biip_workspace_size", "kronq_biip", "kronq_biip_noalloc",
     "kronq_cholinv_workspace_size", "kronq_cholinv",
@@ -83,6 +83,8 @@ def load_library(path: str = LIB_PATH):
         "kronq_device_check": (c_i32, []),
         "kronq_device_error": (c_i32, [c_void_p, c_void_p]),
         "kronq_launch_count": (ctypes.c_uint64, []),
+        "kronq_set_sm_budget": (None, [c_i32]),
+        "kronq_sm_budget": (c_i32, []),
         "kronq_accumulate_workspace_size": (c_sz, [c_i64, c_i32, c_i32, c_i32]),
         "kronq_accumulate": (c_i32, [c_void_p, c_i64, c_void_p, c_i64, c_void_p, c_i64, c_i64,
                                      c_i32, c_i32, c_void_p, c_void_p, c_void_p, c_void_p, c_sz,
@@ -165,6 +167,15 @@ def kronq_device_check():
 
 def kronq_launch_count() -> int:
     return int(load_library().kronq_launch_count())
+
+
+def kronq_set_sm_budget(sms: int) -> None:
+    """At most `sms` CTAs (one per SM) for the persistent kernels launched from now on; 0 = all."""
+    load_library().kronq_set_sm_budget(int(sms))
+
+
+def kronq_sm_budget() -> int:
+    return int(load_library().kronq_sm_budget())
 
 
 def kronq_device_error(stream=None) -> int:
