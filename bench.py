@@ -40,6 +40,12 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="kronq", choices=["kronq", "reference"])
     ap.add_argument("--tokens", type=int, default=None, help=argparse.SUPPRESS)
+    ap.add_argument("--workload", default=WORKLOAD,
+                    choices=["llama2_7b_block", "llama3_8b_block", "llama3_70b_block"],
+                    help="block shape (default: the LLaMA-2-7B block the metric is quoted on)")
+    ap.add_argument("--no-graphs", action="store_true",
+                    help="enqueue the per-sublayer phases eagerly instead of replaying CUDA "
+                         "graphs (each graph keeps its own copies of the phase's outputs)")
     ap.add_argument("--no-e2e", action="store_true", help=argparse.SUPPRESS)
     ap.add_argument("--no-cpu-baseline", action="store_true", help=argparse.SUPPRESS)
     return ap.parse_args()
@@ -180,10 +186,25 @@ class Block:
         self.dev = device
         self.n = n_tokens
         self.ws = ws
-        tag = (WORKLOAD, "rank", rank)
-        self.x = {name: synth.correlated_x(n_tokens, d, synth.seed_for(tag, name, "X"),
-                                           device=device)
-                  for name, d in wl.streams().items()}
+        tag = (wl.name, "rank", rank)
+        self.drift = wl.drift != "none"
+        # X~ (the quantized model's input) in self.x; with the asymmetric term on, also X (the
+        # full-precision model's input) in self.xfp, and D = (X - X~)^T X~ per stream
+        xs = {name: synth.correlated_x(n_tokens, d, synth.seed_for(tag, name, "X"), device=device)
+              for name, d in wl.streams().items()}
+        if self.drift:
+            kind, amount = wl.drift[:3], float(wl.drift[3:])
+            self.xfp = xs
+            self.x = {name: synth.perturbed(x, synth.seed_for(tag, name, "Xq"),
+                                            **({"rel_std": amount} if kind == "rel"
+                                               else {"abs_std": amount}))
+                      for name, x in xs.items()}
+            self.dxx = {name: torch.zeros(d, d, device=device)
+                        for name, d in wl.streams().items()}
+        else:
+            self.xfp = None
+            self.x = xs
+            self.dxx = None
         self.g = {s.name: synth.gradients(n_tokens, s.d_out, synth.seed_for(tag, s.name, "G"),
                                           device=device) for s in wl.sublayers}
         self.w = {s.name: synth.weight(s.d_out, s.d_in, synth.seed_for(tag, s.name, "W"),
@@ -198,10 +219,12 @@ class Block:
         self.acc_events = []        # (start, end, flops) of each statistics call
         self.bits = None
         self.streams = None         # one stream per sublayer for the per-sublayer steps
+        self.use_graphs = True
 
     def input_bytes(self):
         tot = 0
-        for t in list(self.x.values()) + list(self.g.values()) + list(self.w.values()):
+        xfp = list(self.xfp.values()) if self.xfp else []
+        for t in list(self.x.values()) + xfp + list(self.g.values()) + list(self.w.values()):
             tot += t.numel() * t.element_size()
         return tot
 
@@ -213,16 +236,23 @@ class Block:
         wl = self.wl
         x = x_src or self.x
         g = g_src or self.g
+        if not self.use_graphs:
+            self.results = {}       # eager phases allocate new outputs: drop the last step's
         for name, h in self.hx.items():
             h.zero_()
+            if self.drift:
+                self.dxx[name].zero_()
             if time_acc:
                 e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
                 e0.record()
-            P.accumulate(xq=x[name], hx_sum=h, ws=self.ws)
+            P.accumulate(xq=x[name], xfp=self.xfp[name] if self.drift else None, hx_sum=h,
+                         dxx_sum=self.dxx[name] if self.drift else None, ws=self.ws)
             if time_acc:
                 e1.record()
                 d = h.shape[0]
-                self.acc_events.append((e0, e1, self.n * d * (d + 1)))
+                # N d(d+1) for H_X (one triangle), 2 N d^2 for D
+                self.acc_events.append((e0, e1, self.n * d * (d + 1)
+                                        + (2 * self.n * d * d if self.drift else 0)))
         for s in wl.sublayers:
             h = self.hg[s.name]
             h.zero_()
@@ -238,10 +268,13 @@ class Block:
         if self.streams is None:
             # the per-sublayer phases (BiIP; inverse factor + column solve) run side by side on
             # one stream per sublayer, each phase captured once as a CUDA graph and replayed
+            # (or enqueued eagerly every step when graphs are off)
             self.streams = P.SublayerStreams(len(wl.sublayers), self.dev)
-            jobs = [(self.w[s.name], self.hx[s.x_stream], self.hg[s.name], None, inv_n,
+            jobs = [(self.w[s.name], self.hx[s.x_stream], self.hg[s.name],
+                     self.dxx[s.x_stream] if self.drift else None, inv_n,
                      self.si[s.name], self.so[s.name], K.BIIP_FULL) for s in wl.sublayers]
-            self.biip_phase = P.CapturedPhase(lambda: self.streams.biip(jobs))
+            self.biip_phase = (P.CapturedPhase(lambda: self.streams.biip(jobs))
+                               if self.use_graphs else (lambda: self.streams.biip(jobs)))
             self.solve_phases = {}
             self.solve_res = None
         res = self.biip_phase()
@@ -256,6 +289,9 @@ class Block:
         if self.solve_res is not res:       # a new BiIP output set: new solve graphs
             self.solve_res = res
             self.solve_phases = {}
+        if not self.use_graphs:
+            self.streams.solve(res, list(self.bits), 0.01)
+            return
         key = tuple(self.bits)
         if key not in self.solve_phases:
             bits = list(self.bits)
@@ -358,6 +394,20 @@ class Block:
         st["solve"][key]()
 
 
+def describe(wl, n_tok):
+    """The workload in words: shapes, tokens, grid, BiIP, asymmetric term."""
+    shapes = {}
+    for s in wl.sublayers:
+        shapes.setdefault(f"{s.d_out}x{s.d_in}", []).append(s.name.replace("_proj", ""))
+    parts = ", ".join(f"{'/'.join(v)} {k}" for k, v in shapes.items())
+    drift = "drift term off" if wl.drift == "none" else \
+        f"drift term on (X~ = X + noise {wl.drift})"
+    name = {"llama2_7b_block": "LLaMA-2-7B", "llama3_8b_block": "LLaMA-3-8B",
+            "llama3_70b_block": "LLaMA-3-70B"}.get(wl.name, wl.name)
+    return (f"{name}-shaped block: {parts}; {n_tok} tokens; {wl.bits}-bit per-channel grid; "
+            f"BiIP on; {drift}")
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -381,10 +431,11 @@ def run_gpu(args):
     K.load_library()
     K.kronq_device_check()
 
-    wl = synth.WORKLOADS[WORKLOAD]
+    wl = synth.WORKLOADS[args.workload]
     n_tok = args.tokens or wl.n_tokens
     ws = P.Workspace(dev)
     blk = Block(wl, rank, dev, n_tok, ws)
+    blk.use_graphs = not args.no_graphs
     torch.cuda.synchronize()
 
     def barrier():
@@ -420,7 +471,7 @@ def run_gpu(args):
 
     # ---- end to end: host inputs (pinned), host->device copies and the result read-back
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not blk.drift:
         e2e = run_e2e(blk, args, world, dist if world > 1 else None, barrier)
 
     result = None
@@ -440,7 +491,7 @@ def run_gpu(args):
         # launches at d = 4096 and 3 at d = 11008: ncu captures of this kernel version at
         # d = 4096 / 262144 tokens (5.51 GB) and d = 11008 / 131072 tokens (21.2 GB, x2 for
         # 262144 tokens); the accumulate summary under profiles/ has the commands
-        traffic = 15.6e9 if n_tok == 262144 else None
+        traffic = 15.6e9 if (args.workload == WORKLOAD and n_tok == 262144) else None
         acc_tflops = sum(acc_flops) / (sum(acc_ms) / 1e3) / 1e12
         result = {
             "metric": "quantized weight params/s (BiIP+GPTAQ solve); H_X/H_G accumulate TFLOP/s",
@@ -455,12 +506,10 @@ def run_gpu(args):
             "vs_baseline": None,
             "dtype": "bf16 statistics, fp32 solve",
             "data": "synthetic (seeded LLaMA-shaped activations, gradients and weights)",
-            "config": {"workload": "LLaMA-2-7B-shaped block: q/k/v/o 4096x4096, gate/up "
-                                   "11008x4096, down 4096x11008; 262144 tokens; 4-bit "
-                                   "per-channel grid; BiIP on; drift term off",
+            "config": {"workload": describe(wl, n_tok),
                        "tokens": n_tok, "params_per_block": wl.params_per_block,
                        "parallelism": f"one block per GPU x{world}",
-                       "l2": "inputs (34 GB) larger than L2"},
+                       "l2": f"inputs ({blk.input_bytes() / 1e9:.0f} GB) larger than L2"},
             "accumulate_tflops": acc_tflops,
             "roofline": {"bound": "tensor", "kernel": "accumulate_tc_kernel",
                          "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
@@ -470,7 +519,7 @@ def run_gpu(args):
             "clocks": clk,
             "e2e": e2e,
         }
-        if not args.no_cpu_baseline:
+        if not args.no_cpu_baseline and args.workload == WORKLOAD:
             est, desc, threads, spent = oracle_sample()
             result["cpu_baseline"] = {"value": wl.params_per_block / est, "unit": "params/s",
                                       "cores": threads, "kind": "oracle", "sample": desc,

@@ -209,11 +209,11 @@ __global__ void __launch_bounds__(256) fwht_cols_kernel(float* m, int64_t rows, 
 // 64-point over consecutive rows, then (b / 64)-point at row stride 64
 // (H_b = (H_{b/64} (x) I_64)(I_{b/64} (x) H_64)). Every global access is a 128-byte row segment.
 
-// 16-point Walsh-Hadamard butterflies on the low nbits bits of the register index.
-__device__ __forceinline__ void fwht16(float (&x)[16], int nbits) {
+// 16-point Walsh-Hadamard butterflies on register-index bits [h0, h0 + nbits).
+__device__ __forceinline__ void fwht16(float (&x)[16], int nbits, int h0 = 0) {
 #pragma unroll
   for (int h = 0; h < 4; ++h) {
-    if (h < nbits) {
+    if (h >= h0 && h < h0 + nbits) {
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         if (j & (1 << h)) continue;
@@ -291,14 +291,20 @@ __global__ void __launch_bounds__(1024) fwht_rows_reg_kernel(
   }
 #pragma unroll
   for (int k = 0; k < 16; ++k) sb[pad16(16 * t + k)] = x[k];
+  // log2 of the chunk: every round's 16-element window must stay inside it
+  const int log2c = 31 - __clz(chunk);
   for (int R = 1; R < rounds; ++R) {
     __syncthreads();
-    const int sh = 4 * R, s = 1 << sh;
+    // round R transforms index bits [4R, min(4R + 4, log2b)); its window of 4 index bits starts
+    // at 4R, or lower when that would leave the chunk (the last round of b > 4096), in which
+    // case the bits below 4R ride along untouched
+    const int nbits = log2b - 4 * R < 4 ? log2b - 4 * R : 4;
+    const int sh = 4 * R + 4 <= log2c ? 4 * R : log2c - 4;
+    const int s = 1 << sh;
     const int lo = (t & (s - 1)) + ((t >> sh) << (sh + 4));
 #pragma unroll
     for (int k = 0; k < 16; ++k) x[k] = sb[pad16(lo + s * k)];
-    const int nbits = log2b - sh < 4 ? log2b - sh : 4;
-    fwht16(x, nbits);
+    fwht16(x, nbits, 4 * R - sh);
     if (R == rounds - 1) {
 #pragma unroll
       for (int k = 0; k < 16; ++k) {

@@ -27,7 +27,8 @@ namespace {
 
 constexpr int QB = 128;        // column block
 constexpr int QSB = 1024;      // super-block: the rest of W is updated once per QSB columns
-constexpr int QROWS = 32;      // rows per CTA in the block solve
+constexpr int RPL = 1;         // rows per lane in the block solve
+constexpr int QROWS = 32 * RPL; // rows per CTA in the block solve
 constexpr int QT = 4;          // warps per CTA: one column quarter each
 constexpr int QW = QB / QT;    // columns per thread
 constexpr int KS_LD = QB + 4;  // row of the K block in shared memory (16-byte aligned)
@@ -67,17 +68,18 @@ __global__ void striu_kernel(float* __restrict__ m, int d) {
     m[static_cast<int64_t>(i) * d + j] = 0.f;
 }
 
-// One 128-column block of the solve for QROWS rows: lane l of every warp owns row
-// blockIdx.x * QROWS + l, and warp q owns the block's column quarter [32q, 32q + 32) of it, in
-// registers. Quarter by quarter, its warp walks the 32 columns in order (quantize, scaled error,
-// update its own columns to the right) with no exchange, parks the errors in shared memory, and
-// after one barrier every later quarter subtracts those 32 errors times the matching K rows.
-// K rows are read as broadcasts (every lane of a warp reads the same row), so the solve is bound
-// by the per-column dependency chain, not by shared memory.
+// One 128-column block of the solve for QROWS = 32 * RPL rows: lane l of every warp owns rows
+// blockIdx.x * QROWS + 32 r + l (r < RPL), and warp q owns the block's column quarter
+// [32q, 32q + 32) of them, in registers. Quarter by quarter, its warp walks the 32 columns in order (quantize,
+// scaled error, update its own columns to the right) with no exchange, parks the errors in
+// shared memory, and after one barrier every later quarter subtracts those 32 errors times the
+// matching K rows. K rows are read as broadcasts (every lane of a warp reads the same row) and
+// serve all of a lane's rows. With RPL = 1 the solve is bound by the per-column dependency
+// chain; RPL = 2 halves the CTAs but measured slower (the lane's instruction stream doubles).
 //   w_hat  d_out x d_in running weights (in: current values, out: dequantized for the block)
 //   delta  d_out x QB errors scaled by 1/K_pp (row stride ldd), written as three bf16 pieces
 //          (the operand of the lazy trailing updates on the tensor cores)
-__global__ void __launch_bounds__(QROWS * QT) block_solve_kernel(
+__global__ void __launch_bounds__(32 * QT) block_solve_kernel(
     float* __restrict__ w_hat, const float* __restrict__ k, int d_out, int d_in, int b0, int bw,
     const float* __restrict__ scale, const float* __restrict__ zero, float maxq,
     uint8_t* __restrict__ codes, uint16_t* __restrict__ delta0, uint16_t* __restrict__ delta1,
@@ -89,8 +91,6 @@ __global__ void __launch_bounds__(QROWS * QT) block_solve_kernel(
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int q = tid >> 5;              // column quarter of this warp
-  const int row = blockIdx.x * QROWS + lane;
-  const bool active = row < d_out;
 
   // K block (rows/cols beyond bw become identity so that padding never feeds back)
   const bool kvec = (d_in % 4 == 0) && bw == QB && (reinterpret_cast<uintptr_t>(k) & 15u) == 0;
@@ -116,27 +116,31 @@ __global__ void __launch_bounds__(QROWS * QT) block_solve_kernel(
   __syncthreads();
   if (tid < QB) Rd[tid] = 1.f / Ks[tid * KS_LD + tid];
 
-  // this lane's 32 columns of its row
-  float w[QW];
-  float* wrow = w_hat + static_cast<int64_t>(row) * d_in + b0 + QW * q;
-  const bool wvec = active && bw == QB && ((reinterpret_cast<uintptr_t>(wrow) & 15u) == 0);
-  if (wvec) {
+  // this lane's 32 columns of each of its rows
+  float w[RPL][QW];
+  float sc[RPL], zr[RPL];
+  uint32_t packed[RPL][QW / 4];
 #pragma unroll
-    for (int j = 0; j < QW; j += 4) {
-      const float4 v = *reinterpret_cast<const float4*>(wrow + j);
-      w[j] = v.x; w[j + 1] = v.y; w[j + 2] = v.z; w[j + 3] = v.w;
+  for (int r = 0; r < RPL; ++r) {
+    const int row = blockIdx.x * QROWS + 32 * r + lane;
+    const bool active = row < d_out;
+    const float* wrow = w_hat + static_cast<int64_t>(row) * d_in + b0 + QW * q;
+    const bool wvec = active && bw == QB && ((reinterpret_cast<uintptr_t>(wrow) & 15u) == 0);
+    if (wvec) {
+#pragma unroll
+      for (int j = 0; j < QW; j += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(wrow + j);
+        w[r][j] = v.x; w[r][j + 1] = v.y; w[r][j + 2] = v.z; w[r][j + 3] = v.w;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < QW; ++j) w[r][j] = (active && QW * q + j < bw) ? wrow[j] : 0.f;
     }
-  } else {
+    sc[r] = active ? scale[row] : 1.f;
+    zr[r] = active ? zero[row] : 0.f;
 #pragma unroll
-    for (int j = 0; j < QW; ++j) w[j] = (active && QW * q + j < bw) ? wrow[j] : 0.f;
+    for (int j = 0; j < QW / 4; ++j) packed[r][j] = 0u;
   }
-  const float sc = active ? scale[row] : 1.f;
-  const float zr = active ? zero[row] : 0.f;
-  float err[QW];
-  uint32_t packed[QW / 4];
-#pragma unroll
-  for (int j = 0; j < QW / 4; ++j) packed[j] = 0u;
-  float* erow = E + lane * E_LD;
   __syncthreads();   // Rd
 
   for (int qo = 0; qo < QT; ++qo) {
@@ -144,66 +148,85 @@ __global__ void __launch_bounds__(QROWS * QT) block_solve_kernel(
 #pragma unroll
       for (int lp = 0; lp < QW; ++lp) {
         const int p = QW * qo + lp;
-        const float t = __fdiv_rn(w[lp], sc);
-        float code = __fadd_rn(rintf(t), zr);
-        code = fminf(fmaxf(code, 0.f), maxq);
-        const float dq = __fmul_rn(sc, __fsub_rn(code, zr));
-        const float e = __fsub_rn(w[lp], dq) * Rd[p];
-        w[lp] = dq;
-        err[lp] = e;
-        erow[p] = e;
-        packed[lp / 4] |= (static_cast<uint32_t>(code) & 0xFFu) << (8 * (lp % 4));
+        float e[RPL];
+#pragma unroll
+        for (int r = 0; r < RPL; ++r) {
+          const float t = __fdiv_rn(w[r][lp], sc[r]);
+          float code = __fadd_rn(rintf(t), zr[r]);
+          code = fminf(fmaxf(code, 0.f), maxq);
+          const float dq = __fmul_rn(sc[r], __fsub_rn(code, zr[r]));
+          e[r] = __fsub_rn(w[r][lp], dq) * Rd[p];
+          w[r][lp] = dq;
+          E[(32 * r + lane) * E_LD + p] = e[r];
+          packed[r][lp / 4] |= (static_cast<uint32_t>(code) & 0xFFu) << (8 * (lp % 4));
+        }
         // own columns right of lp (a compile-time range)
         const float4* kr = reinterpret_cast<const float4*>(Ks + p * KS_LD + QW * qo);
 #pragma unroll
         for (int j4 = 0; j4 < QW / 4; ++j4) {
           if (4 * j4 + 3 <= lp) continue;
           const float4 kv = kr[j4];
-          if (4 * j4 > lp) w[4 * j4] = fmaf(-e, kv.x, w[4 * j4]);
-          if (4 * j4 + 1 > lp) w[4 * j4 + 1] = fmaf(-e, kv.y, w[4 * j4 + 1]);
-          if (4 * j4 + 2 > lp) w[4 * j4 + 2] = fmaf(-e, kv.z, w[4 * j4 + 2]);
-          if (4 * j4 + 3 > lp) w[4 * j4 + 3] = fmaf(-e, kv.w, w[4 * j4 + 3]);
+#pragma unroll
+          for (int r = 0; r < RPL; ++r) {
+            if (4 * j4 > lp) w[r][4 * j4] = fmaf(-e[r], kv.x, w[r][4 * j4]);
+            if (4 * j4 + 1 > lp) w[r][4 * j4 + 1] = fmaf(-e[r], kv.y, w[r][4 * j4 + 1]);
+            if (4 * j4 + 2 > lp) w[r][4 * j4 + 2] = fmaf(-e[r], kv.z, w[r][4 * j4 + 2]);
+            if (4 * j4 + 3 > lp) w[r][4 * j4 + 3] = fmaf(-e[r], kv.w, w[r][4 * j4 + 3]);
+          }
         }
       }
     }
     __syncthreads();
     if (q > qo) {
       // the finished quarter's 32 errors, applied to this warp's columns
-#pragma unroll 4
+#pragma unroll 2
       for (int p = QW * qo; p < QW * qo + QW; ++p) {
-        const float e = erow[p];
+        float e[RPL];
+#pragma unroll
+        for (int r = 0; r < RPL; ++r) e[r] = E[(32 * r + lane) * E_LD + p];
         const float4* kr = reinterpret_cast<const float4*>(Ks + p * KS_LD + QW * q);
 #pragma unroll
         for (int j4 = 0; j4 < QW / 4; ++j4) {
           const float4 kv = kr[j4];
-          w[4 * j4] = fmaf(-e, kv.x, w[4 * j4]);
-          w[4 * j4 + 1] = fmaf(-e, kv.y, w[4 * j4 + 1]);
-          w[4 * j4 + 2] = fmaf(-e, kv.z, w[4 * j4 + 2]);
-          w[4 * j4 + 3] = fmaf(-e, kv.w, w[4 * j4 + 3]);
+#pragma unroll
+          for (int r = 0; r < RPL; ++r) {
+            w[r][4 * j4] = fmaf(-e[r], kv.x, w[r][4 * j4]);
+            w[r][4 * j4 + 1] = fmaf(-e[r], kv.y, w[r][4 * j4 + 1]);
+            w[r][4 * j4 + 2] = fmaf(-e[r], kv.z, w[r][4 * j4 + 2]);
+            w[r][4 * j4 + 3] = fmaf(-e[r], kv.w, w[r][4 * j4 + 3]);
+          }
         }
       }
     }
   }
+  __syncthreads();   // every quarter's errors are in E
 
-  if (active) {
+#pragma unroll
+  for (int r = 0; r < RPL; ++r) {
+    const int row = blockIdx.x * QROWS + 32 * r + lane;
+    if (row >= d_out) continue;
+    float* wrow = w_hat + static_cast<int64_t>(row) * d_in + b0 + QW * q;
+    const bool wvec = bw == QB && ((reinterpret_cast<uintptr_t>(wrow) & 15u) == 0);
     if (wvec) {
 #pragma unroll
       for (int j = 0; j < QW; j += 4)
-        *reinterpret_cast<float4*>(wrow + j) = make_float4(w[j], w[j + 1], w[j + 2], w[j + 3]);
+        *reinterpret_cast<float4*>(wrow + j) =
+            make_float4(w[r][j], w[r][j + 1], w[r][j + 2], w[r][j + 3]);
     } else {
 #pragma unroll
       for (int j = 0; j < QW; ++j)
-        if (QW * q + j < bw) wrow[j] = w[j];
+        if (QW * q + j < bw) wrow[j] = w[r][j];
     }
-    // the errors, split into three bf16 pieces for the tensor-core trailing update
-    // (8 columns per 16-byte store; the row's 32 columns start on a 64-byte boundary)
+    // the errors of this quarter, split into three bf16 pieces for the tensor-core trailing
+    // update (8 columns per 16-byte store; the row's 32 columns start on a 64-byte boundary)
+    const float* er = E + (32 * r + lane) * E_LD + QW * q;
     const int64_t o = static_cast<int64_t>(row) * ldd + QW * q;
 #pragma unroll
     for (int j8 = 0; j8 < QW; j8 += 8) {
       uint32_t h0[4], h1[4], h2[4];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        const float dv = QW * q + j8 + u < bw ? err[j8 + u] : 0.f;
+        const float dv = QW * q + j8 + u < bw ? er[j8 + u] : 0.f;
         const __nv_bfloat16 p0 = __float2bfloat16_rn(dv);
         const float r1 = dv - __bfloat162float(p0);
         const __nv_bfloat16 p1 = __float2bfloat16_rn(r1);
@@ -220,11 +243,15 @@ __global__ void __launch_bounds__(QROWS * QT) block_solve_kernel(
     }
     uint8_t* cr = codes + static_cast<int64_t>(row) * d_in + b0 + QW * q;
     if (bw == QB && (reinterpret_cast<uintptr_t>(cr) & 15u) == 0) {
-      reinterpret_cast<uint4*>(cr)[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-      reinterpret_cast<uint4*>(cr)[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+      reinterpret_cast<uint4*>(cr)[0] =
+          make_uint4(packed[r][0], packed[r][1], packed[r][2], packed[r][3]);
+      reinterpret_cast<uint4*>(cr)[1] =
+          make_uint4(packed[r][4], packed[r][5], packed[r][6], packed[r][7]);
     } else {
+#pragma unroll
       for (int j = 0; j < QW; ++j)
-        if (QW * q + j < bw) cr[j] = static_cast<uint8_t>((packed[j >> 2] >> (8 * (j & 3))) & 0xFFu);
+        if (QW * q + j < bw)
+          cr[j] = static_cast<uint8_t>((packed[r][j >> 2] >> (8 * (j & 3))) & 0xFFu);
     }
   }
 }
@@ -317,7 +344,7 @@ kronq_status run_quantize(const float* w, const float* k, const float* dxx, int 
     for (int b0 = s0; b0 < s1; b0 += QB) {
       const int bw = d_in - b0 < QB ? d_in - b0 : QB;
       const Split3 db = offset(ds, 0, b0 - s0);
-      block_solve_kernel<<<(d_out + QROWS - 1) / QROWS, QROWS * QT, smem, stream>>>(
+      block_solve_kernel<<<(d_out + QROWS - 1) / QROWS, 32 * QT, smem, stream>>>(
           w_hat, k, d_out, d_in, b0, bw, scale, zero, maxq, codes, db.part[0], db.part[1],
           db.part[2], db.ld);
       KQ_TRY(check_launch("block_solve_kernel"));

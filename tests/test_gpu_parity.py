@@ -378,19 +378,24 @@ def test_drift_term_llama3_8b_width(K):
         assert rel(h64(hx[i0:i0 + 128, j0:j0 + 128]), qa.T @ qb) <= TOL
 
 
-def test_biip_llama3_70b_down_shape(K, P):
-    # down_proj of LLaMA-3-70B: 8192 x 28672 (input Hadamard blocks of 4096, output 8192).
-    # Full-size check through the inverse transforms: (U^T W' V)_ij = s_g,i W_ij s_x,j on
-    # sampled entries, each from a b_out x b_in block of W'; plus the oracle's scales.
-    d_out, d_in, n = 8192, 28672, 2048
-    x = synth.correlated_x(n, d_in, synth.seed_for("b70", "X"), device="cuda")
-    g = synth.gradients(n, d_out, synth.seed_for("b70", "G"), device="cuda")
-    w = synth.weight(d_out, d_in, synth.seed_for("b70", "W"), device="cuda")
-    si = synth.rademacher(d_in, synth.seed_for("b70", "si"), device="cuda")
-    so = synth.rademacher(d_out, synth.seed_for("b70", "so"), device="cuda")
+@pytest.mark.parametrize("d_out,d_in", [(8192, 28672), (1024, 8192), (16384, 16384)])
+def test_biip_llama3_70b_shapes(K, P, d_out, d_in):
+    # LLaMA-3-70B shapes: down_proj 8192 x 28672 (input Hadamard blocks of 4096, output 8192),
+    # k/v 1024 x 8192 (input blocks of 8192: the row pass's widest chunk), and 16384-wide blocks
+    # on both sides. Full-size check through the inverse transforms:
+    # (U^T W' V)_ij = s_g,i W_ij s_x,j and (V^T H_X' V)_ij = (S_X^-1 H_X S_X^-1 / n)_ij on sampled
+    # entries, each from one b x b block; plus the oracle's scales.
+    n = 2048
+    tag = ("b70", d_out, d_in) if d_in != 28672 else "b70"
+    x = synth.correlated_x(n, d_in, synth.seed_for(tag, "X"), device="cuda")
+    g = synth.gradients(n, d_out, synth.seed_for(tag, "G"), device="cuda")
+    w = synth.weight(d_out, d_in, synth.seed_for(tag, "W"), device="cuda")
+    si = synth.rademacher(d_in, synth.seed_for(tag, "si"), device="cuda")
+    so = synth.rademacher(d_out, synth.seed_for(tag, "so"), device="cuda")
     hx = torch.zeros(d_in, d_in, device="cuda"); hg = torch.zeros(d_out, d_out, device="cuda")
     K.kronq_accumulate(x, None, g, hx, hg)
     hx_diag = torch.diagonal(hx).clone(); hg_diag = torch.diagonal(hg).clone()
+    hx_orig = hx.clone()
     r = P.biip(w, hx, hg, None, 1.0 / n, si, so, 15, copy_hx=False)
     torch.cuda.synchronize()
     w64 = h64(w)
@@ -401,22 +406,54 @@ def test_biip_llama3_70b_down_shape(K, P):
     tr_hx = float(np.sum(h64(hx_diag) / n / sx ** 2))
     assert abs(float(r.tr[0]) - tr_hx) <= TOL * tr_hx
     bi, bo = O.hadamard_block_size(d_in), O.hadamard_block_size(d_out)
-    hb_i = O.sylvester(bi) / math.sqrt(bi); hb_o = O.sylvester(bo) / math.sqrt(bo)
+
+    class _Cols:
+        # column k of the normalised Sylvester matrix, (-1)^popcount(i & k) / sqrt(b), built
+        # on demand (the b = 16384 matrix would be 2 GB in fp64)
+        def __init__(self, b):
+            self.b = b
+            self.i = np.arange(b, dtype=np.uint32)
+
+        def __getitem__(self, key):
+            _, k = key
+            par = np.bitwise_count(self.i & np.uint32(k)) & 1
+            return (1.0 - 2.0 * par.astype(np.float64)) / math.sqrt(self.b)
+
+    hb_i = _Cols(bi); hb_o = _Cols(bo)
+    # the on-demand columns agree with the oracle's Sylvester matrix
+    small = O.sylvester(64) / 8.0
+    assert all(np.array_equal(_Cols(64)[:, k], small[:, k]) for k in range(64))
     sin = h64(si); sout = h64(so)
     rng = np.random.default_rng(70)
     got, want = [], []
+    def bilinear(mat, ib, jb, b1, b2, u, v):
+        # u^T mat[ib:ib+b1, jb:jb+b2] v in fp64, on the device (the blocks can be 1 GB)
+        blk = mat[ib:ib + b1, jb:jb + b2].double()
+        uu = torch.from_numpy(u).to(blk.device); vv = torch.from_numpy(v).to(blk.device)
+        return float(uu @ (blk @ vv))
+
     for _ in range(24):
         i = int(rng.integers(0, d_out)); j = int(rng.integers(0, d_in))
         ib, jb = (i // bo) * bo, (j // bi) * bi
-        blk = h64(r.w_prime[ib:ib + bo, jb:jb + bi])
         u_i = hb_o[:, i - ib] * sout[i]          # column i of U = (1/sqrt b)(H_b) diag(sign)
         v_j = hb_i[:, j - jb] * sin[j]
-        got.append(u_i @ blk @ v_j)
+        got.append(bilinear(r.w_prime, ib, jb, bo, bi, u_i, v_j))
         want.append(sg[i] * w64[i, j] * sx[j])
     assert rel(np.array(got), np.array(want)) <= TOL
     # the rotation preserves the Frobenius norm of S_G W S_X
     nrm = float(torch.linalg.vector_norm(r.w_prime.double()))
     assert abs(nrm - np.linalg.norm(sg[:, None] * w64 * sx[None, :])) <= TOL * nrm
+    # H_X' through the inverse input transform, on sampled entries
+    got, want = [], []
+    for _ in range(16):
+        i = int(rng.integers(0, d_in)); j = int(rng.integers(0, d_in))
+        ib, jb = (i // bi) * bi, (j // bi) * bi
+        v_i = hb_i[:, i - ib] * sin[i]
+        v_j = hb_i[:, j - jb] * sin[j]
+        got.append(bilinear(r.hx, ib, jb, bi, bi, v_i, v_j))
+        want.append(float(hx_orig[i, j]) / n / (sx[i] * sx[j]))
+    scale = float(np.max(np.abs(want)))
+    assert np.max(np.abs(np.array(got) - np.array(want))) <= TOL * scale
 
 
 def test_cholinv_llama3_70b_width(K):
