@@ -258,112 +258,259 @@ __device__ __forceinline__ void load16(const __nv_bfloat16* p, bool vec, float (
   }
 }
 
-// src may equal dst (every element is read before the chunk's first write).
-template <typename T>
-__global__ void __launch_bounds__(1024) fwht_rows_reg_kernel(
+// src may equal dst: a chunk is read (the prefetch one iteration earlier) only by the CTA that
+// writes it, before it writes it. A CTA walks chunks grid-stride with two staging buffers: the
+// next chunk streams in (cp.async, no registers) while the current one is transformed and stored.
+// vec = 0 (unaligned operands) takes plain loads instead.
+template <typename T, int NT>
+__global__ void __launch_bounds__(NT) fwht_rows_reg_kernel(
     const T* src, float* dst, int64_t total, int64_t cols, const float* __restrict__ row_f,
     const float* __restrict__ col_f, float scalar, int log2b, int chunk, float out_scale,
     int vec) {
-  extern __shared__ float sb[];
+  extern __shared__ __align__(16) float sb[];
+  float* work = sb;                                                   // padded, chunk + chunk/16
+  T* stage = reinterpret_cast<T*>(sb + chunk + chunk / 16);           // 2 x chunk elements
+  constexpr int PIECES = 16 * sizeof(T) / 16;                         // 16-byte pieces per thread
   const int t = threadIdx.x;
-  const int64_t base = static_cast<int64_t>(blockIdx.x) * chunk;
-  const int rounds = (log2b + 3) >> 2;
-  float x[16];
-  const int64_t f0 = base + 16 * t;
-  if (f0 < total) {   // total is a multiple of b >= 16, so a group is all in or all out
-    load16(src + f0, vec != 0, x);
-    const int64_t r = f0 / cols;
-    const int64_t c0 = f0 - r * cols;
-    const float rf = row_f ? scalar * row_f[r] : scalar;
-#pragma unroll
-    for (int k = 0; k < 16; ++k) x[k] *= col_f ? rf * col_f[c0 + k] : rf;
-  } else {
-#pragma unroll
-    for (int k = 0; k < 16; ++k) x[k] = 0.f;
-  }
-  fwht16(x, log2b < 4 ? log2b : 4);
-  if (rounds == 1) {
-    if (f0 < total) {
-#pragma unroll
-      for (int k = 0; k < 16; ++k) dst[f0 + k] = x[k] * out_scale;
-    }
-    return;
-  }
-#pragma unroll
-  for (int k = 0; k < 16; ++k) sb[pad16(16 * t + k)] = x[k];
-  // log2 of the chunk: every round's 16-element window must stay inside it
+  // log2 of the chunk: every shared-memory window must stay inside it
   const int log2c = 31 - __clz(chunk);
-  for (int R = 1; R < rounds; ++R) {
-    __syncthreads();
-    // round R transforms index bits [4R, min(4R + 4, log2b)); its window of 4 index bits starts
-    // at 4R, or lower when that would leave the chunk (the last round of b > 4096), in which
-    // case the bits below 4R ride along untouched
-    const int nbits = log2b - 4 * R < 4 ? log2b - 4 * R : 4;
-    const int sh = 4 * R + 4 <= log2c ? 4 * R : log2c - 4;
-    const int s = 1 << sh;
-    const int lo = (t & (s - 1)) + ((t >> sh) << (sh + 4));
+  const int64_t nchunks = (total + chunk - 1) / chunk;
+  auto fetch = [&](int64_t c, T* buf) {
+    const int64_t f = c * chunk + 16 * t;
+    if (f < total) {   // total is a multiple of b >= 16: a group of 16 is all in or all out
 #pragma unroll
-    for (int k = 0; k < 16; ++k) x[k] = sb[pad16(lo + s * k)];
-    fwht16(x, nbits, 4 * R - sh);
-    if (R == rounds - 1) {
-#pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const int64_t f = base + lo + static_cast<int64_t>(s) * k;
-        if (f < total) dst[f] = x[k] * out_scale;
+      for (int q = 0; q < PIECES; ++q) {
+        const uint32_t d = static_cast<uint32_t>(
+            __cvta_generic_to_shared(reinterpret_cast<uint8_t*>(buf + 16 * t) + 16 * q));
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d),
+                     "l"(reinterpret_cast<const uint8_t*>(src + f) + 16 * q)
+                     : "memory");
       }
+    }
+  };
+  int cur = 0;
+  int64_t ch = blockIdx.x;
+  if (vec && ch < nchunks) fetch(ch, stage);
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  for (; ch < nchunks; ch += gridDim.x) {
+    const int64_t f0 = ch * chunk + 16 * t;
+    const bool in = f0 < total;
+    float x[16];
+    if (vec) {
+      if (ch + gridDim.x < nchunks) fetch(ch + gridDim.x, stage + (cur ^ 1) * chunk);
+      asm volatile("cp.async.commit_group;" ::: "memory");
+      asm volatile("cp.async.wait_group 1;" ::: "memory");   // this thread's pieces landed
+      if (in) {
+        load16(stage + cur * chunk + 16 * t, true, x);
+      } else {
+#pragma unroll
+        for (int k = 0; k < 16; ++k) x[k] = 0.f;
+      }
+    } else if (in) {
+      load16(src + f0, false, x);
     } else {
 #pragma unroll
-      for (int k = 0; k < 16; ++k) sb[pad16(lo + s * k)] = x[k];
+      for (int k = 0; k < 16; ++k) x[k] = 0.f;
     }
+    if (in) {
+      int64_t r;
+      if (total < (int64_t(1) << 31))
+        r = static_cast<uint32_t>(f0) / static_cast<uint32_t>(cols);
+      else
+        r = f0 / cols;
+      const int64_t c0 = f0 - r * cols;
+      const float rf = row_f ? scalar * row_f[r] : scalar;
+      if (col_f) {
+        float cf[16];
+        load16(col_f + c0, true, cf);  // 16-byte aligned: workspace base, c0 a multiple of 16
+#pragma unroll
+        for (int k = 0; k < 16; ++k) x[k] *= rf * cf[k];
+      } else {
+#pragma unroll
+        for (int k = 0; k < 16; ++k) x[k] *= rf;
+      }
+    }
+    // index bits 0-3: this thread's registers
+    fwht16(x, log2b < 4 ? log2b : 4);
+    // index bits 4-8: the lanes of the warp (lane = bits 4-8 of 16 t)
+    const int lane = t & 31;
+    for (int h = 4; h < log2b && h < 9; ++h) {
+      const int o = 1 << (h - 4);
+      const bool upper = (lane & o) != 0;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const float other = __shfl_xor_sync(0xffffffffu, x[k], o);
+        x[k] = upper ? other - x[k] : x[k] + other;
+      }
+    }
+    // index bits 9 and up: across warps, through shared memory in windows of four bits
+    if (log2b > 9) {
+#pragma unroll
+      for (int k = 0; k < 16; ++k) work[pad16(16 * t + k)] = x[k];
+      for (int hs = 9; hs < log2b; hs += 4) {
+        __syncthreads();
+        // the window of 4 index bits starts at hs, or lower when that would leave the chunk;
+        // bits below hs ride along untouched
+        const int nbits = log2b - hs < 4 ? log2b - hs : 4;
+        const int sh = hs + 4 <= log2c ? hs : log2c - 4;
+        const int s = 1 << sh;
+        const int lo = (t & (s - 1)) + ((t >> sh) << (sh + 4));
+#pragma unroll
+        for (int k = 0; k < 16; ++k) x[k] = work[pad16(lo + s * k)];
+        fwht16(x, nbits, hs - sh);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) work[pad16(lo + s * k)] = x[k];
+      }
+      // back to the first layout: 16 consecutive elements per thread
+      __syncthreads();
+#pragma unroll
+      for (int k = 0; k < 16; ++k) x[k] = work[pad16(16 * t + k)];
+    }
+    if (in) {
+      if (vec) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          reinterpret_cast<float4*>(dst + f0)[q] =
+              make_float4(x[4 * q] * out_scale, x[4 * q + 1] * out_scale,
+                          x[4 * q + 2] * out_scale, x[4 * q + 3] * out_scale);
+      } else {
+#pragma unroll
+        for (int k = 0; k < 16; ++k) dst[f0 + k] = x[k] * out_scale;
+      }
+    }
+    if (log2b > 9) __syncthreads();   // the next chunk overwrites the work buffer
+    cur ^= 1;
   }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
-// P-point transform along rows r_base + rs * j of 32 columns, in place; 2P threads.
+// P-point transform along rows r_base + rs * j of 32-column tiles, in place; 2P threads. The
+// tiles move between global and shared memory in 16-byte pieces (8 per row, 128-byte row
+// segments); the butterflies read and write them column by column in shared memory. A CTA walks
+// tiles grid-stride with two tile buffers: the next tile streams in (cp.async, no registers)
+// while the current one is transformed and stored, so HBM stays busy through the butterflies.
+// vec = 0 (unaligned or ragged columns) takes plain loads into the current buffer instead.
 constexpr int kColTile = 32;
+constexpr int kColLd = kColTile + 4;   // 16-byte aligned rows
+
+__device__ __forceinline__ void cp_async16(float* smem_dst, const float* gmem_src) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
 __global__ void __launch_bounds__(512) fwht_cols_reg_kernel(float* m, int64_t rows, int64_t cols,
-                                                            int log2p, int rs, float out_scale) {
-  extern __shared__ float sb[];
+                                                            int log2p, int rs, float out_scale,
+                                                            int vec) {
+  extern __shared__ __align__(16) float sb[];
   const int P = 1 << log2p;
+  const int nt = 2 * P;
   const int t = threadIdx.x;
-  const int c = t & (kColTile - 1);
-  const int64_t col = static_cast<int64_t>(blockIdx.x) * kColTile + c;
-  const bool cin = col < cols;
-  const int y = blockIdx.y;
-  const int64_t r_base = static_cast<int64_t>(y / rs) * P * rs + (y % rs);
-  constexpr int LDT = kColTile + 1;
-  float x[16];
-  {
-    const int jg = t / kColTile;   // round 0: rows 16 jg .. 16 jg + 15
+  const int tiles_x = static_cast<int>((cols + kColTile - 1) / kColTile);
+  const int num_tiles = tiles_x * static_cast<int>(rows / P);
+  // top-left of a tile (its first row, r_base + rs * 0, and first column)
+  auto origin = [&](int tile, int64_t& col0) {
+    const int y = tile / tiles_x;
+    col0 = static_cast<int64_t>(tile - y * tiles_x) * kColTile;
+    const int64_t r_base = static_cast<int64_t>(y / rs) * P * rs + (y % rs);
+    return m + r_base * cols + col0;
+  };
+  // piece u of this thread in a tile: e = t + nt * u, row j = e / 8, columns 4 (e % 8) ..
+  const int64_t row_step = static_cast<int64_t>(rs) * cols;
+  auto gaddr = [&](float* org, int64_t col0, int u, int64_t& gc) {
+    const int e = t + nt * u, j = e >> 3, c4 = (e & 7) * 4;
+    gc = col0 + c4;
+    return org + j * row_step + c4;
+  };
+  auto soff = [&](int u) {
+    const int e = t + nt * u;
+    return (e >> 3) * kColLd + (e & 7) * 4;
+  };
+  auto fetch_async = [&](int tile, float* buf) {
+    int64_t col0;
+    float* org = origin(tile, col0);
 #pragma unroll
-    for (int k = 0; k < 16; ++k)
-      x[k] = cin ? m[(r_base + static_cast<int64_t>(rs) * (16 * jg + k)) * cols + col] : 0.f;
+    for (int u = 0; u < 4; ++u) {
+      int64_t gc;
+      const float* src = gaddr(org, col0, u, gc);
+      cp_async16(buf + soff(u), src);
+    }
+  };
+  auto fetch_plain = [&](int tile, float* buf) {
+    int64_t col0;
+    float* org = origin(tile, col0);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      int64_t gc;
+      const float* src = gaddr(org, col0, u, gc);
+      float* d = buf + soff(u);
+      d[0] = gc < cols ? src[0] : 0.f;
+      d[1] = gc + 1 < cols ? src[1] : 0.f;
+      d[2] = gc + 2 < cols ? src[2] : 0.f;
+      d[3] = gc + 3 < cols ? src[3] : 0.f;
+    }
+  };
+  const int tile_floats = P * kColLd;
+  int cur = 0;
+  int tile = blockIdx.x;
+  if (vec && tile < num_tiles) fetch_async(tile, sb);
+  cp_async_commit();
+  const int c = t & (kColTile - 1), jg = t / kColTile;
+  for (; tile < num_tiles; tile += gridDim.x) {
+    float* buf = sb + cur * tile_floats;
+    if (vec) {
+      if (tile + gridDim.x < num_tiles) fetch_async(tile + gridDim.x, sb + (cur ^ 1) * tile_floats);
+      cp_async_commit();
+      cp_async_wait1();            // this tile's group has landed (the next may be in flight)
+    } else {
+      fetch_plain(tile, buf);
+    }
+    __syncthreads();
+    float x[16];
+    // round 0: bits 0-3 of j (rows 16 jg .. 16 jg + 15 of column c)
+#pragma unroll
+    for (int k = 0; k < 16; ++k) x[k] = buf[(16 * jg + k) * kColLd + c];
     fwht16(x, 4);
-    if (log2p == 4) {
-      if (cin) {
 #pragma unroll
-        for (int k = 0; k < 16; ++k)
-          m[(r_base + static_cast<int64_t>(rs) * (16 * jg + k)) * cols + col] = x[k] * out_scale;
+    for (int k = 0; k < 16; ++k) buf[(16 * jg + k) * kColLd + c] = x[k];
+    if (log2p > 4) {
+      __syncthreads();
+      // round 1: bits 4.. of j; groups (c, jl), jl in [0, 16), P / 16 elements each
+      const int M = P >> 4, per = 256 / P;
+      for (int w = 0; w < per; ++w) {
+        const int jl = jg * per + w;
+#pragma unroll
+        for (int mm = 0; mm < 16; ++mm) x[mm] = mm < M ? buf[(jl + 16 * mm) * kColLd + c] : 0.f;
+        fwht16(x, log2p - 4);
+#pragma unroll
+        for (int mm = 0; mm < 16; ++mm)
+          if (mm < M) buf[(jl + 16 * mm) * kColLd + c] = x[mm];
       }
-      return;
     }
+    __syncthreads();
+    int64_t col0;
+    float* org = origin(tile, col0);
 #pragma unroll
-    for (int k = 0; k < 16; ++k) sb[(16 * jg + k) * LDT + c] = x[k];
-  }
-  __syncthreads();
-  // round 1: bits 4.. of j; groups (c, jl), jl in [0, 16), P / 16 elements each
-  const int M = P >> 4, per = 256 / P, q = t / kColTile;
-  for (int u = 0; u < per; ++u) {
-    const int jl = q * per + u;
-#pragma unroll
-    for (int mm = 0; mm < 16; ++mm) x[mm] = mm < M ? sb[(jl + 16 * mm) * LDT + c] : 0.f;
-    fwht16(x, log2p - 4);
-    if (cin) {
-#pragma unroll
-      for (int mm = 0; mm < 16; ++mm)
-        if (mm < M)
-          m[(r_base + static_cast<int64_t>(rs) * (jl + 16 * mm)) * cols + col] = x[mm] * out_scale;
+    for (int u = 0; u < 4; ++u) {
+      int64_t gc;
+      float* dst = gaddr(org, col0, u, gc);
+      const float4 v = *reinterpret_cast<const float4*>(buf + soff(u));
+      if (vec) {
+        *reinterpret_cast<float4*>(dst) =
+            make_float4(v.x * out_scale, v.y * out_scale, v.z * out_scale, v.w * out_scale);
+      } else {
+        if (gc < cols) dst[0] = v.x * out_scale;
+        if (gc + 1 < cols) dst[1] = v.y * out_scale;
+        if (gc + 2 < cols) dst[2] = v.z * out_scale;
+        if (gc + 3 < cols) dst[3] = v.w * out_scale;
+      }
     }
+    __syncthreads();   // this buffer is the target of the prefetch two tiles on
+    cur ^= 1;
   }
+  cp_async_wait0();
 }
 
 int ilog2_pow2(int b) {
@@ -383,14 +530,33 @@ kronq_status row_pass(const T* src, float* dst, int64_t rows, int64_t cols, cons
   const float out_scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(b)));
   if (b >= 16 && b <= 16384) {
     const int threads = chunk / 16;
-    const size_t smem = static_cast<size_t>(chunk + chunk / 16) * sizeof(float);
-    if (smem > 48 * 1024)
-      KQ_CUDA_TRY(cudaFuncSetAttribute(fwht_rows_reg_kernel<T>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    // padded work buffer + two staging buffers of the source type
+    const size_t smem = static_cast<size_t>(chunk + chunk / 16) * sizeof(float) +
+                        2 * static_cast<size_t>(chunk) * sizeof(T);
     const int vec = (reinterpret_cast<uintptr_t>(src) & 15u) == 0 &&
                     (reinterpret_cast<uintptr_t>(dst) & 15u) == 0;
-    fwht_rows_reg_kernel<T><<<static_cast<unsigned>(blocks), threads, smem, stream>>>(
-        src, dst, total, cols, row_f, col_f, scalar, ilog2_pow2(b), chunk, out_scale, vec);
+    const int log2b = ilog2_pow2(b);
+    // one instantiation per CTA size, so that each gets the register budget of its size; the
+    // grid is the CTAs that fit at once (each walks chunks grid-stride)
+    auto launch = [&](auto kern) -> kronq_status {
+      if (smem > 48 * 1024)
+        KQ_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem));
+      int per_sm = 1;
+      KQ_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem));
+      if (per_sm < 1) per_sm = 1;
+      const int64_t cap = static_cast<int64_t>(sm_budget()) * per_sm;
+      const unsigned grid = static_cast<unsigned>(blocks < cap ? blocks : cap);
+      kern<<<grid, threads, smem, stream>>>(src, dst, total, cols, row_f, col_f, scalar, log2b,
+                                            chunk, out_scale, vec);
+      return KRONQ_OK;
+    };
+    if (threads == 256)
+      KQ_TRY(launch(fwht_rows_reg_kernel<T, 256>));
+    else if (threads == 512)
+      KQ_TRY(launch(fwht_rows_reg_kernel<T, 512>));
+    else
+      KQ_TRY(launch(fwht_rows_reg_kernel<T, 1024>));
     return check_launch("fwht_rows_reg_kernel");
   }
   const size_t smem = static_cast<size_t>(chunk) * sizeof(float);
@@ -406,10 +572,24 @@ kronq_status row_pass(const T* src, float* dst, int64_t rows, int64_t cols, cons
 kronq_status col_pass_reg(float* m, int64_t rows, int64_t cols, int log2p, int rs, float out_scale,
                           cudaStream_t stream) {
   const int P = 1 << log2p;
-  const size_t smem = static_cast<size_t>(P) * (kColTile + 1) * sizeof(float);
-  dim3 grid(static_cast<unsigned>((cols + kColTile - 1) / kColTile),
-            static_cast<unsigned>(rows / P));
-  fwht_cols_reg_kernel<<<grid, 2 * P, smem, stream>>>(m, rows, cols, log2p, rs, out_scale);
+  const size_t smem = 2 * static_cast<size_t>(P) * kColLd * sizeof(float);   // two tile buffers
+  // 16-byte pieces need aligned rows and whole 32-column tiles
+  const int vec = (reinterpret_cast<uintptr_t>(m) & 15u) == 0 && cols % kColTile == 0;
+  const int64_t tiles = ((cols + kColTile - 1) / kColTile) * (rows / P);
+  static bool attr = false;
+  if (!attr) {
+    KQ_CUDA_TRY(cudaFuncSetAttribute(fwht_cols_reg_kernel,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(2 * 256 * kColLd * sizeof(float))));
+    attr = true;
+  }
+  int per_sm = 1;   // the CTAs that fit at once; each walks tiles grid-stride
+  KQ_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fwht_cols_reg_kernel, 2 * P,
+                                                            smem));
+  if (per_sm < 1) per_sm = 1;
+  const int64_t cap = static_cast<int64_t>(sm_budget()) * per_sm;
+  const unsigned grid = static_cast<unsigned>(tiles < cap ? tiles : cap);
+  fwht_cols_reg_kernel<<<grid, 2 * P, smem, stream>>>(m, rows, cols, log2p, rs, out_scale, vec);
   return check_launch("fwht_cols_reg_kernel");
 }
 
