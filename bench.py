@@ -46,6 +46,9 @@ def parse():
     ap.add_argument("--no-graphs", action="store_true",
                     help="enqueue the per-sublayer phases eagerly instead of replaying CUDA "
                          "graphs (each graph keeps its own copies of the phase's outputs)")
+    ap.add_argument("--overlap", type=int, default=0, metavar="SMS",
+                    help="run each sublayer's BiIP and inverse factor alongside the remaining "
+                         "statistics on SMS reserved SMs (0: phases one after another)")
     ap.add_argument("--no-e2e", action="store_true", help=argparse.SUPPRESS)
     ap.add_argument("--no-cpu-baseline", action="store_true", help=argparse.SUPPRESS)
     return ap.parse_args()
@@ -220,6 +223,8 @@ class Block:
         self.bits = None
         self.streams = None         # one stream per sublayer for the per-sublayer steps
         self.use_graphs = True
+        self.overlap = False        # per-sublayer chains alongside the statistics (see step)
+        self.reserve = 16           # SMs kept free of statistics while overlapping
 
     def input_bytes(self):
         tot = 0
@@ -238,6 +243,9 @@ class Block:
         g = g_src or self.g
         if not self.use_graphs:
             self.results = {}       # eager phases allocate new outputs: drop the last step's
+        if self.overlap:
+            self._step_overlapped(x, g, time_acc=time_acc)
+            return
         for name, h in self.hx.items():
             h.zero_()
             if self.drift:
@@ -303,12 +311,43 @@ class Block:
         """One step with the inputs in pinned host memory, as a user with host data runs it.
 
         Every X / G copy goes over the host link on `copy_stream`, one tensor at a time, in the
-        order the sublayers consume them: longest inverse-factor chain first. Each statistic
-        starts as soon as its input has landed, and each sublayer's BiIP and inverse factor
-        start as soon as its two sums are complete. All of this overlaps the copies still in
-        flight. The column solves follow the bit allocation, which needs every sublayer's
-        traces.
+        order the overlapped step consumes them (longest inverse-factor chain first); each
+        statistic waits only for its own input.
         """
+        import torch
+        main = torch.cuda.current_stream()
+        landed = {}
+        copy_stream.wait_stream(main)
+        for kind, name in self._consumption_order():
+            src, dst = (host_x, dev_x) if kind == "x" else (host_g, dev_g)
+            with torch.cuda.stream(copy_stream):
+                dst[name].copy_(src[name], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(copy_stream)
+            landed[(kind, name)] = ev
+        self._step_overlapped(dev_x, dev_g, landed=landed)
+
+    def _chain_order(self):
+        subs = self.wl.sublayers
+        return sorted(range(len(subs)),
+                      key=lambda i: -(subs[i].d_in ** 3 + 128 * subs[i].d_out * subs[i].d_in))
+
+    def _consumption_order(self):
+        subs = self.wl.sublayers
+        seq, seen = [], set()
+        for i in self._chain_order():
+            if subs[i].x_stream not in seen:
+                seen.add(subs[i].x_stream)
+                seq.append(("x", subs[i].x_stream))
+            seq.append(("g", subs[i].name))
+        return seq
+
+    def _step_overlapped(self, x, g, landed=None, time_acc=False):
+        """Statistics, sublayer by sublayer (longest inverse-factor chain first), on all but
+        `reserve` SMs; as soon as a sublayer's sums are complete its BiIP and inverse factor
+        start on its own stream (a captured graph sized to the reserved SMs), alongside the
+        remaining statistics. The bit allocation needs every sublayer's traces; the column
+        solves follow it on the whole GPU."""
         import torch
 
         from post_quantization_b200 import kronq as K
@@ -317,55 +356,55 @@ class Block:
         subs = wl.sublayers
         inv_n = 1.0 / self.n
         main = torch.cuda.current_stream()
+        sms = torch.cuda.get_device_properties(self.dev).multi_processor_count
         if getattr(self, "_st", None) is None:
             self._st = {}
             st = self._st
-            st["order"] = sorted(range(len(subs)),
-                                 key=lambda i: -(subs[i].d_in ** 3 + 128 * subs[i].d_out * subs[i].d_in))
+            st["order"] = self._chain_order()
             st["streams"] = [torch.cuda.Stream(device=self.dev) for _ in subs]
             st["ws"] = [P.Workspace(self.dev) for _ in subs]
 
             def chain(i):
                 sl = subs[i]
-                r = P.biip(self.w[sl.name], self.hx[sl.x_stream], self.hg[sl.name], None, inv_n,
+                r = P.biip(self.w[sl.name], self.hx[sl.x_stream], self.hg[sl.name],
+                           self.dxx[sl.x_stream] if self.drift else None, inv_n,
                            self.si[sl.name], self.so[sl.name], K.BIIP_FULL, ws=st["ws"][i])
                 P.cholinv(r, 0.01, st["ws"][i])
                 return r
-            st["chain"] = [P.CapturedPhase(lambda i=i: chain(i)) for i in range(len(subs))]
+            st["chain"] = [P.CapturedPhase(lambda i=i: chain(i)) if self.use_graphs
+                           else (lambda i=i: chain(i)) for i in range(len(subs))]
             st["solve"] = {}
             st["solve_res"] = None
         st = self._st
-        seq, seen = [], set()
-        for i in st["order"]:
-            if subs[i].x_stream not in seen:
-                seen.add(subs[i].x_stream)
-                seq.append(("x", subs[i].x_stream))
-            seq.append(("g", subs[i].name))
-        landed = {}
-        copy_stream.wait_stream(main)
-        for kind, name in seq:
-            src, dst = (host_x, dev_x) if kind == "x" else (host_g, dev_g)
-            with torch.cuda.stream(copy_stream):
-                dst[name].copy_(src[name], non_blocking=True)
-                ev = torch.cuda.Event()
-                ev.record(copy_stream)
-            landed[(kind, name)] = ev
         res = [None] * len(subs)
         done = set()
+        acc_budget = sms - self.reserve if self.reserve > 0 else 0
         for i in st["order"]:
             sl = subs[i]
+            K.kronq_set_sm_budget(acc_budget)
             if sl.x_stream not in done:
                 done.add(sl.x_stream)
-                main.wait_event(landed[("x", sl.x_stream)])
-                self.hx[sl.x_stream].zero_()
-                P.accumulate(xq=dev_x[sl.x_stream], hx_sum=self.hx[sl.x_stream], ws=self.ws)
-            main.wait_event(landed[("g", sl.name)])
-            self.hg[sl.name].zero_()
-            P.accumulate(g=dev_g[sl.name], hg_sum=self.hg[sl.name], ws=self.ws)
+                if landed is not None:
+                    main.wait_event(landed[("x", sl.x_stream)])
+                h = self.hx[sl.x_stream]
+                h.zero_()
+                if self.drift:
+                    self.dxx[sl.x_stream].zero_()
+                self._timed_acc(time_acc, h.shape[0], self.drift, lambda: P.accumulate(
+                    xq=x[sl.x_stream], xfp=self.xfp[sl.x_stream] if self.drift else None,
+                    hx_sum=h, dxx_sum=self.dxx[sl.x_stream] if self.drift else None, ws=self.ws))
+            if landed is not None:
+                main.wait_event(landed[("g", sl.name)])
+            h = self.hg[sl.name]
+            h.zero_()
+            self._timed_acc(time_acc, h.shape[0], False,
+                            lambda: P.accumulate(g=g[sl.name], hg_sum=h, ws=self.ws))
             s_i = st["streams"][i]
             s_i.wait_stream(main)
+            K.kronq_set_sm_budget(self.reserve)
             with torch.cuda.stream(s_i):
                 res[i] = st["chain"][i]()
+        K.kronq_set_sm_budget(0)
         for s_i in st["streams"]:
             main.wait_stream(s_i)
         for sl, r in zip(subs, res):
@@ -375,23 +414,38 @@ class Block:
         avg = wl.extra.get("avg_bits", float(wl.bits))
         _, self.bits = K.kronq_score_allocate(tr[:, 0].tolist(), tr[:, 1].tolist(),
                                               [sl.d_out * sl.d_in for sl in subs], choices, avg)
+        bits = list(self.bits)
+
+        def solve():
+            for j in st["order"]:
+                s_j = st["streams"][j]
+                s_j.wait_stream(torch.cuda.current_stream())
+                with torch.cuda.stream(s_j):
+                    P.quantize(res[j], bits[j], st["ws"][j])
+            for s_j in st["streams"]:
+                torch.cuda.current_stream().wait_stream(s_j)
+        if not self.use_graphs:
+            solve()
+            return
         if st["solve_res"] != [id(r) for r in res]:     # new chain outputs: new solve graphs
             st["solve_res"] = [id(r) for r in res]
             st["solve"] = {}
-        key = tuple(self.bits)
+        key = tuple(bits)
         if key not in st["solve"]:
-            bits = list(self.bits)
-
-            def solve():
-                for j in st["order"]:
-                    s_j = st["streams"][j]
-                    s_j.wait_stream(torch.cuda.current_stream())
-                    with torch.cuda.stream(s_j):
-                        P.quantize(res[j], bits[j], st["ws"][j])
-                for s_j in st["streams"]:
-                    torch.cuda.current_stream().wait_stream(s_j)
             st["solve"][key] = P.CapturedPhase(solve)
         st["solve"][key]()
+
+    def _timed_acc(self, time_acc, d, drift, fn):
+        import torch
+        if not time_acc:
+            fn()
+            return
+        e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        # N d(d+1) for a symmetric sum (one triangle), 2 N d^2 for D
+        self.acc_events.append((e0, e1, self.n * d * (d + 1) + (2 * self.n * d * d if drift else 0)))
 
 
 def describe(wl, n_tok):
@@ -436,6 +490,8 @@ def run_gpu(args):
     ws = P.Workspace(dev)
     blk = Block(wl, rank, dev, n_tok, ws)
     blk.use_graphs = not args.no_graphs
+    blk.overlap = args.overlap > 0
+    blk.reserve = args.overlap
     torch.cuda.synchronize()
 
     def barrier():

@@ -401,12 +401,14 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 __device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
-__global__ void __launch_bounds__(512) fwht_cols_reg_kernel(float* m, int64_t rows, int64_t cols,
-                                                            int log2p, int rs, float out_scale,
-                                                            int vec) {
+template <int LOG2P>
+__global__ void __launch_bounds__(2 << LOG2P) fwht_cols_reg_kernel(float* m, int64_t rows,
+                                                                  int64_t cols, int rs,
+                                                                  float out_scale, int vec) {
   extern __shared__ __align__(16) float sb[];
-  const int P = 1 << log2p;
-  const int nt = 2 * P;
+  constexpr int log2p = LOG2P;
+  constexpr int P = 1 << LOG2P;
+  constexpr int nt = 2 * P;
   const int t = threadIdx.x;
   const int tiles_x = static_cast<int>((cols + kColTile - 1) / kColTile);
   const int num_tiles = tiles_x * static_cast<int>(rows / P);
@@ -475,18 +477,27 @@ __global__ void __launch_bounds__(512) fwht_cols_reg_kernel(float* m, int64_t ro
     fwht16(x, 4);
 #pragma unroll
     for (int k = 0; k < 16; ++k) buf[(16 * jg + k) * kColLd + c] = x[k];
-    if (log2p > 4) {
+    if constexpr (LOG2P > 4) {
       __syncthreads();
-      // round 1: bits 4.. of j; groups (c, jl), jl in [0, 16), P / 16 elements each
-      const int M = P >> 4, per = 256 / P;
+      // round 1: bits 4.. of j; groups (c, jl), jl in [0, 16), M = P / 16 elements each
+      constexpr int M = P >> 4, per = 256 / P;
+#pragma unroll
       for (int w = 0; w < per; ++w) {
         const int jl = jg * per + w;
+        float y[M];
 #pragma unroll
-        for (int mm = 0; mm < 16; ++mm) x[mm] = mm < M ? buf[(jl + 16 * mm) * kColLd + c] : 0.f;
-        fwht16(x, log2p - 4);
+        for (int mm = 0; mm < M; ++mm) y[mm] = buf[(jl + 16 * mm) * kColLd + c];
 #pragma unroll
-        for (int mm = 0; mm < 16; ++mm)
-          if (mm < M) buf[(jl + 16 * mm) * kColLd + c] = x[mm];
+        for (int h = 0; h < LOG2P - 4; ++h)
+#pragma unroll
+          for (int mm = 0; mm < M; ++mm) {
+            if (mm & (1 << h)) continue;
+            const float a = y[mm], b = y[mm | (1 << h)];
+            y[mm] = a + b;
+            y[mm | (1 << h)] = a - b;
+          }
+#pragma unroll
+        for (int mm = 0; mm < M; ++mm) buf[(jl + 16 * mm) * kColLd + c] = y[mm];
       }
     }
     __syncthreads();
@@ -576,20 +587,26 @@ kronq_status col_pass_reg(float* m, int64_t rows, int64_t cols, int log2p, int r
   // 16-byte pieces need aligned rows and whole 32-column tiles
   const int vec = (reinterpret_cast<uintptr_t>(m) & 15u) == 0 && cols % kColTile == 0;
   const int64_t tiles = ((cols + kColTile - 1) / kColTile) * (rows / P);
-  static bool attr = false;
-  if (!attr) {
-    KQ_CUDA_TRY(cudaFuncSetAttribute(fwht_cols_reg_kernel,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     static_cast<int>(2 * 256 * kColLd * sizeof(float))));
-    attr = true;
+  auto launch = [&](auto kern) -> kronq_status {
+    if (smem > 48 * 1024)
+      KQ_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem)));
+    int per_sm = 1;   // the CTAs that fit at once; each walks tiles grid-stride
+    KQ_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 2 * P, smem));
+    if (per_sm < 1) per_sm = 1;
+    const int64_t cap = static_cast<int64_t>(sm_budget()) * per_sm;
+    const unsigned grid = static_cast<unsigned>(tiles < cap ? tiles : cap);
+    kern<<<grid, 2 * P, smem, stream>>>(m, rows, cols, rs, out_scale, vec);
+    return KRONQ_OK;
+  };
+  switch (log2p) {
+    case 4: KQ_TRY(launch(fwht_cols_reg_kernel<4>)); break;
+    case 5: KQ_TRY(launch(fwht_cols_reg_kernel<5>)); break;
+    case 6: KQ_TRY(launch(fwht_cols_reg_kernel<6>)); break;
+    case 7: KQ_TRY(launch(fwht_cols_reg_kernel<7>)); break;
+    case 8: KQ_TRY(launch(fwht_cols_reg_kernel<8>)); break;
+    default: return fail(KRONQ_ERR_UNSUPPORTED, "column pass of %d points", P);
   }
-  int per_sm = 1;   // the CTAs that fit at once; each walks tiles grid-stride
-  KQ_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fwht_cols_reg_kernel, 2 * P,
-                                                            smem));
-  if (per_sm < 1) per_sm = 1;
-  const int64_t cap = static_cast<int64_t>(sm_budget()) * per_sm;
-  const unsigned grid = static_cast<unsigned>(tiles < cap ? tiles : cap);
-  fwht_cols_reg_kernel<<<grid, 2 * P, smem, stream>>>(m, rows, cols, log2p, rs, out_scale, vec);
   return check_launch("fwht_cols_reg_kernel");
 }
 
