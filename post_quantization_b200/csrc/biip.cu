@@ -198,11 +198,11 @@ __global__ void __launch_bounds__(256) fwht_cols_kernel(float* m, int64_t rows, 
 
 // ---- register-radix passes (16 <= b <= 16384) ----
 //
-// Row pass: one CTA per chunk of C = max(b, 4096) consecutive elements (whole b-blocks),
-// C / 16 threads. Round 0 takes 16 consecutive elements per thread straight from global
-// memory and transforms index bits 0-3 in registers; round R takes the 16 elements whose index
-// differs in bits 4R..4R+3 (stride 16^R) from shared memory. The last round writes to global
-// memory, coalesced. log2(b) stages cost ceil(log2(b) / 4) - 1 shared-memory round trips.
+// Row pass: chunks of C = max(b, 4096) consecutive elements (whole b-blocks), C / 16 threads per
+// CTA, each CTA walking chunks. A thread takes 16 consecutive elements (streamed in with
+// cp.async one chunk ahead) and transforms index bits 0-3 in registers, bits 4-8 with warp
+// shuffles, and bits 9 and up through shared memory in 4-bit windows; it stores its 16 elements
+// back as 16-byte vectors.
 //
 // Column pass: a P-point transform along rows r_base + rs * j (j < P) of a tile of 32
 // columns, P in [16, 256]. b <= 256 is one pass (P = b, rs = 1); larger b is two passes,
