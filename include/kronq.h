@@ -212,14 +212,22 @@ KRONQ_API kronq_status kronq_cholinv(float* h_to_k, int32_t d, float damp_rel, i
  *   k        (device, fp32) d_in x d_in, upper triangle = K (from kronq_cholinv)
  *   dxx      (device, fp32) d_in x d_in processed drift term, or NULL
  *   bits     2..8;  block: column block width, 128 (others give KRONQ_ERR_UNSUPPORTED)
- *   codes    (device, uint8) d_out x d_in;  scale, zero (device, fp32) d_out each
+ *   group    0: one grid per output row, from W before the solve (as above);
+ *            128 (= block): one grid per row and per 128 consecutive columns ([KronQ-hyper]
+ *            Experiments, g = 128), taken when the solve reaches the group's first column from
+ *            the weights it is about to quantize, i.e. the rows of W (I + P) after the updates
+ *            of every earlier column (lo/hi over the group's columns, same formulas);
+ *            other values give KRONQ_ERR_UNSUPPORTED
+ *   codes    (device, uint8) d_out x d_in
+ *   scale, zero (device, fp32) d_out each (group 0), or d_out x ceil(d_in / group) row-major
  *   w_hat    (device, fp32) d_out x d_in: dequantized weights W^ (also the solve's working copy)
  * ------------------------------------------------------------------------------------- */
 KRONQ_API size_t kronq_quantize_layer_workspace_size(int32_t d_out, int32_t d_in, int32_t block,
                                            int with_dxx);
 KRONQ_API kronq_status kronq_quantize_layer(const float* w, const float* k, const float* dxx,
                                   int32_t d_out, int32_t d_in, int32_t bits, int32_t block,
-                                  uint8_t* codes, float* scale, float* zero, float* w_hat,
+                                  int32_t group, uint8_t* codes, float* scale, float* zero,
+                                  float* w_hat,
                                   void* workspace, size_t workspace_bytes,
                                   kronq_stream_t stream);
 

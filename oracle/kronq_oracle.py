@@ -301,7 +301,8 @@ def dequantize(codes, scale, zero):
     return (scale * (codes - zero)).astype(np.float32)
 
 
-def quantize_layer(w, k, dxx=None, bits: int = 4, follow_codes=None, tie_tol: float = 1e-3):
+def quantize_layer(w, k, dxx=None, bits: int = 4, follow_codes=None, tie_tol: float = 1e-3,
+                   group: int = 0, follow_grid=None, scale_rtol: float = 1e-5):
     """Column-wise OBS / GPTAQ solve onto the per-row grid, literally, one column at a time.
 
     [KronQ-hyper] Method, OBS update:
@@ -313,20 +314,61 @@ def quantize_layer(w, k, dxx=None, bits: int = 4, follow_codes=None, tie_tol: fl
     value sits within tie_tol grid units of a rounding boundary (a half-integer of w/scale) it
     adopts that code instead of its own, and records a near-tie; where it adopts a code that
     differs from its own decision it also records a disagreement. Every other code is its own.
-    Returns dict: codes (uint8), scale, zero, w_hat (fp64), near_tie (bool mask),
-    disagree (bool mask), pre (fp64: each column's value just before it was quantized).
+    group: 0 for one grid per output row (from W before the solve); g > 0 for one grid per row
+    and per g consecutive columns ([KronQ-hyper] Experiments, g = 128). A group's grid is taken
+    when the solve reaches its first column, from the weights that the solve is about to
+    quantize: the current (error-updated) weights plus the P contributions that the group's own
+    earlier columns will still add (the solve quantizes W (I + P), updated). With P = 0 this is
+    the grouped grid of GPTQ.
+    follow_grid: optional (scale, zero) group grids from another implementation (group > 0).
+    A group's grid comes from weights that each side has updated in its own arithmetic, so the
+    two differ by rounding: this oracle adopts the other scale where it agrees with its own to
+    scale_rtol, and the other zero only where its own -lo / scale lies within tie_tol of a
+    rounding boundary (grid_tie counts those rows); anywhere else it keeps its own grid.
+    Returns dict: codes (uint8), scale, zero (d_out, or d_out x groups), w_hat (fp64), near_tie
+    (bool mask), disagree (bool mask), pre (fp64: each column's value just before it was
+    quantized), grid_tie (rows x groups that adopted the other zero).
     """
     w0 = np.asarray(w, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     d_out, d_in = w0.shape
-    scale, zero = grid(w0, bits)
     p_mat = None if dxx is None else p_matrix(dxx, k)
+    grid_tie = None
+    if group:
+        n_groups = (d_in + group - 1) // group
+        scales = np.zeros((d_out, n_groups), dtype=np.float32)
+        zeros = np.zeros((d_out, n_groups), dtype=np.float32)
+        grid_tie = np.zeros((d_out, n_groups), dtype=bool)
+    else:
+        scale, zero = grid(w0, bits)
     cur = w0.copy()
     codes = np.zeros((d_out, d_in), dtype=np.uint8)
     near = np.zeros((d_out, d_in), dtype=bool)
     disagree = np.zeros((d_out, d_in), dtype=bool)
     pre = np.zeros((d_out, d_in))
     for p in range(d_in):
+        if group and p % group == 0:
+            g1 = min(d_in, p + group)
+            target = cur[:, p:g1].copy()
+            if p_mat is not None:
+                # P terms from the group's own columns, not yet added: column j gets
+                # sum over p <= q < j of W_:,q P_q,j
+                target += w0[:, p:g1] @ np.triu(p_mat[p:g1, p:g1], 1)
+            scale, zero = grid(target, bits)
+            if follow_grid is not None:
+                gi = p // group
+                o_s = np.asarray(follow_grid[0], dtype=np.float32).reshape(d_out, -1)[:, gi]
+                o_z = np.asarray(follow_grid[1], dtype=np.float32).reshape(d_out, -1)[:, gi]
+                close = np.abs(o_s.astype(np.float64) - scale) <= scale_rtol * np.abs(scale)
+                lo = target.min(axis=1).astype(np.float32)
+                u = (-lo / scale).astype(np.float64)
+                ztie = np.abs(u - (np.floor(u) + 0.5)) <= tie_tol
+                take_z = close & ztie & (o_z != zero)
+                grid_tie[:, gi] = take_z
+                scale = np.where(close, o_s, scale).astype(np.float32)
+                zero = np.where(take_z, o_z, zero).astype(np.float32)
+            scales[:, p // group] = scale
+            zeros[:, p // group] = zero
         col = cur[:, p].copy()
         pre[:, p] = col
         c = quantize_codes(col, scale, zero, bits)
@@ -346,8 +388,10 @@ def quantize_layer(w, k, dxx=None, bits: int = 4, follow_codes=None, tie_tol: fl
                 cur[:, p + 1:] += np.outer(w0[:, p], p_mat[p, p + 1:])
         cur[:, p] = dq
         codes[:, p] = c.astype(np.uint8)
+    if group:
+        scale, zero = scales, zeros
     return {"codes": codes, "scale": scale, "zero": zero, "w_hat": cur, "near_tie": near,
-            "disagree": disagree, "pre": pre}
+            "disagree": disagree, "pre": pre, "grid_tie": grid_tie}
 
 
 # ------------------------------------------------------------------------------------------

@@ -293,20 +293,22 @@ size_t kronq_quantize_layer_workspace_size(int32_t d_out, int32_t d_in, int32_t 
 
 kronq_status kronq_quantize_layer(const float* w, const float* k, const float* dxx,
                                   int32_t d_out, int32_t d_in, int32_t bits, int32_t block,
-                                  uint8_t* codes, float* scale, float* zero, float* w_hat,
-                                  void* workspace, size_t workspace_bytes,
+                                  int32_t group, uint8_t* codes, float* scale, float* zero,
+                                  float* w_hat, void* workspace, size_t workspace_bytes,
                                   kronq_stream_t stream) {
   if (d_out <= 0 || d_in <= 0) return fail(KRONQ_ERR_SHAPE, "d_out and d_in must be positive");
   if (!w || !k || !codes || !scale || !zero || !w_hat)
     return fail(KRONQ_ERR_INVALID_ARG, "w, k, codes, scale, zero and w_hat are required");
   if (bits < 2 || bits > 8) return fail(KRONQ_ERR_UNSUPPORTED, "bits must be in 2..8");
   if (block != 128) return fail(KRONQ_ERR_UNSUPPORTED, "block must be 128");
+  if (group != 0 && group != block)
+    return fail(KRONQ_ERR_UNSUPPORTED, "group must be 0 (per row) or the block width (128)");
   if (w == w_hat) return fail(KRONQ_ERR_INVALID_ARG, "w and w_hat must not alias");
   KQ_TRY(check_ws(workspace, workspace_bytes,
                   quantize_workspace_bytes(d_out, d_in, block, dxx != nullptr)));
   KQ_TRY(kronq_device_check());
-  return run_quantize(w, k, dxx, d_out, d_in, bits, block, codes, scale, zero, w_hat, workspace,
-                      reinterpret_cast<cudaStream_t>(stream));
+  return run_quantize(w, k, dxx, d_out, d_in, bits, block, group, codes, scale, zero, w_hat,
+                      workspace, reinterpret_cast<cudaStream_t>(stream));
 }
 
 // ----------------------------------------------------------------------------- allocation

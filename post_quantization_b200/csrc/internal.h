@@ -46,8 +46,8 @@ kronq_status run_cholinv(float* a, int d, float damp_rel, int32_t* info, void* w
 // quantize.cu
 size_t quantize_workspace_bytes(int d_out, int d_in, int block, bool with_dxx);
 kronq_status run_quantize(const float* w, const float* k, const float* dxx, int d_out, int d_in,
-                          int bits, int block, uint8_t* codes, float* scale, float* zero,
-                          float* w_hat, void* ws, cudaStream_t stream);
+                          int bits, int block, int group, uint8_t* codes, float* scale,
+                          float* zero, float* w_hat, void* ws, cudaStream_t stream);
 
 // Zero structure of GEMM operands (the zeros must be stored), used to skip K ranges:
 //   GEMM_A_UPPER  A[m][k] = 0 for k < m

@@ -81,7 +81,7 @@ __global__ void striu_kernel(float* __restrict__ m, int d) {
 //          (the operand of the lazy trailing updates on the tensor cores)
 __global__ void __launch_bounds__(32 * QT) block_solve_kernel(
     float* __restrict__ w_hat, const float* __restrict__ k, int d_out, int d_in, int b0, int bw,
-    const float* __restrict__ scale, const float* __restrict__ zero, float maxq,
+    float* __restrict__ scale, float* __restrict__ zero, int grouped, int n_groups, float maxq,
     uint8_t* __restrict__ codes, uint16_t* __restrict__ delta0, uint16_t* __restrict__ delta1,
     uint16_t* __restrict__ delta2, int64_t ldd) {
   extern __shared__ __align__(16) float sm[];
@@ -136,12 +136,49 @@ __global__ void __launch_bounds__(32 * QT) block_solve_kernel(
 #pragma unroll
       for (int j = 0; j < QW; ++j) w[r][j] = (active && QW * q + j < bw) ? wrow[j] : 0.f;
     }
-    sc[r] = active ? scale[row] : 1.f;
-    zr[r] = active ? zero[row] : 0.f;
+    if (!grouped) {
+      sc[r] = active ? scale[row] : 1.f;
+      zr[r] = active ? zero[row] : 0.f;
+    } else {
+      // this quarter's share of the row's lo / hi over the block's columns (E is free until
+      // the solve starts)
+      float lo = INFINITY, hi = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < QW; ++j)
+        if (QW * q + j < bw) {
+          lo = fminf(lo, w[r][j]);
+          hi = fmaxf(hi, w[r][j]);
+        }
+      E[q * QROWS + 32 * r + lane] = lo;
+      E[(QT + q) * QROWS + 32 * r + lane] = hi;
+    }
 #pragma unroll
     for (int j = 0; j < QW / 4; ++j) packed[r][j] = 0u;
   }
-  __syncthreads();   // Rd
+  __syncthreads();   // Rd, and the quarters' lo / hi
+  if (grouped) {
+    // the group's grid, from the weights the solve is about to quantize (same formulas as the
+    // per-row grid, decisions in fp32)
+#pragma unroll
+    for (int r = 0; r < RPL; ++r) {
+      float lo = E[32 * r + lane], hi = E[QT * QROWS + 32 * r + lane];
+#pragma unroll
+      for (int qq = 1; qq < QT; ++qq) {
+        lo = fminf(lo, E[qq * QROWS + 32 * r + lane]);
+        hi = fmaxf(hi, E[(QT + qq) * QROWS + 32 * r + lane]);
+      }
+      float sv = __fdiv_rn(__fsub_rn(hi, lo), maxq);
+      if (hi == lo) sv = 1.f;
+      sc[r] = sv;
+      zr[r] = rintf(__fdiv_rn(-lo, sv));
+      const int row = blockIdx.x * QROWS + 32 * r + lane;
+      if (q == 0 && row < d_out) {
+        scale[static_cast<int64_t>(row) * n_groups + b0 / QB] = sc[r];
+        zero[static_cast<int64_t>(row) * n_groups + b0 / QB] = zr[r];
+      }
+    }
+    __syncthreads();   // every warp has its grid before the solve writes E
+  }
 
   for (int qo = 0; qo < QT; ++qo) {
     if (q == qo) {
@@ -274,17 +311,21 @@ size_t quantize_workspace_bytes(int d_out, int d_in, int block, bool with_dxx) {
 }
 
 kronq_status run_quantize(const float* w, const float* k, const float* dxx, int d_out, int d_in,
-                          int bits, int block, uint8_t* codes, float* scale, float* zero,
-                          float* w_hat, void* ws, cudaStream_t stream) {
+                          int bits, int block, int group, uint8_t* codes, float* scale,
+                          float* zero, float* w_hat, void* ws, cudaStream_t stream) {
   (void)block;
   const float maxq = static_cast<float>((1 << bits) - 1);
   Carve cv{static_cast<uint8_t*>(ws)};
   Split3 ks = cv.split(d_in, d_in);
   Split3 ds = cv.split(d_out, QSB);
 
-  // grid from W before the solve
-  grid_kernel<<<(d_out + 7) / 8, 256, 0, stream>>>(w, d_out, d_in, maxq, scale, zero);
-  KQ_TRY(check_launch("grid_kernel"));
+  const int grouped = group > 0 ? 1 : 0;
+  const int n_groups = grouped ? (d_in + QB - 1) / QB : 1;
+  if (!grouped) {
+    // grid from W before the solve (grouped grids are taken block by block in the solve)
+    grid_kernel<<<(d_out + 7) / 8, 256, 0, stream>>>(w, d_out, d_in, maxq, scale, zero);
+    KQ_TRY(check_launch("grid_kernel"));
+  }
   KQ_TRY(split_bf16x3(k, d_in, d_in, d_in, ks, stream));
 
   KQ_CUDA_TRY(cudaMemcpyAsync(w_hat, w, sizeof(float) * static_cast<size_t>(d_out) * d_in,
@@ -345,8 +386,8 @@ kronq_status run_quantize(const float* w, const float* k, const float* dxx, int 
       const int bw = d_in - b0 < QB ? d_in - b0 : QB;
       const Split3 db = offset(ds, 0, b0 - s0);
       block_solve_kernel<<<(d_out + QROWS - 1) / QROWS, 32 * QT, smem, stream>>>(
-          w_hat, k, d_out, d_in, b0, bw, scale, zero, maxq, codes, db.part[0], db.part[1],
-          db.part[2], db.ld);
+          w_hat, k, d_out, d_in, b0, bw, scale, zero, grouped, n_groups, maxq, codes, db.part[0],
+          db.part[1], db.part[2], db.ld);
       KQ_TRY(check_launch("block_solve_kernel"));
       const int e = b0 + bw;
       if (e < s1) {

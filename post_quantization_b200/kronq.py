@@ -101,8 +101,8 @@ def load_library(path: str = LIB_PATH):
                                   c_void_p]),
         "kronq_quantize_layer_workspace_size": (c_sz, [c_i32, c_i32, c_i32, c_i32]),
         "kronq_quantize_layer": (c_i32, [c_void_p, c_void_p, c_void_p, c_i32, c_i32, c_i32, c_i32,
-                                         c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_sz,
-                                         c_void_p]),
+                                         c_i32, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                         c_sz, c_void_p]),
         "kronq_score_allocate": (c_i32, [c_void_p, c_void_p, c_void_p, c_i32, c_void_p, c_i32,
                                          c_dbl, c_void_p, c_void_p]),
     }
@@ -254,15 +254,15 @@ def kronq_quantize_layer_workspace_size(d_out: int, d_in: int, block: int, with_
 
 
 def kronq_quantize_layer(w, k, dxx, bits, codes, scale, zero, w_hat, block=128, workspace=None,
-                         stream=None):
+                         stream=None, group=0):
     lib = load_library()
     d_out, d_in = w.shape
     ws, wsb = _workspace(lib.kronq_quantize_layer_workspace_size(d_out, d_in, block,
                                                                  int(dxx is not None)),
                          w.device, workspace)
     st = lib.kronq_quantize_layer(_p(w), _p(k), _p(dxx), d_out, d_in, int(bits), int(block),
-                                  _p(codes), _p(scale), _p(zero), _p(w_hat), _p(ws), wsb,
-                                  _stream(stream))
+                                  int(group), _p(codes), _p(scale), _p(zero), _p(w_hat), _p(ws),
+                                  wsb, _stream(stream))
     _check(st, "kronq_quantize_layer")
 
 

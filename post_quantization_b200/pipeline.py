@@ -82,17 +82,22 @@ def cholinv(r: SublayerResult, damp_rel=0.01, ws=None, stream=None, sync=False):
                     workspace=ws.get(wsz) if ws is not None else None, stream=stream)
 
 
-def quantize(r: SublayerResult, bits: int, ws=None, stream=None):
+def quantize(r: SublayerResult, bits: int, ws=None, stream=None, group: int = 0):
+    """Column solve of r (K in r.hx). group 0: one grid per row (scale, zero: d_out); group 128:
+    one grid per row and per 128 columns (scale, zero: d_out x ceil(d_in / 128))."""
     d_out, d_in = r.w_prime.shape
     dev = r.w_prime.device
+    grid_shape = (d_out, (d_in + group - 1) // group) if group else (d_out,)
     if r.codes is None:
         r.codes = torch.empty(d_out, d_in, dtype=torch.uint8, device=dev)
-        r.scale = torch.empty(d_out, dtype=torch.float32, device=dev)
-        r.zero = torch.empty(d_out, dtype=torch.float32, device=dev)
         r.w_hat = torch.empty(d_out, d_in, dtype=torch.float32, device=dev)
+    if r.scale is None or tuple(r.scale.shape) != grid_shape:
+        r.scale = torch.empty(grid_shape, dtype=torch.float32, device=dev)
+        r.zero = torch.empty(grid_shape, dtype=torch.float32, device=dev)
     wsz = K.kronq_quantize_layer_workspace_size(d_out, d_in, 128, r.dxx is not None)
     K.kronq_quantize_layer(r.w_prime, r.hx, r.dxx, bits, r.codes, r.scale, r.zero, r.w_hat,
-                           workspace=ws.get(wsz) if ws is not None else None, stream=stream)
+                           workspace=ws.get(wsz) if ws is not None else None, stream=stream,
+                           group=group)
 
 
 def quantize_sublayer(w, hx_sum, hg_sum, dxx_sum, inv_n, sign_in, sign_out, bits,

@@ -143,15 +143,15 @@ def case_quantize(args):
     P.accumulate(xq=x, hx_sum=hx)
     r = P.biip(w, hx, None, None, 1.0 / n, si, so, K.BIIP_SCALE_IN | K.BIIP_ROTATE_IN | K.BIIP_ROTATE_OUT)
     P.cholinv(r, 0.01, sync=True)
-    P.quantize(r, 4)
+    P.quantize(r, 4, group=args.group)
     torch.cuda.synchronize()
     a, b = ev(), ev()
     a.record()
     for _ in range(args.reps):
-        P.quantize(r, 4)
+        P.quantize(r, 4, group=args.group)
     b.record()
     torch.cuda.synchronize()
-    print(json.dumps({"case": "quantize", "d_out": d_out, "d_in": d_in,
+    print(json.dumps({"case": "quantize", "d_out": d_out, "d_in": d_in, "group": args.group,
                       "ms": a.elapsed_time(b) / args.reps}))
 
 
@@ -163,6 +163,7 @@ def main():
     ap.add_argument("--d-out", type=int, default=4096)
     ap.add_argument("--d-in", type=int, default=4096)
     ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--group", type=int, default=0, help="quantize: 0 (per row) or 128")
     args = ap.parse_args()
     K.load_library()
     K.kronq_device_check()

@@ -66,17 +66,27 @@ def test_workspace_queries(K):
     assert K.kronq_biip_workspace_size(0, 5) == 0
 
 
+def test_sm_budget_is_host_state(K):
+    assert K.kronq_sm_budget() == 0
+    K.kronq_set_sm_budget(16)
+    assert K.kronq_sm_budget() == 16
+    K.kronq_set_sm_budget(-3)                  # non-positive lifts it
+    assert K.kronq_sm_budget() == 0
+
+
 def test_argument_errors_before_device(K):
     lib = K.load_library()
     # quantize: bad bits / block / missing pointers, no device touched
-    assert lib.kronq_quantize_layer(8, 8, None, 16, 16, 9, 128, 8, 8, 8, 16, None, 0, None) \
+    assert lib.kronq_quantize_layer(8, 8, None, 16, 16, 9, 128, 0, 8, 8, 8, 16, None, 0, None) \
         == K.ERR_UNSUPPORTED
-    assert lib.kronq_quantize_layer(8, 8, None, 16, 16, 4, 64, 8, 8, 8, 16, None, 0, None) \
+    assert lib.kronq_quantize_layer(8, 8, None, 16, 16, 4, 64, 0, 8, 8, 8, 16, None, 0, None) \
         == K.ERR_UNSUPPORTED
-    assert lib.kronq_quantize_layer(None, 8, None, 16, 16, 4, 128, 8, 8, 8, 16, None, 0, None) \
+    assert lib.kronq_quantize_layer(None, 8, None, 16, 16, 4, 128, 0, 8, 8, 8, 16, None, 0, None) \
         == K.ERR_INVALID_ARG
-    assert lib.kronq_quantize_layer(8, 8, None, 0, 16, 4, 128, 8, 8, 8, 16, None, 0, None) \
+    assert lib.kronq_quantize_layer(8, 8, None, 0, 16, 4, 128, 0, 8, 8, 8, 16, None, 0, None) \
         == K.ERR_SHAPE
+    assert lib.kronq_quantize_layer(8, 8, None, 16, 16, 4, 128, 64, 8, 8, 8, 16, None, 0, None) \
+        == K.ERR_UNSUPPORTED                                   # group is 0 or the block width
     # biip: SCALE_OUT without hg, rotation without signs, bad dtype, aliasing
     args = [16, 0, 32, 48, None, None, 1.0, None, None, 4, 4]
     tail = [64, 80, 96, 112, None, 0, None]

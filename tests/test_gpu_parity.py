@@ -291,6 +291,42 @@ def test_quantize_matches_oracle(K, P, bits, with_dxx, shape):
     assert rel(h64(r.w_hat), o["w_hat"]) <= TOL
 
 
+@pytest.mark.parametrize("bits", [2, 4])
+@pytest.mark.parametrize("with_dxx", [False, True])
+@pytest.mark.parametrize("shape", [(256, 256), (96, 200), (130, 384)])
+def test_quantize_group128_matches_oracle(K, P, bits, with_dxx, shape):
+    # group-wise grid, g = 128 ([KronQ-hyper] Experiments): one scale / zero per row and per
+    # 128 columns, from the weights the solve is about to quantize. The oracle follows the GPU's
+    # group grid only where the two agree to 1e-5 (scale) and, for the zero, only at a rounding
+    # boundary of -lo / scale; then codes as for the per-row grid
+    d_out, d_in = shape
+    n = 2048
+    xq, xfp, g, w, si, so = layer_inputs(d_out, d_in, n, drift="rel0.05", tag=("qg", shape))
+    hx, hg, dxx = gpu_sums(K, xq, xfp, g, with_dxx=with_dxx)
+    r = P.biip(w, hx, hg, dxx, 1.0 / n, si, so, 15)
+    wp = r.w_prime.clone(); dxx_p = None if dxx is None else r.dxx.clone()
+    P.cholinv(r, 0.01, sync=True)
+    kk = r.hx.clone()
+    P.quantize(r, bits, group=128)
+    torch.cuda.synchronize()
+    ng = (d_in + 127) // 128
+    assert tuple(r.scale.shape) == (d_out, ng)
+    o = O.quantize_layer(h64(wp), h64(kk), None if dxx_p is None else h64(dxx_p), bits,
+                         follow_codes=h64(r.codes), group=128,
+                         follow_grid=(h64(r.scale), h64(r.zero)))
+    assert np.array_equal(h64(r.scale), o["scale"].astype(np.float64))
+    assert np.array_equal(h64(r.zero), o["zero"].astype(np.float64))
+    assert int(o["grid_tie"].sum()) <= 1e-2 * d_out * ng
+    check_codes(r.codes, o, d_out * d_in)
+    assert rel(h64(r.w_hat), o["w_hat"]) <= TOL
+    if not with_dxx:
+        # nothing has touched the first group yet: its grid is the min-max grid of W' over its
+        # columns, bit for bit (with P the first group is taken from W' (I + P) instead)
+        s0, z0 = O.grid(h64(wp)[:, :128].astype(np.float32), bits)
+        assert np.array_equal(h64(r.scale)[:, 0], s0.astype(np.float64))
+        assert np.array_equal(h64(r.zero)[:, 0], z0.astype(np.float64))
+
+
 def test_quantize_llama_shape_sampled_rows(K, P):
     # q_proj of LLaMA-2-7B (4096 x 4096), 4 bits: 48 random rows re-run by the oracle from the
     # GPU's K and W' (rows are independent given K)

@@ -451,3 +451,84 @@ def test_allocation_rejects_nan_and_infeasible_budget():
         O.score_allocate([float("nan")], [1.0], [10], [2, 3], 3)
     with pytest.raises(ValueError):
         O.score_allocate([1.0], [1.0], [10], [2, 3], 1.5)
+
+
+# ------------------------------------------------------------------------------ group-wise grid
+# [KronQ-hyper] Experiments quote 2-bit results with g = 128: one grid per row and per 128
+# consecutive columns, taken when the solve reaches the group (from the weights it is about to
+# quantize).
+
+def test_group_covering_all_columns_is_the_per_row_grid():
+    # with P = 0 and one group spanning the row, the group grid is taken at column 0 from W
+    # itself: the same solve as the per-row grid
+    r = rng(71)
+    d_out, d_in = 6, 37
+    w = 0.02 * r.standard_normal((d_out, d_in))
+    a = r.standard_normal((d_in, d_in))
+    k = O.cholinv(a @ a.T / d_in + 0.1 * np.eye(d_in), 0.01)
+    per_row = O.quantize_layer(w, k, None, 3)
+    one_group = O.quantize_layer(w, k, None, 3, group=d_in)
+    assert np.array_equal(per_row["codes"], one_group["codes"])
+    assert np.array_equal(per_row["w_hat"], one_group["w_hat"])
+    assert np.array_equal(per_row["scale"], one_group["scale"][:, 0])
+    assert np.array_equal(per_row["zero"], one_group["zero"][:, 0])
+
+
+@pytest.mark.parametrize("group", [8, 16, 40])
+def test_group_grid_without_feedback_is_groupwise_rtn(group):
+    # diagonal H: K is diagonal, the error of a column feeds nothing forward, and the solve is
+    # round-to-nearest with each group's own min-max grid (brute force per group, ragged last)
+    r = rng(72 + group)
+    d_out, d_in, bits = 5, 43, 2
+    w = r.standard_normal((d_out, d_in))
+    k = O.cholinv(np.diag(r.uniform(0.5, 2.0, d_in)), 0.01)
+    assert np.count_nonzero(np.triu(k, 1)) == 0
+    res = O.quantize_layer(w, k, None, bits, group=group)
+    maxq = 2 ** bits - 1
+    for g0 in range(0, d_in, group):
+        blk = w[:, g0:g0 + group].astype(np.float32)
+        for i in range(d_out):
+            lo, hi = np.float32(blk[i].min()), np.float32(blk[i].max())
+            s = np.float32((hi - lo) / np.float32(maxq)) if hi != lo else np.float32(1.0)
+            z = np.float32(np.rint(np.float32(-lo) / s))
+            assert res["scale"][i, g0 // group] == s and res["zero"][i, g0 // group] == z
+            for j in range(blk.shape[1]):
+                c = min(max(np.rint(np.float32(blk[i, j]) / s) + z, 0), maxq)
+                assert res["codes"][i, g0 + j] == c
+
+
+def test_group_grid_sees_the_pending_p_terms():
+    # with K diagonal nothing but P moves a column before it is quantized, so the value of each
+    # column at its turn ("pre") is exactly what the group's grid must have been taken from:
+    # a dropped P term, or one from the wrong triangle, changes some group's min or max
+    r = rng(75)
+    n, d_out, d_in, bits, group = 400, 6, 24, 3, 8
+    x = r.standard_normal((n, d_in))
+    xq = x + 0.4 * r.standard_normal((n, d_in))
+    _, _, dxx = O.accumulate(xq, x)
+    dxx /= n
+    k = O.cholinv(np.diag(r.uniform(0.5, 2.0, d_in)), 0.01)
+    w = r.standard_normal((d_out, d_in))
+    res = O.quantize_layer(w, k, dxx, bits, group=group)
+    assert np.abs(O.p_matrix(dxx, k)).max() > 1e-3          # P is not negligible here
+    for g0 in range(0, d_in, group):
+        s, z = O.grid(res["pre"][:, g0:g0 + group], bits)
+        # the two sides sum the same P terms in different orders (fp64): equal up to rounding
+        assert np.allclose(s, res["scale"][:, g0 // group], rtol=1e-6, atol=0)
+        assert np.array_equal(z, res["zero"][:, g0 // group])
+
+
+def test_follow_grid_adopts_only_near_ties():
+    # following another side's group grids changes nothing when that side equals this one, and
+    # a scale further off than scale_rtol is never adopted
+    r = rng(76)
+    d_out, d_in, group = 4, 32, 16
+    w = r.standard_normal((d_out, d_in))
+    a = r.standard_normal((d_in, d_in))
+    k = O.cholinv(a @ a.T / d_in + 0.1 * np.eye(d_in), 0.01)
+    own = O.quantize_layer(w, k, None, 3, group=group)
+    same = O.quantize_layer(w, k, None, 3, group=group, follow_grid=(own["scale"], own["zero"]))
+    assert np.array_equal(same["codes"], own["codes"]) and not same["grid_tie"].any()
+    off = O.quantize_layer(w, k, None, 3, group=group,
+                           follow_grid=(own["scale"] * 1.01, own["zero"] + 1))
+    assert np.array_equal(off["scale"], own["scale"]) and np.array_equal(off["zero"], own["zero"])
