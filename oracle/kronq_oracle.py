@@ -32,6 +32,11 @@ What it computes, step by step, with the passage each step follows. Page names:
   objective       tr[H_G dW H_X dW^T] + 2 tr[H_G W D dW^T]  [KronQ-hyper] Method: objectives
   mu_incoherence  max_ij |Q_ij| over eigenvectors Q of H (mu(H)/sqrt(d))
                                                   [KronQ-hyper] Method: incoherence figure
+  qlinear         the quantized layer on activations, y = S_G^-1 U^T W^' V S_X^-1 x with
+                  W^' = scale (codes - zero): at inference only the orthogonal transforms are
+                  added                                     [KronQ-gist] Limitations
+  pack_codes      the library's packed storage of 2/3/4-bit codes (a format of this library,
+                  defined in the inference-side section below; the pages fix none)
 
 Precision: all continuous arithmetic is fp64. The two places where floating point decides an
 integer (the grid's integer zero point and each quantized code) are evaluated in fp32, the
@@ -392,6 +397,175 @@ def quantize_layer(w, k, dxx=None, bits: int = 4, follow_codes=None, tie_tol: fl
         scale, zero = scales, zeros
     return {"codes": codes, "scale": scale, "zero": zero, "w_hat": cur, "near_tie": near,
             "disagree": disagree, "pre": pre, "grid_tie": grid_tie}
+
+
+# ------------------------------------------------------------------------------------------
+# Inference side: the quantized layer applied to activations
+# ------------------------------------------------------------------------------------------
+#
+# [KronQ-gist] Limitations: at inference the only overhead is the orthogonal transforms (the
+# same ones as QuIP#'s). The layer that was quantized is W' = U S_G W S_X V^T; its quantized
+# form W^' = scale (codes - zero) stands for W^ = S_G^-1 U^T W^' V S_X^-1 in the original basis,
+# so   y = W^ x = S_G^-1 U^T ( W^' ( V S_X^-1 x ) ).
+#
+# Packed code format (a storage format of this library; the pages do not fix one). Codes of
+# b = 2, 3 or 4 bits. Rows are cut into tiles of 128, columns into groups of 128; rows and
+# columns past the matrix hold code 0. Tile t, group g is one blob of 128 x 128 x b bits at byte
+# offset (t * G + g) * 2048 * b (G = ceil(d_in / 128)); inside it, row r takes 16 * b bytes at
+# offset r * 16 * b, read as little-endian 32-bit words w[0 .. 4b). Each word's low 16 bits
+# ("half 0") hold codes of even columns, its high 16 bits ("half 1") codes of odd columns.
+#   b = 2 or 4: the row's 128 columns form 8 chunks of 16; column 16 k + 2 s + h (s = 0..7,
+#     h = 0, 1) sits in word k b / 2 + floor(s b / 16) at bits 16 h + (s b mod 16) and up.
+#   b = 3: 4 chunks of 32 columns; column 32 k + 2 s + h (s = 0..15): for s < 15, word
+#     3 k + floor(s / 5) at bits 16 h + 3 (s mod 5) and up; for s = 15, bit i of the code
+#     (i = 0, 1, 2) is bit 16 h + 15 of word 3 k + i.
+
+PACK_ROWS = 128
+PACK_COLS = 128
+PACK_BITS = (2, 3, 4)
+
+
+def packed_bytes(d_out: int, d_in: int, bits: int) -> int:
+    """Size of the packed form: ceil(d_out/128) * ceil(d_in/128) blobs of 2048 * bits bytes."""
+    if bits not in PACK_BITS:
+        raise ValueError("packed codes have 2, 3 or 4 bits")
+    t = -(-d_out // PACK_ROWS)
+    g = -(-d_in // PACK_COLS)
+    return t * g * 2048 * bits
+
+
+def code_bit_positions(bits: int) -> np.ndarray:
+    """(128, bits) array: for column c of a group and code bit i, the bit index (32 * word +
+    bit in word) of that bit inside the row's 16 * bits bytes, following the format above."""
+    if bits not in PACK_BITS:
+        raise ValueError("packed codes have 2, 3 or 4 bits")
+    pos = np.zeros((PACK_COLS, bits), dtype=np.int64)
+    for c in range(PACK_COLS):
+        if bits == 3:
+            k, s, h = c // 32, (c % 32) // 2, c % 2
+            for i in range(3):
+                if s < 15:
+                    word, bit = 3 * k + s // 5, 16 * h + 3 * (s % 5) + i
+                else:
+                    word, bit = 3 * k + i, 16 * h + 15
+                pos[c, i] = 32 * word + bit
+        else:
+            k, s, h = c // 16, (c % 16) // 2, c % 2
+            for i in range(bits):
+                word = k * bits // 2 + (s * bits) // 16
+                bit = 16 * h + (s * bits) % 16 + i
+                pos[c, i] = 32 * word + bit
+    return pos
+
+
+def _tiled_codes(codes, bits):
+    codes = np.asarray(codes)
+    d_out, d_in = codes.shape
+    if codes.size and int(codes.max()) >= (1 << bits):
+        raise ValueError("code out of range for the bit width")
+    t = -(-d_out // PACK_ROWS)
+    g = -(-d_in // PACK_COLS)
+    full = np.zeros((t * PACK_ROWS, g * PACK_COLS), dtype=np.uint8)
+    full[:d_out, :d_in] = codes
+    # [tile][group][row in tile][column in group]
+    return full.reshape(t, PACK_ROWS, g, PACK_COLS).transpose(0, 2, 1, 3)
+
+
+def pack_codes(codes, bits: int) -> np.ndarray:
+    """Packed form (uint8, packed_bytes(d_out, d_in, bits) bytes) of a d_out x d_in code array."""
+    tiled = _tiled_codes(codes, bits)
+    pos = code_bit_positions(bits)
+    t, g = tiled.shape[:2]
+    bitarr = np.zeros((t, g, PACK_ROWS, PACK_COLS * bits), dtype=np.uint8)
+    for i in range(bits):
+        bitarr[..., pos[:, i]] = (tiled >> i) & 1
+    # bit j of the row's bit string is bit (j mod 8) of byte j // 8 (little-endian words)
+    return np.packbits(bitarr, axis=-1, bitorder="little").reshape(-1)
+
+
+def unpack_codes(packed, d_out: int, d_in: int, bits: int) -> np.ndarray:
+    """Inverse of pack_codes: the d_out x d_in uint8 codes."""
+    packed = np.asarray(packed, dtype=np.uint8).reshape(-1)
+    if packed.size != packed_bytes(d_out, d_in, bits):
+        raise ValueError("packed size does not match the shape")
+    t = -(-d_out // PACK_ROWS)
+    g = -(-d_in // PACK_COLS)
+    bitarr = np.unpackbits(packed.reshape(t, g, PACK_ROWS, 16 * bits), axis=-1,
+                           bitorder="little")
+    pos = code_bit_positions(bits)
+    tiled = np.zeros((t, g, PACK_ROWS, PACK_COLS), dtype=np.uint8)
+    for i in range(bits):
+        tiled |= (bitarr[..., pos[:, i]] << i).astype(np.uint8)
+    full = tiled.transpose(0, 2, 1, 3).reshape(t * PACK_ROWS, g * PACK_COLS)
+    return full[:d_out, :d_in].copy()
+
+
+def dequantize_layer(codes, scale, zero, group: int = 0) -> np.ndarray:
+    """W^' = scale (codes - zero), element by element in fp64. scale/zero: d_out (group 0), or
+    d_out x ceil(d_in / group) with column j on grid j // group."""
+    c = np.asarray(codes, dtype=np.float64)
+    s = np.asarray(scale, dtype=np.float64)
+    z = np.asarray(zero, dtype=np.float64)
+    if group:
+        gi = np.arange(c.shape[1]) // group
+        s = s.reshape(c.shape[0], -1)[:, gi]
+        z = z.reshape(c.shape[0], -1)[:, gi]
+    else:
+        s = s.reshape(-1, 1)
+        z = z.reshape(-1, 1)
+    return s * (c - z)
+
+
+def fwht_last(m) -> np.ndarray:
+    """(I (x) H_b) applied along the last axis (b = largest power of two dividing its length),
+    unnormalised, by the Kronecker factorisation H_b = H_2 (x) ... (x) H_2: each factor adds and
+    subtracts the two halves of one binary index digit."""
+    m = np.array(m, dtype=np.float64)
+    d = m.shape[-1]
+    b = hadamard_block_size(d)
+    lead = m.shape[:-1]
+    v = m.reshape(-1, d // b, b)
+    h = 1
+    while h < b:
+        v = v.reshape(v.shape[0], d // b, b // (2 * h), 2, h)
+        a0 = v[:, :, :, 0, :].copy()
+        a1 = v[:, :, :, 1, :].copy()
+        v[:, :, :, 0, :] = a0 + a1
+        v[:, :, :, 1, :] = a0 - a1
+        h *= 2
+    return v.reshape(lead + (d,))
+
+
+def qlinear_dense(w_hat, x, s_x=None, s_g=None, sign_in=None, sign_out=None,
+                  flags: int = BIIP_FULL) -> np.ndarray:
+    """y = S_G^-1 U^T W^' V S_X^-1 x for each row x of `x` (tokens x d_in) -> tokens x d_out.
+
+    V = (1/sqrt(b_in)) (I (x) H_b_in) diag(sign_in), U likewise on the output side (the
+    transforms of biip); a flag that is off drops its factor.
+    """
+    w_hat = np.asarray(w_hat, dtype=np.float64)
+    d_out, d_in = w_hat.shape
+    xt = np.atleast_2d(np.asarray(x, dtype=np.float64)).copy()
+    if flags & SCALE_IN:
+        xt = xt / np.asarray(s_x, dtype=np.float64)[None, :]
+    if flags & ROTATE_IN:
+        xt = xt * np.asarray(sign_in, dtype=np.float64)[None, :]
+        xt = fwht_last(xt) / math.sqrt(hadamard_block_size(d_in))
+    yp = xt @ w_hat.T
+    if flags & ROTATE_OUT:
+        # U^T = diag(sign_out) (I (x) H_b) / sqrt(b): H_b is symmetric
+        yp = fwht_last(yp) / math.sqrt(hadamard_block_size(d_out))
+        yp = yp * np.asarray(sign_out, dtype=np.float64)[None, :]
+    if flags & SCALE_OUT:
+        yp = yp / np.asarray(s_g, dtype=np.float64)[None, :]
+    return yp
+
+
+def qlinear(x, codes, scale, zero, s_x=None, s_g=None, sign_in=None, sign_out=None,
+            flags: int = BIIP_FULL, group: int = 0) -> np.ndarray:
+    """The quantized layer on activations: qlinear_dense of the dequantized codes."""
+    return qlinear_dense(dequantize_layer(codes, scale, zero, group), x, s_x, s_g, sign_in,
+                         sign_out, flags)
 
 
 # ------------------------------------------------------------------------------------------

@@ -532,3 +532,123 @@ def test_follow_grid_adopts_only_near_ties():
     off = O.quantize_layer(w, k, None, 3, group=group,
                            follow_grid=(own["scale"] * 1.01, own["zero"] + 1))
     assert np.array_equal(off["scale"], own["scale"]) and np.array_equal(off["zero"], own["zero"])
+
+
+# ------------------------------------------------------------------ inference side
+
+@pytest.mark.parametrize("d", [1, 2, 8, 48, 64, 192])
+def test_fwht_matches_explicit_sylvester_blocks(d):
+    # (I (x) H_b) along the last axis equals the product with the textbook Sylvester blocks
+    r = rng(88)
+    m = r.standard_normal((3, d))
+    b = O.hadamard_block_size(d)
+    want = (m.reshape(3, d // b, b) @ O.sylvester(b).T).reshape(3, d)
+    np.testing.assert_allclose(O.fwht_last(m), want, rtol=0, atol=1e-12)
+    # H_b H_b = b I
+    np.testing.assert_allclose(O.fwht_last(O.fwht_last(m)), b * m, atol=1e-11)
+
+
+@pytest.mark.parametrize("flags", [15, 3, 12, 5, 10, 0])
+def test_qlinear_inverts_the_incoherence_processing(flags):
+    # With the unquantized W' = U S_G W S_X V^T in place of W^', the layer gives back W x:
+    # S_G^-1 U^T (U S_G W S_X V^T) V S_X^-1 = W. A transposed U or V, an inverted scale, or a
+    # sign taken on the wrong side of the Hadamard product breaks the identity.
+    r = rng(90)
+    d_out, d_in = 24, 40      # Hadamard blocks of 8 on both sides, several per vector
+    w, hx, hg, dxx, inv_n = _layer(r, d_out, d_in)
+    si = r.choice([-1, 1], d_in); so = r.choice([-1, 1], d_out)
+    out = O.biip(w, hx, hg, dxx, inv_n, si, so, flags)
+    x = 3.0 * r.standard_normal((5, d_in))
+    y = O.qlinear_dense(out["w"], x, out["s_x"], out["s_g"], si, so, flags)
+    np.testing.assert_allclose(y, x @ w.T, rtol=0, atol=1e-12 * np.abs(x @ w.T).max())
+    # the same map with explicit dense transforms
+    u = O.transform_matrix(d_out, so) if flags & O.ROTATE_OUT else np.eye(d_out)
+    v = O.transform_matrix(d_in, si) if flags & O.ROTATE_IN else np.eye(d_in)
+    wh = r.standard_normal((d_out, d_in))
+    dense = np.diag(1 / out["s_g"]) @ u.T @ wh @ v @ np.diag(1 / out["s_x"])
+    np.testing.assert_allclose(O.qlinear_dense(wh, x, out["s_x"], out["s_g"], si, so, flags),
+                               x @ dense.T, rtol=0, atol=1e-12 * np.abs(x @ dense.T).max())
+
+
+@pytest.mark.parametrize("group", [0, 16])
+def test_dequantize_matches_the_solve_and_the_rtn_bound(group):
+    r = rng(91)
+    d_out, d_in, bits = 6, 40, 3
+    w = r.standard_normal((d_out, d_in))
+    # the solve's own dequantized weights, kept in fp32 there
+    res = O.quantize_layer(w, O.cholinv(spd(r, d_in), 0.01), None, bits, group=group)
+    wq = O.dequantize_layer(res["codes"], res["scale"], res["zero"], group)
+    np.testing.assert_allclose(wq, res["w_hat"], rtol=2.0 ** -23, atol=0)
+    # diagonal H: the solve is round-to-nearest, so every element lies within half a step of
+    # its own group's grid (a zero point of the wrong sign or a column mapped to the wrong
+    # group's grid does not)
+    k = O.cholinv(np.diag(r.uniform(0.5, 2.0, d_in)), 0.01)
+    res = O.quantize_layer(w, k, None, bits, group=group)
+    wq = O.dequantize_layer(res["codes"], res["scale"], res["zero"], group)
+    sc = np.asarray(res["scale"], dtype=np.float64).reshape(d_out, -1)
+    per_el = sc[:, np.arange(d_in) // group] if group else np.repeat(sc, d_in, axis=1)
+    assert np.all(np.abs(wq - w) <= 0.5 * per_el * (1 + 1e-6))
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+@pytest.mark.parametrize("shape", [(1, 1), (5, 37), (130, 300), (128, 256)])
+def test_pack_roundtrip_size_and_density(bits, shape):
+    r = rng(92)
+    codes = r.integers(0, 1 << bits, size=shape).astype(np.uint8)
+    p = O.pack_codes(codes, bits)
+    t, g = -(-shape[0] // 128), -(-shape[1] // 128)
+    assert p.dtype == np.uint8 and p.size == O.packed_bytes(*shape, bits) == t * g * 2048 * bits
+    np.testing.assert_array_equal(O.unpack_codes(p, *shape, bits), codes)
+    # every code bit lands on its own bit, padding stays zero
+    pop = lambda a: int(np.unpackbits(a.view(np.uint8)).sum())
+    assert pop(p) == pop(codes)
+
+
+def test_pack_hand_worked_positions():
+    # single codes placed by hand; the expected byte follows the format's wording:
+    # row r of blob (t, g) starts at byte (t G + g) 2048 b + 16 b r; word w is bytes 4w..4w+3
+    def one(bits, shape, row, col, code):
+        c = np.zeros(shape, dtype=np.uint8)
+        c[row, col] = code
+        p = O.pack_codes(c, bits)
+        nz = {int(i): int(p[i]) for i in np.flatnonzero(p)}
+        return nz
+    # b=2, col 1 = 2*0+1: half 1 of word 0, bits 16-17 -> byte 2 holds 0b11
+    assert one(2, (1, 20), 0, 1, 3) == {2: 0x03}
+    # b=2, row 1, col 14 (s=7, h=0): word 0 bits 14-15 of row 1 (byte 32 + 1); code 2 -> bit 15
+    assert one(2, (2, 20), 1, 14, 2) == {33: 0x80}
+    # b=2, col 17 (chunk 1, s=0, h=1): word 1 bit 16 -> byte 6
+    assert one(2, (1, 20), 0, 17, 1) == {6: 0x01}
+    # b=4, col 9 (chunk 0, s=4, h=1): word floor(16/16)=1, bits 16-19 -> byte 6 low nibble
+    assert one(4, (1, 20), 0, 9, 0xA) == {6: 0x0A}
+    # b=3, col 11 (s=5, h=1): word 1, bits 16-18 -> byte 6 holds the code
+    assert one(3, (1, 40), 0, 11, 6) == {6: 0x06}
+    # b=3, col 30 (s=15, h=0): bit i of the code at bit 15 of word i; code 5 = bits 0 and 2
+    assert one(3, (1, 40), 0, 30, 5) == {1: 0x80, 9: 0x80}
+    # b=3, col 31 (s=15, h=1): bit 31 of words 0..2; code 2 = bit 1 -> byte 7, bit 7
+    assert one(3, (1, 40), 0, 31, 2) == {7: 0x80}
+    # b=3, col 32 (chunk 1, s=0): word 3 bits 0-2 -> byte 12
+    assert one(3, (1, 40), 0, 32, 7) == {12: 0x07}
+    # second group of tile 0 (G = 2) and first group of tile 1 (row 128)
+    assert one(2, (1, 200), 0, 128, 1) == {4096: 0x01}
+    assert one(4, (129, 20), 128, 0, 1) == {8192: 0x01}
+
+
+def test_qlinear_of_codes_is_the_dense_layer_of_their_dequantization():
+    r = rng(93)
+    d_out, d_in, bits, group = 16, 48, 2, 16
+    codes = r.integers(0, 4, size=(d_out, d_in)).astype(np.uint8)
+    scale = r.uniform(0.01, 0.1, (d_out, 3)).astype(np.float32)
+    zero = r.integers(-1, 4, (d_out, 3)).astype(np.float32)
+    s_x = r.uniform(0.5, 2, d_in); s_g = r.uniform(0.5, 2, d_out)
+    si = r.choice([-1, 1], d_in); so = r.choice([-1, 1], d_out)
+    x = r.standard_normal((3, d_in))
+    y = O.qlinear(x, codes, scale, zero, s_x, s_g, si, so, O.BIIP_FULL, group)
+    # brute force: element-by-element dequantization, explicit dense transforms
+    wq = np.zeros((d_out, d_in))
+    for i in range(d_out):
+        for j in range(d_in):
+            wq[i, j] = float(scale[i, j // group]) * (int(codes[i, j]) - float(zero[i, j // group]))
+    u = O.transform_matrix(d_out, so); v = O.transform_matrix(d_in, si)
+    want = x @ (np.diag(1 / s_g) @ u.T @ wq @ v @ np.diag(1 / s_x)).T
+    np.testing.assert_allclose(y, want, rtol=0, atol=1e-12 * np.abs(want).max())
