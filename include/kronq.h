@@ -249,6 +249,73 @@ KRONQ_API kronq_status kronq_score_allocate(const double* tr_hx, const double* t
                                   int32_t n_choices, double avg_bits, double* score_out,
                                   int32_t* bits_out);
 
+/* ---------------------------------------------------------------------------------------
+ * 6. The quantized layer at inference: packed codes and y = W^ x.
+ *
+ * [KronQ-gist] Limitations: once quantized, the layer's inference overhead is only the
+ * orthogonal transforms (the same as QuIP#'s). The solve works on W' = U S_G W S_X V^T and
+ * returns codes, scale, zero with W^' = scale (codes - zero); in the original basis the layer is
+ *     y = S_G^-1 U^T W^' V S_X^-1 x,
+ * computed here without forming W^ or W^' in memory: x is transformed, multiplied by the
+ * packed codes on the tensor cores (dequantized on the fly in shared memory), and the result
+ * transformed back.
+ *
+ * Packed code format (this library's storage, the pages fix none). Bits b = 2, 3 or 4. Rows
+ * are cut into tiles of 128 and columns into groups of 128 (past the matrix: code 0). Tile t,
+ * group g is one blob of 2048 b bytes at byte offset (t G + g) 2048 b, G = ceil(d_in / 128).
+ * Inside it, row r takes 16 b bytes at offset 16 b r, read as little-endian 32-bit words w[];
+ * each word's low 16 bits hold codes of even columns, its high 16 bits codes of odd columns:
+ *   b = 2, 4: column 16 k + 2 s + h (s = 0..7, h = 0, 1) at word k b/2 + floor(s b / 16),
+ *             bits 16 h + (s b mod 16) and up;
+ *   b = 3:    column 32 k + 2 s + h (s = 0..15): s < 15 at word 3 k + floor(s / 5), bits
+ *             16 h + 3 (s mod 5) and up; s = 15: code bit i at bit 16 h + 15 of word 3 k + i.
+ * ------------------------------------------------------------------------------------- */
+/* Size in bytes of the packed form of a d_out x d_in code matrix (0 for an unsupported b). */
+KRONQ_API size_t kronq_packed_codes_bytes(int32_t d_out, int32_t d_in, int32_t bits);
+
+/* kronq_pack_codes - codes (device, uint8, d_out x d_in contiguous, each < 2^bits) -> packed
+ * (device, 16-byte aligned, packed_bytes >= kronq_packed_codes_bytes). Bits 2, 3, 4; others
+ * give KRONQ_ERR_UNSUPPORTED. Codes >= 2^bits are not checked (their extra bits spill into
+ * neighbouring codes). */
+KRONQ_API kronq_status kronq_pack_codes(const uint8_t* codes, int32_t d_out, int32_t d_in,
+                                        int32_t bits, void* packed, size_t packed_bytes,
+                                        kronq_stream_t stream);
+
+/* kronq_pack_grid - the grid (scale, zero from kronq_quantize_layer: d_out values each for
+ * group 0, d_out x ceil(d_in / 128) row-major for group 128) re-laid out for kronq_qlinear:
+ * (scale, zero) fp32 pairs, tile by tile of 128 rows, and within a tile group by group (group
+ * 128) or once (group 0): pair (t, g, r) at index (t G' + g) 128 + r, G' = ceil(d_in / 128) or 1;
+ * rows past d_out hold (0, 0). packed_grid: device, 8-byte aligned, at least
+ * kronq_packed_grid_bytes bytes. The values are copied, not changed. */
+KRONQ_API size_t kronq_packed_grid_bytes(int32_t d_out, int32_t d_in, int32_t group);
+KRONQ_API kronq_status kronq_pack_grid(const float* scale, const float* zero, int32_t d_out,
+                                       int32_t d_in, int32_t group, void* packed_grid,
+                                       size_t packed_grid_bytes, kronq_stream_t stream);
+
+/* kronq_qlinear - y = S_G^-1 U^T W^' V S_X^-1 x for n_tok tokens.
+ *
+ *   x        (device) n_tok x d_in, x_dtype KRONQ_DTYPE_BF16 or KRONQ_DTYPE_F32, row stride ld_x
+ *            elements (>= d_in), aligned to its element size
+ *   packed   (device, 16-byte aligned) codes in the packed format above
+ *   packed_grid (device, 8-byte aligned) the grid from kronq_pack_grid with the same group
+ *   s_x, s_g, sign_in, sign_out, flags: the transforms of kronq_biip (KRONQ_BIIP_SCALE_IN,
+ *            _SCALE_OUT, _ROTATE_IN, _ROTATE_OUT; a flag that is off drops its factor and its
+ *            pointer may be NULL). Hadamard blocks up to 16384.
+ *   y        (device, fp32) n_tok x d_out, row stride ld_y (>= d_out)
+ *   Tokens are processed 32 at a time; each group of 32 reads the packed codes once. Deterministic:
+ *   the same inputs give the same bits. Arithmetic: x' = V S_X^-1 x in fp32, split into two bf16
+ *   terms; codes exact in bf16; products on tcgen05 tensor cores with fp32 accumulation; the
+ *   grid, zero point and output transforms in fp32.
+ * ------------------------------------------------------------------------------------- */
+KRONQ_API size_t kronq_qlinear_workspace_size(int32_t d_out, int32_t d_in, int32_t n_tok);
+KRONQ_API kronq_status kronq_qlinear(const void* x, int32_t x_dtype, int64_t ld_x, int32_t n_tok,
+                                     const void* packed, const void* packed_grid,
+                                     int32_t group, const float* s_x, const float* s_g,
+                                     const int8_t* sign_in, const int8_t* sign_out,
+                                     uint32_t flags, int32_t d_out, int32_t d_in, int32_t bits,
+                                     float* y, int64_t ld_y, void* workspace,
+                                     size_t workspace_bytes, kronq_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -411,14 +411,18 @@ def quantize_layer(w, k, dxx=None, bits: int = 4, follow_codes=None, tie_tol: fl
 # Packed code format (a storage format of this library; the pages do not fix one). Codes of
 # b = 2, 3 or 4 bits. Rows are cut into tiles of 128, columns into groups of 128; rows and
 # columns past the matrix hold code 0. Tile t, group g is one blob of 128 x 128 x b bits at byte
-# offset (t * G + g) * 2048 * b (G = ceil(d_in / 128)); inside it, row r takes 16 * b bytes at
-# offset r * 16 * b, read as little-endian 32-bit words w[0 .. 4b). Each word's low 16 bits
-# ("half 0") hold codes of even columns, its high 16 bits ("half 1") codes of odd columns.
-#   b = 2 or 4: the row's 128 columns form 8 chunks of 16; column 16 k + 2 s + h (s = 0..7,
-#     h = 0, 1) sits in word k b / 2 + floor(s b / 16) at bits 16 h + (s b mod 16) and up.
-#   b = 3: 4 chunks of 32 columns; column 32 k + 2 s + h (s = 0..15): for s < 15, word
-#     3 k + floor(s / 5) at bits 16 h + 3 (s mod 5) and up; for s = 15, bit i of the code
-#     (i = 0, 1, 2) is bit 16 h + 15 of word 3 k + i.
+# offset (t * G + g) * 2048 * b (G = ceil(d_in / 128)). Each row of the blob has a string of
+# 16 * b bytes, read as little-endian 32-bit words; the string is stored in 8-byte pieces,
+# piece p of row r at byte 1024 * p + 8 * r of the blob (so that 16 consecutive rows' pieces
+# are contiguous). Inside the words, code j of each run of 4 columns sits in byte j, so that
+# one shift and one mask turn a word into four 8-bit codes of consecutive columns:
+#   b = 2: word w holds columns 16 w .. 16 w + 15; column 16 w + 4 k + j (k, j = 0..3) at
+#          bits 8 j + 2 k and 8 j + 2 k + 1;
+#   b = 4: word w holds columns 8 w .. 8 w + 7; column 8 w + 4 k + j (k = 0, 1) at bits
+#          8 j + 4 k .. 8 j + 4 k + 3;
+#   b = 3: each 32 columns 32 m .. 32 m + 31 take words 3 m, 3 m + 1, 3 m + 2: the low two bits
+#          of columns 32 m .. + 15 and 32 m + 16 .. + 31 in words 3 m and 3 m + 1 as for b = 2,
+#          and the top bit of column 32 m + 4 k + j (k = 0..7) at bit 8 j + k of word 3 m + 2.
 
 PACK_ROWS = 128
 PACK_COLS = 128
@@ -436,25 +440,27 @@ def packed_bytes(d_out: int, d_in: int, bits: int) -> int:
 
 def code_bit_positions(bits: int) -> np.ndarray:
     """(128, bits) array: for column c of a group and code bit i, the bit index (32 * word +
-    bit in word) of that bit inside the row's 16 * bits bytes, following the format above."""
+    bit in word) of that bit inside the row's string of 16 * bits bytes, following the format
+    above."""
     if bits not in PACK_BITS:
         raise ValueError("packed codes have 2, 3 or 4 bits")
     pos = np.zeros((PACK_COLS, bits), dtype=np.int64)
     for c in range(PACK_COLS):
-        if bits == 3:
-            k, s, h = c // 32, (c % 32) // 2, c % 2
-            for i in range(3):
-                if s < 15:
-                    word, bit = 3 * k + s // 5, 16 * h + 3 * (s % 5) + i
-                else:
-                    word, bit = 3 * k + i, 16 * h + 15
-                pos[c, i] = 32 * word + bit
+        if bits == 2:
+            w, k, j = c // 16, (c % 16) // 4, c % 4
+            for i in range(2):
+                pos[c, i] = 32 * w + 8 * j + 2 * k + i
+        elif bits == 4:
+            w, k, j = c // 8, (c % 8) // 4, c % 4
+            for i in range(4):
+                pos[c, i] = 32 * w + 8 * j + 4 * k + i
         else:
-            k, s, h = c // 16, (c % 16) // 2, c % 2
-            for i in range(bits):
-                word = k * bits // 2 + (s * bits) // 16
-                bit = 16 * h + (s * bits) % 16 + i
-                pos[c, i] = 32 * word + bit
+            m, cc = c // 32, c % 32
+            w, k, j = 3 * m + cc // 16, (cc % 16) // 4, cc % 4
+            for i in range(2):
+                pos[c, i] = 32 * w + 8 * j + 2 * k + i
+            k8 = cc // 4
+            pos[c, 2] = 32 * (3 * m + 2) + 8 * j + k8
     return pos
 
 
@@ -480,7 +486,10 @@ def pack_codes(codes, bits: int) -> np.ndarray:
     for i in range(bits):
         bitarr[..., pos[:, i]] = (tiled >> i) & 1
     # bit j of the row's bit string is bit (j mod 8) of byte j // 8 (little-endian words)
-    return np.packbits(bitarr, axis=-1, bitorder="little").reshape(-1)
+    rowstr = np.packbits(bitarr, axis=-1, bitorder="little")       # t, g, 128 rows, 16 b
+    # 8-byte pieces: blob byte 1024 p + 8 r + k holds byte 8 p + k of row r's string
+    pieces = rowstr.reshape(t, g, PACK_ROWS, 2 * bits, 8).transpose(0, 1, 3, 2, 4)
+    return np.ascontiguousarray(pieces).reshape(-1)
 
 
 def unpack_codes(packed, d_out: int, d_in: int, bits: int) -> np.ndarray:
@@ -490,14 +499,33 @@ def unpack_codes(packed, d_out: int, d_in: int, bits: int) -> np.ndarray:
         raise ValueError("packed size does not match the shape")
     t = -(-d_out // PACK_ROWS)
     g = -(-d_in // PACK_COLS)
-    bitarr = np.unpackbits(packed.reshape(t, g, PACK_ROWS, 16 * bits), axis=-1,
-                           bitorder="little")
+    rowstr = packed.reshape(t, g, 2 * bits, PACK_ROWS, 8).transpose(0, 1, 3, 2, 4)
+    bitarr = np.unpackbits(np.ascontiguousarray(rowstr).reshape(t, g, PACK_ROWS, 16 * bits),
+                           axis=-1, bitorder="little")
     pos = code_bit_positions(bits)
     tiled = np.zeros((t, g, PACK_ROWS, PACK_COLS), dtype=np.uint8)
     for i in range(bits):
         tiled |= (bitarr[..., pos[:, i]] << i).astype(np.uint8)
     full = tiled.transpose(0, 2, 1, 3).reshape(t * PACK_ROWS, g * PACK_COLS)
     return full[:d_out, :d_in].copy()
+
+
+def pack_grid(scale, zero, d_out: int, d_in: int, group: int = 0) -> np.ndarray:
+    """The grid as (scale, zero) float32 pairs, tile by tile of 128 rows and, within a tile,
+    group by group (group 128) or once (group 0): pair (t, g, r) at (t G' + g) 128 + r;
+    rows past d_out hold (0, 0). Returns an array of shape (pairs, 2)."""
+    t = -(-d_out // PACK_ROWS)
+    gp = -(-d_in // PACK_COLS) if group else 1
+    sc = np.zeros((t * PACK_ROWS, gp), dtype=np.float32)
+    zr = np.zeros((t * PACK_ROWS, gp), dtype=np.float32)
+    sc[:d_out] = np.asarray(scale, dtype=np.float32).reshape(d_out, gp)
+    zr[:d_out] = np.asarray(zero, dtype=np.float32).reshape(d_out, gp)
+    out = np.zeros((t, gp, PACK_ROWS, 2), dtype=np.float32)
+    for ti in range(t):
+        for gi in range(gp):
+            out[ti, gi, :, 0] = sc[ti * PACK_ROWS:(ti + 1) * PACK_ROWS, gi]
+            out[ti, gi, :, 1] = zr[ti * PACK_ROWS:(ti + 1) * PACK_ROWS, gi]
+    return out.reshape(-1, 2)
 
 
 def dequantize_layer(codes, scale, zero, group: int = 0) -> np.ndarray:
@@ -536,6 +564,32 @@ def fwht_last(m) -> np.ndarray:
     return v.reshape(lead + (d,))
 
 
+def qlinear_input(x, s_x=None, sign_in=None, flags: int = BIIP_FULL) -> np.ndarray:
+    """x' = V S_X^-1 x for each row x of `x` (tokens x d_in), V = (1/sqrt(b)) (I (x) H_b)
+    diag(sign_in) as in biip; a flag that is off drops its factor."""
+    xt = np.atleast_2d(np.asarray(x, dtype=np.float64)).copy()
+    d_in = xt.shape[1]
+    if flags & SCALE_IN:
+        xt = xt / np.asarray(s_x, dtype=np.float64)[None, :]
+    if flags & ROTATE_IN:
+        xt = xt * np.asarray(sign_in, dtype=np.float64)[None, :]
+        xt = fwht_last(xt) / math.sqrt(hadamard_block_size(d_in))
+    return xt
+
+
+def qlinear_output(yp, s_g=None, sign_out=None, flags: int = BIIP_FULL) -> np.ndarray:
+    """y = S_G^-1 U^T y' for each row y' of `yp` (tokens x d_out)."""
+    yp = np.atleast_2d(np.asarray(yp, dtype=np.float64)).copy()
+    d_out = yp.shape[1]
+    if flags & ROTATE_OUT:
+        # U^T = diag(sign_out) (I (x) H_b) / sqrt(b): H_b is symmetric
+        yp = fwht_last(yp) / math.sqrt(hadamard_block_size(d_out))
+        yp = yp * np.asarray(sign_out, dtype=np.float64)[None, :]
+    if flags & SCALE_OUT:
+        yp = yp / np.asarray(s_g, dtype=np.float64)[None, :]
+    return yp
+
+
 def qlinear_dense(w_hat, x, s_x=None, s_g=None, sign_in=None, sign_out=None,
                   flags: int = BIIP_FULL) -> np.ndarray:
     """y = S_G^-1 U^T W^' V S_X^-1 x for each row x of `x` (tokens x d_in) -> tokens x d_out.
@@ -544,21 +598,8 @@ def qlinear_dense(w_hat, x, s_x=None, s_g=None, sign_in=None, sign_out=None,
     transforms of biip); a flag that is off drops its factor.
     """
     w_hat = np.asarray(w_hat, dtype=np.float64)
-    d_out, d_in = w_hat.shape
-    xt = np.atleast_2d(np.asarray(x, dtype=np.float64)).copy()
-    if flags & SCALE_IN:
-        xt = xt / np.asarray(s_x, dtype=np.float64)[None, :]
-    if flags & ROTATE_IN:
-        xt = xt * np.asarray(sign_in, dtype=np.float64)[None, :]
-        xt = fwht_last(xt) / math.sqrt(hadamard_block_size(d_in))
-    yp = xt @ w_hat.T
-    if flags & ROTATE_OUT:
-        # U^T = diag(sign_out) (I (x) H_b) / sqrt(b): H_b is symmetric
-        yp = fwht_last(yp) / math.sqrt(hadamard_block_size(d_out))
-        yp = yp * np.asarray(sign_out, dtype=np.float64)[None, :]
-    if flags & SCALE_OUT:
-        yp = yp / np.asarray(s_g, dtype=np.float64)[None, :]
-    return yp
+    xp = qlinear_input(x, s_x, sign_in, flags)
+    return qlinear_output(xp @ w_hat.T, s_g, sign_out, flags)
 
 
 def qlinear(x, codes, scale, zero, s_x=None, s_g=None, sign_in=None, sign_out=None,

@@ -311,6 +311,108 @@ kronq_status kronq_quantize_layer(const float* w, const float* k, const float* d
                       workspace, reinterpret_cast<cudaStream_t>(stream));
 }
 
+// ----------------------------------------------------------------------------- inference
+size_t kronq_packed_codes_bytes(int32_t d_out, int32_t d_in, int32_t bits) {
+  if (d_out <= 0 || d_in <= 0 || bits < 2 || bits > 4) return 0;
+  return packed_code_bytes(d_out, d_in, bits);
+}
+
+kronq_status kronq_pack_codes(const uint8_t* codes, int32_t d_out, int32_t d_in, int32_t bits,
+                              void* packed, size_t packed_bytes, kronq_stream_t stream) {
+  if (d_out <= 0 || d_in <= 0) return fail(KRONQ_ERR_SHAPE, "d_out and d_in must be positive");
+  if (bits < 2 || bits > 4) return fail(KRONQ_ERR_UNSUPPORTED, "packed codes have 2, 3 or 4 bits");
+  if (!codes || !packed) return fail(KRONQ_ERR_INVALID_ARG, "codes and packed are required");
+  if (!aligned(packed, 16)) return fail(KRONQ_ERR_INVALID_ARG, "packed not 16-byte aligned");
+  if (packed_bytes < packed_code_bytes(d_out, d_in, bits))
+    return fail(KRONQ_ERR_SHAPE, "packed buffer too small: %zu < %zu bytes", packed_bytes,
+                packed_code_bytes(d_out, d_in, bits));
+  KQ_TRY(kronq_device_check());
+  return run_pack_codes(codes, d_out, d_in, bits, packed, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t kronq_packed_grid_bytes(int32_t d_out, int32_t d_in, int32_t group) {
+  if (d_out <= 0 || d_in <= 0 || (group != 0 && group != 128)) return 0;
+  return packed_grid_bytes(d_out, d_in, group);
+}
+
+kronq_status kronq_pack_grid(const float* scale, const float* zero, int32_t d_out, int32_t d_in,
+                             int32_t group, void* packed_grid, size_t packed_grid_bytes_,
+                             kronq_stream_t stream) {
+  if (d_out <= 0 || d_in <= 0) return fail(KRONQ_ERR_SHAPE, "d_out and d_in must be positive");
+  if (group != 0 && group != 128)
+    return fail(KRONQ_ERR_UNSUPPORTED, "group must be 0 (per row) or 128");
+  if (!scale || !zero || !packed_grid)
+    return fail(KRONQ_ERR_INVALID_ARG, "scale, zero and packed_grid are required");
+  if (!aligned(packed_grid, 8)) return fail(KRONQ_ERR_INVALID_ARG, "packed_grid not 8-byte aligned");
+  if (packed_grid_bytes_ < packed_grid_bytes(d_out, d_in, group))
+    return fail(KRONQ_ERR_SHAPE, "packed_grid too small: %zu < %zu bytes", packed_grid_bytes_,
+                packed_grid_bytes(d_out, d_in, group));
+  KQ_TRY(kronq_device_check());
+  return run_pack_grid(scale, zero, d_out, d_in, group, packed_grid,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t kronq_qlinear_workspace_size(int32_t d_out, int32_t d_in, int32_t n_tok) {
+  if (d_out <= 0 || d_in <= 0 || n_tok <= 0) return 0;
+  return qlinear_workspace_bytes(d_out, d_in, n_tok);
+}
+
+kronq_status kronq_qlinear(const void* x, int32_t x_dtype, int64_t ld_x, int32_t n_tok,
+                           const void* packed, const void* packed_grid, int32_t group, const float* s_x, const float* s_g,
+                           const int8_t* sign_in, const int8_t* sign_out, uint32_t flags,
+                           int32_t d_out, int32_t d_in, int32_t bits, float* y, int64_t ld_y,
+                           void* workspace, size_t workspace_bytes, kronq_stream_t stream) {
+  if (d_out <= 0 || d_in <= 0 || n_tok < 0)
+    return fail(KRONQ_ERR_SHAPE, "d_out, d_in must be positive and n_tok >= 0");
+  if (bits < 2 || bits > 4) return fail(KRONQ_ERR_UNSUPPORTED, "packed codes have 2, 3 or 4 bits");
+  if (group != 0 && group != 128)
+    return fail(KRONQ_ERR_UNSUPPORTED, "group must be 0 (per row) or 128");
+  if (flags & ~static_cast<uint32_t>(KRONQ_BIIP_FULL))
+    return fail(KRONQ_ERR_INVALID_ARG, "flags may only hold the four transform bits");
+  if (x_dtype != KRONQ_DTYPE_BF16 && x_dtype != KRONQ_DTYPE_F32)
+    return fail(KRONQ_ERR_INVALID_ARG, "x_dtype must be KRONQ_DTYPE_BF16 or KRONQ_DTYPE_F32");
+  if (n_tok == 0) return KRONQ_OK;
+  if (!x || !packed || !packed_grid || !y)
+    return fail(KRONQ_ERR_INVALID_ARG, "x, packed, packed_grid and y are required");
+  if ((flags & KRONQ_BIIP_SCALE_IN) && !s_x) return fail(KRONQ_ERR_INVALID_ARG, "s_x is NULL");
+  if ((flags & KRONQ_BIIP_SCALE_OUT) && !s_g) return fail(KRONQ_ERR_INVALID_ARG, "s_g is NULL");
+  if ((flags & KRONQ_BIIP_ROTATE_IN) && !sign_in)
+    return fail(KRONQ_ERR_INVALID_ARG, "sign_in is NULL");
+  if ((flags & KRONQ_BIIP_ROTATE_OUT) && !sign_out)
+    return fail(KRONQ_ERR_INVALID_ARG, "sign_out is NULL");
+  if (ld_x < d_in || ld_y < d_out) return fail(KRONQ_ERR_SHAPE, "row stride below the width");
+  if (!aligned(x, x_dtype == KRONQ_DTYPE_BF16 ? 2 : 4) || !aligned(y, 4))
+    return fail(KRONQ_ERR_INVALID_ARG, "x or y not aligned to its element size");
+  if (!aligned(packed, 16)) return fail(KRONQ_ERR_INVALID_ARG, "packed not 16-byte aligned");
+  if (!aligned(packed_grid, 8))
+    return fail(KRONQ_ERR_INVALID_ARG, "packed_grid not 8-byte aligned");
+  const int b_in = d_in & (-d_in), b_out = d_out & (-d_out);
+  if (((flags & KRONQ_BIIP_ROTATE_IN) && b_in > 16384) ||
+      ((flags & KRONQ_BIIP_ROTATE_OUT) && b_out > 16384))
+    return fail(KRONQ_ERR_UNSUPPORTED, "Hadamard blocks above 16384 are not supported");
+  KQ_TRY(check_ws(workspace, workspace_bytes, qlinear_workspace_bytes(d_out, d_in, n_tok)));
+  KQ_TRY(kronq_device_check());
+  QlinearArgs q;
+  q.x = x;
+  q.x_dtype = x_dtype;
+  q.ld_x = ld_x;
+  q.n_tok = n_tok;
+  q.packed = packed;
+  q.grid = packed_grid;
+  q.group = group;
+  q.s_x = s_x;
+  q.s_g = s_g;
+  q.sign_in = sign_in;
+  q.sign_out = sign_out;
+  q.flags = flags;
+  q.d_out = d_out;
+  q.d_in = d_in;
+  q.bits = bits;
+  q.y = y;
+  q.ld_y = ld_y;
+  return run_qlinear(q, workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
 // ----------------------------------------------------------------------------- allocation
 kronq_status kronq_score_allocate(const double* tr_hx, const double* tr_hg,
                                   const int64_t* n_params, int32_t L, const int32_t* choices,

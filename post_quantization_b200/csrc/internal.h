@@ -49,6 +49,33 @@ kronq_status run_quantize(const float* w, const float* k, const float* dxx, int 
                           int bits, int block, int group, uint8_t* codes, float* scale,
                           float* zero, float* w_hat, void* ws, cudaStream_t stream);
 
+// qlinear.cu: the quantized layer at inference (packed codes, input/output transforms).
+struct QlinearArgs {
+  const void* x;
+  int x_dtype;
+  int64_t ld_x;
+  int n_tok;
+  const void* packed;
+  const void* grid;
+  int group;
+  const float* s_x;
+  const float* s_g;
+  const int8_t* sign_in;
+  const int8_t* sign_out;
+  uint32_t flags;
+  int d_out, d_in, bits;
+  float* y;
+  int64_t ld_y;
+};
+size_t packed_code_bytes(int d_out, int d_in, int bits);
+kronq_status run_pack_codes(const uint8_t* codes, int d_out, int d_in, int bits, void* packed,
+                            cudaStream_t stream);
+size_t packed_grid_bytes(int d_out, int d_in, int group);
+kronq_status run_pack_grid(const float* scale, const float* zero, int d_out, int d_in, int group,
+                           void* packed, cudaStream_t stream);
+size_t qlinear_workspace_bytes(int d_out, int d_in, int n_tok);
+kronq_status run_qlinear(const QlinearArgs& q, void* ws, cudaStream_t stream);
+
 // Zero structure of GEMM operands (the zeros must be stored), used to skip K ranges:
 //   GEMM_A_UPPER  A[m][k] = 0 for k < m
 //   GEMM_B_UPPER  op(B)[k][n] = 0 for k > n

@@ -1,0 +1,1042 @@
+// The quantized layer at inference: packed 2/3/4-bit codes and
+//     y = S_G^-1 U^T W^' V S_X^-1 x,   W^' = scale (codes - zero)
+// ([KronQ-gist] Limitations: at inference the only overhead is the orthogonal transforms).
+//
+// Three kernels per pass of up to 32 tokens, chained with programmatic dependent launch so
+// that each one's launch overlaps its predecessor:
+//   qlin_in_kernel   x' = V S_X^-1 x (scale, sign, Hadamard blocks: radix-16 passes in shared
+//                    memory), cut into 128-column groups, each written as three int8 terms
+//                    x' ~ s (q0 + q1 / 128 + q2 / 128^2) with a power-of-two s per group and
+//                    token: the tensor-core B operand, pre-swizzled, plus (s, sum of the terms)
+//                    per group for the zero point.
+//   qlin_mma_kernel  persistent CTAs stream the packed codes (bulk copies of several units at
+//                    once into a ring of stages); eight warps turn each 128 x 128 blob into
+//                    8-bit codes in tensor memory (one shift and one mask per four codes,
+//                    tcgen05.st); tcgen05.mma kind::i8 multiplies them, exactly, with the int8
+//                    terms of x'; four epilogue warps apply the grid, the group scale and the
+//                    within-tile part of U^T, and write one partial per (CTA, row tile). Work is
+//                    split over CTAs as contiguous ranges of (row tile, column group) units.
+//   qlin_out_kernel  sums each tile's partials in a fixed order (deterministic), applies the
+//                    across-tile part of U^T, the signs and S_G^-1.
+// The codes are the MMA's A operand (128 rows per instruction); a tcgen05 MMA costs about the
+// same time for any N up to 256, so the tokens ride along in N, and 8-bit operands (32 columns
+// per instruction, twice bf16's) halve the MMA time per code.
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include <algorithm>
+#include <cmath>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace kq {
+namespace {
+
+constexpr int QL_TILE = 128;            // rows per tile, columns per group
+constexpr int QL_NT_MAX = 32;           // tokens per pass
+constexpr int QL_THREADS = 512;         // 16 warps
+constexpr int QL_EPI_WARP0 = 4;         // warps 4..7: epilogue (TMEM lanes 32 (w % 4) ...)
+constexpr int QL_DQ_WARP0 = 8;          // warps 8..15: dequantization
+constexpr int QL_DQ_THREADS = 256;
+constexpr int QL_MAX_STAGES = 16;
+constexpr int QL_TERMS = 3;             // int8 terms of x'
+
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// 1-D bulk copy global -> shared, completion on `bar` (no multicast).
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes),
+      "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Named barrier that also returns the AND of a predicate over the participating threads.
+__device__ __forceinline__ bool bar_and(int id, int count, bool pred) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.b32 pi, %1, 0;\n\t"
+      "bar.red.and.pred po, %2, %3, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(out)
+      : "r"(pred ? 1u : 0u), "r"(id), "r"(count)
+      : "memory");
+  return out != 0;
+}
+
+// 32 lanes x 16 consecutive 32-bit TMEM columns.
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+// kind::i8: A unsigned 8-bit (codes), B signed 8-bit (terms of x'), both K-major, s32 accumulate.
+__host__ __device__ constexpr uint32_t ql_idesc(int m, int n) {
+  return (2u << 4) | (0u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
+         (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+// ---------------------------------------------------------------------------------------------
+// Packing
+// ---------------------------------------------------------------------------------------------
+// One thread per (padded row, chunk of 16 (b = 2), 8 (b = 4) or 32 (b = 3) columns) -> 1, 1 or 3
+// words, written where the packed format puts them.
+__global__ void pack_codes_kernel(const uint8_t* __restrict__ codes, int d_out, int d_in,
+                                  int bits, int groups, int rows_pad, uint32_t* __restrict__ out) {
+  const int cpg = bits == 2 ? 8 : (bits == 4 ? 16 : 4);     // chunks per 128-column group
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t total = static_cast<int64_t>(rows_pad) * groups * cpg;
+  if (idx >= total) return;
+  const int chunk = static_cast<int>(idx % cpg);
+  const int64_t rg = idx / cpg;
+  const int g = static_cast<int>(rg % groups);
+  const int row = static_cast<int>(rg / groups);
+  const int t = row / QL_TILE, r = row % QL_TILE;
+  const int width = QL_TILE / cpg;
+  const int col0 = g * QL_TILE + chunk * width;
+  auto code = [&](int k) -> uint32_t {
+    const int col = col0 + k;
+    return (row < d_out && col < d_in) ? codes[static_cast<int64_t>(row) * d_in + col] : 0u;
+  };
+  // word j of row r's string in blob (t, g): 8-byte piece j / 2 at 1024 (j / 2) + 8 r, word
+  // j % 2 inside it
+  uint32_t* blob = out + (static_cast<int64_t>(t) * groups + g) * (512 * bits);
+  auto put = [&](int j, uint32_t w) { blob[(j >> 1) * 256 + 2 * r + (j & 1)] = w; };
+  if (bits == 2) {
+    uint32_t w = 0u;
+    for (int k = 0; k < 4; ++k)
+      for (int j = 0; j < 4; ++j) w |= (code(4 * k + j) & 3u) << (8 * j + 2 * k);
+    put(chunk, w);
+  } else if (bits == 4) {
+    uint32_t w = 0u;
+    for (int k = 0; k < 2; ++k)
+      for (int j = 0; j < 4; ++j) w |= (code(4 * k + j) & 15u) << (8 * j + 4 * k);
+    put(chunk, w);
+  } else {
+    uint32_t w[3] = {0u, 0u, 0u};
+    for (int c = 0; c < 32; ++c) {
+      const uint32_t v = code(c);
+      const int cc = c & 15, k = cc >> 2, j = cc & 3;
+      w[c >> 4] |= (v & 3u) << (8 * j + 2 * k);
+      w[2] |= ((v >> 2) & 1u) << (8 * (c & 3) + (c >> 2));
+    }
+    for (int i = 0; i < 3; ++i) put(3 * chunk + i, w[i]);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Input side: x' = V S_X^-1 x, split into the B operand
+// ---------------------------------------------------------------------------------------------
+struct QlInArgs {
+  const void* x;
+  int x_dtype;
+  int64_t ld_x;
+  int n_tok;           // tokens of this pass
+  int d_in;
+  int span;            // columns per CTA: max(b_in, 128)
+  int b_in;
+  const float* s_x;
+  const int8_t* sign_in;
+  uint32_t flags;
+  float inv_sqrt_b;
+  int rows;            // B rows: 3 n_tok rounded up to 8
+  uint8_t* bop;        // groups x [rows][128 bytes]: row 3 t + k = term k of token t
+  float2* sums;        // groups x n_tok: (s, q0 + q1 / 128 + q2 / 128^2 summed over the group)
+};
+
+// One CTA per (span of columns, token), span / 16 threads (at least 32): thread t owns the 16
+// consecutive columns 16t..16t+15 at the end. The Hadamard stages run as radix-16 passes: in
+// the pass over index bits [4p, 4p + 4) each thread gathers the 16 elements that differ only in
+// those bits from shared memory and applies the four stages in registers.
+__global__ void __launch_bounds__(1024) qlin_in_kernel(QlInArgs a) {
+  extern __shared__ float xs[];                 // span floats
+  griddep_launch_dependents();
+  // x may be the output of the kernel before this one; the launch itself overlaps it
+  griddep_wait();
+  const int tid = threadIdx.x;
+  const int nthr = blockDim.x;
+  const int nwork = a.span >> 4;                // threads that own 16 columns
+  const int t = blockIdx.y;
+  const int j0 = blockIdx.x * a.span;
+  const int len = min(a.span, a.d_in - j0);
+  const bool rot = (a.flags & KRONQ_BIIP_ROTATE_IN) != 0;
+  const bool scl = (a.flags & KRONQ_BIIP_SCALE_IN) != 0;
+  for (int j = tid; j < a.span; j += nthr) {
+    float v = 0.f;
+    if (j < len) {
+      const int64_t o = static_cast<int64_t>(t) * a.ld_x + j0 + j;
+      v = a.x_dtype == KRONQ_DTYPE_BF16
+              ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(a.x)[o])
+              : reinterpret_cast<const float*>(a.x)[o];
+      if (scl) v = v / a.s_x[j0 + j];
+      if (rot) v = a.sign_in[j0 + j] < 0 ? -v : v;
+    }
+    xs[j] = v;
+  }
+  __syncthreads();
+  if (rot && a.b_in > 1) {
+    const int L = 31 - __clz(a.b_in);
+    int sh = 0;
+    for (; sh + 4 <= L; sh += 4) {
+      if (tid < nwork) {
+        const int lo = tid & ((1 << sh) - 1);
+        const int base = lo | ((tid >> sh) << (sh + 4));
+        float v[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = xs[base + (j << sh)];
+#pragma unroll
+        for (int h = 1; h < 16; h <<= 1)
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (!(j & h)) {
+              const float u = v[j], w = v[j + h];
+              v[j] = u + w;
+              v[j + h] = u - w;
+            }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) xs[base + (j << sh)] = v[j];
+      }
+      __syncthreads();
+    }
+    for (; sh < L; ++sh) {                      // remaining 1..3 stages, pairwise
+      const int h = 1 << sh;
+      for (int pi = tid; pi < a.span / 2; pi += nthr) {
+        const int i = ((pi >> sh) << (sh + 1)) | (pi & (h - 1));
+        const float u = xs[i], w = xs[i + h];
+        xs[i] = u + w;
+        xs[i + h] = u - w;
+      }
+      __syncthreads();
+    }
+  }
+  // B operand: thread = 16 columns = one 16-byte unit of each of the token's three term rows;
+  // a group's 128 columns belong to 8 consecutive threads (its maximum and sums by shuffles)
+  float xv[16];
+  float amax = 0.f;
+  if (tid < nwork) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float v = 16 * tid + e < len ? (rot ? xs[16 * tid + e] * a.inv_sqrt_b
+                                                : xs[16 * tid + e])
+                                         : 0.f;
+      xv[e] = v;
+      amax = fmaxf(amax, fabsf(v));
+    }
+  }
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  // s = the smallest power of two with 127 s >= max |x'| over the group (1 for a zero group)
+  float sc = 1.f;
+  if (amax > 0.f) {
+    int ex;
+    const float m = frexpf(amax / 127.f, &ex);    // amax / 127 = m 2^ex, m in [0.5, 1)
+    sc = ldexpf(1.f, m == 0.5f ? ex - 1 : ex);
+  }
+  const float inv_sc = 1.f / sc;                 // exact: a power of two
+  int qsum[QL_TERMS] = {0, 0, 0};
+  uint32_t wq[QL_TERMS][4];
+  if (tid < nwork) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      float r = xv[e] * inv_sc;                   // exact; |r| <= 127
+      int q[QL_TERMS];
+#pragma unroll
+      for (int k = 0; k < QL_TERMS; ++k) {
+        q[k] = __float2int_rn(r);                 // |q0| <= 127, |q1|, |q2| <= 64
+        r = (r - static_cast<float>(q[k])) * 128.f;   // exact
+        qsum[k] += q[k];
+      }
+#pragma unroll
+      for (int k = 0; k < QL_TERMS; ++k) {
+        const uint32_t byte = static_cast<uint32_t>(q[k]) & 0xFFu;
+        if ((e & 3) == 0) wq[k][e >> 2] = byte;
+        else wq[k][e >> 2] |= byte << (8 * (e & 3));
+      }
+    }
+    const int c0 = j0 + 16 * tid;                 // 16 columns never straddle a group
+    const int g = c0 / QL_TILE, unit = (c0 % QL_TILE) >> 4;
+    uint8_t* gb = a.bop + static_cast<int64_t>(g) * (128 * a.rows);
+#pragma unroll
+    for (int k = 0; k < QL_TERMS; ++k) {
+      const int rho = QL_TERMS * t + k;
+      *reinterpret_cast<uint4*>(gb + rho * 128 + ((unit ^ (rho & 7)) << 4)) =
+          make_uint4(wq[k][0], wq[k][1], wq[k][2], wq[k][3]);
+    }
+  }
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1)
+#pragma unroll
+    for (int k = 0; k < QL_TERMS; ++k) qsum[k] += __shfl_xor_sync(0xffffffffu, qsum[k], o);
+  if (tid < nwork && (tid & 7) == 0) {
+    // exact integers, combined once in fp32
+    const float qs = static_cast<float>(qsum[0]) + static_cast<float>(qsum[1]) * (1.f / 128.f) +
+                     static_cast<float>(qsum[2]) * (1.f / 16384.f);
+    a.sums[static_cast<int64_t>((j0 + 16 * tid) / QL_TILE) * a.n_tok + t] = make_float2(sc, qs);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// The tensor-core pass over the packed codes
+// ---------------------------------------------------------------------------------------------
+struct QlMmaArgs {
+  const uint8_t* packed;
+  const uint8_t* bop;
+  const float2* sums;
+  const float2* grid;  // packed (scale, zero): [tile][group][128] or [tile][128]
+  float* partial;      // (C + T) segments x n_tok x 128
+  int d_out, T, G;
+  int n_tok, N;        // tokens; MMA N = 3 n_tok rounded up to 16
+  int R;               // B rows in memory: 3 n_tok rounded up to 8
+  int ku;              // units per pipeline stage (one bulk copy of codes, one of B)
+  int grouped;         // 1: grid per row and 128-column group
+  int rotate_out;
+  int b_tile;          // Hadamard block inside a tile: min(b_out, 128) (1 without rotation)
+  int64_t U;           // units = T G
+  int stages;
+  int* err;
+};
+
+__device__ __forceinline__ int64_t unit_begin(int64_t c, int64_t U, int64_t C) {
+  return (c * U) / C;
+}
+
+// Dequantization of one row's half (64 columns) of a 128 x 128 blob into 16 registers of four
+// 8-bit codes each (register j = columns 4j .. 4j + 3 of the half). The row's string is read as
+// 8-byte pieces (piece p of row r at 1024 p + 8 r): the 32 lanes of a warp read 32 consecutive
+// rows, so every read is free of bank conflicts.
+template <int BITS>
+__device__ __forceinline__ void dequant_half_row(const uint8_t* pk, int r, int kh,
+                                                 uint32_t (&o)[16]);
+
+template <>
+__device__ __forceinline__ void dequant_half_row<2>(const uint8_t* pk, int r, int kh,
+                                                    uint32_t (&o)[16]) {
+  const uint2* pc = reinterpret_cast<const uint2*>(pk) + r;
+  const uint2 a = pc[(2 * kh) * 128], b = pc[(2 * kh + 1) * 128];
+  const uint32_t ws[4] = {a.x, a.y, b.x, b.y};            // 16 columns per word
+#pragma unroll
+  for (int w = 0; w < 4; ++w)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) o[4 * w + k] = (ws[w] >> (2 * k)) & 0x03030303u;
+}
+
+template <>
+__device__ __forceinline__ void dequant_half_row<4>(const uint8_t* pk, int r, int kh,
+                                                    uint32_t (&o)[16]) {
+  const uint2* pc = reinterpret_cast<const uint2*>(pk) + r;
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {                            // 8 columns per word
+    const uint2 a = pc[(4 * kh + p) * 128];
+    o[4 * p + 0] = a.x & 0x0F0F0F0Fu;
+    o[4 * p + 1] = (a.x >> 4) & 0x0F0F0F0Fu;
+    o[4 * p + 2] = a.y & 0x0F0F0F0Fu;
+    o[4 * p + 3] = (a.y >> 4) & 0x0F0F0F0Fu;
+  }
+}
+
+template <>
+__device__ __forceinline__ void dequant_half_row<3>(const uint8_t* pk, int r, int kh,
+                                                    uint32_t (&o)[16]) {
+  const uint2* pc = reinterpret_cast<const uint2*>(pk) + r;
+  const uint2 a = pc[(3 * kh) * 128], b = pc[(3 * kh + 1) * 128], e = pc[(3 * kh + 2) * 128];
+  const uint32_t ws[6] = {a.x, a.y, b.x, b.y, e.x, e.y};  // two runs of 32 columns
+#pragma unroll
+  for (int m = 0; m < 2; ++m) {
+    const uint32_t wh = ws[3 * m + 2];                      // top bits of the 32 columns
+#pragma unroll
+    for (int k8 = 0; k8 < 8; ++k8) {                         // columns 4 k8 .. 4 k8 + 3
+      const uint32_t lo = (ws[3 * m + (k8 >> 2)] >> (2 * (k8 & 3))) & 0x03030303u;
+      const uint32_t hi = (k8 >= 2 ? (wh >> (k8 - 2)) : (wh << (2 - k8))) & 0x04040404u;
+      o[8 * m + k8] = lo | hi;
+    }
+  }
+}
+
+// 32 lanes x 16 consecutive 32-bit TMEM columns from registers: thread i -> lane (base + i).
+__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// D(tmem) (+)= A(tmem) * B(smem desc), kind::i8: A is read from tensor memory (K-major, row m
+// in lane m, four 8-bit values per 32-bit column), D is int32.
+__device__ __forceinline__ void umma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Tensor memory of qlin_mma_kernel (512 columns): four A tiles of 128 rows x 128 8-bit codes
+// (32 columns each), then four int32 accumulators of N columns (N <= 96).
+constexpr int QL_NA = 4;
+constexpr int QL_NACC = 4;
+constexpr uint32_t QL_A_COLS = 32;
+constexpr uint32_t QL_ACC_COL0 = QL_NA * QL_A_COLS;
+constexpr uint32_t QL_TMEM_COLS = 512;
+
+// Shared memory of qlin_mma_kernel (offsets from a 1024-byte aligned base). A stage holds ku
+// consecutive units: their B tiles ([R rows][128 B] each, then N rows of slack for the MMA's
+// reads past the last tile's R rows) and their packed blobs, each block filled by one bulk
+// copy (the blobs of consecutive units, and the B tiles of consecutive groups, are contiguous
+// in global memory).
+struct QlSmem {
+  uint32_t stage0;
+  uint32_t stage_bytes;
+  uint32_t b_unit;     // B bytes per unit: 128 R
+  uint32_t a_off;      // offset of the packed blobs inside a stage
+  uint32_t bars;
+  uint32_t xchg;       // 128 rows x 8 tokens of fp32 for the within-tile Hadamard
+  uint32_t total;
+};
+
+__host__ __device__ inline QlSmem ql_smem(int bits, int N, int R, int ku, int stages) {
+  QlSmem s;
+  s.b_unit = 128u * static_cast<uint32_t>(R);
+  s.a_off = static_cast<uint32_t>(ku) * s.b_unit + 128u * static_cast<uint32_t>(N);
+  s.stage_bytes = s.a_off + static_cast<uint32_t>(ku) * 2048u * static_cast<uint32_t>(bits);
+  s.stage0 = 0;
+  s.bars = s.stage0 + static_cast<uint32_t>(stages) * s.stage_bytes;
+  s.xchg = s.bars + 512;
+  s.total = s.xchg + QL_TILE * 8 * 4 + 1024;   // + alignment slack
+  return s;
+}
+
+template <int BITS, int NTC>
+__global__ void __launch_bounds__(QL_THREADS, 1) qlin_mma_kernel(QlMmaArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const QlSmem L = ql_smem(BITS, p.N, p.R, p.ku, p.stages);
+  const int S = p.stages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
+  uint64_t* empty = full + QL_MAX_STAGES;
+  uint64_t* afull = empty + QL_MAX_STAGES;      // QL_NA
+  uint64_t* aempty = afull + QL_NA;             // QL_NA
+  uint64_t* accfull = aempty + QL_NA;           // QL_NACC
+  uint64_t* accempty = accfull + QL_NACC;       // QL_NACC
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(accempty + QL_NACC);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accempty + QL_NACC) + 1;
+  float* xchg = reinterpret_cast<float*>(smem + L.xchg);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t C = gridDim.x;
+  const int64_t u0 = unit_begin(blockIdx.x, p.U, C);
+  const int64_t u1 = unit_begin(blockIdx.x + 1, p.U, C);
+  const int n_units = static_cast<int>(u1 - u0);
+  const int ku = p.ku;
+  const int n_stages = (n_units + ku - 1) / ku;
+  const int g0 = static_cast<int>(u0 % p.G);     // group of the first unit
+  const uint32_t pk_bytes = 2048u * BITS;
+  auto stage_ptr = [&](int s) { return smem + L.stage0 + s * L.stage_bytes; };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < QL_NA; ++i) {
+      mbar_init(&afull[i], QL_DQ_THREADS / 32);
+      mbar_init(&aempty[i], 1);
+    }
+    for (int i = 0; i < QL_NACC; ++i) {
+      mbar_init(&accfull[i], 1);
+      mbar_init(&accempty[i], 4);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, QL_TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ producer
+    if (lane == 0) {
+      const int pre = min(S, n_stages);
+      bool ok = true;
+      // the packed codes do not depend on the preceding kernel: start them before waiting
+      for (int si = 0; si < pre; ++si) {
+        const int i0 = si * ku, nu = min(ku, n_units - i0);
+        mbar_arrive_expect_tx(&full[si], nu * (pk_bytes + L.b_unit));
+        bulk_load(stage_ptr(si) + L.a_off, p.packed + (u0 + i0) * static_cast<int64_t>(pk_bytes),
+                  nu * pk_bytes, &full[si]);
+      }
+      griddep_wait();
+      int si = 0, g = g0;
+      for (; si < n_stages && ok; ++si) {
+        const int s = si % S;
+        const uint32_t ph = (si / S) & 1u;
+        const int i0 = si * ku, nu = min(ku, n_units - i0);
+        uint8_t* st = stage_ptr(s);
+        if (si >= pre) {
+          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.err, DEV_ERR_TMA_WAIT)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], nu * (pk_bytes + L.b_unit));
+          bulk_load(st + L.a_off, p.packed + (u0 + i0) * static_cast<int64_t>(pk_bytes),
+                    nu * pk_bytes, &full[s]);
+        }
+        // B tiles of groups g .. g + nu - 1 (mod G): one copy per contiguous run
+        for (int done = 0; done < nu;) {
+          const int run = min(nu - done, p.G - g);
+          bulk_load(st + done * L.b_unit, p.bop + static_cast<int64_t>(g) * L.b_unit,
+                    run * L.b_unit, &full[s]);
+          done += run;
+          g += run;
+          if (g == p.G) g = 0;
+        }
+      }
+      if (!ok) {
+        // copies already issued complete on their barriers before the CTA leaves
+        for (int j = max(0, si - S); j < si; ++j)
+          mbar_drain(&full[j % S], (j / S) & 1u, 1000000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = ql_idesc(128, p.N);
+      int k = 0, si = 0;
+      // one accumulator per unit (the scale of x' changes from group to group)
+      for (int i = 0; i < n_units; ++i) {
+        const int s = si % S;
+        const uint32_t ph = (si / S) & 1u;
+        const int ab = i % QL_NA;
+        const uint32_t aph = (i / QL_NA) & 1u;
+        const int acc = i % QL_NACC;
+        const uint32_t cph = (i / QL_NACC) & 1u;
+        if (k == 0 && !mbar_wait(&full[s], ph, abort_flag, p.err, DEV_ERR_MMA_WAIT)) break;
+        if (!mbar_wait(&afull[ab], aph, abort_flag, p.err, DEV_ERR_MMA_WAIT)) break;
+        if (!mbar_wait(&accempty[acc], cph ^ 1u, abort_flag, p.err, DEV_ERR_MMA_WAIT)) break;
+        tc_fence_after();
+        const uint32_t a_tmem = tmem_base + ab * QL_A_COLS;
+        const uint32_t bbase = smem_u32(stage_ptr(s) + k * L.b_unit);
+        const uint32_t d_tmem = tmem_base + QL_ACC_COL0 + acc * p.N;
+        // K = 128 in four steps of 32 8-bit values (32 bytes of each A and B row)
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t bd = smem_desc_sw128(bbase + kk * 32, 16, 1024);
+          umma_i8_ts(d_tmem, a_tmem + kk * 8, bd, idesc, kk ? 1u : 0u);
+        }
+        umma_commit(&aempty[ab]);
+        umma_commit(&accfull[acc]);
+        if (k == ku - 1 || i == n_units - 1) {
+          umma_commit(&empty[s]);          // the stage's codes and B tiles are consumed
+          k = 0;
+          ++si;
+        } else {
+          ++k;
+        }
+      }
+    }
+  } else if (warp >= QL_DQ_WARP0) {
+    // ------------------------------------------------------------------ dequantization
+    // warp w writes TMEM lanes 32 (w % 4) .. + 31 (its rows) for column half (w - 8) / 4
+    const int q = warp & 3, kh = (warp - QL_DQ_WARP0) >> 2;
+    const int r = q * 32 + lane;
+    int k = 0, si = 0;
+    for (int i = 0; i < n_units; ++i) {
+      const int s = si % S;
+      const uint32_t ph = (si / S) & 1u;
+      const int ab = i % QL_NA;
+      const uint32_t aph = (i / QL_NA) & 1u;
+      int ok = 1;
+      if (lane == 0) {
+        ok = (k != 0 || mbar_wait(&full[s], ph, abort_flag, p.err, DEV_ERR_MMA_WAIT)) &&
+             mbar_wait(&aempty[ab], aph ^ 1u, abort_flag, p.err, DEV_ERR_MMA_WAIT);
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t o[16];
+      dequant_half_row<BITS>(stage_ptr(s) + L.a_off + k * pk_bytes, r, kh, o);
+      tmem_st_32x32b_x16(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ab * QL_A_COLS +
+                             kh * 16,
+                         o);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&afull[ab]);
+      if (++k == ku) {
+        k = 0;
+        ++si;
+      }
+    }
+  } else if (warp >= QL_EPI_WARP0) {
+    // ------------------------------------------------------------------ epilogue
+    griddep_wait();                                   // the group sums come from qlin_in
+    const int q = warp & 3;
+    const int r = q * 32 + lane;                      // row inside the tile = TMEM lane
+    float yacc[NTC];
+#pragma unroll
+    for (int k = 0; k < NTC; ++k) yacc[k] = 0.f;
+    int g = g0;
+    int tile = static_cast<int>(u0 / p.G);
+    for (int i = 0; i < n_units; ++i) {
+      const int gcur = g;
+      const int tcur = tile;
+      if (++g == p.G) {
+        g = 0;
+        ++tile;
+      }
+      // lane k holds token k's (s, sum of its terms) for this group; and this row's grid; both
+      // loaded before waiting so that their latency overlaps the MMAs
+      float sl = 0.f, ql = 0.f;
+      if (lane < p.n_tok) {
+        const float2 s2 = __ldg(&p.sums[static_cast<int64_t>(gcur) * p.n_tok + lane]);
+        sl = s2.x;
+        ql = s2.y;
+      }
+      const float2 gz = __ldg(&p.grid[p.grouped
+                                          ? (static_cast<int64_t>(tcur) * p.G + gcur) * QL_TILE + r
+                                          : static_cast<int64_t>(tcur) * QL_TILE + r]);
+      const int acc = i % QL_NACC;
+      const uint32_t cph = (i / QL_NACC) & 1u;
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(&accfull[acc], cph, abort_flag, p.err, DEV_ERR_EPI_WAIT);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      // the four epilogue warps leave together (they meet at named barriers below)
+      if (!bar_and(2, 128, ok != 0)) break;
+      tc_fence_after();
+      const float sc = gz.x, z = gz.y;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + QL_ACC_COL0 +
+                             acc * p.N;
+      // tokens in runs of 16 (48 int32 columns = three loads of 16)
+#pragma unroll
+      for (int t0 = 0; t0 < NTC; t0 += 16) {
+        float f[48];
+#pragma unroll
+        for (int cb = 0; cb < 3; ++cb) {
+          if (3 * t0 + 16 * cb < p.N) {
+            uint32_t w[16];
+            tmem_ld_32x32b_x16(taddr + 3 * t0 + 16 * cb, w);
+            tmem_ld_wait();
+            // |value| < 2^22: exact through the 1.5 * 2^23 bias
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              f[16 * cb + j] = __int_as_float(static_cast<int>(w[j]) + 0x4B400000) - 12582912.f;
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) f[16 * cb + j] = 0.f;
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const int tt = t0 + k;
+          if (tt < NTC) {
+            const float st = __shfl_sync(0xffffffffu, sl, tt);
+            const float qt = __shfl_sync(0xffffffffu, ql, tt);
+            if (tt < p.n_tok) {
+              // sum_j c_j x'_j / s = t0 + t1 / 128 + t2 / 128^2 (exact int32 products)
+              const float a = f[3 * k] + f[3 * k + 1] * (1.f / 128.f) +
+                              f[3 * k + 2] * (1.f / 16384.f);
+              yacc[tt] = fmaf(sc * st, fmaf(-z, qt, a), yacc[tt]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&accempty[acc]);
+      // end of this CTA's part of the tile: within-tile Hadamard, then one partial
+      if (i == n_units - 1 || gcur == p.G - 1) {
+        if (p.rotate_out) {
+#pragma unroll
+          for (int h = 1; h < 32; h <<= 1) {
+            if (h >= p.b_tile) break;
+#pragma unroll
+            for (int k = 0; k < NTC; ++k) {
+              const float o = __shfl_xor_sync(0xffffffffu, yacc[k], h);
+              yacc[k] = (lane & h) ? (o - yacc[k]) : (yacc[k] + o);
+            }
+          }
+          for (int h = 32; h < p.b_tile; h <<= 1) {
+#pragma unroll
+            for (int k0 = 0; k0 < NTC; k0 += 8) {
+              named_bar_sync(1, 128);
+#pragma unroll
+              for (int k = 0; k < 8; ++k)
+                if (k0 + k < NTC) xchg[k * QL_TILE + r] = yacc[k0 + k];
+              named_bar_sync(1, 128);
+#pragma unroll
+              for (int k = 0; k < 8; ++k)
+                if (k0 + k < NTC) {
+                  const float o = xchg[k * QL_TILE + (r ^ h)];
+                  yacc[k0 + k] = (r & h) ? (o - yacc[k0 + k]) : (yacc[k0 + k] + o);
+                }
+            }
+          }
+        }
+        const int64_t seg = blockIdx.x + tcur;
+        float* out = p.partial + seg * p.n_tok * QL_TILE + r;
+#pragma unroll
+        for (int k = 0; k < NTC; ++k) {
+          if (k < p.n_tok) out[k * QL_TILE] = yacc[k];
+          yacc[k] = 0.f;
+        }
+      }
+    }
+  }
+
+  griddep_launch_dependents();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, QL_TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Output side: sum of partials, across-tile Hadamard, signs, S_G^-1
+// ---------------------------------------------------------------------------------------------
+struct QlOutArgs {
+  const float* partial;
+  int n_tok, T, G;
+  int64_t U, C;
+  int qb;              // tiles per output Hadamard block (1 when b_out <= 128 or no rotation)
+  int d_out;
+  const float* s_g;
+  const int8_t* sign_out;
+  uint32_t flags;
+  float inv_sqrt_b;
+  float* y;
+  int64_t ld_y;
+};
+
+// CTA that owns unit u under the split c -> [floor(c U / C), floor((c + 1) U / C)): the
+// smallest c with floor((c + 1) U / C) > u, i.e. (c + 1) U >= (u + 1) C.
+__device__ __forceinline__ int64_t cta_of_unit(int64_t u, int64_t U, int64_t C) {
+  return ((u + 1) * C - 1) / U;
+}
+
+// One CTA per (token, output Hadamard block, 16-row slice of the tiles): thread e handles row
+// (e mod 16) of the slice in tile e / 16 of the block.
+__global__ void __launch_bounds__(1024) qlin_out_kernel(QlOutArgs a) {
+  extern __shared__ float ys[];                   // qb x 16, then qb x 2 CTA bounds
+  int* cbound = reinterpret_cast<int*>(ys + a.qb * 16);
+  const int slice = blockIdx.x & 7;
+  const int sb = blockIdx.x >> 3;
+  const int tok = blockIdx.y;
+  griddep_launch_dependents();
+  for (int qi = threadIdx.x; qi < a.qb; qi += blockDim.x) {
+    const int64_t tile = static_cast<int64_t>(sb) * a.qb + qi;
+    cbound[2 * qi] = static_cast<int>(cta_of_unit(tile * a.G, a.U, a.C));
+    cbound[2 * qi + 1] = static_cast<int>(cta_of_unit(tile * a.G + a.G - 1, a.U, a.C));
+  }
+  griddep_wait();
+  __syncthreads();
+  const int n = a.qb * 16;
+  for (int e = threadIdx.x; e < n; e += blockDim.x) {
+    const int qi = e >> 4, r = slice * 16 + (e & 15);
+    const int64_t tile = static_cast<int64_t>(sb) * a.qb + qi;
+    const int c0 = cbound[2 * qi], c1 = cbound[2 * qi + 1];
+    const float* src = a.partial + ((c0 + tile) * a.n_tok + tok) * QL_TILE + r;
+    const int64_t step = static_cast<int64_t>(a.n_tok) * QL_TILE;   // next segment
+    float v0 = 0.f, v1 = 0.f;
+    int c = c0;
+    for (; c + 1 <= c1; c += 2) {               // two independent loads in flight
+      v0 += src[(c - c0) * step];
+      v1 += src[(c + 1 - c0) * step];
+    }
+    if (c <= c1) v0 += src[(c - c0) * step];
+    ys[e] = v0 + v1;
+  }
+  __syncthreads();
+  const bool rot = (a.flags & KRONQ_BIIP_ROTATE_OUT) != 0;
+  if (rot && a.qb > 1) {
+    for (int sh = 0; (1 << sh) < a.qb; ++sh) {
+      const int h = 1 << sh;
+      for (int pidx = threadIdx.x; pidx < n / 2; pidx += blockDim.x) {
+        // pairs of tiles (qi, qi + h) with bit sh of qi clear, same row
+        const int r = pidx & 15, pq = pidx >> 4;
+        const int qi = ((pq >> sh) << (sh + 1)) | (pq & (h - 1));
+        const float u = ys[qi * 16 + r], w = ys[(qi + h) * 16 + r];
+        ys[qi * 16 + r] = u + w;
+        ys[(qi + h) * 16 + r] = u - w;
+      }
+      __syncthreads();
+    }
+  }
+  for (int e = threadIdx.x; e < n; e += blockDim.x) {
+    const int qi = e >> 4, r = slice * 16 + (e & 15);
+    const int64_t i = static_cast<int64_t>(sb * a.qb + qi) * QL_TILE + r;
+    if (i >= a.d_out) continue;
+    float v = ys[e];
+    if (rot) {
+      v *= a.inv_sqrt_b;
+      if (a.sign_out[i] < 0) v = -v;
+    }
+    if (a.flags & KRONQ_BIIP_SCALE_OUT) v = v / a.s_g[i];
+    a.y[tok * a.ld_y + i] = v;
+  }
+}
+
+// (scale, zero) pairs in the order the epilogue reads them: per tile, per group (group-wise
+// grid) or once (per-row grid), 128 rows; rows past d_out get (0, 0).
+__global__ void pack_grid_kernel(const float* __restrict__ scale, const float* __restrict__ zero,
+                                 int d_out, int groups, int rows_pad, float2* __restrict__ out) {
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t total = static_cast<int64_t>(rows_pad) * groups;
+  if (idx >= total) return;
+  const int r = static_cast<int>(idx % QL_TILE);
+  const int64_t tg = idx / QL_TILE;               // tile * groups + g
+  const int g = static_cast<int>(tg % groups);
+  const int t = static_cast<int>(tg / groups);
+  const int row = t * QL_TILE + r;
+  float2 v = make_float2(0.f, 0.f);
+  if (row < d_out) {
+    const int64_t src = static_cast<int64_t>(row) * groups + g;
+    v = make_float2(scale[src], zero[src]);
+  }
+  out[idx] = v;
+}
+
+template <typename Kern, typename... Args>
+kronq_status launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                        bool pdl, const char* what, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  if (e != cudaSuccess) return fail(KRONQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return check_launch(what);
+}
+
+int pow2_factor(int d) { return d & (-d); }
+
+struct QlGeom {
+  int T, G, C;
+  int64_t U;
+  int span;
+  size_t bop_bytes, sums_bytes, partial_bytes;
+};
+
+QlGeom ql_geom(int d_out, int d_in, int n_tok_pass) {
+  QlGeom g;
+  g.T = (d_out + QL_TILE - 1) / QL_TILE;
+  g.G = (d_in + QL_TILE - 1) / QL_TILE;
+  g.U = static_cast<int64_t>(g.T) * g.G;
+  g.C = static_cast<int>(std::min<int64_t>(g.U, sm_budget()));
+  g.span = std::max(pow2_factor(d_in), QL_TILE);
+  g.bop_bytes = align256(static_cast<size_t>(g.G) * 128 * ((3 * n_tok_pass + 7) / 8 * 8));
+  g.sums_bytes = align256(static_cast<size_t>(g.G) * n_tok_pass * sizeof(float2));
+  g.partial_bytes =
+      align256(static_cast<size_t>(g.C + g.T) * n_tok_pass * QL_TILE * sizeof(float));
+  return g;
+}
+
+template <int BITS, int NTC>
+kronq_status launch_mma_t(const QlMmaArgs& p, int C, size_t smem, cudaStream_t stream) {
+  auto kern = qlin_mma_kernel<BITS, NTC>;
+  const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem));
+  if (e != cudaSuccess) return fail(KRONQ_ERR_CUDA, "qlin_mma smem: %s", cudaGetErrorString(e));
+  return launch_pdl(kern, dim3(C), dim3(QL_THREADS), smem, stream, true, "qlin_mma_kernel", p);
+}
+
+kronq_status launch_mma(int bits, int ntc, const QlMmaArgs& p, int C, size_t smem,
+                        cudaStream_t stream) {
+  if (bits == 2) return ntc <= 8 ? launch_mma_t<2, 8>(p, C, smem, stream)
+                                 : launch_mma_t<2, 32>(p, C, smem, stream);
+  if (bits == 3) return ntc <= 8 ? launch_mma_t<3, 8>(p, C, smem, stream)
+                                 : launch_mma_t<3, 32>(p, C, smem, stream);
+  return ntc <= 8 ? launch_mma_t<4, 8>(p, C, smem, stream)
+                  : launch_mma_t<4, 32>(p, C, smem, stream);
+}
+
+}  // namespace
+
+size_t packed_code_bytes(int d_out, int d_in, int bits) {
+  const size_t t = (d_out + QL_TILE - 1) / QL_TILE, g = (d_in + QL_TILE - 1) / QL_TILE;
+  return t * g * 2048 * static_cast<size_t>(bits);
+}
+
+kronq_status run_pack_codes(const uint8_t* codes, int d_out, int d_in, int bits, void* packed,
+                            cudaStream_t stream) {
+  const int groups = (d_in + QL_TILE - 1) / QL_TILE;
+  const int rows_pad = (d_out + QL_TILE - 1) / QL_TILE * QL_TILE;
+  const int cpg = bits == 2 ? 8 : (bits == 4 ? 16 : 4);   // words-chunks per group row
+  const int64_t total = static_cast<int64_t>(rows_pad) * groups * cpg;
+  const int threads = 256;
+  pack_codes_kernel<<<static_cast<unsigned>((total + threads - 1) / threads), threads, 0,
+                      stream>>>(codes, d_out, d_in, bits, groups, rows_pad,
+                                static_cast<uint32_t*>(packed));
+  return check_launch("pack_codes_kernel");
+}
+
+size_t packed_grid_bytes(int d_out, int d_in, int group) {
+  const size_t t = (d_out + QL_TILE - 1) / QL_TILE;
+  const size_t g = group ? (d_in + QL_TILE - 1) / QL_TILE : 1;
+  return t * g * QL_TILE * sizeof(float2);
+}
+
+kronq_status run_pack_grid(const float* scale, const float* zero, int d_out, int d_in, int group,
+                           void* packed, cudaStream_t stream) {
+  const int groups = group ? (d_in + QL_TILE - 1) / QL_TILE : 1;
+  const int rows_pad = (d_out + QL_TILE - 1) / QL_TILE * QL_TILE;
+  const int64_t total = static_cast<int64_t>(rows_pad) * groups;
+  const int threads = 256;
+  pack_grid_kernel<<<static_cast<unsigned>((total + threads - 1) / threads), threads, 0,
+                     stream>>>(scale, zero, d_out, groups, rows_pad,
+                               static_cast<float2*>(packed));
+  return check_launch("pack_grid_kernel");
+}
+
+size_t qlinear_workspace_bytes(int d_out, int d_in, int n_tok) {
+  const int ntp = std::min(std::max(n_tok, 1), QL_NT_MAX);
+  const QlGeom g = ql_geom(d_out, d_in, ntp);
+  return g.bop_bytes + g.sums_bytes + g.partial_bytes;
+}
+
+kronq_status run_qlinear(const QlinearArgs& q, void* ws, cudaStream_t stream) {
+  const int ntp_max = std::min(q.n_tok, QL_NT_MAX);
+  const QlGeom g = ql_geom(q.d_out, q.d_in, ntp_max);
+  Carve cv{static_cast<uint8_t*>(ws)};
+  uint8_t* bop = cv.p;
+  cv.p += g.bop_bytes;
+  float2* sums = reinterpret_cast<float2*>(cv.p);
+  cv.p += g.sums_bytes;
+  float* partial = reinterpret_cast<float*>(cv.p);
+
+  const int b_in = pow2_factor(q.d_in), b_out = pow2_factor(q.d_out);
+  const bool rot_in = (q.flags & KRONQ_BIIP_ROTATE_IN) != 0;
+  const bool rot_out = (q.flags & KRONQ_BIIP_ROTATE_OUT) != 0;
+  if (rot_in && b_in > 16384)
+    return fail(KRONQ_ERR_UNSUPPORTED, "input Hadamard block %d > 16384", b_in);
+  if (rot_out && b_out > 16384)
+    return fail(KRONQ_ERR_UNSUPPORTED, "output Hadamard block %d > 16384", b_out);
+  const int span = rot_in ? g.span : QL_TILE;
+  const size_t in_smem = static_cast<size_t>(span) * sizeof(float);
+  KQ_CUDA_TRY(cudaFuncSetAttribute(qlin_in_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   static_cast<int>(in_smem)));
+  const int qb = (rot_out && b_out > QL_TILE) ? b_out / QL_TILE : 1;
+  const size_t out_smem = static_cast<size_t>(qb) * (16 * sizeof(float) + 2 * sizeof(int));
+
+  int dev = 0, max_smem = 0;
+  KQ_CUDA_TRY(cudaGetDevice(&dev));
+  KQ_CUDA_TRY(cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
+
+  for (int t0 = 0; t0 < q.n_tok; t0 += QL_NT_MAX) {
+    const int nt = std::min(QL_NT_MAX, q.n_tok - t0);
+    QlInArgs ia;
+    ia.x = static_cast<const uint8_t*>(q.x) +
+           static_cast<int64_t>(t0) * q.ld_x * (q.x_dtype == KRONQ_DTYPE_BF16 ? 2 : 4);
+    ia.x_dtype = q.x_dtype;
+    ia.ld_x = q.ld_x;
+    ia.n_tok = nt;
+    ia.d_in = q.d_in;
+    ia.span = span;
+    ia.b_in = rot_in ? b_in : 1;
+    ia.s_x = q.s_x;
+    ia.sign_in = q.sign_in;
+    ia.flags = q.flags;
+    ia.inv_sqrt_b = static_cast<float>(1.0 / std::sqrt(static_cast<double>(b_in)));
+    ia.rows = (3 * nt + 7) / 8 * 8;
+    ia.bop = bop;
+    ia.sums = sums;
+    const dim3 igrid((q.d_in + span - 1) / span, nt);
+    // Chained to the previous kernel too: only the launch overlaps it, since qlin_in waits for
+    // it to complete before reading x (which the previous kernel may have written); so this
+    // call's workspace writes never race with a previous call's reads.
+    KQ_TRY(launch_pdl(qlin_in_kernel, igrid, dim3(std::max(32, span / 16)), in_smem, stream, true,
+                      "qlin_in_kernel", ia));
+
+    QlMmaArgs p;
+    p.packed = static_cast<const uint8_t*>(q.packed);
+    p.bop = bop;
+    p.sums = sums;
+    p.grid = static_cast<const float2*>(q.grid);
+    p.partial = partial;
+    p.d_out = q.d_out;
+    p.T = g.T;
+    p.G = g.G;
+    p.n_tok = nt;
+    p.N = std::max(16, (3 * nt + 15) / 16 * 16);
+    p.grouped = q.group ? 1 : 0;
+    p.rotate_out = rot_out ? 1 : 0;
+    p.b_tile = rot_out ? std::min(b_out, QL_TILE) : 1;
+    p.U = g.U;
+    p.err = device_error_word();
+    p.R = (3 * nt + 7) / 8 * 8;
+    // about 48 KB of stage per bulk-copy pair: few, large copies keep the copy engine busy
+    const int per_unit = 2048 * q.bits + 128 * p.R;
+    p.ku = std::max(1, std::min(8, 49152 / per_unit));
+    QlSmem L0 = ql_smem(q.bits, p.N, p.R, p.ku, 1);
+    const int avail = max_smem - static_cast<int>(L0.total - L0.stage_bytes);
+    p.stages = std::min(QL_MAX_STAGES, avail / static_cast<int>(L0.stage_bytes));
+    if (p.stages < 2) return fail(KRONQ_ERR_UNSUPPORTED, "qlinear: shared memory too small");
+    // at least 117 KB, so that one CTA (and its 512 TMEM columns) fills an SM
+    const size_t smem = std::max<size_t>(ql_smem(q.bits, p.N, p.R, p.ku, p.stages).total,
+                                         117 * 1024);
+    KQ_TRY(launch_mma(q.bits, nt, p, g.C, smem, stream));
+
+    QlOutArgs oa;
+    oa.partial = partial;
+    oa.n_tok = nt;
+    oa.T = g.T;
+    oa.G = g.G;
+    oa.U = g.U;
+    oa.C = g.C;
+    oa.qb = qb;
+    oa.d_out = q.d_out;
+    oa.s_g = q.s_g;
+    oa.sign_out = q.sign_out;
+    oa.flags = q.flags;
+    oa.inv_sqrt_b = static_cast<float>(1.0 / std::sqrt(static_cast<double>(b_out)));
+    oa.y = q.y + static_cast<int64_t>(t0) * q.ld_y;
+    oa.ld_y = q.ld_y;
+    const dim3 ogrid(8 * (g.T / qb), nt);
+    KQ_TRY(launch_pdl(qlin_out_kernel, ogrid, dim3(std::min(1024, std::max(32, qb * 16))),
+                      out_smem, stream, true, "qlin_out_kernel", oa));
+  }
+  return KRONQ_OK;
+}
+
+}  // namespace kq

@@ -46,6 +46,8 @@ SYMBOLS = (
     "kronq_cholinv_workspace_size", "kronq_cholinv",
     "kronq_quantize_layer_workspace_size", "kronq_quantize_layer",
     "kronq_score_allocate",
+    "kronq_packed_codes_bytes", "kronq_pack_codes", "kronq_packed_grid_bytes", "kronq_pack_grid",
+    "kronq_qlinear_workspace_size", "kronq_qlinear",
 )
 
 
@@ -105,6 +107,15 @@ def load_library(path: str = LIB_PATH):
                                          c_sz, c_void_p]),
         "kronq_score_allocate": (c_i32, [c_void_p, c_void_p, c_void_p, c_i32, c_void_p, c_i32,
                                          c_dbl, c_void_p, c_void_p]),
+        "kronq_packed_codes_bytes": (c_sz, [c_i32, c_i32, c_i32]),
+        "kronq_pack_codes": (c_i32, [c_void_p, c_i32, c_i32, c_i32, c_void_p, c_sz, c_void_p]),
+        "kronq_packed_grid_bytes": (c_sz, [c_i32, c_i32, c_i32]),
+        "kronq_pack_grid": (c_i32, [c_void_p, c_void_p, c_i32, c_i32, c_i32, c_void_p, c_sz,
+                                    c_void_p]),
+        "kronq_qlinear_workspace_size": (c_sz, [c_i32, c_i32, c_i32]),
+        "kronq_qlinear": (c_i32, [c_void_p, c_i32, c_i64, c_i32, c_void_p, c_void_p,
+                                  c_i32, c_void_p, c_void_p, c_void_p, c_void_p, c_u32, c_i32,
+                                  c_i32, c_i32, c_void_p, c_i64, c_void_p, c_sz, c_void_p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -281,3 +292,64 @@ def kronq_score_allocate(tr_hx, tr_hg, n_params, choices, avg_bits):
     st = lib.kronq_score_allocate(a, b, n, L, ch, len(choices), float(avg_bits), s, bits)
     _check(st, "kronq_score_allocate")
     return list(s), list(bits)
+
+
+# ------------------------------------------------------------------------------ 6. inference
+
+def kronq_packed_codes_bytes(d_out: int, d_in: int, bits: int) -> int:
+    return load_library().kronq_packed_codes_bytes(d_out, d_in, bits)
+
+
+def kronq_pack_codes(codes, bits, packed=None, stream=None):
+    """codes: d_out x d_in uint8 (contiguous). Returns the packed uint8 tensor."""
+    lib = load_library()
+    d_out, d_in = codes.shape
+    if not codes.is_contiguous():
+        raise ValueError("codes must be contiguous")
+    nbytes = lib.kronq_packed_codes_bytes(d_out, d_in, int(bits))
+    if packed is None:
+        packed = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=codes.device)
+    st = lib.kronq_pack_codes(_p(codes), d_out, d_in, int(bits), _p(packed),
+                              packed.numel() * packed.element_size(), _stream(stream))
+    _check(st, "kronq_pack_codes")
+    return packed
+
+
+def kronq_packed_grid_bytes(d_out: int, d_in: int, group: int) -> int:
+    return load_library().kronq_packed_grid_bytes(d_out, d_in, group)
+
+
+def kronq_pack_grid(scale, zero, d_out, d_in, group, packed=None, stream=None):
+    """scale, zero from kronq_quantize_layer. Returns the packed (scale, zero) pairs (fp32)."""
+    lib = load_library()
+    nbytes = lib.kronq_packed_grid_bytes(d_out, d_in, int(group))
+    if packed is None:
+        packed = torch.empty(max(nbytes // 4, 2), dtype=torch.float32, device=scale.device)
+    st = lib.kronq_pack_grid(_p(scale), _p(zero), d_out, d_in, int(group), _p(packed),
+                             packed.numel() * packed.element_size(), _stream(stream))
+    _check(st, "kronq_pack_grid")
+    return packed
+
+
+def kronq_qlinear_workspace_size(d_out: int, d_in: int, n_tok: int) -> int:
+    return load_library().kronq_qlinear_workspace_size(d_out, d_in, n_tok)
+
+
+def kronq_qlinear(x, packed, packed_grid, s_x, s_g, sign_in, sign_out, flags, d_out, bits, y,
+                  group=0, workspace=None, stream=None):
+    """y (n_tok x d_out fp32) = S_G^-1 U^T W^' V S_X^-1 x for x (n_tok x d_in, bf16 or fp32)."""
+    lib = load_library()
+    n_tok, d_in = x.shape
+    if x.dtype == torch.bfloat16:
+        xd = DTYPE_BF16
+    elif x.dtype == torch.float32:
+        xd = DTYPE_F32
+    else:
+        raise ValueError("x must be bf16 or fp32")
+    ws, wsb = _workspace(lib.kronq_qlinear_workspace_size(d_out, d_in, n_tok), x.device,
+                         workspace)
+    st = lib.kronq_qlinear(_p(x), xd, _rowstride(x), n_tok, _p(packed), _p(packed_grid),
+                           int(group), _p(s_x), _p(s_g), _p(sign_in), _p(sign_out), int(flags),
+                           int(d_out), d_in, int(bits), _p(y), _rowstride(y), _p(ws), wsb,
+                           _stream(stream))
+    _check(st, "kronq_qlinear")

@@ -7,6 +7,8 @@
     python -m post_quantization_b200.profcase biip --d-out 4096 --d-in 4096
     python -m post_quantization_b200.profcase cholinv --d 4096
     python -m post_quantization_b200.profcase quantize --d-out 4096 --d-in 4096
+    python -m post_quantization_b200.profcase qlinear --block --bits 2 --group 128 --tokens 1
+        the quantized layers at inference, per layer (graph replays) and as one block sweep
 Each case runs its call `--reps` times (default 3) after one warm-up call.
 """
 from __future__ import annotations
@@ -155,20 +157,130 @@ def case_quantize(args):
                       "ms": a.elapsed_time(b) / args.reps}))
 
 
+LLAMA3_70B_LINEARS = [("q", 8192, 8192), ("k", 1024, 8192), ("v", 1024, 8192),
+                      ("o", 8192, 8192), ("gate", 28672, 8192), ("up", 28672, 8192),
+                      ("down", 8192, 28672)]
+
+
+def qlinear_bytes(d_out, d_in, bits, group, n_tok, x_bytes=4):
+    """Algorithmic bytes of one kronq_qlinear call: packed codes, grid, x, y, scales, signs."""
+    ng = (d_in + 127) // 128 if group else 1
+    return (K.kronq_packed_codes_bytes(d_out, d_in, bits) + 8 * d_out * ng
+            + n_tok * d_in * x_bytes + n_tok * d_out * 4 + 5 * (d_in + d_out))
+
+
+def case_qlinear(args):
+    """Decode through the linears of one LLaMA-3-70B-shaped block (or one --d-out x --d-in
+    layer) at --bits, --group, --tokens tokens; each layer's call is captured in its own CUDA
+    graph and timed by replays (the block's packed codes, 214 MB at 2 bits, exceed L2)."""
+    dev = torch.device("cuda")
+    n = args.tokens or 1
+    bits, group = args.bits, args.group
+    shapes = LLAMA3_70B_LINEARS if args.block else [("layer", args.d_out, args.d_in)]
+    layers = []
+    for nm, do, di in shapes:
+        tag = ("qlinear-case", nm, do, di, bits)
+        c = synth.codes(do, di, bits, synth.seed_for(tag, "c"), device=dev)
+        packed = K.kronq_pack_codes(c, bits)
+        del c
+        ng = (di + 127) // 128 if group else 0
+        scale, zero = synth.grid_params(do, ng, bits, synth.seed_for(tag, "g"), device=dev)
+        grid = K.kronq_pack_grid(scale, zero, do, di, group)
+        lay = dict(name=nm, d_out=do, d_in=di, packed=packed, grid=grid,
+                   s_x=synth.positive_scales(di, synth.seed_for(tag, "sx"), device=dev),
+                   s_g=synth.positive_scales(do, synth.seed_for(tag, "sg"), device=dev),
+                   si=synth.rademacher(di, synth.seed_for(tag, "si"), device=dev),
+                   so=synth.rademacher(do, synth.seed_for(tag, "so"), device=dev),
+                   x=synth.activations(n, di, synth.seed_for(tag, "x"), device=dev),
+                   y=torch.empty(n, do, device=dev))
+        nb = K.kronq_qlinear_workspace_size(do, di, n)
+        lay["ws"] = P.Workspace(dev).get(nb)
+        layers.append(lay)
+
+    def call(L):
+        K.kronq_qlinear(L["x"], L["packed"], L["grid"], L["s_x"], L["s_g"], L["si"], L["so"],
+                        K.BIIP_FULL, L["d_out"], bits, L["y"], group=group, workspace=L["ws"])
+
+    for L in layers:
+        call(L)
+    torch.cuda.synchronize()
+
+    class Eager:
+        """Stands in for a graph (eager calls), for runs under a profiler."""
+        def __init__(self, L):
+            self.L = L
+
+        def replay(self):
+            call(self.L)
+
+    graphs = []
+    for L in layers:
+        if args.no_graphs:
+            graphs.append(Eager(L))
+            continue
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            call(L)
+        graphs.append(g)
+    for _ in range(3):
+        for g in graphs:
+            g.replay()
+    torch.cuda.synchronize()
+    res = []
+    tot_ms, tot_bytes = 0.0, 0
+    for L, g in zip(layers, graphs):
+        a, b = ev(), ev()
+        # interleave the other layers between timed replays so that this layer's codes are
+        # not in L2 when its replay starts
+        ms = 0.0
+        for _ in range(args.reps):
+            for g2 in graphs:
+                if g2 is not g:
+                    g2.replay()
+            a.record()
+            g.replay()
+            b.record()
+            b.synchronize()
+            ms += a.elapsed_time(b)
+        ms /= args.reps
+        nbytes = qlinear_bytes(L["d_out"], L["d_in"], bits, group, n)
+        tot_ms += ms
+        tot_bytes += nbytes
+        res.append({"layer": L["name"], "d_out": L["d_out"], "d_in": L["d_in"], "us": ms * 1e3,
+                    "GBps": nbytes / ms / 1e6})
+    # the whole block as one sweep of graph replays
+    a, b = ev(), ev()
+    a.record()
+    for _ in range(args.reps):
+        for g in graphs:
+            g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    sweep_ms = a.elapsed_time(b) / args.reps
+    print(json.dumps({"case": "qlinear", "bits": bits, "group": group, "tokens": n,
+                      "layers": res, "sum_us": tot_ms * 1e3, "sweep_us": sweep_ms * 1e3,
+                      "sweep_GBps": tot_bytes / sweep_ms / 1e6,
+                      "launches": K.kronq_launch_count()}))
+    del graphs
+
+
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["stages", "acc", "biip", "cholinv", "quantize"])
+    ap.add_argument("case", choices=["stages", "acc", "biip", "cholinv", "quantize", "qlinear"])
     ap.add_argument("--tokens", type=int, default=None)
     ap.add_argument("--d", type=int, default=4096)
     ap.add_argument("--d-out", type=int, default=4096)
     ap.add_argument("--d-in", type=int, default=4096)
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--group", type=int, default=0, help="quantize: 0 (per row) or 128")
+    ap.add_argument("--bits", type=int, default=2, help="qlinear: code width")
+    ap.add_argument("--block", action="store_true", help="qlinear: the LLaMA-3-70B block")
+    ap.add_argument("--no-graphs", action="store_true", help="qlinear: eager calls")
     args = ap.parse_args()
     K.load_library()
     K.kronq_device_check()
     {"stages": stages, "acc": case_acc, "biip": case_biip, "cholinv": case_cholinv,
-     "quantize": case_quantize}[args.case](args)
+     "quantize": case_quantize, "qlinear": case_qlinear}[args.case](args)
 
 
 if __name__ == "__main__":

@@ -196,3 +196,43 @@ WORKLOADS = {
                                 extra={"choices": (2, 3, 4), "avg_bits": 2.5,
                                        "g_block_multiplier_log10": (-2.0, 1.0)}),
 }
+
+
+# ------------------------------------------------------------------ a quantized layer's storage
+# Stand-ins for what the solve returns (codes, grid) and for the incoherence scales, so that
+# the inference path can be exercised at any size without running the solve first.
+
+def codes(d_out: int, d_in: int, bits: int, seed: int, device="cpu") -> torch.Tensor:
+    """Uniform random b-bit codes (uint8)."""
+    g = _gen(seed, device)
+    return torch.randint(0, 1 << bits, (d_out, d_in), generator=g, device=device,
+                         dtype=torch.int32).to(torch.uint8)
+
+
+def grid_params(d_out: int, n_groups: int, bits: int, seed: int, device="cpu"):
+    """(scale, zero) fp32 of shape d_out (n_groups 0) or d_out x n_groups: scale log-uniform on
+    [1e-3, 1e-1], zero an integer in [-1, 2^bits]."""
+    g = _gen(seed, device)
+    shape = (d_out,) if n_groups == 0 else (d_out, n_groups)
+    scale = torch.exp(torch.empty(shape, device=device).uniform_(math.log(1e-3), math.log(1e-1),
+                                                                generator=g))
+    zero = torch.randint(-1, (1 << bits) + 1, shape, generator=g, device=device).float()
+    return scale.float(), zero
+
+
+def positive_scales(d: int, seed: int, device="cpu", lo: float = 0.25, hi: float = 4.0):
+    """d fp32 values log-uniform on [lo, hi] (stand-ins for the diagonal BiIP scales)."""
+    g = _gen(seed, device)
+    return torch.exp(torch.empty(d, device=device).uniform_(math.log(lo), math.log(hi),
+                                                            generator=g)).float()
+
+
+def activations(n: int, d: int, seed: int, dtype=torch.float32, device="cpu",
+                n_outliers: int = 4, outlier_scale: float = 20.0) -> torch.Tensor:
+    """n x d independent N(0, 1) activations with a few x20 outlier channels (decode-time
+    inputs of a layer; no mixing matrix, so any d is cheap)."""
+    g = _gen(seed, device)
+    x = torch.randn(n, d, generator=g, device=device, dtype=torch.float32)
+    cols = outlier_channels(d, seed_for(seed, "outliers"), n_outliers)
+    x[:, cols] *= outlier_scale
+    return x.to(dtype)

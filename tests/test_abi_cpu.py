@@ -107,6 +107,54 @@ def test_argument_errors_before_device(K):
     assert "no output" in lib.kronq_last_error_detail().decode()
 
 
+def test_inference_calls_host_checks(K):
+    lib = K.load_library()
+    # packed sizes follow the format: 128 x 128 blobs of 2048 * bits bytes
+    for bits in (2, 3, 4):
+        assert K.kronq_packed_codes_bytes(300, 520, bits) == O.packed_bytes(300, 520, bits)
+    assert K.kronq_packed_codes_bytes(128, 128, 5) == 0
+    assert K.kronq_qlinear_workspace_size(4096, 4096, 1) > 0
+    assert K.kronq_qlinear_workspace_size(4096, 4096, 0) == 0
+    # pack: unsupported width, short buffer, misaligned destination
+    assert lib.kronq_pack_codes(16, 8, 8, 5, 256, 4096, None) == K.ERR_UNSUPPORTED
+    assert lib.kronq_pack_codes(16, 8, 8, 2, 256, 16, None) == K.ERR_SHAPE
+    assert lib.kronq_pack_codes(16, 8, 8, 2, 257, 4096, None) == K.ERR_INVALID_ARG
+    # pack_grid: group, size, alignment
+    assert K.kronq_packed_grid_bytes(300, 520, 128) == 3 * 5 * 128 * 8
+    assert K.kronq_packed_grid_bytes(300, 520, 0) == 3 * 128 * 8
+    assert lib.kronq_pack_grid(16, 32, 8, 8, 64, 256, 4096, None) == K.ERR_UNSUPPORTED
+    assert lib.kronq_pack_grid(16, 32, 8, 8, 0, 256, 8, None) == K.ERR_SHAPE
+    assert lib.kronq_pack_grid(16, 32, 8, 8, 0, 260, 4096, None) == K.ERR_INVALID_ARG
+    # qlinear: x, dtype, ld_x, n_tok, packed, grid, group, s_x, s_g, si, so, flags,
+    #          d_out, d_in, bits, y, ld_y, ws, ws_bytes, stream
+    ok = [256, K.DTYPE_F32, 64, 2, 512, 768, 0, 1280, 1536, 1792, 2048, K.BIIP_FULL,
+          32, 64, 2, 2304, 32, None, 0, None]
+
+    def call(**kw):
+        a = list(ok)
+        names = ["x", "dtype", "ld_x", "n_tok", "packed", "grid", "group", "s_x", "s_g",
+                 "si", "so", "flags", "d_out", "d_in", "bits", "y", "ld_y"]
+        for k, v in kw.items():
+            a[names.index(k)] = v
+        return lib.kronq_qlinear(*a)
+    assert call(bits=5) == K.ERR_UNSUPPORTED
+    assert call(group=64) == K.ERR_UNSUPPORTED
+    assert call(flags=16) == K.ERR_INVALID_ARG
+    assert call(dtype=7) == K.ERR_INVALID_ARG
+    assert call(n_tok=0) == K.OK                            # nothing to do
+    assert call(d_out=0) == K.ERR_SHAPE
+    assert call(grid=None) == K.ERR_INVALID_ARG
+    assert call(grid=772) == K.ERR_INVALID_ARG              # 8-byte alignment
+    assert call(s_g=None) == K.ERR_INVALID_ARG              # SCALE_OUT needs s_g
+    assert call(s_g=None, flags=K.BIIP_FULL & ~K.BIIP_SCALE_OUT) == K.ERR_WORKSPACE
+    assert call(si=None) == K.ERR_INVALID_ARG
+    assert call(ld_x=63) == K.ERR_SHAPE
+    assert call(packed=520) == K.ERR_INVALID_ARG            # 16-byte alignment
+    assert call(x=258) == K.ERR_INVALID_ARG                 # fp32 alignment
+    assert call(d_in=3 * 32768, ld_x=3 * 32768) == K.ERR_UNSUPPORTED   # Hadamard block 32768
+    assert call() == K.ERR_WORKSPACE                        # everything else valid
+
+
 def test_allocation_matches_golden_and_oracle(K):
     with open(os.path.join(ROOT, "tests", "golden", "allocation_cases.json")) as f:
         for c in json.load(f)["cases"]:

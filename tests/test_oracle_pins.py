@@ -605,30 +605,38 @@ def test_pack_roundtrip_size_and_density(bits, shape):
 
 
 def test_pack_hand_worked_positions():
-    # single codes placed by hand; the expected byte follows the format's wording:
-    # row r of blob (t, g) starts at byte (t G + g) 2048 b + 16 b r; word w is bytes 4w..4w+3
+    # single codes placed by hand; the expected byte follows the format's wording: byte k of
+    # row r's string sits at (t G + g) 2048 b + 1024 (k // 8) + 8 r + (k mod 8) of the packed
+    # array; word w of the string is its bytes 4w..4w+3
     def one(bits, shape, row, col, code):
         c = np.zeros(shape, dtype=np.uint8)
         c[row, col] = code
         p = O.pack_codes(c, bits)
-        nz = {int(i): int(p[i]) for i in np.flatnonzero(p)}
-        return nz
-    # b=2, col 1 = 2*0+1: half 1 of word 0, bits 16-17 -> byte 2 holds 0b11
-    assert one(2, (1, 20), 0, 1, 3) == {2: 0x03}
-    # b=2, row 1, col 14 (s=7, h=0): word 0 bits 14-15 of row 1 (byte 32 + 1); code 2 -> bit 15
-    assert one(2, (2, 20), 1, 14, 2) == {33: 0x80}
-    # b=2, col 17 (chunk 1, s=0, h=1): word 1 bit 16 -> byte 6
-    assert one(2, (1, 20), 0, 17, 1) == {6: 0x01}
-    # b=4, col 9 (chunk 0, s=4, h=1): word floor(16/16)=1, bits 16-19 -> byte 6 low nibble
-    assert one(4, (1, 20), 0, 9, 0xA) == {6: 0x0A}
-    # b=3, col 11 (s=5, h=1): word 1, bits 16-18 -> byte 6 holds the code
-    assert one(3, (1, 40), 0, 11, 6) == {6: 0x06}
-    # b=3, col 30 (s=15, h=0): bit i of the code at bit 15 of word i; code 5 = bits 0 and 2
-    assert one(3, (1, 40), 0, 30, 5) == {1: 0x80, 9: 0x80}
-    # b=3, col 31 (s=15, h=1): bit 31 of words 0..2; code 2 = bit 1 -> byte 7, bit 7
-    assert one(3, (1, 40), 0, 31, 2) == {7: 0x80}
-    # b=3, col 32 (chunk 1, s=0): word 3 bits 0-2 -> byte 12
-    assert one(3, (1, 40), 0, 32, 7) == {12: 0x07}
+        return {int(i): int(p[i]) for i in np.flatnonzero(p)}
+    # b=2, col 1 (w 0, k 0, j 1): bits 8-9 -> string byte 1, bits 0-1
+    assert one(2, (1, 20), 0, 1, 3) == {1: 0x03}
+    # b=2, col 6 (w 0, k 1, j 2): bits 18-19 -> byte 2, bits 2-3; code 2 -> bit 3
+    assert one(2, (1, 20), 0, 6, 2) == {2: 0x08}
+    # b=2, row 1, col 15 (w 0, k 3, j 3): bits 30-31 -> byte 3, bits 6-7; row 1 of piece 0
+    # starts at byte 8
+    assert one(2, (2, 20), 1, 15, 3) == {11: 0xC0}
+    # b=2, row 3, col 40 (w 2, k 2, j 0): bits 4-5 of word 2 -> string byte 8 = piece 1, k 0:
+    # 1024 + 24
+    assert one(2, (4, 60), 3, 40, 1) == {1048: 0x10}
+    # b=4, col 5 (w 0, k 1, j 1): bits 12-15 -> byte 1 high nibble
+    assert one(4, (1, 20), 0, 5, 0xA) == {1: 0xA0}
+    # b=4, row 2, col 127 (w 15, k 1, j 3): bits 28-31 of word 15 -> string byte 63 = piece 7,
+    # k 7: 7168 + 16 + 7
+    assert one(4, (3, 128), 2, 127, 0x9) == {7191: 0x90}
+    # b=3, col 5 (low bits: w 0, k 1, j 1 -> bits 10-11; top bit: word 2, k 1, j 1 -> bit 9):
+    # code 7 -> byte 1 bits 2-3 and byte 9 bit 1 (piece 1, k 1: 1025)
+    assert one(3, (1, 40), 0, 5, 7) == {1: 0x0C, 1025: 0x02}
+    # b=3, col 30 (low bits: w 1, k 3, j 2 -> bits 22-23 of word 1; top: word 2, k 7, j 2 ->
+    # bit 23): code 4 -> top bit only -> string byte 10 (piece 1, k 2: 1026), bit 7
+    assert one(3, (1, 40), 0, 30, 4) == {1026: 0x80}
+    # b=3, col 33 (chunk 1: w 3, k 0, j 1 -> bits 8-9 of word 3 = string byte 13; top: word 5,
+    # bit 8 = byte 21 = piece 2, k 5: 2048 + 5): code 3 -> low bits only
+    assert one(3, (1, 40), 0, 33, 3) == {1029: 0x03}
     # second group of tile 0 (G = 2) and first group of tile 1 (row 128)
     assert one(2, (1, 200), 0, 128, 1) == {4096: 0x01}
     assert one(4, (129, 20), 128, 0, 1) == {8192: 0x01}
@@ -652,3 +660,20 @@ def test_qlinear_of_codes_is_the_dense_layer_of_their_dequantization():
     u = O.transform_matrix(d_out, so); v = O.transform_matrix(d_in, si)
     want = x @ (np.diag(1 / s_g) @ u.T @ wq @ v @ np.diag(1 / s_x)).T
     np.testing.assert_allclose(y, want, rtol=0, atol=1e-12 * np.abs(want).max())
+
+
+@pytest.mark.parametrize("group", [0, 128])
+def test_pack_grid_places_each_pair(group):
+    # every (row, group) pair is found at (t G' + g) 128 + r and nothing else is non-zero
+    r = rng(94)
+    d_out, d_in = 300, 520
+    gp = -(-d_in // 128) if group else 1
+    sc = r.uniform(0.1, 1, (d_out, gp)).astype(np.float32)
+    zr = r.integers(1, 5, (d_out, gp)).astype(np.float32)
+    pk = O.pack_grid(sc if group else sc[:, 0], zr if group else zr[:, 0], d_out, d_in, group)
+    assert pk.shape == (3 * gp * 128, 2)
+    for row in range(d_out):
+        for g in range(gp):
+            idx = ((row // 128) * gp + g) * 128 + row % 128
+            assert pk[idx, 0] == sc[row, g] and pk[idx, 1] == zr[row, g]
+    assert np.count_nonzero(pk[:, 1]) == d_out * gp
