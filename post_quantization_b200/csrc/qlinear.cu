@@ -77,6 +77,28 @@ __device__ __forceinline__ bool bar_and(int id, int count, bool pred) {
   return out != 0;
 }
 
+// ---- thread-block clusters (distributed shared memory)
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile(
+      "barrier.cluster.arrive.release.aligned;\n\t"
+      "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t map_shared_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float ld_dsmem(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+
 // 32 lanes x 16 consecutive 32-bit TMEM columns.
 __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t* r) {
   asm volatile(
@@ -151,23 +173,31 @@ struct QlInArgs {
   int64_t ld_x;
   int n_tok;           // tokens of this pass
   int d_in;
-  int span;            // columns per CTA: max(b_in, 128)
+  int span;            // columns per CTA (a power of two, at least 128)
   int b_in;
+  int cl;              // CTAs per Hadamard block (a thread-block cluster), b_in = cl span when > 1
   const float* s_x;
   const int8_t* sign_in;
   uint32_t flags;
   float inv_sqrt_b;
   int rows;            // B rows: 3 n_tok rounded up to 8
+  int swz;             // 1: 128-byte swizzle (tensor-core operand), 0: plain rows
   uint8_t* bop;        // groups x [rows][128 bytes]: row 3 t + k = term k of token t
   float2* sums;        // groups x n_tok: (s, q0 + q1 / 128 + q2 / 128^2 summed over the group)
 };
 
-// One CTA per (span of columns, token), span / 16 threads (at least 32): thread t owns the 16
-// consecutive columns 16t..16t+15 at the end. The Hadamard stages run as radix-16 passes: in
-// the pass over index bits [4p, 4p + 4) each thread gathers the 16 elements that differ only in
-// those bits from shared memory and applies the four stages in registers.
+// One CTA per (span of columns, token). Hadamard blocks larger than a span are spread over a
+// cluster of cl CTAs: each applies the stages of the low index bits to its own contiguous span
+// (radix-16 passes: in the pass over bits [4p, 4p + 4) a thread gathers the 16 elements that
+// differ only in those bits and applies four stages in registers), then, after a cluster
+// barrier, combines element e of the cl spans through distributed shared memory:
+// H_b = (H_cl (x) I_span)(I_cl (x) H_span), and this CTA keeps row `rank` of H_cl. At the end
+// thread t (of span / 16) owns the 16 consecutive columns 16t .. 16t + 15.
 __global__ void __launch_bounds__(1024) qlin_in_kernel(QlInArgs a) {
-  extern __shared__ float xs[];                 // span floats
+  // two buffers of span + span / 16 floats: element i at i + i / 16 (one pad per 16 elements,
+  // so that the passes below are free of bank conflicts); the second takes the cluster result
+  extern __shared__ float xs[];
+  auto at = [](int i) { return i + (i >> 4); };
   griddep_launch_dependents();
   // x may be the output of the kernel before this one; the launch itself overlaps it
   griddep_wait();
@@ -179,21 +209,37 @@ __global__ void __launch_bounds__(1024) qlin_in_kernel(QlInArgs a) {
   const int len = min(a.span, a.d_in - j0);
   const bool rot = (a.flags & KRONQ_BIIP_ROTATE_IN) != 0;
   const bool scl = (a.flags & KRONQ_BIIP_SCALE_IN) != 0;
-  for (int j = tid; j < a.span; j += nthr) {
-    float v = 0.f;
-    if (j < len) {
-      const int64_t o = static_cast<int64_t>(t) * a.ld_x + j0 + j;
-      v = a.x_dtype == KRONQ_DTYPE_BF16
-              ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(a.x)[o])
-              : reinterpret_cast<const float*>(a.x)[o];
-      if (scl) v = v / a.s_x[j0 + j];
-      if (rot) v = a.sign_in[j0 + j] < 0 ? -v : v;
+  // at most 16 elements per thread (nthr >= span / 16): all loads issued before any is used
+  {
+    float xv[16], sv[16];
+    int8_t sg[16];
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+      const int j = tid + m * nthr;
+      xv[m] = 0.f;
+      sv[m] = 1.f;
+      sg[m] = 1;
+      if (j < len) {
+        const int64_t o = static_cast<int64_t>(t) * a.ld_x + j0 + j;
+        xv[m] = a.x_dtype == KRONQ_DTYPE_BF16
+                    ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(a.x)[o])
+                    : reinterpret_cast<const float*>(a.x)[o];
+        if (scl) sv[m] = a.s_x[j0 + j];
+        if (rot) sg[m] = a.sign_in[j0 + j];
+      }
     }
-    xs[j] = v;
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+      const int j = tid + m * nthr;
+      if (j < a.span) {
+        float v = scl ? xv[m] / sv[m] : xv[m];
+        xs[at(j)] = sg[m] < 0 ? -v : v;
+      }
+    }
   }
   __syncthreads();
   if (rot && a.b_in > 1) {
-    const int L = 31 - __clz(a.b_in);
+    const int L = 31 - __clz(min(a.b_in, a.span));   // stages inside this CTA's span
     int sh = 0;
     for (; sh + 4 <= L; sh += 4) {
       if (tid < nwork) {
@@ -201,7 +247,7 @@ __global__ void __launch_bounds__(1024) qlin_in_kernel(QlInArgs a) {
         const int base = lo | ((tid >> sh) << (sh + 4));
         float v[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] = xs[base + (j << sh)];
+        for (int j = 0; j < 16; ++j) v[j] = xs[at(base + (j << sh))];
 #pragma unroll
         for (int h = 1; h < 16; h <<= 1)
 #pragma unroll
@@ -212,7 +258,7 @@ __global__ void __launch_bounds__(1024) qlin_in_kernel(QlInArgs a) {
               v[j + h] = u - w;
             }
 #pragma unroll
-        for (int j = 0; j < 16; ++j) xs[base + (j << sh)] = v[j];
+        for (int j = 0; j < 16; ++j) xs[at(base + (j << sh))] = v[j];
       }
       __syncthreads();
     }
@@ -220,12 +266,30 @@ __global__ void __launch_bounds__(1024) qlin_in_kernel(QlInArgs a) {
       const int h = 1 << sh;
       for (int pi = tid; pi < a.span / 2; pi += nthr) {
         const int i = ((pi >> sh) << (sh + 1)) | (pi & (h - 1));
-        const float u = xs[i], w = xs[i + h];
-        xs[i] = u + w;
-        xs[i + h] = u - w;
+        const float u = xs[at(i)], w = xs[at(i + h)];
+        xs[at(i)] = u + w;
+        xs[at(i + h)] = u - w;
       }
       __syncthreads();
     }
+  }
+  float* xf = xs;                               // the transformed span
+  if (rot && a.cl > 1) {
+    float* xo = xs + a.span + a.span / 16;
+    const uint32_t rank = cluster_ctarank();
+    const uint32_t base = smem_u32(xs);
+    cluster_sync_all();                         // every span of the block is transformed
+    for (int e = tid; e < a.span; e += nthr) {
+      const uint32_t off = static_cast<uint32_t>(at(e)) * 4u;
+      float v = 0.f;
+      for (int r2 = 0; r2 < a.cl; ++r2) {
+        const float z = ld_dsmem(map_shared_rank(base + off, static_cast<uint32_t>(r2)));
+        v += (__popc(rank & static_cast<uint32_t>(r2)) & 1) ? -z : z;
+      }
+      xo[at(e)] = v;
+    }
+    cluster_sync_all();                         // no CTA leaves while another still reads it
+    xf = xo;
   }
   // B operand: thread = 16 columns = one 16-byte unit of each of the token's three term rows;
   // a group's 128 columns belong to 8 consecutive threads (its maximum and sums by shuffles)
@@ -234,8 +298,8 @@ __global__ void __launch_bounds__(1024) qlin_in_kernel(QlInArgs a) {
   if (tid < nwork) {
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
-      const float v = 16 * tid + e < len ? (rot ? xs[16 * tid + e] * a.inv_sqrt_b
-                                                : xs[16 * tid + e])
+      const float v = 16 * tid + e < len ? (rot ? xf[17 * tid + e] * a.inv_sqrt_b
+                                                : xf[17 * tid + e])
                                          : 0.f;
       xv[e] = v;
       amax = fmaxf(amax, fabsf(v));
@@ -246,9 +310,12 @@ __global__ void __launch_bounds__(1024) qlin_in_kernel(QlInArgs a) {
   // s = the smallest power of two with 127 s >= max |x'| over the group (1 for a zero group)
   float sc = 1.f;
   if (amax > 0.f) {
-    int ex;
-    const float m = frexpf(amax / 127.f, &ex);    // amax / 127 = m 2^ex, m in [0.5, 1)
-    sc = ldexpf(1.f, m == 0.5f ? ex - 1 : ex);
+    // exponent field of amax / 127, raised by one unless the mantissa is exactly 1; values
+    // below the normal range are not reached by activations and round up to 2^-126
+    const uint32_t bits = __float_as_uint(amax / 127.f);
+    uint32_t e = bits & 0x7F800000u;
+    if ((bits & 0x007FFFFFu) != 0u || e == 0u) e += 0x00800000u;
+    sc = __uint_as_float(e);
   }
   const float inv_sc = 1.f / sc;                 // exact: a power of two
   int qsum[QL_TERMS] = {0, 0, 0};
@@ -277,7 +344,7 @@ __global__ void __launch_bounds__(1024) qlin_in_kernel(QlInArgs a) {
 #pragma unroll
     for (int k = 0; k < QL_TERMS; ++k) {
       const int rho = QL_TERMS * t + k;
-      *reinterpret_cast<uint4*>(gb + rho * 128 + ((unit ^ (rho & 7)) << 4)) =
+      *reinterpret_cast<uint4*>(gb + rho * 128 + ((a.swz ? unit ^ (rho & 7) : unit) << 4)) =
           make_uint4(wq[k][0], wq[k][1], wq[k][2], wq[k][3]);
     }
   }
@@ -441,10 +508,13 @@ __global__ void __launch_bounds__(QL_THREADS, 1) qlin_mma_kernel(QlMmaArgs p) {
   const int S = p.stages;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint64_t* empty = full + QL_MAX_STAGES;
+  // unit i uses A tile and accumulator i % 4: afull (dequantization done), mdone (its MMAs
+  // done: the A tile is free and the accumulator full), accempty (the epilogue drained it)
   uint64_t* afull = empty + QL_MAX_STAGES;      // QL_NA
-  uint64_t* aempty = afull + QL_NA;             // QL_NA
-  uint64_t* accfull = aempty + QL_NA;           // QL_NACC
-  uint64_t* accempty = accfull + QL_NACC;       // QL_NACC
+  uint64_t* mdone = afull + QL_NA;              // QL_NA
+  uint64_t* accfull = mdone;                    // the same barrier, seen by the epilogue
+  uint64_t* accempty = mdone + QL_NA;           // QL_NACC
+  static_assert(QL_NA == 4 && QL_NACC == 4, "unit i uses slot i & 3 of both rings");
   volatile int* abort_flag = reinterpret_cast<volatile int*>(accempty + QL_NACC);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accempty + QL_NACC) + 1;
   float* xchg = reinterpret_cast<float*>(smem + L.xchg);
@@ -467,10 +537,9 @@ __global__ void __launch_bounds__(QL_THREADS, 1) qlin_mma_kernel(QlMmaArgs p) {
     }
     for (int i = 0; i < QL_NA; ++i) {
       mbar_init(&afull[i], QL_DQ_THREADS / 32);
-      mbar_init(&aempty[i], 1);
+      mbar_init(&mdone[i], 1);
     }
     for (int i = 0; i < QL_NACC; ++i) {
-      mbar_init(&accfull[i], 1);
       mbar_init(&accempty[i], 4);
     }
     *abort_flag = 0;
@@ -499,10 +568,9 @@ __global__ void __launch_bounds__(QL_THREADS, 1) qlin_mma_kernel(QlMmaArgs p) {
                   nu * pk_bytes, &full[si]);
       }
       griddep_wait();
-      int si = 0, g = g0;
-      for (; si < n_stages && ok; ++si) {
-        const int s = si % S;
-        const uint32_t ph = (si / S) & 1u;
+      int si = 0, g = g0, s = 0;
+      uint32_t ph = 0;
+      for (; si < n_stages && ok; ++si, s = (s + 1 == S) ? 0 : s + 1, ph ^= (s == 0)) {
         const int i0 = si * ku, nu = min(ku, n_units - i0);
         uint8_t* st = stage_ptr(s);
         if (si >= pre) {
@@ -534,36 +602,40 @@ __global__ void __launch_bounds__(QL_THREADS, 1) qlin_mma_kernel(QlMmaArgs p) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = ql_idesc(128, p.N);
-      int k = 0, si = 0;
+      // descriptor of a stage's first B tile; a tile k and a K step kk add (k b_unit + 32 kk)
+      // bytes, i.e. (k b_unit + 32 kk) / 16 in the descriptor's address field
+      const uint64_t bdesc0 = smem_desc_sw128(smem_u32(stage_ptr(0)), 16, 1024);
+      const uint32_t stage_step = L.stage_bytes >> 4, unit_step = L.b_unit >> 4;
+      int k = 0, s = 0;
+      uint32_t ph = 0;
+      uint64_t bstage = bdesc0;
       // one accumulator per unit (the scale of x' changes from group to group)
       for (int i = 0; i < n_units; ++i) {
-        const int s = si % S;
-        const uint32_t ph = (si / S) & 1u;
-        const int ab = i % QL_NA;
-        const uint32_t aph = (i / QL_NA) & 1u;
-        const int acc = i % QL_NACC;
-        const uint32_t cph = (i / QL_NACC) & 1u;
+        const int b = i & 3;
+        const uint32_t bph = (i >> 2) & 1u;
         if (k == 0 && !mbar_wait(&full[s], ph, abort_flag, p.err, DEV_ERR_MMA_WAIT)) break;
-        if (!mbar_wait(&afull[ab], aph, abort_flag, p.err, DEV_ERR_MMA_WAIT)) break;
-        if (!mbar_wait(&accempty[acc], cph ^ 1u, abort_flag, p.err, DEV_ERR_MMA_WAIT)) break;
+        if (!mbar_wait(&afull[b], bph, abort_flag, p.err, DEV_ERR_MMA_WAIT)) break;
+        if (!mbar_wait(&accempty[b], bph ^ 1u, abort_flag, p.err, DEV_ERR_MMA_WAIT)) break;
         tc_fence_after();
-        const uint32_t a_tmem = tmem_base + ab * QL_A_COLS;
-        const uint32_t bbase = smem_u32(stage_ptr(s) + k * L.b_unit);
-        const uint32_t d_tmem = tmem_base + QL_ACC_COL0 + acc * p.N;
+        const uint32_t a_tmem = tmem_base + b * QL_A_COLS;
+        const uint32_t d_tmem = tmem_base + QL_ACC_COL0 + b * p.N;
+        const uint64_t bd = bstage + k * unit_step;
         // K = 128 in four steps of 32 8-bit values (32 bytes of each A and B row)
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t bd = smem_desc_sw128(bbase + kk * 32, 16, 1024);
-          umma_i8_ts(d_tmem, a_tmem + kk * 8, bd, idesc, kk ? 1u : 0u);
-        }
-        umma_commit(&aempty[ab]);
-        umma_commit(&accfull[acc]);
-        if (k == ku - 1 || i == n_units - 1) {
+        umma_i8_ts(d_tmem, a_tmem, bd, idesc, 0u);
+        umma_i8_ts(d_tmem, a_tmem + 8, bd + 2, idesc, 1u);
+        umma_i8_ts(d_tmem, a_tmem + 16, bd + 4, idesc, 1u);
+        umma_i8_ts(d_tmem, a_tmem + 24, bd + 6, idesc, 1u);
+        umma_commit(&mdone[b]);
+        if (++k == ku || i == n_units - 1) {
           umma_commit(&empty[s]);          // the stage's codes and B tiles are consumed
           k = 0;
-          ++si;
-        } else {
-          ++k;
+          if (++s == S) {
+            s = 0;
+            ph ^= 1u;
+            bstage = bdesc0;
+          } else {
+            bstage += stage_step;
+          }
         }
       }
     }
@@ -572,16 +644,15 @@ __global__ void __launch_bounds__(QL_THREADS, 1) qlin_mma_kernel(QlMmaArgs p) {
     // warp w writes TMEM lanes 32 (w % 4) .. + 31 (its rows) for column half (w - 8) / 4
     const int q = warp & 3, kh = (warp - QL_DQ_WARP0) >> 2;
     const int r = q * 32 + lane;
-    int k = 0, si = 0;
+    int k = 0, s = 0;
+    uint32_t ph = 0;
     for (int i = 0; i < n_units; ++i) {
-      const int s = si % S;
-      const uint32_t ph = (si / S) & 1u;
-      const int ab = i % QL_NA;
-      const uint32_t aph = (i / QL_NA) & 1u;
+      const int ab = i & 3;
+      const uint32_t aph = (i >> 2) & 1u;
       int ok = 1;
       if (lane == 0) {
         ok = (k != 0 || mbar_wait(&full[s], ph, abort_flag, p.err, DEV_ERR_MMA_WAIT)) &&
-             mbar_wait(&aempty[ab], aph ^ 1u, abort_flag, p.err, DEV_ERR_MMA_WAIT);
+             mbar_wait(&mdone[ab], aph ^ 1u, abort_flag, p.err, DEV_ERR_MMA_WAIT);
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
@@ -597,7 +668,10 @@ __global__ void __launch_bounds__(QL_THREADS, 1) qlin_mma_kernel(QlMmaArgs p) {
       if (lane == 0) mbar_arrive(&afull[ab]);
       if (++k == ku) {
         k = 0;
-        ++si;
+        if (++s == S) {
+          s = 0;
+          ph ^= 1u;
+        }
       }
     }
   } else if (warp >= QL_EPI_WARP0) {
@@ -628,8 +702,8 @@ __global__ void __launch_bounds__(QL_THREADS, 1) qlin_mma_kernel(QlMmaArgs p) {
       const float2 gz = __ldg(&p.grid[p.grouped
                                           ? (static_cast<int64_t>(tcur) * p.G + gcur) * QL_TILE + r
                                           : static_cast<int64_t>(tcur) * QL_TILE + r]);
-      const int acc = i % QL_NACC;
-      const uint32_t cph = (i / QL_NACC) & 1u;
+      const int acc = i & 3;
+      const uint32_t cph = (i >> 2) & 1u;
       int ok = 1;
       if (lane == 0) ok = mbar_wait(&accfull[acc], cph, abort_flag, p.err, DEV_ERR_EPI_WAIT);
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -727,6 +801,213 @@ __global__ void __launch_bounds__(QL_THREADS, 1) qlin_mma_kernel(QlMmaArgs p) {
 }
 
 // ---------------------------------------------------------------------------------------------
+// Decode on the CUDA cores (1 or 2 tokens)
+// ---------------------------------------------------------------------------------------------
+// A tensor-core MMA costs the same for any N <= 256 and covers 128 rows x 32 bytes of the code
+// matrix, which caps the tensor-core pass near 22 codes per cycle per SM. For a few tokens the
+// CUDA cores do better: one thread per row and unit, codes masked in place (no shifts: a code in
+// bit pair k of a byte is 4^k c, and each k keeps its own accumulator), and dp4a with the three
+// int8 terms of x' (exact int32 sums, as on the tensor cores).
+struct QlDpArgs {
+  const uint8_t* packed;
+  const uint8_t* bop;      // groups x [rows][128 bytes], plain rows, row 3 t + k = term k
+  const float2* sums;      // groups x n_tok: (s, sum of the three terms)
+  const float2* grid;
+  float* partial;          // (C + T) segments x n_tok x 128
+  int d_out, G, n_tok, rows;
+  int grouped, rotate_out, b_tile;
+  int64_t U;
+};
+
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// exact int -> float for |v| < 2^22
+__device__ __forceinline__ float i2f_small(int v) {
+  return __int_as_float(v + 0x4B400000) - 12582912.f;
+}
+
+template <int BITS>
+struct DpCodes {
+  static constexpr int PIECES = 2 * BITS;   // 8-byte pieces per row and unit
+  uint2 p[PIECES];
+};
+
+template <int BITS>
+__device__ __forceinline__ void dp_load(const uint8_t* blob, int r, DpCodes<BITS>& c) {
+  const uint2* pc = reinterpret_cast<const uint2*>(blob) + r;
+#pragma unroll
+  for (int i = 0; i < DpCodes<BITS>::PIECES; ++i) c.p[i] = __ldg(pc + i * 128);
+}
+
+// acc[term][part] += codes . x' terms over the unit's 128 columns; the parts carry the codes'
+// bit-position factors (2 bits: 4^k, 4 bits: 16^k, 3 bits: 1)
+template <int BITS, int NT>
+__device__ __forceinline__ void dp_unit(const DpCodes<BITS>& c, const uint8_t* xg,
+                                        int n_tok, int (&acc)[NT][QL_TERMS][4]) {
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(c.p);
+#pragma unroll
+  for (int t = 0; t < NT; ++t)
+#pragma unroll
+    for (int k = 0; k < QL_TERMS; ++k)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[t][k][j] = 0;
+#pragma unroll
+  for (int t = 0; t < NT; ++t) {
+    if (t >= n_tok) break;
+#pragma unroll
+    for (int term = 0; term < QL_TERMS; ++term) {
+      const uint4* xr = reinterpret_cast<const uint4*>(xg + (3 * t + term) * 128);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {                  // 16 columns per step
+        const uint4 xv = xr[q];                       // x' bytes of columns 16q .. 16q + 15
+        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+        if (BITS == 2) {
+          // word q: columns 16q + 4k + j at bits 8j + 2k
+          const uint32_t wd = w[q];
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            acc[t][term][k] = dp4a_us(wd & (0x03030303u << (2 * k)), xw[k], acc[t][term][k]);
+        } else if (BITS == 4) {
+          // words 2q, 2q + 1: columns 8w + 4k + j at bits 8j + 4k
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t wd = w[2 * q + h];
+            acc[t][term][0] = dp4a_us(wd & 0x0F0F0F0Fu, xw[2 * h], acc[t][term][0]);
+            acc[t][term][1] = dp4a_us(wd & 0xF0F0F0F0u, xw[2 * h + 1], acc[t][term][1]);
+          }
+        } else {
+          // 32 columns per three words: low bits in words 3m, 3m + 1, top bits in word 3m + 2
+          const int m = q >> 1, half = q & 1;
+          const uint32_t wl = w[3 * m + half], wh = w[3 * m + 2];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int k8 = 4 * half + k;
+            const uint32_t lo = (wl >> (2 * k)) & 0x03030303u;
+            const uint32_t hi = (k8 >= 2 ? (wh >> (k8 - 2)) : (wh << (2 - k8))) & 0x04040404u;
+            acc[t][term][0] = dp4a_us(lo | hi, xw[k], acc[t][term][0]);
+          }
+        }
+      }
+    }
+  }
+}
+
+template <int BITS, int NT>
+__global__ void __launch_bounds__(128, 4) qlin_dp4a_kernel(QlDpArgs p) {
+  __shared__ float ys[NT][QL_TILE];
+  // x' terms of the groups this CTA visits: groups g0 .. g0 + n_units - 1 (mod G) in visiting
+  // order, or all G groups at their own index when the CTA visits every group
+  extern __shared__ __align__(16) uint8_t xstage[];
+  const int r = threadIdx.x;                          // row of the tile
+  const int lane = r & 31;
+  const int64_t C = gridDim.x;
+  const int64_t u0 = unit_begin(blockIdx.x, p.U, C);
+  const int64_t u1 = unit_begin(blockIdx.x + 1, p.U, C);
+  const int n_units = static_cast<int>(u1 - u0);
+  constexpr int D = BITS == 2 ? 4 : 2;                // units of codes in flight per thread
+  const int64_t blob = 2048 * BITS;
+  DpCodes<BITS> buf[D];
+  // the packed codes do not depend on the preceding kernel: load them before waiting
+#pragma unroll
+  for (int d = 0; d < D; ++d)
+    if (d < n_units) dp_load<BITS>(p.packed + (u0 + d) * blob, r, buf[d]);
+  griddep_wait();                                     // x' and its sums come from qlin_in
+  const int gb = 128 * p.rows;                         // bytes of one group's terms
+  const bool all_groups = n_units >= p.G;
+  {
+    const int gstart = all_groups ? 0 : static_cast<int>(u0 % p.G);
+    const int ng = all_groups ? p.G : n_units;
+    const int words = ng * gb / 16;
+    for (int w = threadIdx.x; w < words; w += blockDim.x) {
+      const int gi = w / (gb / 16), off = w % (gb / 16);
+      int gsrc = gstart + gi;
+      if (gsrc >= p.G) gsrc -= p.G;
+      reinterpret_cast<uint4*>(xstage)[w] =
+          __ldg(reinterpret_cast<const uint4*>(p.bop + static_cast<int64_t>(gsrc) * gb) + off);
+    }
+    __syncthreads();
+  }
+  float y[NT];
+#pragma unroll
+  for (int t = 0; t < NT; ++t) y[t] = 0.f;
+  int g = static_cast<int>(u0 % p.G);
+  int tile = static_cast<int>(u0 / p.G);
+  for (int i0 = 0; i0 < n_units; i0 += D) {
+#pragma unroll
+    for (int d = 0; d < D; ++d) {
+      const int i = i0 + d;
+      if (i >= n_units) break;
+      const int row = tile * QL_TILE + r;
+      const float2 gz = __ldg(&p.grid[p.grouped
+                                          ? (static_cast<int64_t>(tile) * p.G + g) * QL_TILE + r
+                                          : static_cast<int64_t>(tile) * QL_TILE + r]);
+      int acc[NT][QL_TERMS][4];
+      dp_unit<BITS, NT>(buf[d], xstage + (all_groups ? g : i) * gb, p.n_tok, acc);
+      if (i + D < n_units) dp_load<BITS>(p.packed + (u0 + i + D) * blob, r, buf[d]);
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        if (t >= p.n_tok) break;
+        const float2 sq = __ldg(&p.sums[static_cast<int64_t>(g) * p.n_tok + t]);
+        float a[QL_TERMS];
+#pragma unroll
+        for (int term = 0; term < QL_TERMS; ++term) {
+          // each part is an exact multiple of its bit-position factor
+          int v = acc[t][term][0];
+          if (BITS == 2)
+            v += (acc[t][term][1] >> 2) + (acc[t][term][2] >> 4) + (acc[t][term][3] >> 6);
+          else if (BITS == 4)
+            v += acc[t][term][1] >> 4;
+          a[term] = i2f_small(v);
+        }
+        const float dot = a[0] + a[1] * (1.f / 128.f) + a[2] * (1.f / 16384.f);
+        if (row < p.d_out) y[t] = fmaf(gz.x * sq.x, fmaf(-gz.y, sq.y, dot), y[t]);
+      }
+      // end of this CTA's part of the tile: within-tile Hadamard, then one partial
+      const bool seg_end = (i == n_units - 1) || (g == p.G - 1);
+      if (seg_end) {
+        if (p.rotate_out) {
+#pragma unroll
+          for (int h = 1; h < 32; h <<= 1) {
+            if (h >= p.b_tile) break;
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+              const float o = __shfl_xor_sync(0xffffffffu, y[t], h);
+              y[t] = (lane & h) ? (o - y[t]) : (y[t] + o);
+            }
+          }
+          for (int h = 32; h < p.b_tile; h <<= 1) {
+            __syncthreads();
+#pragma unroll
+            for (int t = 0; t < NT; ++t) ys[t][r] = y[t];
+            __syncthreads();
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+              const float o = ys[t][r ^ h];
+              y[t] = (r & h) ? (o - y[t]) : (y[t] + o);
+            }
+          }
+        }
+        float* out = p.partial + (static_cast<int64_t>(blockIdx.x) + tile) * p.n_tok * QL_TILE + r;
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          if (t < p.n_tok) out[t * QL_TILE] = y[t];
+          y[t] = 0.f;
+        }
+      }
+      if (++g == p.G) {
+        g = 0;
+        ++tile;
+      }
+    }
+  }
+  griddep_launch_dependents();
+}
+
+// ---------------------------------------------------------------------------------------------
 // Output side: sum of partials, across-tile Hadamard, signs, S_G^-1
 // ---------------------------------------------------------------------------------------------
 struct QlOutArgs {
@@ -734,6 +1015,7 @@ struct QlOutArgs {
   int n_tok, T, G;
   int64_t U, C;
   int qb;              // tiles per output Hadamard block (1 when b_out <= 128 or no rotation)
+  int tpe;             // threads per output element in the partial-sum gather (power of two)
   int d_out;
   const float* s_g;
   const int8_t* sign_out;
@@ -763,26 +1045,50 @@ __global__ void __launch_bounds__(1024) qlin_out_kernel(QlOutArgs a) {
     cbound[2 * qi] = static_cast<int>(cta_of_unit(tile * a.G, a.U, a.C));
     cbound[2 * qi + 1] = static_cast<int>(cta_of_unit(tile * a.G + a.G - 1, a.U, a.C));
   }
+  // output scale of this thread's first row (most CTAs give one row per thread), read while
+  // the preceding kernel still runs
+  const bool rot = (a.flags & KRONQ_BIIP_ROTATE_OUT) != 0;
+  float oscale = 1.f;
+  {
+    const int e = threadIdx.x;
+    const int64_t i = static_cast<int64_t>(sb * a.qb + (e >> 4)) * QL_TILE + slice * 16 + (e & 15);
+    if (e < a.qb * 16 && i < a.d_out) {
+      if (rot) oscale = a.sign_out[i] < 0 ? -a.inv_sqrt_b : a.inv_sqrt_b;
+      if (a.flags & KRONQ_BIIP_SCALE_OUT) oscale = oscale / a.s_g[i];
+    }
+  }
   griddep_wait();
   __syncthreads();
   const int n = a.qb * 16;
-  for (int e = threadIdx.x; e < n; e += blockDim.x) {
-    const int qi = e >> 4, r = slice * 16 + (e & 15);
-    const int64_t tile = static_cast<int64_t>(sb) * a.qb + qi;
-    const int c0 = cbound[2 * qi], c1 = cbound[2 * qi + 1];
-    const float* src = a.partial + ((c0 + tile) * a.n_tok + tok) * QL_TILE + r;
-    const int64_t step = static_cast<int64_t>(a.n_tok) * QL_TILE;   // next segment
-    float v0 = 0.f, v1 = 0.f;
-    int c = c0;
-    for (; c + 1 <= c1; c += 2) {               // two independent loads in flight
-      v0 += src[(c - c0) * step];
-      v1 += src[(c + 1 - c0) * step];
+  // a.tpe consecutive threads share an element: each sums every tpe-th of its segments, with
+  // four loads in flight, then the tpe sums are combined by shuffles in a fixed order
+  const int tpe = a.tpe;
+  const int epw = 32 / tpe;                     // elements per warp and step
+  const int wid = threadIdx.x >> 5, lid = threadIdx.x & 31;
+  for (int base = wid * epw; base < n; base += (blockDim.x >> 5) * epw) {   // warp-uniform
+    const int e0 = base + lid / tpe, sub = lid % tpe;
+    float tot = 0.f;
+    if (e0 < n) {
+      const int qi = e0 >> 4, r = slice * 16 + (e0 & 15);
+      const int64_t tile = static_cast<int64_t>(sb) * a.qb + qi;
+      const int c0 = cbound[2 * qi], c1 = cbound[2 * qi + 1];
+      const int64_t seg = static_cast<int64_t>(a.n_tok) * QL_TILE;      // next segment
+      const float* ps = a.partial + ((c0 + tile) * a.n_tok + tok) * QL_TILE + r + sub * seg;
+      const int64_t step = seg * tpe;                                     // next own segment
+      const int cnt = c1 - c0 + 1;
+      float v[4] = {0.f, 0.f, 0.f, 0.f};
+      int k = sub;
+      for (; k + 3 * tpe < cnt; k += 4 * tpe, ps += 4 * step) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v[j] += ps[j * step];
+      }
+      for (int j = 0; k < cnt; k += tpe, ++j, ps += step) v[j & 3] += *ps;
+      tot = (v[0] + v[1]) + (v[2] + v[3]);
     }
-    if (c <= c1) v0 += src[(c - c0) * step];
-    ys[e] = v0 + v1;
+    for (int o = 1; o < tpe; o <<= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+    if (e0 < n && sub == 0) ys[e0] = tot;
   }
   __syncthreads();
-  const bool rot = (a.flags & KRONQ_BIIP_ROTATE_OUT) != 0;
   if (rot && a.qb > 1) {
     for (int sh = 0; (1 << sh) < a.qb; ++sh) {
       const int h = 1 << sh;
@@ -801,13 +1107,13 @@ __global__ void __launch_bounds__(1024) qlin_out_kernel(QlOutArgs a) {
     const int qi = e >> 4, r = slice * 16 + (e & 15);
     const int64_t i = static_cast<int64_t>(sb * a.qb + qi) * QL_TILE + r;
     if (i >= a.d_out) continue;
-    float v = ys[e];
-    if (rot) {
-      v *= a.inv_sqrt_b;
-      if (a.sign_out[i] < 0) v = -v;
+    float os = oscale;
+    if (e != threadIdx.x) {                     // rows past the first: scale read now
+      os = 1.f;
+      if (rot) os = a.sign_out[i] < 0 ? -a.inv_sqrt_b : a.inv_sqrt_b;
+      if (a.flags & KRONQ_BIIP_SCALE_OUT) os = os / a.s_g[i];
     }
-    if (a.flags & KRONQ_BIIP_SCALE_OUT) v = v / a.s_g[i];
-    a.y[tok * a.ld_y + i] = v;
+    a.y[tok * a.ld_y + i] = ys[e] * os;
   }
 }
 
@@ -831,25 +1137,40 @@ __global__ void pack_grid_kernel(const float* __restrict__ scale, const float* _
   out[idx] = v;
 }
 
-template <typename Kern, typename... Args>
+template <typename Kern, typename Arg>
 kronq_status launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
-                        bool pdl, const char* what, Args... args) {
+                        bool pdl, const char* what, Arg arg, int cluster = 1) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (cluster > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = static_cast<unsigned>(cluster);
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  cfg.numAttrs = na;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, arg);
   if (e != cudaSuccess) return fail(KRONQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
   return check_launch(what);
 }
 
 int pow2_factor(int d) { return d & (-d); }
+
+constexpr int QL_DP_MAX_TOK = 2;   // up to this many tokens: the CUDA-core decode kernel
+constexpr int QL_DP_CTAS_PER_SM = 4;
+constexpr int QL_DP_MAX_UNITS = 48;   // units per CTA (its x' groups are staged in shared memory)
 
 struct QlGeom {
   int T, G, C;
@@ -863,7 +1184,15 @@ QlGeom ql_geom(int d_out, int d_in, int n_tok_pass) {
   g.T = (d_out + QL_TILE - 1) / QL_TILE;
   g.G = (d_in + QL_TILE - 1) / QL_TILE;
   g.U = static_cast<int64_t>(g.T) * g.G;
-  g.C = static_cast<int>(std::min<int64_t>(g.U, sm_budget()));
+  // CTAs (one partial per CTA and tile): one per SM for the tensor-core pass, several per SM
+  // for the CUDA-core decode kernel
+  const bool decode = n_tok_pass <= QL_DP_MAX_TOK;
+  const int per_sm = decode ? QL_DP_CTAS_PER_SM : 1;
+  g.C = static_cast<int>(std::min<int64_t>(g.U, static_cast<int64_t>(per_sm) * sm_budget()));
+  if (decode) {
+    // at most QL_DP_MAX_UNITS units (and staged groups) per CTA
+    g.C = static_cast<int>(std::max<int64_t>(g.C, (g.U + QL_DP_MAX_UNITS - 1) / QL_DP_MAX_UNITS));
+  }
   g.span = std::max(pow2_factor(d_in), QL_TILE);
   g.bop_bytes = align256(static_cast<size_t>(g.G) * 128 * ((3 * n_tok_pass + 7) / 8 * 8));
   g.sums_bytes = align256(static_cast<size_t>(g.G) * n_tok_pass * sizeof(float2));
@@ -879,6 +1208,24 @@ kronq_status launch_mma_t(const QlMmaArgs& p, int C, size_t smem, cudaStream_t s
                                              static_cast<int>(smem));
   if (e != cudaSuccess) return fail(KRONQ_ERR_CUDA, "qlin_mma smem: %s", cudaGetErrorString(e));
   return launch_pdl(kern, dim3(C), dim3(QL_THREADS), smem, stream, true, "qlin_mma_kernel", p);
+}
+
+template <int BITS, int NT>
+kronq_status launch_dp_t(const QlDpArgs& p, int C, size_t smem, cudaStream_t stream) {
+  auto kern = qlin_dp4a_kernel<BITS, NT>;
+  const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem));
+  if (e != cudaSuccess) return fail(KRONQ_ERR_CUDA, "qlin_dp4a smem: %s", cudaGetErrorString(e));
+  return launch_pdl(kern, dim3(C), dim3(QL_TILE), smem, stream, true, "qlin_dp4a_kernel", p);
+}
+
+kronq_status launch_dp(int bits, int nt, const QlDpArgs& p, int C, size_t smem,
+                       cudaStream_t stream) {
+  if (bits == 2)
+    return nt <= 1 ? launch_dp_t<2, 1>(p, C, smem, stream) : launch_dp_t<2, 2>(p, C, smem, stream);
+  if (bits == 3)
+    return nt <= 1 ? launch_dp_t<3, 1>(p, C, smem, stream) : launch_dp_t<3, 2>(p, C, smem, stream);
+  return nt <= 1 ? launch_dp_t<4, 1>(p, C, smem, stream) : launch_dp_t<4, 2>(p, C, smem, stream);
 }
 
 kronq_status launch_mma(int bits, int ntc, const QlMmaArgs& p, int C, size_t smem,
@@ -952,8 +1299,18 @@ kronq_status run_qlinear(const QlinearArgs& q, void* ws, cudaStream_t stream) {
     return fail(KRONQ_ERR_UNSUPPORTED, "input Hadamard block %d > 16384", b_in);
   if (rot_out && b_out > 16384)
     return fail(KRONQ_ERR_UNSUPPORTED, "output Hadamard block %d > 16384", b_out);
-  const int span = rot_in ? g.span : QL_TILE;
-  const size_t in_smem = static_cast<size_t>(span) * sizeof(float);
+  // columns per CTA and CTAs per Hadamard block (a cluster of at most 8)
+  int span = QL_TILE, cl = 1;
+  if (rot_in) {
+    if (b_in <= 1024) {
+      span = std::max(QL_TILE, b_in);
+    } else {
+      span = std::max(1024, b_in / 8);
+      cl = b_in / span;
+    }
+  }
+  const int in_threads = std::max(32, span / 4);
+  const size_t in_smem = static_cast<size_t>(2 * (span + span / 16)) * sizeof(float);
   KQ_CUDA_TRY(cudaFuncSetAttribute(qlin_in_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    static_cast<int>(in_smem)));
   const int qb = (rot_out && b_out > QL_TILE) ? b_out / QL_TILE : 1;
@@ -963,6 +1320,7 @@ kronq_status run_qlinear(const QlinearArgs& q, void* ws, cudaStream_t stream) {
   KQ_CUDA_TRY(cudaGetDevice(&dev));
   KQ_CUDA_TRY(cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
 
+  const bool decode = q.n_tok <= QL_DP_MAX_TOK;
   for (int t0 = 0; t0 < q.n_tok; t0 += QL_NT_MAX) {
     const int nt = std::min(QL_NT_MAX, q.n_tok - t0);
     QlInArgs ia;
@@ -974,20 +1332,41 @@ kronq_status run_qlinear(const QlinearArgs& q, void* ws, cudaStream_t stream) {
     ia.d_in = q.d_in;
     ia.span = span;
     ia.b_in = rot_in ? b_in : 1;
+    ia.cl = cl;
     ia.s_x = q.s_x;
     ia.sign_in = q.sign_in;
     ia.flags = q.flags;
     ia.inv_sqrt_b = static_cast<float>(1.0 / std::sqrt(static_cast<double>(b_in)));
     ia.rows = (3 * nt + 7) / 8 * 8;
+    ia.swz = decode ? 0 : 1;
     ia.bop = bop;
     ia.sums = sums;
     const dim3 igrid((q.d_in + span - 1) / span, nt);
     // Chained to the previous kernel too: only the launch overlaps it, since qlin_in waits for
     // it to complete before reading x (which the previous kernel may have written); so this
     // call's workspace writes never race with a previous call's reads.
-    KQ_TRY(launch_pdl(qlin_in_kernel, igrid, dim3(std::max(32, span / 16)), in_smem, stream, true,
-                      "qlin_in_kernel", ia));
+    KQ_TRY(launch_pdl(qlin_in_kernel, igrid, dim3(in_threads), in_smem, stream, true,
+                      "qlin_in_kernel", ia, cl));
 
+    if (decode) {
+      QlDpArgs dpa;
+      dpa.packed = static_cast<const uint8_t*>(q.packed);
+      dpa.bop = bop;
+      dpa.sums = sums;
+      dpa.grid = static_cast<const float2*>(q.grid);
+      dpa.partial = partial;
+      dpa.d_out = q.d_out;
+      dpa.G = g.G;
+      dpa.n_tok = nt;
+      dpa.rows = ia.rows;
+      dpa.grouped = q.group ? 1 : 0;
+      dpa.rotate_out = rot_out ? 1 : 0;
+      dpa.b_tile = rot_out ? std::min(b_out, QL_TILE) : 1;
+      dpa.U = g.U;
+      const int64_t upc = (g.U + g.C - 1) / g.C;          // units of the largest CTA
+      const size_t dsmem = static_cast<size_t>(std::min<int64_t>(upc, g.G)) * 128 * dpa.rows;
+      KQ_TRY(launch_dp(q.bits, nt, dpa, g.C, dsmem, stream));
+    } else {
     QlMmaArgs p;
     p.packed = static_cast<const uint8_t*>(q.packed);
     p.bop = bop;
@@ -1016,6 +1395,7 @@ kronq_status run_qlinear(const QlinearArgs& q, void* ws, cudaStream_t stream) {
     const size_t smem = std::max<size_t>(ql_smem(q.bits, p.N, p.R, p.ku, p.stages).total,
                                          117 * 1024);
     KQ_TRY(launch_mma(q.bits, nt, p, g.C, smem, stream));
+    }
 
     QlOutArgs oa;
     oa.partial = partial;
@@ -1032,9 +1412,16 @@ kronq_status run_qlinear(const QlinearArgs& q, void* ws, cudaStream_t stream) {
     oa.inv_sqrt_b = static_cast<float>(1.0 / std::sqrt(static_cast<double>(b_out)));
     oa.y = q.y + static_cast<int64_t>(t0) * q.ld_y;
     oa.ld_y = q.ld_y;
+    // threads per element: enough to give each at most about four segments, within 1024
+    // threads per CTA (qb * 16 elements)
+    const int64_t segs = (g.C + g.T - 1) / g.T + 1;     // partials per tile, at most
+    int tpe = 1;
+    while (tpe < 32 && tpe * 4 < segs && qb * 16 * tpe * 2 <= 1024) tpe *= 2;
+    oa.tpe = tpe;
     const dim3 ogrid(8 * (g.T / qb), nt);
-    KQ_TRY(launch_pdl(qlin_out_kernel, ogrid, dim3(std::min(1024, std::max(32, qb * 16))),
-                      out_smem, stream, true, "qlin_out_kernel", oa));
+    KQ_TRY(launch_pdl(qlin_out_kernel, ogrid,
+                      dim3(std::min(1024, std::max(32, qb * 16 * tpe))), out_smem, stream, true,
+                      "qlin_out_kernel", oa));
   }
   return KRONQ_OK;
 }

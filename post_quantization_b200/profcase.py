@@ -257,9 +257,32 @@ def case_qlinear(args):
     b.record()
     torch.cuda.synchronize()
     sweep_ms = a.elapsed_time(b) / args.reps
+    # the whole block in one graph (the layers' kernels chained back to back, as in a decode
+    # step); replayed with the other copies of the codes in between so that L2 starts cold
+    block_us = None
+    if not args.no_graphs:
+        gb = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gb):
+            for L in layers:
+                call(L)
+        for _ in range(3):
+            gb.replay()
+        torch.cuda.synchronize()
+        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+        tot = 0.0
+        for _ in range(args.reps):
+            flush.zero_()                      # 256 MB through L2
+            a.record()
+            gb.replay()
+            b.record()
+            b.synchronize()
+            tot += a.elapsed_time(b)
+        block_us = tot / args.reps * 1e3
+        del gb, flush
     print(json.dumps({"case": "qlinear", "bits": bits, "group": group, "tokens": n,
                       "layers": res, "sum_us": tot_ms * 1e3, "sweep_us": sweep_ms * 1e3,
-                      "sweep_GBps": tot_bytes / sweep_ms / 1e6,
+                      "sweep_GBps": tot_bytes / sweep_ms / 1e6, "block_graph_us": block_us,
+                      "block_graph_GBps": tot_bytes / block_us / 1e3 if block_us else None,
                       "launches": K.kronq_launch_count()}))
     del graphs
 
