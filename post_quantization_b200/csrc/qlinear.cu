@@ -199,8 +199,6 @@ __global__ void __launch_bounds__(1024) qlin_in_kernel(QlInArgs a) {
   extern __shared__ float xs[];
   auto at = [](int i) { return i + (i >> 4); };
   griddep_launch_dependents();
-  // x may be the output of the kernel before this one; the launch itself overlaps it
-  griddep_wait();
   const int tid = threadIdx.x;
   const int nthr = blockDim.x;
   const int nwork = a.span >> 4;                // threads that own 16 columns
@@ -209,23 +207,32 @@ __global__ void __launch_bounds__(1024) qlin_in_kernel(QlInArgs a) {
   const int len = min(a.span, a.d_in - j0);
   const bool rot = (a.flags & KRONQ_BIIP_ROTATE_IN) != 0;
   const bool scl = (a.flags & KRONQ_BIIP_SCALE_IN) != 0;
-  // at most 16 elements per thread (nthr >= span / 16): all loads issued before any is used
+  // at most 16 elements per thread (nthr >= span / 16): all loads issued before any is used;
+  // the layer's scales and signs while the preceding kernel still runs, x (which that kernel
+  // may have written) after waiting for it
   {
     float xv[16], sv[16];
     int8_t sg[16];
 #pragma unroll
     for (int m = 0; m < 16; ++m) {
       const int j = tid + m * nthr;
-      xv[m] = 0.f;
       sv[m] = 1.f;
       sg[m] = 1;
+      if (j < len) {
+        if (scl) sv[m] = a.s_x[j0 + j];
+        if (rot) sg[m] = a.sign_in[j0 + j];
+      }
+    }
+    griddep_wait();
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+      const int j = tid + m * nthr;
+      xv[m] = 0.f;
       if (j < len) {
         const int64_t o = static_cast<int64_t>(t) * a.ld_x + j0 + j;
         xv[m] = a.x_dtype == KRONQ_DTYPE_BF16
                     ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(a.x)[o])
                     : reinterpret_cast<const float*>(a.x)[o];
-        if (scl) sv[m] = a.s_x[j0 + j];
-        if (rot) sg[m] = a.sign_in[j0 + j];
       }
     }
 #pragma unroll
@@ -279,14 +286,24 @@ __global__ void __launch_bounds__(1024) qlin_in_kernel(QlInArgs a) {
     const uint32_t rank = cluster_ctarank();
     const uint32_t base = smem_u32(xs);
     cluster_sync_all();                         // every span of the block is transformed
-    for (int e = tid; e < a.span; e += nthr) {
-      const uint32_t off = static_cast<uint32_t>(at(e)) * 4u;
+    // all of a thread's remote loads (at most 4 elements x 8 spans) are issued before any sum
+    constexpr int EPT = 4;                      // elements per thread: nthr = span / 4
+    float z[EPT][8];
+#pragma unroll
+    for (int m = 0; m < EPT; ++m) {
+      const uint32_t off = static_cast<uint32_t>(at(tid + m * nthr)) * 4u;
+#pragma unroll
+      for (int r2 = 0; r2 < 8; ++r2)
+        z[m][r2] = r2 < a.cl ? ld_dsmem(map_shared_rank(base + off, static_cast<uint32_t>(r2)))
+                             : 0.f;
+    }
+#pragma unroll
+    for (int m = 0; m < EPT; ++m) {
       float v = 0.f;
-      for (int r2 = 0; r2 < a.cl; ++r2) {
-        const float z = ld_dsmem(map_shared_rank(base + off, static_cast<uint32_t>(r2)));
-        v += (__popc(rank & static_cast<uint32_t>(r2)) & 1) ? -z : z;
-      }
-      xo[at(e)] = v;
+#pragma unroll
+      for (int r2 = 0; r2 < 8; ++r2)
+        v += (__popc(rank & static_cast<uint32_t>(r2)) & 1) ? -z[m][r2] : z[m][r2];
+      xo[at(tid + m * nthr)] = v;
     }
     cluster_sync_all();                         // no CTA leaves while another still reads it
     xf = xo;
@@ -855,41 +872,45 @@ __device__ __forceinline__ void dp_unit(const DpCodes<BITS>& c, const uint8_t* x
     for (int k = 0; k < QL_TERMS; ++k)
 #pragma unroll
       for (int j = 0; j < 4; ++j) acc[t][k][j] = 0;
+  // 16 columns per step: the step's codes are masked once and used for every token and term
 #pragma unroll
-  for (int t = 0; t < NT; ++t) {
-    if (t >= n_tok) break;
+  for (int q = 0; q < 8; ++q) {
+    uint32_t cm[4];                               // four 4-column code words of the step
+    if (BITS == 2) {
+      // word q: columns 16q + 4k + j at bits 8j + 2k (code scaled by 4^k)
 #pragma unroll
-    for (int term = 0; term < QL_TERMS; ++term) {
-      const uint4* xr = reinterpret_cast<const uint4*>(xg + (3 * t + term) * 128);
+      for (int k = 0; k < 4; ++k) cm[k] = w[q] & (0x03030303u << (2 * k));
+    } else if (BITS == 4) {
+      // words 2q, 2q + 1: columns 8w + 4k + j at bits 8j + 4k (code scaled by 16^k)
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {                  // 16 columns per step
-        const uint4 xv = xr[q];                       // x' bytes of columns 16q .. 16q + 15
-        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-        if (BITS == 2) {
-          // word q: columns 16q + 4k + j at bits 8j + 2k
-          const uint32_t wd = w[q];
+      for (int h = 0; h < 2; ++h) {
+        cm[2 * h] = w[2 * q + h] & 0x0F0F0F0Fu;
+        cm[2 * h + 1] = w[2 * q + h] & 0xF0F0F0F0u;
+      }
+    } else {
+      // 32 columns per three words: low bits in words 3m, 3m + 1, top bits in word 3m + 2
+      const int m = q >> 1, half = q & 1;
+      const uint32_t wl = w[3 * m + half], wh = w[3 * m + 2];
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            acc[t][term][k] = dp4a_us(wd & (0x03030303u << (2 * k)), xw[k], acc[t][term][k]);
-        } else if (BITS == 4) {
-          // words 2q, 2q + 1: columns 8w + 4k + j at bits 8j + 4k
+      for (int k = 0; k < 4; ++k) {
+        const int k8 = 4 * half + k;
+        const uint32_t lo = (wl >> (2 * k)) & 0x03030303u;
+        const uint32_t hi = (k8 >= 2 ? (wh >> (k8 - 2)) : (wh << (2 - k8))) & 0x04040404u;
+        cm[k] = lo | hi;
+      }
+    }
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint32_t wd = w[2 * q + h];
-            acc[t][term][0] = dp4a_us(wd & 0x0F0F0F0Fu, xw[2 * h], acc[t][term][0]);
-            acc[t][term][1] = dp4a_us(wd & 0xF0F0F0F0u, xw[2 * h + 1], acc[t][term][1]);
-          }
-        } else {
-          // 32 columns per three words: low bits in words 3m, 3m + 1, top bits in word 3m + 2
-          const int m = q >> 1, half = q & 1;
-          const uint32_t wl = w[3 * m + half], wh = w[3 * m + 2];
+    for (int t = 0; t < NT; ++t) {
+      if (t >= n_tok) break;
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int k8 = 4 * half + k;
-            const uint32_t lo = (wl >> (2 * k)) & 0x03030303u;
-            const uint32_t hi = (k8 >= 2 ? (wh >> (k8 - 2)) : (wh << (2 - k8))) & 0x04040404u;
-            acc[t][term][0] = dp4a_us(lo | hi, xw[k], acc[t][term][0]);
-          }
+      for (int term = 0; term < QL_TERMS; ++term) {
+        const uint4 xv = reinterpret_cast<const uint4*>(xg + (3 * t + term) * 128)[q];
+        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};   // columns 16q + 4k .. + 3
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          // part: 2 bits -> k (factor 4^k); 4 bits -> k & 1 (factor 16^(k & 1)); 3 bits -> 0
+          const int part = BITS == 2 ? k : (BITS == 4 ? (k & 1) : 0);
+          acc[t][term][part] = dp4a_us(cm[k], xw[k], acc[t][term][part]);
         }
       }
     }
@@ -911,16 +932,25 @@ __global__ void __launch_bounds__(128, 4) qlin_dp4a_kernel(QlDpArgs p) {
   constexpr int D = BITS == 2 ? 4 : 2;                // units of codes in flight per thread
   const int64_t blob = 2048 * BITS;
   DpCodes<BITS> buf[D];
-  // the packed codes do not depend on the preceding kernel: load them before waiting
+  float2 gbuf[D];                                     // this row's grid for those units
+  // unit i's grid entry: (tile, group) of the unit for group-wise grids, tile for per-row
+  auto grid_of = [&](int64_t u) {
+    return __ldg(&p.grid[p.grouped ? u * QL_TILE + r : (u / p.G) * QL_TILE + r]);
+  };
+  // the packed codes and the grid do not depend on the preceding kernel: load them first
 #pragma unroll
   for (int d = 0; d < D; ++d)
-    if (d < n_units) dp_load<BITS>(p.packed + (u0 + d) * blob, r, buf[d]);
+    if (d < n_units) {
+      dp_load<BITS>(p.packed + (u0 + d) * blob, r, buf[d]);
+      gbuf[d] = grid_of(u0 + d);
+    }
   griddep_wait();                                     // x' and its sums come from qlin_in
   const int gb = 128 * p.rows;                         // bytes of one group's terms
   const bool all_groups = n_units >= p.G;
+  const int ng = all_groups ? p.G : n_units;
+  float2* sstage = reinterpret_cast<float2*>(xstage + ng * gb);   // (s, sum) per group, token
   {
     const int gstart = all_groups ? 0 : static_cast<int>(u0 % p.G);
-    const int ng = all_groups ? p.G : n_units;
     const int words = ng * gb / 16;
     for (int w = threadIdx.x; w < words; w += blockDim.x) {
       const int gi = w / (gb / 16), off = w % (gb / 16);
@@ -928,6 +958,11 @@ __global__ void __launch_bounds__(128, 4) qlin_dp4a_kernel(QlDpArgs p) {
       if (gsrc >= p.G) gsrc -= p.G;
       reinterpret_cast<uint4*>(xstage)[w] =
           __ldg(reinterpret_cast<const uint4*>(p.bop + static_cast<int64_t>(gsrc) * gb) + off);
+    }
+    for (int w = threadIdx.x; w < ng * p.n_tok; w += blockDim.x) {
+      int gsrc = gstart + w / p.n_tok;
+      if (gsrc >= p.G) gsrc -= p.G;
+      sstage[w] = __ldg(&p.sums[static_cast<int64_t>(gsrc) * p.n_tok + w % p.n_tok]);
     }
     __syncthreads();
   }
@@ -942,16 +977,18 @@ __global__ void __launch_bounds__(128, 4) qlin_dp4a_kernel(QlDpArgs p) {
       const int i = i0 + d;
       if (i >= n_units) break;
       const int row = tile * QL_TILE + r;
-      const float2 gz = __ldg(&p.grid[p.grouped
-                                          ? (static_cast<int64_t>(tile) * p.G + g) * QL_TILE + r
-                                          : static_cast<int64_t>(tile) * QL_TILE + r]);
+      const float2 gz = gbuf[d];
+      const int si = all_groups ? g : i;                // staged group index
       int acc[NT][QL_TERMS][4];
-      dp_unit<BITS, NT>(buf[d], xstage + (all_groups ? g : i) * gb, p.n_tok, acc);
-      if (i + D < n_units) dp_load<BITS>(p.packed + (u0 + i + D) * blob, r, buf[d]);
+      dp_unit<BITS, NT>(buf[d], xstage + si * gb, p.n_tok, acc);
+      if (i + D < n_units) {
+        dp_load<BITS>(p.packed + (u0 + i + D) * blob, r, buf[d]);
+        gbuf[d] = grid_of(u0 + i + D);
+      }
 #pragma unroll
       for (int t = 0; t < NT; ++t) {
         if (t >= p.n_tok) break;
-        const float2 sq = __ldg(&p.sums[static_cast<int64_t>(g) * p.n_tok + t]);
+        const float2 sq = sstage[si * p.n_tok + t];
         float a[QL_TERMS];
 #pragma unroll
         for (int term = 0; term < QL_TERMS; ++term) {
@@ -1364,7 +1401,8 @@ kronq_status run_qlinear(const QlinearArgs& q, void* ws, cudaStream_t stream) {
       dpa.b_tile = rot_out ? std::min(b_out, QL_TILE) : 1;
       dpa.U = g.U;
       const int64_t upc = (g.U + g.C - 1) / g.C;          // units of the largest CTA
-      const size_t dsmem = static_cast<size_t>(std::min<int64_t>(upc, g.G)) * 128 * dpa.rows;
+      const size_t dsmem = static_cast<size_t>(std::min<int64_t>(upc, g.G)) *
+                           (128 * dpa.rows + sizeof(float2) * nt);
       KQ_TRY(launch_dp(q.bits, nt, dpa, g.C, dsmem, stream));
     } else {
     QlMmaArgs p;
