@@ -524,6 +524,304 @@ __global__ void __launch_bounds__(2 << LOG2P) fwht_cols_reg_kernel(float* m, int
   cp_async_wait0();
 }
 
+// ---- tiled row pass (32 <= b <= 8192, 16-byte aligned operands) ----
+//
+// A chunk is RB = max(1, 4096 / b) matrix rows of one b-wide column band (one Hadamard block per
+// row), C = RB b = max(4096, b) elements, seen as C / 32 tile rows of 32: tile row r is matrix
+// row RB-row r / (b / 32), columns 32 (r % (b / 32)) .. + 31 of the band. Sylvester's H_b factors
+// over index bits, H_b = H_{b/32} (x) H_32, so the transform is a 32-point butterfly along every
+// tile row (index bits 0-4) and a (b/32)-point one down the tile columns inside each matrix row
+// (bits 5 and up). C / 32 threads; each holds 32 elements in every step:
+//   loads     TMA copies the chunk (a box of 32 x b/32 x RB) into one of several stages, up to
+//             stages - 1 chunks ahead, completion on the stage's mbarrier; rows past the matrix
+//             read as zeros
+//   row step  a thread takes one tile row: the scaling (row factor x column factors x scalar x
+//             1/sqrt(b); first, as the column factors differ inside a block), the five row bits
+//             in registers, then into the fp32 tile (in place for fp32 sources)
+//   rounds    a thread takes 2^m tile rows r0 + k 2^h0 (k < 2^m) of 32 / 2^m adjacent columns,
+//             so the lanes of a warp cover whole tile rows; butterflies on the low n bits of k.
+//             The last round stores to global memory, each tile row one 128-byte segment.
+// The CTAs take contiguous ranges of chunks ordered band by band, so a thread's 32 columns stay
+// the same from chunk to chunk and their factors stay in registers.
+// Shared layouts are XOR-swizzled so that eight lanes reading eight tile rows at one offset and
+// lanes reading along one tile row are both free of bank conflicts: 16-byte piece q of 128-byte
+// fp32 tile row r sits at q ^ (r % 8) (TMA's 128-byte swizzle), piece q of a 64-byte bf16 row at
+// q ^ ((r / 2) % 4) (TMA's 64-byte swizzle).
+template <int LOG2B, bool F32>
+struct RowTma {
+  static constexpr int kLog2S = LOG2B - 5;                        // log2 tile rows per matrix row
+  static constexpr int kSegs = 1 << kLog2S;
+  static constexpr int kRB = LOG2B >= 12 ? 1 : 1 << (12 - LOG2B);  // matrix rows per chunk
+  static constexpr int kLog2C = LOG2B > 12 ? LOG2B : 12;
+  static constexpr int kC = 1 << kLog2C;
+  static constexpr int kThreads = kC / 32;                         // = tile rows
+  static constexpr int kStages = (!F32 && kLog2C == 12) ? 4 : 3;
+  static constexpr int kStageBytes = kC * (F32 ? 4 : 2);
+  static constexpr int kWorkBytes = F32 ? 0 : kC * 4;              // bf16: separate fp32 tile
+  static constexpr int kMinBlocks = kLog2C == 12 ? 4 : 2;          // fits an SM's shared memory
+  static constexpr size_t kSmem = 1024 + static_cast<size_t>(kStages) * kStageBytes + kWorkBytes + 64;
+};
+
+__device__ __forceinline__ void fwht32(float (&x)[32]) {
+#pragma unroll
+  for (int h = 0; h < 5; ++h)
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      if (j & (1 << h)) continue;
+      const float a = x[j], b = x[j | (1 << h)];
+      x[j] = a + b;
+      x[j | (1 << h)] = a - b;
+    }
+}
+
+// float offset of 16-byte piece q of tile row r (128-byte rows, 128-byte swizzle)
+__device__ __forceinline__ int tpos(int r, int q) { return r * 32 + 4 * (q ^ (r & 7)); }
+
+// One round: tile rows r0 + (k << H0), k < 2^MLOG, butterflies on the low NB bits of k. The last
+// round writes tile row r to dst row (row0 + r / segs), columns col0 + 32 (r % segs) ..
+template <int H0, int MLOG, int NB, bool LAST, int LOG2S>
+__device__ __forceinline__ void tile_round(float* work, float* dst, int64_t rows, int64_t cols,
+                                           int64_t row0, int64_t col0, int t) {
+  constexpr int M = 1 << MLOG, W = 32 / M;
+  const int g = t & (M - 1), s = t >> MLOG;
+  const int r0 = (s & ((1 << H0) - 1)) | ((s >> H0) << (H0 + MLOG));
+  // float offset of this lane's W columns in tile row r
+  auto at = [&](int r) {
+    if constexpr (W == 4) return tpos(r, g);
+    else if constexpr (W == 2) return tpos(r, g >> 1) + 2 * (g & 1);
+    else return tpos(r, g >> 2) + (g & 3);
+  };
+  float y[M][W];
+#pragma unroll
+  for (int k = 0; k < M; ++k) {
+    const float* p = work + at(r0 + (k << H0));
+    if constexpr (W == 4) {
+      const float4 v = *reinterpret_cast<const float4*>(p);
+      y[k][0] = v.x; y[k][1] = v.y; y[k][2] = v.z; y[k][3] = v.w;
+    } else if constexpr (W == 2) {
+      const float2 v = *reinterpret_cast<const float2*>(p);
+      y[k][0] = v.x; y[k][1] = v.y;
+    } else {
+      y[k][0] = p[0];
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < NB; ++h)
+#pragma unroll
+    for (int k = 0; k < M; ++k) {
+      if (k & (1 << h)) continue;
+#pragma unroll
+      for (int e = 0; e < W; ++e) {
+        const float a = y[k][e], b = y[k | (1 << h)][e];
+        y[k][e] = a + b;
+        y[k | (1 << h)][e] = a - b;
+      }
+    }
+#pragma unroll
+  for (int k = 0; k < M; ++k) {
+    const int r = r0 + (k << H0);
+    float* p;
+    if constexpr (LAST) {
+      const int64_t row = row0 + (r >> LOG2S);
+      if (row >= rows) continue;
+      p = dst + row * cols + col0 + 32 * (r & ((1 << LOG2S) - 1)) + W * g;
+    } else {
+      p = work + at(r);
+    }
+    if constexpr (W == 4)
+      *reinterpret_cast<float4*>(p) = make_float4(y[k][0], y[k][1], y[k][2], y[k][3]);
+    else if constexpr (W == 2)
+      *reinterpret_cast<float2*>(p) = make_float2(y[k][0], y[k][1]);
+    else
+      p[0] = y[k][0];
+  }
+}
+
+// dst may be the source matrix itself (fp32): a chunk is loaded (by TMA, up to stages - 1 chunks
+// ahead) and written only by the CTA that owns it, load before store.
+template <typename T, int LOG2B>
+__global__ void __launch_bounds__(RowTma<LOG2B, sizeof(T) == 4>::kThreads,
+                                  RowTma<LOG2B, sizeof(T) == 4>::kMinBlocks)
+    fwht_rows_tma_kernel(const __grid_constant__ CUtensorMap src_map, float* dst, int64_t rows,
+                         int64_t cols, const float* __restrict__ row_f,
+                         const float* __restrict__ col_f, float scalar, float out_scale,
+                         int* err_word) {
+  constexpr bool kF32 = sizeof(T) == 4;
+  using S = RowTma<LOG2B, kF32>;
+  constexpr int L = LOG2B - 5, LOG2S = S::kLog2S, NST = S::kStages;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  unsigned char* stages = sm;
+  float* work_bf = reinterpret_cast<float*>(sm + NST * S::kStageBytes);   // bf16 sources only
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + NST * S::kStageBytes + S::kWorkBytes);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(full + NST);
+  const int t = threadIdx.x;
+
+  const int64_t nrg = (rows + S::kRB - 1) / S::kRB;        // row groups per band
+  const int64_t nchunks = (cols >> LOG2B) * nrg;
+  const int64_t k0 = nchunks * blockIdx.x / gridDim.x;
+  const int64_t k1 = nchunks * (blockIdx.x + 1) / gridDim.x;
+  const int n = static_cast<int>(k1 - k0);
+  if (n <= 0) return;
+
+  if (t == 0) {
+    prefetch_tensormap(&src_map);
+    for (int i = 0; i < NST; ++i) mbar_init(&full[i], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  // chunk k0 + j: band, row group
+  auto issue = [&](int j) {
+    const int64_t k = k0 + j;
+    const int64_t band = k / nrg, rg = k - band * nrg;
+    uint64_t* bar = &full[j % NST];
+    mbar_arrive_expect_tx(bar, S::kStageBytes);
+    tma_load_3d(stages + (j % NST) * S::kStageBytes, &src_map, bar, 0,
+                static_cast<int32_t>(band << LOG2S), static_cast<int32_t>(rg * S::kRB));
+  };
+  if (t == 0)
+    for (int j = 0; j < NST - 1 && j < n; ++j) issue(j);
+
+  const int rr = t >> LOG2S, seg = t & (S::kSegs - 1);    // row step: matrix row, segment
+  int64_t band = k0 / nrg, rg = k0 - band * nrg;
+  int64_t cf_band = -1;
+  float cf[32];
+  bool aborted = false;
+  int i = 0;
+  for (; i < n; ++i) {
+    const int st = i % NST;
+    if (t == 0 && i + NST - 1 < n) issue(i + NST - 1);   // its stage was freed by chunk i - 1
+    const int64_t row0 = rg * S::kRB, col0 = band << LOG2B;
+    const int64_t row = row0 + rr;
+    const float rf = (row_f && row < rows) ? row_f[row] : 1.f;
+    if (band != cf_band) {   // column factors x scalar x 1/sqrt(b) of this thread's 32 columns
+      const float sc = scalar * out_scale;
+      if (col_f) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 v = *reinterpret_cast<const float4*>(col_f + col0 + 32 * seg + 4 * q);
+          cf[4 * q] = v.x * sc; cf[4 * q + 1] = v.y * sc; cf[4 * q + 2] = v.z * sc;
+          cf[4 * q + 3] = v.w * sc;
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < 32; ++k) cf[k] = sc;
+      }
+      cf_band = band;
+    }
+    const bool ok = mbar_wait(&full[st], (i / NST) & 1, abort_flag, err_word, DEV_ERR_LOAD_WAIT);
+    float* work = kF32 ? reinterpret_cast<float*>(stages + st * S::kStageBytes) : work_bf;
+    if (ok) {
+      float x[32];
+      if constexpr (kF32) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 v = *reinterpret_cast<const float4*>(work + tpos(t, q));
+          x[4 * q] = v.x; x[4 * q + 1] = v.y; x[4 * q + 2] = v.z; x[4 * q + 3] = v.w;
+        }
+      } else {
+        const T* sg = reinterpret_cast<const T*>(stages + st * S::kStageBytes) + 32 * t;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 v = *reinterpret_cast<const uint4*>(sg + 8 * (q ^ ((t >> 1) & 3)));
+          const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            x[8 * q + 2 * e] = __uint_as_float(u[e] << 16);
+            x[8 * q + 2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
+          }
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 32; ++k) x[k] *= rf * cf[k];
+      fwht32(x);
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        *reinterpret_cast<float4*>(work + tpos(t, q)) =
+            make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+    }
+    if (__syncthreads_or(!ok)) {
+      aborted = true;
+      break;
+    }
+    // rounds over the index bits above the tile row; a round of MLOG bits needs h0 + MLOG <=
+    // log2 of the tile rows (7 for C = 4096, 8 for C = 8192)
+    if constexpr (L == 0) {
+      tile_round<0, 3, 0, true, LOG2S>(work, dst, rows, cols, row0, col0, t);
+    } else if constexpr (L <= 3) {
+      tile_round<0, 3, L, true, LOG2S>(work, dst, rows, cols, row0, col0, t);
+    } else if constexpr (L == 4 || L == 5) {
+      tile_round<0, L, L, true, LOG2S>(work, dst, rows, cols, row0, col0, t);
+    } else if constexpr (L == 6) {
+      tile_round<0, 3, 3, false, LOG2S>(work, dst, rows, cols, row0, col0, t);
+      __syncthreads();
+      tile_round<3, 3, 3, true, LOG2S>(work, dst, rows, cols, row0, col0, t);
+    } else if constexpr (L == 7) {
+      tile_round<0, 3, 3, false, LOG2S>(work, dst, rows, cols, row0, col0, t);
+      __syncthreads();
+      tile_round<3, 4, 4, true, LOG2S>(work, dst, rows, cols, row0, col0, t);
+    } else {
+      static_assert(L == 8, "tiled row pass covers 32 <= b <= 8192");
+      tile_round<0, 4, 4, false, LOG2S>(work, dst, rows, cols, row0, col0, t);
+      __syncthreads();
+      tile_round<4, 4, 4, true, LOG2S>(work, dst, rows, cols, row0, col0, t);
+    }
+    if constexpr (kF32) fence_proxy_async_smem();   // the stage was written in place; TMA refills it
+    __syncthreads();
+    if (++rg == nrg) {
+      rg = 0;
+      ++band;
+    }
+  }
+  if (aborted && t == 0) {
+    // let the loads already issued (chunks i .. i + stages - 2) land before the CTA exits
+    for (int j = i; j < n && j < i + NST - 1; ++j)
+      mbar_drain(&full[j % NST], (j / NST) & 1, kWaitLimitNs);
+  }
+}
+
+template <typename T>
+kronq_status row_pass_tile(const T* src, float* dst, int64_t rows, int64_t cols,
+                           const float* row_f, const float* col_f, float scalar, int log2b,
+                           float out_scale, cudaStream_t stream) {
+  constexpr bool kF32 = sizeof(T) == 4;
+  CUtensorMap map;
+  const uint64_t dims[3] = {32, static_cast<uint64_t>(cols / 32), static_cast<uint64_t>(rows)};
+  const uint64_t strides[2] = {32 * sizeof(T), static_cast<uint64_t>(cols) * sizeof(T)};
+  const int b = 1 << log2b;
+  const uint32_t box[3] = {32, static_cast<uint32_t>(b / 32),
+                           static_cast<uint32_t>(log2b >= 12 ? 1 : 4096 / b)};
+  KQ_TRY(encode_tiled_map(&map, kF32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                          3, src, dims, strides, box,
+                          kF32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B));
+  int* err = device_error_word();
+  const int64_t rb = log2b >= 12 ? 1 : 4096 / b;
+  const int64_t nchunks = (cols / b) * ((rows + rb - 1) / rb);
+  auto launch = [&](auto kern, int nt, size_t smem) -> kronq_status {
+    KQ_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(smem)));
+    int per_sm = 1;   // the CTAs that fit at once; each takes a contiguous range of chunks
+    KQ_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, nt, smem));
+    if (per_sm < 1) per_sm = 1;
+    const int64_t cap = static_cast<int64_t>(sm_budget()) * per_sm;
+    const unsigned grid = static_cast<unsigned>(nchunks < cap ? nchunks : cap);
+    kern<<<grid, nt, smem, stream>>>(map, dst, rows, cols, row_f, col_f, scalar, out_scale, err);
+    return check_launch("fwht_rows_tma_kernel");
+  };
+#define KQ_ROW_TMA(LB)                                                      \
+  case LB:                                                                  \
+    return launch(fwht_rows_tma_kernel<T, LB>, RowTma<LB, kF32>::kThreads, \
+                  RowTma<LB, kF32>::kSmem);
+  switch (log2b) {
+    KQ_ROW_TMA(5) KQ_ROW_TMA(6) KQ_ROW_TMA(7) KQ_ROW_TMA(8) KQ_ROW_TMA(9)
+    KQ_ROW_TMA(10) KQ_ROW_TMA(11) KQ_ROW_TMA(12) KQ_ROW_TMA(13)
+    default: return fail(KRONQ_ERR_UNSUPPORTED, "tiled row pass: block size out of range");
+  }
+#undef KQ_ROW_TMA
+}
+
 int ilog2_pow2(int b) {
   int l = 0;
   while ((1 << l) < b) ++l;
@@ -539,6 +837,11 @@ kronq_status row_pass(const T* src, float* dst, int64_t rows, int64_t cols, cons
   const int64_t total = rows * cols;
   const int64_t blocks = (total + chunk - 1) / chunk;
   const float out_scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(b)));
+  const bool aligned = (reinterpret_cast<uintptr_t>(src) & 15u) == 0 &&
+                       (reinterpret_cast<uintptr_t>(dst) & 15u) == 0;
+  if (aligned && b >= 32 && b <= 8192 && rows < (int64_t(1) << 31))
+    return row_pass_tile(src, dst, rows, cols, row_f, col_f, scalar, ilog2_pow2(b), out_scale,
+                         stream);
   if (b >= 16 && b <= 16384) {
     const int threads = chunk / 16;
     // padded work buffer + two staging buffers of the source type

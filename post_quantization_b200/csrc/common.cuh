@@ -31,6 +31,12 @@ kronq_status check_launch(const char* what);
     if (s_ != KRONQ_OK) return s_;          \
   } while (0)
 
+// Tiled tensor map (zero fill out of bounds, 256-byte L2 promotion). dims[0] is the contiguous
+// dimension; strides[i] is the byte stride of dimension i + 1 (rank - 1 entries).
+kronq_status encode_tiled_map(CUtensorMap* map, CUtensorMapDataType dtype, int rank,
+                              const void* base, const uint64_t* dims, const uint64_t* strides,
+                              const uint32_t* box, CUtensorMapSwizzle swizzle);
+
 // Device-side error word: kernels that give up a bounded wait record a code here.
 int* device_error_word();   // device address of the word (current device)
 // SMs that persistent kernels may size their grids to: the device's SM count, or less while
@@ -43,6 +49,7 @@ enum DeviceError : int {
   DEV_ERR_TMA_WAIT = 1,     // producer waited too long for a free pipeline stage
   DEV_ERR_MMA_WAIT = 2,     // MMA issuer waited too long for operands or an accumulator
   DEV_ERR_EPI_WAIT = 3,     // epilogue waited too long for an accumulator
+  DEV_ERR_LOAD_WAIT = 4,    // a streaming pass waited too long for a tile load
 };
 
 // ---------------------------------------------------------------------------------------------
@@ -129,6 +136,22 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
+}
+
+// 3-D tiled TMA load global -> shared (this CTA), completion signalled on `bar` (no multicast).
+__device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
+                                            int32_t x, int32_t y, int32_t z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Orders this thread's generic-proxy shared-memory writes before later async-proxy (TMA)
+// accesses of the same bytes.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {

@@ -165,6 +165,26 @@ def test_biip_matches_oracle(K, P, flags, shape, w_dtype):
         assert torch.equal(hg_in, hg)          # read-only without WRITE_HG
 
 
+@pytest.mark.parametrize("d_out,d_in", [(24, 96), (40, 192), (9, 640), (7, 1536), (5, 1024),
+                                        (3, 6144), (33, 4096)])
+@pytest.mark.parametrize("w_dtype", [torch.float32, torch.bfloat16])
+def test_biip_row_block_sizes(K, P, d_out, d_in, w_dtype):
+    # every input Hadamard block size of the row pass's tiled kernel (b = 32 .. 4096), with
+    # chunks of W that end part-way (d_out * d_in not a multiple of the 4096-element chunk)
+    n = 256
+    xq, xfp, g, w, si, so = layer_inputs(d_out, d_in, n, w_dtype=w_dtype,
+                                         tag=("biip-b", d_out, d_in))
+    hx, hg, dxx = gpu_sums(K, xq, xfp, g)
+    hg_in = hg.clone()
+    r = run_biip(K, P, w, hx, hg_in, dxx, 1.0 / n, si, so, 15 | 16)
+    o = O.biip(h64(w), h64(hx), h64(hg), h64(dxx), 1.0 / n, h64(si), h64(so), 15)
+    assert rel(h64(r.w_prime), o["w"]) <= TOL
+    assert rel(h64(r.hx), o["hx"]) <= TOL
+    assert rel(h64(r.dxx), o["dxx"]) <= TOL
+    assert rel(h64(hg_in), o["hg"]) <= TOL
+    assert K.kronq_device_error() == 0
+
+
 def test_biip_llama_gate_shape(K, P):
     # gate_proj of LLaMA-2-7B: 11008 x 4096 (output Hadamard blocks of 256, input 4096)
     d_out, d_in, n = 11008, 4096, 4096
