@@ -27,8 +27,7 @@ namespace kq {
 
 namespace {
 
-constexpr int kNormRows = 64;
-constexpr int kNormCols = 256;
+constexpr int kNormRows = 256;   // rows per CTA of the norms pass
 
 template <typename T>
 __device__ __forceinline__ float load_as_float(const T* p, int64_t i);
@@ -41,35 +40,77 @@ __device__ __forceinline__ float load_as_float<__nv_bfloat16>(const __nv_bfloat1
   return __bfloat162float(p[i]);
 }
 
-// Partial squared column and row norms of a 64 x 256 tile, added into fp64 accumulators.
+// Squared column and row norms of a contiguous rows x cols W, added into fp64 accumulators. A CTA
+// takes a panel of 32 V columns (V elements = one 16-byte load per lane) and kNormRows rows; warp
+// w takes rows w, w + 8, .. of it. Per row the warp sums its lanes' squares with five shuffles
+// and one lane adds the row's panel sum; per column the lanes keep running sums, which the 8
+// warps combine in shared memory at the end, one addition per column and CTA.
 template <typename T>
-__global__ void __launch_bounds__(256) colrow_norms_kernel(const T* __restrict__ w, int rows,
-                                                           int cols, double* __restrict__ col_sq,
+__global__ void __launch_bounds__(256, 3) colrow_norms_kernel(const T* __restrict__ w, int rows,
+                                                           int cols, int vec,
+                                                           double* __restrict__ col_sq,
                                                            double* __restrict__ row_sq) {
-  __shared__ float part[8][kNormRows];
-  const int c = blockIdx.x * kNormCols + threadIdx.x;
+  constexpr int V = 16 / sizeof(T);
+  constexpr int PW = 32 * V;   // panel width
+  __shared__ float part[8][PW];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int c0 = blockIdx.x * PW + lane * V;
   const int r0 = blockIdx.y * kNormRows;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float colacc = 0.f;
-  for (int r = 0; r < kNormRows; ++r) {
-    const int row = r0 + r;
-    float v = 0.f;
-    if (row < rows && c < cols) v = load_as_float(w, static_cast<int64_t>(row) * cols + c);
-    const float sq = v * v;
-    colacc += sq;
-    float rs = sq;
+  const int r1 = rows - r0 < kNormRows ? rows : r0 + kNormRows;
+  const bool whole = vec && c0 + V <= cols;   // one aligned 16-byte load
+  float colacc[V];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) rs += __shfl_xor_sync(0xffffffffu, rs, o);
-    if (lane == 0) part[warp][r] = rs;
+  for (int e = 0; e < V; ++e) colacc[e] = 0.f;
+  // batches of 8 rows per warp, their loads issued together
+  for (int rb = r0 + warp; rb < r1; rb += 64) {
+    uint4 u[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int r = rb + 8 * j;
+      if (whole && r < r1)
+        u[j] = *reinterpret_cast<const uint4*>(w + static_cast<int64_t>(r) * cols + c0);
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int r = rb + 8 * j;
+      if (r >= r1) break;
+      float v[V];
+      if (whole) {
+        const uint32_t q[4] = {u[j].x, u[j].y, u[j].z, u[j].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if constexpr (V == 8) {
+            v[2 * e] = __uint_as_float(q[e] << 16);
+            v[2 * e + 1] = __uint_as_float(q[e] & 0xFFFF0000u);
+          } else {
+            v[e] = __uint_as_float(q[e]);
+          }
+        }
+      } else {
+        const T* p = w + static_cast<int64_t>(r) * cols + c0;
+#pragma unroll
+        for (int e = 0; e < V; ++e) v[e] = c0 + e < cols ? load_as_float(p, e) : 0.f;
+      }
+      float sq = 0.f;
+#pragma unroll
+      for (int e = 0; e < V; ++e) {
+        colacc[e] = fmaf(v[e], v[e], colacc[e]);
+        sq = fmaf(v[e], v[e], sq);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+      if (lane == 0) atomicAdd(&row_sq[r], static_cast<double>(sq));
+    }
   }
-  if (c < cols) atomicAdd(&col_sq[c], static_cast<double>(colacc));
-  __syncthreads();
-  if (threadIdx.x < kNormRows) {
-    const int row = r0 + threadIdx.x;
-    float s = 0.f;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) s += part[k][threadIdx.x];
-    if (row < rows) atomicAdd(&row_sq[row], static_cast<double>(s));
+  for (int e = 0; e < V; ++e) part[warp][lane * V + e] = colacc[e];
+  __syncthreads();
+  for (int c = threadIdx.x; c < PW; c += blockDim.x) {
+    float sum = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) sum += part[k][c];
+    const int col = blockIdx.x * PW + c;
+    if (col < cols) atomicAdd(&col_sq[col], static_cast<double>(sum));
   }
 }
 
@@ -103,6 +144,7 @@ __global__ void side_trace_kernel(int d, const float* __restrict__ h, const doub
                                   double inv_n, int do_scale, double* __restrict__ tr) {
   __shared__ double red[32];
   double acc = 0.0;
+#pragma unroll 8
   for (int i = threadIdx.x; i < d; i += blockDim.x) {
     const double hii = static_cast<double>(h[static_cast<int64_t>(i) * d + i]) * inv_n;
     double s = 1.0;
@@ -578,10 +620,10 @@ __device__ __forceinline__ void fwht32(float (&x)[32]) {
 __device__ __forceinline__ int tpos(int r, int q) { return r * 32 + 4 * (q ^ (r & 7)); }
 
 // One round: tile rows r0 + (k << H0), k < 2^MLOG, butterflies on the low NB bits of k. The last
-// round writes tile row r to dst row (row0 + r / segs), columns col0 + 32 (r % segs) ..
-template <int H0, int MLOG, int NB, bool LAST, int LOG2S>
-__device__ __forceinline__ void tile_round(float* work, float* dst, int64_t rows, int64_t cols,
-                                           int64_t row0, int64_t col0, int t) {
+// round stores tile row r's W columns at out(r, column offset) (skipped where that is null),
+// times `scale`; the others write back to the tile.
+template <int H0, int MLOG, int NB, bool LAST, typename Out>
+__device__ __forceinline__ void tile_round(float* work, int t, float scale, const Out& out) {
   constexpr int M = 1 << MLOG, W = 32 / M;
   const int g = t & (M - 1), s = t >> MLOG;
   const int r0 = (s & ((1 << H0) - 1)) | ((s >> H0) << (H0 + MLOG));
@@ -622,9 +664,10 @@ __device__ __forceinline__ void tile_round(float* work, float* dst, int64_t rows
     const int r = r0 + (k << H0);
     float* p;
     if constexpr (LAST) {
-      const int64_t row = row0 + (r >> LOG2S);
-      if (row >= rows) continue;
-      p = dst + row * cols + col0 + 32 * (r & ((1 << LOG2S) - 1)) + W * g;
+      p = out(r, W * g);
+      if (!p) continue;
+#pragma unroll
+      for (int e = 0; e < W; ++e) y[k][e] *= scale;
     } else {
       p = work + at(r);
     }
@@ -634,6 +677,32 @@ __device__ __forceinline__ void tile_round(float* work, float* dst, int64_t rows
       *reinterpret_cast<float2*>(p) = make_float2(y[k][0], y[k][1]);
     else
       p[0] = y[k][0];
+  }
+}
+
+// Butterflies on the low L bits of the tile-row index (L <= log2 of the tile rows, at least 7),
+// in one or two rounds; a round of m bits starting at bit h0 needs h0 + m <= log2 tile rows.
+template <int L, typename Out>
+__device__ __forceinline__ void tile_rounds(float* work, int t, float scale, const Out& out) {
+  if constexpr (L == 0) {
+    tile_round<0, 3, 0, true>(work, t, scale, out);
+  } else if constexpr (L <= 3) {
+    tile_round<0, 3, L, true>(work, t, scale, out);
+  } else if constexpr (L == 4 || L == 5) {
+    tile_round<0, L, L, true>(work, t, scale, out);
+  } else if constexpr (L == 6) {
+    tile_round<0, 3, 3, false>(work, t, scale, out);
+    __syncthreads();
+    tile_round<3, 3, 3, true>(work, t, scale, out);
+  } else if constexpr (L == 7) {
+    tile_round<0, 3, 3, false>(work, t, scale, out);
+    __syncthreads();
+    tile_round<3, 4, 4, true>(work, t, scale, out);
+  } else {
+    static_assert(L == 8, "tile rounds cover up to 8 index bits");
+    tile_round<0, 4, 4, false>(work, t, scale, out);
+    __syncthreads();
+    tile_round<4, 4, 4, true>(work, t, scale, out);
   }
 }
 
@@ -746,28 +815,12 @@ __global__ void __launch_bounds__(RowTma<LOG2B, sizeof(T) == 4>::kThreads,
       aborted = true;
       break;
     }
-    // rounds over the index bits above the tile row; a round of MLOG bits needs h0 + MLOG <=
-    // log2 of the tile rows (7 for C = 4096, 8 for C = 8192)
-    if constexpr (L == 0) {
-      tile_round<0, 3, 0, true, LOG2S>(work, dst, rows, cols, row0, col0, t);
-    } else if constexpr (L <= 3) {
-      tile_round<0, 3, L, true, LOG2S>(work, dst, rows, cols, row0, col0, t);
-    } else if constexpr (L == 4 || L == 5) {
-      tile_round<0, L, L, true, LOG2S>(work, dst, rows, cols, row0, col0, t);
-    } else if constexpr (L == 6) {
-      tile_round<0, 3, 3, false, LOG2S>(work, dst, rows, cols, row0, col0, t);
-      __syncthreads();
-      tile_round<3, 3, 3, true, LOG2S>(work, dst, rows, cols, row0, col0, t);
-    } else if constexpr (L == 7) {
-      tile_round<0, 3, 3, false, LOG2S>(work, dst, rows, cols, row0, col0, t);
-      __syncthreads();
-      tile_round<3, 4, 4, true, LOG2S>(work, dst, rows, cols, row0, col0, t);
-    } else {
-      static_assert(L == 8, "tiled row pass covers 32 <= b <= 8192");
-      tile_round<0, 4, 4, false, LOG2S>(work, dst, rows, cols, row0, col0, t);
-      __syncthreads();
-      tile_round<4, 4, 4, true, LOG2S>(work, dst, rows, cols, row0, col0, t);
-    }
+    // the index bits above the tile row; the last round writes tile row r to matrix row
+    // row0 + r / segs, columns col0 + 32 (r % segs) ..
+    tile_rounds<L>(work, t, 1.0f, [&](int r, int c) -> float* {
+      const int64_t row = row0 + (r >> LOG2S);
+      return row < rows ? dst + row * cols + col0 + 32 * (r & (S::kSegs - 1)) + c : nullptr;
+    });
     if constexpr (kF32) fence_proxy_async_smem();   // the stage was written in place; TMA refills it
     __syncthreads();
     if (++rg == nrg) {
@@ -820,6 +873,140 @@ kronq_status row_pass_tile(const T* src, float* dst, int64_t rows, int64_t cols,
     default: return fail(KRONQ_ERR_UNSUPPORTED, "tiled row pass: block size out of range");
   }
 #undef KQ_ROW_TMA
+}
+
+// ---- tiled column pass (P = 16 .. 256 rows at stride rs, in place) ----
+//
+// A chunk is CT = max(1, 128 / P) adjacent 32-column tiles of the P rows r_base + rs j (j < P):
+// CT TMA boxes of 32 x P from the view {cols, rs, rows / rs} of the matrix, stacked so that tile
+// row ct P + j holds row j of column tile ct. The P-point butterflies run on the low log2 P bits
+// of the tile-row index with the rounds of the row pass; the last one scales by out_scale and
+// stores each tile row as one 128-byte segment. Columns past the matrix read as zeros and are not
+// stored. Same pipeline as the row pass: CTAs take contiguous ranges of chunks (column groups of
+// one row block, then the next row block), loads run up to stages - 1 chunks ahead.
+template <int LP>
+struct ColTma {
+  static constexpr int kP = 1 << LP;
+  static constexpr int kCT = LP >= 7 ? 1 : 1 << (7 - LP);   // column tiles per chunk
+  static constexpr int kThreads = kCT * kP;                  // = tile rows
+  static constexpr int kStages = 3;
+  static constexpr int kStageBytes = kThreads * 128;
+  static constexpr int kMinBlocks = LP == 8 ? 2 : 4;         // fits an SM's shared memory
+  static constexpr size_t kSmem = 1024 + static_cast<size_t>(kStages) * kStageBytes + 64;
+};
+
+template <int LP>
+__global__ void __launch_bounds__(ColTma<LP>::kThreads, ColTma<LP>::kMinBlocks)
+    fwht_cols_tma_kernel(const __grid_constant__ CUtensorMap map, float* m, int64_t rows,
+                         int64_t cols, int rs, float out_scale, int* err_word) {
+  using S = ColTma<LP>;
+  constexpr int P = S::kP, CT = S::kCT, NST = S::kStages;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* stages = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(stages + NST * S::kStageBytes);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(full + NST);
+  const int t = threadIdx.x;
+
+  const int ntiles = static_cast<int>((cols + 31) / 32);
+  const int ncg = (ntiles + CT - 1) / CT;                  // column groups per row block
+  const int64_t nchunks = (rows / P) * ncg;
+  const int64_t k0 = nchunks * blockIdx.x / gridDim.x;
+  const int64_t k1 = nchunks * (blockIdx.x + 1) / gridDim.x;
+  const int n = static_cast<int>(k1 - k0);
+  if (n <= 0) return;
+
+  if (t == 0) {
+    prefetch_tensormap(&map);
+    for (int i = 0; i < NST; ++i) mbar_init(&full[i], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  // chunk k0 + j: row block y (rows (y / rs) P rs + (y % rs) + rs j), column group cg
+  auto issue = [&](int j) {
+    const int64_t k = k0 + j;
+    const int64_t y = k / ncg;
+    const int cg = static_cast<int>(k - y * ncg);
+    const int a = static_cast<int>(y % rs);
+    const int z = static_cast<int>((y / rs) * P);
+    const int nt = ntiles - cg * CT < CT ? ntiles - cg * CT : CT;
+    uint64_t* bar = &full[j % NST];
+    unsigned char* dst = stages + (j % NST) * S::kStageBytes;
+    mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nt) * P * 128);
+    for (int ct = 0; ct < nt; ++ct)
+      tma_load_3d(dst + ct * P * 128, &map, bar, (cg * CT + ct) * 32, a, z);
+  };
+  if (t == 0)
+    for (int j = 0; j < NST - 1 && j < n; ++j) issue(j);
+
+  int64_t y = k0 / ncg;
+  int cg = static_cast<int>(k0 - y * ncg);
+  bool aborted = false;
+  int i = 0;
+  for (; i < n; ++i) {
+    const int st = i % NST;
+    if (t == 0 && i + NST - 1 < n) issue(i + NST - 1);   // its stage was freed by chunk i - 1
+    const bool ok = mbar_wait(&full[st], (i / NST) & 1, abort_flag, err_word, DEV_ERR_LOAD_WAIT);
+    if (__syncthreads_or(!ok)) {
+      aborted = true;
+      break;
+    }
+    float* work = reinterpret_cast<float*>(stages + st * S::kStageBytes);
+    const int64_t rbase = (y / rs) * P * rs + (y % rs);
+    const int64_t c0 = static_cast<int64_t>(cg) * CT * 32;
+    tile_rounds<LP>(work, t, out_scale, [&](int r, int c) -> float* {
+      const int64_t col = c0 + 32 * (r >> LP) + c;
+      return col < cols ? m + (rbase + static_cast<int64_t>(rs) * (r & (P - 1))) * cols + col
+                        : nullptr;
+    });
+    fence_proxy_async_smem();   // the stage was written in place; TMA refills it
+    __syncthreads();
+    if (++cg == ncg) {
+      cg = 0;
+      ++y;
+    }
+  }
+  if (aborted && t == 0) {
+    for (int j = i; j < n && j < i + NST - 1; ++j)
+      mbar_drain(&full[j % NST], (j / NST) & 1, kWaitLimitNs);
+  }
+}
+
+kronq_status col_pass_tma(float* m, int64_t rows, int64_t cols, int log2p, int rs, float out_scale,
+                          cudaStream_t stream) {
+  CUtensorMap map;
+  const uint64_t dims[3] = {static_cast<uint64_t>(cols), static_cast<uint64_t>(rs),
+                            static_cast<uint64_t>(rows / rs)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(cols) * 4,
+                               static_cast<uint64_t>(cols) * 4 * rs};
+  const uint32_t box[3] = {32, 1, static_cast<uint32_t>(1 << log2p)};
+  KQ_TRY(encode_tiled_map(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, m, dims, strides, box,
+                          CU_TENSOR_MAP_SWIZZLE_128B));
+  int* err = device_error_word();
+  const int P = 1 << log2p;
+  const int ct = log2p >= 7 ? 1 : 1 << (7 - log2p);
+  const int64_t ncg = ((cols + 31) / 32 + ct - 1) / ct;
+  const int64_t nchunks = (rows / P) * ncg;
+  auto launch = [&](auto kern, int nt, size_t smem) -> kronq_status {
+    KQ_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(smem)));
+    int per_sm = 1;   // the CTAs that fit at once; each takes a contiguous range of chunks
+    KQ_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, nt, smem));
+    if (per_sm < 1) per_sm = 1;
+    const int64_t cap = static_cast<int64_t>(sm_budget()) * per_sm;
+    const unsigned grid = static_cast<unsigned>(nchunks < cap ? nchunks : cap);
+    kern<<<grid, nt, smem, stream>>>(map, m, rows, cols, rs, out_scale, err);
+    return check_launch("fwht_cols_tma_kernel");
+  };
+#define KQ_COL_TMA(LPV) \
+  case LPV:             \
+    return launch(fwht_cols_tma_kernel<LPV>, ColTma<LPV>::kThreads, ColTma<LPV>::kSmem);
+  switch (log2p) {
+    KQ_COL_TMA(4) KQ_COL_TMA(5) KQ_COL_TMA(6) KQ_COL_TMA(7) KQ_COL_TMA(8)
+    default: return fail(KRONQ_ERR_UNSUPPORTED, "tiled column pass: block size out of range");
+  }
+#undef KQ_COL_TMA
 }
 
 int ilog2_pow2(int b) {
@@ -918,10 +1105,18 @@ kronq_status col_pass(float* m, int64_t rows, int64_t cols, int b, cudaStream_t 
   const float out_scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(b)));
   if (b >= 16 && b <= 16384) {
     const int L = ilog2_pow2(b);
-    if (L <= 8) return col_pass_reg(m, rows, cols, L, 1, out_scale, stream);
+    // TMA needs a 16-byte aligned base and row stride and row indices below 2^31; its boxes
+    // are 32 columns wide
+    const bool tma = (reinterpret_cast<uintptr_t>(m) & 15u) == 0 && cols % 4 == 0 &&
+                     cols >= 32 && rows < (int64_t(1) << 31);
+    auto pass = [&](int lp, int rs, float sc) {
+      return tma ? col_pass_tma(m, rows, cols, lp, rs, sc, stream)
+                 : col_pass_reg(m, rows, cols, lp, rs, sc, stream);
+    };
+    if (L <= 8) return pass(L, 1, out_scale);
     const int l1 = (L + 1) / 2, l2 = L / 2;   // H_b = (H_P2 (x) I_P1)(I_P2 (x) H_P1)
-    KQ_TRY(col_pass_reg(m, rows, cols, l1, 1, 1.0f, stream));
-    return col_pass_reg(m, rows, cols, l2, 1 << l1, out_scale, stream);
+    KQ_TRY(pass(l1, 1, 1.0f));
+    return pass(l2, 1 << l1, out_scale);
   }
   int cw = 32768 / b;
   if (cw > 64) cw = 64;
@@ -982,13 +1177,16 @@ kronq_status run_biip(const BiipArgs& a, void* ws_raw, cudaStream_t stream) {
   KQ_CUDA_TRY(cudaMemsetAsync(ws.col_sq, 0, sizeof(double) * a.d_in, stream));
   KQ_CUDA_TRY(cudaMemsetAsync(ws.row_sq, 0, sizeof(double) * a.d_out, stream));
   {
-    dim3 grid((a.d_in + kNormCols - 1) / kNormCols, (a.d_out + kNormRows - 1) / kNormRows);
-    if (a.w_dtype == KRONQ_DTYPE_BF16)
+    const bool bf = a.w_dtype == KRONQ_DTYPE_BF16;
+    const int esz = bf ? 2 : 4, pw = 32 * (16 / esz);
+    const int vec = (reinterpret_cast<uintptr_t>(a.w) & 15u) == 0 && (a.d_in * esz) % 16 == 0;
+    dim3 grid((a.d_in + pw - 1) / pw, (a.d_out + kNormRows - 1) / kNormRows);
+    if (bf)
       colrow_norms_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
-          static_cast<const __nv_bfloat16*>(a.w), a.d_out, a.d_in, ws.col_sq, ws.row_sq);
+          static_cast<const __nv_bfloat16*>(a.w), a.d_out, a.d_in, vec, ws.col_sq, ws.row_sq);
     else
-      colrow_norms_kernel<float><<<grid, 256, 0, stream>>>(static_cast<const float*>(a.w),
-                                                           a.d_out, a.d_in, ws.col_sq, ws.row_sq);
+      colrow_norms_kernel<float><<<grid, 256, 0, stream>>>(
+          static_cast<const float*>(a.w), a.d_out, a.d_in, vec, ws.col_sq, ws.row_sq);
     KQ_TRY(check_launch("colrow_norms_kernel"));
   }
 

@@ -170,7 +170,7 @@ def test_biip_matches_oracle(K, P, flags, shape, w_dtype):
 @pytest.mark.parametrize("w_dtype", [torch.float32, torch.bfloat16])
 def test_biip_row_block_sizes(K, P, d_out, d_in, w_dtype):
     # every input Hadamard block size of the row pass's tiled kernel (b = 32 .. 4096), with
-    # chunks of W that end part-way (d_out * d_in not a multiple of the 4096-element chunk)
+    # matrices whose row count is not a multiple of the rows a chunk takes (4096 / b)
     n = 256
     xq, xfp, g, w, si, so = layer_inputs(d_out, d_in, n, w_dtype=w_dtype,
                                          tag=("biip-b", d_out, d_in))
@@ -182,6 +182,24 @@ def test_biip_row_block_sizes(K, P, d_out, d_in, w_dtype):
     assert rel(h64(r.hx), o["hx"]) <= TOL
     assert rel(h64(r.dxx), o["dxx"]) <= TOL
     assert rel(h64(hg_in), o["hg"]) <= TOL
+    assert K.kronq_device_error() == 0
+
+
+@pytest.mark.parametrize("d_out,d_in", [(4096, 100), (256, 36), (96, 68), (1024, 20),
+                                        (2048, 44)])
+def test_biip_col_pass_ragged(K, P, d_out, d_in):
+    # the column pass over output Hadamard blocks of 32 .. 4096 rows (one pass up to 256, two
+    # above), on W widths that end part-way through a 32-column tile; H_G written back
+    n = 256
+    xq, xfp, g, w, si, so = layer_inputs(d_out, d_in, n, tag=("biip-c", d_out, d_in))
+    hx, hg, dxx = gpu_sums(K, xq, xfp, g)
+    hg_in = hg.clone()
+    r = run_biip(K, P, w, hx, hg_in, dxx, 1.0 / n, si, so, 15 | 16)
+    o = O.biip(h64(w), h64(hx), h64(hg), h64(dxx), 1.0 / n, h64(si), h64(so), 15)
+    assert rel(h64(r.w_prime), o["w"]) <= TOL
+    assert rel(h64(r.hx), o["hx"]) <= TOL
+    assert rel(h64(hg_in), o["hg"]) <= TOL
+    assert abs(float(r.tr[1]) - o["tr_hg"]) <= TOL * abs(o["tr_hg"])
     assert K.kronq_device_error() == 0
 
 
