@@ -121,46 +121,50 @@ __device__ __forceinline__ double biip_scale(double diag_raw, double inv_n, doub
   return sqrt(sqrt(dg / norm_sq));
 }
 
-// Scales and factor vectors for one side (d entries).
+// Scales and factor vectors for one side (d entries), 256 threads per block.
 //   s        = S (fp32 output)
 //   fw       = S * sign            (factor on W)
 //   fh       = sign / S            (factor on the Hessian, both sides)
-__global__ void side_scales_kernel(int d, const float* __restrict__ h, const double* __restrict__ nsq,
-                                   double inv_n, int do_scale, const int8_t* __restrict__ sign,
-                                   float* __restrict__ s_out, float* __restrict__ fw,
-                                   float* __restrict__ fh) {
+//   tr_part  (if given) this block's share of tr(S^-1 (inv_n H) S^-1) = sum_i inv_n H_ii / s_i^2
+__global__ void __launch_bounds__(256) side_scales_kernel(int d, const float* __restrict__ h,
+                                                          const double* __restrict__ nsq,
+                                                          double inv_n, int do_scale,
+                                                          const int8_t* __restrict__ sign,
+                                                          float* __restrict__ s_out,
+                                                          float* __restrict__ fw,
+                                                          float* __restrict__ fh,
+                                                          double* __restrict__ tr_part) {
+  __shared__ double red[8];
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= d) return;
-  double s = 1.0;
-  if (do_scale) s = biip_scale(h[static_cast<int64_t>(i) * d + i], inv_n, nsq[i]);
-  const double sg = sign ? static_cast<double>(sign[i]) : 1.0;
-  s_out[i] = static_cast<float>(s);
-  fw[i] = static_cast<float>(s * sg);
-  fh[i] = static_cast<float>(sg / s);
-}
-
-// tr(S^-1 (inv_n H) S^-1) = sum_i inv_n H_ii / s_i^2, in fp64 (one block).
-__global__ void side_trace_kernel(int d, const float* __restrict__ h, const double* __restrict__ nsq,
-                                  double inv_n, int do_scale, double* __restrict__ tr) {
-  __shared__ double red[32];
-  double acc = 0.0;
-#pragma unroll 8
-  for (int i = threadIdx.x; i < d; i += blockDim.x) {
-    const double hii = static_cast<double>(h[static_cast<int64_t>(i) * d + i]) * inv_n;
+  double contrib = 0.0;
+  if (i < d) {
     double s = 1.0;
     if (do_scale) s = biip_scale(h[static_cast<int64_t>(i) * d + i], inv_n, nsq[i]);
-    acc += hii / (s * s);
+    const double sg = sign ? static_cast<double>(sign[i]) : 1.0;
+    s_out[i] = static_cast<float>(s);
+    fw[i] = static_cast<float>(s * sg);
+    fh[i] = static_cast<float>(sg / s);
+    if (tr_part) contrib = static_cast<double>(h[static_cast<int64_t>(i) * d + i]) * inv_n / (s * s);
   }
+  if (!tr_part) return;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  for (int o = 16; o > 0; o >>= 1) contrib += __shfl_xor_sync(0xffffffffu, contrib, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = contrib;
   __syncthreads();
-  if (threadIdx.x < 32) {
-    double v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.0;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (threadIdx.x == 0) *tr = v;
+  if (threadIdx.x == 0) {
+    double v = 0.0;
+    for (int k = 0; k < 8; ++k) v += red[k];
+    tr_part[blockIdx.x] = v;
   }
+}
+
+// tr = sum of the n block shares, in a fixed order (one warp).
+__global__ void trace_sum_kernel(const double* __restrict__ part, int n, double* __restrict__ tr) {
+  double v = 0.0;
+  for (int k = threadIdx.x; k < n; k += 32) v += part[k];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if (threadIdx.x == 0) *tr = v;
 }
 
 // Row pass over a rows x cols matrix seen as a flat array of b-blocks (b divides cols):
@@ -604,15 +608,29 @@ struct RowTma {
   static constexpr size_t kSmem = 1024 + static_cast<size_t>(kStages) * kStageBytes + kWorkBytes + 64;
 };
 
-__device__ __forceinline__ void fwht32(float (&x)[32]) {
+// Butterfly on two independent pairs at once with Blackwell's packed fp32 arithmetic:
+// (a, b) <- (a + b, a - b) per component, rounded exactly as the scalar sum and difference (the
+// difference is a fused b * -1 + a, whose product is exact).
+__device__ __forceinline__ void bfly2(float2& a, float2& b) {
+  const float2 s = __fadd2_rn(a, b);
+  b = __ffma2_rn(b, make_float2(-1.f, -1.f), a);
+  a = s;
+}
+
+// 32-point Walsh-Hadamard butterflies on x[2 i + c] = x2[i].c: index bit 0 inside each pair
+// (scalar), bits 1-4 between pairs (packed).
+__device__ __forceinline__ void fwht32(float2 (&x)[16]) {
 #pragma unroll
-  for (int h = 0; h < 5; ++h)
+  for (int i = 0; i < 16; ++i) {
+    const float a = x[i].x, b = x[i].y;
+    x[i] = make_float2(a + b, a - b);
+  }
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      if (j & (1 << h)) continue;
-      const float a = x[j], b = x[j | (1 << h)];
-      x[j] = a + b;
-      x[j | (1 << h)] = a - b;
+  for (int h = 0; h < 4; ++h)
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      if (i & (1 << h)) continue;
+      bfly2(x[i], x[i | (1 << h)]);
     }
 }
 
@@ -621,8 +639,8 @@ __device__ __forceinline__ int tpos(int r, int q) { return r * 32 + 4 * (q ^ (r 
 
 // One round: tile rows r0 + (k << H0), k < 2^MLOG, butterflies on the low NB bits of k. The last
 // round stores tile row r's W columns at out(r, column offset) (skipped where that is null),
-// times `scale`; the others write back to the tile.
-template <int H0, int MLOG, int NB, bool LAST, typename Out>
+// times `scale` if SCALE; the others write back to the tile.
+template <int H0, int MLOG, int NB, bool LAST, bool SCALE, typename Out>
 __device__ __forceinline__ void tile_round(float* work, int t, float scale, const Out& out) {
   constexpr int M = 1 << MLOG, W = 32 / M;
   const int g = t & (M - 1), s = t >> MLOG;
@@ -633,76 +651,98 @@ __device__ __forceinline__ void tile_round(float* work, int t, float scale, cons
     else if constexpr (W == 2) return tpos(r, g >> 1) + 2 * (g & 1);
     else return tpos(r, g >> 2) + (g & 3);
   };
-  float y[M][W];
-#pragma unroll
-  for (int k = 0; k < M; ++k) {
-    const float* p = work + at(r0 + (k << H0));
-    if constexpr (W == 4) {
-      const float4 v = *reinterpret_cast<const float4*>(p);
-      y[k][0] = v.x; y[k][1] = v.y; y[k][2] = v.z; y[k][3] = v.w;
-    } else if constexpr (W == 2) {
-      const float2 v = *reinterpret_cast<const float2*>(p);
-      y[k][0] = v.x; y[k][1] = v.y;
-    } else {
-      y[k][0] = p[0];
-    }
-  }
-#pragma unroll
-  for (int h = 0; h < NB; ++h)
+  if constexpr (W >= 2) {
+    constexpr int Y = W / 2;   // column pairs per row, butterflied packed
+    float2 y[M][Y];
 #pragma unroll
     for (int k = 0; k < M; ++k) {
-      if (k & (1 << h)) continue;
-#pragma unroll
-      for (int e = 0; e < W; ++e) {
-        const float a = y[k][e], b = y[k | (1 << h)][e];
-        y[k][e] = a + b;
-        y[k | (1 << h)][e] = a - b;
+      const float* p = work + at(r0 + (k << H0));
+      if constexpr (W == 4) {
+        const float4 v = *reinterpret_cast<const float4*>(p);
+        y[k][0] = make_float2(v.x, v.y);
+        y[k][Y - 1] = make_float2(v.z, v.w);
+      } else {
+        y[k][0] = *reinterpret_cast<const float2*>(p);
       }
     }
 #pragma unroll
-  for (int k = 0; k < M; ++k) {
-    const int r = r0 + (k << H0);
-    float* p;
-    if constexpr (LAST) {
-      p = out(r, W * g);
-      if (!p) continue;
+    for (int h = 0; h < NB; ++h)
 #pragma unroll
-      for (int e = 0; e < W; ++e) y[k][e] *= scale;
-    } else {
-      p = work + at(r);
+      for (int k = 0; k < M; ++k) {
+        if (k & (1 << h)) continue;
+#pragma unroll
+        for (int e = 0; e < Y; ++e) bfly2(y[k][e], y[k | (1 << h)][e]);
+      }
+#pragma unroll
+    for (int k = 0; k < M; ++k) {
+      const int r = r0 + (k << H0);
+      float* p;
+      if constexpr (LAST) {
+        p = out(r, W * g);
+        if (!p) continue;
+        if constexpr (SCALE) {
+#pragma unroll
+          for (int e = 0; e < Y; ++e) y[k][e] = __fmul2_rn(y[k][e], make_float2(scale, scale));
+        }
+      } else {
+        p = work + at(r);
+      }
+      if constexpr (W == 4)
+        *reinterpret_cast<float4*>(p) = make_float4(y[k][0].x, y[k][0].y, y[k][Y - 1].x,
+                                                    y[k][Y - 1].y);
+      else
+        *reinterpret_cast<float2*>(p) = y[k][0];
     }
-    if constexpr (W == 4)
-      *reinterpret_cast<float4*>(p) = make_float4(y[k][0], y[k][1], y[k][2], y[k][3]);
-    else if constexpr (W == 2)
-      *reinterpret_cast<float2*>(p) = make_float2(y[k][0], y[k][1]);
-    else
-      p[0] = y[k][0];
+  } else {
+    float y[M];
+#pragma unroll
+    for (int k = 0; k < M; ++k) y[k] = work[at(r0 + (k << H0))];
+#pragma unroll
+    for (int h = 0; h < NB; ++h)
+#pragma unroll
+      for (int k = 0; k < M; ++k) {
+        if (k & (1 << h)) continue;
+        const float a = y[k], b = y[k | (1 << h)];
+        y[k] = a + b;
+        y[k | (1 << h)] = a - b;
+      }
+#pragma unroll
+    for (int k = 0; k < M; ++k) {
+      const int r = r0 + (k << H0);
+      if constexpr (LAST) {
+        float* p = out(r, g);
+        if (!p) continue;
+        *p = SCALE ? y[k] * scale : y[k];
+      } else {
+        work[at(r)] = y[k];
+      }
+    }
   }
 }
 
 // Butterflies on the low L bits of the tile-row index (L <= log2 of the tile rows, at least 7),
 // in one or two rounds; a round of m bits starting at bit h0 needs h0 + m <= log2 tile rows.
-template <int L, typename Out>
+template <int L, bool SCALE, typename Out>
 __device__ __forceinline__ void tile_rounds(float* work, int t, float scale, const Out& out) {
   if constexpr (L == 0) {
-    tile_round<0, 3, 0, true>(work, t, scale, out);
+    tile_round<0, 3, 0, true, SCALE>(work, t, scale, out);
   } else if constexpr (L <= 3) {
-    tile_round<0, 3, L, true>(work, t, scale, out);
+    tile_round<0, 3, L, true, SCALE>(work, t, scale, out);
   } else if constexpr (L == 4 || L == 5) {
-    tile_round<0, L, L, true>(work, t, scale, out);
+    tile_round<0, L, L, true, SCALE>(work, t, scale, out);
   } else if constexpr (L == 6) {
-    tile_round<0, 3, 3, false>(work, t, scale, out);
+    tile_round<0, 3, 3, false, SCALE>(work, t, scale, out);
     __syncthreads();
-    tile_round<3, 3, 3, true>(work, t, scale, out);
+    tile_round<3, 3, 3, true, SCALE>(work, t, scale, out);
   } else if constexpr (L == 7) {
-    tile_round<0, 3, 3, false>(work, t, scale, out);
+    tile_round<0, 3, 3, false, SCALE>(work, t, scale, out);
     __syncthreads();
-    tile_round<3, 4, 4, true>(work, t, scale, out);
+    tile_round<3, 4, 4, true, SCALE>(work, t, scale, out);
   } else {
     static_assert(L == 8, "tile rounds cover up to 8 index bits");
-    tile_round<0, 4, 4, false>(work, t, scale, out);
+    tile_round<0, 4, 4, false, SCALE>(work, t, scale, out);
     __syncthreads();
-    tile_round<4, 4, 4, true>(work, t, scale, out);
+    tile_round<4, 4, 4, true, SCALE>(work, t, scale, out);
   }
 }
 
@@ -756,7 +796,7 @@ __global__ void __launch_bounds__(RowTma<LOG2B, sizeof(T) == 4>::kThreads,
   const int rr = t >> LOG2S, seg = t & (S::kSegs - 1);    // row step: matrix row, segment
   int64_t band = k0 / nrg, rg = k0 - band * nrg;
   int64_t cf_band = -1;
-  float cf[32];
+  float2 cf[16];   // factors of this thread's 32 columns, in pairs
   bool aborted = false;
   int i = 0;
   for (; i < n; ++i) {
@@ -771,24 +811,25 @@ __global__ void __launch_bounds__(RowTma<LOG2B, sizeof(T) == 4>::kThreads,
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           const float4 v = *reinterpret_cast<const float4*>(col_f + col0 + 32 * seg + 4 * q);
-          cf[4 * q] = v.x * sc; cf[4 * q + 1] = v.y * sc; cf[4 * q + 2] = v.z * sc;
-          cf[4 * q + 3] = v.w * sc;
+          cf[2 * q] = make_float2(v.x * sc, v.y * sc);
+          cf[2 * q + 1] = make_float2(v.z * sc, v.w * sc);
         }
       } else {
 #pragma unroll
-        for (int k = 0; k < 32; ++k) cf[k] = sc;
+        for (int i = 0; i < 16; ++i) cf[i] = make_float2(sc, sc);
       }
       cf_band = band;
     }
     const bool ok = mbar_wait(&full[st], (i / NST) & 1, abort_flag, err_word, DEV_ERR_LOAD_WAIT);
     float* work = kF32 ? reinterpret_cast<float*>(stages + st * S::kStageBytes) : work_bf;
     if (ok) {
-      float x[32];
+      float2 x[16];   // x[i] = elements 2 i, 2 i + 1 of tile row t
       if constexpr (kF32) {
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           const float4 v = *reinterpret_cast<const float4*>(work + tpos(t, q));
-          x[4 * q] = v.x; x[4 * q + 1] = v.y; x[4 * q + 2] = v.z; x[4 * q + 3] = v.w;
+          x[2 * q] = make_float2(v.x, v.y);
+          x[2 * q + 1] = make_float2(v.z, v.w);
         }
       } else {
         const T* sg = reinterpret_cast<const T*>(stages + st * S::kStageBytes) + 32 * t;
@@ -797,19 +838,24 @@ __global__ void __launch_bounds__(RowTma<LOG2B, sizeof(T) == 4>::kThreads,
           const uint4 v = *reinterpret_cast<const uint4*>(sg + 8 * (q ^ ((t >> 1) & 3)));
           const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            x[8 * q + 2 * e] = __uint_as_float(u[e] << 16);
-            x[8 * q + 2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
-          }
+          for (int e = 0; e < 4; ++e)
+            x[4 * q + e] = make_float2(__uint_as_float(u[e] << 16),
+                                       __uint_as_float(u[e] & 0xFFFF0000u));
         }
       }
+      if constexpr (S::kRB == 1) {   // one matrix row per chunk: its factor joins the store
 #pragma unroll
-      for (int k = 0; k < 32; ++k) x[k] *= rf * cf[k];
+        for (int i = 0; i < 16; ++i) x[i] = __fmul2_rn(x[i], cf[i]);
+      } else {
+        const float2 rf2 = make_float2(rf, rf);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) x[i] = __fmul2_rn(x[i], __fmul2_rn(cf[i], rf2));
+      }
       fwht32(x);
 #pragma unroll
       for (int q = 0; q < 8; ++q)
         *reinterpret_cast<float4*>(work + tpos(t, q)) =
-            make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+            make_float4(x[2 * q].x, x[2 * q].y, x[2 * q + 1].x, x[2 * q + 1].y);
     }
     if (__syncthreads_or(!ok)) {
       aborted = true;
@@ -817,7 +863,7 @@ __global__ void __launch_bounds__(RowTma<LOG2B, sizeof(T) == 4>::kThreads,
     }
     // the index bits above the tile row; the last round writes tile row r to matrix row
     // row0 + r / segs, columns col0 + 32 (r % segs) ..
-    tile_rounds<L>(work, t, 1.0f, [&](int r, int c) -> float* {
+    tile_rounds<L, S::kRB == 1>(work, t, rf, [&](int r, int c) -> float* {
       const int64_t row = row0 + (r >> LOG2S);
       return row < rows ? dst + row * cols + col0 + 32 * (r & (S::kSegs - 1)) + c : nullptr;
     });
@@ -955,11 +1001,15 @@ __global__ void __launch_bounds__(ColTma<LP>::kThreads, ColTma<LP>::kMinBlocks)
     float* work = reinterpret_cast<float*>(stages + st * S::kStageBytes);
     const int64_t rbase = (y / rs) * P * rs + (y % rs);
     const int64_t c0 = static_cast<int64_t>(cg) * CT * 32;
-    tile_rounds<LP>(work, t, out_scale, [&](int r, int c) -> float* {
+    auto out = [&](int r, int c) -> float* {
       const int64_t col = c0 + 32 * (r >> LP) + c;
       return col < cols ? m + (rbase + static_cast<int64_t>(rs) * (r & (P - 1))) * cols + col
                         : nullptr;
-    });
+    };
+    if (out_scale != 1.0f)
+      tile_rounds<LP, true>(work, t, out_scale, out);
+    else
+      tile_rounds<LP, false>(work, t, 1.0f, out);
     fence_proxy_async_smem();   // the stage was written in place; TMA refills it
     __syncthreads();
     if (++cg == ncg) {
@@ -1137,6 +1187,8 @@ struct BiipWs {
   float* fh_in;     // d_in   sign_in / S_X
   float* fw_out;    // d_out  S_G * sign_out
   float* fh_out;    // d_out  sign_out / S_G
+  double* tr_in;    // ceil(d_in / 256)   block shares of tr(H_X')
+  double* tr_out;   // ceil(d_out / 256)  block shares of tr(H_G')
 };
 
 BiipWs carve(void* ws, int d_out, int d_in) {
@@ -1153,6 +1205,10 @@ BiipWs carve(void* ws, int d_out, int d_in) {
   w.fw_out = reinterpret_cast<float*>(p);
   p += align256(sizeof(float) * d_out);
   w.fh_out = reinterpret_cast<float*>(p);
+  p += align256(sizeof(float) * d_out);
+  w.tr_in = reinterpret_cast<double*>(p);
+  p += align256(sizeof(double) * ((d_in + 255) / 256));
+  w.tr_out = reinterpret_cast<double*>(p);
   return w;
 }
 
@@ -1160,7 +1216,9 @@ BiipWs carve(void* ws, int d_out, int d_in) {
 
 size_t biip_workspace_bytes(int d_out, int d_in) {
   return align256(sizeof(double) * d_in) + align256(sizeof(double) * d_out) +
-         2 * align256(sizeof(float) * d_in) + 2 * align256(sizeof(float) * d_out);
+         2 * align256(sizeof(float) * d_in) + 2 * align256(sizeof(float) * d_out) +
+         align256(sizeof(double) * ((d_in + 255) / 256)) +
+         align256(sizeof(double) * ((d_out + 255) / 256));
 }
 
 kronq_status run_biip(const BiipArgs& a, void* ws_raw, cudaStream_t stream) {
@@ -1191,20 +1249,23 @@ kronq_status run_biip(const BiipArgs& a, void* ws_raw, cudaStream_t stream) {
   }
 
   // 2. scales, factors and traces (from the un-transformed diagonals)
-  side_scales_kernel<<<(a.d_in + 255) / 256, 256, 0, stream>>>(
+  const int nb_in = (a.d_in + 255) / 256, nb_out = (a.d_out + 255) / 256;
+  side_scales_kernel<<<nb_in, 256, 0, stream>>>(
       a.d_in, a.hx, ws.col_sq, a.inv_n, scale_in, rot_in ? a.sign_in : nullptr, a.s_x, ws.fw_in,
-      ws.fh_in);
+      ws.fh_in, a.tr_hx ? ws.tr_in : nullptr);
   KQ_TRY(check_launch("side_scales_kernel(in)"));
-  side_trace_kernel<<<1, 1024, 0, stream>>>(a.d_in, a.hx, ws.col_sq, a.inv_n, scale_in, a.tr_hx);
-  KQ_TRY(check_launch("side_trace_kernel(in)"));
-  side_scales_kernel<<<(a.d_out + 255) / 256, 256, 0, stream>>>(
+  if (a.tr_hx) {
+    trace_sum_kernel<<<1, 32, 0, stream>>>(ws.tr_in, nb_in, a.tr_hx);
+    KQ_TRY(check_launch("trace_sum_kernel(in)"));
+  }
+  const bool tr_g = a.hg && a.tr_hg;
+  side_scales_kernel<<<nb_out, 256, 0, stream>>>(
       a.d_out, a.hg, ws.row_sq, a.inv_n, scale_out, rot_out ? a.sign_out : nullptr, a.s_g,
-      ws.fw_out, ws.fh_out);
+      ws.fw_out, ws.fh_out, tr_g ? ws.tr_out : nullptr);
   KQ_TRY(check_launch("side_scales_kernel(out)"));
-  if (a.hg && a.tr_hg) {
-    side_trace_kernel<<<1, 1024, 0, stream>>>(a.d_out, a.hg, ws.row_sq, a.inv_n, scale_out,
-                                              a.tr_hg);
-    KQ_TRY(check_launch("side_trace_kernel(out)"));
+  if (tr_g) {
+    trace_sum_kernel<<<1, 32, 0, stream>>>(ws.tr_out, nb_out, a.tr_hg);
+    KQ_TRY(check_launch("trace_sum_kernel(out)"));
   }
 
   // 3. W' = U S_G W S_X V^T: row pass (scales, output signs, input-side FWHT), column pass
