@@ -90,7 +90,11 @@ KRONQ_API void kronq_set_sm_budget(int32_t sms);
 KRONQ_API int32_t kronq_sm_budget(void);
 
 /* Reads and clears the device-side error word (bounded waits that gave up). Synchronizes
- * `stream`. *code_out = 0 when no kernel reported an error since the last call. */
+ * `stream`. *code_out = 0 when no kernel reported an error since the last call, else the first
+ * code recorded: 1 a TMA producer found no free pipeline stage, 2 a tensor-core issuer waited for
+ * operands or an accumulator, 3 an epilogue waited for an accumulator, 4 a streaming pass (the
+ * Hadamard passes of kronq_biip) waited for a tile load. Each wait gives up after 4 s; the kernel
+ * then lets its copies in flight land and returns, leaving its outputs incomplete. */
 KRONQ_API kronq_status kronq_device_error(int32_t* code_out, kronq_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------
@@ -161,7 +165,7 @@ KRONQ_API kronq_status kronq_biip(const void* w, int32_t w_dtype, float* w_out, 
  * services that reserve all device memory up front. This variant takes the same arguments as
  * kronq_biip minus the workspace and uses a fixed scratch array of 1 MiB that lives in device
  * memory (every GPU that loads this library holds it until the process exits). That limits it
- * to 16 * (d_out + d_in) + about 1.5 KB <= 1 MiB (d_out + d_in up to about 65000, every LLaMA
+ * to about 16.03 * (d_out + d_in) + 2 KB <= 1 MiB (d_out + d_in up to about 65000, every LLaMA
  * shape); larger layers get KRONQ_ERR_UNSUPPORTED with the needed size in the error detail.
  * The first call on a device looks up the array's device address; make that first call before
  * any stream capture. All calls in the process share the one array, so calls whose execution
