@@ -12,8 +12,11 @@
 //   rows    for every row: multiply by row and column factors, FWHT along the row in b-blocks
 //   cols    for every b-row block of every column: FWHT along the column (in place; one pass
 //           for b <= 256, two for larger b)
-// The passes work in registers (16-point butterflies per thread) with a shared-memory exchange
-// between groups of four stages; b outside [16, 16384] takes plain shared-memory kernels.
+// The row and column passes stream TMA-loaded chunks through shared memory: 32-point
+// butterflies along 128-byte tile rows in registers, the higher index bits in vectorised rounds
+// down the tile columns (fwht_rows_tma_kernel, fwht_cols_tma_kernel). b = 16 or 16384,
+// unaligned operands and matrices narrower than 32 columns take register/shuffle kernels
+// (fwht_rows_reg_kernel, fwht_cols_reg_kernel); b outside [16, 16384] plain shared-memory ones.
 // W' = rows(W) then cols; H_X and dXX^T = rows then cols (in place); H_G likewise if asked.
 #include <cuda_bf16.h>
 
