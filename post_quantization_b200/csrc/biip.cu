@@ -819,14 +819,14 @@ __global__ void __launch_bounds__(RowTma<LOG2B, sizeof(T) == 4>::kThreads,
         }
       } else {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) cf[i] = make_float2(sc, sc);
+        for (int p = 0; p < 16; ++p) cf[p] = make_float2(sc, sc);
       }
       cf_band = band;
     }
     const bool ok = mbar_wait(&full[st], (i / NST) & 1, abort_flag, err_word, DEV_ERR_LOAD_WAIT);
     float* work = kF32 ? reinterpret_cast<float*>(stages + st * S::kStageBytes) : work_bf;
     if (ok) {
-      float2 x[16];   // x[i] = elements 2 i, 2 i + 1 of tile row t
+      float2 x[16];   // x[p] = elements 2 p, 2 p + 1 of tile row t
       if constexpr (kF32) {
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
@@ -848,11 +848,11 @@ __global__ void __launch_bounds__(RowTma<LOG2B, sizeof(T) == 4>::kThreads,
       }
       if constexpr (S::kRB == 1) {   // one matrix row per chunk: its factor joins the store
 #pragma unroll
-        for (int i = 0; i < 16; ++i) x[i] = __fmul2_rn(x[i], cf[i]);
+        for (int p = 0; p < 16; ++p) x[p] = __fmul2_rn(x[p], cf[p]);
       } else {
         const float2 rf2 = make_float2(rf, rf);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) x[i] = __fmul2_rn(x[i], __fmul2_rn(cf[i], rf2));
+        for (int p = 0; p < 16; ++p) x[p] = __fmul2_rn(x[p], __fmul2_rn(cf[p], rf2));
       }
       fwht32(x);
 #pragma unroll
@@ -878,8 +878,9 @@ __global__ void __launch_bounds__(RowTma<LOG2B, sizeof(T) == 4>::kThreads,
     }
   }
   if (aborted && t == 0) {
-    // let the loads already issued (chunks i .. i + stages - 2) land before the CTA exits
-    for (int j = i; j < n && j < i + NST - 1; ++j)
+    // let the loads already issued (chunks i .. i + stages - 1, one per stage) land before the
+    // CTA exits
+    for (int j = i; j < n && j < i + NST; ++j)
       mbar_drain(&full[j % NST], (j / NST) & 1, kWaitLimitNs);
   }
 }
@@ -1021,7 +1022,8 @@ __global__ void __launch_bounds__(ColTma<LP>::kThreads, ColTma<LP>::kMinBlocks)
     }
   }
   if (aborted && t == 0) {
-    for (int j = i; j < n && j < i + NST - 1; ++j)
+    // let the loads already issued (chunks i .. i + stages - 1) land before the CTA exits
+    for (int j = i; j < n && j < i + NST; ++j)
       mbar_drain(&full[j % NST], (j / NST) & 1, kWaitLimitNs);
   }
 }
