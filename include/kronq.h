@@ -64,6 +64,7 @@ enum {
   KRONQ_BIIP_ROTATE_IN = 4,   /* W <- W V^T,  H_X <- V H_X V^T, dXX^T <- V dXX^T V^T         */
   KRONQ_BIIP_ROTATE_OUT = 8,  /* W <- U W,    H_G <- U H_G U^T                               */
   KRONQ_BIIP_WRITE_HG = 16,   /* also write the normalised, transformed H_G into `hg`        */
+  KRONQ_BIIP_HG_DIAG = 32,    /* `hg` is only the d_out diagonal sums (kronq_accumulate_diag) */
   KRONQ_BIIP_FULL = 15        /* the four transforms of BiIP                                  */
 };
 
@@ -125,6 +126,31 @@ KRONQ_API kronq_status kronq_accumulate(const void* xq, int64_t ld_xq, const voi
                               void* workspace, size_t workspace_bytes, kronq_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------
+ * 1b. kronq_accumulate_diag - the diagonal of H_G alone.
+ *
+ * [KronQ-hyper] Method: S_G (BiIP equations) and the sensitivity tr(H_G) read only the diagonal
+ * of H_G, and Proposition 1 takes H_G out of the column update. A caller that quantizes without
+ * evaluating the objective or the incoherence of H_G therefore needs diag(G^T G) only. This call
+ * adds, over n tokens,
+ *     diag_sum[j] += sum_t G[t][j]^2        (j < d)
+ * in one streaming read of G instead of the G^T G product. Pass the result to kronq_biip as `hg`
+ * with KRONQ_BIIP_HG_DIAG.
+ *
+ *   g         (device, bf16) n x d, row stride ld_g elements (ld_g >= d, ld_g*2 bytes a multiple
+ *             of 16, base 16-byte aligned); one token per row
+ *   diag_sum  (device, fp32) d entries, += the column sums of squares (un-normalised)
+ *   workspace kronq_accumulate_diag_workspace_size(n, d) bytes (partial sums of blocks of 2048
+ *             tokens); NULL when that size is 0. n = 0 is a no-op.
+ *   Accumulation: squares of bf16 values are exact in fp32; each block of 2048 tokens is summed
+ *   in fp32, the blocks are added in a fixed order in fp64, so the result does not depend on
+ *   scheduling.
+ * ------------------------------------------------------------------------------------- */
+KRONQ_API size_t kronq_accumulate_diag_workspace_size(int64_t n, int32_t d);
+KRONQ_API kronq_status kronq_accumulate_diag(const void* g, int64_t ld_g, int64_t n, int32_t d,
+                                             float* diag_sum, void* workspace,
+                                             size_t workspace_bytes, kronq_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
  * 2. kronq_biip - normalisation and bidirectional incoherence processing of one sublayer.
  *
  * [KronQ-hyper] Method, BiIP equations:
@@ -142,7 +168,9 @@ KRONQ_API kronq_status kronq_accumulate(const void* xq, int64_t ld_xq, const voi
  *   hx       (device, fp32) d_in x d_in: in: raw sum X~^T X~; out: V S_X^-1 (inv_n hx) S_X^-1 V^T
  *   hg       (device, fp32) d_out x d_out raw sum G^T G, or NULL (then SCALE_OUT is invalid).
  *            Read-only unless KRONQ_BIIP_WRITE_HG, in which case it is replaced by
- *            U S_G^-1 (inv_n hg) S_G^-1 U^T.
+ *            U S_G^-1 (inv_n hg) S_G^-1 U^T. With KRONQ_BIIP_HG_DIAG it is instead the d_out
+ *            raw diagonal sums from kronq_accumulate_diag: S_G and tr_hg need only those, and
+ *            WRITE_HG is then invalid.
  *   dxx      (device, fp32) d_in x d_in raw drift sum or NULL; out: V S_X^-1 (inv_n dxx) S_X^-1 V^T
  *   inv_n    1 / total token count
  *   sign_in  (device, int8 +-1) d_in; needed with ROTATE_IN. sign_out likewise d_out.

@@ -13,6 +13,9 @@ What it computes, step by step, with the passage each step follows. Page names:
   accumulate      H_X = E[x x^T], H_G = E[g g^T] under the K-FAC split H ~ H_X (x) H_G, and the
                   asymmetric term E[(x - x~) x~^T]            [KronQ-hyper] Method: Fisher eq.,
                                                               K-FAC split, asymmetric objective
+  accumulate_diag the diagonal of G^T G alone: S_G and tr(H_G) read only the diagonal, and H_G
+                  cancels from the column update           [KronQ-hyper] Method: BiIP equations,
+                                                              sensitivity, Proposition 1
   biip            W <- S_G W S_X with S_X = diag(H_X,jj/|W_:,j|^2)^(1/4), S_G likewise on rows;
                   then W <- U W V^T, H_X <- V H_X V^T, H_G <- U H_G U^T, dXX^T <- V dXX^T V^T
                   with U, V random-sign Hadamard          [KronQ-hyper] Method: BiIP equations
@@ -101,6 +104,17 @@ def accumulate(xq, xfp=None, g=None):
         xfp = np.asarray(xfp, dtype=np.float64)
         dxx = (xfp - xq).T @ xq
     return hx, hg, dxx
+
+
+def accumulate_diag(g):
+    """Raw diagonal sums diag(G^T G)_j = sum_t G_tj^2 over the N tokens (rows).
+
+    [KronQ-hyper] Method: S_G = diag(H_G,ii / |W_i,:|^2)^(1/4) and the sensitivity tr(H_G) use
+    only the diagonal of H_G, and Proposition 1 removes H_G from the column update, so a
+    quantization that skips the objective and the incoherence figure needs only these sums.
+    """
+    g = np.asarray(g, dtype=np.float64)
+    return np.einsum("tj,tj->j", g, g)
 
 
 def fisher_kron(x, g):

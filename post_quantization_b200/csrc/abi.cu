@@ -255,6 +255,24 @@ kronq_status kronq_accumulate(const void* xq, int64_t ld_xq, const void* xfp, in
   return KRONQ_OK;
 }
 
+size_t kronq_accumulate_diag_workspace_size(int64_t n, int32_t d) {
+  return accumulate_diag_workspace_bytes(n, d);
+}
+
+kronq_status kronq_accumulate_diag(const void* g, int64_t ld_g, int64_t n, int32_t d,
+                                   float* diag_sum, void* workspace, size_t workspace_bytes,
+                                   kronq_stream_t stream) {
+  if (n < 0) return fail(KRONQ_ERR_SHAPE, "n < 0");
+  if (d <= 0) return fail(KRONQ_ERR_SHAPE, "d <= 0");
+  if (!diag_sum) return fail(KRONQ_ERR_INVALID_ARG, "diag_sum is required");
+  if (n == 0) return KRONQ_OK;
+  KQ_TRY(check_bf16_matrix(g, ld_g, d, "g"));
+  KQ_TRY(check_ws(workspace, workspace_bytes, accumulate_diag_workspace_bytes(n, d)));
+  KQ_TRY(kronq_device_check());
+  return launch_accumulate_diag(g, ld_g, n, d, diag_sum, workspace,
+                                reinterpret_cast<cudaStream_t>(stream));
+}
+
 // ----------------------------------------------------------------------------- biip
 size_t kronq_biip_workspace_size(int32_t d_out, int32_t d_in) {
   if (d_out <= 0 || d_in <= 0) return 0;
@@ -271,10 +289,14 @@ kronq_status kronq_biip(const void* w, int32_t w_dtype, float* w_out, float* hx,
     return fail(KRONQ_ERR_INVALID_ARG, "w, w_out, hx, s_x, s_g and tr_hx are required");
   if (w_dtype != KRONQ_DTYPE_BF16 && w_dtype != KRONQ_DTYPE_F32)
     return fail(KRONQ_ERR_INVALID_ARG, "w_dtype must be KRONQ_DTYPE_BF16 or KRONQ_DTYPE_F32");
-  if (flags & ~static_cast<uint32_t>(31))
+  if (flags & ~static_cast<uint32_t>(63))
     return fail(KRONQ_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
   if ((flags & KRONQ_BIIP_SCALE_OUT) && !hg)
     return fail(KRONQ_ERR_INVALID_ARG, "KRONQ_BIIP_SCALE_OUT needs hg");
+  if ((flags & KRONQ_BIIP_HG_DIAG) && !hg)
+    return fail(KRONQ_ERR_INVALID_ARG, "KRONQ_BIIP_HG_DIAG needs hg (the diagonal sums)");
+  if ((flags & KRONQ_BIIP_HG_DIAG) && (flags & KRONQ_BIIP_WRITE_HG))
+    return fail(KRONQ_ERR_INVALID_ARG, "KRONQ_BIIP_WRITE_HG needs the full H_G, not its diagonal");
   if ((flags & KRONQ_BIIP_ROTATE_IN) && !sign_in)
     return fail(KRONQ_ERR_INVALID_ARG, "KRONQ_BIIP_ROTATE_IN needs sign_in");
   if ((flags & KRONQ_BIIP_ROTATE_OUT) && !sign_out)

@@ -314,6 +314,73 @@ __global__ void drift_split_kernel(const __nv_bfloat16* __restrict__ xfp, int64_
   }
 }
 
+// Column sums of squares of G (n x d bf16), the diagonal of G^T G. A block takes a panel of 256
+// columns (8 per lane, one 16-byte load per token) and up to kDiagTokens tokens; warp w takes
+// tokens w, w + 8, .. of them, eight loads in flight per lane. The 8 warps' sums meet in shared
+// memory and the block writes its partial sums to part[split][column]; no atomics, so the result
+// does not depend on the order blocks run in.
+constexpr int kDiagTokens = 2048;
+
+__global__ void __launch_bounds__(256, 3) diag_partial_kernel(const uint16_t* __restrict__ g,
+                                                           int64_t ld, int64_t n, int d, int vec,
+                                                           float* __restrict__ part) {
+  __shared__ float red[8][256];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int c0 = blockIdx.x * 256 + lane * 8;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.y) * kDiagTokens;
+  const int64_t t1 = n - t0 < kDiagTokens ? n : t0 + kDiagTokens;
+  const bool whole = vec && c0 + 8 <= d;
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  for (int64_t tb = t0 + warp; tb < t1; tb += 64) {
+    uint4 u[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int64_t t = tb + 8 * j;
+      if (whole && t < t1) u[j] = *reinterpret_cast<const uint4*>(g + t * ld + c0);
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int64_t t = tb + 8 * j;
+      if (t >= t1) break;
+      float v[8];
+      if (whole) {
+        const uint32_t q[4] = {u[j].x, u[j].y, u[j].z, u[j].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          v[2 * e] = __uint_as_float(q[e] << 16);
+          v[2 * e + 1] = __uint_as_float(q[e] & 0xFFFF0000u);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          v[e] = c0 + e < d ? __uint_as_float(static_cast<uint32_t>(g[t * ld + c0 + e]) << 16) : 0.f;
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = fmaf(v[e], v[e], acc[e]);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) red[warp][lane * 8 + e] = acc[e];
+  __syncthreads();
+  const int col = blockIdx.x * 256 + threadIdx.x;
+  float sum = 0.f;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) sum += red[k][threadIdx.x];
+  if (col < d) part[static_cast<int64_t>(blockIdx.y) * d + col] = sum;
+}
+
+// diag_sum[j] += sum over splits of part[split][j], added in split order in fp64.
+__global__ void diag_finalize_kernel(const float* __restrict__ part, int splits, int d,
+                                     float* __restrict__ diag_sum) {
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= d) return;
+  double s = 0.0;
+  for (int k = 0; k < splits; ++k) s += part[static_cast<int64_t>(k) * d + j];
+  diag_sum[j] = static_cast<float>(static_cast<double>(diag_sum[j]) + s);
+}
+
 // ---------------------------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------------------------
@@ -410,6 +477,25 @@ kronq_status launch_drift_split(const void* xfp, int64_t ld_xfp, const void* xq,
       static_cast<const __nv_bfloat16*>(xfp), ld_xfp, static_cast<const __nv_bfloat16*>(xq), ld_xq,
       rows, cols, static_cast<__nv_bfloat16*>(hi), static_cast<__nv_bfloat16*>(lo), ld_out);
   return check_launch("drift_split_kernel");
+}
+
+size_t accumulate_diag_workspace_bytes(int64_t n, int d) {
+  if (n <= 0 || d <= 0) return 0;
+  const int64_t splits = (n + kDiagTokens - 1) / kDiagTokens;
+  return static_cast<size_t>(splits) * d * sizeof(float);
+}
+
+kronq_status launch_accumulate_diag(const void* g, int64_t ld, int64_t n, int d, float* diag_sum,
+                                    void* ws, cudaStream_t stream) {
+  if (n <= 0) return KRONQ_OK;
+  const int splits = static_cast<int>((n + kDiagTokens - 1) / kDiagTokens);
+  const int vec = (reinterpret_cast<uintptr_t>(g) & 15u) == 0 && (ld * 2) % 16 == 0;
+  float* part = static_cast<float*>(ws);
+  diag_partial_kernel<<<dim3((d + 255) / 256, splits), 256, 0, stream>>>(
+      static_cast<const uint16_t*>(g), ld, n, d, vec, part);
+  KQ_TRY(check_launch("diag_partial_kernel"));
+  diag_finalize_kernel<<<(d + 255) / 256, 256, 0, stream>>>(part, splits, d, diag_sum);
+  return check_launch("diag_finalize_kernel");
 }
 
 }  // namespace kq

@@ -129,7 +129,9 @@ __device__ __forceinline__ double biip_scale(double diag_raw, double inv_n, doub
 //   fw       = S * sign            (factor on W)
 //   fh       = sign / S            (factor on the Hessian, both sides)
 //   tr_part  (if given) this block's share of tr(S^-1 (inv_n H) S^-1) = sum_i inv_n H_ii / s_i^2
+// H_ii is h[i * hstep]: hstep = d + 1 for the full matrix, 1 for a vector of its diagonal.
 __global__ void __launch_bounds__(256) side_scales_kernel(int d, const float* __restrict__ h,
+                                                          int64_t hstep,
                                                           const double* __restrict__ nsq,
                                                           double inv_n, int do_scale,
                                                           const int8_t* __restrict__ sign,
@@ -142,12 +144,12 @@ __global__ void __launch_bounds__(256) side_scales_kernel(int d, const float* __
   double contrib = 0.0;
   if (i < d) {
     double s = 1.0;
-    if (do_scale) s = biip_scale(h[static_cast<int64_t>(i) * d + i], inv_n, nsq[i]);
+    if (do_scale) s = biip_scale(h[i * hstep], inv_n, nsq[i]);
     const double sg = sign ? static_cast<double>(sign[i]) : 1.0;
     s_out[i] = static_cast<float>(s);
     fw[i] = static_cast<float>(s * sg);
     fh[i] = static_cast<float>(sg / s);
-    if (tr_part) contrib = static_cast<double>(h[static_cast<int64_t>(i) * d + i]) * inv_n / (s * s);
+    if (tr_part) contrib = static_cast<double>(h[i * hstep]) * inv_n / (s * s);
   }
   if (!tr_part) return;
 #pragma unroll
@@ -1232,7 +1234,8 @@ kronq_status run_biip(const BiipArgs& a, void* ws_raw, cudaStream_t stream) {
   const bool scale_out = a.flags & KRONQ_BIIP_SCALE_OUT;
   const bool rot_in = a.flags & KRONQ_BIIP_ROTATE_IN;
   const bool rot_out = a.flags & KRONQ_BIIP_ROTATE_OUT;
-  const bool write_hg = (a.flags & KRONQ_BIIP_WRITE_HG) && a.hg;
+  const bool hg_diag = a.flags & KRONQ_BIIP_HG_DIAG;   // hg holds the diagonal only
+  const bool write_hg = (a.flags & KRONQ_BIIP_WRITE_HG) && a.hg && !hg_diag;
   const int b_in = rot_in ? largest_pow2_divisor(a.d_in) : 1;
   const int b_out = rot_out ? largest_pow2_divisor(a.d_out) : 1;
 
@@ -1256,7 +1259,7 @@ kronq_status run_biip(const BiipArgs& a, void* ws_raw, cudaStream_t stream) {
   // 2. scales, factors and traces (from the un-transformed diagonals)
   const int nb_in = (a.d_in + 255) / 256, nb_out = (a.d_out + 255) / 256;
   side_scales_kernel<<<nb_in, 256, 0, stream>>>(
-      a.d_in, a.hx, ws.col_sq, a.inv_n, scale_in, rot_in ? a.sign_in : nullptr, a.s_x, ws.fw_in,
+      a.d_in, a.hx, static_cast<int64_t>(a.d_in) + 1, ws.col_sq, a.inv_n, scale_in, rot_in ? a.sign_in : nullptr, a.s_x, ws.fw_in,
       ws.fh_in, a.tr_hx ? ws.tr_in : nullptr);
   KQ_TRY(check_launch("side_scales_kernel(in)"));
   if (a.tr_hx) {
@@ -1265,7 +1268,7 @@ kronq_status run_biip(const BiipArgs& a, void* ws_raw, cudaStream_t stream) {
   }
   const bool tr_g = a.hg && a.tr_hg;
   side_scales_kernel<<<nb_out, 256, 0, stream>>>(
-      a.d_out, a.hg, ws.row_sq, a.inv_n, scale_out, rot_out ? a.sign_out : nullptr, a.s_g,
+      a.d_out, a.hg, hg_diag ? 1 : static_cast<int64_t>(a.d_out) + 1, ws.row_sq, a.inv_n, scale_out, rot_out ? a.sign_out : nullptr, a.s_g,
       ws.fw_out, ws.fh_out, tr_g ? ws.tr_out : nullptr);
   KQ_TRY(check_launch("side_scales_kernel(out)"));
   if (tr_g) {

@@ -16,6 +16,9 @@ kronq_status launch_mirror_upper(float* c, int64_t ldc, int d, cudaStream_t stre
 kronq_status launch_drift_split(const void* xfp, int64_t ld_xfp, const void* xq, int64_t ld_xq,
                                 int64_t rows, int cols, void* hi, void* lo, int64_t ld_out,
                                 cudaStream_t stream);
+size_t accumulate_diag_workspace_bytes(int64_t n, int d);
+kronq_status launch_accumulate_diag(const void* g, int64_t ld, int64_t n, int d, float* diag_sum,
+                                    void* ws, cudaStream_t stream);
 
 // biip.cu
 struct BiipArgs {

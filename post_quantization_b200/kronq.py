@@ -33,6 +33,7 @@ BIIP_SCALE_OUT = 2
 BIIP_ROTATE_IN = 4
 BIIP_ROTATE_OUT = 8
 BIIP_WRITE_HG = 16
+BIIP_HG_DIAG = 32
 BIIP_FULL = 15
 
 CHOLINV_SYNC = 1
@@ -42,6 +43,7 @@ SYMBOLS = (
     "kronq_status_string", "kronq_last_error_detail", "kronq_version", "kronq_device_check",
     "kronq_device_error", "kronq_launch_count", "kronq_set_sm_budget", "kronq_sm_budget",
     "kronq_accumulate_workspace_size", "kronq_accumulate",
+    "kronq_accumulate_diag_workspace_size", "kronq_accumulate_diag",
     "kronq_biip_workspace_size", "kronq_biip", "kronq_biip_noalloc",
     "kronq_cholinv_workspace_size", "kronq_cholinv",
     "kronq_quantize_layer_workspace_size", "kronq_quantize_layer",
@@ -91,6 +93,9 @@ def load_library(path: str = LIB_PATH):
         "kronq_accumulate": (c_i32, [c_void_p, c_i64, c_void_p, c_i64, c_void_p, c_i64, c_i64,
                                      c_i32, c_i32, c_void_p, c_void_p, c_void_p, c_void_p, c_sz,
                                      c_void_p]),
+        "kronq_accumulate_diag_workspace_size": (c_sz, [c_i64, c_i32]),
+        "kronq_accumulate_diag": (c_i32, [c_void_p, c_i64, c_i64, c_i32, c_void_p, c_void_p, c_sz,
+                                          c_void_p]),
         "kronq_biip_workspace_size": (c_sz, [c_i32, c_i32]),
         "kronq_biip": (c_i32, [c_void_p, c_i32, c_void_p, c_void_p, c_void_p, c_void_p, c_dbl,
                                c_void_p, c_void_p, c_i32, c_i32, c_u32, c_void_p, c_void_p,
@@ -217,6 +222,20 @@ def kronq_accumulate(xq=None, xfp=None, g=None, hx_sum=None, hg_sum=None, dxx_su
                               _rowstride(g), n, d_in, d_out, _p(hx_sum), _p(hg_sum),
                               _p(dxx_sum), _p(ws), wsb, _stream(stream))
     _check(st, "kronq_accumulate")
+
+
+def kronq_accumulate_diag_workspace_size(n: int, d: int) -> int:
+    return load_library().kronq_accumulate_diag_workspace_size(n, d)
+
+
+def kronq_accumulate_diag(g, diag_sum, workspace=None, stream=None):
+    """diag_sum[j] += sum_t g[t, j]^2 (the diagonal of g^T g; bf16 in, fp32 sums)."""
+    lib = load_library()
+    n, d = g.shape
+    ws, wsb = _workspace(lib.kronq_accumulate_diag_workspace_size(n, d), g.device, workspace)
+    st = lib.kronq_accumulate_diag(_p(g), _rowstride(g), n, d, _p(diag_sum), _p(ws), wsb,
+                                   _stream(stream))
+    _check(st, "kronq_accumulate_diag")
 
 
 # ------------------------------------------------------------------------------ 2. biip

@@ -56,6 +56,13 @@ def accumulate(xq=None, xfp=None, g=None, hx_sum=None, hg_sum=None, dxx_sum=None
                        workspace=ws.get(wsz) if ws is not None else None, stream=stream)
 
 
+def accumulate_diag(g, hg_diag_sum, ws=None, stream=None):
+    """hg_diag_sum += the diagonal of g^T g (for biip with K.BIIP_HG_DIAG)."""
+    wsz = K.kronq_accumulate_diag_workspace_size(g.shape[0], g.shape[1])
+    K.kronq_accumulate_diag(g, hg_diag_sum, workspace=ws.get(wsz) if ws is not None else None,
+                            stream=stream)
+
+
 def biip(w, hx_sum, hg_sum, dxx_sum, inv_n, sign_in, sign_out, flags=K.BIIP_FULL, ws=None,
          stream=None, copy_hx=True):
     """Runs kronq_biip on copies of the sums (hx is copied unless copy_hx is False)."""

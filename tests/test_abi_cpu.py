@@ -64,6 +64,9 @@ def test_workspace_queries(K):
     assert K.kronq_accumulate_workspace_size(1000, 256, 256, False) == 0
     assert K.kronq_accumulate_workspace_size(1000, 256, 256, True) > 0
     assert K.kronq_biip_workspace_size(0, 5) == 0
+    # diagonal sums: one fp32 partial per column and block of 2048 tokens
+    assert K.kronq_accumulate_diag_workspace_size(4097, 100) == 3 * 100 * 4
+    assert K.kronq_accumulate_diag_workspace_size(0, 100) == 0
 
 
 def test_sm_budget_is_host_state(K):
@@ -105,6 +108,17 @@ def test_argument_errors_before_device(K):
     assert lib.kronq_accumulate(256, 16, None, 0, None, 0, 10, 12, 0, None, None, None, None, 0,
                                 None) == K.ERR_INVALID_ARG
     assert "no output" in lib.kronq_last_error_detail().decode()
+    # accumulate_diag: missing output, bad width, misaligned stride, short workspace
+    assert lib.kronq_accumulate_diag(256, 16, 10, 16, None, None, 0, None) == K.ERR_INVALID_ARG
+    assert lib.kronq_accumulate_diag(256, 16, 10, 0, 512, None, 0, None) == K.ERR_SHAPE
+    assert lib.kronq_accumulate_diag(256, 12, 10, 12, 512, None, 0, None) == K.ERR_INVALID_ARG
+    assert lib.kronq_accumulate_diag(256, 16, 10, 16, 512, None, 0, None) == K.ERR_WORKSPACE
+    assert lib.kronq_accumulate_diag(256, 16, 0, 16, 512, None, 0, None) == K.OK   # n = 0
+    # biip: the diagonal form of H_G needs hg and cannot be written back
+    assert lib.kronq_biip(*args, K.BIIP_HG_DIAG, *tail) == K.ERR_INVALID_ARG
+    withhg = list(args); withhg[4] = 128
+    assert lib.kronq_biip(*withhg, K.BIIP_HG_DIAG | K.BIIP_WRITE_HG, *tail) == K.ERR_INVALID_ARG
+    assert "diagonal" in lib.kronq_last_error_detail().decode()
 
 
 def test_inference_calls_host_checks(K):

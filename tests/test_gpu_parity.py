@@ -133,6 +133,28 @@ def test_accumulate_llama_width_sampled(K, d):
     assert abs(float(torch.trace(h.double())) - tr) <= TOL * tr
 
 
+@pytest.mark.parametrize("n,d", [(5000, 4096), (3000, 200), (77, 36), (4100, 11008)])
+def test_accumulate_diag_matches_oracle(K, n, d):
+    # diag(G^T G) in one streaming pass: against the oracle's sums, and against the diagonal of
+    # the tensor-core G^T G; "+=" onto a non-zero start; 2048-token blocks with a ragged last one,
+    # widths that end part-way through a lane's 8 columns (36, 200)
+    g = padded(synth.gradients(n, d, synth.seed_for("diag", n, d), device="cuda"))
+    start = torch.rand(d, device="cuda")
+    dg = start.clone()
+    K.kronq_accumulate_diag(g, dg)
+    hg = torch.zeros(d, d, device="cuda")
+    K.kronq_accumulate(None, None, g, None, hg)
+    torch.cuda.synchronize()
+    o = O.accumulate_diag(h64(g))
+    assert rel(h64(dg) - h64(start), o) <= TOL
+    assert rel(h64(dg) - h64(start), h64(torch.diagonal(hg))) <= TOL
+    dg2 = start.clone()
+    K.kronq_accumulate_diag(g, dg2)
+    torch.cuda.synchronize()
+    assert torch.equal(dg, dg2)                      # fixed summation order
+    assert K.kronq_device_error() == 0
+
+
 # ------------------------------------------------------------------------------ biip
 
 def run_biip(K, P, w, hx_sum, hg_sum, dxx_sum, inv_n, si, so, flags):
@@ -199,6 +221,29 @@ def test_biip_col_pass_ragged(K, P, d_out, d_in):
     assert rel(h64(r.w_prime), o["w"]) <= TOL
     assert rel(h64(r.hx), o["hx"]) <= TOL
     assert rel(h64(hg_in), o["hg"]) <= TOL
+    assert abs(float(r.tr[1]) - o["tr_hg"]) <= TOL * abs(o["tr_hg"])
+    assert K.kronq_device_error() == 0
+
+
+@pytest.mark.parametrize("shape", [(256, 384), (11008, 256)])
+def test_biip_with_diagonal_hg(K, P, shape):
+    # KRONQ_BIIP_HG_DIAG: only diag(G^T G) from kronq_accumulate_diag; W', H_X', S_G and the
+    # traces against the oracle run on that diagonal
+    d_out, d_in = shape
+    n = 1024
+    xq, xfp, g, w, si, so = layer_inputs(d_out, d_in, n, w_dtype=torch.bfloat16,
+                                         tag=("biip-diag", d_out, d_in))
+    hx = torch.zeros(d_in, d_in, device="cuda")
+    K.kronq_accumulate(xq, None, None, hx)
+    hgd = torch.zeros(d_out, device="cuda")
+    K.kronq_accumulate_diag(g, hgd)
+    torch.cuda.synchronize()
+    r = run_biip(K, P, w, hx, hgd, None, 1.0 / n, si, so, K.BIIP_FULL | K.BIIP_HG_DIAG)
+    o = O.biip(h64(w), h64(hx), np.diag(h64(hgd)), None, 1.0 / n, h64(si), h64(so), 15)
+    assert rel(h64(r.w_prime), o["w"]) <= TOL
+    assert rel(h64(r.hx), o["hx"]) <= TOL
+    assert rel(h64(r.s_g), o["s_g"]) <= TOL and rel(h64(r.s_x), o["s_x"]) <= TOL
+    assert abs(float(r.tr[0]) - o["tr_hx"]) <= TOL * abs(o["tr_hx"])
     assert abs(float(r.tr[1]) - o["tr_hg"]) <= TOL * abs(o["tr_hg"])
     assert K.kronq_device_error() == 0
 

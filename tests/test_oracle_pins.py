@@ -60,6 +60,38 @@ def test_accumulate_trace_symmetry_psd():
     assert np.linalg.eigvalsh(hx).min() > -1e-12
 
 
+def test_accumulate_diag_closed_form():
+    # G_tj = (t + 1)(j + 1)  =>  sum_t G_tj^2 = (j + 1)^2 n (n + 1)(2n + 1) / 6
+    n, d = 11, 6
+    t = np.arange(1, n + 1, dtype=np.float64)[:, None]
+    j = np.arange(1, d + 1, dtype=np.float64)[None, :]
+    got = O.accumulate_diag(t * j)
+    np.testing.assert_allclose(got, (j[0] ** 2) * n * (n + 1) * (2 * n + 1) / 6, rtol=1e-15)
+
+
+def test_biip_needs_only_the_diagonal_of_hg():
+    # S_G = diag(H_G,ii / |W_i,:|^2)^(1/4) and tr(H_G') = sum_i H_G,ii / s_i^2 read only the
+    # diagonal ([KronQ-hyper] Method: BiIP equations, sensitivity): BiIP with diag(H_G) alone
+    # gives the same W', H_X', S_G and traces as with the full H_G; and the diagonal sums equal
+    # the diagonal of the full (brute-force pinned) G^T G.
+    r = rng(31)
+    n, d_out, d_in = 40, 16, 8
+    x = r.standard_normal((n, d_in)); g = r.standard_normal((n, d_out)) * r.uniform(0.1, 3, d_out)
+    w = r.standard_normal((d_out, d_in))
+    hx, hg, _ = O.accumulate(x, None, g)
+    dg = O.accumulate_diag(g)
+    np.testing.assert_allclose(dg, np.diag(hg), rtol=1e-13)
+    si = np.where(r.standard_normal(d_in) > 0, 1.0, -1.0)
+    so = np.where(r.standard_normal(d_out) > 0, 1.0, -1.0)
+    full = O.biip(w, hx, hg, None, 1.0 / n, si, so, O.BIIP_FULL)
+    diag = O.biip(w, hx, np.diag(dg), None, 1.0 / n, si, so, O.BIIP_FULL)
+    for key in ("w", "hx", "s_x", "s_g"):
+        np.testing.assert_allclose(diag[key], full[key], rtol=1e-12, atol=1e-14)
+    assert abs(diag["tr_hg"] - full["tr_hg"]) <= 1e-12 * abs(full["tr_hg"])
+    assert abs(diag["tr_hx"] - full["tr_hx"]) <= 1e-12 * abs(full["tr_hx"])
+    assert not np.allclose(diag["hg"], full["hg"])          # the off-diagonal part is not there
+
+
 def test_drift_term_sign_for_shrunk_input():
     # x~ = (1 - eps) x  =>  D = sum (x - x~) x~^T = eps (1 - eps) X^T X
     r = rng(3)
