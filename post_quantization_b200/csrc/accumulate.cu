@@ -447,12 +447,9 @@ kronq_status launch_accumulate_tc(const void* a, int64_t ld_a, const void* b, in
   p.err = device_error_word();
   if (!p.err) return fail(KRONQ_ERR_CUDA, "device error word unavailable");
 
-  static bool attr_set = false;
-  if (!attr_set) {
-    KQ_CUDA_TRY(cudaFuncSetAttribute(accumulate_tc_kernel,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
-    attr_set = true;
-  }
+  // per device and cheap on the host, so set on every launch
+  KQ_CUDA_TRY(cudaFuncSetAttribute(accumulate_tc_kernel,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
   const int budget = sm_budget();
   const int grid = p.num_units < budget ? p.num_units : budget;
   accumulate_tc_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(ma, mb, p);

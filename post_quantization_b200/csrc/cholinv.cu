@@ -570,12 +570,9 @@ kronq_status run_cholinv(float* a, int d, float damp_rel, int32_t* info, void* w
     prep_kernel<<<grid, 256, 0, stream>>>(a, d, lam);
     KQ_TRY(check_launch("prep_kernel"));
   }
-  static bool attr = false;
-  if (!attr) {
-    KQ_CUDA_TRY(cudaFuncSetAttribute(leaf_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     static_cast<int>(LEAF_SMEM)));
-    attr = true;
-  }
+  // per device and cheap on the host, so set on every call
+  KQ_CUDA_TRY(cudaFuncSetAttribute(leaf_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   static_cast<int>(LEAF_SMEM)));
   Ctx c{d, t, info, stream};
   return chol_inv_rec(c, a, d, 0, p);
 }

@@ -370,13 +370,10 @@ kronq_status run_quantize(const float* w, const float* k, const float* dxx, int 
     }
   }
 
-  static bool attr = false;
   const size_t smem = sizeof(float) * (QB * KS_LD + QROWS * E_LD + QB);
-  if (!attr) {
-    KQ_CUDA_TRY(cudaFuncSetAttribute(block_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)smem));
-    attr = true;
-  }
+  // per device and cheap on the host, so set on every call
+  KQ_CUDA_TRY(cudaFuncSetAttribute(block_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)smem));
   // Two-level lazy updates: after a 128-column block only the rest of its super-block is
   // updated (K = 128); after a super-block, the rest of W at once (K = QSB), so the fp32 W is
   // read and written once per super-block instead of once per block.

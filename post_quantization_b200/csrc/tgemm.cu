@@ -404,12 +404,9 @@ kronq_status tgemm(int m, int n, int k, float alpha, Split3 a, Split3 b, bool b_
   p.skip = skip;
   p.err = device_error_word();
   if (!p.err) return fail(KRONQ_ERR_CUDA, "device error word unavailable");
-  static bool attr = false;
-  if (!attr) {
-    KQ_CUDA_TRY(cudaFuncSetAttribute(tgemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     SMEM_BYTES));
-    attr = true;
-  }
+  // per device and cheap on the host, so set on every launch
+  KQ_CUDA_TRY(cudaFuncSetAttribute(tgemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   SMEM_BYTES));
   // As few CTAs as the minimal number of tile waves needs: each CTA holds a whole SM (shared
   // memory), and SMs this GEMM does not need stay free for other streams' work.
   const int tiles = p.tiles_m * p.tiles_n;
