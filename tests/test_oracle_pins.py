@@ -347,6 +347,48 @@ def test_p_matrix_structure_and_drift_cancellation():
     np.testing.assert_allclose(full, w / (1 - eps), rtol=1e-9)
 
 
+def test_p_matrix_golden_cases():
+    # [KronQ-hyper] Method, OBS update: the W_:,p [P]_p,p+1: term. P = striu(D K^T) K is the
+    # reading of the undefined GPTAQ matrix (causal part of the exact shift w D (H + lambda I)^-1);
+    # the cases are worked by hand in tests/golden/p_matrix_cases.json. A transposed or swapped
+    # operand (K striu(D K^T), striu(K^T D) K, striu(D K) K, striu(M) K^T) or a non-strict
+    # triangle changes at least one entry of these small-integer cases.
+    with open(os.path.join(GOLDEN, "p_matrix_cases.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        k = np.array(c["k"], dtype=np.float64)
+        d = np.array(c["d"], dtype=np.float64)
+        p = O.p_matrix(d, k)
+        np.testing.assert_array_equal(p, np.array(c["p"], dtype=np.float64), err_msg=c["name"])
+        w = np.array(c["w"], dtype=np.float64)
+        np.testing.assert_array_equal(w @ (np.eye(3) + p), np.array(c["w_preshift"], dtype=np.float64),
+                                      err_msg=c["name"])
+
+
+@pytest.mark.parametrize("seed", [64, 65, 66])
+def test_p_matrix_is_causal_part_of_exact_shift(seed):
+    # [KronQ-hyper] Method, OBS update, with the reading of P as the causal part of the exact
+    # row shift w D (H + lambda I)^-1. In the K basis (right-multiplying by K^-1) that shift is
+    # w D (H + lambda I)^-1 K^-1; P K^-1 must equal its strictly upper part and vanish on and
+    # below the diagonal. (H + lambda I)^-1 is taken from a plain matrix inverse here, not from
+    # K, so a slip in how p_matrix combines D and K cannot cancel out.
+    r = rng(seed)
+    d = 7
+    h = spd(r, d, cond=50.0)
+    lam = O.damping(h, 0.01)
+    dxx = r.standard_normal((d, d))
+    k = O.cholinv(h, 0.01)
+    p = O.p_matrix(dxx, k)
+    kinv = np.linalg.inv(k)
+    shift = dxx @ np.linalg.inv(h + lam * np.eye(d)) @ kinv
+    got = p @ kinv
+    np.testing.assert_allclose(got, np.triu(shift, 1), rtol=0, atol=1e-10 * np.abs(shift).max())
+    # the full (untruncated) shift recovers the exact optimum w + w D (H + lambda I)^-1
+    w = r.standard_normal((3, d))
+    np.testing.assert_allclose(w + (w @ dxx @ k.T) @ k,
+                               w + w @ dxx @ np.linalg.inv(h + lam * np.eye(d)), rtol=1e-9)
+
+
 def _plain_gptq(w, k, bits):
     scale, zero = O.grid(w, bits)
     cur = w.copy(); codes = np.zeros(w.shape)
