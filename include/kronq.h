@@ -289,18 +289,22 @@ KRONQ_API kronq_status kronq_score_allocate(const double* tr_hx, const double* t
  * returns codes, scale, zero with W^' = scale (codes - zero); in the original basis the layer is
  *     y = S_G^-1 U^T W^' V S_X^-1 x,
  * computed here without forming W^ or W^' in memory: x is transformed, multiplied by the
- * packed codes on the tensor cores (dequantized on the fly in shared memory), and the result
- * transformed back.
+ * packed codes as 8-bit integers, and the result transformed back.
  *
  * Packed code format (this library's storage, the pages fix none). Bits b = 2, 3 or 4. Rows
  * are cut into tiles of 128 and columns into groups of 128 (past the matrix: code 0). Tile t,
  * group g is one blob of 2048 b bytes at byte offset (t G + g) 2048 b, G = ceil(d_in / 128).
- * Inside it, row r takes 16 b bytes at offset 16 b r, read as little-endian 32-bit words w[];
- * each word's low 16 bits hold codes of even columns, its high 16 bits codes of odd columns:
- *   b = 2, 4: column 16 k + 2 s + h (s = 0..7, h = 0, 1) at word k b/2 + floor(s b / 16),
- *             bits 16 h + (s b mod 16) and up;
- *   b = 3:    column 32 k + 2 s + h (s = 0..15): s < 15 at word 3 k + floor(s / 5), bits
- *             16 h + 3 (s mod 5) and up; s = 15: code bit i at bit 16 h + 15 of word 3 k + i.
+ *   Row strings: row r (0..127) of the blob owns a string of 16 b bytes, read as little-endian
+ *   32-bit words w[0 .. 4b-1]. The string is stored in 8-byte pieces: byte 8 p + k of row r's
+ *   string (p = 0 .. 2b-1, k = 0..7) is blob byte 1024 p + 8 r + k, so the 32 rows a warp
+ *   reads at once are contiguous.
+ *   Codes in the words: the code of column c (0..127 within the group) sits in byte lane
+ *   j = c mod 4 of its word, so one mask gives the codes of four consecutive columns:
+ *     b = 2: word floor(c / 16), bits 8 j + 2 q and 8 j + 2 q + 1, q = floor((c mod 16) / 4);
+ *     b = 4: word floor(c / 8), bits 8 j + 4 q .. 8 j + 4 q + 3, q = floor((c mod 8) / 4);
+ *     b = 3: with m = floor(c / 32), e = c mod 32: code bits 0 and 1 as for b = 2 in word
+ *            3 m + floor(e / 16) (q = floor((e mod 16) / 4)); code bit 2 in word 3 m + 2 at
+ *            bit 8 j + floor(e / 4).
  * ------------------------------------------------------------------------------------- */
 /* Size in bytes of the packed form of a d_out x d_in code matrix (0 for an unsupported b). */
 KRONQ_API size_t kronq_packed_codes_bytes(int32_t d_out, int32_t d_in, int32_t bits);
@@ -334,10 +338,14 @@ KRONQ_API kronq_status kronq_pack_grid(const float* scale, const float* zero, in
  *            _SCALE_OUT, _ROTATE_IN, _ROTATE_OUT; a flag that is off drops its factor and its
  *            pointer may be NULL). Hadamard blocks up to 16384.
  *   y        (device, fp32) n_tok x d_out, row stride ld_y (>= d_out)
- *   Tokens are processed 32 at a time; each group of 32 reads the packed codes once. Deterministic:
- *   the same inputs give the same bits. Arithmetic: x' = V S_X^-1 x in fp32, split into two bf16
- *   terms; codes exact in bf16; products on tcgen05 tensor cores with fp32 accumulation; the
- *   grid, zero point and output transforms in fp32.
+ *   Tokens are processed 32 at a time; each pass of up to 32 tokens reads the packed codes
+ *   once. Deterministic: the same inputs give the same bits.
+ *   Arithmetic: x' = V S_X^-1 x in fp32; each 128-column group of x' and each token is written
+ *   as three int8 terms, x' ~ s (q0 + q1 / 128 + q2 / 128^2) with a power-of-two s per group and
+ *   token (relative error about 1e-6 of the group's largest entry). The codes multiply the terms
+ *   exactly in int32: with 1 or 2 tokens on the CUDA cores (dp4a, u8 codes x s8 terms), with 3
+ *   to 32 tokens on the tensor cores (tcgen05.mma kind::i8, codes as the A operand in tensor
+ *   memory). The grid, zero point, group scale and output transforms are applied in fp32.
  * ------------------------------------------------------------------------------------- */
 KRONQ_API size_t kronq_qlinear_workspace_size(int32_t d_out, int32_t d_in, int32_t n_tok);
 KRONQ_API kronq_status kronq_qlinear(const void* x, int32_t x_dtype, int64_t ld_x, int32_t n_tok,

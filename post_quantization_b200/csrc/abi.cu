@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <mutex>
 #include <vector>
 
 #include "common.cuh"
@@ -19,6 +20,7 @@ thread_local char g_detail[512] = "";
 __device__ int g_device_error_word = 0;
 constexpr int kMaxDevices = 64;
 int* g_err_ptr[kMaxDevices] = {nullptr};
+std::mutex g_err_mu;
 }  // namespace
 
 void set_detail(const char* fmt, ...) {
@@ -102,6 +104,9 @@ kronq_status encode_tiled_map(CUtensorMap* map, CUtensorMapDataType dtype, int r
 int* device_error_word() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  // the address is per device; host threads making their first call on one device together
+  // look it up under the lock
+  std::lock_guard<std::mutex> lock(g_err_mu);
   if (!g_err_ptr[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_device_error_word) != cudaSuccess) return nullptr;
@@ -266,6 +271,10 @@ kronq_status kronq_accumulate_diag(const void* g, int64_t ld_g, int64_t n, int32
   if (d <= 0) return fail(KRONQ_ERR_SHAPE, "d <= 0");
   if (!diag_sum) return fail(KRONQ_ERR_INVALID_ARG, "diag_sum is required");
   if (n == 0) return KRONQ_OK;
+  if (n > kMaxDiagTokens)
+    return fail(KRONQ_ERR_SHAPE, "n = %lld tokens exceeds the %lld tokens one call takes; "
+                "split the tokens over several calls (the sums add)", (long long)n,
+                (long long)kMaxDiagTokens);
   KQ_TRY(check_bf16_matrix(g, ld_g, d, "g"));
   KQ_TRY(check_ws(workspace, workspace_bytes, accumulate_diag_workspace_bytes(n, d)));
   KQ_TRY(kronq_device_check());

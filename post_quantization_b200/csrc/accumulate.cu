@@ -395,17 +395,6 @@ kronq_status make_map(CUtensorMap* map, const void* base, int64_t rows, int cols
                           CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-int num_sms() {
-  static int sms = 0;
-  if (!sms) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms <= 0) sms = 148;
-  }
-  return sms;
-}
-
 }  // namespace
 
 // C (m x n, fp32, ldc) += A^T B with A: k x m bf16 (ld_a), B: k x n bf16 (ld_b).
@@ -434,7 +423,7 @@ kronq_status launch_accumulate_tc(const void* a, int64_t ld_a, const void* b, in
   } else {
     p.num_tiles = p.tiles_m * p.tiles_n;
   }
-  const int sms = num_sms();
+  const int sms = device_sms();
   const int kblocks = static_cast<int>((k + BK - 1) / BK);
   // Token chunk per unit: about 16K tokens, fewer when there are too few tiles to fill the GPU.
   int per = 256;

@@ -17,6 +17,10 @@ kronq_status launch_drift_split(const void* xfp, int64_t ld_xfp, const void* xq,
                                 int64_t rows, int cols, void* hi, void* lo, int64_t ld_out,
                                 cudaStream_t stream);
 size_t accumulate_diag_workspace_bytes(int64_t n, int d);
+// tokens one kronq_accumulate_diag call takes: 2048 per block row of the grid, 65535 rows
+constexpr int64_t kMaxDiagTokens = 65535LL * 2048;
+// SM count of the current device (queried per call; 148 if the query fails)
+int device_sms();
 kronq_status launch_accumulate_diag(const void* g, int64_t ld, int64_t n, int d, float* diag_sum,
                                     void* ws, cudaStream_t stream);
 

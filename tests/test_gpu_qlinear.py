@@ -72,6 +72,49 @@ def test_pack_codes_bit_exact(K, bits, shape):
     np.testing.assert_array_equal(got, want)
 
 
+def _header_bit_positions(bits, d_in, row, col):
+    """Byte offset and bit of each code bit of (row, col), read off the packed-format text of
+    include/kronq.h (blob, 8-byte pieces of the row string, byte lanes of 32-bit words)."""
+    G = (d_in + 127) // 128
+    t, r = divmod(row, 128)
+    g, c = divmod(col, 128)
+    blob = (t * G + g) * 2048 * bits
+    j = c % 4
+    if bits == 2:
+        where = [(c // 16, 8 * j + 2 * ((c % 16) // 4) + i) for i in range(2)]
+    elif bits == 4:
+        where = [(c // 8, 8 * j + 4 * ((c % 8) // 4) + i) for i in range(4)]
+    else:
+        m, e = divmod(c, 32)
+        where = [(3 * m + e // 16, 8 * j + 2 * ((e % 16) // 4) + i) for i in range(2)]
+        where.append((3 * m + 2, 8 * j + e // 4))
+    out = []
+    for word, bit in where:
+        sbyte = 4 * word + bit // 8           # byte of the row string (little-endian words)
+        p, k = divmod(sbyte, 8)
+        out.append((blob + 1024 * p + 8 * r + k, bit % 8))
+    return out
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_pack_codes_follow_the_header_text(K, bits):
+    # one code at a time, all others zero: its bits must appear exactly where the format text
+    # of the C header puts them, and nowhere else
+    d_out, d_in = 300, 520
+    placements = [(0, 0), (1, 1), (127, 127), (128, 5), (37, 130), (299, 519), (64, 255),
+                  (5, 33), (200, 62)]
+    for row, col in placements:
+        value = (1 << bits) - 1 if (row + col) % 2 else (1 << (bits - 1)) | 1
+        c = torch.zeros(d_out, d_in, dtype=torch.uint8, device="cuda")
+        c[row, col] = value
+        got = K.kronq_pack_codes(c, bits).cpu().numpy()[:O.packed_bytes(d_out, d_in, bits)]
+        want = np.zeros_like(got)
+        for i, (byte, bit) in enumerate(_header_bit_positions(bits, d_in, row, col)):
+            if (value >> i) & 1:
+                want[byte] |= np.uint8(1 << bit)
+        np.testing.assert_array_equal(got, want, err_msg=f"bits {bits} at ({row}, {col})")
+
+
 @pytest.mark.parametrize("group", [0, 128])
 @pytest.mark.parametrize("shape", [(1, 1), (300, 520), (1024, 4096)])
 def test_pack_grid_bit_exact(K, group, shape):
