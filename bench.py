@@ -1,17 +1,20 @@
 """KronQ layer-path benchmark on B200.
 
-One step = the whole hot path over one LLaMA-2-7B-shaped transformer block (7 sublayers:
-q/k/v/o 4096x4096, gate/up 11008x4096, down 4096x11008; 262144 calibration tokens; 4-bit
-per-channel grid; BiIP on; X~ = X so the drift term is off):
-  Kronecker-factor sums for the 4 distinct inputs (q/k/v share one) and the 7 output-gradient
-  streams -> BiIP of every sublayer -> traces to the host -> scores and bit allocation ->
-  damped inverse factor -> column solve of every sublayer. The per-sublayer steps of the 7
-  sublayers run side by side on one CUDA stream each.
+One step = the whole hot path over one LLaMA-3-70B-shaped transformer block (7 sublayers:
+q/o 8192x8192, k/v 1024x8192, gate/up 28672x8192, down 8192x28672; 262144 calibration tokens;
+2-bit per-channel grid; BiIP on; X~ = X + N(0, (0.05 rms X)^2), so the drift term and the GPTAQ
+pre-shift are active):
+  Kronecker-factor sums (H_X and the drift sum D for the 4 distinct inputs - q/k/v share one,
+  gate/up share one - and H_G for the 7 output-gradient streams) -> BiIP of every sublayer ->
+  traces to the host -> scores and bit allocation -> damped inverse factor -> P pre-shift and
+  column solve of every sublayer. The per-sublayer steps run side by side, one CUDA stream each.
 Metric: quantized weight params/s (whole job: params of all ranks' blocks / max step time).
 Each rank quantizes its own block (weak scaling, no collective on the data path).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
 
+--workload llama2_7b_block / llama3_8b_block select the smaller blocks; llama2_7b_stack runs
+the 32-block mixed-precision stack (see run_stack).
 --impl reference times the fp64 CPU oracle on a bounded sample of the same workload (see
 oracle_sample) on the host cores.
 """
@@ -30,7 +33,7 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-WORKLOAD = "llama2_7b_block"
+WORKLOAD = "llama3_70b_block"
 
 
 def parse():
@@ -41,11 +44,14 @@ def parse():
     ap.add_argument("--impl", default="kronq", choices=["kronq", "reference"])
     ap.add_argument("--tokens", type=int, default=None, help=argparse.SUPPRESS)
     ap.add_argument("--workload", default=WORKLOAD,
-                    choices=["llama2_7b_block", "llama3_8b_block", "llama3_70b_block"],
-                    help="block shape (default: the LLaMA-2-7B block the metric is quoted on)")
-    ap.add_argument("--no-graphs", action="store_true",
-                    help="enqueue the per-sublayer phases eagerly instead of replaying CUDA "
-                         "graphs (each graph keeps its own copies of the phase's outputs)")
+                    choices=["llama2_7b_block", "llama3_8b_block", "llama3_70b_block",
+                             "llama2_7b_stack"],
+                    help="block shape (default: the LLaMA-3-70B block)")
+    ap.add_argument("--graphs", default="auto", choices=["auto", "on", "off"],
+                    help="replay the per-sublayer phases as CUDA graphs (each graph keeps its own "
+                         "copies of the phase's outputs); auto: on when the block's inputs "
+                         "take less than 60 GB of device memory")
+    ap.add_argument("--no-graphs", action="store_true", help=argparse.SUPPRESS)
     ap.add_argument("--overlap", type=int, default=0, metavar="SMS",
                     help="run each sublayer's BiIP and inverse factor alongside the remaining "
                          "statistics on SMS reserved SMs (0: phases one after another)")
@@ -56,69 +62,146 @@ def parse():
 
 # ---------------------------------------------------------------------------------- oracle
 
-def oracle_sample(seconds_hint: float = 12.0):
-    """Time the fp64 oracle on a bounded sample of the block and scale it to one full step.
+PROXY_D = 2048        # proxy sublayer of the oracle sample: d_out = d_in = 2048
+PROXY_TOKENS = 8192
+PROXY_ROWS = 128
 
-    Sample: q_proj (4096 x 4096) with 4096 calibration tokens for the statistics, the whole
-    BiIP and damped inverse factor of that sublayer, and the column solve of 32 output rows.
-    Each stage's time is scaled to the full block by its work ratio (accumulation ~ N d^2 per
-    stream, BiIP ~ dense Hadamard cost, inverse ~ d^3, solve ~ d_out d_in^2).
-    Returns (estimated seconds per full step, description, threads).
-    """
-    import numpy as np
-    import torch
+
+def _biip_flops(d_out, d_in, drift):
+    """Flops of the oracle's BiIP: dense b x b Hadamard-block products on each side of W, on both
+    sides of H_X (and D), and of H_G."""
+    bi = d_in & -d_in
+    bo = d_out & -d_out
+    f = 2 * d_out * d_in * (bi + bo) + 4 * d_in * d_in * bi + 4 * d_out * d_out * bo
+    return f + (4 * d_in * d_in * bi if drift else 0)
+
+
+def cpu_info():
+    model = ""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
     from threadpoolctl import threadpool_info
+    threads = max([int(i.get("num_threads", 0)) for i in threadpool_info()] or [0])
+    return model, os.cpu_count() or 1, threads or (os.cpu_count() or 1)
 
+
+def oracle_layer256():
+    """The 256 x 256 layer (2048 tokens, 2 bits, drift term on) through the whole oracle, BiIP on
+    and off: seconds per stage."""
+    from oracle import kronq_oracle as O
+    from post_quantization_b200 import synth
+    tag = ("bench-oracle", "layer256")
+    d, n = 256, 2048
+    xt = synth.correlated_x(n, d, synth.seed_for(tag, "X"))
+    xfp = xt.double().numpy()
+    xq = synth.perturbed(xt, synth.seed_for(tag, "Xq"), abs_std=0.01).double().numpy()
+    g = synth.gradients(n, d, synth.seed_for(tag, "G")).double().numpy()
+    w = synth.weight(d, d, synth.seed_for(tag, "W"), dtype=__import__("torch").float32).double().numpy()
+    si = synth.rademacher(d, synth.seed_for(tag, "si")).numpy()
+    so = synth.rademacher(d, synth.seed_for(tag, "so")).numpy()
+    out = {}
+    for name, flags in (("biip_on", O.BIIP_FULL), ("biip_off", 0)):
+        t = {}
+        t0 = time.perf_counter()
+        hx, hg, dxx = O.accumulate(xq, xfp, g)
+        t["statistics"] = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        b = O.biip(w, hx, hg, dxx, 1.0 / n, si, so, flags)
+        t["biip"] = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        k = O.cholinv(b["hx"], 0.01)
+        t["cholinv"] = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        O.quantize_layer(b["w"], k, b["dxx"], 2)
+        t["solve"] = time.perf_counter() - t0
+        out[name] = {key: round(v, 4) for key, v in t.items()}
+    return out
+
+
+def oracle_sample(wl_name: str = WORKLOAD):
+    """Time the fp64 oracle, stage by stage, on a proxy sublayer and report its measured rates.
+
+    Sample: a 2048 x 2048 sublayer (one Hadamard block per side, like the hidden-size sublayers)
+    with 8192 calibration tokens: the statistics (with the drift sum when the workload has it),
+    the whole BiIP, the damped inverse factor, GPTAQ's P (drift workloads), and the column solve
+    of 128 output rows (rows are independent given K). Each stage gives a measured rate: GFLOP/s
+    of the oracle's own arithmetic for the statistics and BiIP, seconds at d = 2048 for the
+    inverse factor and P, rows/s for the solve.
+
+    The block estimate divides the block's work in each stage by that stage's measured rate:
+    statistics and BiIP by their flop counts, the inverse factor and P by d_in^3, the solve by
+    d_out d_in^2. It is an estimate, labelled as one; the measured quantities are the rates.
+    Returns (estimated seconds per block step, record dict, seconds spent measuring).
+    """
     from oracle import kronq_oracle as O
     from post_quantization_b200 import synth
 
-    wl = synth.WORKLOADS[WORKLOAD]
-    d = 4096
-    n_s = 4096
-    rows = 32
-    tag = ("bench-oracle",)
-    x = synth.correlated_x(n_s, d, synth.seed_for(tag, "X")).double().numpy()
+    wl = synth.WORKLOADS[wl_name]
+    drift = wl.drift != "none"
+    d, n_s, rows = PROXY_D, PROXY_TOKENS, PROXY_ROWS
+    tag = ("bench-oracle", wl_name)
+    xt = synth.correlated_x(n_s, d, synth.seed_for(tag, "X"))
+    xfp = xt.double().numpy()
+    xq = (synth.perturbed(xt, synth.seed_for(tag, "Xq"), rel_std=0.05).double().numpy()
+          if drift else xfp)
+    del xt
     g = synth.gradients(n_s, d, synth.seed_for(tag, "G")).double().numpy()
     w = synth.weight(d, d, synth.seed_for(tag, "W")).double().numpy()
     si = synth.rademacher(d, synth.seed_for(tag, "si")).numpy()
     so = synth.rademacher(d, synth.seed_for(tag, "so")).numpy()
 
+    spent0 = time.perf_counter()
     t0 = time.perf_counter()
-    hx, hg, _ = O.accumulate(x, None, g)
+    hx, hg, dxx = O.accumulate(xq, xfp if drift else None, g)
     t_acc = time.perf_counter() - t0
     t0 = time.perf_counter()
-    b = O.biip(w, hx, hg, None, 1.0 / n_s, si, so, O.BIIP_FULL)
+    b = O.biip(w, hx, hg, dxx, 1.0 / n_s, si, so, O.BIIP_FULL)
     t_biip = time.perf_counter() - t0
     t0 = time.perf_counter()
     k = O.cholinv(b["hx"], 0.01)
     t_chol = time.perf_counter() - t0
+    t_p = 0.0
+    if drift:
+        t0 = time.perf_counter()
+        O.p_matrix(b["dxx"], k)
+        t_p = time.perf_counter() - t0
     t0 = time.perf_counter()
-    O.quantize_layer(b["w"][:rows], k, None, wl.bits)
-    t_q = time.perf_counter() - t0
+    O.quantize_layer(b["w"][:rows], k, b["dxx"] if drift else None, wl.bits)
+    t_q = time.perf_counter() - t0 - t_p         # quantize_layer forms P itself
+    t_q = max(t_q, 1e-9)
+    spent = time.perf_counter() - spent0
 
+    # measured rates
+    acc_fl = 2.0 * n_s * d * d * (3 if drift else 2)      # X~^T X~, G^T G (and D), full matrices
+    r_acc = acc_fl / t_acc
+    r_biip = _biip_flops(d, d, drift) / t_biip
+    rows_per_s = rows / t_q
+
+    # block estimate from those rates
     N = wl.n_tokens
-    # accumulation: this sample did one X and one G stream of width 4096 over n_s tokens
-    acc_work = sum(N * dd * dd for dd in wl.streams().values()) + \
-        sum(N * s.d_out * s.d_out for s in wl.sublayers)
-    acc_scale = acc_work / (2 * n_s * d * d)
-
-    def biip_cost(s):
-        bi = s.d_in & -s.d_in; bo = s.d_out & -s.d_out
-        return s.d_out * s.d_in * (bi + bo) + 2 * s.d_in * s.d_in * bi + 2 * s.d_out * s.d_out * bo
-
-    ref = synth.Sublayer("q", d, d, "x")
-    biip_scale = sum(biip_cost(s) for s in wl.sublayers) / biip_cost(ref)
-    chol_scale = sum(s.d_in ** 3 for s in wl.sublayers) / d ** 3
-    q_scale = sum(s.d_out * s.d_in ** 2 for s in wl.sublayers) / (rows * d * d)
-    est = t_acc * acc_scale + t_biip * biip_scale + t_chol * chol_scale + t_q * q_scale
-    threads = 0
-    for info in threadpool_info():
-        threads = max(threads, int(info.get("num_threads", 0)))
-    desc = (f"q_proj 4096x4096: statistics over {n_s} tokens, full BiIP and inverse factor, "
-            f"column solve of {rows} rows; stage times ({t_acc:.2f}s, {t_biip:.2f}s, "
-            f"{t_chol:.2f}s, {t_q:.2f}s) scaled by work ratios ({acc_scale:.0f}, "
-            f"{biip_scale:.1f}, {chol_scale:.1f}, {q_scale:.0f}) to one {WORKLOAD} step")
-    return est, desc, threads or (os.cpu_count() or 1), t_acc + t_biip + t_chol + t_q
+    e_acc = sum(2.0 * N * dd * dd * (2 if drift else 1) for dd in wl.streams().values())
+    e_acc += sum(2.0 * N * s.d_out * s.d_out for s in wl.sublayers)
+    est = e_acc / r_acc
+    est += sum(_biip_flops(s.d_out, s.d_in, drift) for s in wl.sublayers) / r_biip
+    est += sum((s.d_in / d) ** 3 for s in wl.sublayers) * t_chol
+    if drift:
+        est += sum((s.d_in / d) ** 3 for s in wl.sublayers) * t_p
+    est += sum(s.d_out * (s.d_in / d) ** 2 for s in wl.sublayers) / rows_per_s
+    rec = {
+        "statistics_gflops": round(r_acc / 1e9, 2),
+        "biip_gflops": round(r_biip / 1e9, 2),
+        f"cholinv_s_d{d}": round(t_chol, 3),
+        f"p_matrix_s_d{d}": round(t_p, 3) if drift else None,
+        f"solve_rows_per_s_d{d}": round(rows_per_s, 2),
+        "estimated_s_per_step": round(est, 1),
+    }
+    return est, rec, spent
 
 
 # ---------------------------------------------------------------------------------- clocks
@@ -233,18 +316,26 @@ class Block:
             tot += t.numel() * t.element_size()
         return tot
 
-    def step(self, time_acc=False, x_src=None, g_src=None):
+    def inputs(self):
+        """(kind, stream or sublayer name, device tensor) of every calibration input: X~, X (drift
+        workloads) and G."""
+        out = [("x", k, v) for k, v in self.x.items()]
+        if self.xfp:
+            out += [("xfp", k, v) for k, v in self.xfp.items()]
+        out += [("g", k, v) for k, v in self.g.items()]
+        return out
+
+    def step(self, time_acc=False):
         import torch
 
         from post_quantization_b200 import kronq as K
         from post_quantization_b200 import pipeline as P
         wl = self.wl
-        x = x_src or self.x
-        g = g_src or self.g
+        x, g = self.x, self.g
         if not self.use_graphs:
             self.results = {}       # eager phases allocate new outputs: drop the last step's
         if self.overlap:
-            self._step_overlapped(x, g, time_acc=time_acc)
+            self._step_overlapped(time_acc=time_acc)
             return
         for name, h in self.hx.items():
             h.zero_()
@@ -307,25 +398,26 @@ class Block:
                 lambda: self.streams.solve(res, bits, 0.01))
         self.solve_phases[key]()
 
-    def step_streamed(self, host_x, host_g, dev_x, dev_g, copy_stream):
-        """One step with the inputs in pinned host memory, as a user with host data runs it.
+    def step_streamed(self, host, copy_stream):
+        """One step with the inputs in page-locked host memory, as a user with host data runs it.
 
-        Every X / G copy goes over the host link on `copy_stream`, one tensor at a time, in the
-        order the overlapped step consumes them (longest inverse-factor chain first); each
-        statistic waits only for its own input.
+        host[(kind, name)] is the host copy of the device input of the same key (see inputs()).
+        Every copy goes over the host link on `copy_stream`, one tensor at a time, in the order
+        the overlapped step consumes them (longest inverse-factor chain first); each statistic
+        waits only for its own inputs.
         """
         import torch
         main = torch.cuda.current_stream()
+        dev = {(kind, name): t for kind, name, t in self.inputs()}
         landed = {}
         copy_stream.wait_stream(main)
-        for kind, name in self._consumption_order():
-            src, dst = (host_x, dev_x) if kind == "x" else (host_g, dev_g)
+        for key in self._consumption_order():
             with torch.cuda.stream(copy_stream):
-                dst[name].copy_(src[name], non_blocking=True)
+                dev[key].copy_(host[key], non_blocking=True)
                 ev = torch.cuda.Event()
                 ev.record(copy_stream)
-            landed[(kind, name)] = ev
-        self._step_overlapped(dev_x, dev_g, landed=landed)
+            landed[key] = ev
+        self._step_overlapped(landed=landed)
 
     def _chain_order(self):
         subs = self.wl.sublayers
@@ -339,10 +431,12 @@ class Block:
             if subs[i].x_stream not in seen:
                 seen.add(subs[i].x_stream)
                 seq.append(("x", subs[i].x_stream))
+                if self.drift:
+                    seq.append(("xfp", subs[i].x_stream))
             seq.append(("g", subs[i].name))
         return seq
 
-    def _step_overlapped(self, x, g, landed=None, time_acc=False):
+    def _step_overlapped(self, landed=None, time_acc=False):
         """Statistics, sublayer by sublayer (longest inverse-factor chain first), on all but
         `reserve` SMs; as soon as a sublayer's sums are complete its BiIP and inverse factor
         start on its own stream (a captured graph sized to the reserved SMs), alongside the
@@ -354,6 +448,7 @@ class Block:
         from post_quantization_b200 import pipeline as P
         wl = self.wl
         subs = wl.sublayers
+        x, g = self.x, self.g
         inv_n = 1.0 / self.n
         main = torch.cuda.current_stream()
         sms = torch.cuda.get_device_properties(self.dev).multi_processor_count
@@ -386,6 +481,8 @@ class Block:
                 done.add(sl.x_stream)
                 if landed is not None:
                     main.wait_event(landed[("x", sl.x_stream)])
+                    if self.drift:
+                        main.wait_event(landed[("xfp", sl.x_stream)])
                 h = self.hx[sl.x_stream]
                 h.zero_()
                 if self.drift:
@@ -489,7 +586,10 @@ def run_gpu(args):
     n_tok = args.tokens or wl.n_tokens
     ws = P.Workspace(dev)
     blk = Block(wl, rank, dev, n_tok, ws)
-    blk.use_graphs = not args.no_graphs
+    graphs = args.graphs
+    if args.no_graphs:
+        graphs = "off"
+    blk.use_graphs = graphs == "on" or (graphs == "auto" and blk.input_bytes() < 60e9)
     blk.overlap = args.overlap > 0
     blk.reserve = args.overlap
     torch.cuda.synchronize()
@@ -525,9 +625,9 @@ def run_gpu(args):
     params = wl.params_per_block * world
     value = params * args.steps / elapsed_max
 
-    # ---- end to end: host inputs (pinned), host->device copies and the result read-back
+    # ---- end to end: host inputs (page-locked), host->device copies and the result read-back
     e2e = None
-    if not args.no_e2e and not blk.drift:
+    if not args.no_e2e:
         e2e = run_e2e(blk, args, world, dist if world > 1 else None, barrier)
 
     result = None
@@ -542,13 +642,8 @@ def run_gpu(args):
         if not peak:
             peak = 1400.0
             peak_src = "fallback (sustained bf16)"
-        achieved = sum(acc_flops) / (sum(acc_ms) / 1e3) / 1e12
-        # DRAM bytes (read + write) per accumulate_tc_kernel launch, averaged over a step's 8
-        # launches at d = 4096 and 3 at d = 11008: ncu captures of this kernel version at
-        # d = 4096 / 262144 tokens (5.51 GB) and d = 11008 / 131072 tokens (21.2 GB, x2 for
-        # 262144 tokens); the accumulate summary under profiles/ has the commands
-        traffic = 15.6e9 if (args.workload == WORKLOAD and n_tok == 262144) else None
         acc_tflops = sum(acc_flops) / (sum(acc_ms) / 1e3) / 1e12
+        traffic = TRAFFIC.get((args.workload, n_tok))
         result = {
             "metric": "quantized weight params/s (BiIP+GPTAQ solve); H_X/H_G accumulate TFLOP/s",
             "value": value,
@@ -560,112 +655,340 @@ def run_gpu(args):
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
-            "dtype": "bf16 statistics, fp32 solve",
+            "dtype": "bf16 statistics (fp16 drift operands), fp32 solve",
             "data": "synthetic (seeded LLaMA-shaped activations, gradients and weights)",
             "config": {"workload": describe(wl, n_tok),
                        "tokens": n_tok, "params_per_block": wl.params_per_block,
                        "parallelism": f"one block per GPU x{world}",
+                       "graphs": blk.use_graphs,
                        "l2": f"inputs ({blk.input_bytes() / 1e9:.0f} GB) larger than L2"},
             "accumulate_tflops": acc_tflops,
             "roofline": {"bound": "tensor", "kernel": "accumulate_tc_kernel",
-                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "peak_source": peak_src, "traffic": traffic,
-                         "traffic_unit": "bytes per launch"},
+                         "achieved": acc_tflops, "peak": peak, "unit": "TFLOP/s",
+                         "frac": acc_tflops / peak, "peak_source": peak_src,
+                         "achieved_basis": "algorithmic flops of the statistics calls (N d(d+1) "
+                                           "per symmetric sum, 2 N d^2 per drift sum) / their "
+                                           "CUDA-event time",
+                         "traffic": traffic, "traffic_unit": "bytes per launch"},
             "gpu_launches": launches,
             "clocks": clk,
             "e2e": e2e,
         }
-        if not args.no_cpu_baseline and args.workload == WORKLOAD:
-            est, desc, threads, spent = oracle_sample()
-            result["cpu_baseline"] = {"value": wl.params_per_block / est, "unit": "params/s",
-                                      "cores": threads, "kind": "oracle", "sample": desc,
-                                      "sample_seconds": spent}
+        if not args.no_cpu_baseline:
+            samples = [oracle_sample(args.workload) for _ in range(3)]
+            est = statistics.mean(e for e, _, _ in samples)
+            rec = samples[-1][1]
+            spent = sum(sp for _, _, sp in samples)
+            model, nproc, threads = cpu_info()
+            result["cpu_baseline"] = {
+                "value": wl.params_per_block / est, "unit": "params/s", "cores": threads,
+                "kind": "oracle",
+                "value_kind": "estimate: the block's work per stage / the oracle's measured "
+                              "rate per stage (rates measured on the sample)",
+                "sample": (f"fp64 oracle on a {PROXY_D}x{PROXY_D} sublayer, {PROXY_TOKENS} "
+                           f"tokens: statistics, BiIP, inverse factor"
+                           + (", P" if blk.drift else "") +
+                           f", column solve of {PROXY_ROWS} rows; 3 samples, {spent:.1f} s"),
+                "rates": rec, "cpu_model": model, "nproc": nproc,
+                "layer256_full_s": oracle_layer256()}
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     return result
 
 
+# DRAM bytes (read + write) per accumulate_tc_kernel launch, averaged over the launches of one
+# step, from ncu captures of this kernel version (commands in the accumulate profile summary
+# under profiles/); keyed by (workload, tokens)
+TRAFFIC = {}
+
+
+def _mem_available():
+    try:
+        with open("/proc/meminfo") as f:
+            for line in f:
+                if line.startswith("MemAvailable:"):
+                    return int(line.split()[1]) * 1024
+    except OSError:
+        pass
+    return None
+
+
 def run_e2e(blk, args, world, dist, barrier):
-    """Same step through the same API, inputs starting in pinned host memory every step."""
+    """Same step through the same API, the inputs starting in page-locked host memory every
+    step: every X~, X and G tensor is copied to the device inside the timed region, and the
+    codes and grid of every sublayer are read back."""
     import torch
-    def pinned(v):
-        h = torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
-        h.copy_(v)
-        return h
+    # the streamed step runs the overlapped phases with their own outputs and workspaces: free
+    # the resident step's first (the LLaMA-3-70B block does not hold both sets)
+    blk.results = {}
+    blk.streams = None
+    blk.biip_phase = None
+    blk.solve_phases = {}
+    blk.solve_res = None
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    items = blk.inputs()
+    sizes = [t.numel() * t.element_size() for _, _, t in items]
+    offs, total = [], 0
+    for sz in sizes:
+        offs.append(total)
+        total += (sz + 4095) // 4096 * 4096
+    avail = _mem_available()
+    # one host buffer for all inputs, page-locked by registration (the pinned-tensor allocator
+    # would round each tensor up to a power of two)
+    if avail is not None and total > avail - 24e9:
+        return {"value": None, "unit": "params/s",
+                "skipped": f"needs {total / 1e9:.0f} GB of page-locked host memory, "
+                           f"{avail / 1e9:.0f} GB available"}
+    host_buf = torch.empty(total, dtype=torch.uint8)
+    cudart = torch.cuda.cudart()
+    rc = cudart.cudaHostRegister(host_buf.data_ptr(), total, 0)
+    if int(rc) != 0:
+        return {"value": None, "unit": "params/s", "skipped": f"cudaHostRegister failed ({rc})"}
+    try:
+        host = {}
+        for (kind, name, t), off, sz in zip(items, offs, sizes):
+            h = host_buf[off:off + sz].view(t.dtype).view(t.shape)
+            h.copy_(t)
+            host[(kind, name)] = h
+        assert all(h.is_pinned() for h in host.values())
+        h2d = sum(sizes)
+        # the device copies are written by every streamed step (same shapes, same addresses)
+        copy_stream = torch.cuda.Stream(device=blk.dev)
+        outs = None
 
-    host_x = {k: pinned(v) for k, v in blk.x.items()}
-    host_g = {k: pinned(v) for k, v in blk.g.items()}
-    dev_x = {k: torch.empty_like(v) for k, v in blk.x.items()}
-    dev_g = {k: torch.empty_like(v) for k, v in blk.g.items()}
-    # free the resident copies to keep device memory flat
-    blk.x = dev_x
-    blk.g = dev_g
-    h2d = sum(t.numel() * t.element_size() for t in list(host_x.values()) + list(host_g.values()))
-    d2h = 0
+        def one():
+            nonlocal outs
+            blk.step_streamed(host, copy_stream)
+            if outs is None:
+                outs = []
+                for sl in blk.wl.sublayers:
+                    r = blk.results[sl.name]
+                    outs += [torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+                             for t in (r.codes, r.scale, r.zero)]
+            k = 0
+            for sl in blk.wl.sublayers:
+                r = blk.results[sl.name]
+                for t in (r.codes, r.scale, r.zero):
+                    outs[k].copy_(t, non_blocking=True)
+                    k += 1
+            torch.cuda.current_stream().synchronize()
 
-    copy_stream = torch.cuda.Stream(device=blk.dev)
-
-    def one():
-        nonlocal d2h
-        blk.step_streamed(host_x, host_g, dev_x, dev_g, copy_stream)
-        outs = []
-        for s in blk.wl.sublayers:
-            r = blk.results[s.name]
-            outs.append(r.codes.to("cpu", non_blocking=True))
-            outs.append(r.scale.to("cpu", non_blocking=True))
-            outs.append(r.zero.to("cpu", non_blocking=True))
-        torch.cuda.current_stream().synchronize()
+        for _ in range(2):          # first step allocates and (with graphs) captures
+            one()
+        barrier()
+        steps = max(2, min(args.steps, 10))
+        e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            one()
+        e1.record()
+        barrier()
+        el = e0.elapsed_time(e1) / 1e3
         d2h = sum(o.numel() * o.element_size() for o in outs)
+        t = torch.tensor([el], dtype=torch.float64, device=blk.dev)
+        if dist is not None:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        value = blk.wl.params_per_block * world * steps / float(t)
+        return {"value": value, "unit": "params/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": steps,
+                "ms_per_step": float(t) / steps * 1e3}
+    finally:
+        torch.cuda.synchronize()
+        cudart.cudaHostUnregister(host_buf.data_ptr())
 
-    for _ in range(3):          # eager, capture, replay: the timed steps only replay
-        one()
+
+# ---------------------------------------------------------------------------------- stack
+
+def run_stack(args):
+    """The mixed-precision stack: 32 LLaMA-2-7B-shaped blocks (224 sublayers, 6.5B weights),
+    every sublayer with its own X and G (65536 tokens; per-block G scale log-uniform on
+    [1e-2, 1e1]). One step: statistics and BiIP of every sublayer, the traces of all 224 to the
+    host (gathered over ranks), one {2,3,4}-bit allocation at 2.5 average bits over the whole
+    stack, then the inverse factor and column solve of every sublayer with its width.
+
+    Blocks are split over ranks (strong scaling). The stack's calibration inputs (330 GB) do not
+    fit in device memory, so each sublayer's X and G are generated on the device just before its
+    statistics; the timed intervals (CUDA events on the one stream that runs everything) cover
+    the library calls only, and the step time is their sum.
+    """
+    import torch
+    import torch.distributed as dist
+
+    from post_quantization_b200 import build
+    from post_quantization_b200 import dist as D
+    from post_quantization_b200 import kronq as K
+    from post_quantization_b200 import pipeline as P
+    from post_quantization_b200 import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=600))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    K.load_library()
+    K.kronq_device_check()
+
+    wl = synth.WORKLOADS["llama2_7b_stack"]
+    n = args.tokens or wl.n_tokens
+    subs = wl.sublayers
+    lo, hi = wl.extra["g_block_multiplier_log10"]
+    blocks = D.shard(wl.n_blocks, rank, world)
+    sizes = [s.d_out * s.d_in for _ in range(wl.n_blocks) for s in subs]
+    owned = [b * len(subs) + j for b in blocks for j in range(len(subs))]
+    w, si, so, mult = {}, {}, {}, {}
+    for b in blocks:
+        mult[b] = synth.block_g_multiplier(b, lo, hi, synth.seed_for(wl.name))
+        for j, sl in enumerate(subs):
+            tag = (wl.name, b, sl.name)
+            i = b * len(subs) + j
+            w[i] = synth.weight(sl.d_out, sl.d_in, synth.seed_for(tag, "W"), device=dev)
+            si[i] = synth.rademacher(sl.d_in, synth.seed_for(tag, "si"), device=dev)
+            so[i] = synth.rademacher(sl.d_out, synth.seed_for(tag, "so"), device=dev)
+    ws = P.Workspace(dev)
+    streams = P.SublayerStreams(len(subs), dev)
+    state = {"bits": None}
+
+    def step():
+        timed = []
+        res = {}
+
+        def timed_call(fn):
+            e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            out = fn()
+            e1.record()
+            timed.append((e0, e1))
+            return out
+
+        for b in blocks:
+            for j, sl in enumerate(subs):
+                i = b * len(subs) + j
+                tag = (wl.name, b, sl.name)
+                x = synth.correlated_x(n, sl.d_in, synth.seed_for(tag, "X"), device=dev)
+                g = synth.gradients(n, sl.d_out, synth.seed_for(tag, "G"), device=dev,
+                                    multiplier=mult[b])
+                hx = torch.zeros(sl.d_in, sl.d_in, device=dev)
+                hg = torch.zeros(sl.d_out, sl.d_out, device=dev)
+
+                def stats_and_biip():
+                    P.accumulate(xq=x, g=g, hx_sum=hx, hg_sum=hg, ws=ws)
+                    return P.biip(w[i], hx, hg, None, 1.0 / n, si[i], so[i], K.BIIP_FULL,
+                                  ws=ws, copy_hx=False)
+                res[i] = timed_call(stats_and_biip)
+                del x, g, hg
+
+        def allocate_and_solve():
+            tr = torch.stack([res[i].tr for i in owned]).cpu()
+            local_tr = {i: (float(tr[k, 0]), float(tr[k, 1])) for k, i in enumerate(owned)}
+            _, bits = P.allocate_global(local_tr, sizes, wl.extra["choices"],
+                                        wl.extra["avg_bits"], device=dev)
+            state["bits"] = bits
+            for b in blocks:
+                idx = [b * len(subs) + j for j in range(len(subs))]
+                streams.solve([res[i] for i in idx], [bits[i] for i in idx], 0.01)
+        timed_call(allocate_and_solve)
+        return timed, res
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step()
     barrier()
-    e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
-    steps = max(1, min(args.steps, 3))
-    e0.record()
-    for _ in range(steps):
-        one()
-    e1.record()
+    assert K.kronq_device_error() == 0
+    clocks = ClockSampler(local)
+    clocks.start()
+    launches0 = K.kronq_launch_count()
+    total_s = 0.0
+    for _ in range(args.steps):
+        timed, res = step()
+        torch.cuda.synchronize()
+        total_s += sum(a.elapsed_time(b) for a, b in timed) / 1e3
+        del res
     barrier()
-    el = e0.elapsed_time(e1) / 1e3
-    t = torch.tensor([el], dtype=torch.float64, device=blk.dev)
-    if dist is not None:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    value = blk.wl.params_per_block * world * steps / float(t)
-    return {"value": value, "unit": "params/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "steps": steps}
+    clk = clocks.stop()
+    launches = K.kronq_launch_count() - launches0
+    t_max = D.max_over_ranks(total_s, device=dev)
+    params = sum(sizes)
+    bits = state["bits"]
+    hist = {str(b): sum(1 for v in bits if v == b) for b in sorted(set(bits))}
+    avg = sum(b * s for b, s in zip(bits, sizes)) / params
+    result = None
+    if rank == 0:
+        result = {
+            "metric": "quantized weight params/s (BiIP+GPTAQ solve); H_X/H_G accumulate TFLOP/s",
+            "value": params * args.steps / t_max, "unit": "params/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": t_max / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "bf16 statistics, fp32 solve",
+            "data": "synthetic (seeded LLaMA-shaped activations, gradients and weights)",
+            "config": {"workload": f"mixed-precision stack: {wl.n_blocks} LLaMA-2-7B-shaped "
+                                   f"blocks, {len(sizes)} sublayers, {params} weights, own X "
+                                   f"and G per sublayer, {n} tokens, {{2,3,4}} bits at "
+                                   f"{wl.extra['avg_bits']} average; BiIP on; drift term off",
+                       "parallelism": f"blocks split over {world} GPU(s)",
+                       "timing": "sum of CUDA-event intervals around the library calls; the "
+                                 "per-sublayer input generation between them is not timed",
+                       "l2": "inputs larger than L2"},
+            "allocation": {"bits_histogram": hist, "average_bits": avg},
+            "gpu_launches": launches, "clocks": clk,
+            "e2e": {"value": None, "unit": "params/s",
+                    "skipped": "the stack's 330 GB of calibration inputs exceed host memory"},
+        }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
 
 
 # ---------------------------------------------------------------------------------- reference
 
 def run_reference(args):
+    """The oracle as it stands on the host cores, one bounded sample per step (oracle_sample):
+    value = the block estimate from the measured stage rates; ms_per_step = the measured time
+    of one sample."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return None
     from post_quantization_b200 import synth
-    wl = synth.WORKLOADS[WORKLOAD]
-    times = []
-    threads = 1
-    desc = ""
+    wl = synth.WORKLOADS[args.workload]
+    ests, spents = [], []
+    rec = {}
     for i in range(args.warmup + args.steps):
-        est, desc, threads, spent = oracle_sample()
+        est, rec, spent = oracle_sample(args.workload)
         if i >= args.warmup:
-            times.append(est)
-    est = statistics.mean(times)
+            ests.append(est)
+            spents.append(spent)
+    est = statistics.mean(ests)
     value = wl.params_per_block / est
+    model, nproc, threads = cpu_info()
+    sample = (f"fp64 oracle on a {PROXY_D}x{PROXY_D} sublayer, {PROXY_TOKENS} tokens: "
+              f"statistics, BiIP, inverse factor" + (", P" if wl.drift != "none" else "") +
+              f", column solve of {PROXY_ROWS} rows, per step")
     return {
         "impl": "reference",
         "metric": "quantized weight params/s (BiIP+GPTAQ solve); H_X/H_G accumulate TFLOP/s",
         "value": value, "unit": "params/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": est * 1e3,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": statistics.mean(spents) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded LLaMA-shaped activations, gradients and weights)",
-        "config": {"workload": "LLaMA-2-7B-shaped block: q/k/v/o 4096x4096, gate/up "
-                               "11008x4096, down 4096x11008; 262144 tokens; 4-bit per-channel "
-                               "grid; BiIP on; drift term off"},
+        "config": {"workload": describe(wl, wl.n_tokens)},
+        "value_kind": "estimate: the block's work per stage / the oracle's measured rate per "
+                      "stage; ms_per_step is the measured time of one sample",
+        "estimated_s_per_block": est,
         "cpu_baseline": {"value": value, "unit": "params/s", "cores": threads, "kind": "oracle",
-                         "sample": desc},
+                         "sample": sample, "rates": rec, "cpu_model": model, "nproc": nproc},
         "e2e": {"value": value, "unit": "params/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -675,6 +998,8 @@ def main():
     args = parse()
     if args.impl == "reference":
         res = run_reference(args)
+    elif args.workload == "llama2_7b_stack":
+        res = run_stack(args)
     else:
         res = run_gpu(args)
     if res is not None:

@@ -116,8 +116,12 @@ KRONQ_API kronq_status kronq_device_error(int32_t* code_out, kronq_stream_t stre
  *            Both triangles of hx_sum / hg_sum are valid on return (symmetric).
  *   Requirements: strides >= width, stride*2 bytes a multiple of 16, base pointers 16-byte
  *   aligned; hx_sum needs xq; dxx_sum needs xq and xfp; hg_sum needs g. n = 0 is a no-op.
- *   Accumulation: bf16 products, fp32 sums on tcgen05 tensor cores; the drift X - X~ is split
- *   into two bf16 terms so that (X - X~)^T X~ is formed without rounding X - X~.
+ *   Accumulation: bf16 products (exact), fp32 sums on tcgen05 tensor cores. For the drift
+ *   term, X~ and X - X~ are first rescaled by powers of two chosen from their largest magnitude
+ *   over the n tokens and converted to fp16: X~ stays exact, X - X~ is rounded once to 2^-11
+ *   relative; the fp16 products are summed in fp32 and the rescale is undone exactly. Inputs
+ *   must be finite. Scratch for the drift term (kronq_accumulate_workspace_size): 256 bytes
+ *   plus two fp16 copies of up to 32768 tokens of width d_in.
  * ------------------------------------------------------------------------------------- */
 KRONQ_API size_t kronq_accumulate_workspace_size(int64_t n, int32_t d_in, int32_t d_out, int with_dxx);
 KRONQ_API kronq_status kronq_accumulate(const void* xq, int64_t ld_xq, const void* xfp, int64_t ld_xfp,

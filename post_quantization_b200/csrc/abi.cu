@@ -138,14 +138,15 @@ kronq_status check_bf16_matrix(const void* p, int64_t ld, int cols, const char* 
   return KRONQ_OK;
 }
 
-constexpr int64_t kDriftChunk = 32768;   // tokens per drift split (workspace bound)
+constexpr int64_t kDriftChunk = 32768;   // tokens per fp16 conversion (workspace bound)
 
 size_t drift_ld(int d_in) { return static_cast<size_t>((d_in + 7) / 8 * 8); }
 
+// [amax pair: 256 B][fp16 X - X~ chunk][fp16 X~ chunk]
 size_t drift_ws(int64_t n, int d_in) {
   const int64_t rows = std::min<int64_t>(n, kDriftChunk);
   if (rows <= 0) return 0;
-  return 2 * align256(static_cast<size_t>(rows) * drift_ld(d_in) * 2);
+  return 256 + 2 * align256(static_cast<size_t>(rows) * drift_ld(d_in) * 2);
 }
 
 }  // namespace
@@ -241,20 +242,22 @@ kronq_status kronq_accumulate(const void* xq, int64_t ld_xq, const void* xfp, in
     KQ_TRY(launch_mirror_upper(hg_sum, d_out, d_out, s));
   }
   if (dxx_sum) {
+    // D += (X - X~)^T X~ as one fp16 product per token chunk: both operands rescaled by powers
+    // of two from their largest magnitude over all n tokens (X~ exact, X - X~ rounded once)
     const int64_t ld = static_cast<int64_t>(drift_ld(d_in));
     const int64_t rows = std::min<int64_t>(n, kDriftChunk);
-    uint8_t* hi = static_cast<uint8_t*>(workspace);
-    uint8_t* lo = hi + align256(static_cast<size_t>(rows) * ld * 2);
+    float* amax = static_cast<float*>(workspace);
+    uint8_t* da = static_cast<uint8_t*>(workspace) + 256;
+    uint8_t* xb = da + align256(static_cast<size_t>(rows) * ld * 2);
     const uint16_t* xq16 = static_cast<const uint16_t*>(xq);
     const uint16_t* xf16 = static_cast<const uint16_t*>(xfp);
+    KQ_TRY(launch_drift_amax(xfp, ld_xfp, xq, ld_xq, n, d_in, amax, s));
     for (int64_t t0 = 0; t0 < n; t0 += kDriftChunk) {
       const int64_t cnt = std::min<int64_t>(kDriftChunk, n - t0);
-      KQ_TRY(launch_drift_split(xf16 + t0 * ld_xfp, ld_xfp, xq16 + t0 * ld_xq, ld_xq, cnt, d_in, hi,
-                                lo, ld, s));
-      KQ_TRY(launch_accumulate_tc(hi, ld, xq16 + t0 * ld_xq, ld_xq, cnt, d_in, d_in, dxx_sum, d_in,
-                                  false, s));
-      KQ_TRY(launch_accumulate_tc(lo, ld, xq16 + t0 * ld_xq, ld_xq, cnt, d_in, d_in, dxx_sum, d_in,
-                                  false, s));
+      KQ_TRY(launch_drift_fp16(xf16 + t0 * ld_xfp, ld_xfp, xq16 + t0 * ld_xq, ld_xq, cnt, d_in,
+                               amax, da, xb, ld, s));
+      KQ_TRY(launch_accumulate_tc(da, ld, xb, ld, cnt, d_in, d_in, dxx_sum, d_in, false, s,
+                                  true, amax));
     }
   }
   return KRONQ_OK;

@@ -18,7 +18,15 @@
 //                 TMEM full, the next unit's MMAs wait for the drain (a few percent of a unit).
 // Work unit = (output tile, token chunk). For symmetric outputs only tiles touching the upper
 // triangle are computed and a mirror kernel fills the strict lower triangle afterwards.
+//
+// The drift term D = (X - X~)^T X~ multiplies a difference of two bf16 tensors, which bf16 cannot
+// hold to the 1e-3 the sums are held to (its rounding error is ~2^-9 per element). Both operands
+// therefore go to the tensor cores as fp16 after a power-of-two rescale taken from their largest
+// magnitude (drift_amax_kernel): X~ is exact in fp16 at that scale (bf16's 8 significant bits fit
+// fp16's 11), and X - X~ is rounded once, to 2^-11 relative. One GEMM then does what two bf16
+// GEMMs (a hi and a lo part of X - X~) would, and its epilogue undoes the rescale exactly.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "common.cuh"
 #include "internal.h"
@@ -53,8 +61,24 @@ struct AccParams {
   int kblocks_per_unit;   // BK-blocks per token chunk
   int k_splits;
   int num_units;
+  int fp16;               // operands are fp16 (else bf16)
+  const float* amax;      // drift product: {max |A source|, max |B source|}; the epilogue scales
+                          // by 2^-(fp16_shift(amax[0]) + fp16_shift(amax[1])). NULL: no scale
   int* err;
 };
+
+// Power-of-two exponent e with amax * 2^e in [2^14, 2^15), so that values scaled by 2^e stay
+// below fp16's largest finite value (65504) and lose no precision to fp16's small-number range.
+// 0 for a zero or non-finite amax; clamped to [-100, 100] (a tensor whose largest value is below
+// 2^-85 is zero for every purpose here).
+__device__ __forceinline__ int fp16_shift(float amax) {
+  if (!(amax > 0.f) || !(amax <= 3.0e38f)) return 0;
+  const int k = static_cast<int>((__float_as_uint(amax) >> 23) & 0xffu) - 126;  // amax in [2^(k-1), 2^k)
+  return max(-100, min(100, 15 - k));
+}
+__device__ __forceinline__ float pow2f(int e) {   // 2^e for e in [-126, 127]
+  return __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
+}
 
 // Map a computed-tile index to (tm, tn). Symmetric: row tm holds tiles tn >= tn_min(tm).
 // Tiles are visited in groups of GROUP tile rows, column by column inside a group, so that the
@@ -176,7 +200,7 @@ __global__ void __launch_bounds__(acc::THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32_mn_mn(HM, BN);
+      const uint32_t idesc = p.fp16 ? idesc_f16_f32_mn_mn(HM, BN) : idesc_bf16_f32_mn_mn(HM, BN);
       uint32_t it = 0;
       uint32_t ui = 0;
       bool ok = true;
@@ -223,6 +247,12 @@ __global__ void __launch_bounds__(acc::THREADS, 1)
   } else {
     // ------------------------------------------------------------------ epilogue (warps 2..5)
     const int q = warp & 3;            // TMEM lane quarter this warp may access
+    // undo the operands' power-of-two rescale (two exact multiplications)
+    float unscale_a = 1.f, unscale_b = 1.f;
+    if (p.amax) {
+      unscale_a = pow2f(-fp16_shift(p.amax[0]));
+      unscale_b = pow2f(-fp16_shift(p.amax[1]));
+    }
     uint32_t ui = 0;
     for (int u = blockIdx.x; u < p.num_units; u += gridDim.x, ++ui) {
       const int t = u % p.num_tiles;
@@ -246,6 +276,11 @@ __global__ void __launch_bounds__(acc::THREADS, 1)
           uint32_t v[32];
           tmem_ld_32x32b_x32(taddr + cb * 32, v);
           tmem_ld_wait();
+          if (p.amax) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              v[j] = __float_as_uint(__uint_as_float(v[j]) * unscale_a * unscale_b);
+          }
           const int col0 = tn * BN + cb * 32;
           if (row < p.m && col0 < p.n) {
             float* dst = p.c + static_cast<int64_t>(row) * p.ldc + col0;
@@ -297,20 +332,91 @@ __global__ void mirror_upper_kernel(float* c, int64_t ldc, int d) {
   }
 }
 
-// X - X~ split into two bf16 terms: hi = bf16(x - xq), lo = bf16((x - xq) - hi).
-__global__ void drift_split_kernel(const __nv_bfloat16* __restrict__ xfp, int64_t ld_xfp,
-                                   const __nv_bfloat16* __restrict__ xq, int64_t ld_xq,
-                                   int64_t rows, int cols, __nv_bfloat16* __restrict__ hi,
-                                   __nv_bfloat16* __restrict__ lo, int64_t ld_out) {
-  const int64_t total = rows * cols;
+// Largest |X~| and |X - X~| over a token range (bf16 in): the scales of the fp16 drift operands.
+// amax_bits[0] = max |x - x~|, amax_bits[1] = max |x~|, as fp32 bit patterns (non-negative
+// floats order like their bits), combined with atomicMax: the result does not depend on order.
+__global__ void drift_amax_kernel(const uint16_t* __restrict__ xfp, int64_t ld_xfp,
+                                  const uint16_t* __restrict__ xq, int64_t ld_xq, int64_t rows,
+                                  int cols, unsigned int* __restrict__ amax_bits) {
+  const int groups = (cols + 7) / 8;
+  const int64_t total = rows * groups;
+  float md = 0.f, mq = 0.f;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = i / cols;
-    const int c = static_cast<int>(i - r * cols);
-    const float d = __bfloat162float(xfp[r * ld_xfp + c]) - __bfloat162float(xq[r * ld_xq + c]);
-    const __nv_bfloat16 h = __float2bfloat16_rn(d);
-    hi[r * ld_out + c] = h;
-    lo[r * ld_out + c] = __float2bfloat16_rn(d - __bfloat162float(h));
+    const int64_t r = i / groups;
+    const int c0 = static_cast<int>(i - r * groups) * 8;
+    const uint16_t* pf = xfp + r * ld_xfp + c0;
+    const uint16_t* pq = xq + r * ld_xq + c0;
+    if (c0 + 8 <= cols) {
+      const uint4 uf = *reinterpret_cast<const uint4*>(pf);
+      const uint4 uq = *reinterpret_cast<const uint4*>(pq);
+      const uint32_t f[4] = {uf.x, uf.y, uf.z, uf.w}, qv[4] = {uq.x, uq.y, uq.z, uq.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float x0 = __uint_as_float(f[e] << 16), x1 = __uint_as_float(f[e] & 0xFFFF0000u);
+        const float q0 = __uint_as_float(qv[e] << 16), q1 = __uint_as_float(qv[e] & 0xFFFF0000u);
+        md = fmaxf(md, fmaxf(fabsf(x0 - q0), fabsf(x1 - q1)));
+        mq = fmaxf(mq, fmaxf(fabsf(q0), fabsf(q1)));
+      }
+    } else {
+      for (int e = 0; c0 + e < cols; ++e) {
+        const float x = __uint_as_float(static_cast<uint32_t>(pf[e]) << 16);
+        const float q = __uint_as_float(static_cast<uint32_t>(pq[e]) << 16);
+        md = fmaxf(md, fabsf(x - q));
+        mq = fmaxf(mq, fabsf(q));
+      }
+    }
+  }
+  const unsigned bd = __reduce_max_sync(0xffffffffu, __float_as_uint(md));
+  const unsigned bq = __reduce_max_sync(0xffffffffu, __float_as_uint(mq));
+  if ((threadIdx.x & 31) == 0) {
+    atomicMax(&amax_bits[0], bd);
+    atomicMax(&amax_bits[1], bq);
+  }
+}
+
+// The fp16 operands of the drift product over a token range: da = (x - x~) 2^ea and
+// xb = x~ 2^eb, with ea, eb = fp16_shift of the amax pair; row stride ld_out (a multiple of 8).
+__global__ void drift_fp16_kernel(const uint16_t* __restrict__ xfp, int64_t ld_xfp,
+                                  const uint16_t* __restrict__ xq, int64_t ld_xq, int64_t rows,
+                                  int cols, const float* __restrict__ amax,
+                                  __half* __restrict__ da, __half* __restrict__ xb,
+                                  int64_t ld_out) {
+  const float sa = pow2f(fp16_shift(amax[0])), sb = pow2f(fp16_shift(amax[1]));
+  const int groups = (cols + 7) / 8;
+  const int64_t total = rows * groups;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / groups;
+    const int c0 = static_cast<int>(i - r * groups) * 8;
+    const uint16_t* pf = xfp + r * ld_xfp + c0;
+    const uint16_t* pq = xq + r * ld_xq + c0;
+    __half* oa = da + r * ld_out + c0;
+    __half* ob = xb + r * ld_out + c0;
+    if (c0 + 8 <= cols) {
+      const uint4 uf = *reinterpret_cast<const uint4*>(pf);
+      const uint4 uq = *reinterpret_cast<const uint4*>(pq);
+      const uint32_t f[4] = {uf.x, uf.y, uf.z, uf.w}, qv[4] = {uq.x, uq.y, uq.z, uq.w};
+      uint32_t ra[4], rb[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float x0 = __uint_as_float(f[e] << 16), x1 = __uint_as_float(f[e] & 0xFFFF0000u);
+        const float q0 = __uint_as_float(qv[e] << 16), q1 = __uint_as_float(qv[e] & 0xFFFF0000u);
+        const __half2 a2 = __floats2half2_rn((x0 - q0) * sa, (x1 - q1) * sa);
+        const __half2 b2 = __floats2half2_rn(q0 * sb, q1 * sb);
+        ra[e] = *reinterpret_cast<const uint32_t*>(&a2);
+        rb[e] = *reinterpret_cast<const uint32_t*>(&b2);
+      }
+      *reinterpret_cast<uint4*>(oa) = make_uint4(ra[0], ra[1], ra[2], ra[3]);
+      *reinterpret_cast<uint4*>(ob) = make_uint4(rb[0], rb[1], rb[2], rb[3]);
+    } else {
+      for (int e = 0; c0 + e < cols; ++e) {
+        const float x = __uint_as_float(static_cast<uint32_t>(pf[e]) << 16);
+        const float q = __uint_as_float(static_cast<uint32_t>(pq[e]) << 16);
+        oa[e] = __float2half_rn((x - q) * sa);
+        ob[e] = __float2half_rn(q * sb);
+      }
+    }
   }
 }
 
@@ -386,13 +492,15 @@ __global__ void diag_finalize_kernel(const float* __restrict__ part, int splits,
 // ---------------------------------------------------------------------------------------------
 namespace {
 
-// Tensor map over a rows x cols bf16 matrix (row stride ld elements), 64 x 64 boxes, 128B swizzle.
-kronq_status make_map(CUtensorMap* map, const void* base, int64_t rows, int cols, int64_t ld) {
+// Tensor map over a rows x cols bf16 (or fp16) matrix (row stride ld elements), 64 x 64 boxes,
+// 128B swizzle.
+kronq_status make_map(CUtensorMap* map, const void* base, int64_t rows, int cols, int64_t ld,
+                      bool f16) {
   const uint64_t dims[2] = {static_cast<uint64_t>(cols), static_cast<uint64_t>(rows)};
   const uint64_t strides[1] = {static_cast<uint64_t>(ld) * 2};
   const uint32_t box[2] = {static_cast<uint32_t>(acc::BOX), static_cast<uint32_t>(acc::BK)};
-  return encode_tiled_map(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box,
-                          CU_TENSOR_MAP_SWIZZLE_128B);
+  return encode_tiled_map(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                          2, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 }  // namespace
@@ -400,12 +508,12 @@ kronq_status make_map(CUtensorMap* map, const void* base, int64_t rows, int cols
 // C (m x n, fp32, ldc) += A^T B with A: k x m bf16 (ld_a), B: k x n bf16 (ld_b).
 kronq_status launch_accumulate_tc(const void* a, int64_t ld_a, const void* b, int64_t ld_b,
                                   int64_t k, int m, int n, float* c, int64_t ldc, bool symmetric,
-                                  cudaStream_t stream) {
+                                  cudaStream_t stream, bool f16, const float* amax) {
   using namespace acc;
   if (k <= 0 || m <= 0 || n <= 0) return KRONQ_OK;
   CUtensorMap ma, mb;
-  KQ_TRY(make_map(&ma, a, k, m, ld_a));
-  KQ_TRY(make_map(&mb, b, k, n, ld_b));
+  KQ_TRY(make_map(&ma, a, k, m, ld_a, f16));
+  KQ_TRY(make_map(&mb, b, k, n, ld_b, f16));
 
   AccParams p{};
   p.c = c;
@@ -433,6 +541,8 @@ kronq_status launch_accumulate_tc(const void* a, int64_t ld_a, const void* b, in
   p.kblocks_per_unit = per;
   p.k_splits = (kblocks + per - 1) / per;
   p.num_units = p.num_tiles * p.k_splits;
+  p.fp16 = f16 ? 1 : 0;
+  p.amax = amax;
   p.err = device_error_word();
   if (!p.err) return fail(KRONQ_ERR_CUDA, "device error word unavailable");
 
@@ -452,17 +562,32 @@ kronq_status launch_mirror_upper(float* c, int64_t ldc, int d, cudaStream_t stre
   return check_launch("mirror_upper_kernel");
 }
 
-kronq_status launch_drift_split(const void* xfp, int64_t ld_xfp, const void* xq, int64_t ld_xq,
-                                int64_t rows, int cols, void* hi, void* lo, int64_t ld_out,
-                                cudaStream_t stream) {
-  const int64_t total = rows * cols;
+kronq_status launch_drift_amax(const void* xfp, int64_t ld_xfp, const void* xq, int64_t ld_xq,
+                               int64_t rows, int cols, float* amax, cudaStream_t stream) {
+  KQ_CUDA_TRY(cudaMemsetAsync(amax, 0, 2 * sizeof(float), stream));
+  const int64_t total = rows * ((cols + 7) / 8);
   if (total <= 0) return KRONQ_OK;
   int64_t blocks = (total + 255) / 256;
-  if (blocks > 148 * 16) blocks = 148 * 16;
-  drift_split_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(xfp), ld_xfp, static_cast<const __nv_bfloat16*>(xq), ld_xq,
-      rows, cols, static_cast<__nv_bfloat16*>(hi), static_cast<__nv_bfloat16*>(lo), ld_out);
-  return check_launch("drift_split_kernel");
+  const int64_t cap = static_cast<int64_t>(device_sms()) * 8;
+  if (blocks > cap) blocks = cap;
+  drift_amax_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(
+      static_cast<const uint16_t*>(xfp), ld_xfp, static_cast<const uint16_t*>(xq), ld_xq, rows,
+      cols, reinterpret_cast<unsigned int*>(amax));
+  return check_launch("drift_amax_kernel");
+}
+
+kronq_status launch_drift_fp16(const void* xfp, int64_t ld_xfp, const void* xq, int64_t ld_xq,
+                               int64_t rows, int cols, const float* amax, void* da, void* xb,
+                               int64_t ld_out, cudaStream_t stream) {
+  const int64_t total = rows * ((cols + 7) / 8);
+  if (total <= 0) return KRONQ_OK;
+  int64_t blocks = (total + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(device_sms()) * 8;
+  if (blocks > cap) blocks = cap;
+  drift_fp16_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(
+      static_cast<const uint16_t*>(xfp), ld_xfp, static_cast<const uint16_t*>(xq), ld_xq, rows,
+      cols, amax, static_cast<__half*>(da), static_cast<__half*>(xb), ld_out);
+  return check_launch("drift_fp16_kernel");
 }
 
 size_t accumulate_diag_workspace_bytes(int64_t n, int d) {

@@ -244,4 +244,14 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32_mn_mn(int m, int n) {
          | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
 }
 
+// The same for fp16 A/B (kind::f16 takes either 16-bit type, the same for both operands).
+__host__ __device__ constexpr uint32_t idesc_f16_f32_mn_mn(int m, int n) {
+  return (1u << 4)       // D format: f32
+         | (0u << 7)     // A format: f16
+         | (0u << 10)    // B format: f16
+         | (1u << 15)    // A major: MN
+         | (1u << 16)    // B major: MN
+         | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
+}
+
 }  // namespace kq

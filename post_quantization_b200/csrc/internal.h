@@ -9,13 +9,22 @@
 namespace kq {
 
 // accumulate.cu
+// C (m x n, fp32, ldc) += A^T B with A: k x m, B: k x n, token-major (ld_a, ld_b elements),
+// bf16 (f16 false) or fp16 (f16 true). amax (device, 2 floats, may be NULL): the operands were
+// scaled by powers of two taken from these magnitudes (launch_drift_fp16); the epilogue divides
+// the products by the same powers.
 kronq_status launch_accumulate_tc(const void* a, int64_t ld_a, const void* b, int64_t ld_b,
                                   int64_t k, int m, int n, float* c, int64_t ldc, bool symmetric,
-                                  cudaStream_t stream);
+                                  cudaStream_t stream, bool f16 = false,
+                                  const float* amax = nullptr);
 kronq_status launch_mirror_upper(float* c, int64_t ldc, int d, cudaStream_t stream);
-kronq_status launch_drift_split(const void* xfp, int64_t ld_xfp, const void* xq, int64_t ld_xq,
-                                int64_t rows, int cols, void* hi, void* lo, int64_t ld_out,
-                                cudaStream_t stream);
+// amax[0] = max |xfp - xq|, amax[1] = max |xq| over rows x cols bf16 (amax zeroed first)
+kronq_status launch_drift_amax(const void* xfp, int64_t ld_xfp, const void* xq, int64_t ld_xq,
+                               int64_t rows, int cols, float* amax, cudaStream_t stream);
+// da = fp16((xfp - xq) 2^ea), xb = fp16(xq 2^eb), rows x cols, row stride ld_out elements
+kronq_status launch_drift_fp16(const void* xfp, int64_t ld_xfp, const void* xq, int64_t ld_xq,
+                               int64_t rows, int cols, const float* amax, void* da, void* xb,
+                               int64_t ld_out, cudaStream_t stream);
 size_t accumulate_diag_workspace_bytes(int64_t n, int d);
 // tokens one kronq_accumulate_diag call takes: 2048 per block row of the grid, 65535 rows
 constexpr int64_t kMaxDiagTokens = 65535LL * 2048;
@@ -105,9 +114,11 @@ kronq_status split_bf16x3(const float* src, int64_t lds, int rows, int cols, Spl
 kronq_status split_bf16x3_2(const float* src0, int64_t lds0, int rows0, int cols0, Split3 dst0,
                             const float* src1, int64_t lds1, int rows1, int cols1, Split3 dst1,
                             cudaStream_t stream);
+// products: 6 (fp32-accurate: every term down to 2^-16 relative) or 3 (a0 b0 + a0 b1 + a1 b0,
+// ~2^-16 relative; the third pieces are not read).
 kronq_status tgemm(int m, int n, int k, float alpha, Split3 a, Split3 b, bool b_mn_major,
                    float beta, float* c, int64_t ldc, bool upper_only, int tri,
-                   const int32_t* skip, cudaStream_t stream);
+                   const int32_t* skip, cudaStream_t stream, int products = 6);
 // the sub-matrix of a split operand starting at (row, col)
 inline Split3 offset(Split3 s, int64_t row, int64_t col) {
   for (int i = 0; i < 3; ++i) s.part[i] += row * s.ld + col;

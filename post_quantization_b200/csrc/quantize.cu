@@ -338,13 +338,17 @@ kronq_status run_quantize(const float* w, const float* k, const float* dxx, int 
     float* mm = cv.floats(static_cast<size_t>(d_in) * d_in);
     Split3 ms = cv.split(d_in, d_in);
     float* t1 = cv.floats(static_cast<size_t>(d_out) * d_in);
+    // The pre-shift W (I + P) is W plus a correction of a few percent of W, computed from
+    // products that keep the leading three bf16 terms (~2^-16 relative): its error is far below
+    // fp32 rounding of W itself. Only the strict upper triangle of M = D K^T is formed (the
+    // tiles below the diagonal are skipped, and K^T's zero triangle bounds each tile's K range).
     // M = D K^T, striu(M)
     {
       Carve r{r1_base};
       Split3 dsp = r.split(d_in, d_in);
       KQ_TRY(split_bf16x3(dxx, d_in, d_in, d_in, dsp, stream));
-      KQ_TRY(tgemm(d_in, d_in, d_in, 1.f, dsp, ks, false, 0.f, mm, d_in, false, GEMM_B_LOWER,
-                   nullptr, stream));
+      KQ_TRY(tgemm(d_in, d_in, d_in, 1.f, dsp, ks, false, 0.f, mm, d_in, true, GEMM_B_LOWER,
+                   nullptr, stream, 3));
     }
     {
       dim3 g((d_in + 255) / 256, d_in);
@@ -358,7 +362,7 @@ kronq_status run_quantize(const float* w, const float* k, const float* dxx, int 
       Split3 wsp = r.split(d_out, d_in);
       KQ_TRY(split_bf16x3(w, d_in, d_out, d_in, wsp, stream));
       KQ_TRY(tgemm(d_out, d_in, d_in, 1.f, wsp, ms, true, 0.f, t1, d_in, false, GEMM_B_UPPER,
-                   nullptr, stream));
+                   nullptr, stream, 3));
     }
     // W~ = W + T1 K
     {
@@ -366,7 +370,7 @@ kronq_status run_quantize(const float* w, const float* k, const float* dxx, int 
       Split3 tsp = r.split(d_out, d_in);
       KQ_TRY(split_bf16x3(t1, d_in, d_out, d_in, tsp, stream));
       KQ_TRY(tgemm(d_out, d_in, d_in, 1.f, tsp, ks, true, 1.f, w_hat, d_in, false, GEMM_B_UPPER,
-                   nullptr, stream));
+                   nullptr, stream, 3));
     }
   }
 

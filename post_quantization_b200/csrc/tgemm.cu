@@ -5,7 +5,9 @@
 //
 // Each fp32 operand x is split beforehand into three bf16 pieces x = x0 + x1 + x2 (each the
 // bf16 rounding of what the previous pieces left), which carry its 24 significant bits. The
-// product keeps every term down to 2^-16 relative, a0 b0 + a0 b1 + a1 b0 + a0 b2 + a1 b1 + a2 b0;
+// product keeps every term down to 2^-16 relative, a0 b0 + a0 b1 + a1 b0 + a0 b2 + a1 b1 + a2 b0
+// (a call may ask for the first three only, ~2^-16 relative, where the result is a small
+// correction to a value held exactly elsewhere);
 // bf16 x bf16 products are exact, the dropped terms are ~2^-24 relative, and the sums are the
 // tensor core's fp32 accumulation (measured ~1e-5 relative at K = 1024, close to a CUDA-core
 // fp32 GEMM). This is what the damped inverse factor and the trailing update of the column
@@ -44,6 +46,7 @@ struct TgParams {
   int b_mn_major;
   int upper_only;
   int tri;
+  int products;           // 6: every term down to 2^-16 relative; 3: a0 b0 + a0 b1 + a1 b0
   const int32_t* skip;
   int* err;
 };
@@ -142,10 +145,13 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
             break;
           }
           uint8_t* st = smem + s * STAGE_BYTES;
-          mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+          // three products read only the first two pieces of each operand
+          const int pieces = p.products == 3 ? 2 : 3;
+          mbar_arrive_expect_tx(&full[s], pieces * 2 * PIECE_BYTES);
           const int k0 = kb * BK;
 #pragma unroll
           for (int i = 0; i < 3; ++i) {
+            if (i >= pieces) break;
             tma_load_2d(st + i * PIECE_BYTES, &maps.a[i], &full[s], k0, ti.tm * BM);
             uint8_t* bp = st + (3 + i) * PIECE_BYTES;
             if (!p.b_mn_major) {
@@ -200,12 +206,18 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
                                    : smem_desc_sw128(bb + kk * 32, 16, 1024);
             }
             const uint32_t first = (kb == ti.kb0 && kk == 0) ? 0u : 1u;
-            umma_f16(d_tmem, ad[2], bd[0], idesc, first);   // smallest terms first
-            umma_f16(d_tmem, ad[1], bd[1], idesc, 1u);
-            umma_f16(d_tmem, ad[0], bd[2], idesc, 1u);
-            umma_f16(d_tmem, ad[1], bd[0], idesc, 1u);
-            umma_f16(d_tmem, ad[0], bd[1], idesc, 1u);
-            umma_f16(d_tmem, ad[0], bd[0], idesc, 1u);
+            if (p.products == 3) {
+              umma_f16(d_tmem, ad[1], bd[0], idesc, first);   // smallest terms first
+              umma_f16(d_tmem, ad[0], bd[1], idesc, 1u);
+              umma_f16(d_tmem, ad[0], bd[0], idesc, 1u);
+            } else {
+              umma_f16(d_tmem, ad[2], bd[0], idesc, first);
+              umma_f16(d_tmem, ad[1], bd[1], idesc, 1u);
+              umma_f16(d_tmem, ad[0], bd[2], idesc, 1u);
+              umma_f16(d_tmem, ad[1], bd[0], idesc, 1u);
+              umma_f16(d_tmem, ad[0], bd[1], idesc, 1u);
+              umma_f16(d_tmem, ad[0], bd[0], idesc, 1u);
+            }
           }
           umma_commit(&empty[s]);
         }
@@ -376,10 +388,11 @@ kronq_status split_bf16x3_2(const float* src0, int64_t lds0, int rows0, int cols
 
 kronq_status tgemm(int m, int n, int k, float alpha, Split3 a, Split3 b, bool b_mn_major,
                    float beta, float* c, int64_t ldc, bool upper_only, int tri,
-                   const int32_t* skip, cudaStream_t stream) {
+                   const int32_t* skip, cudaStream_t stream, int products) {
   using namespace tg;
   if (m <= 0 || n <= 0) return KRONQ_OK;
   if (k <= 0) return fail(KRONQ_ERR_SHAPE, "tensor-core GEMM needs k >= 1");
+  if (products != 3 && products != 6) return fail(KRONQ_ERR_INVALID_ARG, "products must be 3 or 6");
   TgMaps maps;
   for (int i = 0; i < 3; ++i) {
     KQ_TRY(map_bf16(&maps.a[i], a.part[i], m, k, a.ld, BK, BM));
@@ -401,6 +414,7 @@ kronq_status tgemm(int m, int n, int k, float alpha, Split3 a, Split3 b, bool b_
   p.b_mn_major = b_mn_major ? 1 : 0;
   p.upper_only = upper_only ? 1 : 0;
   p.tri = tri;
+  p.products = products;
   p.skip = skip;
   p.err = device_error_word();
   if (!p.err) return fail(KRONQ_ERR_CUDA, "device error word unavailable");

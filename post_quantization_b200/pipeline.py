@@ -115,6 +115,20 @@ def quantize_sublayer(w, hx_sum, hg_sum, dxx_sum, inv_n, sign_in, sign_out, bits
     return r
 
 
+def allocate_global(local_traces: dict, n_params: list, choices, avg_bits: float, device=None):
+    """Bit widths of every sublayer of a stack whose sublayers are spread over ranks.
+
+    local_traces maps a global sublayer index to (tr H_X', tr H_G') for the sublayers this rank
+    processed. The traces of all ranks are gathered (dist.gather_traces) and every rank runs
+    kronq_score_allocate on the same full list, so every rank gets the same bits.
+    Returns (scores, bits) for all len(n_params) sublayers.
+    """
+    from . import dist as D
+    traces = D.gather_traces(local_traces, len(n_params), device=device)
+    return K.kronq_score_allocate([a for a, _ in traces], [b for _, b in traces], list(n_params),
+                                  choices, avg_bits)
+
+
 class SublayerStreams:
     """Runs the per-sublayer steps of a block on one CUDA stream per sublayer.
 

@@ -198,6 +198,13 @@ WORKLOADS = {
 }
 
 
+def block_g_multiplier(block: int, log10_lo: float, log10_hi: float, seed: int) -> float:
+    """Per-block output-gradient scale of a stack, log-uniform on [10^lo, 10^hi]."""
+    g = _gen(seed_for(seed, "block", block), "cpu")
+    u = float(torch.rand(1, generator=g, dtype=torch.float64))
+    return 10.0 ** (log10_lo + (log10_hi - log10_lo) * u)
+
+
 # ------------------------------------------------------------------ a quantized layer's storage
 # Stand-ins for what the solve returns (codes, grid) and for the incoherence scales, so that
 # the inference path can be exercised at any size without running the solve first.

@@ -1,8 +1,9 @@
 """Multi-rank host logic on CPU: two gloo ranks (no GPU).
 
 Sharding covers every block once, the reported step time is the maximum over ranks, and a
-stack's bit allocation computed on every rank from the all-reduced traces is identical on
-both ranks and equal to the single-process allocation.
+stack's bit allocation - the library's kronq_score_allocate run on every rank over the
+all-reduced traces (pipeline.allocate_global) - is identical on both ranks and equal to the
+oracle's allocation of all the traces in one process.
 """
 import os
 import socket
@@ -39,13 +40,12 @@ def _worker(rank, world_size, port, out):
             for s in range(7):
                 i = b * 7 + s
                 local[i] = (1.0 + 0.1 * i, 0.5 + ((i * 7919) % 13) / 3.0)
-        traces = D.gather_traces(local, n_blocks * 7)
-        from oracle import kronq_oracle as O
+        from post_quantization_b200 import pipeline as P
         sizes = [4096 * 4096] * 4 + [11008 * 4096] * 3
         sizes = sizes * n_blocks
-        _, bits = O.score_allocate([a for a, _ in traces], [b for _, b in traces], sizes,
-                                   [2, 3, 4], 2.5)
-        out[rank] = (mine, t, bits)
+        # the library's allocation (host code of the C ABI) on the gathered traces
+        _, bits = P.allocate_global(local, sizes, [2, 3, 4], 2.5)
+        out[rank] = (mine, t, list(bits))
     finally:
         dist.destroy_process_group()
 

@@ -497,6 +497,58 @@ def test_drift_term_llama3_8b_width(K):
         assert rel(h64(hx[i0:i0 + 128, j0:j0 + 128]), qa.T @ qb) <= TOL
 
 
+@pytest.mark.parametrize("scale", [1.0, 2.0 ** 40, 2.0 ** -40])
+def test_drift_term_across_chunks_and_magnitudes(K, scale):
+    # The drift product runs in fp16 after a power-of-two rescale taken from the largest
+    # magnitude over all n tokens. 70000 tokens span three conversion chunks (the largest value
+    # of the whole call sets the scale of each); inputs scaled by 2^40 would overflow fp16
+    # without the rescale and inputs scaled by 2^-40 would vanish in it. The width 136 is ragged (17 groups of 8, padded
+    # stride). The oracle sums the same bf16 values in fp64.
+    n, d = 70000, 136
+    tag = ("drift-chunks", scale)
+    x = padded((synth.correlated_x(n, d, synth.seed_for(tag, "X"), device="cuda").float()
+                * scale).to(torch.bfloat16))
+    xq = padded(synth.perturbed(x, synth.seed_for(tag, "Xq"), rel_std=0.05))
+    hx = torch.zeros(d, d, device="cuda"); dxx = torch.zeros(d, d, device="cuda")
+    K.kronq_accumulate(xq, x, None, hx, None, dxx)
+    torch.cuda.synchronize()
+    assert torch.isfinite(dxx).all()
+    o_hx, _, o_dxx = O.accumulate(h64(xq), h64(x))
+    assert rel(h64(dxx), o_dxx) <= TOL
+    assert rel(h64(hx), o_hx) <= TOL
+    # the largest value late in the tokens: the scale must come from all of them, not the
+    # first chunk
+    x2 = x.clone(); x2[-5, 3] = x2[-5, 3] * 64
+    xq2 = xq.clone(); xq2[-7, 11] = xq2[-7, 11] * 64
+    d2 = torch.zeros(d, d, device="cuda")
+    K.kronq_accumulate(xq2, x2, None, None, None, d2)
+    torch.cuda.synchronize()
+    assert rel(h64(d2), O.accumulate(h64(xq2), h64(x2))[2]) <= TOL
+
+
+@pytest.mark.parametrize("d", [8192, 28672])
+def test_drift_term_llama3_70b_width_sampled(K, d):
+    # LLaMA-3-70B input widths (hidden 8192; MLP 28672 for down_proj), X~ = X + N(0, (0.05 rms
+    # X)^2), 8192 tokens: 12 sampled 128 x 128 tiles of D = (X - X~)^T X~ and of H_X, each against
+    # fp64 sums of the same bf16 values; and the trace of H_X against its closed form.
+    n = 8192
+    x = synth.correlated_x(n, d, synth.seed_for("drift70b", d, "X"), device="cuda")
+    xq = synth.perturbed(x, synth.seed_for("drift70b", d, "Xq"), rel_std=0.05)
+    hx = torch.zeros(d, d, device="cuda"); dxx = torch.zeros(d, d, device="cuda")
+    K.kronq_accumulate(xq, x, None, hx, None, dxx)
+    torch.cuda.synchronize()
+    r = np.random.default_rng(d + 1)
+    for t in range(12):
+        i0 = int(r.integers(0, d // 128)) * 128
+        j0 = i0 if t == 0 else int(r.integers(0, d // 128)) * 128   # one diagonal tile
+        xa = h64(x[:, i0:i0 + 128]); qa = h64(xq[:, i0:i0 + 128]); qb = h64(xq[:, j0:j0 + 128])
+        assert rel(h64(dxx[i0:i0 + 128, j0:j0 + 128]), (xa - qa).T @ qb) <= TOL, (i0, j0)
+        assert rel(h64(hx[i0:i0 + 128, j0:j0 + 128]), qa.T @ qb) <= TOL, (i0, j0)
+    tr = float(np.sum(h64(xq) ** 2))
+    assert abs(float(torch.trace(hx.double())) - tr) <= TOL * tr
+    del hx, dxx
+
+
 @pytest.mark.parametrize("d_out,d_in", [(8192, 28672), (1024, 8192), (16384, 16384)])
 def test_biip_llama3_70b_shapes(K, P, d_out, d_in):
     # LLaMA-3-70B shapes: down_proj 8192 x 28672 (input Hadamard blocks of 4096, output 8192),
@@ -635,6 +687,37 @@ def test_quantize_with_drift_llama3_8b_kv(K, P):
     torch.cuda.synchronize()
     rows = np.random.default_rng(8).choice(d_out, 32, replace=False)
     o = O.quantize_layer(h64(wp[rows]), h64(r.hx), h64(dp), 3, follow_codes=h64(r.codes[rows]))
+    check_codes(r.codes[rows], o, 32 * d_in)
+    assert rel(h64(r.w_hat[rows]), o["w_hat"]) <= TOL
+
+
+@pytest.mark.parametrize("d_out,d_in", [(8192, 28672), (28672, 8192)])
+def test_quantize_llama3_70b_with_drift_sampled_rows(K, P, d_out, d_in):
+    # LLaMA-3-70B down_proj (8192 x 28672: the 28672-wide inverse factor, P and pre-shift) and
+    # gate_proj (28672 x 8192: 28672 output rows), 2 bits, drifted input (X~ = X + N(0, (0.05
+    # rms X)^2)) so P is active. 32 rows re-run by the oracle - the literal column update with
+    # the P term, P = striu(D K^T) K formed in fp64 - from the GPU's K, W' and D'.
+    n = 8192
+    tag = ("q70b", d_out, d_in)
+    x = synth.correlated_x(n, d_in, synth.seed_for(tag, "X"), device="cuda")
+    xq = synth.perturbed(x, synth.seed_for(tag, "Xq"), rel_std=0.05)
+    g = synth.gradients(n, d_out, synth.seed_for(tag, "G"), device="cuda")
+    w = synth.weight(d_out, d_in, synth.seed_for(tag, "W"), device="cuda")
+    si = synth.rademacher(d_in, synth.seed_for(tag, "si"), device="cuda")
+    so = synth.rademacher(d_out, synth.seed_for(tag, "so"), device="cuda")
+    hx = torch.zeros(d_in, d_in, device="cuda"); dxx = torch.zeros(d_in, d_in, device="cuda")
+    hg = torch.zeros(d_out, device="cuda")
+    K.kronq_accumulate(xq, x, None, hx, None, dxx)
+    K.kronq_accumulate_diag(g, hg)
+    del x, xq, g
+    r = P.biip(w, hx, hg, dxx, 1.0 / n, si, so, 15 | K.BIIP_HG_DIAG, copy_hx=False)
+    del hx, dxx
+    wp = r.w_prime.clone(); dp = r.dxx.clone()
+    P.cholinv(r, 0.01, sync=True)
+    P.quantize(r, 2)
+    torch.cuda.synchronize()
+    rows = np.random.default_rng(d_out + d_in).choice(d_out, 32, replace=False)
+    o = O.quantize_layer(h64(wp[rows]), h64(r.hx), h64(dp), 2, follow_codes=h64(r.codes[rows]))
     check_codes(r.codes[rows], o, 32 * d_in)
     assert rel(h64(r.w_hat[rows]), o["w_hat"]) <= TOL
 
