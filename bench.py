@@ -471,6 +471,8 @@ class Block:
             st["solve"] = {}
             st["solve_res"] = None
         st = self._st
+        if not self.use_graphs:
+            self.results = {}       # eager chains allocate new outputs: drop the last step's
         res = [None] * len(subs)
         done = set()
         acc_budget = sms - self.reserve if self.reserve > 0 else 0

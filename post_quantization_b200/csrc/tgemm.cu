@@ -21,20 +21,37 @@
 // while the next tile accumulates in the other TMEM buffer.
 #include <cuda_bf16.h>
 
+#include <cstdlib>
+#include <cstring>
+
 #include "common.cuh"
 #include "internal.h"
 
 namespace kq {
 
 namespace tg {
-constexpr int BM = 128, BN = 128, BK = 64, UK = 16, STAGES = 2;
-constexpr int PIECE_BYTES = 128 * BK * 2;         // 16 KB: one bf16 piece of one operand tile
-constexpr int STAGE_BYTES = 6 * PIECE_BYTES;      // A0, A1, A2, B0, B1, B2
-constexpr int MN_BOX_BYTES = 64 * BK * 2;         // 8 KB: 64 columns x BK rows (MN-major B)
-constexpr int THREADS = 192;
-constexpr int TMEM_COLS = 256;                    // two 128-column fp32 accumulators
+constexpr int BM = 128, UK = 16, STAGES = 2, THREADS = 192;
 constexpr int EPI_BYTES = 4 * 32 * 33 * 4;        // per epilogue warp: a 32 x 32 transpose tile
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024 + 256;
+
+// Two tile shapes. A tcgen05 MMA takes about the same time for any N up to 256, so the 128 x 256
+// tile runs the tensor pipe at twice the rate of the 128 x 128 one. Its operand pieces are
+// K = 32 deep (64-byte rows, 64-byte swizzle) so that two pipeline stages of the six pieces still
+// fit in shared memory; the 128 x 128 tile keeps K = 64 (128-byte rows, 128-byte swizzle).
+template <int BN_>
+struct Cfg {
+  static constexpr int BN = BN_;
+  static constexpr int BK = BN_ == 256 ? 32 : 64;
+  static constexpr int ROW_BYTES = BK * 2;                  // one K-major row of a piece
+  static constexpr uint32_t KSW = BN_ == 256 ? 4u : 2u;     // descriptor layout: 64B / 128B swizzle
+  static constexpr uint32_t KSBO = 8 * ROW_BYTES;           // bytes per 8-row swizzle atom
+  static constexpr int A_PIECE = BM * BK * 2;
+  static constexpr int B_PIECE = BN_ * BK * 2;
+  static constexpr int STAGE_BYTES = 3 * (A_PIECE + B_PIECE);   // A0, A1, A2, B0, B1, B2
+  static constexpr int MN_BOX_BYTES = 64 * BK * 2;          // 64 columns x BK rows (MN-major B)
+  static constexpr int TMEM_COLS = 2 * BN_;                 // two fp32 accumulators
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024 + 256;
+};
+static_assert(Cfg<256>::SMEM_BYTES <= 227 * 1024, "128 x 256 tile: shared memory");
 }  // namespace tg
 
 struct TgParams {
@@ -64,17 +81,18 @@ struct TileInfo {
   int tm, tn, kb0, kb1;   // K blocks [kb0, kb1) of BK
 };
 
+template <class C>
 __device__ __forceinline__ bool tile_info(const TgParams& p, int t, TileInfo& ti) {
   ti.tm = t / p.tiles_n;
   ti.tn = t % p.tiles_n;
-  const int bm = ti.tm * tg::BM, bn = ti.tn * tg::BN;
-  if (p.upper_only && bm > bn + tg::BN - 1) return false;   // entirely below the diagonal
+  const int bm = ti.tm * tg::BM, bn = ti.tn * C::BN;
+  if (p.upper_only && bm > bn + C::BN - 1) return false;   // entirely below the diagonal
   int k_lo = 0, k_hi = p.k;
   if (p.tri & GEMM_A_UPPER) k_lo = max(k_lo, bm);
   if (p.tri & GEMM_B_LOWER) k_lo = max(k_lo, bn);
-  if (p.tri & GEMM_B_UPPER) k_hi = min(k_hi, bn + tg::BN);
-  ti.kb0 = k_lo / tg::BK;
-  ti.kb1 = k_hi > k_lo ? (k_hi + tg::BK - 1) / tg::BK : ti.kb0;
+  if (p.tri & GEMM_B_UPPER) k_hi = min(k_hi, bn + C::BN);
+  ti.kb0 = k_lo / C::BK;
+  ti.kb1 = k_hi > k_lo ? (k_hi + C::BK - 1) / C::BK : ti.kb0;
   return true;
 }
 
@@ -83,9 +101,13 @@ struct TgMaps {
   CUtensorMap b[3];
 };
 
+template <int BN_>
 __global__ void __launch_bounds__(tg::THREADS, 1)
     tgemm_kernel(const __grid_constant__ TgMaps maps, const TgParams p) {
   using namespace tg;
+  using C = Cfg<BN_>;
+  constexpr int BN = C::BN, BK = C::BK, STAGE_BYTES = C::STAGE_BYTES, TMEM_COLS = C::TMEM_COLS;
+  constexpr int A_PIECE = C::A_PIECE, B_PIECE = C::B_PIECE, MN_BOX_BYTES = C::MN_BOX_BYTES;
   if (p.skip && *p.skip >= 0) return;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -136,7 +158,7 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
         TileInfo ti;
-        if (!tile_info(p, t, ti)) continue;
+        if (!tile_info<C>(p, t, ti)) continue;
         for (int kb = ti.kb0; kb < ti.kb1; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
@@ -147,18 +169,19 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
           uint8_t* st = smem + s * STAGE_BYTES;
           // three products read only the first two pieces of each operand
           const int pieces = p.products == 3 ? 2 : 3;
-          mbar_arrive_expect_tx(&full[s], pieces * 2 * PIECE_BYTES);
+          mbar_arrive_expect_tx(&full[s], pieces * (A_PIECE + B_PIECE));
           const int k0 = kb * BK;
 #pragma unroll
           for (int i = 0; i < 3; ++i) {
             if (i >= pieces) break;
-            tma_load_2d(st + i * PIECE_BYTES, &maps.a[i], &full[s], k0, ti.tm * BM);
-            uint8_t* bp = st + (3 + i) * PIECE_BYTES;
+            tma_load_2d(st + i * A_PIECE, &maps.a[i], &full[s], k0, ti.tm * BM);
+            uint8_t* bp = st + 3 * A_PIECE + i * B_PIECE;
             if (!p.b_mn_major) {
               tma_load_2d(bp, &maps.b[i], &full[s], k0, ti.tn * BN);
             } else {
-              tma_load_2d(bp, &maps.b[i], &full[s], ti.tn * BN, k0);
-              tma_load_2d(bp + MN_BOX_BYTES, &maps.b[i], &full[s], ti.tn * BN + 64, k0);
+#pragma unroll
+              for (int bx = 0; bx < BN / 64; ++bx)
+                tma_load_2d(bp + bx * MN_BOX_BYTES, &maps.b[i], &full[s], ti.tn * BN + 64 * bx, k0);
             }
           }
         }
@@ -176,7 +199,7 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
         TileInfo ti;
-        if (!tile_info(p, t, ti)) continue;
+        if (!tile_info<C>(p, t, ti)) continue;
         const uint32_t a = ui & 1u;
         const uint32_t aph = (ui >> 1) & 1u;
         ++ui;
@@ -197,13 +220,13 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
             uint64_t ad[3], bd[3];
 #pragma unroll
             for (int i = 0; i < 3; ++i) {
-              // A: K-major, 128 rows x 128 bytes, 8-row atoms of 1 KB; K step = 32 bytes.
-              ad[i] = smem_desc_sw128(base + i * PIECE_BYTES + kk * 32, 16, 1024);
-              const uint32_t bb = base + (3 + i) * PIECE_BYTES;
-              // B: K-major like A, or MN-major in two 64-column boxes (LBO = box), K step =
-              // 16 rows = 2 KB.
+              // A: K-major, 128 rows of BK elements, 8-row swizzle atoms; K step = 32 bytes.
+              ad[i] = smem_desc(base + i * A_PIECE + kk * 32, 16, C::KSBO, C::KSW);
+              const uint32_t bb = base + 3 * A_PIECE + i * B_PIECE;
+              // B: K-major like A, or MN-major in 64-column boxes of 128-byte rows (LBO = box),
+              // K step = 16 rows = 2 KB.
               bd[i] = p.b_mn_major ? smem_desc_sw128(bb + kk * 2048, MN_BOX_BYTES, 1024)
-                                   : smem_desc_sw128(bb + kk * 32, 16, 1024);
+                                   : smem_desc(bb + kk * 32, 16, C::KSBO, C::KSW);
             }
             const uint32_t first = (kb == ti.kb0 && kk == 0) ? 0u : 1u;
             if (p.products == 3) {
@@ -231,7 +254,7 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
     uint32_t ui = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
       TileInfo ti;
-      if (!tile_info(p, t, ti)) continue;
+      if (!tile_info<C>(p, t, ti)) continue;
       const uint32_t a = ui & 1u;
       const uint32_t aph = (ui >> 1) & 1u;
       ++ui;
@@ -349,7 +372,7 @@ __global__ void __launch_bounds__(128) split_bf16x3_kernel(SplitJob j0, SplitJob
 namespace {
 
 // bf16 tensor map: rows x cols (cols contiguous, row stride ld elements), box = box_cols x
-// box_rows, 128-byte swizzle.
+// box_rows; the swizzle spans the box's row (64 or 128 bytes).
 kronq_status map_bf16(CUtensorMap* map, const uint16_t* base, int64_t rows, int64_t cols,
                       int64_t ld, int box_cols, int box_rows) {
   if ((reinterpret_cast<uintptr_t>(base) & 15u) || (ld * 2) % 16)
@@ -358,7 +381,50 @@ kronq_status map_bf16(CUtensorMap* map, const uint16_t* base, int64_t rows, int6
   const uint64_t strides[1] = {static_cast<uint64_t>(ld) * 2};
   const uint32_t box[2] = {static_cast<uint32_t>(box_cols), static_cast<uint32_t>(box_rows)};
   return encode_tiled_map(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box,
-                          CU_TENSOR_MAP_SWIZZLE_128B);
+                          box_cols * 2 == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// The 128 x 256 tile is the default; KRONQ_TGEMM_TILE=128 in the environment selects the
+// 128 x 128 tile (same results to rounding order; kept to compare the two).
+bool tgemm_wide_tiles() {
+  const char* v = std::getenv("KRONQ_TGEMM_TILE");
+  return !(v && std::strcmp(v, "128") == 0);
+}
+
+template <int BN_>
+kronq_status launch_tgemm(const Split3& a, const Split3& b, TgParams p, bool b_mn_major,
+                          cudaStream_t stream) {
+  using C = tg::Cfg<BN_>;
+  TgMaps maps;
+  for (int i = 0; i < 3; ++i) {
+    KQ_TRY(map_bf16(&maps.a[i], a.part[i], p.m, p.k, a.ld, C::BK, tg::BM));
+    if (!b_mn_major)
+      KQ_TRY(map_bf16(&maps.b[i], b.part[i], p.n, p.k, b.ld, C::BK, C::BN));
+    else
+      KQ_TRY(map_bf16(&maps.b[i], b.part[i], p.k, p.n, b.ld, 64, C::BK));
+  }
+  p.tiles_m = (p.m + tg::BM - 1) / tg::BM;
+  p.tiles_n = (p.n + C::BN - 1) / C::BN;
+  // per device and cheap on the host, so set on every launch
+  KQ_CUDA_TRY(cudaFuncSetAttribute(tgemm_kernel<BN_>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   C::SMEM_BYTES));
+  // As few CTAs as the minimal number of tile waves needs: each CTA holds a whole SM (shared
+  // memory), and SMs this GEMM does not need stay free for other streams' work.
+  const int tiles = p.tiles_m * p.tiles_n;
+  int work = tiles;
+  if (p.upper_only) {
+    work = 0;
+    for (int tm = 0; tm < p.tiles_m; ++tm)
+      for (int tn = 0; tn < p.tiles_n; ++tn)
+        if (tm * tg::BM <= tn * C::BN + C::BN - 1) ++work;
+  }
+  const int sms = sm_budget();
+  const int waves = (work + sms - 1) / sms;
+  int grid = waves > 0 ? (tiles + waves - 1) / waves : 1;
+  if (grid > sms) grid = sms;
+  if (grid < 1) grid = 1;
+  tgemm_kernel<BN_><<<grid, tg::THREADS, C::SMEM_BYTES, stream>>>(maps, p);
+  return check_launch("tgemm_kernel");
 }
 
 
@@ -389,18 +455,9 @@ kronq_status split_bf16x3_2(const float* src0, int64_t lds0, int rows0, int cols
 kronq_status tgemm(int m, int n, int k, float alpha, Split3 a, Split3 b, bool b_mn_major,
                    float beta, float* c, int64_t ldc, bool upper_only, int tri,
                    const int32_t* skip, cudaStream_t stream, int products) {
-  using namespace tg;
   if (m <= 0 || n <= 0) return KRONQ_OK;
   if (k <= 0) return fail(KRONQ_ERR_SHAPE, "tensor-core GEMM needs k >= 1");
   if (products != 3 && products != 6) return fail(KRONQ_ERR_INVALID_ARG, "products must be 3 or 6");
-  TgMaps maps;
-  for (int i = 0; i < 3; ++i) {
-    KQ_TRY(map_bf16(&maps.a[i], a.part[i], m, k, a.ld, BK, BM));
-    if (!b_mn_major)
-      KQ_TRY(map_bf16(&maps.b[i], b.part[i], n, k, b.ld, BK, BN));
-    else
-      KQ_TRY(map_bf16(&maps.b[i], b.part[i], k, n, b.ld, 64, BK));
-  }
   TgParams p{};
   p.c = c;
   p.ldc = ldc;
@@ -409,8 +466,6 @@ kronq_status tgemm(int m, int n, int k, float alpha, Split3 a, Split3 b, bool b_
   p.k = k;
   p.alpha = alpha;
   p.beta = beta;
-  p.tiles_m = (m + BM - 1) / BM;
-  p.tiles_n = (n + BN - 1) / BN;
   p.b_mn_major = b_mn_major ? 1 : 0;
   p.upper_only = upper_only ? 1 : 0;
   p.tri = tri;
@@ -418,26 +473,9 @@ kronq_status tgemm(int m, int n, int k, float alpha, Split3 a, Split3 b, bool b_
   p.skip = skip;
   p.err = device_error_word();
   if (!p.err) return fail(KRONQ_ERR_CUDA, "device error word unavailable");
-  // per device and cheap on the host, so set on every launch
-  KQ_CUDA_TRY(cudaFuncSetAttribute(tgemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   SMEM_BYTES));
-  // As few CTAs as the minimal number of tile waves needs: each CTA holds a whole SM (shared
-  // memory), and SMs this GEMM does not need stay free for other streams' work.
-  const int tiles = p.tiles_m * p.tiles_n;
-  int work = tiles;
-  if (upper_only) {
-    work = 0;
-    for (int tm = 0; tm < p.tiles_m; ++tm)
-      for (int tn = 0; tn < p.tiles_n; ++tn)
-        if (tm * BM <= tn * BN + BN - 1) ++work;
-  }
-  const int sms = sm_budget();
-  const int waves = (work + sms - 1) / sms;
-  int grid = waves > 0 ? (tiles + waves - 1) / waves : 1;
-  if (grid > sms) grid = sms;
-  if (grid < 1) grid = 1;
-  tgemm_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(maps, p);
-  return check_launch("tgemm_kernel");
+  // 128 x 256 tiles where the output is wide enough to fill them
+  if (n > 128 && tgemm_wide_tiles()) return launch_tgemm<256>(a, b, p, b_mn_major, stream);
+  return launch_tgemm<128>(a, b, p, b_mn_major, stream);
 }
 
 }  // namespace kq

@@ -84,17 +84,52 @@ def case_acc(args):
     n, d = args.tokens or 16384, args.d
     x = synth.correlated_x(n, d, synth.seed_for("profcase-acc", d), device="cuda")
     h = torch.zeros(d, d, device="cuda")
-    P.accumulate(xq=x, hx_sum=h)
+    ws = P.Workspace(torch.device("cuda"))
+    if args.drift:
+        # the drift sum D += (X - X~)^T X~ alone (X~ = X + N(0, (0.05 rms X)^2))
+        xq = synth.perturbed(x, synth.seed_for("profcase-acc", d, "q"), rel_std=0.05)
+        call = lambda: P.accumulate(xq=xq, xfp=x, dxx_sum=h, ws=ws)
+        flops = 2.0 * n * d * d
+    else:
+        call = lambda: P.accumulate(xq=x, hx_sum=h, ws=ws)
+        flops = float(n) * d * (d + 1)
+    call()
     torch.cuda.synchronize()
     a, b = ev(), ev()
     a.record()
     for _ in range(args.reps):
-        P.accumulate(xq=x, hx_sum=h)
+        call()
     b.record()
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / args.reps
-    print(json.dumps({"case": "acc", "d": d, "tokens": n, "ms": ms,
-                      "tflops": n * d * (d + 1) / ms / 1e9}))
+    print(json.dumps({"case": "acc", "d": d, "tokens": n, "drift": args.drift, "ms": ms,
+                      "tflops": flops / ms / 1e9}))
+
+
+def case_peaks(args):
+    """torch (cuBLAS) matmul rates, 8192^3, best of 10 after 3 warm-ups: bf16, fp16, TF32 and
+    fp32 (the denominators of the fp32-accurate tensor-core GEMM)."""
+    n = 8192
+    out = {"case": "peaks", "n": n}
+    for name, dt, tf32 in (("bf16", torch.bfloat16, False), ("fp16", torch.float16, False),
+                           ("tf32", torch.float32, True), ("fp32", torch.float32, False)):
+        torch.backends.cuda.matmul.allow_tf32 = tf32
+        a = torch.randn(n, n, device="cuda", dtype=dt)
+        b = torch.randn(n, n, device="cuda", dtype=dt)
+        for _ in range(3):
+            a @ b
+        best = 1e30
+        for _ in range(10):
+            e0, e1 = ev(), ev()
+            e0.record()
+            a @ b
+            e1.record()
+            torch.cuda.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        out[name + "_tflops"] = 2.0 * n ** 3 / best / 1e9
+        del a, b
+    torch.backends.cuda.matmul.allow_tf32 = False
+    print(json.dumps(out))
 
 
 def case_biip(args):
@@ -142,8 +177,15 @@ def case_quantize(args):
     w = synth.weight(d_out, d_in, synth.seed_for("pc-q", "w"), device="cuda")
     si = synth.rademacher(d_in, 1, device="cuda"); so = synth.rademacher(d_out, 2, device="cuda")
     hx = torch.zeros(d_in, d_in, device="cuda")
-    P.accumulate(xq=x, hx_sum=hx)
-    r = P.biip(w, hx, None, None, 1.0 / n, si, so, K.BIIP_SCALE_IN | K.BIIP_ROTATE_IN | K.BIIP_ROTATE_OUT)
+    dxx = None
+    if args.drift:
+        xq = synth.perturbed(x, synth.seed_for("pc-q", "xq"), rel_std=0.05)
+        dxx = torch.zeros(d_in, d_in, device="cuda")
+        P.accumulate(xq=xq, xfp=x, hx_sum=hx, dxx_sum=dxx)
+    else:
+        P.accumulate(xq=x, hx_sum=hx)
+    r = P.biip(w, hx, None, dxx, 1.0 / n, si, so,
+               K.BIIP_SCALE_IN | K.BIIP_ROTATE_IN | K.BIIP_ROTATE_OUT)
     P.cholinv(r, 0.01, sync=True)
     P.quantize(r, 4, group=args.group)
     torch.cuda.synchronize()
@@ -154,7 +196,7 @@ def case_quantize(args):
     b.record()
     torch.cuda.synchronize()
     print(json.dumps({"case": "quantize", "d_out": d_out, "d_in": d_in, "group": args.group,
-                      "ms": a.elapsed_time(b) / args.reps}))
+                      "drift": args.drift, "ms": a.elapsed_time(b) / args.reps}))
 
 
 LLAMA3_70B_LINEARS = [("q", 8192, 8192), ("k", 1024, 8192), ("v", 1024, 8192),
@@ -289,7 +331,10 @@ def case_qlinear(args):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["stages", "acc", "biip", "cholinv", "quantize", "qlinear"])
+    ap.add_argument("case", choices=["stages", "acc", "biip", "cholinv", "quantize", "qlinear",
+                                     "peaks"])
+    ap.add_argument("--drift", action="store_true", help="acc: the drift sum D alone; "
+                                                          "quantize: with D (P pre-shift)")
     ap.add_argument("--tokens", type=int, default=None)
     ap.add_argument("--d", type=int, default=4096)
     ap.add_argument("--d-out", type=int, default=4096)
@@ -303,7 +348,7 @@ def main():
     K.load_library()
     K.kronq_device_check()
     {"stages": stages, "acc": case_acc, "biip": case_biip, "cholinv": case_cholinv,
-     "quantize": case_quantize, "qlinear": case_qlinear}[args.case](args)
+     "quantize": case_quantize, "qlinear": case_qlinear, "peaks": case_peaks}[args.case](args)
 
 
 if __name__ == "__main__":

@@ -243,3 +243,79 @@ def activations(n: int, d: int, seed: int, dtype=torch.float32, device="cpu",
     cols = outlier_channels(d, seed_for(seed, "outliers"), n_outliers)
     x[:, cols] *= outlier_scale
     return x.to(dtype)
+
+
+# ------------------------------------------------------------ a synthetic block's own backward
+# The KronQ pages obtain G from one backward pass of the model over the calibration set. This
+# stands in for that with a random-weight LLaMA-style block (no trained weights, no dataset):
+# its forward over correlated synthetic inputs gives each linear's input X, and its backward
+# from a synthetic gradient of the block output gives each linear's output gradient G. It is
+# input generation, like the generators above: plain torch ops in fp32, stored as bf16.
+
+def _rms_norm(x: torch.Tensor, eps: float = 1e-5) -> torch.Tensor:
+    return x * torch.rsqrt(x.pow(2).mean(dim=-1, keepdim=True) + eps)
+
+
+def block_calibration(wl: Workload, n: int, seed: int, device="cpu", seq_len: int = 2048,
+                      head_dim: int = 128, seqs_per_chunk: int = 4, dtype=torch.bfloat16):
+    """X (per input stream) and G (per sublayer) of one forward + backward of a random-weight block.
+
+    Block: u = x + o_proj(attn(q_proj(n1), k_proj(n1), v_proj(n1))) with n1 = rmsnorm(x), causal
+    attention per sequence of seq_len tokens (k/v heads shared by groups of query heads when
+    k_proj is narrower than q_proj); y = u + down_proj(silu(gate_proj(n2)) * up_proj(n2)) with
+    n2 = rmsnorm(u). x is the correlated synthetic activation of the block input; the gradient
+    of the block output dL/dy is the log-uniform per-channel synthetic gradient. Weights are
+    N(0, 0.02^2) (wl's shapes; the same seeds as the quantized weights, so W is the layer the
+    statistics belong to). Returns ({stream: X}, {sublayer: G}) with the streams of wl: the
+    inputs of q/k/v, o, gate/up and down.
+    """
+    subs = {s.name: s for s in wl.sublayers}
+    h = subs["q_proj"].d_in
+    heads = subs["q_proj"].d_out // head_dim
+    kv_heads = subs["k_proj"].d_out // head_dim
+    f32 = torch.float32
+    w = {name: weight(s.d_out, s.d_in, seed_for(seed, name, "W"), dtype=dtype, device=device)
+         for name, s in subs.items()}
+    x_all = correlated_x(n, h, seed_for(seed, "x"), dtype=dtype, device=device)
+    gy_all = gradients(n, h, seed_for(seed, "gy"), dtype=dtype, device=device)
+    stream_of = {s.name: s.x_stream for s in wl.sublayers}
+    xs = {st: torch.empty(n, subs[name].d_in, dtype=dtype, device=device)
+          for name, st in stream_of.items()}
+    gs = {name: torch.empty(n, s.d_out, dtype=dtype, device=device) for name, s in subs.items()}
+    chunk = seq_len * seqs_per_chunk
+    for c0 in range(0, n, chunk):
+        c1 = min(n, c0 + chunk)
+        nb = (c1 - c0) // seq_len
+        x = x_all[c0:c1].to(f32).requires_grad_(True)    # so that every output carries a grad
+        outs = {}
+
+        def lin(name, inp):
+            out = inp @ w[name].to(f32).t()
+            out.retain_grad()
+            outs[name] = (inp, out)
+            return out
+
+        with torch.enable_grad():
+            n1 = _rms_norm(x)
+            q = lin("q_proj", n1)
+            k = lin("k_proj", n1)
+            v = lin("v_proj", n1)
+            qh = q.view(nb, seq_len, heads, head_dim).transpose(1, 2)
+            kh = k.view(nb, seq_len, kv_heads, head_dim).transpose(1, 2)
+            vh = v.view(nb, seq_len, kv_heads, head_dim).transpose(1, 2)
+            if kv_heads != heads:
+                kh = kh.repeat_interleave(heads // kv_heads, dim=1)
+                vh = vh.repeat_interleave(heads // kv_heads, dim=1)
+            att = torch.nn.functional.scaled_dot_product_attention(qh, kh, vh, is_causal=True)
+            att = att.transpose(1, 2).reshape(c1 - c0, heads * head_dim)
+            u = x + lin("o_proj", att)
+            n2 = _rms_norm(u)
+            a = lin("gate_proj", n2)
+            b = lin("up_proj", n2)
+            y = u + lin("down_proj", torch.nn.functional.silu(a) * b)
+            y.backward(gy_all[c0:c1].to(f32))
+        for name, (inp, out) in outs.items():
+            xs[stream_of[name]][c0:c1] = inp.detach().to(dtype)
+            gs[name][c0:c1] = out.grad.to(dtype)
+        del outs, x
+    return xs, gs
