@@ -55,6 +55,12 @@ def parse():
     ap.add_argument("--overlap", type=int, default=0, metavar="SMS",
                     help="run each sublayer's BiIP and inverse factor alongside the remaining "
                          "statistics on SMS reserved SMs (0: phases one after another)")
+    ap.add_argument("--calibration", default="synthetic", choices=["synthetic", "backward"],
+                    help="synthetic: seeded X and G generators; backward: X and G of every linear "
+                         "from the forward and backward of a random-weight block")
+    ap.add_argument("--hg-diag", action="store_true",
+                    help="diagonal-only H_G: sum diag(G^T G) in one streaming pass instead of "
+                         "the G^T G product (BiIP's scales and the trace need only the diagonal)")
     ap.add_argument("--no-e2e", action="store_true", help=argparse.SUPPRESS)
     ap.add_argument("--no-cpu-baseline", action="store_true", help=argparse.SUPPRESS)
     return ap.parse_args()
@@ -264,9 +270,10 @@ class ClockSampler:
 class Block:
     """Device-resident inputs and buffers of one block; `step` runs the whole path."""
 
-    def __init__(self, wl, rank, device, n_tokens, ws):
+    def __init__(self, wl, rank, device, n_tokens, ws, calibration="synthetic", hg_diag=False):
         import torch
 
+        from post_quantization_b200 import kronq as K
         from post_quantization_b200 import synth
         self.wl = wl
         self.dev = device
@@ -274,10 +281,20 @@ class Block:
         self.ws = ws
         tag = (wl.name, "rank", rank)
         self.drift = wl.drift != "none"
+        self.hg_diag = hg_diag
+        self.biip_flags = K.BIIP_FULL | (K.BIIP_HG_DIAG if hg_diag else 0)
+        self.w = {s.name: synth.weight(s.d_out, s.d_in, synth.seed_for(tag, s.name, "W"),
+                                       dtype=wl.w_dtype, device=device) for s in wl.sublayers}
         # X~ (the quantized model's input) in self.x; with the asymmetric term on, also X (the
         # full-precision model's input) in self.xfp, and D = (X - X~)^T X~ per stream
-        xs = {name: synth.correlated_x(n_tokens, d, synth.seed_for(tag, name, "X"), device=device)
-              for name, d in wl.streams().items()}
+        if calibration == "backward":
+            # X and G from the forward and backward of a random-weight block with these weights
+            xs, gs = synth.block_calibration(wl, n_tokens, synth.seed_for(tag, "block"),
+                                             device=device, weights=self.w)
+        else:
+            xs = {name: synth.correlated_x(n_tokens, d, synth.seed_for(tag, name, "X"),
+                                           device=device) for name, d in wl.streams().items()}
+            gs = None
         if self.drift:
             kind, amount = wl.drift[:3], float(wl.drift[3:])
             self.xfp = xs
@@ -291,18 +308,20 @@ class Block:
             self.xfp = None
             self.x = xs
             self.dxx = None
-        self.g = {s.name: synth.gradients(n_tokens, s.d_out, synth.seed_for(tag, s.name, "G"),
-                                          device=device) for s in wl.sublayers}
-        self.w = {s.name: synth.weight(s.d_out, s.d_in, synth.seed_for(tag, s.name, "W"),
-                                       dtype=wl.w_dtype, device=device) for s in wl.sublayers}
+        self.g = gs if gs is not None else {
+            s.name: synth.gradients(n_tokens, s.d_out, synth.seed_for(tag, s.name, "G"),
+                                    device=device) for s in wl.sublayers}
         self.si = {s.name: synth.rademacher(s.d_in, synth.seed_for(tag, s.name, "si"),
                                             device=device) for s in wl.sublayers}
         self.so = {s.name: synth.rademacher(s.d_out, synth.seed_for(tag, s.name, "so"),
                                             device=device) for s in wl.sublayers}
         self.hx = {name: torch.zeros(d, d, device=device) for name, d in wl.streams().items()}
-        self.hg = {s.name: torch.zeros(s.d_out, s.d_out, device=device) for s in wl.sublayers}
+        # H_G sums, or only their diagonals in the diagonal-only mode
+        self.hg = {s.name: torch.zeros((s.d_out,) if hg_diag else (s.d_out, s.d_out),
+                                       device=device) for s in wl.sublayers}
         self.results = {}
-        self.acc_events = []        # (start, end, flops) of each statistics call
+        self.acc_events = []        # (start, end, flops) of each tensor-core statistics call
+        self.diag_events = []       # (start, end, bytes) of each diagonal-only H_G call
         self.bits = None
         self.streams = None         # one stream per sublayer for the per-sublayer steps
         self.use_graphs = True
@@ -355,14 +374,7 @@ class Block:
         for s in wl.sublayers:
             h = self.hg[s.name]
             h.zero_()
-            if time_acc:
-                e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
-                e0.record()
-            P.accumulate(g=g[s.name], hg_sum=h, ws=self.ws)
-            if time_acc:
-                e1.record()
-                d = h.shape[0]
-                self.acc_events.append((e0, e1, self.n * d * (d + 1)))
+            self._hg_sum(time_acc, g[s.name], h)
         inv_n = 1.0 / self.n
         if self.streams is None:
             # the per-sublayer phases (BiIP; inverse factor + column solve) run side by side on
@@ -371,7 +383,7 @@ class Block:
             self.streams = P.SublayerStreams(len(wl.sublayers), self.dev)
             jobs = [(self.w[s.name], self.hx[s.x_stream], self.hg[s.name],
                      self.dxx[s.x_stream] if self.drift else None, inv_n,
-                     self.si[s.name], self.so[s.name], K.BIIP_FULL) for s in wl.sublayers]
+                     self.si[s.name], self.so[s.name], self.biip_flags) for s in wl.sublayers]
             self.biip_phase = (P.CapturedPhase(lambda: self.streams.biip(jobs))
                                if self.use_graphs else (lambda: self.streams.biip(jobs)))
             self.solve_phases = {}
@@ -463,7 +475,7 @@ class Block:
                 sl = subs[i]
                 r = P.biip(self.w[sl.name], self.hx[sl.x_stream], self.hg[sl.name],
                            self.dxx[sl.x_stream] if self.drift else None, inv_n,
-                           self.si[sl.name], self.so[sl.name], K.BIIP_FULL, ws=st["ws"][i])
+                           self.si[sl.name], self.so[sl.name], self.biip_flags, ws=st["ws"][i])
                 P.cholinv(r, 0.01, st["ws"][i])
                 return r
             st["chain"] = [P.CapturedPhase(lambda i=i: chain(i)) if self.use_graphs
@@ -496,8 +508,7 @@ class Block:
                 main.wait_event(landed[("g", sl.name)])
             h = self.hg[sl.name]
             h.zero_()
-            self._timed_acc(time_acc, h.shape[0], False,
-                            lambda: P.accumulate(g=g[sl.name], hg_sum=h, ws=self.ws))
+            self._hg_sum(time_acc, g[sl.name], h)
             s_i = st["streams"][i]
             s_i.wait_stream(main)
             K.kronq_set_sm_budget(self.reserve)
@@ -533,6 +544,28 @@ class Block:
         if key not in st["solve"]:
             st["solve"][key] = P.CapturedPhase(solve)
         st["solve"][key]()
+
+    def _hg_sum(self, time_acc, g, h):
+        """H_G += G^T G (tensor cores), or its diagonal alone in the diagonal-only mode."""
+        import torch
+
+        from post_quantization_b200 import pipeline as P
+        if self.hg_diag:
+            fn = lambda: P.accumulate_diag(g, h, ws=self.ws)
+        else:
+            fn = lambda: P.accumulate(g=g, hg_sum=h, ws=self.ws)
+        if not time_acc:
+            fn()
+            return
+        e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        if self.hg_diag:
+            self.diag_events.append((e0, e1, g.numel() * g.element_size()))
+        else:
+            d = h.shape[0]
+            self.acc_events.append((e0, e1, self.n * d * (d + 1)))
 
     def _timed_acc(self, time_acc, d, drift, fn):
         import torch
@@ -587,7 +620,7 @@ def run_gpu(args):
     wl = synth.WORKLOADS[args.workload]
     n_tok = args.tokens or wl.n_tokens
     ws = P.Workspace(dev)
-    blk = Block(wl, rank, dev, n_tok, ws)
+    blk = Block(wl, rank, dev, n_tok, ws, calibration=args.calibration, hg_diag=args.hg_diag)
     graphs = args.graphs
     if args.no_graphs:
         graphs = "off"
@@ -622,6 +655,15 @@ def run_gpu(args):
     elapsed = t_start.elapsed_time(t_end) / 1e3
     acc_ms = [a.elapsed_time(b) for a, b, _ in blk.acc_events]
     acc_flops = [f for _, _, f in blk.acc_events]
+    diag = None
+    if blk.diag_events:
+        d_s = sum(a.elapsed_time(b) for a, b, _ in blk.diag_events) / 1e3
+        diag = {"kernel": "diag_partial_kernel (+ diag_finalize_kernel)",
+                "achieved_gbs": sum(nb for _, _, nb in blk.diag_events) / d_s / 1e9,
+                "basis": "bytes of G read / CUDA-event time of the diagonal-sum calls",
+                "ms_per_step": d_s * 1e3 / args.steps}
+    scores = {sl.name: float(blk.results[sl.name].tr[0] * blk.results[sl.name].tr[1])
+              for sl in wl.sublayers if sl.name in blk.results}
     from post_quantization_b200 import dist as D
     elapsed_max = D.max_over_ranks(elapsed, device=dev)
     params = wl.params_per_block * world
@@ -663,6 +705,10 @@ def run_gpu(args):
                        "tokens": n_tok, "params_per_block": wl.params_per_block,
                        "parallelism": f"one block per GPU x{world}",
                        "graphs": blk.use_graphs,
+                       "calibration": ("X and G from the forward and backward of a random-weight "
+                                       "block" if args.calibration == "backward" else
+                                       "seeded synthetic X and G"),
+                       "hg": "diagonal only" if args.hg_diag else "full G^T G",
                        "l2": f"inputs ({blk.input_bytes() / 1e9:.0f} GB) larger than L2"},
             "accumulate_tflops": acc_tflops,
             "roofline": {"bound": "tensor", "kernel": "accumulate_tc_kernel",
@@ -675,7 +721,12 @@ def run_gpu(args):
             "gpu_launches": launches,
             "clocks": clk,
             "e2e": e2e,
+            "scores": scores,
         }
+        if diag is not None:
+            hbm = peaks.get("hbm_gbs") or 6650.0
+            diag.update({"peak_gbs": hbm, "frac": diag["achieved_gbs"] / hbm})
+            result["hg_diag"] = diag
         if not args.no_cpu_baseline:
             samples = [oracle_sample(args.workload) for _ in range(3)]
             est = statistics.mean(e for e, _, _ in samples)

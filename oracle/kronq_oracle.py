@@ -33,6 +33,9 @@ What it computes, step by step, with the passage each step follows. Page names:
                                                   [KronQ-gist] Experimental results (upgrade the
                                                   higher-scored sublayer first)
   objective       tr[H_G dW H_X dW^T] + 2 tr[H_G W D dW^T]  [KronQ-hyper] Method: objectives
+  yaqa_round      comparison variant (prior art, not KronQ): rounding with input- and
+                  output-side feedback, the fixed point W^ = Q(W + L_O'^T D L_I' + L_O'^T D +
+                  D L_I')                       [YAQA notes] generalized LDLQ
   mu_incoherence  max_ij |Q_ij| over eigenvectors Q of H (mu(H)/sqrt(d))
                                                   [KronQ-hyper] Method: incoherence figure
   qlinear         the quantized layer on activations, y = S_G^-1 U^T W^' V S_X^-1 x with
@@ -621,6 +624,90 @@ def qlinear(x, codes, scale, zero, s_x=None, s_g=None, sign_in=None, sign_out=No
     """The quantized layer on activations: qlinear_dense of the dequantized codes."""
     return qlinear_dense(dequantize_layer(codes, scale, zero, group), x, s_x, s_g, sign_in,
                          sign_out, flags)
+
+
+# ------------------------------------------------------------------------------------------
+# Comparison variant: rounding with output-side feedback as well (prior art, not KronQ)
+# ------------------------------------------------------------------------------------------
+
+def udu_factor(h):
+    """Unit upper triangular U and diagonal d with H = U diag(d) U^T.
+
+    The triangular factor of H in the orientation that makes the natural column order causal:
+    row p of U - I holds the feedback from column p to the later columns. Computed as the
+    Cholesky factor of the index-reversed matrix, reversed back: J H J = L L^T gives
+    H = (J L J)(J L J)^T with J L J upper triangular.
+    """
+    h = np.asarray(h, dtype=np.float64)
+    rev = np.arange(h.shape[0])[::-1]
+    try:
+        l = np.linalg.cholesky(h[np.ix_(rev, rev)])
+    except np.linalg.LinAlgError as e:
+        raise NotPositiveDefinite(str(e))
+    u = l[np.ix_(rev, rev)]
+    dg = np.diag(u).copy()
+    return u / dg[None, :], dg * dg
+
+
+def quantize_matrix(t, scale, zero, bits):
+    """Per-row grid codes of a whole matrix: clamp(rint(t/scale) + zero, 0, 2^b - 1) in fp32."""
+    maxq = np.float32(2 ** bits - 1)
+    s = np.asarray(scale, dtype=np.float32)[:, None]
+    z = np.asarray(zero, dtype=np.float32)[:, None]
+    c = np.rint(np.asarray(t).astype(np.float32) / s)
+    return np.clip(c + z, np.float32(0), maxq).astype(np.float32)
+
+
+def yaqa_round(w, h_out, h_in, bits: int, damp_rel: float = 0.01, follow_codes=None,
+               tie_tol: float = 1e-3):
+    """Rounding with feedback on both the input and the output side, for comparison with KronQ.
+
+    [YAQA notes], generalized LDLQ: for a Kronecker proxy H_O (x) H_I of the layer Hessian,
+    with the triangular factors L_O, L_I of H_O and H_I and L' = L - I, the quantized W^ is the
+    fixed point of
+        W^ = Q(W + L_O'^T D L_I' + L_O'^T D + D L_I'),    D = W - W^,
+    which is reached in at most m + n - 1 iterations. Here H_O = H_G' and H_I = H_X' (after
+    incoherence processing), each damped by damp_rel * mean diag, L the unit upper triangular
+    factor of udu_factor (so that L_I' is the input-side feedback of the column solve, which
+    with H_O = I is KronQ's solve without P), Q the per-row grid of W (grid). The iteration
+    starts from W^ = Q(W) and stops when an iteration changes nothing.
+    follow_codes / tie_tol: as in quantize_layer, at every iteration.
+    Returns dict: codes, scale, zero, w_hat (fp64), iterations, near_tie, disagree.
+    """
+    w = np.asarray(w, dtype=np.float64)
+    m, n = w.shape
+    ho = np.asarray(h_out, dtype=np.float64)
+    hi = np.asarray(h_in, dtype=np.float64)
+    ho = ho + damping(ho, damp_rel) * np.eye(m)
+    hi = hi + damping(hi, damp_rel) * np.eye(n)
+    lo = udu_factor(ho)[0] - np.eye(m)
+    li = udu_factor(hi)[0] - np.eye(n)
+    scale, zero = grid(w, bits)
+    s64 = scale.astype(np.float64)[:, None]
+
+    def deq(c):   # scale (c - zero) in fp32, as the column solve dequantizes
+        return dequantize(c, scale[:, None], zero[:, None]).astype(np.float64)
+
+    codes = quantize_matrix(w, scale, zero, bits)
+    near = np.zeros((m, n), dtype=bool)
+    disagree = np.zeros((m, n), dtype=bool)
+    iterations = 0
+    for _ in range(m + n):
+        delta = w - deq(codes)
+        target = w + lo.T @ delta @ li + lo.T @ delta + delta @ li
+        new = quantize_matrix(target, scale, zero, bits)
+        if follow_codes is not None:
+            u = target / s64
+            near = np.abs(u - (np.floor(u) + 0.5)) <= tie_tol
+            fc = np.asarray(follow_codes, dtype=np.float32)
+            disagree = near & (fc != new)
+            new = np.where(near, fc, new).astype(np.float32)
+        iterations += 1
+        if np.array_equal(new, codes):
+            break
+        codes = new
+    return {"codes": codes.astype(np.uint8), "scale": scale, "zero": zero, "w_hat": deq(codes),
+            "iterations": iterations, "near_tie": near, "disagree": disagree}
 
 
 # ------------------------------------------------------------------------------------------

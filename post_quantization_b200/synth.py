@@ -257,7 +257,8 @@ def _rms_norm(x: torch.Tensor, eps: float = 1e-5) -> torch.Tensor:
 
 
 def block_calibration(wl: Workload, n: int, seed: int, device="cpu", seq_len: int = 2048,
-                      head_dim: int = 128, seqs_per_chunk: int = 4, dtype=torch.bfloat16):
+                      head_dim: int = 128, seqs_per_chunk: int = 4, dtype=torch.bfloat16,
+                      weights: dict | None = None):
     """X (per input stream) and G (per sublayer) of one forward + backward of a random-weight block.
 
     Block: u = x + o_proj(attn(q_proj(n1), k_proj(n1), v_proj(n1))) with n1 = rmsnorm(x), causal
@@ -265,17 +266,18 @@ def block_calibration(wl: Workload, n: int, seed: int, device="cpu", seq_len: in
     k_proj is narrower than q_proj); y = u + down_proj(silu(gate_proj(n2)) * up_proj(n2)) with
     n2 = rmsnorm(u). x is the correlated synthetic activation of the block input; the gradient
     of the block output dL/dy is the log-uniform per-channel synthetic gradient. Weights are
-    N(0, 0.02^2) (wl's shapes; the same seeds as the quantized weights, so W is the layer the
-    statistics belong to). Returns ({stream: X}, {sublayer: G}) with the streams of wl: the
-    inputs of q/k/v, o, gate/up and down.
+    N(0, 0.02^2) in wl's shapes, or `weights` ({sublayer: W}) when given, so that the statistics
+    belong to the layers being quantized. Returns ({stream: X}, {sublayer: G}) with the streams
+    of wl: the inputs of q/k/v, o, gate/up and down.
     """
     subs = {s.name: s for s in wl.sublayers}
     h = subs["q_proj"].d_in
     heads = subs["q_proj"].d_out // head_dim
     kv_heads = subs["k_proj"].d_out // head_dim
     f32 = torch.float32
-    w = {name: weight(s.d_out, s.d_in, seed_for(seed, name, "W"), dtype=dtype, device=device)
-         for name, s in subs.items()}
+    w = weights if weights is not None else {
+        name: weight(s.d_out, s.d_in, seed_for(seed, name, "W"), dtype=dtype, device=device)
+        for name, s in subs.items()}
     x_all = correlated_x(n, h, seed_for(seed, "x"), dtype=dtype, device=device)
     gy_all = gradients(n, h, seed_for(seed, "gy"), dtype=dtype, device=device)
     stream_of = {s.name: s.x_stream for s in wl.sublayers}

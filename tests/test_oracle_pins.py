@@ -751,3 +751,73 @@ def test_pack_grid_places_each_pair(group):
             idx = ((row // 128) * gp + g) * 128 + row % 128
             assert pk[idx, 0] == sc[row, g] and pk[idx, 1] == zr[row, g]
     assert np.count_nonzero(pk[:, 1]) == d_out * gp
+
+
+# ------------------------------------------------------------------ output-side feedback (comparison variant)
+
+def test_udu_factor_is_the_inverse_factor_rescaled():
+    # H = U diag(d) U^T with U unit upper triangular; the same U follows from the damped inverse
+    # factor, K^T K = H^-1  =>  H = K^-1 K^-T, so U = K^-1 diag(K_pp) and d = 1 / K_pp^2.
+    r = rng(80)
+    h = spd(r, 9, cond=40.0)
+    u, dg = O.udu_factor(h)
+    np.testing.assert_allclose(u @ np.diag(dg) @ u.T, h, rtol=0, atol=1e-12 * np.abs(h).max())
+    np.testing.assert_array_equal(np.tril(u, -1), 0)
+    np.testing.assert_allclose(np.diag(u), 1.0, rtol=0, atol=1e-15)
+    k = O.cholinv(h, 0.0)
+    np.testing.assert_allclose(u, np.linalg.inv(k) * np.diag(k)[None, :], rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(dg, 1.0 / np.diag(k) ** 2, rtol=1e-9)
+
+
+@pytest.mark.parametrize("seed,bits", [(81, 2), (82, 3), (83, 4)])
+def test_output_feedback_rounding_reduces_to_the_column_solve(seed, bits):
+    # [YAQA notes]: with H_O = I the output-side terms vanish and the fixed point is LDLQ, i.e.
+    # the column-wise OBS solve without P (GPTQ); same grid, so the same codes.
+    r = rng(seed)
+    m, n = 7, 12
+    w = r.standard_normal((m, n))
+    hi = spd(r, n, cond=50.0)
+    res = O.yaqa_round(w, np.eye(m), hi, bits)
+    ref = O.quantize_layer(w, O.cholinv(hi, 0.01), None, bits)
+    np.testing.assert_array_equal(res["codes"], ref["codes"])
+    np.testing.assert_allclose(res["w_hat"], ref["w_hat"], rtol=0, atol=1e-12)
+
+
+def _yaqa_elementwise(w, ho, hi, bits, damp_rel=0.01):
+    """The fixed point evaluated element by element in row-major order (a valid order: element
+    (i, j) reads the errors of elements (k, l) with k <= i and l <= j only), scalar loops."""
+    m, n = w.shape
+    ho = ho + O.damping(ho, damp_rel) * np.eye(m)
+    hi = hi + O.damping(hi, damp_rel) * np.eye(n)
+    uo = O.udu_factor(ho)[0]
+    ui = O.udu_factor(hi)[0]
+    scale, zero = O.grid(w, bits)
+    maxq = np.float32(2 ** bits - 1)
+    delta = np.zeros((m, n))
+    codes = np.zeros((m, n), dtype=np.float32)
+    for i in range(m):
+        for j in range(n):
+            t = w[i, j]
+            for k in range(i + 1):
+                for l in range(j + 1):
+                    if (k, l) != (i, j):
+                        t += uo[k, i] * delta[k, l] * ui[l, j]
+            c = np.clip(np.rint(np.float32(t) / scale[i]) + zero[i], np.float32(0), maxq)
+            codes[i, j] = c
+            delta[i, j] = w[i, j] - float(np.float32(scale[i] * (c - zero[i])))
+    return codes
+
+
+@pytest.mark.parametrize("seed", [84, 85, 86])
+def test_output_feedback_fixed_point_equals_elementwise_order(seed):
+    r = rng(seed)
+    m, n, bits = 5, 6, 2
+    w = r.standard_normal((m, n))
+    ho = spd(r, m, cond=20.0); hi = spd(r, n, cond=20.0)
+    res = O.yaqa_round(w, ho, hi, bits)
+    np.testing.assert_array_equal(res["codes"], _yaqa_elementwise(w, ho, hi, bits))
+    # reached within m + n - 1 updates (+1 iteration that finds nothing to change)
+    assert res["iterations"] <= m + n
+    # a fixed point: one more update changes no code
+    again = O.yaqa_round(w, ho, hi, bits, follow_codes=res["codes"], tie_tol=0.0)
+    np.testing.assert_array_equal(again["codes"], res["codes"])
