@@ -286,6 +286,40 @@ KRONQ_API kronq_status kronq_score_allocate(const double* tr_hx, const double* t
                                   int32_t* bits_out);
 
 /* ---------------------------------------------------------------------------------------
+ * 5b. Comparison variant (prior art, not KronQ): rounding with output-side feedback too.
+ *
+ * [YAQA notes], generalized LDLQ: for a Kronecker proxy H_O (x) H_I of the layer Hessian with
+ * unit upper triangular factors L_O, L_I (H = L diag L^T) and L' = L - I, the quantized W^ is
+ * the fixed point of
+ *     W^ = Q(W + L_O'^T D L_I' + L_O'^T D + D L_I'),   D = W - W^,
+ * reached within d_out + d_in - 1 updates of all elements at once. KronQ's own solve
+ * (kronq_quantize_layer) keeps only the input side, the D L_I' term: with H_G it cancels
+ * ([KronQ-hyper] Method, Proposition 1). This call takes H_I = H_X' and H_O = H_G' through their
+ * damped inverse factors and exists to measure what the output side adds.
+ *
+ *   w        (device, fp32) d_out x d_in, W' from kronq_biip (contiguous)
+ *   k_in     (device, fp32) d_in x d_in, kronq_cholinv of H_X' (upper, K^T K = (H_X'+lI)^-1)
+ *   k_out    (device, fp32) d_out x d_out, kronq_cholinv of the full H_G' (kronq_biip with
+ *            KRONQ_BIIP_WRITE_HG gives H_G')
+ *   bits 2..8; grid: one per row from w (as kronq_quantize_layer with group 0)
+ *   codes (uint8), scale, zero (d_out), w_hat (fp32): outputs as for kronq_quantize_layer
+ *   iterations (host, may be NULL): the update passes run, the last one changing no code
+ *   Arithmetic: L from the inverse factors (the inverse factor of K K^T is K^-1, U U^T = H +
+ *   lambda I); each update is two fp32-accurate tensor-core products with the strictly
+ *   triangular parts of L_I and L_O; decisions in fp32. Synchronizes `stream` once per update
+ *   (it reads how many codes changed). d_out, d_in <= 65535.
+ *   Errors: KRONQ_ERR_CUDA if no fixed point is reached within d_out + d_in updates.
+ * ------------------------------------------------------------------------------------- */
+KRONQ_API size_t kronq_quantize_layer_twosided_workspace_size(int32_t d_out, int32_t d_in);
+KRONQ_API kronq_status kronq_quantize_layer_twosided(const float* w, const float* k_in,
+                                                     const float* k_out, int32_t d_out,
+                                                     int32_t d_in, int32_t bits, uint8_t* codes,
+                                                     float* scale, float* zero, float* w_hat,
+                                                     int32_t* iterations, void* workspace,
+                                                     size_t workspace_bytes,
+                                                     kronq_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
  * 6. The quantized layer at inference: packed codes and y = W^ x.
  *
  * [KronQ-gist] Limitations: once quantized, the layer's inference overhead is only the

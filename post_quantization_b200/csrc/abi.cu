@@ -378,6 +378,30 @@ kronq_status kronq_quantize_layer(const float* w, const float* k, const float* d
                       workspace, reinterpret_cast<cudaStream_t>(stream));
 }
 
+// ----------------------------------------------------------------------------- two-sided
+size_t kronq_quantize_layer_twosided_workspace_size(int32_t d_out, int32_t d_in) {
+  if (d_out <= 0 || d_in <= 0) return 0;
+  return twosided_workspace_bytes(d_out, d_in);
+}
+
+kronq_status kronq_quantize_layer_twosided(const float* w, const float* k_in, const float* k_out,
+                                           int32_t d_out, int32_t d_in, int32_t bits,
+                                           uint8_t* codes, float* scale, float* zero,
+                                           float* w_hat, int32_t* iterations, void* workspace,
+                                           size_t workspace_bytes, kronq_stream_t stream) {
+  if (d_out <= 0 || d_in <= 0) return fail(KRONQ_ERR_SHAPE, "d_out and d_in must be positive");
+  if (!w || !k_in || !k_out || !codes || !scale || !zero || !w_hat)
+    return fail(KRONQ_ERR_INVALID_ARG, "w, k_in, k_out, codes, scale, zero and w_hat are required");
+  if (bits < 2 || bits > 8) return fail(KRONQ_ERR_UNSUPPORTED, "bits must be in 2..8");
+  if (w == w_hat) return fail(KRONQ_ERR_INVALID_ARG, "w and w_hat must not alias");
+  if (d_out > 65535 || d_in > 65535)
+    return fail(KRONQ_ERR_SHAPE, "two-sided rounding takes at most 65535 rows and columns");
+  KQ_TRY(check_ws(workspace, workspace_bytes, twosided_workspace_bytes(d_out, d_in)));
+  KQ_TRY(kronq_device_check());
+  return run_twosided(w, k_in, k_out, d_out, d_in, bits, codes, scale, zero, w_hat, iterations,
+                      workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
 // ----------------------------------------------------------------------------- inference
 size_t kronq_packed_codes_bytes(int32_t d_out, int32_t d_in, int32_t bits) {
   if (d_out <= 0 || d_in <= 0 || bits < 2 || bits > 4) return 0;

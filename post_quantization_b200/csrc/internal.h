@@ -65,6 +65,12 @@ kronq_status run_quantize(const float* w, const float* k, const float* dxx, int 
                           int bits, int block, int group, uint8_t* codes, float* scale,
                           float* zero, float* w_hat, void* ws, cudaStream_t stream);
 
+// quantize.cu: rounding with feedback on both sides (comparison variant, not KronQ)
+size_t twosided_workspace_bytes(int d_out, int d_in);
+kronq_status run_twosided(const float* w, const float* k_in, const float* k_out, int d_out,
+                          int d_in, int bits, uint8_t* codes, float* scale, float* zero,
+                          float* w_hat, int32_t* iterations, void* ws, cudaStream_t stream);
+
 // qlinear.cu: the quantized layer at inference (packed codes, input/output transforms).
 struct QlinearArgs {
   const void* x;
@@ -96,7 +102,8 @@ kronq_status run_qlinear(const QlinearArgs& q, void* ws, cudaStream_t stream);
 //   GEMM_A_UPPER  A[m][k] = 0 for k < m
 //   GEMM_B_UPPER  op(B)[k][n] = 0 for k > n
 //   GEMM_B_LOWER  op(B)[k][n] = 0 for k < n
-enum { GEMM_A_UPPER = 1, GEMM_B_UPPER = 2, GEMM_B_LOWER = 4 };
+//   GEMM_A_LOWER  A[m][k] = 0 for k > m
+enum { GEMM_A_UPPER = 1, GEMM_B_UPPER = 2, GEMM_B_LOWER = 4, GEMM_A_LOWER = 8 };
 
 // tgemm.cu: fp32-accurate GEMM on tcgen05 tensor cores (bf16 x3 split, six products).
 //   An fp32 operand x is first split (split_bf16x3) into three bf16 pieces x0 + x1 + x2 that

@@ -406,4 +406,206 @@ kronq_status run_quantize(const float* w, const float* k, const float* dxx, int 
   return KRONQ_OK;
 }
 
+// ---------------------------------------------------------------------------------------------
+// Comparison variant (prior art, not KronQ): rounding with feedback on both sides.
+//
+// [YAQA notes], generalized LDLQ: for a Kronecker proxy H_O (x) H_I of the layer Hessian the
+// quantized W^ is the fixed point of
+//     W^ = Q(W + L_O'^T D L_I' + L_O'^T D + D L_I'),    D = W - W^,  L' = L - I,
+// L the unit upper triangular factor of H (H = L diag L^T), reached within m + n - 1 updates of
+// all elements at once, each update a pair of matrix products. Here H_I = H_X' and H_O = H_G'
+// (damped), so L = U diag(U)^-1 with U U^T = H + lambda I, U upper; U = K^-1 for the inverse
+// factor K of kronq_cholinv, and it is obtained with the same routine: by uniqueness of the
+// factorization, the inverse factor of K K^T is K^-1.
+// One update: S = D + D L_I' and T = W + (S - D) + L_O'^T S, then codes = Q(T) per row and
+// D = W - deq(codes). Both products read only the strictly triangular parts, so an element's
+// target never reads its own or a later element's error, and once no code changes the state is
+// the fixed point (the test that ends the loop).
+
+namespace {
+
+// The strictly triangular unit factor L' of U (upper, d x d), split into three bf16 pieces:
+// transpose 0: L'[i][j] = U[i][j] / U[j][j] for i < j, else 0;
+// transpose 1: the transpose, L'^T[i][j] = U[j][i] / U[i][i] for j < i, else 0.
+__global__ void unit_factor_split_kernel(const float* __restrict__ u, int d, int transpose,
+                                         uint16_t* __restrict__ p0, uint16_t* __restrict__ p1,
+                                         uint16_t* __restrict__ p2, int64_t ld) {
+  __shared__ float tile[32][33];
+  const int bx = blockIdx.x * 32, by = blockIdx.y * 32;   // output tile: rows by.., cols bx..
+  const int tx = threadIdx.x, ty = threadIdx.y;            // 32 x 8
+  if (transpose) {
+    // read the mirrored tile U[bx.., by..] row by row (coalesced), write it transposed
+    for (int r = ty; r < 32; r += 8) {
+      const int i = bx + r, j = by + tx;
+      tile[r][tx] = (i < d && j < d) ? u[static_cast<int64_t>(i) * d + j] : 0.f;
+    }
+    __syncthreads();
+  }
+  for (int r = ty; r < 32; r += 8) {
+    const int i = by + r, j = bx + tx;   // output element (i, j)
+    if (i >= d || j >= d) continue;
+    float v = 0.f;
+    if (!transpose) {
+      if (i < j) v = __fdiv_rn(u[static_cast<int64_t>(i) * d + j], u[static_cast<int64_t>(j) * d + j]);
+    } else {
+      if (j < i) v = __fdiv_rn(tile[tx][r], u[static_cast<int64_t>(i) * d + i]);
+    }
+    const __nv_bfloat16 b0 = __float2bfloat16_rn(v);
+    const float r1 = v - __bfloat162float(b0);
+    const __nv_bfloat16 b1 = __float2bfloat16_rn(r1);
+    const __nv_bfloat16 b2 = __float2bfloat16_rn(r1 - __bfloat162float(b1));
+    const int64_t o = static_cast<int64_t>(i) * ld + j;
+    p0[o] = __bfloat16_as_ushort(b0);
+    p1[o] = __bfloat16_as_ushort(b1);
+    p2[o] = __bfloat16_as_ushort(b2);
+  }
+}
+
+// One update of all elements (init: T = W). T = W + (S - D) + P2, code = Q(T) on the row's grid
+// (decisions in fp32, like the column solve), D = W - deq(code); counts the codes that changed.
+__global__ void twosided_step_kernel(const float* __restrict__ w, const float* __restrict__ s,
+                                     const float* __restrict__ p2, float* __restrict__ delta,
+                                     uint8_t* __restrict__ codes, float* __restrict__ w_hat,
+                                     const float* __restrict__ scale,
+                                     const float* __restrict__ zero, int d_out, int d_in,
+                                     float maxq, int init, unsigned int* __restrict__ changed) {
+  const int64_t total = static_cast<int64_t>(d_out) * d_in;
+  unsigned int local = 0;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int row = static_cast<int>(e / d_in);
+    const float wv = w[e];
+    float t = wv;
+    if (!init) t = __fadd_rn(__fadd_rn(wv, __fsub_rn(s[e], delta[e])), p2[e]);
+    const float sc = scale[row], zr = zero[row];
+    float code = __fadd_rn(rintf(__fdiv_rn(t, sc)), zr);
+    code = fminf(fmaxf(code, 0.f), maxq);
+    const float dq = __fmul_rn(sc, __fsub_rn(code, zr));
+    const uint8_t c8 = static_cast<uint8_t>(code);
+    if (init || c8 != codes[e]) ++local;
+    codes[e] = c8;
+    w_hat[e] = dq;
+    delta[e] = __fsub_rn(wv, dq);
+  }
+  local = __reduce_add_sync(0xffffffffu, local);
+  if ((threadIdx.x & 31) == 0 && local) atomicAdd(changed, local);
+}
+
+}  // namespace
+
+namespace {
+struct TwoWs {
+  float* u_in;       // d_in^2: K_in K_in^T, then its inverse factor U_in
+  float* u_out;      // d_out^2
+  Split3 kt;         // a split K (for K K^T), max(d_in, d_out)^2
+  Split3 li;         // L_I' split, d_in^2
+  Split3 lot;        // L_O'^T split, d_out^2
+  float* delta;      // d_out x d_in
+  float* s;
+  float* p2;
+  Split3 ms;         // split of D, then of S (d_out x d_in)
+  unsigned int* changed;
+  uint8_t* chol_ws;
+};
+
+size_t two_chol_bytes(int d_out, int d_in) {
+  const size_t a = cholinv_workspace_bytes(d_in), b = cholinv_workspace_bytes(d_out);
+  return a > b ? a : b;
+}
+
+TwoWs two_carve(void* ws, int d_out, int d_in) {
+  Carve cv{static_cast<uint8_t*>(ws)};
+  TwoWs t;
+  const int dm = d_in > d_out ? d_in : d_out;
+  t.u_in = cv.floats(static_cast<size_t>(d_in) * d_in);
+  t.u_out = cv.floats(static_cast<size_t>(d_out) * d_out);
+  t.kt = cv.split(dm, dm);
+  t.li = cv.split(d_in, d_in);
+  t.lot = cv.split(d_out, d_out);
+  t.delta = cv.floats(static_cast<size_t>(d_out) * d_in);
+  t.s = cv.floats(static_cast<size_t>(d_out) * d_in);
+  t.p2 = cv.floats(static_cast<size_t>(d_out) * d_in);
+  t.ms = cv.split(d_out, d_in);
+  t.changed = reinterpret_cast<unsigned int*>(cv.floats(64));
+  t.chol_ws = cv.p;
+  return t;
+}
+
+// U with U U^T = H + lambda I (upper), from the inverse factor K of H: U = chol_inv(K K^T).
+kronq_status inverse_of_factor(const float* k, int d, float* u, Split3 kt, void* chol_ws,
+                               int32_t* info, cudaStream_t stream) {
+  KQ_TRY(split_bf16x3(k, d, d, d, kt, stream));
+  // K K^T: A = K (upper), B given K-major as K itself (op(B)[k][n] = K[n][k], zero for k < n)
+  KQ_TRY(tgemm(d, d, d, 1.f, kt, kt, false, 0.f, u, d, false, GEMM_A_UPPER | GEMM_B_LOWER,
+               nullptr, stream));
+  KQ_TRY(run_cholinv(u, d, 0.f, info, chol_ws, stream));
+  return KRONQ_OK;
+}
+}  // namespace
+
+size_t twosided_workspace_bytes(int d_out, int d_in) {
+  const int dm = d_in > d_out ? d_in : d_out;
+  const size_t mn = static_cast<size_t>(d_out) * d_in;
+  return align256(sizeof(float) * static_cast<size_t>(d_in) * d_in) +
+         align256(sizeof(float) * static_cast<size_t>(d_out) * d_out) + split_bytes(dm, dm) +
+         split_bytes(d_in, d_in) + split_bytes(d_out, d_out) + 3 * align256(sizeof(float) * mn) +
+         split_bytes(d_out, d_in) + align256(sizeof(float) * 64) + two_chol_bytes(d_out, d_in);
+}
+
+kronq_status run_twosided(const float* w, const float* k_in, const float* k_out, int d_out,
+                          int d_in, int bits, uint8_t* codes, float* scale, float* zero,
+                          float* w_hat, int32_t* iterations, void* ws, cudaStream_t stream) {
+  const float maxq = static_cast<float>((1 << bits) - 1);
+  TwoWs t = two_carve(ws, d_out, d_in);
+  int32_t* info = reinterpret_cast<int32_t*>(t.changed + 16);
+  KQ_TRY(inverse_of_factor(k_in, d_in, t.u_in, t.kt, t.chol_ws, info, stream));
+  KQ_TRY(inverse_of_factor(k_out, d_out, t.u_out, t.kt, t.chol_ws, info, stream));
+  {
+    dim3 b(32, 8);
+    unit_factor_split_kernel<<<dim3((d_in + 31) / 32, (d_in + 31) / 32), b, 0, stream>>>(
+        t.u_in, d_in, 0, t.li.part[0], t.li.part[1], t.li.part[2], t.li.ld);
+    KQ_TRY(check_launch("unit_factor_split_kernel"));
+    unit_factor_split_kernel<<<dim3((d_out + 31) / 32, (d_out + 31) / 32), b, 0, stream>>>(
+        t.u_out, d_out, 1, t.lot.part[0], t.lot.part[1], t.lot.part[2], t.lot.ld);
+    KQ_TRY(check_launch("unit_factor_split_kernel"));
+  }
+  grid_kernel<<<(d_out + 7) / 8, 256, 0, stream>>>(w, d_out, d_in, maxq, scale, zero);
+  KQ_TRY(check_launch("grid_kernel"));
+  const int64_t total = static_cast<int64_t>(d_out) * d_in;
+  int64_t blocks = (total + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(device_sms()) * 8;
+  if (blocks > cap) blocks = cap;
+  const size_t mn_bytes = sizeof(float) * static_cast<size_t>(total);
+  int it = 0;
+  bool done = false;
+  // init: codes = Q(W), D = W - deq; then updates until no code changes (at most m + n)
+  for (; it <= d_out + d_in && !done; ++it) {
+    if (it > 0) {
+      // S = D + D L_I'
+      KQ_CUDA_TRY(cudaMemcpyAsync(t.s, t.delta, mn_bytes, cudaMemcpyDeviceToDevice, stream));
+      KQ_TRY(split_bf16x3(t.delta, d_in, d_out, d_in, t.ms, stream));
+      KQ_TRY(tgemm(d_out, d_in, d_in, 1.f, t.ms, t.li, true, 1.f, t.s, d_in, false,
+                   GEMM_B_UPPER, nullptr, stream));
+      // P2 = L_O'^T S
+      KQ_TRY(split_bf16x3(t.s, d_in, d_out, d_in, t.ms, stream));
+      KQ_TRY(tgemm(d_out, d_in, d_out, 1.f, t.lot, t.ms, true, 0.f, t.p2, d_in, false,
+                   GEMM_A_LOWER, nullptr, stream));
+    }
+    KQ_CUDA_TRY(cudaMemsetAsync(t.changed, 0, sizeof(unsigned int), stream));
+    twosided_step_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(
+        w, t.s, t.p2, t.delta, codes, w_hat, scale, zero, d_out, d_in, maxq, it == 0 ? 1 : 0,
+        t.changed);
+    KQ_TRY(check_launch("twosided_step_kernel"));
+    unsigned int host = 0;
+    KQ_CUDA_TRY(cudaMemcpyAsync(&host, t.changed, sizeof(host), cudaMemcpyDeviceToHost, stream));
+    KQ_CUDA_TRY(cudaStreamSynchronize(stream));
+    if (it > 0 && host == 0) done = true;
+  }
+  if (iterations) *iterations = it - 1;   // update passes, the last one changing no code
+  if (!done)
+    return fail(KRONQ_ERR_CUDA, "two-sided rounding did not reach its fixed point in %d updates",
+                d_out + d_in);
+  return KRONQ_OK;
+}
+
 }  // namespace kq

@@ -89,6 +89,7 @@ __device__ __forceinline__ bool tile_info(const TgParams& p, int t, TileInfo& ti
   if (p.upper_only && bm > bn + C::BN - 1) return false;   // entirely below the diagonal
   int k_lo = 0, k_hi = p.k;
   if (p.tri & GEMM_A_UPPER) k_lo = max(k_lo, bm);
+  if (p.tri & GEMM_A_LOWER) k_hi = min(k_hi, bm + tg::BM);
   if (p.tri & GEMM_B_LOWER) k_lo = max(k_lo, bn);
   if (p.tri & GEMM_B_UPPER) k_hi = min(k_hi, bn + C::BN);
   ti.kb0 = k_lo / C::BK;

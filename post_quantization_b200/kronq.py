@@ -48,6 +48,7 @@ SYMBOLS = (
     "kronq_cholinv_workspace_size", "kronq_cholinv",
     "kronq_quantize_layer_workspace_size", "kronq_quantize_layer",
     "kronq_score_allocate",
+    "kronq_quantize_layer_twosided_workspace_size", "kronq_quantize_layer_twosided",
     "kronq_packed_codes_bytes", "kronq_pack_codes", "kronq_packed_grid_bytes", "kronq_pack_grid",
     "kronq_qlinear_workspace_size", "kronq_qlinear",
 )
@@ -112,6 +113,10 @@ def load_library(path: str = LIB_PATH):
                                          c_sz, c_void_p]),
         "kronq_score_allocate": (c_i32, [c_void_p, c_void_p, c_void_p, c_i32, c_void_p, c_i32,
                                          c_dbl, c_void_p, c_void_p]),
+        "kronq_quantize_layer_twosided_workspace_size": (c_sz, [c_i32, c_i32]),
+        "kronq_quantize_layer_twosided": (c_i32, [c_void_p, c_void_p, c_void_p, c_i32, c_i32,
+                                                  c_i32, c_void_p, c_void_p, c_void_p, c_void_p,
+                                                  c_void_p, c_void_p, c_sz, c_void_p]),
         "kronq_packed_codes_bytes": (c_sz, [c_i32, c_i32, c_i32]),
         "kronq_pack_codes": (c_i32, [c_void_p, c_i32, c_i32, c_i32, c_void_p, c_sz, c_void_p]),
         "kronq_packed_grid_bytes": (c_sz, [c_i32, c_i32, c_i32]),
@@ -311,6 +316,30 @@ def kronq_score_allocate(tr_hx, tr_hg, n_params, choices, avg_bits):
     st = lib.kronq_score_allocate(a, b, n, L, ch, len(choices), float(avg_bits), s, bits)
     _check(st, "kronq_score_allocate")
     return list(s), list(bits)
+
+
+# ------------------------------------------------------------------------------ comparison variant
+
+def kronq_quantize_layer_twosided(w, k_in, k_out, bits, codes=None, scale=None, zero=None,
+                                  w_hat=None, workspace=None, stream=None):
+    """Rounding with input- and output-side feedback (prior art, for comparison).
+    Returns (codes, scale, zero, w_hat, iterations)."""
+    lib = load_library()
+    d_out, d_in = w.shape
+    dev = w.device
+    codes = codes if codes is not None else torch.empty(d_out, d_in, dtype=torch.uint8, device=dev)
+    scale = scale if scale is not None else torch.empty(d_out, dtype=torch.float32, device=dev)
+    zero = zero if zero is not None else torch.empty(d_out, dtype=torch.float32, device=dev)
+    w_hat = w_hat if w_hat is not None else torch.empty(d_out, d_in, dtype=torch.float32,
+                                                        device=dev)
+    ws, wsb = _workspace(lib.kronq_quantize_layer_twosided_workspace_size(d_out, d_in), dev,
+                         workspace)
+    it = ctypes.c_int32(0)
+    st = lib.kronq_quantize_layer_twosided(_p(w), _p(k_in), _p(k_out), d_out, d_in, int(bits),
+                                           _p(codes), _p(scale), _p(zero), _p(w_hat),
+                                           ctypes.byref(it), _p(ws), wsb, _stream(stream))
+    _check(st, "kronq_quantize_layer_twosided")
+    return codes, scale, zero, w_hat, it.value
 
 
 # ------------------------------------------------------------------------------ 6. inference

@@ -7,6 +7,8 @@
     python -m post_quantization_b200.profcase biip --d-out 4096 --d-in 4096
     python -m post_quantization_b200.profcase cholinv --d 4096
     python -m post_quantization_b200.profcase quantize --d-out 4096 --d-in 4096
+    python -m post_quantization_b200.profcase twosided --d-out 1024 --d-in 1024 --bits 2
+        the comparison variant with output-side feedback against the column solve
     python -m post_quantization_b200.profcase qlinear --block --bits 2 --group 128 --tokens 1
         the quantized layers at inference, per layer (graph replays) and as one block sweep
 Each case runs its call `--reps` times (default 3) after one warm-up call.
@@ -104,6 +106,49 @@ def case_acc(args):
     ms = a.elapsed_time(b) / args.reps
     print(json.dumps({"case": "acc", "d": d, "tokens": n, "drift": args.drift, "ms": ms,
                       "tflops": flops / ms / 1e9}))
+
+
+def case_twosided(args):
+    """The comparison variant (output-side feedback too) against KronQ's column solve on one
+    layer: time per call, update passes, and the Kronecker objective tr[H_G dW H_X dW^T] of both
+    (fp64 on the device; a measurement, not part of the library)."""
+    d_out, d_in, n, bits = args.d_out, args.d_in, max(2 * args.d_in, 4096), args.bits
+    x = synth.correlated_x(n, d_in, synth.seed_for("pc-2s", "x"), device="cuda")
+    g = synth.gradients(n, d_out, synth.seed_for("pc-2s", "g"), device="cuda")
+    w = synth.weight(d_out, d_in, synth.seed_for("pc-2s", "w"), device="cuda")
+    si = synth.rademacher(d_in, 1, device="cuda"); so = synth.rademacher(d_out, 2, device="cuda")
+    hx = torch.zeros(d_in, d_in, device="cuda"); hg = torch.zeros(d_out, d_out, device="cuda")
+    P.accumulate(xq=x, g=g, hx_sum=hx, hg_sum=hg)
+    r = P.biip(w, hx, hg, None, 1.0 / n, si, so, K.BIIP_FULL | K.BIIP_WRITE_HG)
+    hx_p, hg_p = r.hx.clone(), hg.clone()
+    P.cholinv(r, 0.01, sync=True)
+    k_out = hg.clone()
+    info = torch.empty(1, dtype=torch.int32, device="cuda")
+    K.kronq_cholinv(k_out, 0.01, info, K.CHOLINV_SYNC)
+    out = K.kronq_quantize_layer_twosided(r.w_prime, r.hx, k_out, bits)
+    P.quantize(r, bits)
+    torch.cuda.synchronize()
+    a, b = ev(), ev()
+    a.record()
+    out = K.kronq_quantize_layer_twosided(r.w_prime, r.hx, k_out, bits)
+    b.record()
+    torch.cuda.synchronize()
+    ms2 = a.elapsed_time(b)
+    a.record()
+    P.quantize(r, bits)
+    b.record()
+    torch.cuda.synchronize()
+    ms1 = a.elapsed_time(b)
+    wp = r.w_prime.double()
+
+    def obj(wh):
+        dw = wp - wh.double()
+        return float(torch.trace(hg_p.double() @ dw @ hx_p.double() @ dw.T))
+    o1, o2 = obj(r.w_hat), obj(out[3])
+    print(json.dumps({"case": "twosided", "d_out": d_out, "d_in": d_in, "bits": bits,
+                      "updates": out[4], "ms_twosided": ms2, "ms_column_solve": ms1,
+                      "objective_column_solve": o1, "objective_twosided": o2,
+                      "objective_ratio": o2 / o1}))
 
 
 def case_peaks(args):
@@ -332,7 +377,7 @@ def case_qlinear(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("case", choices=["stages", "acc", "biip", "cholinv", "quantize", "qlinear",
-                                     "peaks"])
+                                     "peaks", "twosided"])
     ap.add_argument("--drift", action="store_true", help="acc: the drift sum D alone; "
                                                           "quantize: with D (P pre-shift)")
     ap.add_argument("--tokens", type=int, default=None)
@@ -348,7 +393,8 @@ def main():
     K.load_library()
     K.kronq_device_check()
     {"stages": stages, "acc": case_acc, "biip": case_biip, "cholinv": case_cholinv,
-     "quantize": case_quantize, "qlinear": case_qlinear, "peaks": case_peaks}[args.case](args)
+     "quantize": case_quantize, "qlinear": case_qlinear, "peaks": case_peaks,
+     "twosided": case_twosided}[args.case](args)
 
 
 if __name__ == "__main__":
