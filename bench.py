@@ -757,14 +757,29 @@ TRAFFIC = {}
 
 
 def _mem_available():
+    """Host memory this process may still use: MemAvailable, capped by the container's memory
+    limit (cgroup v2 memory.max - memory.current, or v1 limit - usage) when there is one."""
+    avail = None
     try:
         with open("/proc/meminfo") as f:
             for line in f:
                 if line.startswith("MemAvailable:"):
-                    return int(line.split()[1]) * 1024
+                    avail = int(line.split()[1]) * 1024
     except OSError:
         pass
-    return None
+    for lim_f, use_f in (("/sys/fs/cgroup/memory.max", "/sys/fs/cgroup/memory.current"),
+                         ("/sys/fs/cgroup/memory/memory.limit_in_bytes",
+                          "/sys/fs/cgroup/memory/memory.usage_in_bytes")):
+        try:
+            lim = open(lim_f).read().strip()
+            use = int(open(use_f).read().strip())
+        except (OSError, ValueError):
+            continue
+        if lim.isdigit() and int(lim) < (1 << 60):
+            room = int(lim) - use
+            avail = room if avail is None else min(avail, room)
+        break
+    return avail
 
 
 def run_e2e(blk, args, world, dist, barrier):
@@ -805,7 +820,7 @@ def run_e2e(blk, args, world, dist, barrier):
             h = host_buf[off:off + sz].view(t.dtype).view(t.shape)
             h.copy_(t)
             host[(kind, name)] = h
-        assert all(h.is_pinned() for h in host.values())
+        pinned = all(h.is_pinned() for h in host.values())
         h2d = sum(sizes)
         # the device copies are written by every streamed step (same shapes, same addresses)
         copy_stream = torch.cuda.Stream(device=blk.dev)
@@ -846,7 +861,9 @@ def run_e2e(blk, args, world, dist, barrier):
         value = blk.wl.params_per_block * world * steps / float(t)
         return {"value": value, "unit": "params/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": steps,
-                "ms_per_step": float(t) / steps * 1e3}
+                "ms_per_step": float(t) / steps * 1e3,
+                "host_inputs": "one registered (page-locked) buffer" if pinned else
+                               "registered buffer not reported page-locked: staged copies"}
     finally:
         torch.cuda.synchronize()
         cudart.cudaHostUnregister(host_buf.data_ptr())
