@@ -31,6 +31,10 @@
 #include "common.cuh"
 #include "internal.h"
 
+#ifndef KQ_ACC_UNIT_KBLOCKS
+#define KQ_ACC_UNIT_KBLOCKS 256   // 16384 tokens
+#endif
+
 namespace kq {
 
 namespace acc {
@@ -533,8 +537,9 @@ kronq_status launch_accumulate_tc(const void* a, int64_t ld_a, const void* b, in
   }
   const int sms = device_sms();
   const int kblocks = static_cast<int>((k + BK - 1) / BK);
-  // Token chunk per unit: about 16K tokens, fewer when there are too few tiles to fill the GPU.
-  int per = 256;
+  // Token chunk per unit: at most KQ_ACC_UNIT_KBLOCKS blocks of 64 tokens, fewer when there are
+  // too few tiles to fill the GPU.
+  int per = KQ_ACC_UNIT_KBLOCKS;
   while (per > 8 && static_cast<int64_t>(p.num_tiles) * ((kblocks + per - 1) / per) < 8 * sms)
     per >>= 1;
   if (per > kblocks) per = kblocks;
