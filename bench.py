@@ -751,9 +751,9 @@ def run_gpu(args):
 
 
 # DRAM bytes (read + write) per accumulate_tc_kernel launch, averaged over the launches of one
-# step, from ncu captures of this kernel version (commands in the accumulate profile summary
-# under profiles/); keyed by (workload, tokens)
-TRAFFIC = {}
+# step: bounded ncu captures of this kernel version scaled to the step's launches (commands and
+# scaling in the accumulate profile summaries under profiles/); keyed by (workload, tokens)
+TRAFFIC = {("llama3_70b_block", 262144): 29.9e9}
 
 
 def _mem_available():
@@ -798,26 +798,25 @@ def run_e2e(blk, args, world, dist, barrier):
     torch.cuda.empty_cache()
     items = blk.inputs()
     sizes = [t.numel() * t.element_size() for _, _, t in items]
-    offs, total = [], 0
-    for sz in sizes:
-        offs.append(total)
-        total += (sz + 4095) // 4096 * 4096
+    total = sum((sz + 4095) // 4096 * 4096 for sz in sizes)
     avail = _mem_available()
-    # one host buffer for all inputs, page-locked by registration (the pinned-tensor allocator
-    # would round each tensor up to a power of two)
+    # host copies of the inputs, each page-locked by registration (the pinned-tensor allocator
+    # would round every tensor up to a power of two)
     if avail is not None and total > avail - 24e9:
         return {"value": None, "unit": "params/s",
                 "skipped": f"needs {total / 1e9:.0f} GB of page-locked host memory, "
                            f"{avail / 1e9:.0f} GB available"}
-    host_buf = torch.empty(total, dtype=torch.uint8)
     cudart = torch.cuda.cudart()
-    rc = cudart.cudaHostRegister(host_buf.data_ptr(), total, 0)
-    if int(rc) != 0:
-        return {"value": None, "unit": "params/s", "skipped": f"cudaHostRegister failed ({rc})"}
+    registered = []
     try:
         host = {}
-        for (kind, name, t), off, sz in zip(items, offs, sizes):
-            h = host_buf[off:off + sz].view(t.dtype).view(t.shape)
+        for (kind, name, t), sz in zip(items, sizes):
+            h = torch.empty(t.shape, dtype=t.dtype)
+            rc = cudart.cudaHostRegister(h.data_ptr(), sz, 0)
+            if int(rc) != 0:
+                return {"value": None, "unit": "params/s",
+                        "skipped": f"cudaHostRegister failed ({rc})"}
+            registered.append(h)
             h.copy_(t)
             host[(kind, name)] = h
         pinned = all(h.is_pinned() for h in host.values())
@@ -862,11 +861,12 @@ def run_e2e(blk, args, world, dist, barrier):
         return {"value": value, "unit": "params/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": steps,
                 "ms_per_step": float(t) / steps * 1e3,
-                "host_inputs": "one registered (page-locked) buffer" if pinned else
+                "host_inputs": "registered (page-locked) host tensors" if pinned else
                                "registered buffer not reported page-locked: staged copies"}
     finally:
         torch.cuda.synchronize()
-        cudart.cudaHostUnregister(host_buf.data_ptr())
+        for h in registered:
+            cudart.cudaHostUnregister(h.data_ptr())
 
 
 # ---------------------------------------------------------------------------------- stack

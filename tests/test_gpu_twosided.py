@@ -37,11 +37,22 @@ def h64(t):
     return t.detach().double().cpu().numpy()
 
 
+def padded(t):
+    """Same values in storage whose row stride is a multiple of 8 elements (16 bytes), as the
+    statistics call requires of its bf16 inputs."""
+    c = t.shape[1]
+    if c % 8 == 0:
+        return t
+    base = torch.zeros(t.shape[0], (c + 7) // 8 * 8, dtype=t.dtype, device=t.device)
+    base[:, :c] = t
+    return base[:, :c]
+
+
 def layer(K, d_out, d_in, n, tag):
     """W', H_X' and the full H_G' of a synthetic layer through the library (fp32 on device)."""
     from post_quantization_b200 import pipeline as P
-    x = synth.correlated_x(n, d_in, synth.seed_for(tag, "X"), device="cuda")
-    g = synth.gradients(n, d_out, synth.seed_for(tag, "G"), device="cuda")
+    x = padded(synth.correlated_x(n, d_in, synth.seed_for(tag, "X"), device="cuda"))
+    g = padded(synth.gradients(n, d_out, synth.seed_for(tag, "G"), device="cuda"))
     w = synth.weight(d_out, d_in, synth.seed_for(tag, "W"), dtype=torch.float32, device="cuda")
     si = synth.rademacher(d_in, synth.seed_for(tag, "si"), device="cuda")
     so = synth.rademacher(d_out, synth.seed_for(tag, "so"), device="cuda")
