@@ -52,9 +52,13 @@ def parse():
                          "copies of the phase's outputs); auto: on when the block's inputs "
                          "take less than 60 GB of device memory")
     ap.add_argument("--no-graphs", action="store_true", help=argparse.SUPPRESS)
+    ap.add_argument("--schedule", default="phases", choices=["phases", "overlapped"],
+                    help="phases: all statistics, then every sublayer's BiIP, inverse factor and "
+                         "solve; overlapped: each sublayer's chain starts when its sums are "
+                         "complete, beside the remaining statistics")
     ap.add_argument("--overlap", type=int, default=0, metavar="SMS",
-                    help="run each sublayer's BiIP and inverse factor alongside the remaining "
-                         "statistics on SMS reserved SMs (0: phases one after another)")
+                    help="overlapped schedule with SMS SMs kept free of statistics for the "
+                         "chains (0: no reservation)")
     ap.add_argument("--calibration", default="synthetic", choices=["synthetic", "backward"],
                     help="synthetic: seeded X and G generators; backward: X and G of every linear "
                          "from the forward and backward of a random-weight block")
@@ -471,12 +475,19 @@ class Block:
             st["streams"] = [torch.cuda.Stream(device=self.dev) for _ in subs]
             st["ws"] = [P.Workspace(self.dev) for _ in subs]
 
+            # with one bit width the allocation is known before any trace: each sublayer's
+            # solve then follows its inverse factor at once, beside the remaining statistics
+            st["fixed_bits"] = wl.extra.get("choices", (wl.bits,))
+            st["fixed_bits"] = st["fixed_bits"][0] if len(st["fixed_bits"]) == 1 else None
+
             def chain(i):
                 sl = subs[i]
                 r = P.biip(self.w[sl.name], self.hx[sl.x_stream], self.hg[sl.name],
                            self.dxx[sl.x_stream] if self.drift else None, inv_n,
                            self.si[sl.name], self.so[sl.name], self.biip_flags, ws=st["ws"][i])
                 P.cholinv(r, 0.01, st["ws"][i])
+                if st["fixed_bits"] is not None:
+                    P.quantize(r, st["fixed_bits"], st["ws"][i])
                 return r
             st["chain"] = [P.CapturedPhase(lambda i=i: chain(i)) if self.use_graphs
                            else (lambda i=i: chain(i)) for i in range(len(subs))]
@@ -525,6 +536,8 @@ class Block:
         _, self.bits = K.kronq_score_allocate(tr[:, 0].tolist(), tr[:, 1].tolist(),
                                               [sl.d_out * sl.d_in for sl in subs], choices, avg)
         bits = list(self.bits)
+        if st["fixed_bits"] is not None:
+            return                  # every sublayer was solved in its chain
 
         def solve():
             for j in st["order"]:
@@ -625,7 +638,7 @@ def run_gpu(args):
     if args.no_graphs:
         graphs = "off"
     blk.use_graphs = graphs == "on" or (graphs == "auto" and blk.input_bytes() < 60e9)
-    blk.overlap = args.overlap > 0
+    blk.overlap = args.overlap > 0 or args.schedule == "overlapped"
     blk.reserve = args.overlap
     torch.cuda.synchronize()
 
@@ -705,6 +718,9 @@ def run_gpu(args):
                        "tokens": n_tok, "params_per_block": wl.params_per_block,
                        "parallelism": f"one block per GPU x{world}",
                        "graphs": blk.use_graphs,
+                       "schedule": ("overlapped" + (f", {blk.reserve} SMs reserved"
+                                                    if blk.reserve else "")
+                                    if blk.overlap else "phases"),
                        "calibration": ("X and G from the forward and backward of a random-weight "
                                        "block" if args.calibration == "backward" else
                                        "seeded synthetic X and G"),

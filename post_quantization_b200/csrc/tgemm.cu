@@ -30,16 +30,21 @@
 namespace kq {
 
 namespace tg {
-constexpr int BM = 128, UK = 16, STAGES = 2, THREADS = 192;
-constexpr int EPI_BYTES = 4 * 32 * 33 * 4;        // per epilogue warp: a 32 x 32 transpose tile
+constexpr int BM = 128, UK = 16, THREADS = 192;
 
 // Two tile shapes. A tcgen05 MMA takes about the same time for any N up to 256, so the 128 x 256
 // tile runs the tensor pipe at twice the rate of the 128 x 128 one. Its operand pieces are
 // K = 32 deep (64-byte rows, 64-byte swizzle) so that two pipeline stages of the six pieces still
 // fit in shared memory; the 128 x 128 tile keeps K = 64 (128-byte rows, 128-byte swizzle).
+// The 128 x 256 tile keeps three stages in flight: its epilogue stages 32 x 16 halves of each
+// 32-column chunk (the 128 x 128 tile stages whole 32 x 32 chunks, with two stages).
 template <int BN_>
 struct Cfg {
   static constexpr int BN = BN_;
+  static constexpr int STAGES = BN_ == 256 ? 3 : 2;
+  static constexpr int EPI_COLS = BN_ == 256 ? 16 : 32;     // columns staged per pass
+  static constexpr int EPI_LD = EPI_COLS + 1;
+  static constexpr int EPI_BYTES = 4 * 32 * EPI_LD * 4;     // per warp: 32 rows x EPI_COLS
   static constexpr int BK = BN_ == 256 ? 32 : 64;
   static constexpr int ROW_BYTES = BK * 2;                  // one K-major row of a piece
   static constexpr uint32_t KSW = BN_ == 256 ? 4u : 2u;     // descriptor layout: 64B / 128B swizzle
@@ -108,6 +113,7 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
   using namespace tg;
   using C = Cfg<BN_>;
   constexpr int BN = C::BN, BK = C::BK, STAGE_BYTES = C::STAGE_BYTES, TMEM_COLS = C::TMEM_COLS;
+  constexpr int STAGES = C::STAGES, EPI_BYTES = C::EPI_BYTES, EPI_LD = C::EPI_LD;
   constexpr int A_PIECE = C::A_PIECE, B_PIECE = C::B_PIECE, MN_BOX_BYTES = C::MN_BOX_BYTES;
   if (p.skip && *p.skip >= 0) return;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -268,32 +274,64 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
       const bool has_k = ti.kb1 > ti.kb0;
       const int row0 = ti.tm * BM + q * 32;        // this warp's 32 rows
       const uint32_t taddr = tmem_base + ((q * 32u) << 16) + a * BN;
-      float* tw = epi + q * (32 * 33);              // transpose tile of this warp
+      float* tw = epi + q * (32 * EPI_LD);          // transpose tile of this warp
 #pragma unroll 1
       for (int cb = 0; cb < BN / 32; ++cb) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(taddr + cb * 32, v);
         tmem_ld_wait();
-        // lane = row: stage the 32 x 32 chunk, then lane = column for coalesced C traffic
+        if constexpr (C::EPI_COLS == 32) {
+          // lane = row: stage the 32 x 32 chunk, then lane = column for coalesced C traffic
 #pragma unroll
-        for (int j = 0; j < 32; ++j) tw[lane * 33 + j] = has_k ? __uint_as_float(v[j]) : 0.f;
-        __syncwarp();
-        const int col = ti.tn * BN + cb * 32 + lane;
-        float* cbase = p.c + static_cast<int64_t>(row0) * p.ldc + col;
-        float old[32];
-        // all 32 loads of C are issued before any is used
+          for (int j = 0; j < 32; ++j) tw[lane * EPI_LD + j] = has_k ? __uint_as_float(v[j]) : 0.f;
+          __syncwarp();
+          const int col = ti.tn * BN + cb * 32 + lane;
+          float* cbase = p.c + static_cast<int64_t>(row0) * p.ldc + col;
+          float old[32];
+          // all 32 loads of C are issued before any is used
 #pragma unroll
-        for (int r = 0; r < 32; ++r) {
-          const bool ok_rc = col < p.n && row0 + r < p.m && !(p.upper_only && col < row0 + r);
-          old[r] = (ok_rc && p.beta != 0.f) ? cbase[static_cast<int64_t>(r) * p.ldc] : 0.f;
+          for (int r = 0; r < 32; ++r) {
+            const bool ok_rc = col < p.n && row0 + r < p.m && !(p.upper_only && col < row0 + r);
+            old[r] = (ok_rc && p.beta != 0.f) ? cbase[static_cast<int64_t>(r) * p.ldc] : 0.f;
+          }
+#pragma unroll
+          for (int r = 0; r < 32; ++r) {
+            const bool ok_rc = col < p.n && row0 + r < p.m && !(p.upper_only && col < row0 + r);
+            if (ok_rc)
+              cbase[static_cast<int64_t>(r) * p.ldc] =
+                  fmaf(p.beta, old[r], p.alpha * tw[r * EPI_LD + lane]);
+          }
+          __syncwarp();
+        } else {
+          // two 32 x 16 halves: lane = row to stage, then lanes 0..15 and 16..31 take the 16
+          // columns of two rows at a time (two 64-byte segments per access)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              tw[lane * EPI_LD + j] = has_k ? __uint_as_float(v[16 * h + j]) : 0.f;
+            __syncwarp();
+            const int cl = lane & 15, rh = lane >> 4;
+            const int col = ti.tn * BN + cb * 32 + 16 * h + cl;
+            float* cbase = p.c + static_cast<int64_t>(row0 + rh) * p.ldc + col;
+            float old[16];
+#pragma unroll
+            for (int it = 0; it < 16; ++it) {
+              const int r = 2 * it + rh;
+              const bool ok_rc = col < p.n && row0 + r < p.m && !(p.upper_only && col < row0 + r);
+              old[it] = (ok_rc && p.beta != 0.f) ? cbase[static_cast<int64_t>(2 * it) * p.ldc] : 0.f;
+            }
+#pragma unroll
+            for (int it = 0; it < 16; ++it) {
+              const int r = 2 * it + rh;
+              const bool ok_rc = col < p.n && row0 + r < p.m && !(p.upper_only && col < row0 + r);
+              if (ok_rc)
+                cbase[static_cast<int64_t>(2 * it) * p.ldc] =
+                    fmaf(p.beta, old[it], p.alpha * tw[r * EPI_LD + cl]);
+            }
+            __syncwarp();
+          }
         }
-#pragma unroll
-        for (int r = 0; r < 32; ++r) {
-          const bool ok_rc = col < p.n && row0 + r < p.m && !(p.upper_only && col < row0 + r);
-          if (ok_rc)
-            cbase[static_cast<int64_t>(r) * p.ldc] = fmaf(p.beta, old[r], p.alpha * tw[r * 33 + lane]);
-        }
-        __syncwarp();
       }
       tc_fence_before();
       __syncwarp();
