@@ -417,10 +417,12 @@ kronq_status run_quantize(const float* w, const float* k, const float* dxx, int 
 // (damped), so L = U diag(U)^-1 with U U^T = H + lambda I, U upper; U = K^-1 for the inverse
 // factor K of kronq_cholinv, and it is obtained with the same routine: by uniqueness of the
 // factorization, the inverse factor of K K^T is K^-1.
-// One update: S = D + D L_I' and T = W + (S - D) + L_O'^T S, then codes = Q(T) per row and
-// D = W - deq(codes). Both products read only the strictly triangular parts, so an element's
-// target never reads its own or a later element's error, and once no code changes the state is
-// the fixed point (the test that ends the loop).
+// One update: P1 = D L_I', S = D + P1, P2 = L_O'^T S, T = W + P1 + P2, then codes = Q(T) per
+// row and D = W - deq(codes). Both products read only the strictly triangular parts, and T
+// reads P1 and P2 directly (not S - D, whose rounding would carry the element's own error), so
+// an element's target reads only strictly earlier elements' errors: in floating point too, the
+// iteration settles within d_out + d_in - 1 updates, and once no code changes the state is the
+// fixed point (the test that ends the loop).
 
 namespace {
 
@@ -461,9 +463,17 @@ __global__ void unit_factor_split_kernel(const float* __restrict__ u, int d, int
   }
 }
 
-// One update of all elements (init: T = W). T = W + (S - D) + P2, code = Q(T) on the row's grid
+// S = D + P1, elementwise.
+__global__ void add_kernel(const float* __restrict__ a, const float* __restrict__ b,
+                           float* __restrict__ out, int64_t total) {
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    out[e] = __fadd_rn(a[e], b[e]);
+}
+
+// One update of all elements (init: T = W). T = W + P1 + P2, code = Q(T) on the row's grid
 // (decisions in fp32, like the column solve), D = W - deq(code); counts the codes that changed.
-__global__ void twosided_step_kernel(const float* __restrict__ w, const float* __restrict__ s,
+__global__ void twosided_step_kernel(const float* __restrict__ w, const float* __restrict__ p1,
                                      const float* __restrict__ p2, float* __restrict__ delta,
                                      uint8_t* __restrict__ codes, float* __restrict__ w_hat,
                                      const float* __restrict__ scale,
@@ -476,7 +486,7 @@ __global__ void twosided_step_kernel(const float* __restrict__ w, const float* _
     const int row = static_cast<int>(e / d_in);
     const float wv = w[e];
     float t = wv;
-    if (!init) t = __fadd_rn(__fadd_rn(wv, __fsub_rn(s[e], delta[e])), p2[e]);
+    if (!init) t = __fadd_rn(__fadd_rn(wv, p1[e]), p2[e]);
     const float sc = scale[row], zr = zero[row];
     float code = __fadd_rn(rintf(__fdiv_rn(t, sc)), zr);
     code = fminf(fmaxf(code, 0.f), maxq);
@@ -501,6 +511,7 @@ struct TwoWs {
   Split3 li;         // L_I' split, d_in^2
   Split3 lot;        // L_O'^T split, d_out^2
   float* delta;      // d_out x d_in
+  float* p1;
   float* s;
   float* p2;
   Split3 ms;         // split of D, then of S (d_out x d_in)
@@ -523,6 +534,7 @@ TwoWs two_carve(void* ws, int d_out, int d_in) {
   t.li = cv.split(d_in, d_in);
   t.lot = cv.split(d_out, d_out);
   t.delta = cv.floats(static_cast<size_t>(d_out) * d_in);
+  t.p1 = cv.floats(static_cast<size_t>(d_out) * d_in);
   t.s = cv.floats(static_cast<size_t>(d_out) * d_in);
   t.p2 = cv.floats(static_cast<size_t>(d_out) * d_in);
   t.ms = cv.split(d_out, d_in);
@@ -548,7 +560,7 @@ size_t twosided_workspace_bytes(int d_out, int d_in) {
   const size_t mn = static_cast<size_t>(d_out) * d_in;
   return align256(sizeof(float) * static_cast<size_t>(d_in) * d_in) +
          align256(sizeof(float) * static_cast<size_t>(d_out) * d_out) + split_bytes(dm, dm) +
-         split_bytes(d_in, d_in) + split_bytes(d_out, d_out) + 3 * align256(sizeof(float) * mn) +
+         split_bytes(d_in, d_in) + split_bytes(d_out, d_out) + 4 * align256(sizeof(float) * mn) +
          split_bytes(d_out, d_in) + align256(sizeof(float) * 64) + two_chol_bytes(d_out, d_in);
 }
 
@@ -575,17 +587,17 @@ kronq_status run_twosided(const float* w, const float* k_in, const float* k_out,
   int64_t blocks = (total + 255) / 256;
   const int64_t cap = static_cast<int64_t>(device_sms()) * 8;
   if (blocks > cap) blocks = cap;
-  const size_t mn_bytes = sizeof(float) * static_cast<size_t>(total);
   int it = 0;
   bool done = false;
   // init: codes = Q(W), D = W - deq; then updates until no code changes (at most m + n)
   for (; it <= d_out + d_in && !done; ++it) {
     if (it > 0) {
-      // S = D + D L_I'
-      KQ_CUDA_TRY(cudaMemcpyAsync(t.s, t.delta, mn_bytes, cudaMemcpyDeviceToDevice, stream));
+      // P1 = D L_I', S = D + P1
       KQ_TRY(split_bf16x3(t.delta, d_in, d_out, d_in, t.ms, stream));
-      KQ_TRY(tgemm(d_out, d_in, d_in, 1.f, t.ms, t.li, true, 1.f, t.s, d_in, false,
+      KQ_TRY(tgemm(d_out, d_in, d_in, 1.f, t.ms, t.li, true, 0.f, t.p1, d_in, false,
                    GEMM_B_UPPER, nullptr, stream));
+      add_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(t.delta, t.p1, t.s, total);
+      KQ_TRY(check_launch("add_kernel"));
       // P2 = L_O'^T S
       KQ_TRY(split_bf16x3(t.s, d_in, d_out, d_in, t.ms, stream));
       KQ_TRY(tgemm(d_out, d_in, d_out, 1.f, t.lot, t.ms, true, 0.f, t.p2, d_in, false,
@@ -593,7 +605,7 @@ kronq_status run_twosided(const float* w, const float* k_in, const float* k_out,
     }
     KQ_CUDA_TRY(cudaMemsetAsync(t.changed, 0, sizeof(unsigned int), stream));
     twosided_step_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(
-        w, t.s, t.p2, t.delta, codes, w_hat, scale, zero, d_out, d_in, maxq, it == 0 ? 1 : 0,
+        w, t.p1, t.p2, t.delta, codes, w_hat, scale, zero, d_out, d_in, maxq, it == 0 ? 1 : 0,
         t.changed);
     KQ_TRY(check_launch("twosided_step_kernel"));
     unsigned int host = 0;
