@@ -769,7 +769,7 @@ def run_gpu(args):
 # DRAM bytes (read + write) per accumulate_tc_kernel launch, averaged over the launches of one
 # step: bounded ncu captures of this kernel version scaled to the step's launches (commands and
 # scaling in the accumulate profile summaries under profiles/); keyed by (workload, tokens)
-TRAFFIC = {("llama3_70b_block", 262144): 25.5e9}
+TRAFFIC = {("llama3_70b_block", 262144): 24.7e9}
 
 
 def _mem_available():

@@ -21,8 +21,11 @@
 // while the next tile accumulates in the other TMEM buffer.
 #include <cuda_bf16.h>
 
+#include <algorithm>
 #include <cstdlib>
 #include <cstring>
+#include <utility>
+#include <vector>
 
 #include "common.cuh"
 #include "internal.h"
@@ -71,7 +74,17 @@ struct TgParams {
   int products;           // 6: every term down to 2^-16 relative; 3: a0 b0 + a0 b1 + a1 b0
   const int32_t* skip;
   int* err;
+  // Tile schedule: slot j = blockIdx.x + i * gridDim.x holds the CTA's i-th tile. With n_order
+  // > 0, order[j] is that tile (kTgNoTile for none); otherwise slot j is tile j.
+  int n_slots;
+  int n_order;
+  uint16_t order[1024];
 };
+constexpr uint16_t kTgNoTile = 0xFFFF;
+
+__device__ __forceinline__ int slot_tile(const TgParams& p, int j) {
+  return p.n_order ? (p.order[j] == kTgNoTile ? -1 : static_cast<int>(p.order[j])) : j;
+}
 
 __host__ __device__ constexpr uint32_t idesc_bf16(int m, int n, bool b_mn) {
   return (1u << 4)                 // D: f32
@@ -106,6 +119,7 @@ struct TgMaps {
   CUtensorMap a[3];
   CUtensorMap b[3];
 };
+static_assert(sizeof(TgMaps) + sizeof(TgParams) <= 4096, "tgemm kernel parameters above 4 KB");
 
 template <int BN_>
 __global__ void __launch_bounds__(tg::THREADS, 1)
@@ -129,7 +143,6 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int num_tiles = p.tiles_m * p.tiles_n;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -163,9 +176,10 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
     if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+      for (int j = blockIdx.x; j < p.n_slots && ok; j += gridDim.x) {
+        const int t = slot_tile(p, j);
         TileInfo ti;
-        if (!tile_info<C>(p, t, ti)) continue;
+        if (t < 0 || !tile_info<C>(p, t, ti)) continue;
         for (int kb = ti.kb0; kb < ti.kb1; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
@@ -204,9 +218,10 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
       const uint32_t idesc = idesc_bf16(BM, BN, p.b_mn_major != 0);
       uint32_t it = 0, ui = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+      for (int j = blockIdx.x; j < p.n_slots && ok; j += gridDim.x) {
+        const int t = slot_tile(p, j);
         TileInfo ti;
-        if (!tile_info<C>(p, t, ti)) continue;
+        if (t < 0 || !tile_info<C>(p, t, ti)) continue;
         const uint32_t a = ui & 1u;
         const uint32_t aph = (ui >> 1) & 1u;
         ++ui;
@@ -259,9 +274,10 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
     // ------------------------------------------------------------------ epilogue (warps 2..5)
     const int q = warp & 3;
     uint32_t ui = 0;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+    for (int j = blockIdx.x; j < p.n_slots; j += gridDim.x) {
+      const int t = slot_tile(p, j);
       TileInfo ti;
-      if (!tile_info<C>(p, t, ti)) continue;
+      if (t < 0 || !tile_info<C>(p, t, ti)) continue;
       const uint32_t a = ui & 1u;
       const uint32_t aph = (ui >> 1) & 1u;
       ++ui;
@@ -447,21 +463,52 @@ kronq_status launch_tgemm(const Split3& a, const Split3& b, TgParams p, bool b_m
   // per device and cheap on the host, so set on every launch
   KQ_CUDA_TRY(cudaFuncSetAttribute(tgemm_kernel<BN_>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    C::SMEM_BYTES));
+  // The tiles that have work, with their K lengths (the same rule as tile_info): triangular
+  // operands make the lengths differ by up to the whole K.
+  const int tiles = p.tiles_m * p.tiles_n;
+  std::vector<std::pair<int, int>> work;   // (K blocks, tile)
+  work.reserve(tiles);
+  for (int t = 0; t < tiles; ++t) {
+    const int tm = t / p.tiles_n, tn = t % p.tiles_n;
+    const int bm = tm * tg::BM, bn = tn * C::BN;
+    if (p.upper_only && bm > bn + C::BN - 1) continue;
+    int k_lo = 0, k_hi = p.k;
+    if (p.tri & GEMM_A_UPPER) k_lo = std::max(k_lo, bm);
+    if (p.tri & GEMM_A_LOWER) k_hi = std::min(k_hi, bm + tg::BM);
+    if (p.tri & GEMM_B_LOWER) k_lo = std::max(k_lo, bn);
+    if (p.tri & GEMM_B_UPPER) k_hi = std::min(k_hi, bn + C::BN);
+    const int kb = k_hi > k_lo ? (k_hi + C::BK - 1) / C::BK - k_lo / C::BK : 0;
+    work.emplace_back(kb, t);
+  }
   // As few CTAs as the minimal number of tile waves needs: each CTA holds a whole SM (shared
   // memory), and SMs this GEMM does not need stay free for other streams' work.
-  const int tiles = p.tiles_m * p.tiles_n;
-  int work = tiles;
-  if (p.upper_only) {
-    work = 0;
-    for (int tm = 0; tm < p.tiles_m; ++tm)
-      for (int tn = 0; tn < p.tiles_n; ++tn)
-        if (tm * tg::BM <= tn * C::BN + C::BN - 1) ++work;
-  }
+  const int n_work = static_cast<int>(work.size());
   const int sms = sm_budget();
-  const int waves = (work + sms - 1) / sms;
-  int grid = waves > 0 ? (tiles + waves - 1) / waves : 1;
+  const int waves = (n_work + sms - 1) / sms;
+  int grid = waves > 0 ? (n_work + waves - 1) / waves : 1;
   if (grid > sms) grid = sms;
   if (grid < 1) grid = 1;
+  // Longest tiles first, dealt to the CTAs in a snake (wave w forward when w is even, backward
+  // when odd): each CTA gets a mix of long and short tiles, so that no CTA holds only the long
+  // ones. The table fits the kernel's parameters up to 1024 slots; larger launches have enough
+  // tiles per CTA for the plain order to even out.
+  p.n_order = 0;
+  p.n_slots = tiles;
+  const int slots = waves * grid;
+  if (slots <= static_cast<int>(sizeof(p.order) / sizeof(p.order[0])) && n_work > 0) {
+    std::stable_sort(work.begin(), work.end(),
+                     [](const std::pair<int, int>& x, const std::pair<int, int>& y) {
+                       return x.first > y.first;
+                     });
+    for (int j = 0; j < slots; ++j) p.order[j] = kTgNoTile;
+    for (int r = 0; r < n_work; ++r) {
+      const int w = r / grid, i = r % grid;
+      const int cta = (w & 1) ? grid - 1 - i : i;
+      p.order[w * grid + cta] = static_cast<uint16_t>(work[r].second);
+    }
+    p.n_order = 1;
+    p.n_slots = slots;
+  }
   tgemm_kernel<BN_><<<grid, tg::THREADS, C::SMEM_BYTES, stream>>>(maps, p);
   return check_launch("tgemm_kernel");
 }
@@ -512,8 +559,11 @@ kronq_status tgemm(int m, int n, int k, float alpha, Split3 a, Split3 b, bool b_
   p.skip = skip;
   p.err = device_error_word();
   if (!p.err) return fail(KRONQ_ERR_CUDA, "device error word unavailable");
-  // 128 x 256 tiles where the output is wide enough to fill them
-  if (n > 128 && tgemm_wide_tiles()) return launch_tgemm<256>(a, b, p, b_mn_major, stream);
+  // 128 x 256 tiles where they still give every SM a tile (fewer, wider tiles halve the CTAs
+  // of a small product, which then runs longer)
+  const int64_t wide_tiles = static_cast<int64_t>((m + 127) / 128) * ((n + 255) / 256);
+  if (n > 128 && wide_tiles >= sm_budget() && tgemm_wide_tiles())
+    return launch_tgemm<256>(a, b, p, b_mn_major, stream);
   return launch_tgemm<128>(a, b, p, b_mn_major, stream);
 }
 
