@@ -570,8 +570,16 @@ kronq_status run_twosided(const float* w, const float* k_in, const float* k_out,
   const float maxq = static_cast<float>((1 << bits) - 1);
   TwoWs t = two_carve(ws, d_out, d_in);
   int32_t* info = reinterpret_cast<int32_t*>(t.changed + 16);
-  KQ_TRY(inverse_of_factor(k_in, d_in, t.u_in, t.kt, t.chol_ws, info, stream));
-  KQ_TRY(inverse_of_factor(k_out, d_out, t.u_out, t.kt, t.chol_ws, info, stream));
+  for (int side = 0; side < 2; ++side) {
+    KQ_TRY(inverse_of_factor(side ? k_out : k_in, side ? d_out : d_in, side ? t.u_out : t.u_in,
+                             t.kt, t.chol_ws, info, stream));
+    int32_t bad = -1;
+    KQ_CUDA_TRY(cudaMemcpyAsync(&bad, info, sizeof(bad), cudaMemcpyDeviceToHost, stream));
+    KQ_CUDA_TRY(cudaStreamSynchronize(stream));
+    if (bad >= 0)
+      return fail(KRONQ_ERR_NOT_PD, "%s: K K^T has a non-positive pivot at %d (is it an inverse "
+                  "factor from kronq_cholinv?)", side ? "k_out" : "k_in", bad);
+  }
   {
     dim3 b(32, 8);
     unit_factor_split_kernel<<<dim3((d_in + 31) / 32, (d_in + 31) / 32), b, 0, stream>>>(

@@ -722,6 +722,38 @@ def test_quantize_llama3_70b_with_drift_sampled_rows(K, P, d_out, d_in):
     assert rel(h64(r.w_hat[rows]), o["w_hat"]) <= TOL
 
 
+def test_quantize_group128_llama3_70b_gate_sampled_rows(K, P):
+    # LLaMA-3-70B gate_proj (28672 x 8192), 2 bits, group-wise grid g = 128 ([KronQ-hyper]
+    # Experiments: the 2-bit results use g = 128), drifted input so P is active. 32 rows re-run
+    # by the oracle in follow mode (codes and group grids) from the GPU's K, W' and D'.
+    d_out, d_in, n, bits = 28672, 8192, 8192, 2
+    tag = ("qg70b",)
+    x = synth.correlated_x(n, d_in, synth.seed_for(tag, "X"), device="cuda")
+    xq = synth.perturbed(x, synth.seed_for(tag, "Xq"), rel_std=0.05)
+    g = synth.gradients(n, d_out, synth.seed_for(tag, "G"), device="cuda")
+    w = synth.weight(d_out, d_in, synth.seed_for(tag, "W"), device="cuda")
+    si = synth.rademacher(d_in, synth.seed_for(tag, "si"), device="cuda")
+    so = synth.rademacher(d_out, synth.seed_for(tag, "so"), device="cuda")
+    hx = torch.zeros(d_in, d_in, device="cuda"); dxx = torch.zeros(d_in, d_in, device="cuda")
+    hg = torch.zeros(d_out, device="cuda")
+    K.kronq_accumulate(xq, x, None, hx, None, dxx)
+    K.kronq_accumulate_diag(g, hg)
+    del x, xq, g
+    r = P.biip(w, hx, hg, dxx, 1.0 / n, si, so, 15 | K.BIIP_HG_DIAG, copy_hx=False)
+    wp = r.w_prime.clone(); dp = r.dxx.clone()
+    P.cholinv(r, 0.01, sync=True)
+    P.quantize(r, bits, group=128)
+    torch.cuda.synchronize()
+    rows = np.random.default_rng(77).choice(d_out, 32, replace=False)
+    o = O.quantize_layer(h64(wp[rows]), h64(r.hx), h64(dp), bits, follow_codes=h64(r.codes[rows]),
+                         group=128, follow_grid=(h64(r.scale[rows]), h64(r.zero[rows])))
+    assert np.array_equal(h64(r.scale[rows]), o["scale"].astype(np.float64))
+    assert np.array_equal(h64(r.zero[rows]), o["zero"].astype(np.float64))
+    assert int(o["grid_tie"].sum()) <= 1e-2 * 32 * (d_in // 128)
+    check_codes(r.codes[rows], o, 32 * d_in)
+    assert rel(h64(r.w_hat[rows]), o["w_hat"]) <= TOL
+
+
 def test_stack_scores_and_allocation(K, P):
     # Two blocks of the LLaMA-2-7B mixed-precision stack (14 sublayers, each its own X and G,
     # 65536 tokens, per-block G scale log-uniform on [1e-2, 1e1]): traces after BiIP against
