@@ -308,7 +308,9 @@ KRONQ_API kronq_status kronq_score_allocate(const double* tr_hx, const double* t
  *   lambda I); each update is two fp32-accurate tensor-core products with the strictly
  *   triangular parts of L_I and L_O; decisions in fp32. Synchronizes `stream` once per update
  *   (it reads how many codes changed). d_out, d_in <= 65535.
- *   Errors: KRONQ_ERR_CUDA if no fixed point is reached within d_out + d_in updates.
+ *   Errors: KRONQ_ERR_NOT_PD if k_in or k_out is not an invertible upper factor (its K K^T
+ *   has a non-positive pivot); KRONQ_ERR_CUDA if no fixed point is reached within d_out + d_in
+ *   updates.
  * ------------------------------------------------------------------------------------- */
 KRONQ_API size_t kronq_quantize_layer_twosided_workspace_size(int32_t d_out, int32_t d_in);
 KRONQ_API kronq_status kronq_quantize_layer_twosided(const float* w, const float* k_in,
@@ -371,7 +373,7 @@ KRONQ_API kronq_status kronq_pack_grid(const float* scale, const float* zero, in
  *   x        (device) n_tok x d_in, x_dtype KRONQ_DTYPE_BF16 or KRONQ_DTYPE_F32, row stride ld_x
  *            elements (>= d_in), aligned to its element size
  *   packed   (device, 16-byte aligned) codes in the packed format above
- *   packed_grid (device, 8-byte aligned) the grid from kronq_pack_grid with the same group
+ *   packed_grid (device, 16-byte aligned) the grid from kronq_pack_grid with the same group
  *   s_x, s_g, sign_in, sign_out, flags: the transforms of kronq_biip (KRONQ_BIIP_SCALE_IN,
  *            _SCALE_OUT, _ROTATE_IN, _ROTATE_OUT; a flag that is off drops its factor and its
  *            pointer may be NULL). Hadamard blocks up to 16384.

@@ -475,8 +475,8 @@ kronq_status kronq_qlinear(const void* x, int32_t x_dtype, int64_t ld_x, int32_t
   if (!aligned(x, x_dtype == KRONQ_DTYPE_BF16 ? 2 : 4) || !aligned(y, 4))
     return fail(KRONQ_ERR_INVALID_ARG, "x or y not aligned to its element size");
   if (!aligned(packed, 16)) return fail(KRONQ_ERR_INVALID_ARG, "packed not 16-byte aligned");
-  if (!aligned(packed_grid, 8))
-    return fail(KRONQ_ERR_INVALID_ARG, "packed_grid not 8-byte aligned");
+  if (!aligned(packed_grid, 16))
+    return fail(KRONQ_ERR_INVALID_ARG, "packed_grid not 16-byte aligned");
   const int b_in = d_in & (-d_in), b_out = d_out & (-d_out);
   if (((flags & KRONQ_BIIP_ROTATE_IN) && b_in > 16384) ||
       ((flags & KRONQ_BIIP_ROTATE_OUT) && b_out > 16384))

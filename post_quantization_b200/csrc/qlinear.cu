@@ -41,6 +41,9 @@ constexpr int QL_DQ_WARP0 = 8;          // warps 8..15: dequantization
 constexpr int QL_DQ_THREADS = 256;
 constexpr int QL_MAX_STAGES = 16;
 constexpr int QL_TERMS = 3;             // int8 terms of x'
+constexpr int QL_DP_THREADS = 160;      // decode kernel: 4 consumer warps + 1 producer warp
+constexpr int QL_DP_CTAS_PER_SM = 5;
+constexpr int QL_DP_MAX_STAGES = 8;
 
 __device__ __forceinline__ void griddep_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -833,7 +836,9 @@ struct QlDpArgs {
   float* partial;          // (C + T) segments x n_tok x 128
   int d_out, G, n_tok, rows;
   int grouped, rotate_out, b_tile;
+  int stages;              // ring stages (<= QL_DP_MAX_STAGES)
   int64_t U;
+  int* err;
 };
 
 __device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
@@ -917,74 +922,139 @@ __device__ __forceinline__ void dp_unit(const DpCodes<BITS>& c, const uint8_t* x
   }
 }
 
+// Shared-memory layout of the decode kernel: the x' terms of the groups the CTA visits (3 n_tok
+// rows of 128 bytes each), their (s, sum) pairs, then a ring of stages, each one unit's packed
+// codes (2048 b bytes) and its 128 grid pairs, filled by bulk copies; the stages' full and
+// empty barriers and the abort flag come last.
+struct DpSmem {
+  int x, sums, ring, stage, bars, total;
+};
+__host__ __device__ inline DpSmem dp_smem(int bits, int ng, int n_tok, int stages) {
+  DpSmem L;
+  L.x = 0;
+  L.sums = ng * 384 * n_tok;
+  L.ring = (L.sums + ng * n_tok * 8 + 127) / 128 * 128;
+  L.stage = 2048 * bits + QL_TILE * 8;
+  L.bars = L.ring + stages * L.stage;
+  L.total = L.bars + 2 * QL_DP_MAX_STAGES * 8 + 16;
+  return L;
+}
+
+// Four consumer warps (one thread per row of the 128-row unit) and one producer warp, whose
+// first lane streams the CTA's units into the ring with bulk copies; the codes therefore need
+// no registers while in flight, and the copies run as far ahead as the ring is deep.
 template <int BITS, int NT>
-__global__ void __launch_bounds__(128, 4) qlin_dp4a_kernel(QlDpArgs p) {
+__global__ void __launch_bounds__(QL_DP_THREADS, QL_DP_CTAS_PER_SM) qlin_dp4a_kernel(QlDpArgs p) {
   __shared__ float ys[NT][QL_TILE];
-  // x' terms of the groups this CTA visits: groups g0 .. g0 + n_units - 1 (mod G) in visiting
-  // order, or all G groups at their own index when the CTA visits every group
-  extern __shared__ __align__(16) uint8_t xstage[];
-  const int r = threadIdx.x;                          // row of the tile
-  const int lane = r & 31;
+  extern __shared__ __align__(128) uint8_t dsm[];
+  const int tid = threadIdx.x;
+  const int r = tid;                                  // row of the tile (consumer threads)
+  const int lane = tid & 31, warp = tid >> 5;
   const int64_t C = gridDim.x;
   const int64_t u0 = unit_begin(blockIdx.x, p.U, C);
   const int64_t u1 = unit_begin(blockIdx.x + 1, p.U, C);
   const int n_units = static_cast<int>(u1 - u0);
-  constexpr int D = BITS == 2 ? 4 : 2;                // units of codes in flight per thread
-  const int64_t blob = 2048 * BITS;
-  DpCodes<BITS> buf[D];
-  float2 gbuf[D];                                     // this row's grid for those units
-  // unit i's grid entry: (tile, group) of the unit for group-wise grids, tile for per-row
-  auto grid_of = [&](int64_t u) {
-    return __ldg(&p.grid[p.grouped ? u * QL_TILE + r : (u / p.G) * QL_TILE + r]);
-  };
-  // the packed codes and the grid do not depend on the preceding kernel: load them first
-#pragma unroll
-  for (int d = 0; d < D; ++d)
-    if (d < n_units) {
-      dp_load<BITS>(p.packed + (u0 + d) * blob, r, buf[d]);
-      gbuf[d] = grid_of(u0 + d);
-    }
-  griddep_wait();                                     // x' and its sums come from qlin_in
-  const int gb = 128 * p.rows;                         // bytes of one group's terms
   const bool all_groups = n_units >= p.G;
   const int ng = all_groups ? p.G : n_units;
-  float2* sstage = reinterpret_cast<float2*>(xstage + ng * gb);   // (s, sum) per group, token
+  const int S = p.stages;
+  const DpSmem L = dp_smem(BITS, ng, p.n_tok, S);
+  uint8_t* xstage = dsm + L.x;                        // group i: 3 n_tok rows of 128 bytes
+  float2* sstage = reinterpret_cast<float2*>(dsm + L.sums);
+  uint64_t* full = reinterpret_cast<uint64_t*>(dsm + L.bars);
+  uint64_t* empty = full + QL_DP_MAX_STAGES;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + QL_DP_MAX_STAGES);
+  const uint32_t pk = 2048u * BITS;
+  auto stage_ptr = [&](int s) { return dsm + L.ring + s * L.stage; };
+  auto grid_src = [&](int64_t u) {
+    return p.grid + (p.grouped ? u * QL_TILE : (u / p.G) * QL_TILE);
+  };
+  auto issue = [&](int i, int s) {
+    mbar_arrive_expect_tx(&full[s], pk + QL_TILE * 8);
+    bulk_load(stage_ptr(s), p.packed + (u0 + i) * static_cast<int64_t>(pk), pk, &full[s]);
+    bulk_load(stage_ptr(s) + pk, grid_src(u0 + i), QL_TILE * 8, &full[s]);
+  };
+
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], QL_TILE / 32);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const bool producer = warp == QL_TILE / 32;
+  // the packed codes and the grid do not depend on the preceding kernel: start them first
+  const int pre = min(S, n_units);
+  if (producer && lane == 0)
+    for (int i = 0; i < pre; ++i) issue(i, i);
+  griddep_wait();                                     // x' and its sums come from qlin_in
   {
+    // x' terms of the groups this CTA visits: groups g0 .. g0 + ng - 1 (mod G) in visiting
+    // order, or all G groups at their own index when the CTA visits every group; the scale
+    // s carries 4^-(parts - 1) and the sum 4^(parts - 1), the factor of the combined parts
     const int gstart = all_groups ? 0 : static_cast<int>(u0 % p.G);
-    const int words = ng * gb / 16;
-    for (int w = threadIdx.x; w < words; w += blockDim.x) {
-      const int gi = w / (gb / 16), off = w % (gb / 16);
+    const int tr = 3 * p.n_tok;                       // term rows per group
+    const int words = ng * tr * 8;                    // 16-byte words
+    for (int w = tid; w < words; w += blockDim.x) {
+      const int gi = w / (tr * 8), off = w % (tr * 8);
       int gsrc = gstart + gi;
       if (gsrc >= p.G) gsrc -= p.G;
-      reinterpret_cast<uint4*>(xstage)[w] =
-          __ldg(reinterpret_cast<const uint4*>(p.bop + static_cast<int64_t>(gsrc) * gb) + off);
+      reinterpret_cast<uint4*>(xstage)[w] = __ldg(
+          reinterpret_cast<const uint4*>(p.bop + static_cast<int64_t>(gsrc) * 128 * p.rows) + off);
     }
-    for (int w = threadIdx.x; w < ng * p.n_tok; w += blockDim.x) {
+    constexpr float kPart = BITS == 2 ? 64.f : (BITS == 4 ? 16.f : 1.f);
+    for (int w = tid; w < ng * p.n_tok; w += blockDim.x) {
       int gsrc = gstart + w / p.n_tok;
       if (gsrc >= p.G) gsrc -= p.G;
-      sstage[w] = __ldg(&p.sums[static_cast<int64_t>(gsrc) * p.n_tok + w % p.n_tok]);
+      const float2 v = __ldg(&p.sums[static_cast<int64_t>(gsrc) * p.n_tok + w % p.n_tok]);
+      sstage[w] = make_float2(v.x * (1.f / kPart), v.y * kPart);
     }
     __syncthreads();
   }
-  float y[NT];
-#pragma unroll
-  for (int t = 0; t < NT; ++t) y[t] = 0.f;
-  int g = static_cast<int>(u0 % p.G);
-  int tile = static_cast<int>(u0 / p.G);
-  for (int i0 = 0; i0 < n_units; i0 += D) {
-#pragma unroll
-    for (int d = 0; d < D; ++d) {
-      const int i = i0 + d;
-      if (i >= n_units) break;
-      const int row = tile * QL_TILE + r;
-      const float2 gz = gbuf[d];
-      const int si = all_groups ? g : i;                // staged group index
-      int acc[NT][QL_TERMS][4];
-      dp_unit<BITS, NT>(buf[d], xstage + si * gb, p.n_tok, acc);
-      if (i + D < n_units) {
-        dp_load<BITS>(p.packed + (u0 + i + D) * blob, r, buf[d]);
-        gbuf[d] = grid_of(u0 + i + D);
+
+  if (producer) {
+    // ------------------------------------------------------------------ producer
+    if (lane == 0) {
+      int i = pre;
+      for (; i < n_units; ++i) {
+        const int s = i % S;
+        if (!mbar_wait(&empty[s], ((i / S) & 1u) ^ 1u, abort_flag, p.err, DEV_ERR_TMA_WAIT))
+          break;
+        issue(i, s);
       }
+      if (i < n_units) {
+        // copies already issued complete on their barriers before the CTA leaves
+        for (int j = max(0, i - S); j < i; ++j)
+          mbar_drain(&full[j % S], (j / S) & 1u, 1000000000ull);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ consumers
+    // Every consumer runs every unit, also after an abort (then on whatever the stage holds),
+    // so that the named barriers of the within-tile Hadamard are always reached by all 128.
+    float y[NT];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) y[t] = 0.f;
+    int g = static_cast<int>(u0 % p.G);
+    int tile = static_cast<int>(u0 / p.G);
+    const int xb = 384 * p.n_tok;                    // staged bytes per group
+    for (int i = 0; i < n_units; ++i) {
+      const int s = i % S;
+      mbar_wait(&full[s], (i / S) & 1u, abort_flag, p.err, DEV_ERR_LOAD_WAIT);
+      DpCodes<BITS> cb;
+      {
+        const uint2* pc = reinterpret_cast<const uint2*>(stage_ptr(s)) + r;
+#pragma unroll
+        for (int k = 0; k < DpCodes<BITS>::PIECES; ++k) cb.p[k] = pc[k * 128];
+      }
+      const float2 gz = reinterpret_cast<const float2*>(stage_ptr(s) + pk)[r];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      const int row = tile * QL_TILE + r;
+      const int si = all_groups ? g : i;              // staged group index
+      int acc[NT][QL_TERMS][4];
+      dp_unit<BITS, NT>(cb, xstage + si * xb, p.n_tok, acc);
 #pragma unroll
       for (int t = 0; t < NT; ++t) {
         if (t >= p.n_tok) break;
@@ -992,12 +1062,12 @@ __global__ void __launch_bounds__(128, 4) qlin_dp4a_kernel(QlDpArgs p) {
         float a[QL_TERMS];
 #pragma unroll
         for (int term = 0; term < QL_TERMS; ++term) {
-          // each part is an exact multiple of its bit-position factor
+          // the parts combined at the factor of the highest one (exact: |v| < 2^22)
           int v = acc[t][term][0];
           if (BITS == 2)
-            v += (acc[t][term][1] >> 2) + (acc[t][term][2] >> 4) + (acc[t][term][3] >> 6);
+            v = (v << 6) + (acc[t][term][1] << 4) + (acc[t][term][2] << 2) + acc[t][term][3];
           else if (BITS == 4)
-            v += acc[t][term][1] >> 4;
+            v = (v << 4) + acc[t][term][1];
           a[term] = i2f_small(v);
         }
         const float dot = a[0] + a[1] * (1.f / 128.f) + a[2] * (1.f / 16384.f);
@@ -1017,10 +1087,10 @@ __global__ void __launch_bounds__(128, 4) qlin_dp4a_kernel(QlDpArgs p) {
             }
           }
           for (int h = 32; h < p.b_tile; h <<= 1) {
-            __syncthreads();
+            named_bar_sync(1, QL_TILE);
 #pragma unroll
             for (int t = 0; t < NT; ++t) ys[t][r] = y[t];
-            __syncthreads();
+            named_bar_sync(1, QL_TILE);
 #pragma unroll
             for (int t = 0; t < NT; ++t) {
               const float o = ys[t][r ^ h];
@@ -1042,6 +1112,7 @@ __global__ void __launch_bounds__(128, 4) qlin_dp4a_kernel(QlDpArgs p) {
     }
   }
   griddep_launch_dependents();
+  __syncthreads();
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -1206,7 +1277,6 @@ kronq_status launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStr
 int pow2_factor(int d) { return d & (-d); }
 
 constexpr int QL_DP_MAX_TOK = 2;   // up to this many tokens: the CUDA-core decode kernel
-constexpr int QL_DP_CTAS_PER_SM = 4;
 constexpr int QL_DP_MAX_UNITS = 48;   // units per CTA (its x' groups are staged in shared memory)
 
 struct QlGeom {
@@ -1253,7 +1323,7 @@ kronq_status launch_dp_t(const QlDpArgs& p, int C, size_t smem, cudaStream_t str
   const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(smem));
   if (e != cudaSuccess) return fail(KRONQ_ERR_CUDA, "qlin_dp4a smem: %s", cudaGetErrorString(e));
-  return launch_pdl(kern, dim3(C), dim3(QL_TILE), smem, stream, true, "qlin_dp4a_kernel", p);
+  return launch_pdl(kern, dim3(C), dim3(QL_DP_THREADS), smem, stream, true, "qlin_dp4a_kernel", p);
 }
 
 kronq_status launch_dp(int bits, int nt, const QlDpArgs& p, int C, size_t smem,
@@ -1400,9 +1470,23 @@ kronq_status run_qlinear(const QlinearArgs& q, void* ws, cudaStream_t stream) {
       dpa.rotate_out = rot_out ? 1 : 0;
       dpa.b_tile = rot_out ? std::min(b_out, QL_TILE) : 1;
       dpa.U = g.U;
-      const int64_t upc = (g.U + g.C - 1) / g.C;          // units of the largest CTA
-      const size_t dsmem = static_cast<size_t>(std::min<int64_t>(upc, g.G)) *
-                           (128 * dpa.rows + sizeof(float2) * nt);
+      dpa.err = device_error_word();
+      if (!dpa.err) return fail(KRONQ_ERR_CUDA, "device error word unavailable");
+      // the largest CTA's staged groups, and as many ring stages as leave room for
+      // QL_DP_CTAS_PER_SM CTAs per SM (at least 2)
+      const int64_t upc = (g.U + g.C - 1) / g.C;
+      const int ng = static_cast<int>(std::min<int64_t>(upc, g.G));
+      int per_sm_smem = 0;
+      KQ_CUDA_TRY(cudaDeviceGetAttribute(&per_sm_smem, cudaDevAttrMaxSharedMemoryPerMultiprocessor,
+                                         dev));
+      const int budget = per_sm_smem / QL_DP_CTAS_PER_SM - 1024 -
+                         static_cast<int>(sizeof(float)) * nt * QL_TILE;
+      const DpSmem L1 = dp_smem(q.bits, ng, nt, 1);
+      dpa.stages = std::max(2, std::min(QL_DP_MAX_STAGES, (budget - (L1.total - L1.stage)) /
+                                                              L1.stage));
+      const size_t dsmem = static_cast<size_t>(dp_smem(q.bits, ng, nt, dpa.stages).total);
+      if (static_cast<int>(dsmem) > max_smem)
+        return fail(KRONQ_ERR_UNSUPPORTED, "qlinear decode: shared memory too small");
       KQ_TRY(launch_dp(q.bits, nt, dpa, g.C, dsmem, stream));
     } else {
     QlMmaArgs p;

@@ -346,7 +346,7 @@ def case_qlinear(args):
     sweep_ms = a.elapsed_time(b) / args.reps
     # the whole block in one graph (the layers' kernels chained back to back, as in a decode
     # step); replayed with the other copies of the codes in between so that L2 starts cold
-    block_us = None
+    block_us = conc_us = None
     if not args.no_graphs:
         gb = torch.cuda.CUDAGraph()
         with torch.cuda.graph(gb):
@@ -365,11 +365,48 @@ def case_qlinear(args):
             b.synchronize()
             tot += a.elapsed_time(b)
         block_us = tot / args.reps * 1e3
-        del gb, flush
+        del gb
+        if args.block:
+            # the block's own dependency order: q, k and v read the same input and run as
+            # three branches, then o, then gate and up as two branches, then down
+            stages = [["q", "k", "v"], ["o"], ["gate", "up"], ["down"]]
+            by_name = {L["name"]: L for L in layers}
+            side = [torch.cuda.Stream() for _ in range(3)]
+            gc = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gc):
+                main = torch.cuda.current_stream()
+                for names in stages:
+                    if len(names) == 1:
+                        call(by_name[names[0]])
+                        continue
+                    fork = torch.cuda.Event()
+                    fork.record(main)
+                    for st, nm in zip(side, names):
+                        st.wait_event(fork)
+                        with torch.cuda.stream(st):
+                            call(by_name[nm])
+                    for st in side[:len(names)]:
+                        main.wait_stream(st)
+            for _ in range(3):
+                gc.replay()
+            torch.cuda.synchronize()
+            tot = 0.0
+            for _ in range(args.reps):
+                flush.zero_()
+                a.record()
+                gc.replay()
+                b.record()
+                b.synchronize()
+                tot += a.elapsed_time(b)
+            conc_us = tot / args.reps * 1e3
+            del gc
+        del flush
     print(json.dumps({"case": "qlinear", "bits": bits, "group": group, "tokens": n,
                       "layers": res, "sum_us": tot_ms * 1e3, "sweep_us": sweep_ms * 1e3,
                       "sweep_GBps": tot_bytes / sweep_ms / 1e6, "block_graph_us": block_us,
                       "block_graph_GBps": tot_bytes / block_us / 1e3 if block_us else None,
+                      "block_branches_us": conc_us,
+                      "block_branches_GBps": tot_bytes / conc_us / 1e3 if conc_us else None,
                       "launches": K.kronq_launch_count()}))
     del graphs
 

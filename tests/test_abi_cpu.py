@@ -158,7 +158,8 @@ def test_inference_calls_host_checks(K):
     assert call(n_tok=0) == K.OK                            # nothing to do
     assert call(d_out=0) == K.ERR_SHAPE
     assert call(grid=None) == K.ERR_INVALID_ARG
-    assert call(grid=772) == K.ERR_INVALID_ARG              # 8-byte alignment
+    assert call(grid=772) == K.ERR_INVALID_ARG              # 16-byte alignment
+    assert call(grid=776) == K.ERR_INVALID_ARG
     assert call(s_g=None) == K.ERR_INVALID_ARG              # SCALE_OUT needs s_g
     assert call(s_g=None, flags=K.BIIP_FULL & ~K.BIIP_SCALE_OUT) == K.ERR_WORKSPACE
     assert call(si=None) == K.ERR_INVALID_ARG
@@ -209,3 +210,18 @@ def test_llama2_stack_allocation_shape(K):
     s, bits = K.kronq_score_allocate(tr_hx, tr_hg, sizes, [2, 3, 4], 2.5)
     assert sum(b * n for b, n in zip(bits, sizes)) <= math.floor(2.5 * sum(sizes))
     assert bits == O.score_allocate(tr_hx, tr_hg, sizes, [2, 3, 4], 2.5)[1]
+
+
+def test_twosided_argument_errors_before_device(K):
+    lib = K.load_library()
+    f = lib.kronq_quantize_layer_twosided
+    # (w, k_in, k_out, d_out, d_in, bits, codes, scale, zero, w_hat, iterations, ws, bytes, stream)
+    assert f(8, 8, 8, 0, 16, 2, 8, 8, 8, 16, None, None, 0, None) == K.ERR_SHAPE
+    assert f(8, 8, 8, 16, 16, 9, 8, 8, 8, 16, None, None, 0, None) == K.ERR_UNSUPPORTED
+    assert f(8, None, 8, 16, 16, 2, 8, 8, 8, 16, None, None, 0, None) == K.ERR_INVALID_ARG
+    assert f(8, 8, 8, 16, 16, 2, 8, 8, 8, 8, None, None, 0, None) == K.ERR_INVALID_ARG   # w == w_hat
+    assert f(8, 8, 8, 70000, 16, 2, 8, 8, 8, 16, None, None, 0, None) == K.ERR_SHAPE
+    assert f(8, 8, 8, 16, 16, 2, 8, 8, 8, 16, None, None, 0, None) == K.ERR_WORKSPACE
+    need = K.load_library().kronq_quantize_layer_twosided_workspace_size(300, 200)
+    # two factors, their splits, four fp32 d_out x d_in buffers and a split of one
+    assert need >= 4 * 300 * 200 * 4 + 3 * 300 * 200 * 2 + (300 * 300 + 200 * 200) * 4
