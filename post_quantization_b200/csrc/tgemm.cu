@@ -74,16 +74,23 @@ struct TgParams {
   int products;           // 6: every term down to 2^-16 relative; 3: a0 b0 + a0 b1 + a1 b0
   const int32_t* skip;
   int* err;
-  // Tile schedule: slot j = blockIdx.x + i * gridDim.x holds the CTA's i-th tile. With n_order
-  // > 0, order[j] is that tile (kTgNoTile for none); otherwise slot j is tile j.
+  // Tile schedule: slot j = blockIdx.x + i * gridDim.x holds the CTA's i-th tile; slot j is
+  // tile j, unless the launch passes a table (TgOrder<true>).
   int n_slots;
-  int n_order;
-  uint16_t order[1024];
+};
+
+// The table: order[j] is slot j's tile (kTgNoTile for none). A separate kernel parameter, so
+// that launches without one keep a small parameter block.
+template <bool SCHED>
+struct TgOrder {
+  uint16_t order[SCHED ? 1536 : 2];
 };
 constexpr uint16_t kTgNoTile = 0xFFFF;
 
-__device__ __forceinline__ int slot_tile(const TgParams& p, int j) {
-  return p.n_order ? (p.order[j] == kTgNoTile ? -1 : static_cast<int>(p.order[j])) : j;
+template <bool SCHED>
+__device__ __forceinline__ int slot_tile(const TgOrder<SCHED>& o, int j) {
+  if constexpr (SCHED) return o.order[j] == kTgNoTile ? -1 : static_cast<int>(o.order[j]);
+  return j;
 }
 
 __host__ __device__ constexpr uint32_t idesc_bf16(int m, int n, bool b_mn) {
@@ -119,11 +126,13 @@ struct TgMaps {
   CUtensorMap a[3];
   CUtensorMap b[3];
 };
-static_assert(sizeof(TgMaps) + sizeof(TgParams) <= 4096, "tgemm kernel parameters above 4 KB");
+static_assert(sizeof(TgMaps) + sizeof(TgParams) + sizeof(TgOrder<true>) <= 4096,
+              "tgemm kernel parameters above 4 KB");
 
-template <int BN_>
+template <int BN_, bool SCHED>
 __global__ void __launch_bounds__(tg::THREADS, 1)
-    tgemm_kernel(const __grid_constant__ TgMaps maps, const TgParams p) {
+    tgemm_kernel(const __grid_constant__ TgMaps maps, const TgParams p,
+                 const __grid_constant__ TgOrder<SCHED> sched) {
   using namespace tg;
   using C = Cfg<BN_>;
   constexpr int BN = C::BN, BK = C::BK, STAGE_BYTES = C::STAGE_BYTES, TMEM_COLS = C::TMEM_COLS;
@@ -177,7 +186,7 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
       uint32_t it = 0;
       bool ok = true;
       for (int j = blockIdx.x; j < p.n_slots && ok; j += gridDim.x) {
-        const int t = slot_tile(p, j);
+        const int t = slot_tile<SCHED>(sched, j);
         TileInfo ti;
         if (t < 0 || !tile_info<C>(p, t, ti)) continue;
         for (int kb = ti.kb0; kb < ti.kb1; ++kb, ++it) {
@@ -219,7 +228,7 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
       uint32_t it = 0, ui = 0;
       bool ok = true;
       for (int j = blockIdx.x; j < p.n_slots && ok; j += gridDim.x) {
-        const int t = slot_tile(p, j);
+        const int t = slot_tile<SCHED>(sched, j);
         TileInfo ti;
         if (t < 0 || !tile_info<C>(p, t, ti)) continue;
         const uint32_t a = ui & 1u;
@@ -275,7 +284,7 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
     const int q = warp & 3;
     uint32_t ui = 0;
     for (int j = blockIdx.x; j < p.n_slots; j += gridDim.x) {
-      const int t = slot_tile(p, j);
+      const int t = slot_tile<SCHED>(sched, j);
       TileInfo ti;
       if (t < 0 || !tile_info<C>(p, t, ti)) continue;
       const uint32_t a = ui & 1u;
@@ -461,8 +470,10 @@ kronq_status launch_tgemm(const Split3& a, const Split3& b, TgParams p, bool b_m
   p.tiles_m = (p.m + tg::BM - 1) / tg::BM;
   p.tiles_n = (p.n + C::BN - 1) / C::BN;
   // per device and cheap on the host, so set on every launch
-  KQ_CUDA_TRY(cudaFuncSetAttribute(tgemm_kernel<BN_>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   C::SMEM_BYTES));
+  KQ_CUDA_TRY(cudaFuncSetAttribute(tgemm_kernel<BN_, false>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
+  KQ_CUDA_TRY(cudaFuncSetAttribute(tgemm_kernel<BN_, true>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
   // The tiles that have work, with their K lengths (the same rule as tile_info): triangular
   // operands make the lengths differ by up to the whole K.
   const int tiles = p.tiles_m * p.tiles_n;
@@ -480,36 +491,45 @@ kronq_status launch_tgemm(const Split3& a, const Split3& b, TgParams p, bool b_m
     const int kb = k_hi > k_lo ? (k_hi + C::BK - 1) / C::BK - k_lo / C::BK : 0;
     work.emplace_back(kb, t);
   }
-  // As few CTAs as the minimal number of tile waves needs: each CTA holds a whole SM (shared
-  // memory), and SMs this GEMM does not need stay free for other streams' work.
   const int n_work = static_cast<int>(work.size());
   const int sms = sm_budget();
-  const int waves = (n_work + sms - 1) / sms;
-  int grid = waves > 0 ? (n_work + waves - 1) / waves : 1;
-  if (grid > sms) grid = sms;
-  if (grid < 1) grid = 1;
-  // Longest tiles first, dealt to the CTAs in a snake (wave w forward when w is even, backward
-  // when odd): each CTA gets a mix of long and short tiles, so that no CTA holds only the long
-  // ones. The table fits the kernel's parameters up to 1024 slots; larger launches have enough
-  // tiles per CTA for the plain order to even out.
-  p.n_order = 0;
+  bool uniform = true;
+  for (const auto& w : work) uniform = uniform && w.first == work[0].first;
+  TgOrder<true> order;
+  constexpr int kMaxSlots = static_cast<int>(sizeof(order.order) / sizeof(order.order[0]));
   p.n_slots = tiles;
-  const int slots = waves * grid;
-  if (slots <= static_cast<int>(sizeof(p.order) / sizeof(p.order[0])) && n_work > 0) {
+  int grid = 1;
+  if (!uniform && n_work > 0 && ((n_work + sms - 1) / sms) * std::min(sms, n_work) <= kMaxSlots) {
+    // Tiles of different K lengths (triangular operands): every SM takes part, and the tiles,
+    // longest first, are dealt to the CTAs in a snake (wave w forward when w is even, backward
+    // when odd), so that each CTA gets a mix of long and short tiles and no CTA holds only the
+    // long ones. The order travels as a table in the kernel's parameters.
+    grid = std::min(sms, n_work);
+    const int waves = (n_work + grid - 1) / grid;
     std::stable_sort(work.begin(), work.end(),
                      [](const std::pair<int, int>& x, const std::pair<int, int>& y) {
                        return x.first > y.first;
                      });
-    for (int j = 0; j < slots; ++j) p.order[j] = kTgNoTile;
+    const int slots = waves * grid;
+    for (int j = 0; j < slots; ++j) order.order[j] = kTgNoTile;
     for (int r = 0; r < n_work; ++r) {
       const int w = r / grid, i = r % grid;
       const int cta = (w & 1) ? grid - 1 - i : i;
-      p.order[w * grid + cta] = static_cast<uint16_t>(work[r].second);
+      order.order[w * grid + cta] = static_cast<uint16_t>(work[r].second);
     }
-    p.n_order = 1;
     p.n_slots = slots;
+    tgemm_kernel<BN_, true><<<grid, tg::THREADS, C::SMEM_BYTES, stream>>>(maps, p, order);
+    return check_launch("tgemm_kernel");
+  } else {
+    // Equal tiles, or too many for the table (then enough per CTA for the plain order to even
+    // out): as few CTAs as the minimal number of tile waves needs. Each CTA holds a whole SM
+    // (shared memory), and SMs this GEMM does not need stay free for other streams' work.
+    const int waves = (n_work + sms - 1) / sms;
+    grid = waves > 0 ? (tiles + waves - 1) / waves : 1;
+    grid = std::max(1, std::min(grid, sms));
   }
-  tgemm_kernel<BN_><<<grid, tg::THREADS, C::SMEM_BYTES, stream>>>(maps, p);
+  tgemm_kernel<BN_, false><<<grid, tg::THREADS, C::SMEM_BYTES, stream>>>(maps, p,
+                                                                          TgOrder<false>{});
   return check_launch("tgemm_kernel");
 }
 

@@ -205,7 +205,9 @@ def case_cholinv(args):
     h /= n
     info = torch.empty(1, dtype=torch.int32, device="cuda")
     k = h.clone()
+    n0 = K.kronq_launch_count()
     K.kronq_cholinv(k, 0.01, info, K.CHOLINV_SYNC)
+    per_call = K.kronq_launch_count() - n0
     a, b = ev(), ev()
     a.record()
     for _ in range(args.reps):
@@ -213,7 +215,23 @@ def case_cholinv(args):
         K.kronq_cholinv(k, 0.01, info, 0)
     b.record()
     torch.cuda.synchronize()
-    print(json.dumps({"case": "cholinv", "d": d, "ms": a.elapsed_time(b) / args.reps}))
+    ms = a.elapsed_time(b) / args.reps
+    # the same calls replayed from a CUDA graph: the difference is the launch gaps
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        k.copy_(h)
+        K.kronq_cholinv(k, 0.01, info, 0)
+    g.replay()
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(args.reps):
+        g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    print(json.dumps({"case": "cholinv", "d": d, "ms": ms,
+                      "graph_ms": a.elapsed_time(b) / args.reps,
+                      "launches_per_call": per_call}))
+    del g
 
 
 def case_quantize(args):
