@@ -858,17 +858,24 @@ struct DpCodes {
   uint2 p[PIECES];
 };
 
-template <int BITS>
-__device__ __forceinline__ void dp_load(const uint8_t* blob, int r, DpCodes<BITS>& c) {
-  const uint2* pc = reinterpret_cast<const uint2*>(blob) + r;
-#pragma unroll
-  for (int i = 0; i < DpCodes<BITS>::PIECES; ++i) c.p[i] = __ldg(pc + i * 128);
+__device__ __forceinline__ uint2 lds_u2(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint4 lds_u4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
 }
 
 // acc[term][part] += codes . x' terms over the unit's 128 columns; the parts carry the codes'
 // bit-position factors (2 bits: 4^k, 4 bits: 16^k, 3 bits: 1)
 template <int BITS, int NT>
-__device__ __forceinline__ void dp_unit(const DpCodes<BITS>& c, const uint8_t* xg,
+__device__ __forceinline__ void dp_unit(const DpCodes<BITS>& c, uint32_t xg,
                                         int n_tok, int (&acc)[NT][QL_TERMS][4]) {
   const uint32_t* w = reinterpret_cast<const uint32_t*>(c.p);
 #pragma unroll
@@ -909,7 +916,7 @@ __device__ __forceinline__ void dp_unit(const DpCodes<BITS>& c, const uint8_t* x
       if (t >= n_tok) break;
 #pragma unroll
       for (int term = 0; term < QL_TERMS; ++term) {
-        const uint4 xv = reinterpret_cast<const uint4*>(xg + (3 * t + term) * 128)[q];
+        const uint4 xv = lds_u4(xg + (3 * t + term) * 128 + 16 * q);
         const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};   // columns 16q + 4k .. + 3
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -1016,12 +1023,17 @@ __global__ void __launch_bounds__(QL_DP_THREADS, QL_DP_CTAS_PER_SM) qlin_dp4a_ke
   if (producer) {
     // ------------------------------------------------------------------ producer
     if (lane == 0) {
-      int i = pre;
+      // unit i >= S refills stage i % S once the consumers released unit i - S: the empty
+      // barrier's completion number i / S - 1, parity (i / S - 1) & 1
+      int i = pre, s = 0;
+      uint32_t eph = 0;
       for (; i < n_units; ++i) {
-        const int s = i % S;
-        if (!mbar_wait(&empty[s], ((i / S) & 1u) ^ 1u, abort_flag, p.err, DEV_ERR_TMA_WAIT))
-          break;
+        if (!mbar_wait(&empty[s], eph, abort_flag, p.err, DEV_ERR_TMA_WAIT)) break;
         issue(i, s);
+        if (++s == S) {
+          s = 0;
+          eph ^= 1u;
+        }
       }
       if (i < n_units) {
         // copies already issued complete on their barriers before the CTA leaves
@@ -1039,22 +1051,28 @@ __global__ void __launch_bounds__(QL_DP_THREADS, QL_DP_CTAS_PER_SM) qlin_dp4a_ke
     int g = static_cast<int>(u0 % p.G);
     int tile = static_cast<int>(u0 / p.G);
     const int xb = 384 * p.n_tok;                    // staged bytes per group
+    const uint32_t xs0 = smem_u32(xstage);
+    const uint32_t ring_row = smem_u32(stage_ptr(0)) + 8 * r;   // this row's piece 0, stage 0
+    int s = 0;                                       // stage of unit i, and its fill parity
+    uint32_t ph = 0;
     for (int i = 0; i < n_units; ++i) {
-      const int s = i % S;
-      mbar_wait(&full[s], (i / S) & 1u, abort_flag, p.err, DEV_ERR_LOAD_WAIT);
+      mbar_wait(&full[s], ph, abort_flag, p.err, DEV_ERR_LOAD_WAIT);
       DpCodes<BITS> cb;
-      {
-        const uint2* pc = reinterpret_cast<const uint2*>(stage_ptr(s)) + r;
+      const uint32_t st = ring_row + s * L.stage;
 #pragma unroll
-        for (int k = 0; k < DpCodes<BITS>::PIECES; ++k) cb.p[k] = pc[k * 128];
-      }
-      const float2 gz = reinterpret_cast<const float2*>(stage_ptr(s) + pk)[r];
+      for (int k = 0; k < DpCodes<BITS>::PIECES; ++k) cb.p[k] = lds_u2(st + 1024 * k);
+      const uint2 gzu = lds_u2(st + pk);             // (scale, zero) of this row
+      const float2 gz = make_float2(__uint_as_float(gzu.x), __uint_as_float(gzu.y));
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
+      if (++s == S) {
+        s = 0;
+        ph ^= 1u;
+      }
       const int row = tile * QL_TILE + r;
       const int si = all_groups ? g : i;              // staged group index
       int acc[NT][QL_TERMS][4];
-      dp_unit<BITS, NT>(cb, xstage + si * xb, p.n_tok, acc);
+      dp_unit<BITS, NT>(cb, xs0 + si * xb, p.n_tok, acc);
 #pragma unroll
       for (int t = 0; t < NT; ++t) {
         if (t >= p.n_tok) break;
