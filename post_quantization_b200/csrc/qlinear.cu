@@ -875,8 +875,8 @@ __device__ __forceinline__ uint4 lds_u4(uint32_t addr) {
 // acc[term][part] += codes . x' terms over the unit's 128 columns; the parts carry the codes'
 // bit-position factors (2 bits: 4^k, 4 bits: 16^k, 3 bits: 1)
 template <int BITS, int NT>
-__device__ __forceinline__ void dp_unit(const DpCodes<BITS>& c, uint32_t xg,
-                                        int n_tok, int (&acc)[NT][QL_TERMS][4]) {
+__device__ __forceinline__ void dp_unit(const DpCodes<BITS>& c, uint32_t xg, int n_tok,
+                                        int (&acc)[NT][QL_TERMS][4]) {
   const uint32_t* w = reinterpret_cast<const uint32_t*>(c.p);
 #pragma unroll
   for (int t = 0; t < NT; ++t)
@@ -913,7 +913,8 @@ __device__ __forceinline__ void dp_unit(const DpCodes<BITS>& c, uint32_t xg,
     }
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
-      if (t >= n_tok) break;
+      // a run-time bound for two tokens keeps their loads apart (no spills); none for one
+      if (NT > 1 && t >= n_tok) break;
 #pragma unroll
       for (int term = 0; term < QL_TERMS; ++term) {
         const uint4 xv = lds_u4(xg + (3 * t + term) * 128 + 16 * q);
@@ -1050,7 +1051,8 @@ __global__ void __launch_bounds__(QL_DP_THREADS, QL_DP_CTAS_PER_SM) qlin_dp4a_ke
     for (int t = 0; t < NT; ++t) y[t] = 0.f;
     int g = static_cast<int>(u0 % p.G);
     int tile = static_cast<int>(u0 / p.G);
-    const int xb = 384 * p.n_tok;                    // staged bytes per group
+    // the kernel is instantiated for the call's token count: NT == p.n_tok
+    constexpr int xb = 384 * NT;                     // staged bytes per group
     const uint32_t xs0 = smem_u32(xstage);
     const uint32_t ring_row = smem_u32(stage_ptr(0)) + 8 * r;   // this row's piece 0, stage 0
     int s = 0;                                       // stage of unit i, and its fill parity
@@ -1075,8 +1077,8 @@ __global__ void __launch_bounds__(QL_DP_THREADS, QL_DP_CTAS_PER_SM) qlin_dp4a_ke
       dp_unit<BITS, NT>(cb, xs0 + si * xb, p.n_tok, acc);
 #pragma unroll
       for (int t = 0; t < NT; ++t) {
-        if (t >= p.n_tok) break;
-        const float2 sq = sstage[si * p.n_tok + t];
+        if (NT > 1 && t >= p.n_tok) break;
+        const float2 sq = sstage[si * NT + t];
         float a[QL_TERMS];
 #pragma unroll
         for (int term = 0; term < QL_TERMS; ++term) {
@@ -1116,10 +1118,10 @@ __global__ void __launch_bounds__(QL_DP_THREADS, QL_DP_CTAS_PER_SM) qlin_dp4a_ke
             }
           }
         }
-        float* out = p.partial + (static_cast<int64_t>(blockIdx.x) + tile) * p.n_tok * QL_TILE + r;
+        float* out = p.partial + (static_cast<int64_t>(blockIdx.x) + tile) * NT * QL_TILE + r;
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
-          if (t < p.n_tok) out[t * QL_TILE] = y[t];
+          out[t * QL_TILE] = y[t];
           y[t] = 0.f;
         }
       }
@@ -1346,6 +1348,7 @@ kronq_status launch_dp_t(const QlDpArgs& p, int C, size_t smem, cudaStream_t str
 
 kronq_status launch_dp(int bits, int nt, const QlDpArgs& p, int C, size_t smem,
                        cudaStream_t stream) {
+  if (nt != 1 && nt != 2) return fail(KRONQ_ERR_INVALID_ARG, "decode kernel: 1 or 2 tokens");
   if (bits == 2)
     return nt <= 1 ? launch_dp_t<2, 1>(p, C, smem, stream) : launch_dp_t<2, 2>(p, C, smem, stream);
   if (bits == 3)
