@@ -30,7 +30,6 @@ namespace kq {
 
 namespace {
 
-constexpr int kNormRows = 256;   // rows per CTA of the norms pass
 
 template <typename T>
 __device__ __forceinline__ float load_as_float(const T* p, int64_t i);
@@ -44,13 +43,14 @@ __device__ __forceinline__ float load_as_float<__nv_bfloat16>(const __nv_bfloat1
 }
 
 // Squared column and row norms of a contiguous rows x cols W, added into fp64 accumulators. A CTA
-// takes a panel of 32 V columns (V elements = one 16-byte load per lane) and kNormRows rows; warp
-// w takes rows w, w + 8, .. of it. Per row the warp sums its lanes' squares with five shuffles
+// takes a panel of 32 V columns (V elements = one 16-byte load per lane) and chunk_rows rows (the
+// host sizes the chunks so that the grid is one wave of resident CTAs); warp w takes rows w,
+// w + 8, .. of it. Per row the warp sums its lanes' squares with five shuffles
 // and one lane adds the row's panel sum; per column the lanes keep running sums, which the 8
 // warps combine in shared memory at the end, one addition per column and CTA.
 template <typename T>
 __global__ void __launch_bounds__(256, 3) colrow_norms_kernel(const T* __restrict__ w, int rows,
-                                                           int cols, int vec,
+                                                           int cols, int vec, int chunk_rows,
                                                            double* __restrict__ col_sq,
                                                            double* __restrict__ row_sq) {
   constexpr int V = 16 / sizeof(T);
@@ -58,8 +58,8 @@ __global__ void __launch_bounds__(256, 3) colrow_norms_kernel(const T* __restric
   __shared__ float part[8][PW];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int c0 = blockIdx.x * PW + lane * V;
-  const int r0 = blockIdx.y * kNormRows;
-  const int r1 = rows - r0 < kNormRows ? rows : r0 + kNormRows;
+  const int r0 = blockIdx.y * chunk_rows;
+  const int r1 = rows - r0 < chunk_rows ? rows : r0 + chunk_rows;
   const bool whole = vec && c0 + V <= cols;   // one aligned 16-byte load
   float colacc[V];
 #pragma unroll
@@ -457,7 +457,6 @@ __global__ void __launch_bounds__(2 << LOG2P) fwht_cols_reg_kernel(float* m, int
                                                                   int64_t cols, int rs,
                                                                   float out_scale, int vec) {
   extern __shared__ __align__(16) float sb[];
-  constexpr int log2p = LOG2P;
   constexpr int P = 1 << LOG2P;
   constexpr int nt = 2 * P;
   const int t = threadIdx.x;
@@ -1246,13 +1245,19 @@ kronq_status run_biip(const BiipArgs& a, void* ws_raw, cudaStream_t stream) {
     const bool bf = a.w_dtype == KRONQ_DTYPE_BF16;
     const int esz = bf ? 2 : 4, pw = 32 * (16 / esz);
     const int vec = (reinterpret_cast<uintptr_t>(a.w) & 15u) == 0 && (a.d_in * esz) % 16 == 0;
-    dim3 grid((a.d_in + pw - 1) / pw, (a.d_out + kNormRows - 1) / kNormRows);
+    // row chunks (multiples of 64 rows) such that panels x chunks fills the 3 CTAs per SM once
+    const int panels = (a.d_in + pw - 1) / pw;
+    const int chunks = std::max(1, 3 * device_sms() / panels);
+    int chunk_rows = (a.d_out + chunks - 1) / chunks;
+    chunk_rows = std::max(64, (chunk_rows + 63) / 64 * 64);
+    dim3 grid(panels, (a.d_out + chunk_rows - 1) / chunk_rows);
     if (bf)
       colrow_norms_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
-          static_cast<const __nv_bfloat16*>(a.w), a.d_out, a.d_in, vec, ws.col_sq, ws.row_sq);
+          static_cast<const __nv_bfloat16*>(a.w), a.d_out, a.d_in, vec, chunk_rows, ws.col_sq,
+          ws.row_sq);
     else
       colrow_norms_kernel<float><<<grid, 256, 0, stream>>>(
-          static_cast<const float*>(a.w), a.d_out, a.d_in, vec, ws.col_sq, ws.row_sq);
+          static_cast<const float*>(a.w), a.d_out, a.d_in, vec, chunk_rows, ws.col_sq, ws.row_sq);
     KQ_TRY(check_launch("colrow_norms_kernel"));
   }
 
