@@ -549,6 +549,34 @@ def test_drift_term_llama3_70b_width_sampled(K, d):
     del hx, dxx
 
 
+@pytest.mark.parametrize("d", [8192, 28672])
+def test_accumulate_llama3_70b_bench_size_sampled(K, d):
+    # The benchmark's launch configuration: 262144 tokens at the LLaMA-3-70B widths, X~ = X +
+    # N(0, (0.05 rms X)^2). H_X runs as four 65536-token work units per output tile whose fp32
+    # partials meet by atomic adds; D = (X - X~)^T X~ as eight 32768-token fp16 products. 8
+    # sampled 128 x 128 tiles of each (one diagonal) against fp64 sums of the same bf16 values,
+    # and the trace of H_X against ||X~||^2 summed in fp64.
+    n = 262144
+    x = synth.correlated_x(n, d, synth.seed_for("acc70b-bench", d), device="cuda")
+    xq = synth.perturbed(x, synth.seed_for("acc70b-bench", d, "q"), rel_std=0.05)
+    hx = torch.zeros(d, d, device="cuda"); dxx = torch.zeros(d, d, device="cuda")
+    K.kronq_accumulate(xq, x, None, hx, None, dxx)
+    torch.cuda.synchronize()
+    r = np.random.default_rng(d + 7)
+    for t in range(8):
+        i0 = int(r.integers(0, d // 128)) * 128
+        j0 = i0 if t == 0 else int(r.integers(0, d // 128)) * 128
+        qa = h64(xq[:, i0:i0 + 128]); qb = qa if j0 == i0 else h64(xq[:, j0:j0 + 128])
+        assert rel(h64(hx[i0:i0 + 128, j0:j0 + 128]), qa.T @ qb) <= TOL, (i0, j0)
+        xa = h64(x[:, i0:i0 + 128])
+        assert rel(h64(dxx[i0:i0 + 128, j0:j0 + 128]), (xa - qa).T @ qb) <= TOL, (i0, j0)
+    tr = 0.0
+    for c0 in range(0, n, 16384):
+        tr += float(torch.sum(xq[c0:c0 + 16384].double() ** 2))
+    assert abs(float(torch.trace(hx.double())) - tr) <= TOL * tr
+    del x, xq, hx, dxx
+
+
 @pytest.mark.parametrize("d_out,d_in", [(8192, 28672), (1024, 8192), (16384, 16384)])
 def test_biip_llama3_70b_shapes(K, P, d_out, d_in):
     # LLaMA-3-70B shapes: down_proj 8192 x 28672 (input Hadamard blocks of 4096, output 8192),
