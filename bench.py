@@ -700,7 +700,8 @@ def run_gpu(args):
             peak = 1400.0
             peak_src = "fallback (sustained bf16)"
         acc_tflops = sum(acc_flops) / (sum(acc_ms) / 1e3) / 1e12
-        traffic = TRAFFIC.get((args.workload, n_tok))
+        # the captures cover the full-H_G step only (the diagonal mode has other launches)
+        traffic = None if args.hg_diag else TRAFFIC.get((args.workload, n_tok))
         result = {
             "metric": "quantized weight params/s (BiIP+GPTAQ solve); H_X/H_G accumulate TFLOP/s",
             "value": value,
