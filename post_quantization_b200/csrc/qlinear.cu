@@ -16,6 +16,10 @@
 //                    terms of x'; four epilogue warps apply the grid, the group scale and the
 //                    within-tile part of U^T, and write one partial per (CTA, row tile). Work is
 //                    split over CTAs as contiguous ranges of (row tile, column group) units.
+//   qlin_dp4a_kernel (one or two tokens, in place of qlin_mma_kernel) a producer warp streams
+//                    each CTA's units of packed codes and grid into a shared-memory ring with
+//                    bulk copies; four warps, one thread per row, take exact int32 dot products
+//                    of the codes with the int8 terms (dp4a) and write the same partials.
 //   qlin_out_kernel  sums each tile's partials in a fixed order (deterministic), applies the
 //                    across-tile part of U^T, the signs and S_G^-1.
 // The codes are the MMA's A operand (128 rows per instruction); a tcgen05 MMA costs about the
