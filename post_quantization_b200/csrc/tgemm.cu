@@ -499,11 +499,14 @@ kronq_status launch_tgemm(const Split3& a, const Split3& b, TgParams p, bool b_m
   constexpr int kMaxSlots = static_cast<int>(sizeof(order.order) / sizeof(order.order[0]));
   p.n_slots = tiles;
   int grid = 1;
-  if (!uniform && n_work > 0 && ((n_work + sms - 1) / sms) * std::min(sms, n_work) <= kMaxSlots) {
-    // Tiles of different K lengths (triangular operands): every SM takes part, and the tiles,
-    // longest first, are dealt to the CTAs in a snake (wave w forward when w is even, backward
-    // when odd), so that each CTA gets a mix of long and short tiles and no CTA holds only the
-    // long ones. The order travels as a table in the kernel's parameters.
+  if ((!uniform || n_work < tiles) && n_work > 0 &&
+      ((n_work + sms - 1) / sms) * std::min(sms, n_work) <= kMaxSlots) {
+    // Tiles of different K lengths (triangular operands), or only some tiles with work (the
+    // upper triangle): every SM takes part, and the tiles that have work, longest first, are
+    // dealt to the CTAs in a snake (wave w forward when w is even, backward when odd), so that
+    // each CTA gets a mix of long and short tiles and no CTA holds only the long ones. (In the
+    // plain order a CTA's slots would fall on the skipped triangle unevenly.) The order travels
+    // as a table in the kernel's parameters.
     grid = std::min(sms, n_work);
     const int waves = (n_work + grid - 1) / grid;
     std::stable_sort(work.begin(), work.end(),
@@ -521,8 +524,8 @@ kronq_status launch_tgemm(const Split3& a, const Split3& b, TgParams p, bool b_m
     tgemm_kernel<BN_, true><<<grid, tg::THREADS, C::SMEM_BYTES, stream>>>(maps, p, order);
     return check_launch("tgemm_kernel");
   } else {
-    // Equal tiles, or too many for the table (then enough per CTA for the plain order to even
-    // out): as few CTAs as the minimal number of tile waves needs. Each CTA holds a whole SM
+    // Equal tiles that all have work, or too many for the table (then enough per CTA for the
+    // plain order to even out): as few CTAs as the minimal number of tile waves needs. Each CTA holds a whole SM
     // (shared memory), and SMs this GEMM does not need stay free for other streams' work.
     const int waves = (n_work + sms - 1) / sms;
     grid = waves > 0 ? (tiles + waves - 1) / waves : 1;
