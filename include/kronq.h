@@ -362,7 +362,8 @@ KRONQ_API kronq_status kronq_pack_codes(const uint8_t* codes, int32_t d_out, int
  * (scale, zero) fp32 pairs, tile by tile of 128 rows, and within a tile group by group (group
  * 128) or once (group 0): pair (t, g, r) at index (t G' + g) 128 + r, G' = ceil(d_in / 128) or 1;
  * rows past d_out hold (0, 0). packed_grid: device, 8-byte aligned, at least
- * kronq_packed_grid_bytes bytes. The values are copied, not changed. */
+ * kronq_packed_grid_bytes bytes (kronq_qlinear reads it with bulk copies and needs it 16-byte
+ * aligned). The values are copied, not changed. */
 KRONQ_API size_t kronq_packed_grid_bytes(int32_t d_out, int32_t d_in, int32_t group);
 KRONQ_API kronq_status kronq_pack_grid(const float* scale, const float* zero, int32_t d_out,
                                        int32_t d_in, int32_t group, void* packed_grid,
