@@ -557,6 +557,7 @@ def test_accumulate_llama3_70b_bench_size_sampled(K, d):
     # sampled 128 x 128 tiles of each (one diagonal) against fp64 sums of the same bf16 values,
     # and the trace of H_X against ||X~||^2 summed in fp64.
     n = 262144
+    torch.cuda.empty_cache()                 # ~40 GB below: start from released memory
     x = synth.correlated_x(n, d, synth.seed_for("acc70b-bench", d), device="cuda")
     xq = synth.perturbed(x, synth.seed_for("acc70b-bench", d, "q"), rel_std=0.05)
     hx = torch.zeros(d, d, device="cuda"); dxx = torch.zeros(d, d, device="cuda")
@@ -575,6 +576,7 @@ def test_accumulate_llama3_70b_bench_size_sampled(K, d):
         tr += float(torch.sum(xq[c0:c0 + 16384].double() ** 2))
     assert abs(float(torch.trace(hx.double())) - tr) <= TOL * tr
     del x, xq, hx, dxx
+    torch.cuda.empty_cache()
 
 
 @pytest.mark.parametrize("d_out,d_in", [(8192, 28672), (1024, 8192), (16384, 16384)])
